@@ -1,0 +1,294 @@
+"""Pins for the SLA oracle: closed forms, special cases, library routines, hand examples.
+
+None of these re-types the oracle's own formulas: each checks it against
+something fixed independently (torch SDPA, the quadratic form of linear
+attention, hand-worked rows, an independent loop implementation on a tiny case).
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import sla
+
+
+def _rng(seed):
+    return np.random.default_rng(seed)
+
+
+def _bf16ish(x):
+    return torch.tensor(x, dtype=torch.float32).to(torch.bfloat16).double().numpy()
+
+
+# ---------------------------------------------------------------- counts
+
+@pytest.mark.parametrize("nkb,pc,pn,kc,kn", [
+    (4, 0.25, 0.25, 1, 1),        # tiny workload: 25 % / 25 % of 4 blocks
+    (512, 0.05, 0.10, 26, 51),    # 32k-token workload: 5 % / 10 % of 512 blocks
+    (1800, 0.05, 0.10, 90, 180),  # 115k-token workload: 5 % / 10 % of 1800 blocks
+    (1, 0.05, 0.10, 1, 0),        # at least one critical block per row
+    (20, 1.0, 0.0, 20, 0),        # dense mode: everything critical
+    (10, 0.6, 0.6, 6, 4),         # kc + kn capped at Nkb
+])
+def test_block_counts(nkb, pc, pn, kc, kn):
+    assert sla.block_counts(nkb, pc, pn) == (kc, kn)
+
+
+# ---------------------------------------------------------------- pooling
+
+def test_pool_constant_block_is_the_token():
+    rng = _rng(1)
+    tok = rng.standard_normal(8)
+    x = np.tile(tok, (128, 1))
+    x[64:] = rng.standard_normal((64, 8))
+    out = sla.pool_blocks(x, np.ones(128, bool))
+    np.testing.assert_allclose(out[0], tok, rtol=1e-14, atol=0)
+
+
+def test_pool_excludes_pads_closed_form():
+    # block of 64 tokens, 56 valid, channel 0 holds the token index: mean = 27.5
+    x = np.zeros((64, 3))
+    x[:, 0] = np.arange(64)
+    x[:, 1] = 1.0
+    valid = sla.valid_tokens(1, 56, 64)
+    out = sla.pool_blocks(x, valid)
+    assert out[0, 0] == 27.5
+    assert out[0, 1] == 1.0
+
+
+def test_valid_tokens_segments():
+    v = sla.valid_tokens(3, 5, 8)
+    assert v.tolist() == ([True] * 5 + [False] * 3) * 3
+
+
+# ---------------------------------------------------------------- classification
+
+def _golden_rows(golden_dir):
+    rows = []
+    with open(os.path.join(golden_dir, "classify_ties.txt")) as f:
+        for line in f:
+            if line.startswith("#") or not line.strip():
+                continue
+            a, b, c = line.split("|")
+            kc, kn = map(int, a.split())
+            rows.append((kc, kn, [float(x) for x in b.split()], [int(x) for x in c.split()]))
+    return rows
+
+
+def test_classify_hand_examples(golden_dir):
+    for kc, kn, scores, expect in _golden_rows(golden_dir):
+        got = sla.classify(np.array([scores]), kc, kn)[0]
+        assert got.tolist() == expect, (scores, kc, kn)
+
+
+def test_classify_invariants_random():
+    rng = _rng(7)
+    for nk, kc, kn in [(37, 2, 3), (64, 4, 7), (512, 26, 51)]:
+        logits = rng.standard_normal((16, nk))
+        p = sla.row_softmax(logits)
+        m = sla.classify(logits, kc, kn)
+        for i in range(16):
+            assert (m[i] == 1).sum() == kc
+            assert (m[i] == -1).sum() == kn
+            crit, marg, negl = p[i][m[i] == 1], p[i][m[i] == 0], p[i][m[i] == -1]
+            assert crit.min() >= marg.max() >= negl.max() if marg.size else True
+            if marg.size:
+                assert marg.min() >= negl.max() if negl.size else True
+
+
+def test_classify_on_probabilities_equals_on_logits():
+    # the page ranks P_c; ranking its logits must give the same labels
+    rng = _rng(8)
+    logits = rng.standard_normal((32, 200)) * 3
+    p = sla.row_softmax(logits)
+    assert np.array_equal(sla.classify(logits, 10, 20), sla.classify(p, 10, 20))
+
+
+def test_threshold_band():
+    logits = np.array([[3.0, 1.0, 2.0, 0.0]])
+    p = sla.row_softmax(logits)
+    m = sla.classify(logits, 1, 1)
+    tc, tn = sla.threshold_band(p, m)
+    assert tc[0] == p[0, 0] and tn[0] == p[0, 3]
+
+
+# ---------------------------------------------------------------- sparse branch
+
+def _sdpa(q, k, v, key_valid):
+    qt = torch.tensor(q)[None, None]
+    kt = torch.tensor(k)[None, None]
+    vt = torch.tensor(v)[None, None]
+    mask = torch.tensor(key_valid)[None, None, None, :].expand(1, 1, q.shape[0], k.shape[0])
+    return torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, attn_mask=mask)[0, 0].numpy()
+
+
+def test_all_blocks_listed_equals_sdpa():
+    rng = _rng(3)
+    n, d = 256, 16
+    q, k, v = (_bf16ish(rng.standard_normal((n, d))) for _ in range(3))
+    valid = sla.valid_tokens(2, 100, 128)
+    q[~valid] = k[~valid] = v[~valid] = 0
+    nb = n // 64
+    out = sla.block_sparse_attention(q, k, v, valid, [list(range(nb))] * nb)
+    ref = _sdpa(q, k, v, valid)
+    ref[~valid] = 0
+    np.testing.assert_allclose(out, ref, rtol=0, atol=1e-12)
+
+
+def test_softmax_rows_sum_to_one_with_identity_values():
+    rng = _rng(4)
+    n, d = 128, 8
+    q, k = rng.standard_normal((n, d)), rng.standard_normal((n, d))
+    v = np.eye(n)              # output row = attention probabilities
+    valid = np.ones(n, bool)
+    out = sla.block_sparse_attention(q, k, v, valid, [[1], [0, 1]])
+    np.testing.assert_allclose(out.sum(axis=1), 1.0, rtol=0, atol=1e-12)
+    assert (out >= 0).all()
+    assert np.abs(out[:64, :64]).max() == 0.0      # block 0 only attends key block 1
+
+
+def test_identical_keys_give_mean_of_values():
+    rng = _rng(5)
+    n, d = 128, 8
+    q = rng.standard_normal((n, d))
+    k = np.tile(rng.standard_normal(d), (n, 1))
+    v = rng.standard_normal((n, d))
+    valid = np.ones(n, bool)
+    out = sla.block_sparse_attention(q, k, v, valid, [[1], [1]])
+    np.testing.assert_allclose(out, np.tile(v[64:].mean(axis=0), (n, 1)), rtol=0, atol=1e-13)
+
+
+def test_empty_list_gives_zero():
+    rng = _rng(6)
+    q = k = v = rng.standard_normal((128, 4))
+    out = sla.block_sparse_attention(q, k, v, np.ones(128, bool), [[], [0]])
+    assert np.abs(out[:64]).max() == 0 and np.abs(out[64:]).max() > 0
+
+
+# ---------------------------------------------------------------- linear branch
+
+def test_phi_values():
+    x = np.array([0.0, 1.0, -1.0, 2.5, -50.0])
+    np.testing.assert_allclose(sla.phi_elu1(x), [1.0, 2.0, math.exp(-1), 3.5, math.exp(-50)], rtol=1e-15)
+
+
+def test_all_marginal_equals_quadratic_linear_attention():
+    rng = _rng(9)
+    n, d = 192, 12
+    q, k, v = (rng.standard_normal((n, d)) for _ in range(3))
+    valid = sla.valid_tokens(1, 180, 192)
+    q[~valid] = k[~valid] = v[~valid] = 0
+    nb = n // 64
+    out = sla.linear_attention(q, k, v, valid, np.ones((nb, nb), bool))
+    # textbook form: weights phi(q).phi(k) over valid keys, normalised per row
+    fq = np.where(q > 0, q + 1, np.exp(q))
+    fk = np.where(k > 0, k + 1, np.exp(k))
+    w = (fq @ fk.T) * valid[None, :]
+    ref = (w @ v) / w.sum(axis=1, keepdims=True)
+    ref[~valid] = 0
+    np.testing.assert_allclose(out, ref, rtol=1e-12, atol=1e-13)
+
+
+def test_linear_constant_values_reproduced():
+    rng = _rng(10)
+    n, d = 128, 6
+    q, k = rng.standard_normal((n, d)), rng.standard_normal((n, d))
+    c = rng.standard_normal(d)
+    v = np.tile(c, (n, 1))
+    out = sla.linear_attention(q, k, v, np.ones(n, bool), np.array([[False, True], [True, True]]))
+    np.testing.assert_allclose(out, np.tile(c, (n, 1)), rtol=1e-13, atol=1e-14)
+
+
+def test_linear_no_marginal_gives_zero():
+    rng = _rng(11)
+    q = k = v = rng.standard_normal((128, 4))
+    out = sla.linear_attention(q, k, v, np.ones(128, bool), np.array([[False, False], [True, False]]))
+    assert np.abs(out[:64]).max() == 0 and np.abs(out[64:]).max() > 0
+
+
+# ---------------------------------------------------------------- combination
+
+def _tiny_inputs(seed, n=256, d=16):
+    rng = _rng(seed)
+    return tuple(_bf16ish(rng.standard_normal((n, d))) for _ in range(3))
+
+
+def test_w_proj_zero_gives_sparse_only_and_identity_gives_sum():
+    q, k, v = _tiny_inputs(12)
+    valid = np.ones(256, bool)
+    r0 = sla.sla_head(q, k, v, np.zeros((16, 16)), valid, 0.25, 0.25)
+    np.testing.assert_array_equal(r0["o"], r0["o_s"])
+    r1 = sla.sla_head(q, k, v, np.eye(16), valid, 0.25, 0.25)
+    np.testing.assert_allclose(r1["o"], r1["o_s"] + r1["o_l"], rtol=0, atol=0)
+
+
+def test_dense_mode_is_full_attention():
+    q, k, v = _tiny_inputs(13)
+    valid = sla.valid_tokens(1, 250, 256)
+    q[~valid] = k[~valid] = v[~valid] = 0
+    r = sla.sla_head(q, k, v, np.eye(16), valid, 1.0, 0.0)
+    assert (r["mask"] == 1).all()
+    ref = _sdpa(q, k, v, valid)
+    ref[~valid] = 0
+    np.testing.assert_allclose(r["o"], ref, rtol=0, atol=1e-12)
+
+
+def _loop_sla(q, k, v, w, valid, kc, kn):
+    """Independent loop-by-loop SLA on a tiny case (brute force pin)."""
+    n, d = q.shape
+    nb = n // 64
+    pooled = []
+    for x in (q, k):
+        pb = []
+        for b in range(nb):
+            acc, cnt = [0.0] * d, 0
+            for t in range(b * 64, b * 64 + 64):
+                if valid[t]:
+                    cnt += 1
+                    for c in range(d):
+                        acc[c] += x[t, c]
+            pb.append([a / cnt for a in acc])
+        pooled.append(pb)
+    qb, kb = pooled
+    out = np.zeros((n, d))
+    for i in range(nb):
+        sc = []
+        for j in range(nb):
+            sc.append(sum(qb[i][c] * kb[j][c] for c in range(d)) / math.sqrt(d))
+        order = sorted(range(nb), key=lambda j: (-sc[j], j))
+        crit = set(order[:kc])
+        negl = set(order[nb - kn:]) if kn else set()
+        marg = [j for j in range(nb) if j not in crit and j not in negl]
+        keys_c = [u for j in sorted(crit) for u in range(j * 64, j * 64 + 64) if valid[u]]
+        keys_m = [u for j in marg for u in range(j * 64, j * 64 + 64) if valid[u]]
+        for t in range(i * 64, i * 64 + 64):
+            if not valid[t]:
+                continue
+            logit = [sum(q[t, c] * k[u, c] for c in range(d)) / math.sqrt(d) for u in keys_c]
+            mx = max(logit)
+            e = [math.exp(x - mx) for x in logit]
+            s = sum(e)
+            o_s = [sum(e[a] * v[u, c] for a, u in enumerate(keys_c)) / s for c in range(d)]
+            o_l = [0.0] * d
+            if keys_m:
+                phi = lambda x: x + 1 if x > 0 else math.exp(x)
+                wts = [sum(phi(q[t, c]) * phi(k[u, c]) for c in range(d)) for u in keys_m]
+                tot = sum(wts)
+                o_l = [sum(wts[a] * v[u, c] for a, u in enumerate(keys_m)) / tot for c in range(d)]
+            for c in range(d):
+                out[t, c] = o_s[c] + sum(o_l[a] * w[a, c] for a in range(d))
+    return out
+
+
+def test_brute_force_loops_tiny():
+    rng = _rng(14)
+    n, d = 256, 4
+    q, k, v = (_bf16ish(rng.standard_normal((n, d))) for _ in range(3))
+    w = rng.standard_normal((d, d)) / 2
+    valid = sla.valid_tokens(1, 240, 256)
+    q[~valid] = k[~valid] = v[~valid] = 0
+    r = sla.sla_head(q, k, v, w, valid, 0.25, 0.25)
+    ref = _loop_sla(q, k, v, w, valid, r["kc"], r["kn"])
+    np.testing.assert_allclose(r["o"], ref, rtol=1e-10, atol=1e-12)
