@@ -1,0 +1,246 @@
+// k_classify.cu -- SLA's compressed scores and percentile classification.
+//
+// SLA page section 3: the pooled Q and K give a compressed attention-weight
+// matrix P_c = softmax(pool(Q) pool(K)^T / sqrt(d)); within each query-block row
+// the top 5 % positions are labelled critical (1), the bottom 10 % negligible
+// (-1), the rest marginal (0).  Softmax is strictly increasing along a row, so
+// the labels are taken on the fp64 logits; ties rank the lower key-block index
+// first.  Both the logits and the selection are fp64 so that the labels agree
+// with an fp64 evaluation of the same definition.
+//
+// block_logits_kernel: 64x64 output tiles of qbar kbar^T / sqrt(d) (fp64 FMA).
+// classify_rows_kernel: one warp per row; two MSB-first radix selections over
+//   order-preserving 64-bit keys (8 passes of 8-bit digits) find the kc-th
+//   largest and kn-th smallest key; one pass in index order applies the
+//   thresholds with index tie-breaking and emits the mask row, the ascending
+//   critical list, the marginal indicator row (bf16 1/0 for the tensor-core
+//   contraction) and, on request, P_c in fp32.
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <math.h>
+
+#include "launch.h"
+#include "sm100.cuh"
+
+namespace slr {
+namespace {
+
+__global__ void __launch_bounds__(256)
+block_logits_kernel(const double* __restrict__ qbar, const double* __restrict__ kbar,
+                    double* __restrict__ logits, int nb, int d, double sqrt_d) {
+  __shared__ double As[16][64 + 1];
+  __shared__ double Bs[16][64 + 1];
+  const int bh = blockIdx.z;
+  const int i0 = blockIdx.y * 64, j0 = blockIdx.x * 64;
+  const double* A = qbar + (size_t)bh * nb * d;
+  const double* B = kbar + (size_t)bh * nb * d;
+  const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
+  double acc[4][4];
+  #pragma unroll
+  for (int a = 0; a < 4; ++a)
+    #pragma unroll
+    for (int b = 0; b < 4; ++b) acc[a][b] = 0.0;
+  for (int c0 = 0; c0 < d; c0 += 16) {
+    for (int e = threadIdx.x; e < 64 * 16; e += 256) {
+      const int row = e / 16, col = e % 16;
+      As[col][row] = (i0 + row < nb) ? A[(size_t)(i0 + row) * d + c0 + col] : 0.0;
+      Bs[col][row] = (j0 + row < nb) ? B[(size_t)(j0 + row) * d + c0 + col] : 0.0;
+    }
+    __syncthreads();
+    #pragma unroll
+    for (int c = 0; c < 16; ++c) {
+      double a[4], b[4];
+      #pragma unroll
+      for (int u = 0; u < 4; ++u) { a[u] = As[c][ty * 4 + u]; b[u] = Bs[c][tx * 4 + u]; }
+      #pragma unroll
+      for (int u = 0; u < 4; ++u)
+        #pragma unroll
+        for (int w = 0; w < 4; ++w) acc[u][w] = fma(a[u], b[w], acc[u][w]);
+    }
+    __syncthreads();
+  }
+  #pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int i = i0 + ty * 4 + u;
+    if (i >= nb) continue;
+    #pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      const int j = j0 + tx * 4 + w;
+      if (j < nb) logits[((size_t)bh * nb + i) * nb + j] = acc[u][w] / sqrt_d;
+    }
+  }
+}
+
+// Order-preserving map of an fp64 value onto uint64 (larger value -> larger key);
+// -0 is folded onto +0 so that equal values give equal keys.
+__device__ __forceinline__ uint64_t order_key(double x) {
+  if (x == 0.0) x = 0.0;
+  const uint64_t b = (uint64_t)__double_as_longlong(x);
+  return (b >> 63) ? ~b : (b | 0x8000000000000000ull);
+}
+
+__device__ __forceinline__ int warp_incl_scan(int v, int lane) {
+  #pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xFFFFFFFFu, v, o);
+    if (lane >= o) v += y;
+  }
+  return v;
+}
+
+// MSB-first radix selection of the k-th largest (largest=true) or k-th smallest
+// key among keys[0..n).  Returns the key value T, how many of the keys equal to
+// T are taken (take), and how many keys equal T in total (eq_total).
+__device__ void radix_select(const uint64_t* keys, int n, int k, bool largest, unsigned* hist, int lane,
+                             uint64_t& T, int& take, int& eq_total) {
+  uint64_t prefix = 0, pmask = 0;
+  int kk = k, last = 0;
+  for (int shift = 56; shift >= 0; shift -= 8) {
+    for (int b = lane; b < 256; b += 32) hist[b] = 0;
+    __syncwarp();
+    for (int j = lane; j < n; j += 32) {
+      const uint64_t u = keys[j];
+      if ((u & pmask) == prefix) atomicAdd(&hist[(u >> shift) & 255], 1u);
+    }
+    __syncwarp();
+    int cnt[8], lsum = 0;
+    #pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const int bin = largest ? 255 - (lane * 8 + q) : lane * 8 + q;
+      cnt[q] = (int)hist[bin];
+      lsum += cnt[q];
+    }
+    const int incl = warp_incl_scan(lsum, lane);
+    const int excl = incl - lsum;
+    const bool has = excl < kk && incl >= kk;
+    const unsigned bal = __ballot_sync(0xFFFFFFFFu, has);
+    const int src = __ffs(bal) - 1;
+    int sel = 0, before = 0;
+    if (lane == src) {
+      int acc = excl;
+      #pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        if (acc + cnt[q] >= kk) { sel = largest ? 255 - (lane * 8 + q) : lane * 8 + q; before = acc; break; }
+        acc += cnt[q];
+      }
+    }
+    sel = __shfl_sync(0xFFFFFFFFu, sel, src);
+    before = __shfl_sync(0xFFFFFFFFu, before, src);
+    kk -= before;
+    last = (int)hist[sel];
+    prefix |= (uint64_t)sel << shift;
+    pmask |= (uint64_t)0xFF << shift;
+    __syncwarp();
+  }
+  T = prefix;
+  take = kk;
+  eq_total = last;
+}
+
+constexpr int kRowsPerCta = 4;
+
+__global__ void __launch_bounds__(128)
+classify_rows_kernel(const double* __restrict__ logits, int rows, int nb, int kc, int kn,
+                     int8_t* __restrict__ mask, int32_t* __restrict__ crit_idx, int32_t* __restrict__ crit_cnt,
+                     __nv_bfloat16* __restrict__ m01, int ld_m01, float* __restrict__ scores) {
+  extern __shared__ uint8_t smem[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  uint64_t* keys = reinterpret_cast<uint64_t*>(smem) + (size_t)warp * nb;
+  unsigned* hist = reinterpret_cast<unsigned*>(reinterpret_cast<uint64_t*>(smem) + (size_t)kRowsPerCta * nb) + warp * 256;
+  const int row = blockIdx.x * kRowsPerCta + warp;
+  if (row >= rows) return;
+  const double* lg = logits + (size_t)row * nb;
+  double mx = -INFINITY;
+  for (int j = lane; j < nb; j += 32) {
+    const double x = lg[j];
+    keys[j] = order_key(x);
+    mx = fmax(mx, x);
+  }
+  #pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = fmax(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
+  double sum = 0.0;
+  if (scores) {
+    for (int j = lane; j < nb; j += 32) sum += exp(lg[j] - mx);
+    #pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
+  }
+  __syncwarp();
+  uint64_t Tc = 0, Tn = 0;
+  int take_c = 0, eq_c = 0, take_n = 0, eq_n = 0;
+  radix_select(keys, nb, kc, true, hist, lane, Tc, take_c, eq_c);
+  if (kn > 0) radix_select(keys, nb, kn, false, hist, lane, Tn, take_n, eq_n);
+  const unsigned lt_mask = (1u << lane) - 1u;
+  int seen_c = 0, seen_n = 0, written = 0;
+  for (int base = 0; base < nb; base += 32) {
+    const int j = base + lane;
+    const bool in = j < nb;
+    const uint64_t u = in ? keys[j] : 0;
+    const bool eqc = in && u == Tc;
+    const unsigned bc = __ballot_sync(0xFFFFFFFFu, eqc);
+    const bool crit = (in && u > Tc) || (eqc && seen_c + __popc(bc & lt_mask) < take_c);
+    seen_c += __popc(bc);
+    bool negl = false;
+    if (kn > 0) {
+      const bool eqn = in && u == Tn;
+      const unsigned bn = __ballot_sync(0xFFFFFFFFu, eqn);
+      negl = (in && u < Tn) || (eqn && seen_n + __popc(bn & lt_mask) >= eq_n - take_n);
+      seen_n += __popc(bn);
+    }
+    if (in) {
+      const int8_t m = crit ? 1 : (negl ? -1 : 0);
+      mask[(size_t)row * nb + j] = m;
+      if (m01) m01[(size_t)row * ld_m01 + j] = __float2bfloat16_rn(m == 0 ? 1.f : 0.f);
+      if (scores) scores[(size_t)row * nb + j] = (float)(exp(lg[j] - mx) / sum);
+    }
+    const unsigned bcrit = __ballot_sync(0xFFFFFFFFu, crit);
+    if (crit) crit_idx[(size_t)row * kc + written + __popc(bcrit & lt_mask)] = j;
+    written += __popc(bcrit);
+  }
+  if (m01)
+    for (int j = nb + lane; j < ld_m01; j += 32) m01[(size_t)row * ld_m01 + j] = __float2bfloat16_rn(0.f);
+  if (lane == 0) crit_cnt[row] = kc;
+}
+
+__global__ void mask_to_m01_kernel(const int8_t* __restrict__ mask, __nv_bfloat16* __restrict__ m01,
+                                   int rows, int nb, int ld) {
+  const size_t total = (size_t)rows * ld;
+  for (size_t e = blockIdx.x * (size_t)blockDim.x + threadIdx.x; e < total; e += (size_t)gridDim.x * blockDim.x) {
+    const size_t r = e / ld;
+    const int j = (int)(e % ld);
+    const float v = (j < nb && mask[r * nb + j] == 0) ? 1.f : 0.f;
+    m01[e] = __float2bfloat16_rn(v);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_block_logits(const double* qbar, const double* kbar, double* logits,
+                                int BH, int nb, int d, cudaStream_t st) {
+  dim3 grid((nb + 63) / 64, (nb + 63) / 64, BH);
+  block_logits_kernel<<<grid, 256, 0, st>>>(qbar, kbar, logits, nb, d, sqrt((double)d));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_classify_rows(const double* logits, int BH, int nb, int kc, int kn,
+                                 int8_t* mask, int32_t* crit_idx, int32_t* crit_cnt,
+                                 __nv_bfloat16* m01, int ld_m01, float* scores, cudaStream_t st) {
+  const int rows = BH * nb;
+  const size_t smem = (size_t)kRowsPerCta * nb * sizeof(uint64_t) + (size_t)kRowsPerCta * 256 * sizeof(unsigned);
+  cudaError_t e = cudaFuncSetAttribute(classify_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  classify_rows_kernel<<<(rows + kRowsPerCta - 1) / kRowsPerCta, 128, smem, st>>>(
+      logits, rows, nb, kc, kn, mask, crit_idx, crit_cnt, m01, ld_m01, scores);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_mask_to_m01(const int8_t* mask, __nv_bfloat16* m01, int BH, int nb, int ld_m01,
+                               cudaStream_t st) {
+  const int rows = BH * nb;
+  const size_t total = (size_t)rows * ld_m01;
+  int blocks = (int)((total + 255) / 256);
+  if (blocks > 148 * 16) blocks = 148 * 16;
+  mask_to_m01_kernel<<<blocks, 256, 0, st>>>(mask, m01, rows, nb, ld_m01);
+  return cudaGetLastError();
+}
+
+}  // namespace slr

@@ -1,0 +1,520 @@
+// k_marginal.cu -- the linear-attention branch of SLA on tcgen05 (sm_100a).
+//
+// SLA page section 3 ("边缘权重 ... 线性注意力"): for marginal block pairs the
+// attention is replaced by linear attention with feature map phi, evaluated as
+// "K^T V first, then apply Q".  Three kernels:
+//
+//  key_states_kernel    per key block j: h_j^T = V_j^T phi(K_j) (d x d, one MMA
+//                       M=128 N=d K=64 with both operands MN-major straight from
+//                       the TMA tiles; phi is applied in place in shared memory)
+//                       and z_j = sum_t phi(K_j,t); written as bf16 rows
+//                       [h_j^T ; z_j] of (d+1)*d elements.
+//  reduce_states_kernel per head: Hs = M01 . h, a plain tensor-core GEMM with
+//                       the 0/1 marginal indicator M01 [Nqb x Nkb] (K-major) and
+//                       h [Nkb x (d+1)d] (MN-major), fp32 accumulation in TMEM,
+//                       bf16 out.  Row i of Hs is [H_i^T ; Z_i].
+//  linear_apply_kernel  per query block i: O_l^T = H_i^T phi(Q_i)^T (MMA M=128 over
+//                       the output channel, N=64 tokens), normalised by
+//                       phi(q_t).Z_i, then optionally projected,
+//                       (O_l W)^T = W^T O_l^T (second MMA, W MN-major), written
+//                       as fp32 [token][channel].
+// d = 64 runs the same M=128 MMAs with the upper 64 rows of A zero-filled.
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+
+#include "launch.h"
+#include "sm100.cuh"
+
+namespace slr {
+namespace {
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+// Block-wide bounded wait: every thread polls; any timeout aborts all.
+__device__ __forceinline__ bool cta_wait(uint64_t* bar, uint32_t parity, volatile int* abort, int* status) {
+  return __all_sync(0xFFFFFFFFu, mbar_wait(bar, parity, abort, status));
+}
+
+// ------------------------------------------------------------------ key states
+constexpr int kKsBytes = 2 * 8192 + 2 * 8192 + 16 * 128 * 4 + 256 + 1024;
+constexpr int kKsSmemRequest = 56 * 1024;   // keeps at most 4 CTAs (4 x 128 TMEM columns) per SM
+
+template <int D>
+__global__ void __launch_bounds__(128, 4)
+key_states_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                  __nv_bfloat16* __restrict__ h, SeqShape s, int* status) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint8_t* sK = smem;                      // phi(K_j) after the transform, 64 rows (t) x D
+  uint8_t* sV = smem + 2 * 8192;           // V_j, 64 rows (t) x D; chunk 1 zero when D = 64
+  float* zred = reinterpret_cast<float*>(smem + 4 * 8192);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 4 * 8192 + 16 * 128 * 4);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  const int blk = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x, warp = tid >> 5;
+
+  if (tid == 0) {
+    mbar_init(&bars[0], 1);
+    mbar_init(&bars[1], 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (D == 64)
+    for (int i = tid; i < 8192 / 16; i += 128) reinterpret_cast<uint4*>(sV + 8192)[i] = make_uint4(0, 0, 0, 0);
+  if (warp == 0) { tmem_alloc(tmem_slot, 128); tmem_relinquish(); }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (tid == 0) {
+    mbar_arrive_expect_tx(&bars[0], 2 * (D / 64) * 8192);
+    for (int c = 0; c < D / 64; ++c) {
+      tma_load_3d(sK + c * 8192, &tmK, &bars[0], c * 64, blk * 64, bh);
+      tma_load_3d(sV + c * 8192, &tmV, &bars[0], c * 64, blk * 64, bh);
+    }
+  }
+  bool ok = cta_wait(&bars[0], 0, abort_flag, status);
+
+  // phi in place (pad tokens -> 0) and column sums z
+  constexpr int kCPR = D / 8, kRS = 128 / kCPR;
+  const int g = tid % kCPR, rs = tid / kCPR;
+  const int chunk = g >> 3, q8 = g & 7;
+  const int nvalid = block_valid_count(s, blk);
+  float z[8];
+  #pragma unroll
+  for (int i = 0; i < 8; ++i) z[i] = 0.f;
+  if (ok) {
+    for (int t = rs; t < 64; t += kRS) {
+      uint4* p = reinterpret_cast<uint4*>(sK + chunk * 8192 + sw128_offset(t, q8));
+      const uint4 u = *p;
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+      uint32_t o[4];
+      #pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float a = t < nvalid ? phi_elu1(bf16_lo(w[i])) : 0.f;
+        const float b = t < nvalid ? phi_elu1(bf16_hi(w[i])) : 0.f;
+        z[2 * i] += a;
+        z[2 * i + 1] += b;
+        o[i] = pack_bf16(a, b);
+      }
+      *p = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+  }
+  #pragma unroll
+  for (int i = 0; i < 8; ++i) zred[rs * D + g * 8 + i] = z[i];
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+
+  if (tid == 0 && ok) {
+    tc_fence_after();
+    constexpr uint32_t id = idesc_bf16(128, D, true, true);
+    #pragma unroll
+    for (int kk = 0; kk < 4; ++kk) {
+      const uint64_t a = desc_mnmajor(smem_u32(sV) + kk * 2048, 8192);
+      const uint64_t b = desc_mnmajor(smem_u32(sK) + kk * 2048, 8192);
+      mma_bf16_ss(tmem, a, b, id, kk > 0 ? 1u : 0u);
+    }
+    mma_commit(&bars[1]);
+  }
+  __nv_bfloat16* hrow = h + ((size_t)bh * s.n_blocks + blk) * (size_t)(D + 1) * D;
+  for (int a = tid; a < D; a += 128) {
+    float sum = 0.f;
+    #pragma unroll
+    for (int r = 0; r < kRS; ++r) sum += zred[r * D + a];
+    hrow[(size_t)D * D + a] = __float2bfloat16_rn(sum);
+  }
+  if (ok) ok = cta_wait(&bars[1], 0, abort_flag, status);
+  tc_fence_after();
+  if (ok && warp * 32 < D) {
+    const int c = tid;                       // TMEM lane = output row (value channel)
+    #pragma unroll 1
+    for (int cc = 0; cc < D / 32; ++cc) {
+      uint32_t r[32];
+      tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + cc * 32, r);
+      tmem_wait_ld();
+      uint4* dst = reinterpret_cast<uint4*>(hrow + (size_t)c * D + cc * 32);
+      #pragma unroll
+      for (int i = 0; i < 4; ++i)
+        dst[i] = make_uint4(pack_bf16(__uint_as_float(r[8 * i]), __uint_as_float(r[8 * i + 1])),
+                            pack_bf16(__uint_as_float(r[8 * i + 2]), __uint_as_float(r[8 * i + 3])),
+                            pack_bf16(__uint_as_float(r[8 * i + 4]), __uint_as_float(r[8 * i + 5])),
+                            pack_bf16(__uint_as_float(r[8 * i + 6]), __uint_as_float(r[8 * i + 7])));
+    }
+  }
+  if (!ok && tid == 0) {
+    mma_commit(&bars[1]);
+    const long long t0 = clock64();
+    while (!mbar_try_wait(&bars[1], 0) && clock64() - t0 < kWaitBudgetCycles) {}
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) { tc_fence_after(); tmem_dealloc(tmem, 128); }
+}
+
+// ------------------------------------------------------------------ reduce states (GEMM)
+constexpr int kGemmStages = 2;
+constexpr int kGemmBN = 256;
+constexpr int kGemmABytes = 128 * 128;          // 128 rows x 64 bf16
+constexpr int kGemmBBytes = 4 * 64 * 128;       // 4 chunks of 64 K-rows x 64 bf16
+constexpr int kGemmSmem = kGemmStages * (kGemmABytes + kGemmBBytes) + 256 + 1024;
+
+__global__ void __launch_bounds__(192, 2)
+reduce_states_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                     __nv_bfloat16* __restrict__ Hs, int nb, int ntot, int* status) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + kGemmStages * kGemmABytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kGemmStages * (kGemmABytes + kGemmBBytes));
+  uint64_t* full = bars;
+  uint64_t* empty = bars + kGemmStages;
+  uint64_t* acc = bars + 2 * kGemmStages;
+  uint64_t* drain = acc + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m0 = blockIdx.x * 128, n0 = blockIdx.y * kGemmBN, bh = blockIdx.z;
+  const int kt_total = (nb + 63) / 64;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kGemmStages; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+    mbar_init(acc, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 5) { tmem_alloc(tmem_slot, 256); tmem_relinquish(); }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 4) {
+    if (lane == 0) {
+      int kt = 0;
+      for (; kt < kt_total; ++kt) {
+        const int s = kt % kGemmStages;
+        if (kt >= kGemmStages && !mbar_wait(&empty[s], ((kt / kGemmStages) - 1) & 1, abort_flag, status)) break;
+        mbar_arrive_expect_tx(&full[s], kGemmABytes + kGemmBBytes);
+        tma_load_3d(sA + s * kGemmABytes, &tmA, &full[s], kt * 64, m0, bh);
+        for (int c = 0; c < 4; ++c)
+          tma_load_3d(sB + s * kGemmBBytes + c * 8192, &tmB, &full[s], n0 + c * 64, kt * 64, bh);
+      }
+      if (*abort_flag) {
+        for (int i = (kt - kGemmStages > 0 ? kt - kGemmStages : 0); i < kt; ++i) {
+          const long long t0 = clock64();
+          while (!mbar_try_wait(&full[i % kGemmStages], (i / kGemmStages) & 1) && clock64() - t0 < kWaitBudgetCycles) {}
+        }
+      }
+    }
+  } else if (warp == 5) {
+    if (lane == 0) {
+      constexpr uint32_t id = idesc_bf16(128, kGemmBN, false, true);
+      bool ok = true;
+      for (int kt = 0; kt < kt_total; ++kt) {
+        const int s = kt % kGemmStages;
+        if (!mbar_wait(&full[s], (kt / kGemmStages) & 1, abort_flag, status)) { ok = false; break; }
+        tc_fence_after();
+        #pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint64_t a = desc_kmajor(smem_u32(sA + s * kGemmABytes) + kk * 32);
+          const uint64_t b = desc_mnmajor(smem_u32(sB + s * kGemmBBytes) + kk * 2048, 8192);
+          mma_bf16_ss(tmem, a, b, id, (kt > 0 || kk > 0) ? 1u : 0u);
+        }
+        mma_commit(&empty[s]);
+      }
+      mma_commit(ok ? acc : drain);
+      if (!ok) {
+        const long long t0 = clock64();
+        while (!mbar_try_wait(drain, 0) && clock64() - t0 < kWaitBudgetCycles) {}
+      }
+    }
+  } else {
+    const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(acc, 0, abort_flag, status));
+    tc_fence_after();
+    const int r = threadIdx.x;
+    const int m = m0 + r;
+    if (ok) {
+      #pragma unroll 1
+      for (int cc = 0; cc < kGemmBN / 32; ++cc) {
+        uint32_t v[32];
+        tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + cc * 32, v);
+        tmem_wait_ld();
+        const int n = n0 + cc * 32;
+        if (m < nb && n < ntot) {
+          uint4* dst = reinterpret_cast<uint4*>(Hs + ((size_t)bh * nb + m) * ntot + n);
+          #pragma unroll
+          for (int i = 0; i < 4; ++i)
+            dst[i] = make_uint4(pack_bf16(__uint_as_float(v[8 * i]), __uint_as_float(v[8 * i + 1])),
+                                pack_bf16(__uint_as_float(v[8 * i + 2]), __uint_as_float(v[8 * i + 3])),
+                                pack_bf16(__uint_as_float(v[8 * i + 4]), __uint_as_float(v[8 * i + 5])),
+                                pack_bf16(__uint_as_float(v[8 * i + 6]), __uint_as_float(v[8 * i + 7])));
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) { tc_fence_after(); tmem_dealloc(tmem, 256); }
+}
+
+// ------------------------------------------------------------------ linear apply (+ projection)
+template <int D>
+struct ApplyLayout {
+  static constexpr int kQOff = 0;                         // phi(Q_i): D/64 chunks x 64 rows
+  static constexpr int kHOff = kQOff + 2 * 8192;          // H_i^T: D/64 chunks x 128 rows
+  static constexpr int kWOff = kHOff + 2 * 16384;         // W (MN-major): 2 chunks x D rows
+  static constexpr int kOOff = kWOff + 2 * D * 128;       // O_l (K-major): D/64 chunks x 64 rows
+  static constexpr int kZOff = kOOff + 2 * 8192;          // z (D floats) + den (64 floats)
+  static constexpr int kBarOff = kZOff + (D + 64) * 4;
+  static constexpr int kBytes = kBarOff + 64 + 1024;
+};
+
+template <int D>
+__global__ void __launch_bounds__(128, 2)
+linear_apply_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmH,
+                    const __grid_constant__ CUtensorMap tmW, const __nv_bfloat16* __restrict__ Hs,
+                    float* __restrict__ o_lin, SeqShape s, int has_w, int* status) {
+  using L = ApplyLayout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint8_t* sQ = smem + L::kQOff;
+  uint8_t* sH = smem + L::kHOff;
+  uint8_t* sW = smem + L::kWOff;
+  uint8_t* sO = smem + L::kOOff;
+  float* zs = reinterpret_cast<float*>(smem + L::kZOff);
+  float* den = zs + D;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  const int blk = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x, warp = tid >> 5;
+  const size_t hs_row = (size_t)bh * s.n_blocks + blk;
+
+  if (tid == 0) {
+    for (int i = 0; i < 3; ++i) mbar_init(&bars[i], 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (D == 64 && has_w)
+    for (int i = tid; i < 8192 / 16; i += 128) reinterpret_cast<uint4*>(sW + D * 128)[i] = make_uint4(0, 0, 0, 0);
+  if (warp == 0) { tmem_alloc(tmem_slot, 128); tmem_relinquish(); }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (tid == 0) {
+    const uint32_t bytes = (D / 64) * (8192 + 16384) + (has_w ? (D / 64) * D * 128 : 0);
+    mbar_arrive_expect_tx(&bars[0], bytes);
+    for (int c = 0; c < D / 64; ++c) {
+      tma_load_3d(sQ + c * 8192, &tmQ, &bars[0], c * 64, blk * 64, bh);
+      tma_load_3d(sH + c * 16384, &tmH, &bars[0], c * 64, 0, (int)hs_row);
+      if (has_w) tma_load_3d(sW + c * D * 128, &tmW, &bars[0], c * 64, 0, 0);
+    }
+  }
+  for (int a = tid; a < D; a += 128) zs[a] = __bfloat162float(Hs[(hs_row * (D + 1) + D) * D + a]);
+  bool ok = cta_wait(&bars[0], 0, abort_flag, status);
+
+  // phi(Q_i) in place; pad tokens -> 0
+  constexpr int kCPR = D / 8, kRS = 128 / kCPR;
+  const int nvalid = block_valid_count(s, blk);
+  {
+    const int g = tid % kCPR, rs = tid / kCPR, chunk = g >> 3, q8 = g & 7;
+    if (ok)
+      for (int t = rs; t < 64; t += kRS) {
+        uint4* p = reinterpret_cast<uint4*>(sQ + chunk * 8192 + sw128_offset(t, q8));
+        const uint4 u = *p;
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+        uint32_t o[4];
+        #pragma unroll
+        for (int i = 0; i < 4; ++i)
+          o[i] = t < nvalid ? pack_bf16(phi_elu1(bf16_lo(w[i])), phi_elu1(bf16_hi(w[i]))) : 0u;
+        *p = make_uint4(o[0], o[1], o[2], o[3]);
+      }
+  }
+  __syncthreads();
+  // den[t] = phi(q_t) . Z_i  (two threads per token)
+  {
+    const int t = tid >> 1, hlf = tid & 1;
+    float part = 0.f;
+    for (int g = hlf * (kCPR / 2); g < (hlf + 1) * (kCPR / 2); ++g) {
+      const uint4 u = *reinterpret_cast<const uint4*>(sQ + (g >> 3) * 8192 + sw128_offset(t, g & 7));
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+      #pragma unroll
+      for (int i = 0; i < 4; ++i) part += bf16_lo(w[i]) * zs[g * 8 + 2 * i] + bf16_hi(w[i]) * zs[g * 8 + 2 * i + 1];
+    }
+    part += __shfl_xor_sync(0xFFFFFFFFu, part, 1);
+    if (hlf == 0) den[t] = part;
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  if (tid == 0 && ok) {
+    tc_fence_after();
+    constexpr uint32_t id = idesc_bf16(128, 64, false, false);
+    #pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+      const uint64_t a = desc_kmajor(smem_u32(sH) + (kk >> 2) * 16384 + (kk & 3) * 32);
+      const uint64_t b = desc_kmajor(smem_u32(sQ) + (kk >> 2) * 8192 + (kk & 3) * 32);
+      mma_bf16_ss(tmem, a, b, id, kk > 0 ? 1u : 0u);
+    }
+    mma_commit(&bars[1]);
+  }
+  if (ok) ok = cta_wait(&bars[1], 0, abort_flag, status);
+  tc_fence_after();
+  const int c = tid;                              // TMEM lane = output channel
+  const bool lane_active = warp * 32 < D;
+  float vals[64];
+  if (lane_active) {
+    if (ok) {
+      uint32_t r[32];
+      tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16), r);
+      tmem_wait_ld();
+      #pragma unroll
+      for (int t = 0; t < 32; ++t) vals[t] = den[t] > 0.f ? __uint_as_float(r[t]) / den[t] : 0.f;
+      tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + 32, r);
+      tmem_wait_ld();
+      #pragma unroll
+      for (int t = 0; t < 32; ++t) vals[32 + t] = den[32 + t] > 0.f ? __uint_as_float(r[t]) / den[32 + t] : 0.f;
+    } else {
+      #pragma unroll
+      for (int t = 0; t < 64; ++t) vals[t] = 0.f;
+    }
+  }
+  float* out = o_lin + ((size_t)bh * s.n_pad + (size_t)blk * 64) * D;
+  if (!has_w) {
+    if (lane_active)
+      #pragma unroll 4
+      for (int t = 0; t < 64; ++t) out[(size_t)t * D + c] = t < nvalid ? vals[t] : 0.f;
+  } else {
+    if (lane_active) {
+      __nv_bfloat16* base = reinterpret_cast<__nv_bfloat16*>(sO + (c >> 6) * 8192);
+      const int q8 = (c & 63) >> 3, e = c & 7;
+      #pragma unroll 8
+      for (int t = 0; t < 64; ++t)
+        base[(sw128_offset(t, q8) >> 1) + e] = __float2bfloat16_rn(vals[t]);
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0 && ok) {
+      tc_fence_after();
+      constexpr uint32_t id = idesc_bf16(128, 64, true, false);
+      #pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint64_t a = desc_mnmajor(smem_u32(sW) + kk * 2048, D * 128);
+        const uint64_t b = desc_kmajor(smem_u32(sO) + (kk >> 2) * 8192 + (kk & 3) * 32);
+        mma_bf16_ss(tmem + 64, a, b, id, kk > 0 ? 1u : 0u);
+      }
+      mma_commit(&bars[2]);
+    }
+    if (ok) ok = cta_wait(&bars[2], 0, abort_flag, status);
+    tc_fence_after();
+    if (lane_active) {
+      if (ok) {
+        #pragma unroll 1
+        for (int h2 = 0; h2 < 2; ++h2) {
+          uint32_t r[32];
+          tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + 64 + h2 * 32, r);
+          tmem_wait_ld();
+          #pragma unroll 4
+          for (int t = 0; t < 32; ++t) {
+            const int tt = h2 * 32 + t;
+            out[(size_t)tt * D + c] = tt < nvalid ? __uint_as_float(r[t]) : 0.f;
+          }
+        }
+      } else {
+        for (int t = 0; t < 64; ++t) out[(size_t)t * D + c] = 0.f;
+      }
+    }
+  }
+  if (!ok && tid == 0) {
+    mma_commit(&bars[2]);
+    const long long t0 = clock64();
+    while (!mbar_try_wait(&bars[2], has_w ? 1 : 0) && clock64() - t0 < kWaitBudgetCycles) {}
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) { tc_fence_after(); tmem_dealloc(tmem, 128); }
+}
+
+}  // namespace
+
+cudaError_t launch_key_states(const void* k, const void* v, __nv_bfloat16* h, int BH, int d, SeqShape s,
+                              int* status, cudaStream_t st) {
+  CUtensorMap mk, mv;
+  const uint64_t dims[3] = {(uint64_t)d, (uint64_t)s.n_pad, (uint64_t)BH};
+  const uint64_t strides[2] = {(uint64_t)d * 2, (uint64_t)d * 2 * s.n_pad};
+  const uint32_t box[3] = {64, 64, 1};
+  if (!make_tile_map(&mk, k, 3, dims, strides, box) || !make_tile_map(&mv, v, 3, dims, strides, box))
+    return cudaErrorInvalidValue;
+  dim3 grid(s.n_blocks, BH);
+  if (d == 128) {
+    cudaError_t e = cudaFuncSetAttribute(key_states_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, kKsSmemRequest);
+    if (e != cudaSuccess) return e;
+    key_states_kernel<128><<<grid, 128, kKsSmemRequest, st>>>(mk, mv, h, s, status);
+  } else {
+    cudaError_t e = cudaFuncSetAttribute(key_states_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, kKsSmemRequest);
+    if (e != cudaSuccess) return e;
+    key_states_kernel<64><<<grid, 128, kKsSmemRequest, st>>>(mk, mv, h, s, status);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_reduce_states(const __nv_bfloat16* m01, int ld_m01, const __nv_bfloat16* h,
+                                 __nv_bfloat16* Hs, int BH, int nb, int d, int* status, cudaStream_t st) {
+  const int ntot = (d + 1) * d;
+  CUtensorMap ma, mb;
+  const uint64_t adims[3] = {(uint64_t)ld_m01, (uint64_t)nb, (uint64_t)BH};
+  const uint64_t astr[2] = {(uint64_t)ld_m01 * 2, (uint64_t)ld_m01 * 2 * nb};
+  const uint32_t abox[3] = {64, 128, 1};
+  const uint64_t bdims[3] = {(uint64_t)ntot, (uint64_t)nb, (uint64_t)BH};
+  const uint64_t bstr[2] = {(uint64_t)ntot * 2, (uint64_t)ntot * 2 * nb};
+  const uint32_t bbox[3] = {64, 64, 1};
+  if (!make_tile_map(&ma, m01, 3, adims, astr, abox) || !make_tile_map(&mb, h, 3, bdims, bstr, bbox))
+    return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(reduce_states_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem);
+  if (e != cudaSuccess) return e;
+  dim3 grid((nb + 127) / 128, (ntot + kGemmBN - 1) / kGemmBN, BH);
+  reduce_states_kernel<<<grid, 192, kGemmSmem, st>>>(ma, mb, Hs, nb, ntot, status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_linear_apply(const void* q, const __nv_bfloat16* Hs, const void* w_proj,
+                                float* o_lin, int BH, int d, SeqShape s, int* status, cudaStream_t st) {
+  CUtensorMap mq, mh, mw;
+  const uint64_t qdims[3] = {(uint64_t)d, (uint64_t)s.n_pad, (uint64_t)BH};
+  const uint64_t qstr[2] = {(uint64_t)d * 2, (uint64_t)d * 2 * s.n_pad};
+  const uint32_t qbox[3] = {64, 64, 1};
+  const uint64_t hdims[3] = {(uint64_t)d, (uint64_t)(d + 1), (uint64_t)BH * s.n_blocks};
+  const uint64_t hstr[2] = {(uint64_t)d * 2, (uint64_t)d * 2 * (d + 1)};
+  const uint32_t hbox[3] = {64, 128, 1};
+  if (!make_tile_map(&mq, q, 3, qdims, qstr, qbox) || !make_tile_map(&mh, Hs, 3, hdims, hstr, hbox))
+    return cudaErrorInvalidValue;
+  if (w_proj) {
+    const uint64_t wdims[3] = {(uint64_t)d, (uint64_t)d, 1};
+    const uint64_t wstr[2] = {(uint64_t)d * 2, (uint64_t)d * 2 * d};
+    const uint32_t wbox[3] = {64, (uint32_t)d, 1};
+    if (!make_tile_map(&mw, w_proj, 3, wdims, wstr, wbox)) return cudaErrorInvalidValue;
+  } else {
+    mw = mq;
+  }
+  dim3 grid(s.n_blocks, BH);
+  const int has_w = w_proj ? 1 : 0;
+  if (d == 128) {
+    cudaError_t e = cudaFuncSetAttribute(linear_apply_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, ApplyLayout<128>::kBytes);
+    if (e != cudaSuccess) return e;
+    linear_apply_kernel<128><<<grid, 128, ApplyLayout<128>::kBytes, st>>>(mq, mh, mw, Hs, o_lin, s, has_w, status);
+  } else {
+    cudaError_t e = cudaFuncSetAttribute(linear_apply_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, ApplyLayout<64>::kBytes);
+    if (e != cudaSuccess) return e;
+    linear_apply_kernel<64><<<grid, 128, ApplyLayout<64>::kBytes, st>>>(mq, mh, mw, Hs, o_lin, s, has_w, status);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace slr

@@ -1,0 +1,123 @@
+// k_pool.cu -- bandwidth-bound pooling kernels.
+//
+// pool_means_kernel: the block mean-pooling of Q and K that feeds SLA's
+// compressed score matrix (SLA page section 3: "对查询（Q）和键（K）矩阵进行平均
+// 池化").  One CTA reads one 64-token block (16-byte vector loads, valid tokens
+// only) and writes its mean in fp64.  Sums of at most 64 bf16 values are exact
+// in fp64, so the pooled means do not depend on summation order.
+//
+// far_pool_kernel: the far field of the RoPeSLR gated mode -- K and V averaged
+// over cells of (cf, ch, cw) raster tokens (aixinbiao page: K and V compressed
+// by token mean-pooling into a small low-rank set), rounded to bf16 because
+// they are tensor-core operands of the attention kernel.
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+
+#include "launch.h"
+#include "sm100.cuh"
+
+namespace slr {
+namespace {
+
+template <int D>
+__global__ void __launch_bounds__(128)
+pool_means_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
+                  double* __restrict__ qbar, double* __restrict__ kbar, SeqShape s) {
+  constexpr int kCPR = D / 8;          // 16-byte chunks per row
+  constexpr int kRG = 128 / kCPR;      // row groups
+  __shared__ double red[kRG][D];
+  const int blk = blockIdx.x, bh = blockIdx.y;
+  const __nv_bfloat16* x = (blockIdx.z == 0 ? q : k) + ((size_t)bh * s.n_pad + (size_t)blk * kBlock) * D;
+  double* out = (blockIdx.z == 0 ? qbar : kbar) + ((size_t)bh * s.n_blocks + blk) * D;
+  const int chunk = threadIdx.x % kCPR, rg = threadIdx.x / kCPR;
+  const int nvalid = block_valid_count(s, blk);   // valid tokens form a prefix of the block
+  double acc[8];
+  #pragma unroll
+  for (int i = 0; i < 8; ++i) acc[i] = 0.0;
+  for (int r = rg; r < nvalid; r += kRG) {
+    const uint4 u = __ldg(reinterpret_cast<const uint4*>(x + (size_t)r * D + chunk * 8));
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+    #pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      acc[2 * i] += (double)bf16_lo(w[i]);
+      acc[2 * i + 1] += (double)bf16_hi(w[i]);
+    }
+  }
+  #pragma unroll
+  for (int i = 0; i < 8; ++i) red[rg][chunk * 8 + i] = acc[i];
+  __syncthreads();
+  for (int c = threadIdx.x; c < D; c += 128) {
+    double sum = 0.0;
+    #pragma unroll
+    for (int g = 0; g < kRG; ++g) sum += red[g][c];
+    out[c] = sum / (double)nvalid;
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(128)
+far_pool_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
+                __nv_bfloat16* __restrict__ kf, __nv_bfloat16* __restrict__ vf,
+                int F, int Hh, int Ww, int cf, int ch, int cw) {
+  constexpr int kCPR = D / 8;
+  constexpr int kRG = 128 / kCPR;
+  __shared__ float red[kRG][D];
+  const int cell = blockIdx.x, bh = blockIdx.y;
+  const int gh = Hh / ch, gw = Ww / cw;
+  const int c_f = cell / (gh * gw), c_h = (cell / gw) % gh, c_w = cell % gw;
+  const size_t n = (size_t)F * Hh * Ww;
+  const __nv_bfloat16* x = (blockIdx.z == 0 ? k : v) + (size_t)bh * n * D;
+  __nv_bfloat16* out = (blockIdx.z == 0 ? kf : vf) + ((size_t)bh * gridDim.x + cell) * D;
+  const int chunk = threadIdx.x % kCPR, rg = threadIdx.x / kCPR;
+  const int per_cell = cf * ch * cw;
+  float acc[8];
+  #pragma unroll
+  for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+  for (int r = rg; r < per_cell; r += kRG) {
+    const int df = r / (ch * cw), dh = (r / cw) % ch, dw = r % cw;
+    const size_t tok = ((size_t)(c_f * cf + df) * Hh + (c_h * ch + dh)) * Ww + (c_w * cw + dw);
+    const uint4 u = __ldg(reinterpret_cast<const uint4*>(x + tok * D + chunk * 8));
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+    #pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      acc[2 * i] += bf16_lo(w[i]);
+      acc[2 * i + 1] += bf16_hi(w[i]);
+    }
+  }
+  #pragma unroll
+  for (int i = 0; i < 8; ++i) red[rg][chunk * 8 + i] = acc[i];
+  __syncthreads();
+  for (int c = threadIdx.x; c < D; c += 128) {
+    float sum = 0.f;
+    #pragma unroll
+    for (int g = 0; g < kRG; ++g) sum += red[g][c];
+    out[c] = __float2bfloat16_rn(sum / (float)per_cell);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_pool_means(const void* q, const void* k, double* qbar, double* kbar,
+                              int BH, int d, SeqShape s, cudaStream_t st) {
+  dim3 grid(s.n_blocks, BH, 2);
+  if (d == 128)
+    pool_means_kernel<128><<<grid, 128, 0, st>>>((const __nv_bfloat16*)q, (const __nv_bfloat16*)k, qbar, kbar, s);
+  else
+    pool_means_kernel<64><<<grid, 128, 0, st>>>((const __nv_bfloat16*)q, (const __nv_bfloat16*)k, qbar, kbar, s);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_far_pool(const void* k, const void* v, void* kf, void* vf, int BH, int d,
+                            int F, int Hh, int Ww, int cf, int ch, int cw, cudaStream_t st) {
+  const int ncells = (F / cf) * (Hh / ch) * (Ww / cw);
+  dim3 grid(ncells, BH, 2);
+  if (d == 128)
+    far_pool_kernel<128><<<grid, 128, 0, st>>>((const __nv_bfloat16*)k, (const __nv_bfloat16*)v,
+                                               (__nv_bfloat16*)kf, (__nv_bfloat16*)vf, F, Hh, Ww, cf, ch, cw);
+  else
+    far_pool_kernel<64><<<grid, 128, 0, st>>>((const __nv_bfloat16*)k, (const __nv_bfloat16*)v,
+                                              (__nv_bfloat16*)kf, (__nv_bfloat16*)vf, F, Hh, Ww, cf, ch, cw);
+  return cudaGetLastError();
+}
+
+}  // namespace slr

@@ -1,0 +1,109 @@
+// launch.h -- host-side launch interface between the C ABI (slr_api.cu) and the
+// kernels (k_*.cu).  Every launcher queues its kernels on `stream` and returns a
+// cudaError_t from the launch; none synchronises.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace slr {
+
+// ------------------------------------------------------------ tensor maps
+// A tile map over a bf16 tensor whose innermost dimension is contiguous.
+// dims[0] is the innermost extent (elements), strides are in bytes for dims 1..rank-1.
+bool make_tile_map(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
+                   const uint64_t* strides_bytes, const uint32_t* box);
+
+// ------------------------------------------------------------ pooling (k_pool.cu)
+// Means of the valid tokens of every 64-token block of q and k, fp64 [BH][Nb][d].
+cudaError_t launch_pool_means(const void* q, const void* k, double* qbar, double* kbar,
+                              int BH, int d, SeqShape s, cudaStream_t st);
+
+// Far-field K/V: means over cells of (cf, ch, cw) tokens of the raster (F, Hh, Ww),
+// bf16 [BH][ncells][d], cells in raster order of the cell grid.
+cudaError_t launch_far_pool(const void* k, const void* v, void* kf, void* vf, int BH, int d,
+                            int F, int Hh, int Ww, int cf, int ch, int cw, cudaStream_t st);
+
+// ------------------------------------------------------------ classification (k_classify.cu)
+// logits[bh][i][j] = qbar_i . kbar_j / sqrt(d) in fp64.
+cudaError_t launch_block_logits(const double* qbar, const double* kbar, double* logits,
+                                int BH, int nb, int d, cudaStream_t st);
+
+// Per row: top kc -> 1, bottom kn -> -1, rest 0; critical list ascending; the
+// marginal indicator m01 (bf16 1/0, row stride ld_m01, pad columns 0); optional
+// P_c in fp32.
+cudaError_t launch_classify_rows(const double* logits, int BH, int nb, int kc, int kn,
+                                 int8_t* mask, int32_t* crit_idx, int32_t* crit_cnt,
+                                 __nv_bfloat16* m01, int ld_m01, float* scores, cudaStream_t st);
+
+// m01 = (mask == 0) as bf16 with row stride ld_m01 (pad columns zeroed).
+cudaError_t launch_mask_to_m01(const int8_t* mask, __nv_bfloat16* m01, int BH, int nb, int ld_m01,
+                               cudaStream_t st);
+
+// ------------------------------------------------------------ block lists (k_lists.cu)
+// Entries of a pair list: key block index in bits [0,30), bit 30 = the first query
+// block of the pair attends it, bit 31 = the second does.
+enum ListMode { kListExplicit = 0, kListLvsa = 1, kListTile3d = 2 };
+
+struct ListArgs {
+  int mode;
+  int n_qb, n_kb, n_pairs, cap;
+  // explicit
+  const int32_t* kv_idx;   // [BH][n_qb][kv_max]
+  const int32_t* kv_cnt;   // [BH][n_qb]
+  int kv_max;
+  // lvsa
+  const int32_t* sets;     // [T][set_cap]
+  const int32_t* set_cnt;  // [T]
+  int set_cap, blocks_per_frame;
+  // tile3d: tile grid (TF, TH, TW), tile id = (th*TW + tw)*TF + tf
+  int TF, TH, TW, radius;
+  uint32_t* list;          // [heads][n_pairs][cap]
+  int32_t* list_cnt;       // [heads][n_pairs]
+  int* status;
+};
+cudaError_t launch_pair_lists(const ListArgs& a, int heads, cudaStream_t st);
+
+// LVSA attention sets on the device (one thread per frame).
+cudaError_t launch_lvsa_sets(int T, int C, int W, int step, int32_t* sets, int32_t* counts, int cap,
+                             cudaStream_t st);
+
+// ------------------------------------------------------------ attention (k_attn.cu)
+struct AttnArgs {
+  const void* q; const void* k; const void* v;
+  const void* kf; const void* vf;      // far-field pooled K/V, bf16 [BH][64][d] (gated mode)
+  int BH, d;
+  SeqShape s;
+  int n_qb, n_kb, n_pairs;
+  const uint32_t* list;                // null = dense
+  const int32_t* list_cnt;
+  int list_cap, list_per_head;         // list_per_head = 0 when one list serves all heads
+  const float* addend;                 // fp32 [BH][n_pad][d] added to the output, or null
+  void* out;                           // bf16 [BH][n_pad][d]
+  float* lse;                          // fp32 [BH][n_pad] or null
+  int tile3d;                          // 1: blocks are 4x4x4 tiles of raster (F, Hh, Ww)
+  int F, Hh, Ww;
+  int gated;                           // 1: add the far-field branch and gate
+  float gate;
+  int* status;
+};
+cudaError_t launch_attention(const AttnArgs& a, cudaStream_t st);
+
+// ------------------------------------------------------------ marginal branch (k_marginal.cu)
+// h[bh][j] = [ (phi(K_j)^T V_j)^T (d rows of d) ; z_j (1 row) ] in bf16, [BH][nb][(d+1)*d].
+cudaError_t launch_key_states(const void* k, const void* v, __nv_bfloat16* h, int BH, int d, SeqShape s,
+                              int* status, cudaStream_t st);
+
+// Hs[bh][i] = sum_j m01[bh][i][j] * h[bh][j]  (bf16 out, fp32 accumulate), [BH][nb][(d+1)*d].
+cudaError_t launch_reduce_states(const __nv_bfloat16* m01, int ld_m01, const __nv_bfloat16* h,
+                                 __nv_bfloat16* Hs, int BH, int nb, int d, int* status, cudaStream_t st);
+
+// o_lin[bh][t] = (phi(q_t) H_i / (phi(q_t).Z_i)) [@ W_proj] for every valid token t of block i.
+cudaError_t launch_linear_apply(const void* q, const __nv_bfloat16* Hs, const void* w_proj,
+                                float* o_lin, int BH, int d, SeqShape s, int* status, cudaStream_t st);
+
+}  // namespace slr

@@ -1,0 +1,600 @@
+// slr_api.cu -- the C ABI of libslr (declared in include/slr.h): argument
+// validation, workspace layout, and the launch sequence of every entry point.
+// Nothing here synchronises or allocates (except slr_check_status, which is
+// documented to synchronise).
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include "../../include/slr.h"
+#include "launch.h"
+#include "lvsa_sets.cuh"
+
+namespace slr {
+
+// ------------------------------------------------------------------ tensor maps
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+bool make_tile_map(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
+                   const uint64_t* strides_bytes, const uint32_t* box) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t gdim[5], gstr[4];
+  cuuint32_t bdim[5], estr[5];
+  for (int i = 0; i < rank; ++i) { gdim[i] = dims[i]; bdim[i] = box[i]; estr[i] = 1; }
+  for (int i = 0; i < rank - 1; ++i) gstr[i] = strides_bytes[i];
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base), gdim, gstr,
+                  bdim, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+}  // namespace slr
+
+using namespace slr;
+
+namespace {
+
+constexpr size_t kAlign = 256;
+
+size_t align_up(size_t x) { return (x + kAlign - 1) & ~(kAlign - 1); }
+
+// Sequential carving of the caller's workspace.  With base == nullptr it only counts.
+struct Carve {
+  uint8_t* base;
+  size_t off;
+  explicit Carve(void* b) : base(static_cast<uint8_t*>(b)), off(0) {}
+  template <class T>
+  T* take(size_t count) {
+    const size_t at = off;
+    off = align_up(off + count * sizeof(T));
+    return base ? reinterpret_cast<T*>(base + at) : nullptr;
+  }
+};
+
+struct Shape {
+  int B, H, BH, d, n_seg, seg_len, seg_stride, n_pad, nb, npairs;
+  SeqShape s;
+};
+
+slr_status check_seq(const slr_seq* q, Shape& sh) {
+  if (!q) return SLR_ERR_ARG;
+  if (q->B < 1 || q->H < 1 || q->n_seg < 1 || q->seg_len < 1 || q->seg_stride < 1) return SLR_ERR_ARG;
+  if (q->d != 64 && q->d != 128) return SLR_ERR_UNSUPPORTED;
+  if (q->block != kBlock) return SLR_ERR_UNSUPPORTED;
+  if (q->seg_stride % kBlock != 0) return SLR_ERR_UNSUPPORTED;
+  if (q->seg_len > q->seg_stride || q->seg_len <= q->seg_stride - kBlock) return SLR_ERR_UNSUPPORTED;
+  const long long n_pad = (long long)q->n_seg * q->seg_stride;
+  if (n_pad / kBlock > kMaxKeyBlocks) return SLR_ERR_UNSUPPORTED;
+  const long long bh = (long long)q->B * q->H;
+  if (bh > 65535) return SLR_ERR_UNSUPPORTED;
+  sh.B = q->B; sh.H = q->H; sh.BH = (int)bh; sh.d = q->d;
+  sh.n_seg = q->n_seg; sh.seg_len = q->seg_len; sh.seg_stride = q->seg_stride;
+  sh.n_pad = (int)n_pad; sh.nb = (int)(n_pad / kBlock); sh.npairs = (sh.nb + 1) / 2;
+  sh.s = SeqShape{sh.n_pad, sh.seg_len, sh.seg_stride, sh.nb};
+  return SLR_OK;
+}
+
+bool aligned16(const void* p) { return p && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+slr_status counts(int nb, float crit, float negl, int* kc, int* kn) {
+  if (!(crit >= 0.f && crit <= 1.f && negl >= 0.f && negl <= 1.f)) return SLR_ERR_ARG;
+  if ((double)crit + (double)negl > 1.0 + 1e-6) return SLR_ERR_ARG;
+  const double c = (double)crit * nb, n = (double)negl * nb;
+  int a = (int)ceil(c - 1e-3);
+  if (a < 1) a = 1;
+  if (a > nb) a = nb;
+  int b = (int)floor(n + 1e-3);
+  if (b < 0) b = 0;
+  if (b > nb - a) b = nb - a;
+  *kc = a;
+  *kn = b;
+  return SLR_OK;
+}
+
+int ld_m01(int nb) { return (nb + 63) / 64 * 64; }
+
+// ---------------------------------------------------------------- workspace plans
+
+struct ClassifyWs {
+  double *qbar, *kbar, *logits;
+  __nv_bfloat16* m01;
+};
+
+void plan_classify(Carve& c, const Shape& sh, ClassifyWs& w) {
+  w.qbar = c.take<double>((size_t)sh.BH * sh.nb * sh.d);
+  w.kbar = c.take<double>((size_t)sh.BH * sh.nb * sh.d);
+  w.logits = c.take<double>((size_t)sh.BH * sh.nb * sh.nb);
+  w.m01 = c.take<__nv_bfloat16>((size_t)sh.BH * sh.nb * ld_m01(sh.nb));
+}
+
+struct MarginalWs {
+  __nv_bfloat16 *h, *Hs;
+};
+
+void plan_marginal(Carve& c, const Shape& sh, MarginalWs& w) {
+  const size_t per = (size_t)(sh.d + 1) * sh.d;
+  w.h = c.take<__nv_bfloat16>((size_t)sh.BH * sh.nb * per);
+  w.Hs = c.take<__nv_bfloat16>((size_t)sh.BH * sh.nb * per);
+}
+
+struct SlaWs {
+  int* status;
+  ClassifyWs cls;
+  int8_t* mask;
+  int32_t *crit_idx, *crit_cnt;
+  uint32_t* list;
+  int32_t* list_cnt;
+  int cap;
+  MarginalWs mar;
+  float* olin;
+};
+
+void plan_sla(Carve& c, const Shape& sh, int kc, int kn, bool own_mask, SlaWs& w) {
+  w.status = c.take<int>(64);
+  const bool dense = kc == sh.nb;
+  w.cap = dense ? 0 : (2 * kc < sh.nb ? 2 * kc : sh.nb);
+  if (dense) return;
+  plan_classify(c, sh, w.cls);
+  w.mask = own_mask ? c.take<int8_t>((size_t)sh.BH * sh.nb * sh.nb) : nullptr;
+  w.crit_idx = c.take<int32_t>((size_t)sh.BH * sh.nb * kc);
+  w.crit_cnt = c.take<int32_t>((size_t)sh.BH * sh.nb);
+  w.list = c.take<uint32_t>((size_t)sh.BH * sh.npairs * w.cap);
+  w.list_cnt = c.take<int32_t>((size_t)sh.BH * sh.npairs);
+  if (sh.nb - kc - kn > 0) {
+    plan_marginal(c, sh, w.mar);
+    w.olin = c.take<float>((size_t)sh.BH * sh.n_pad * sh.d);
+  } else {
+    w.mar.h = w.mar.Hs = nullptr;
+    w.olin = nullptr;
+  }
+}
+
+struct FrameWs {
+  int* status;
+  int32_t *sets, *set_cnt;
+  int set_cap;
+  uint32_t* list;
+  int32_t* list_cnt;
+  int cap;
+  void *kf, *vf;
+};
+
+slr_status check_mask(const slr_mask_desc* m, const Shape& sh) {
+  if (!m) return SLR_ERR_ARG;
+  if (m->kind == SLR_MASK_LVSA) {
+    if (m->T != sh.n_seg || m->W < 0 || m->step < 0 || m->C <= 2 * m->W + 1) return SLR_ERR_ARG;
+    return SLR_OK;
+  }
+  if (m->kind == SLR_MASK_TILE3D) {
+    if (sh.n_seg != 1 || sh.seg_len != sh.seg_stride) return SLR_ERR_UNSUPPORTED;
+    if (m->F < 1 || m->Hh < 1 || m->Ww < 1) return SLR_ERR_ARG;
+    if ((long long)m->F * m->Hh * m->Ww != sh.n_pad) return SLR_ERR_ARG;
+    if (m->tile[0] != 4 || m->tile[1] != 4 || m->tile[2] != 4) return SLR_ERR_UNSUPPORTED;
+    if (m->F % 4 || m->Hh % 4 || m->Ww % 4) return SLR_ERR_UNSUPPORTED;
+    if (m->radius < 0) return SLR_ERR_ARG;
+    const int* c = m->cell;
+    if (c[0] < 1 || c[1] < 1 || c[2] < 1 || m->F % c[0] || m->Hh % c[1] || m->Ww % c[2]) return SLR_ERR_ARG;
+    if ((m->F / c[0]) * (m->Hh / c[1]) * (m->Ww / c[2]) != 64) return SLR_ERR_UNSUPPORTED;
+    if (!(m->gate >= 0.f && m->gate <= 1.f)) return SLR_ERR_ARG;
+    return SLR_OK;
+  }
+  return SLR_ERR_ARG;
+}
+
+void plan_frame(Carve& c, const Shape& sh, const slr_mask_desc* m, FrameWs& w) {
+  w.status = c.take<int>(64);
+  w.sets = w.set_cnt = nullptr;
+  w.kf = w.vf = nullptr;
+  if (m->kind == SLR_MASK_LVSA) {
+    const LvsaGlobals g = lvsa_globals(m->T, m->C, m->W, m->step);
+    const int win = (2 * m->W + 1 < m->T - g.count) ? 2 * m->W + 1 : m->T - g.count;
+    w.set_cap = g.count + win;
+    w.sets = c.take<int32_t>((size_t)m->T * w.set_cap);
+    w.set_cnt = c.take<int32_t>((size_t)m->T);
+    const int bpf = sh.seg_stride / kBlock;
+    const long long cap = 2LL * w.set_cap * bpf;
+    w.cap = cap < sh.nb ? (int)cap : sh.nb;
+  } else {
+    const int side = 2 * m->radius + 1;
+    const long long cap = 2LL * side * side * side;
+    w.cap = cap < sh.nb ? (int)cap : sh.nb;
+    w.kf = c.take<__nv_bfloat16>((size_t)sh.BH * 64 * sh.d);
+    w.vf = c.take<__nv_bfloat16>((size_t)sh.BH * 64 * sh.d);
+    w.set_cap = 0;
+  }
+  w.list = c.take<uint32_t>((size_t)sh.npairs * w.cap);
+  w.list_cnt = c.take<int32_t>((size_t)sh.npairs);
+}
+
+slr_status ws_check(void* ws, size_t have, size_t need) {
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & (kAlign - 1))) return SLR_ERR_WORKSPACE;
+  if (have < need) return SLR_ERR_WORKSPACE;
+  return SLR_OK;
+}
+
+#define SLR_TRY(expr)                                   \
+  do {                                                  \
+    if ((expr) != cudaSuccess) return SLR_ERR_CUDA;     \
+  } while (0)
+
+// ---------------------------------------------------------------- per-kernel profiler
+enum KernelKind {
+  kKPool, kKLogits, kKClassify, kKLists, kKKeyStates, kKReduce, kKApply, kKAttention, kKLvsaSets,
+  kKFarPool, kKMaskToM01, kKNumKinds
+};
+const char* const kKindNames[kKNumKinds] = {
+    "pool_means", "block_logits", "classify_rows", "pair_lists", "key_states", "reduce_states",
+    "linear_apply", "attention", "lvsa_sets", "far_pool", "mask_to_m01"};
+
+struct ProfRec {
+  int kind;
+  cudaEvent_t a, b;
+};
+bool g_prof = false;
+cudaEvent_t g_pool[4096];
+int g_pool_n = 0;
+ProfRec g_pending[2048];
+int g_pending_n = 0;
+int g_launches[kKNumKinds];
+double g_ms[kKNumKinds];
+
+cudaEvent_t prof_event() {
+  if (g_pool_n > 0) return g_pool[--g_pool_n];
+  cudaEvent_t e = nullptr;
+  cudaEventCreate(&e);
+  return e;
+}
+
+void prof_drain() {
+  for (int i = 0; i < g_pending_n; ++i) {
+    ProfRec& r = g_pending[i];
+    float ms = 0.f;
+    if (cudaEventSynchronize(r.b) == cudaSuccess && cudaEventElapsedTime(&ms, r.a, r.b) == cudaSuccess) {
+      g_launches[r.kind] += 1;
+      g_ms[r.kind] += ms;
+    }
+    if (g_pool_n + 2 <= 4096) { g_pool[g_pool_n++] = r.a; g_pool[g_pool_n++] = r.b; }
+  }
+  g_pending_n = 0;
+}
+
+struct ProfScope {
+  int kind;
+  cudaStream_t st;
+  cudaEvent_t a = nullptr;
+  ProfScope(int k, cudaStream_t s) : kind(k), st(s) {
+    if (g_prof) {
+      if (g_pending_n >= 2048) prof_drain();
+      a = prof_event();
+      cudaEventRecord(a, st);
+    }
+  }
+  ~ProfScope() {
+    if (a) {
+      cudaEvent_t b = prof_event();
+      cudaEventRecord(b, st);
+      g_pending[g_pending_n++] = ProfRec{kind, a, b};
+    }
+  }
+};
+
+// Launch `expr` (a launcher call) bracketed by profiler events when profiling is on.
+#define SLR_LAUNCH(kind, stream, expr)                  \
+  do {                                                  \
+    ProfScope _ps(kind, stream);                        \
+    if ((expr) != cudaSuccess) return SLR_ERR_CUDA;     \
+  } while (0)
+
+AttnArgs attn_base(const Shape& sh, const void* q, const void* k, const void* v, void* out, int* status) {
+  AttnArgs a;
+  memset(&a, 0, sizeof(a));
+  a.q = q; a.k = k; a.v = v;
+  a.BH = sh.BH; a.d = sh.d; a.s = sh.s;
+  a.n_qb = sh.nb; a.n_kb = sh.nb; a.n_pairs = sh.npairs;
+  a.out = out;
+  a.status = status;
+  a.gate = 1.f;
+  return a;
+}
+
+}  // namespace
+
+extern "C" {
+
+int slr_version(void) { return 100; }
+
+slr_status slr_profile_enable(int on) {
+  g_prof = on != 0;
+  return SLR_OK;
+}
+
+int slr_profile_collect(const char** names, int* launches, double* total_ms, int max) {
+  prof_drain();
+  int n = 0;
+  for (int k = 0; k < kKNumKinds; ++k) {
+    if (g_launches[k] == 0) continue;
+    if (n < max) {
+      if (names) names[n] = kKindNames[k];
+      if (launches) launches[n] = g_launches[k];
+      if (total_ms) total_ms[n] = g_ms[k];
+      ++n;
+    }
+    g_launches[k] = 0;
+    g_ms[k] = 0.0;
+  }
+  return n;
+}
+
+const char* slr_status_string(slr_status s) {
+  switch (s) {
+    case SLR_OK: return "ok";
+    case SLR_ERR_ARG: return "invalid argument";
+    case SLR_ERR_UNSUPPORTED: return "unsupported shape";
+    case SLR_ERR_WORKSPACE: return "workspace too small or misaligned";
+    case SLR_ERR_CUDA: return "CUDA error";
+    case SLR_ERR_TIMEOUT: return "device wait timed out";
+    case SLR_ERR_INDEX: return "block index out of range";
+    default: return "unknown status";
+  }
+}
+
+slr_status slr_block_counts(int n_kb, float crit_frac, float negl_frac, int* kc, int* kn) {
+  if (n_kb < 1 || !kc || !kn) return SLR_ERR_ARG;
+  return counts(n_kb, crit_frac, negl_frac, kc, kn);
+}
+
+slr_status slr_lvsa_attention_sets(int T, int C, int W, int step, int32_t* sets, int32_t* cnts, int cap) {
+  if (T < 1 || W < 0 || step < 0 || C <= 2 * W + 1 || !sets || !cnts || cap < 1) return SLR_ERR_ARG;
+  for (int t = 0; t < T; ++t) {
+    const int n = lvsa_attention_set(T, C, W, step, t, sets + (size_t)t * cap, cap);
+    if (n < 0) return SLR_ERR_ARG;
+    cnts[t] = n;
+  }
+  return SLR_OK;
+}
+
+size_t slr_workspace_bytes(int op, const slr_seq* seq, const void* params) {
+  Shape sh;
+  if (check_seq(seq, sh) != SLR_OK) return 0;
+  Carve c(nullptr);
+  switch (op) {
+    case SLR_OP_POOL_CLASSIFY: {
+      if (sh.nb > kMaxClassifyBlocks || !params) return 0;
+      c.take<int>(64);
+      ClassifyWs w;
+      plan_classify(c, sh, w);
+      return c.off;
+    }
+    case SLR_OP_BLOCK_SPARSE: {
+      c.take<int>(64);
+      const int kv_max = params ? *static_cast<const int*>(params) : sh.nb;
+      const int cap = 2 * kv_max < sh.nb ? 2 * kv_max : sh.nb;
+      c.take<uint32_t>((size_t)sh.BH * sh.npairs * (cap > 0 ? cap : 1));
+      c.take<int32_t>((size_t)sh.BH * sh.npairs);
+      return c.off;
+    }
+    case SLR_OP_LINEAR_MARGINAL: {
+      c.take<int>(64);
+      c.take<__nv_bfloat16>((size_t)sh.BH * sh.nb * ld_m01(sh.nb));
+      MarginalWs w;
+      plan_marginal(c, sh, w);
+      return c.off;
+    }
+    case SLR_OP_SPARSE_LINEAR: {
+      if (!params) return 0;
+      const slr_fracs* f = static_cast<const slr_fracs*>(params);
+      int kc, kn;
+      if (counts(sh.nb, f->crit_frac, f->negl_frac, &kc, &kn) != SLR_OK) return 0;
+      if (kc != sh.nb && sh.nb > kMaxClassifyBlocks) return 0;
+      SlaWs w;
+      plan_sla(c, sh, kc, kn, true, w);
+      return c.off;
+    }
+    case SLR_OP_FRAME_MASK: {
+      const slr_mask_desc* m = static_cast<const slr_mask_desc*>(params);
+      if (check_mask(m, sh) != SLR_OK) return 0;
+      FrameWs w;
+      plan_frame(c, sh, m, w);
+      return c.off;
+    }
+    default:
+      return 0;
+  }
+}
+
+slr_status slr_check_status(void* ws, void* stream) {
+  if (!ws) return SLR_ERR_ARG;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return SLR_ERR_CUDA;
+  int code = 0;
+  if (cudaMemcpy(&code, ws, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return SLR_ERR_CUDA;
+  if (cudaMemset(ws, 0, sizeof(int)) != cudaSuccess) return SLR_ERR_CUDA;
+  return code == 0 ? SLR_OK : -code;
+}
+
+slr_status slr_pool_classify(const void* q, const void* k, const slr_seq* seq, float crit_frac, float negl_frac,
+                             int8_t* mask, int32_t* crit_idx, int32_t* crit_cnt, float* scores_opt,
+                             void* ws, size_t ws_bytes, void* stream) {
+  Shape sh;
+  slr_status st = check_seq(seq, sh);
+  if (st != SLR_OK) return st;
+  if (sh.nb > kMaxClassifyBlocks) return SLR_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !mask || !crit_idx || !crit_cnt) return SLR_ERR_ARG;
+  int kc, kn;
+  if ((st = counts(sh.nb, crit_frac, negl_frac, &kc, &kn)) != SLR_OK) return st;
+  const slr_fracs f{crit_frac, negl_frac};
+  if ((st = ws_check(ws, ws_bytes, slr_workspace_bytes(SLR_OP_POOL_CLASSIFY, seq, &f))) != SLR_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  Carve c(ws);
+  int* status = c.take<int>(64);
+  ClassifyWs w;
+  plan_classify(c, sh, w);
+  SLR_TRY(cudaMemsetAsync(status, 0, sizeof(int), s));
+  SLR_LAUNCH(kKPool, s, launch_pool_means(q, k, w.qbar, w.kbar, sh.BH, sh.d, sh.s, s));
+  SLR_LAUNCH(kKLogits, s, launch_block_logits(w.qbar, w.kbar, w.logits, sh.BH, sh.nb, sh.d, s));
+  SLR_LAUNCH(kKClassify, s, launch_classify_rows(w.logits, sh.BH, sh.nb, kc, kn, mask, crit_idx, crit_cnt, w.m01, ld_m01(sh.nb),
+                               scores_opt, s));
+  return SLR_OK;
+}
+
+slr_status slr_block_sparse_attn(const void* q, const void* k, const void* v, const slr_seq* seq,
+                                 const int32_t* kv_idx, const int32_t* kv_cnt, int kv_max,
+                                 void* o, float* lse_opt, void* ws, size_t ws_bytes, void* stream) {
+  Shape sh;
+  slr_status st = check_seq(seq, sh);
+  if (st != SLR_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return SLR_ERR_ARG;
+  if (kv_idx && (!kv_cnt || kv_max < 1)) return SLR_ERR_ARG;
+  const int km = kv_idx ? kv_max : sh.nb;
+  if ((st = ws_check(ws, ws_bytes, slr_workspace_bytes(SLR_OP_BLOCK_SPARSE, seq, &km))) != SLR_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  Carve c(ws);
+  int* status = c.take<int>(64);
+  const int cap = 2 * km < sh.nb ? 2 * km : sh.nb;
+  uint32_t* list = c.take<uint32_t>((size_t)sh.BH * sh.npairs * cap);
+  int32_t* list_cnt = c.take<int32_t>((size_t)sh.BH * sh.npairs);
+  SLR_TRY(cudaMemsetAsync(status, 0, sizeof(int), s));
+  AttnArgs a = attn_base(sh, q, k, v, o, status);
+  a.lse = lse_opt;
+  if (kv_idx) {
+    ListArgs la;
+    memset(&la, 0, sizeof(la));
+    la.mode = kListExplicit;
+    la.n_qb = sh.nb; la.n_kb = sh.nb; la.n_pairs = sh.npairs; la.cap = cap;
+    la.kv_idx = kv_idx; la.kv_cnt = kv_cnt; la.kv_max = kv_max;
+    la.list = list; la.list_cnt = list_cnt; la.status = status;
+    SLR_LAUNCH(kKLists, s, launch_pair_lists(la, sh.BH, s));
+    a.list = list; a.list_cnt = list_cnt; a.list_cap = cap; a.list_per_head = 1;
+  }
+  SLR_LAUNCH(kKAttention, s, launch_attention(a, s));
+  return SLR_OK;
+}
+
+slr_status slr_linear_marginal(const void* q, const void* k, const void* v, const slr_seq* seq,
+                               const int8_t* mask, int phi, const void* w_proj_opt,
+                               float* o_lin, void* ws, size_t ws_bytes, void* stream) {
+  Shape sh;
+  slr_status st = check_seq(seq, sh);
+  if (st != SLR_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !mask || !aligned16(o_lin)) return SLR_ERR_ARG;
+  if (w_proj_opt && !aligned16(w_proj_opt)) return SLR_ERR_ARG;
+  if (phi != SLR_PHI_ELU1) return SLR_ERR_UNSUPPORTED;
+  if ((st = ws_check(ws, ws_bytes, slr_workspace_bytes(SLR_OP_LINEAR_MARGINAL, seq, nullptr))) != SLR_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  Carve c(ws);
+  int* status = c.take<int>(64);
+  __nv_bfloat16* m01 = c.take<__nv_bfloat16>((size_t)sh.BH * sh.nb * ld_m01(sh.nb));
+  MarginalWs w;
+  plan_marginal(c, sh, w);
+  SLR_TRY(cudaMemsetAsync(status, 0, sizeof(int), s));
+  SLR_LAUNCH(kKMaskToM01, s, launch_mask_to_m01(mask, m01, sh.BH, sh.nb, ld_m01(sh.nb), s));
+  SLR_LAUNCH(kKKeyStates, s, launch_key_states(k, v, w.h, sh.BH, sh.d, sh.s, status, s));
+  SLR_LAUNCH(kKReduce, s, launch_reduce_states(m01, ld_m01(sh.nb), w.h, w.Hs, sh.BH, sh.nb, sh.d, status, s));
+  SLR_LAUNCH(kKApply, s, launch_linear_apply(q, w.Hs, w_proj_opt, o_lin, sh.BH, sh.d, sh.s, status, s));
+  return SLR_OK;
+}
+
+slr_status slr_sparse_linear_attn(const void* q, const void* k, const void* v, const void* w_proj,
+                                  const slr_seq* seq, float crit_frac, float negl_frac, int phi,
+                                  void* out, int8_t* mask_out_opt, void* ws, size_t ws_bytes, void* stream) {
+  Shape sh;
+  slr_status st = check_seq(seq, sh);
+  if (st != SLR_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return SLR_ERR_ARG;
+  if (phi != SLR_PHI_ELU1) return SLR_ERR_UNSUPPORTED;
+  int kc, kn;
+  if ((st = counts(sh.nb, crit_frac, negl_frac, &kc, &kn)) != SLR_OK) return st;
+  const bool dense = kc == sh.nb;
+  const bool marginal = !dense && sh.nb - kc - kn > 0;
+  if (marginal && !aligned16(w_proj)) return SLR_ERR_ARG;
+  if (!dense && sh.nb > kMaxClassifyBlocks) return SLR_ERR_UNSUPPORTED;
+  const slr_fracs f{crit_frac, negl_frac};
+  if ((st = ws_check(ws, ws_bytes, slr_workspace_bytes(SLR_OP_SPARSE_LINEAR, seq, &f))) != SLR_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  Carve c(ws);
+  SlaWs w;
+  plan_sla(c, sh, kc, kn, true, w);
+  SLR_TRY(cudaMemsetAsync(w.status, 0, sizeof(int), s));
+  AttnArgs a = attn_base(sh, q, k, v, out, w.status);
+  if (dense) {
+    if (mask_out_opt) SLR_TRY(cudaMemsetAsync(mask_out_opt, 1, (size_t)sh.BH * sh.nb * sh.nb, s));
+    SLR_LAUNCH(kKAttention, s, launch_attention(a, s));
+    return SLR_OK;
+  }
+  int8_t* mask = mask_out_opt ? mask_out_opt : w.mask;
+  SLR_LAUNCH(kKPool, s, launch_pool_means(q, k, w.cls.qbar, w.cls.kbar, sh.BH, sh.d, sh.s, s));
+  SLR_LAUNCH(kKLogits, s, launch_block_logits(w.cls.qbar, w.cls.kbar, w.cls.logits, sh.BH, sh.nb, sh.d, s));
+  SLR_LAUNCH(kKClassify, s, launch_classify_rows(w.cls.logits, sh.BH, sh.nb, kc, kn, mask, w.crit_idx, w.crit_cnt, w.cls.m01,
+                               ld_m01(sh.nb), nullptr, s));
+  ListArgs la;
+  memset(&la, 0, sizeof(la));
+  la.mode = kListExplicit;
+  la.n_qb = sh.nb; la.n_kb = sh.nb; la.n_pairs = sh.npairs; la.cap = w.cap;
+  la.kv_idx = w.crit_idx; la.kv_cnt = w.crit_cnt; la.kv_max = kc;
+  la.list = w.list; la.list_cnt = w.list_cnt; la.status = w.status;
+  SLR_LAUNCH(kKLists, s, launch_pair_lists(la, sh.BH, s));
+  if (marginal) {
+    SLR_LAUNCH(kKKeyStates, s, launch_key_states(k, v, w.mar.h, sh.BH, sh.d, sh.s, w.status, s));
+    SLR_LAUNCH(kKReduce, s, launch_reduce_states(w.cls.m01, ld_m01(sh.nb), w.mar.h, w.mar.Hs, sh.BH, sh.nb, sh.d, w.status, s));
+    SLR_LAUNCH(kKApply, s, launch_linear_apply(q, w.mar.Hs, w_proj, w.olin, sh.BH, sh.d, sh.s, w.status, s));
+    a.addend = w.olin;
+  }
+  a.list = w.list; a.list_cnt = w.list_cnt; a.list_cap = w.cap; a.list_per_head = 1;
+  SLR_LAUNCH(kKAttention, s, launch_attention(a, s));
+  return SLR_OK;
+}
+
+slr_status slr_frame_mask_attn(const void* q, const void* k, const void* v, const slr_seq* seq,
+                               const slr_mask_desc* m, void* out, void* ws, size_t ws_bytes, void* stream) {
+  Shape sh;
+  slr_status st = check_seq(seq, sh);
+  if (st != SLR_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return SLR_ERR_ARG;
+  if ((st = check_mask(m, sh)) != SLR_OK) return st;
+  if ((st = ws_check(ws, ws_bytes, slr_workspace_bytes(SLR_OP_FRAME_MASK, seq, m))) != SLR_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  Carve c(ws);
+  FrameWs w;
+  plan_frame(c, sh, m, w);
+  SLR_TRY(cudaMemsetAsync(w.status, 0, sizeof(int), s));
+  ListArgs la;
+  memset(&la, 0, sizeof(la));
+  la.n_qb = sh.nb; la.n_kb = sh.nb; la.n_pairs = sh.npairs; la.cap = w.cap;
+  la.list = w.list; la.list_cnt = w.list_cnt; la.status = w.status;
+  AttnArgs a = attn_base(sh, q, k, v, out, w.status);
+  if (m->kind == SLR_MASK_LVSA) {
+    SLR_LAUNCH(kKLvsaSets, s, launch_lvsa_sets(m->T, m->C, m->W, m->step, w.sets, w.set_cnt, w.set_cap, s));
+    la.mode = kListLvsa;
+    la.sets = w.sets; la.set_cnt = w.set_cnt; la.set_cap = w.set_cap;
+    la.blocks_per_frame = sh.seg_stride / kBlock;
+  } else {
+    la.mode = kListTile3d;
+    la.TF = m->F / 4; la.TH = m->Hh / 4; la.TW = m->Ww / 4; la.radius = m->radius;
+    SLR_LAUNCH(kKFarPool, s, launch_far_pool(k, v, w.kf, w.vf, sh.BH, sh.d, m->F, m->Hh, m->Ww, m->cell[0], m->cell[1], m->cell[2], s));
+    a.tile3d = 1; a.F = m->F; a.Hh = m->Hh; a.Ww = m->Ww;
+    a.gated = 1; a.gate = m->gate; a.kf = w.kf; a.vf = w.vf;
+  }
+  SLR_LAUNCH(kKLists, s, launch_pair_lists(la, 1, s));
+  a.list = w.list; a.list_cnt = w.list_cnt; a.list_cap = w.cap; a.list_per_head = 0;
+  SLR_LAUNCH(kKAttention, s, launch_attention(a, s));
+  return SLR_OK;
+}
+
+}  // extern "C"

@@ -124,18 +124,20 @@ def lists_from_mask(mask: np.ndarray, value: int) -> list[np.ndarray]:
     return [np.nonzero(mask[i] == value)[0] for i in range(mask.shape[0])]
 
 
-def block_sparse_attention(q, k, v, valid, key_blocks, rows=None, block: int = BLOCK):
+def block_sparse_attention(q, k, v, valid, key_blocks, rows=None, block: int = BLOCK, return_lse=False):
     """Exact softmax attention of every query block over the listed key blocks.
 
     ``key_blocks[i]`` is a set of key-block indices for query block i (duplicates
     count once).  Only valid keys enter the softmax; pad queries and query blocks
     with no valid key give 0 (SLA page sec. 3, critical branch; LVSA page step 6
     writes the same normalised sum).  ``rows`` restricts the work to some query
-    blocks; the others are left 0.
+    blocks; the others are left 0.  With ``return_lse`` also returns the natural
+    log-sum-exp of each valid query's scaled logits (-inf with no key, 0 for pads).
     """
     n, d = q.shape
     nb = n // block
     out = np.zeros((n, v.shape[1]))
+    lse = np.zeros(n)
     scale = 1.0 / math.sqrt(d)
     rows = range(nb) if rows is None else rows
     for i in rows:
@@ -143,15 +145,16 @@ def block_sparse_attention(q, k, v, valid, key_blocks, rows=None, block: int = B
         qrows = np.arange(t0, t0 + block)
         qrows = qrows[valid[qrows]]
         blocks = np.unique(np.asarray(key_blocks[i], dtype=np.int64))
-        if blocks.size == 0 or qrows.size == 0:
-            continue
         keys = (blocks[:, None] * block + np.arange(block)[None, :]).reshape(-1)
-        keys = keys[valid[keys]]
-        if keys.size == 0:
+        keys = keys[valid[keys]] if keys.size else keys
+        if keys.size == 0 or qrows.size == 0:
+            lse[qrows] = -np.inf
             continue
         s = (q[qrows] @ k[keys].T) * scale
         out[qrows] = row_softmax(s) @ v[keys]
-    return out
+        m = s.max(axis=1)
+        lse[qrows] = m + np.log(np.exp(s - m[:, None]).sum(axis=1))
+    return (out, lse) if return_lse else out
 
 
 def phi_elu1(x: np.ndarray) -> np.ndarray:

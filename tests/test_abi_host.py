@@ -1,0 +1,129 @@
+"""CPU tests of the C ABI: the library loads, exports every symbol include/slr.h
+declares, its host-only helpers agree with the oracle, and argument errors are
+rejected on the host before any CUDA call (no GPU is needed for these)."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import block_sparse_linear_02_b200 as slr
+from oracle import lvsa as olvsa
+from oracle import sla as osla
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _header_symbols():
+    text = open(os.path.join(ROOT, "include", "slr.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(slr_[a-z_0-9]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(slr.LIB_PATH):
+        from block_sparse_linear_02_b200 import build
+        build.build()
+    return slr.lib()
+
+
+def test_exports_every_declared_symbol(lib):
+    syms = _header_symbols()
+    assert len(syms) >= 11
+    for s in syms:
+        assert hasattr(lib, s), s
+    assert set(syms) == set(slr.EXPORTS)
+
+
+def test_version_and_strings(lib):
+    assert lib.slr_version() >= 100
+    for code in range(0, -7, -1):
+        assert slr.status_string(code) not in ("", "unknown status")
+
+
+@pytest.mark.parametrize("nkb", [1, 2, 3, 4, 7, 64, 100, 512, 1800, 3025, 4096])
+@pytest.mark.parametrize("fr", [(0.05, 0.10), (0.25, 0.25), (1.0, 0.0), (0.0, 0.0), (0.5, 0.5), (0.33, 0.2)])
+def test_block_counts_match_oracle(lib, nkb, fr):
+    assert slr.slr_block_counts(nkb, *fr) == osla.block_counts(nkb, *fr)
+
+
+def test_block_counts_rejects_bad_fractions(lib):
+    for fr in [(-0.1, 0.1), (0.5, 0.6), (1.5, 0.0), (float("nan"), 0.1)]:
+        with pytest.raises(slr.SlrError):
+            slr.slr_block_counts(100, *fr)
+
+
+@pytest.mark.parametrize("T,C,W", [(121, 21, 3), (10, 6, 1), (9, 6, 1), (5, 6, 1), (37, 9, 2), (200, 30, 4),
+                                   (4, 9, 1), (13, 8, 3), (3, 9, 2), (1, 5, 1), (64, 12, 2)])
+def test_lvsa_sets_match_oracle(lib, T, C, W):
+    tper = olvsa.global_period(T, C, W)
+    for s in range(0, 2 * tper + 2):
+        assert slr.slr_lvsa_attention_sets(T, C, W, s) == olvsa.attention_sets(T, C, W, s), (T, C, W, s)
+
+
+def test_lvsa_sets_rejects_bad_budget(lib):
+    with pytest.raises(slr.SlrError):
+        slr.slr_lvsa_attention_sets(10, 3, 1, 0)     # C <= 2W+1
+
+
+def test_workspace_bytes(lib):
+    good = slr.make_seq(1, 12, 128, 1, 32760, 32768)
+    n = slr.slr_workspace_bytes(slr.SLR_OP_SPARSE_LINEAR, good, slr.SlrFracs(0.05, 0.10))
+    # at least h and H (bf16, (d+1)d per block per head) and the fp32 linear output
+    assert n >= 2 * 12 * 512 * 129 * 128 * 2 + 12 * 32768 * 128 * 4
+    dense = slr.slr_workspace_bytes(slr.SLR_OP_SPARSE_LINEAR, good, slr.SlrFracs(1.0, 0.0))
+    assert 0 < dense <= 4096
+    for bad in [slr.make_seq(1, 1, 96, 1, 64, 64),          # d unsupported
+                slr.make_seq(1, 1, 64, 1, 60, 100),         # stride not a multiple of 64
+                slr.make_seq(1, 1, 64, 1, 10, 128),         # a block with no valid token
+                slr.make_seq(0, 1, 64, 1, 64, 64)]:
+        assert slr.slr_workspace_bytes(slr.SLR_OP_SPARSE_LINEAR, bad, slr.SlrFracs(0.05, 0.1)) == 0
+    m = slr.lvsa_mask(121, 21, 3, 0)
+    assert slr.slr_workspace_bytes(slr.SLR_OP_FRAME_MASK, slr.make_seq(1, 12, 128, 121, 1560, 1600), m) > 0
+    assert slr.slr_workspace_bytes(slr.SLR_OP_FRAME_MASK, slr.make_seq(1, 12, 128, 120, 1560, 1600), m) == 0
+    t3 = slr.tile3d_mask(8, 64, 64)
+    assert slr.slr_workspace_bytes(slr.SLR_OP_FRAME_MASK, slr.make_seq(1, 16, 128, 1, 32768, 32768), t3) > 0
+    t3bad = slr.tile3d_mask(8, 64, 64, cell=(2, 8, 8))      # 256 cells, not 64
+    assert slr.slr_workspace_bytes(slr.SLR_OP_FRAME_MASK, slr.make_seq(1, 16, 128, 1, 32768, 32768), t3bad) == 0
+
+
+def test_invalid_arguments_rejected_before_cuda(lib):
+    seq = slr.make_seq(1, 1, 64, 1, 256, 256)
+    vp = ctypes.c_void_p
+    fake = vp(0x1000)           # never dereferenced: validation fails first
+    ws = vp(0x100000)
+    # null q
+    assert lib.slr_block_sparse_attn(None, fake, fake, ctypes.byref(seq), None, None, 0, fake, None, ws, 1 << 20,
+                                     None) == slr.SLR_ERR_ARG
+    # misaligned output
+    assert lib.slr_block_sparse_attn(fake, fake, fake, ctypes.byref(seq), None, None, 0, vp(0x1001), None, ws,
+                                     1 << 20, None) == slr.SLR_ERR_ARG
+    # workspace too small / misaligned
+    assert lib.slr_block_sparse_attn(fake, fake, fake, ctypes.byref(seq), None, None, 0, fake, None, ws, 16,
+                                     None) == slr.SLR_ERR_WORKSPACE
+    assert lib.slr_block_sparse_attn(fake, fake, fake, ctypes.byref(seq), None, None, 0, fake, None, vp(0x100010),
+                                     1 << 20, None) == slr.SLR_ERR_WORKSPACE
+    # unsupported head size
+    bad = slr.make_seq(1, 1, 32, 1, 256, 256)
+    assert lib.slr_sparse_linear_attn(fake, fake, fake, fake, ctypes.byref(bad), 0.05, 0.1, 0, fake, None, ws,
+                                      1 << 20, None) == slr.SLR_ERR_UNSUPPORTED
+    # fractions that do not fit
+    assert lib.slr_sparse_linear_attn(fake, fake, fake, fake, ctypes.byref(seq), 0.7, 0.5, 0, fake, None, ws,
+                                      1 << 20, None) == slr.SLR_ERR_ARG
+    # unknown feature map
+    assert lib.slr_sparse_linear_attn(fake, fake, fake, fake, ctypes.byref(seq), 0.05, 0.1, 7, fake, None, ws,
+                                      1 << 20, None) == slr.SLR_ERR_UNSUPPORTED
+    # mask kind
+    m = slr.SlrMaskDesc()
+    m.kind = 9
+    assert lib.slr_frame_mask_attn(fake, fake, fake, ctypes.byref(seq), ctypes.byref(m), fake, ws, 1 << 20,
+                                   None) == slr.SLR_ERR_ARG
+    # LVSA frame count must equal the number of segments
+    m = slr.lvsa_mask(5, 6, 1, 0)
+    assert lib.slr_frame_mask_attn(fake, fake, fake, ctypes.byref(seq), ctypes.byref(m), fake, ws, 1 << 20,
+                                   None) == slr.SLR_ERR_ARG
+    # linear branch needs a mask
+    assert lib.slr_linear_marginal(fake, fake, fake, ctypes.byref(seq), None, 0, None, fake, ws, 1 << 20,
+                                   None) == slr.SLR_ERR_ARG

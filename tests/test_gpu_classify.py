@@ -1,0 +1,76 @@
+"""GPU parity of slr_pool_classify against the fp64 oracle: the three-way block
+mask (exact outside the 1e-5 threshold band), the ascending critical lists,
+the counts and P_c, on the tiny workload, a ragged multi-segment case, a fully
+tied case, the 32k-token workload at full size and the largest supported
+block count."""
+import numpy as np
+import pytest
+import torch
+
+import block_sparse_linear_02_b200 as slr
+import workloads
+from gpu_common import check_mask, cuda, make_inputs, status_ok, to64, valid_np
+from oracle import sla as osla
+
+pytestmark = pytest.mark.gpu
+
+
+def _run_and_check(q, k, seq, crit, negl, with_scores=True):
+    mask, ci, cc, sc = slr.slr_pool_classify(cuda(q), cuda(k), seq, crit, negl, scores=with_scores)
+    status_ok()
+    valid = valid_np(seq.n_seg, seq.seg_len, seq.seg_stride)
+    mask, ci, cc = mask.cpu().numpy(), ci.cpu().numpy(), cc.cpu().numpy()
+    flips = 0
+    for b in range(seq.B):
+        for h in range(seq.H):
+            qbar = osla.pool_blocks(to64(q[b, h]), valid)
+            kbar = osla.pool_blocks(to64(k[b, h]), valid)
+            lg = osla.block_logits(qbar, kbar)
+            p = osla.row_softmax(lg)
+            kc, kn = osla.block_counts(kbar.shape[0], crit, negl)
+            ref = osla.classify(lg, kc, kn)
+            tc, tn = osla.threshold_band(p, ref)
+            flips += check_mask(mask[b, h], ref, p, tc, tn, kc, kn)
+            assert (cc[b, h] == kc).all()
+            for i in range(mask.shape[2]):
+                assert ci[b, h, i].tolist() == np.nonzero(mask[b, h, i] == 1)[0].tolist()
+            if sc is not None:
+                assert np.abs(sc[b, h].cpu().double().numpy() - p).max() < 1e-6
+    return flips
+
+
+def test_tiny_workload():
+    w = workloads.TINY
+    q, k, _ = workloads.make_qkv(w)
+    assert _run_and_check(q, k, slr.make_seq(**{k_: v for k_, v in w.seq().items() if k_ != "block"}),
+                          w.crit_frac, w.negl_frac) == 0
+
+
+def test_ragged_segments():
+    q, k, _ = make_inputs(1, 2, 128, 3, 600, 640, seed=11)
+    assert _run_and_check(q, k, slr.make_seq(1, 2, 128, 3, 600, 640), 0.1, 0.2) == 0
+
+
+def test_full_tie_breaks_by_index():
+    n = 512
+    q = torch.zeros(1, 1, n, 64, dtype=torch.bfloat16)         # every logit is 0
+    k = make_inputs(1, 1, 64, 1, n, n, seed=12)[1]
+    mask, ci, _, _ = slr.slr_pool_classify(cuda(q), cuda(k), slr.make_seq(1, 1, 64, 1, n, n), 0.25, 0.25)
+    status_ok()
+    row = mask[0, 0].cpu().numpy()
+    assert (row == np.array([1, 1, 0, 0, 0, 0, -1, -1], np.int8)[None, :]).all()
+    assert (ci[0, 0].cpu().numpy() == np.array([0, 1])[None, :]).all()
+
+
+def test_wan_workload_full_size():
+    w = workloads.WAN
+    q, k, _ = workloads.make_qkv(w)
+    flips = _run_and_check(q, k, slr.make_seq(1, w.heads, w.d, w.n_seg, w.seg_len, w.seg_stride),
+                           w.crit_frac, w.negl_frac, with_scores=False)
+    assert flips == 0
+
+
+def test_largest_classified_block_count():
+    n = 4096 * 64
+    q, k, _ = make_inputs(1, 1, 64, 1, n, n, seed=13)
+    assert _run_and_check(q, k, slr.make_seq(1, 1, 64, 1, n, n), 0.05, 0.1, with_scores=False) == 0

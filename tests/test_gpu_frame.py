@@ -1,0 +1,82 @@
+"""GPU parity of slr_frame_mask_attn against the fp64 oracle: LVSA frame masks
+(small case in full for four denoising steps, the 121-frame workload on sampled
+query blocks) and the gated tile neighbourhood + far field (small grids in
+full, including an odd tile count, and the 8x64x64 workload on sampled tiles)."""
+import numpy as np
+import pytest
+import torch
+
+import block_sparse_linear_02_b200 as slr
+import workloads
+from gpu_common import assert_close, cuda, make_inputs, rows_of_blocks, status_ok, to64, valid_np
+from oracle import lvsa as olvsa
+from oracle import tile3d as otile
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("step", [0, 1, 2, 3])
+def test_lvsa_small_full(step):
+    T, C, W, seg_len, stride, H, d = 10, 6, 1, 100, 128, 2, 128
+    q, k, v = make_inputs(1, H, d, T, seg_len, stride, seed=41)
+    seq = slr.make_seq(1, H, d, T, seg_len, stride)
+    out = slr.slr_frame_mask_attn(cuda(q), cuda(k), cuda(v), seq, slr.lvsa_mask(T, C, W, step))
+    status_ok()
+    sets = olvsa.attention_sets(T, C, W, step)
+    for h in range(H):
+        ref = olvsa.frame_mask_attention(to64(q[0, h]), to64(k[0, h]), to64(v[0, h]), T, seg_len, stride, sets)
+        assert_close(to64(out[0, h]), ref, f"step {step} head {h}")
+
+
+@pytest.mark.parametrize("step", [0, 3])
+def test_lvsa_workload_sampled(step):
+    w = workloads.LVSA
+    q, k, v = workloads.make_qkv(w)
+    seq = slr.make_seq(1, w.heads, w.d, w.n_seg, w.seg_len, w.seg_stride)
+    out = slr.slr_frame_mask_attn(cuda(q), cuda(k), cuda(v), seq, slr.lvsa_mask(w.frames, w.lvsa_C, w.lvsa_W, step))
+    status_ok()
+    sets = olvsa.attention_sets(w.frames, w.lvsa_C, w.lvsa_W, step)
+    bpf = w.seg_stride // 64
+    rows = [0, 24, 25, 60 * bpf + 7, 120 * bpf + 24, w.n_blocks - 1]
+    sel = rows_of_blocks(rows)
+    outs, refs = [], []
+    for h in range(w.heads):
+        ref = olvsa.frame_mask_attention(to64(q[0, h]), to64(k[0, h]), to64(v[0, h]), w.n_seg, w.seg_len,
+                                         w.seg_stride, sets, rows=rows)
+        outs.append(to64(out[0, h])[sel])
+        refs.append(ref[sel])
+    assert_close(np.concatenate(outs), np.concatenate(refs), "lvsa workload")
+    pad = ~valid_np(w.n_seg, w.seg_len, w.seg_stride)
+    assert torch.count_nonzero(out[0, 0, torch.from_numpy(pad)]).item() == 0
+
+
+@pytest.mark.parametrize("F,Hh,Ww,cell,gate", [(8, 16, 16, (2, 4, 4), 0.55), (12, 8, 8, (3, 2, 2), 0.3),
+                                               (4, 16, 32, (1, 4, 8), 1.0), (8, 8, 16, (2, 2, 4), 0.0)])
+def test_tile3d_small_full(F, Hh, Ww, cell, gate):
+    H, d = 2, 128
+    n = F * Hh * Ww
+    q, k, v = make_inputs(1, H, d, 1, n, n, seed=51)
+    seq = slr.make_seq(1, H, d, 1, n, n)
+    out = slr.slr_frame_mask_attn(cuda(q), cuda(k), cuda(v), seq, slr.tile3d_mask(F, Hh, Ww, 1, cell, gate))
+    status_ok()
+    for h in range(H):
+        r = otile.gated_head(to64(q[0, h]), to64(k[0, h]), to64(v[0, h]), F, Hh, Ww, cell=cell, gate=gate)
+        assert_close(to64(out[0, h]), r["o"], f"tile3d head {h}")
+
+
+def test_tile3d_workload_sampled():
+    w = workloads.ROPESLR
+    q, k, v = workloads.make_qkv(w)
+    seq = slr.make_seq(1, w.heads, w.d, 1, w.seg_len, w.seg_stride)
+    out = slr.slr_frame_mask_attn(cuda(q), cuda(k), cuda(v), seq,
+                                  slr.tile3d_mask(w.frames, w.fh, w.fw, w.radius, w.cell, w.gate))
+    status_ok()
+    rng = np.random.default_rng(5)
+    toks = sorted(set(rng.choice(w.n_pad, 300, replace=False).tolist() + [0, w.n_pad - 1, 64 * 64 * 4 - 1]))
+    outs, refs = [], []
+    for h in range(0, w.heads, 3):
+        r = otile.gated_head(to64(q[0, h]), to64(k[0, h]), to64(v[0, h]), w.frames, w.fh, w.fw,
+                             w.tile, w.radius, w.cell, w.gate, rows=toks)
+        outs.append(to64(out[0, h])[toks])
+        refs.append(r["o"][toks])
+    assert_close(np.concatenate(outs), np.concatenate(refs), "tile3d workload")

@@ -292,3 +292,24 @@ def test_brute_force_loops_tiny():
     r = sla.sla_head(q, k, v, w, valid, 0.25, 0.25)
     ref = _loop_sla(q, k, v, w, valid, r["kc"], r["kn"])
     np.testing.assert_allclose(r["o"], ref, rtol=1e-10, atol=1e-12)
+
+
+def test_lse_matches_scipy_logsumexp():
+    from scipy.special import logsumexp
+    rng = _rng(15)
+    n, d = 192, 8
+    q, k, v = (rng.standard_normal((n, d)) * 2 for _ in range(3))
+    valid = sla.valid_tokens(3, 50, 64)
+    lists = [[0, 2], [], [1]]
+    _, lse = sla.block_sparse_attention(q, k, v, valid, lists, return_lse=True)
+    for t in range(n):
+        if not valid[t]:
+            assert lse[t] == 0
+            continue
+        i = t // 64
+        keys = [u for j in lists[i] for u in range(j * 64, j * 64 + 64) if valid[u]]
+        if not keys:
+            assert lse[t] == -np.inf
+        else:
+            ref = logsumexp([q[t] @ k[u] / math.sqrt(d) for u in keys])
+            assert abs(lse[t] - ref) < 1e-12
