@@ -41,7 +41,7 @@ EXPORTS = (
     "slr_pool_classify", "slr_block_sparse_attn", "slr_linear_marginal", "slr_sparse_linear_attn",
     "slr_frame_mask_attn", "slr_workspace_bytes", "slr_check_status", "slr_block_counts",
     "slr_lvsa_attention_sets", "slr_status_string", "slr_version", "slr_profile_enable",
-    "slr_profile_collect",
+    "slr_profile_collect", "slr_block_sparse_attn_noalloc",
 )
 
 
@@ -84,6 +84,8 @@ def lib() -> ctypes.CDLL:
         L.slr_linear_marginal.argtypes = [vp, vp, vp, seqp, vp, i, vp, vp, vp, sz, vp]
         L.slr_sparse_linear_attn.argtypes = [vp, vp, vp, vp, seqp, f, f, i, vp, vp, vp, sz, vp]
         L.slr_frame_mask_attn.argtypes = [vp, vp, vp, seqp, maskp, vp, vp, sz, vp]
+        L.slr_block_sparse_attn_noalloc.argtypes = [vp, vp, vp, seqp, vp, vp, i, vp, vp, vp, vp]
+        L.slr_block_sparse_attn_noalloc.restype = i
         L.slr_workspace_bytes.argtypes = [i, seqp, vp]
         L.slr_workspace_bytes.restype = sz
         L.slr_check_status.argtypes = [vp, vp]
@@ -324,3 +326,24 @@ def slr_frame_mask_attn(q, k, v, seq: SlrSeq, mask: SlrMaskDesc, out=None, ws=No
     _check(lib().slr_frame_mask_attn(_ptr(q), _ptr(k), _ptr(v), ctypes.byref(seq), ctypes.byref(mask), _ptr(o),
                                      wp, wn, _stream(q)), "slr_frame_mask_attn")
     return o
+
+
+def slr_block_sparse_attn_noalloc(q, k, v, seq: SlrSeq, kv_idx=None, kv_cnt=None, out=None, lse: bool = False,
+                                  status=None):
+    """slr_block_sparse_attn without a workspace (static device scratch); returns (o, lse).
+
+    ``status``: optional int32 CUDA tensor of one element that receives the device status.
+    Outputs are allocated here only when not given; the library call itself allocates nothing.
+    """
+    import torch
+    _check_qkv(q, k, v)
+    o = torch.empty_like(q) if out is None else out
+    l = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device) if lse else None
+    kv_max = 0
+    if kv_idx is not None:
+        kv_idx, kv_cnt = kv_idx.contiguous(), kv_cnt.contiguous()
+        kv_max = kv_idx.shape[-1]
+    _check(lib().slr_block_sparse_attn_noalloc(_ptr(q), _ptr(k), _ptr(v), ctypes.byref(seq), _ptr(kv_idx),
+                                               _ptr(kv_cnt), kv_max, _ptr(o), _ptr(l), _ptr(status), _stream(q)),
+           "slr_block_sparse_attn_noalloc")
+    return o, l

@@ -186,6 +186,38 @@ slr_status slr_frame_mask_attn(const void* q, const void* k, const void* v, cons
                                const slr_mask_desc* mask, void* out,
                                void* ws, size_t ws_bytes, void* stream);
 
+/*
+ * slr_block_sparse_attn_noalloc -- slr_block_sparse_attn without a workspace.
+ * The source pages have no counterpart to this call; it exists for callers
+ * that cannot allocate device memory for the library: a host application that
+ * owns the whole device-memory budget (for example an inference server that
+ * reserves the GPU's memory at start-up and forbids further cudaMalloc), or a
+ * plug-in whose interface passes only input and output tensors.
+ *
+ * It computes exactly what slr_block_sparse_attn computes, with the same
+ * arguments except `ws`/`ws_bytes`.  Its scratch (the per-pair key-block lists
+ * and, when status_opt is NULL, the status word) lives in one static device
+ * array of SLR_NOALLOC_SCRATCH_BYTES that every GPU which loads the library
+ * holds until the process exits; the call allocates nothing.
+ *   status_opt  int device pointer or NULL: zeroed by the call, then receives
+ *               the device status (0, or 5 / 6 for a timeout / an out-of-range
+ *               index: the negated SLR_ERR_TIMEOUT / SLR_ERR_INDEX).
+ * Returns SLR_ERR_WORKSPACE when the lists of this shape need more than the
+ * static scratch: 256 + B*H*ceil(Nb/2)*(min(Nb, 2*kv_max) + 1)*4 bytes (each
+ * part rounded up to 256) must fit in SLR_NOALLOC_SCRATCH_BYTES; the dense mode
+ * (kv_idx NULL) needs no lists.
+ * The first call on each device looks up the device address of the static
+ * array (cudaGetSymbolAddress, with that device current) and caches it; make
+ * that first call before any stream capture.  All calls in the process share
+ * the one array, which keeps the last call's lists: calls that can overlap on
+ * the GPU (different streams, or different host threads on one device) race on
+ * it and must be serialised by the caller.
+ */
+#define SLR_NOALLOC_SCRATCH_BYTES (4u << 20)
+slr_status slr_block_sparse_attn_noalloc(const void* q, const void* k, const void* v, const slr_seq* seq,
+                                         const int32_t* kv_idx, const int32_t* kv_cnt, int kv_max,
+                                         void* o, float* lse_opt, int* status_opt, void* stream);
+
 /* ------------------------------------------------------------------ helpers */
 
 /* Bytes of scratch the call `op` needs for this shape (0 on invalid input). */
