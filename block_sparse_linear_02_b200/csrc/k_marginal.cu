@@ -2,22 +2,26 @@
 //
 // SLA page section 3 ("边缘权重 ... 线性注意力"): for marginal block pairs the
 // attention is replaced by linear attention with feature map phi, evaluated as
-// "K^T V first, then apply Q".  Three kernels:
+// "K^T V first, then apply Q"; its output passes through the learnable
+// projection W_proj before it is added (same section, projection paragraph).
+// Because linear attention is a normalised weighted sum of value rows,
+// (sum w v / sum w) W = sum w (v W) / sum w, so W_proj is folded into V here.
 //
-//  key_states_kernel    per key block j: h_j^T = V_j^T phi(K_j) (d x d, one MMA
-//                       M=128 N=d K=64 with both operands MN-major straight from
-//                       the TMA tiles; phi is applied in place in shared memory)
-//                       and z_j = sum_t phi(K_j,t); written as bf16 rows
-//                       [h_j^T ; z_j] of (d+1)*d elements.
+//  key_states_kernel    per key block j: (V_j W)^T by one MMA (M=128 channels,
+//                       N=64 tokens, K=d), then h_j'^T = (V_j W)^T phi(K_j)
+//                       (M=128, N=d, K=64 tokens; phi applied in place in shared
+//                       memory) and z_j = sum_t phi(K_j,t); written as bf16 rows
+//                       [h_j'^T ; z_j] of (d+1)*d elements.  Without W the first
+//                       MMA is skipped and V_j^T is read MN-major from the tile.
 //  reduce_states_kernel per head: Hs = M01 . h, a plain tensor-core GEMM with
 //                       the 0/1 marginal indicator M01 [Nqb x Nkb] (K-major) and
 //                       h [Nkb x (d+1)d] (MN-major), fp32 accumulation in TMEM,
-//                       bf16 out.  Row i of Hs is [H_i^T ; Z_i].
-//  linear_apply_kernel  per query block i: O_l^T = H_i^T phi(Q_i)^T (MMA M=128 over
-//                       the output channel, N=64 tokens), normalised by
-//                       phi(q_t).Z_i, then optionally projected,
-//                       (O_l W)^T = W^T O_l^T (second MMA, W MN-major), written
-//                       as fp32 [token][channel].
+//                       bf16 out.  Row i of Hs is [H_i'^T ; Z_i].
+//  linear_apply_kernel  per pair of query blocks: phi(Q) times the rows
+//                       [H_i'^T ; Z_i] (M=128 tokens, N=d+16), whose column d is
+//                       the denominator phi(q_t).Z_i; fp32 [token][channel] out.
+//                       (The SLA call does this step inside the attention
+//                       kernel's epilogue instead.)
 // d = 64 runs the same M=128 MMAs with the upper 64 rows of A zero-filled.
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
@@ -38,45 +42,65 @@ __device__ __forceinline__ bool cta_wait(uint64_t* bar, uint32_t parity, volatil
 }
 
 // ------------------------------------------------------------------ key states
-constexpr int kKsBytes = 2 * 8192 + 2 * 8192 + 16 * 128 * 4 + 256 + 1024;
-constexpr int kKsSmemRequest = 56 * 1024;   // keeps at most 4 CTAs (4 x 128 TMEM columns) per SM
+// Shared-memory plan (bytes): K/phi(K) 16K | V 16K | W 32K | V'^T 16K | z partials 8K | barriers.
+constexpr int kKsK = 0, kKsV = 16384, kKsW = 32768, kKsVp = 65536, kKsZ = 81920, kKsBar = 81920 + 8192;
+constexpr int kKsSmemRequest = 100 * 1024;   // at most 2 CTAs (2 x 256 TMEM columns) per SM
 
-template <int D>
-__global__ void __launch_bounds__(128, 4)
+template <int D, bool PROJ>
+__global__ void __launch_bounds__(128)
 key_states_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-                  __nv_bfloat16* __restrict__ h, SeqShape s, int* status) {
+                  const __grid_constant__ CUtensorMap tmW, __nv_bfloat16* __restrict__ h, SeqShape s, int* status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
-  uint8_t* sK = smem;                      // phi(K_j) after the transform, 64 rows (t) x D
-  uint8_t* sV = smem + 2 * 8192;           // V_j, 64 rows (t) x D; chunk 1 zero when D = 64
-  float* zred = reinterpret_cast<float*>(smem + 4 * 8192);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 4 * 8192 + 16 * 128 * 4);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2);
+  uint8_t* sK = smem + kKsK;               // phi(K_j) after the transform, 64 rows (t) x D
+  uint8_t* sV = smem + kKsV;               // V_j, 64 rows (t) x D; chunk 1 zero when D = 64
+  uint8_t* sW = smem + kKsW;               // W_proj MN-major: rows c_in, 64 c_out per chunk (chunk stride D*128)
+  uint8_t* sVp = smem + kKsVp;             // (V_j W)^T, K-major: 128 rows (c_out) x 64 t
+  float* zred = reinterpret_cast<float*>(smem + kKsZ);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kKsBar);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 4);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   const int blk = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x, warp = tid >> 5;
+  constexpr uint32_t kColP = 0;            // (V W)^T: 64 columns
+  constexpr uint32_t kColH = 64;           // h^T: D columns
 
   if (tid == 0) {
-    mbar_init(&bars[0], 1);
-    mbar_init(&bars[1], 1);
+    for (int i = 0; i < 4; ++i) mbar_init(&bars[i], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (D == 64)
-    for (int i = tid; i < 8192 / 16; i += 128) reinterpret_cast<uint4*>(sV + 8192)[i] = make_uint4(0, 0, 0, 0);
-  if (warp == 0) { tmem_alloc(tmem_slot, 128); tmem_relinquish(); }
+  if (D == 64) {
+    // upper half of the M = 128 operand must be zero
+    uint4* z = reinterpret_cast<uint4*>(PROJ ? sW + D * 128 : sV + 8192);
+    for (int i = tid; i < 8192 / 16; i += 128) z[i] = make_uint4(0, 0, 0, 0);
+  }
+  if (warp == 0) { tmem_alloc(tmem_slot, 256); tmem_relinquish(); }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
   if (tid == 0) {
-    mbar_arrive_expect_tx(&bars[0], 2 * (D / 64) * 8192);
+    mbar_arrive_expect_tx(&bars[0], 2 * (D / 64) * 8192 + (PROJ ? (D / 64) * D * 128 : 0));
     for (int c = 0; c < D / 64; ++c) {
       tma_load_3d(sK + c * 8192, &tmK, &bars[0], c * 64, blk * 64, bh);
       tma_load_3d(sV + c * 8192, &tmV, &bars[0], c * 64, blk * 64, bh);
+      if (PROJ) tma_load_3d(sW + c * D * 128, &tmW, &bars[0], c * 64, 0, 0);
     }
   }
   bool ok = cta_wait(&bars[0], 0, abort_flag, status);
+  if (PROJ && tid == 0 && ok) {
+    // (V_j W)^T = W^T V_j^T: M = c_out (128), N = t (64), K = c_in (D)
+    tc_fence_after();
+    constexpr uint32_t id = idesc_bf16(128, 64, true, false);
+    #pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+      const uint64_t a = desc_mnmajor(smem_u32(sW) + kk * 2048, D * 128);
+      const uint64_t b = desc_kmajor(smem_u32(sV) + (kk >> 2) * 8192 + (kk & 3) * 32);
+      mma_bf16_ss(tmem + kColP, a, b, id, kk > 0 ? 1u : 0u);
+    }
+    mma_commit(&bars[1]);
+  }
 
   // phi in place (pad tokens -> 0) and column sums z
   constexpr int kCPR = D / 8, kRS = 128 / kCPR;
@@ -105,20 +129,42 @@ key_states_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
   }
   #pragma unroll
   for (int i = 0; i < 8; ++i) zred[rs * D + g * 8 + i] = z[i];
+  if (PROJ) {
+    // (V W)^T from TMEM into shared memory as the K-major A operand of the next MMA
+    if (ok) ok = cta_wait(&bars[1], 0, abort_flag, status);
+    tc_fence_after();
+    if (ok) {
+      uint32_t r[32], r2[32];
+      tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + kColP, r);
+      tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + kColP + 32, r2);
+      tmem_wait_ld();
+      #pragma unroll
+      for (int c8 = 0; c8 < 8; ++c8) {
+        const uint32_t* src = c8 < 4 ? r : r2;
+        const int b = (c8 & 3) * 8;
+        *reinterpret_cast<uint4*>(sVp + sw128_offset(tid, c8)) =
+            make_uint4(pack_bf16(__uint_as_float(src[b]), __uint_as_float(src[b + 1])),
+                       pack_bf16(__uint_as_float(src[b + 2]), __uint_as_float(src[b + 3])),
+                       pack_bf16(__uint_as_float(src[b + 4]), __uint_as_float(src[b + 5])),
+                       pack_bf16(__uint_as_float(src[b + 6]), __uint_as_float(src[b + 7])));
+      }
+    }
+  }
   fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
 
   if (tid == 0 && ok) {
+    // h^T = A^T-product: M = c (128), N = a (D), K = t (64)
     tc_fence_after();
-    constexpr uint32_t id = idesc_bf16(128, D, true, true);
+    constexpr uint32_t id = idesc_bf16(128, D, !PROJ, true);
     #pragma unroll
     for (int kk = 0; kk < 4; ++kk) {
-      const uint64_t a = desc_mnmajor(smem_u32(sV) + kk * 2048, 8192);
+      const uint64_t a = PROJ ? desc_kmajor(smem_u32(sVp) + kk * 32) : desc_mnmajor(smem_u32(sV) + kk * 2048, 8192);
       const uint64_t b = desc_mnmajor(smem_u32(sK) + kk * 2048, 8192);
-      mma_bf16_ss(tmem, a, b, id, kk > 0 ? 1u : 0u);
+      mma_bf16_ss(tmem + kColH, a, b, id, kk > 0 ? 1u : 0u);
     }
-    mma_commit(&bars[1]);
+    mma_commit(&bars[2]);
   }
   __nv_bfloat16* hrow = h + ((size_t)bh * s.n_blocks + blk) * (size_t)(D + 1) * D;
   for (int a = tid; a < D; a += 128) {
@@ -127,14 +173,14 @@ key_states_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
     for (int r = 0; r < kRS; ++r) sum += zred[r * D + a];
     hrow[(size_t)D * D + a] = __float2bfloat16_rn(sum);
   }
-  if (ok) ok = cta_wait(&bars[1], 0, abort_flag, status);
+  if (ok) ok = cta_wait(&bars[2], 0, abort_flag, status);
   tc_fence_after();
   if (ok && warp * 32 < D) {
     const int c = tid;                       // TMEM lane = output row (value channel)
     #pragma unroll 1
     for (int cc = 0; cc < D / 32; ++cc) {
       uint32_t r[32];
-      tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + cc * 32, r);
+      tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + kColH + cc * 32, r);
       tmem_wait_ld();
       uint4* dst = reinterpret_cast<uint4*>(hrow + (size_t)c * D + cc * 32);
       #pragma unroll
@@ -146,13 +192,13 @@ key_states_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
     }
   }
   if (!ok && tid == 0) {
-    mma_commit(&bars[1]);
+    mma_commit(&bars[3]);
     const long long t0 = clock64();
-    while (!mbar_try_wait(&bars[1], 0) && clock64() - t0 < kWaitBudgetCycles) {}
+    while (!mbar_try_wait(&bars[3], 0) && clock64() - t0 < kWaitBudgetCycles) {}
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) { tc_fence_after(); tmem_dealloc(tmem, 128); }
+  if (warp == 0) { tc_fence_after(); tmem_dealloc(tmem, 256); }
 }
 
 // ------------------------------------------------------------------ reduce states (GEMM)
@@ -262,207 +308,171 @@ reduce_states_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
   if (warp == 5) { tc_fence_after(); tmem_dealloc(tmem, 256); }
 }
 
-// ------------------------------------------------------------------ linear apply (+ projection)
+// ------------------------------------------------------------------ linear apply
+// One CTA per pair of query blocks: D_lin[t][c] = phi(q_t) . row c of [H_i'^T ; Z_i]
+// (M = 128 tokens, N = d + 16, K = d), the first query block's rows written with
+// TMEM lanes 64-127 masked off and the second's with lanes 0-63 masked off;
+// column d holds the denominator phi(q_t) . Z_i.
 template <int D>
 struct ApplyLayout {
-  static constexpr int kQOff = 0;                         // phi(Q_i): D/64 chunks x 64 rows
-  static constexpr int kHOff = kQOff + 2 * 8192;          // H_i^T: D/64 chunks x 128 rows
-  static constexpr int kWOff = kHOff + 2 * 16384;         // W (MN-major): 2 chunks x D rows
-  static constexpr int kOOff = kWOff + 2 * D * 128;       // O_l (K-major): D/64 chunks x 64 rows
-  static constexpr int kZOff = kOOff + 2 * 8192;          // z (D floats) + den (64 floats)
-  static constexpr int kBarOff = kZOff + (D + 64) * 4;
+  static constexpr int kNL = D + 16;
+  static constexpr int kQOff = 0;                              // phi(Q): D/64 chunks x 128 rows
+  static constexpr int kHOff = kQOff + (D / 64) * 16384;       // two state tiles: D/64 chunks x kNL rows
+  static constexpr int kHTile = (D / 64) * kNL * 128;
+  static constexpr int kBarOff = kHOff + 2 * kHTile;
   static constexpr int kBytes = kBarOff + 64 + 1024;
 };
 
+__device__ __forceinline__ void mma_masked(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc,
+                                           uint32_t m0, uint32_t m1, uint32_t m2, uint32_t m3) {
+  asm volatile("{\n\t.reg .pred p;\n\t"
+               "setp.ne.b32 p, %4, 0;\n\t"
+               "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}"
+               :: "r"(d_tmem), "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(m0), "r"(m1), "r"(m2), "r"(m3) : "memory");
+}
+
 template <int D>
-__global__ void __launch_bounds__(128, 2)
+__global__ void __launch_bounds__(128)
 linear_apply_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmH,
-                    const __grid_constant__ CUtensorMap tmW, const __nv_bfloat16* __restrict__ Hs,
-                    float* __restrict__ o_lin, SeqShape s, int has_w, int* status) {
+                    float* __restrict__ o_lin, SeqShape s, int* status) {
   using L = ApplyLayout<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint8_t* sQ = smem + L::kQOff;
   uint8_t* sH = smem + L::kHOff;
-  uint8_t* sW = smem + L::kWOff;
-  uint8_t* sO = smem + L::kOOff;
-  float* zs = reinterpret_cast<float*>(smem + L::kZOff);
-  float* den = zs + D;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  const int blk = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x, warp = tid >> 5;
-  const size_t hs_row = (size_t)bh * s.n_blocks + blk;
+  const int pair = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x, warp = tid >> 5;
+  const bool second = 2 * pair + 1 < s.n_blocks;
 
   if (tid == 0) {
     for (int i = 0; i < 3; ++i) mbar_init(&bars[i], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (D == 64 && has_w)
-    for (int i = tid; i < 8192 / 16; i += 128) reinterpret_cast<uint4*>(sW + D * 128)[i] = make_uint4(0, 0, 0, 0);
-  if (warp == 0) { tmem_alloc(tmem_slot, 128); tmem_relinquish(); }
+  if (warp == 0) { tmem_alloc(tmem_slot, 256); tmem_relinquish(); }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
   if (tid == 0) {
-    const uint32_t bytes = (D / 64) * (8192 + 16384) + (has_w ? (D / 64) * D * 128 : 0);
-    mbar_arrive_expect_tx(&bars[0], bytes);
+    const int nblk = second ? 2 : 1;
+    mbar_arrive_expect_tx(&bars[0], (D / 64) * 16384 + nblk * L::kHTile);
     for (int c = 0; c < D / 64; ++c) {
-      tma_load_3d(sQ + c * 8192, &tmQ, &bars[0], c * 64, blk * 64, bh);
-      tma_load_3d(sH + c * 16384, &tmH, &bars[0], c * 64, 0, (int)hs_row);
-      if (has_w) tma_load_3d(sW + c * D * 128, &tmW, &bars[0], c * 64, 0, 0);
+      tma_load_3d(sQ + c * 16384, &tmQ, &bars[0], c * 64, pair * 128, bh);
+      for (int b = 0; b < nblk; ++b)
+        tma_load_3d(sH + b * L::kHTile + c * L::kNL * 128, &tmH, &bars[0], c * 64, 0, bh * s.n_blocks + 2 * pair + b);
     }
   }
-  for (int a = tid; a < D; a += 128) zs[a] = __bfloat162float(Hs[(hs_row * (D + 1) + D) * D + a]);
   bool ok = cta_wait(&bars[0], 0, abort_flag, status);
-
-  // phi(Q_i) in place; pad tokens -> 0
-  constexpr int kCPR = D / 8, kRS = 128 / kCPR;
-  const int nvalid = block_valid_count(s, blk);
-  {
-    const int g = tid % kCPR, rs = tid / kCPR, chunk = g >> 3, q8 = g & 7;
-    if (ok)
-      for (int t = rs; t < 64; t += kRS) {
-        uint4* p = reinterpret_cast<uint4*>(sQ + chunk * 8192 + sw128_offset(t, q8));
-        const uint4 u = *p;
-        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-        uint32_t o[4];
-        #pragma unroll
-        for (int i = 0; i < 4; ++i)
-          o[i] = t < nvalid ? pack_bf16(phi_elu1(bf16_lo(w[i])), phi_elu1(bf16_hi(w[i]))) : 0u;
-        *p = make_uint4(o[0], o[1], o[2], o[3]);
-      }
-  }
-  __syncthreads();
-  // den[t] = phi(q_t) . Z_i  (two threads per token)
-  {
-    const int t = tid >> 1, hlf = tid & 1;
-    float part = 0.f;
-    for (int g = hlf * (kCPR / 2); g < (hlf + 1) * (kCPR / 2); ++g) {
-      const uint4 u = *reinterpret_cast<const uint4*>(sQ + (g >> 3) * 8192 + sw128_offset(t, g & 7));
+  // phi(Q) in place, one row per thread; pad rows -> 0
+  const int r = tid;
+  const int tok = pair * 128 + r;
+  const bool valid = tok < s.n_pad && token_valid(s, tok);
+  if (ok) {
+    #pragma unroll
+    for (int gg = 0; gg < D / 8; ++gg) {
+      uint4* ptr = reinterpret_cast<uint4*>(sQ + (gg >> 3) * 16384 + sw128_offset(r, gg & 7));
+      const uint4 u = *ptr;
       const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+      uint32_t o4[4];
       #pragma unroll
-      for (int i = 0; i < 4; ++i) part += bf16_lo(w[i]) * zs[g * 8 + 2 * i] + bf16_hi(w[i]) * zs[g * 8 + 2 * i + 1];
+      for (int i = 0; i < 4; ++i) o4[i] = valid ? pack_bf16(phi_elu1(bf16_lo(w[i])), phi_elu1(bf16_hi(w[i]))) : 0u;
+      *ptr = make_uint4(o4[0], o4[1], o4[2], o4[3]);
     }
-    part += __shfl_xor_sync(0xFFFFFFFFu, part, 1);
-    if (hlf == 0) den[t] = part;
   }
   fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
   if (tid == 0 && ok) {
     tc_fence_after();
-    constexpr uint32_t id = idesc_bf16(128, 64, false, false);
+    constexpr uint32_t id = idesc_bf16(128, L::kNL, false, false);
     #pragma unroll
     for (int kk = 0; kk < D / 16; ++kk) {
-      const uint64_t a = desc_kmajor(smem_u32(sH) + (kk >> 2) * 16384 + (kk & 3) * 32);
-      const uint64_t b = desc_kmajor(smem_u32(sQ) + (kk >> 2) * 8192 + (kk & 3) * 32);
-      mma_bf16_ss(tmem, a, b, id, kk > 0 ? 1u : 0u);
+      const uint64_t a = desc_kmajor(smem_u32(sQ) + (kk >> 2) * 16384 + (kk & 3) * 32);
+      const uint64_t b = desc_kmajor(smem_u32(sH) + (kk >> 2) * L::kNL * 128 + (kk & 3) * 32);
+      mma_masked(tmem, a, b, id, kk > 0 ? 1u : 0u, 0u, 0u, 0xFFFFFFFFu, 0xFFFFFFFFu);
+    }
+    if (second) {
+      #pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint64_t a = desc_kmajor(smem_u32(sQ) + (kk >> 2) * 16384 + (kk & 3) * 32);
+        const uint64_t b = desc_kmajor(smem_u32(sH) + L::kHTile + (kk >> 2) * L::kNL * 128 + (kk & 3) * 32);
+        mma_masked(tmem, a, b, id, kk > 0 ? 1u : 0u, 0xFFFFFFFFu, 0xFFFFFFFFu, 0u, 0u);
+      }
     }
     mma_commit(&bars[1]);
   }
   if (ok) ok = cta_wait(&bars[1], 0, abort_flag, status);
   tc_fence_after();
-  const int c = tid;                              // TMEM lane = output channel
-  const bool lane_active = warp * 32 < D;
-  float vals[64];
-  if (lane_active) {
-    if (ok) {
-      uint32_t r[32];
-      tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16), r);
-      tmem_wait_ld();
-      #pragma unroll
-      for (int t = 0; t < 32; ++t) vals[t] = den[t] > 0.f ? __uint_as_float(r[t]) / den[t] : 0.f;
-      tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + 32, r);
-      tmem_wait_ld();
-      #pragma unroll
-      for (int t = 0; t < 32; ++t) vals[32 + t] = den[32 + t] > 0.f ? __uint_as_float(r[t]) / den[32 + t] : 0.f;
-    } else {
-      #pragma unroll
-      for (int t = 0; t < 64; ++t) vals[t] = 0.f;
-    }
+  const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
+  float inv_den = 0.f;
+  if (ok) {
+    uint32_t dv;
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(dv) : "r"(lane_addr + D));
+    tmem_wait_ld();
+    const float den = __uint_as_float(dv);
+    inv_den = den > 0.f ? 1.f / den : 0.f;
   }
-  float* out = o_lin + ((size_t)bh * s.n_pad + (size_t)blk * 64) * D;
-  if (!has_w) {
-    if (lane_active)
-      #pragma unroll 4
-      for (int t = 0; t < 64; ++t) out[(size_t)t * D + c] = t < nvalid ? vals[t] : 0.f;
-  } else {
-    if (lane_active) {
-      __nv_bfloat16* base = reinterpret_cast<__nv_bfloat16*>(sO + (c >> 6) * 8192);
-      const int q8 = (c & 63) >> 3, e = c & 7;
-      #pragma unroll 8
-      for (int t = 0; t < 64; ++t)
-        base[(sw128_offset(t, q8) >> 1) + e] = __float2bfloat16_rn(vals[t]);
+  const bool row_exists = tok < s.n_pad;
+  float* out = o_lin + ((size_t)bh * s.n_pad + (row_exists ? tok : 0)) * D;
+  #pragma unroll 1
+  for (int cc = 0; cc < D / 32; ++cc) {
+    uint32_t v[32];
+    if (ok) {
+      tmem_ld32(lane_addr + cc * 32, v);
+      tmem_wait_ld();
     }
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    if (tid == 0 && ok) {
-      tc_fence_after();
-      constexpr uint32_t id = idesc_bf16(128, 64, true, false);
-      #pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        const uint64_t a = desc_mnmajor(smem_u32(sW) + kk * 2048, D * 128);
-        const uint64_t b = desc_kmajor(smem_u32(sO) + (kk >> 2) * 8192 + (kk & 3) * 32);
-        mma_bf16_ss(tmem + 64, a, b, id, kk > 0 ? 1u : 0u);
-      }
-      mma_commit(&bars[2]);
-    }
-    if (ok) ok = cta_wait(&bars[2], 0, abort_flag, status);
-    tc_fence_after();
-    if (lane_active) {
-      if (ok) {
-        #pragma unroll 1
-        for (int h2 = 0; h2 < 2; ++h2) {
-          uint32_t r[32];
-          tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + 64 + h2 * 32, r);
-          tmem_wait_ld();
-          #pragma unroll 4
-          for (int t = 0; t < 32; ++t) {
-            const int tt = h2 * 32 + t;
-            out[(size_t)tt * D + c] = tt < nvalid ? __uint_as_float(r[t]) : 0.f;
-          }
-        }
-      } else {
-        for (int t = 0; t < 64; ++t) out[(size_t)t * D + c] = 0.f;
-      }
+    if (!row_exists) continue;
+    float4* dst = reinterpret_cast<float4*>(out + cc * 32);
+    #pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (ok && valid)
+        f = make_float4(__uint_as_float(v[4 * i]) * inv_den, __uint_as_float(v[4 * i + 1]) * inv_den,
+                        __uint_as_float(v[4 * i + 2]) * inv_den, __uint_as_float(v[4 * i + 3]) * inv_den);
+      dst[i] = f;
     }
   }
   if (!ok && tid == 0) {
     mma_commit(&bars[2]);
     const long long t0 = clock64();
-    while (!mbar_try_wait(&bars[2], has_w ? 1 : 0) && clock64() - t0 < kWaitBudgetCycles) {}
+    while (!mbar_try_wait(&bars[2], 0) && clock64() - t0 < kWaitBudgetCycles) {}
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) { tc_fence_after(); tmem_dealloc(tmem, 128); }
+  if (warp == 0) { tc_fence_after(); tmem_dealloc(tmem, 256); }
 }
 
 }  // namespace
 
-cudaError_t launch_key_states(const void* k, const void* v, __nv_bfloat16* h, int BH, int d, SeqShape s,
-                              int* status, cudaStream_t st) {
-  CUtensorMap mk, mv;
+cudaError_t launch_key_states(const void* k, const void* v, const void* w_proj, __nv_bfloat16* h, int BH, int d,
+                              SeqShape s, int* status, cudaStream_t st) {
+  CUtensorMap mk, mv, mw;
   const uint64_t dims[3] = {(uint64_t)d, (uint64_t)s.n_pad, (uint64_t)BH};
   const uint64_t strides[2] = {(uint64_t)d * 2, (uint64_t)d * 2 * s.n_pad};
   const uint32_t box[3] = {64, 64, 1};
   if (!make_tile_map(&mk, k, 3, dims, strides, box) || !make_tile_map(&mv, v, 3, dims, strides, box))
     return cudaErrorInvalidValue;
-  dim3 grid(s.n_blocks, BH);
-  if (d == 128) {
-    cudaError_t e = cudaFuncSetAttribute(key_states_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, kKsSmemRequest);
-    if (e != cudaSuccess) return e;
-    key_states_kernel<128><<<grid, 128, kKsSmemRequest, st>>>(mk, mv, h, s, status);
+  if (w_proj) {
+    const uint64_t wdims[3] = {(uint64_t)d, (uint64_t)d, 1};
+    const uint64_t wstr[2] = {(uint64_t)d * 2, (uint64_t)d * 2 * d};
+    const uint32_t wbox[3] = {64, (uint32_t)d, 1};
+    if (!make_tile_map(&mw, w_proj, 3, wdims, wstr, wbox)) return cudaErrorInvalidValue;
   } else {
-    cudaError_t e = cudaFuncSetAttribute(key_states_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, kKsSmemRequest);
-    if (e != cudaSuccess) return e;
-    key_states_kernel<64><<<grid, 128, kKsSmemRequest, st>>>(mk, mv, h, s, status);
+    mw = mk;
   }
-  return cudaGetLastError();
+  dim3 grid(s.n_blocks, BH);
+  auto go = [&](auto kern) -> cudaError_t {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kKsSmemRequest);
+    if (e != cudaSuccess) return e;
+    kern<<<grid, 128, kKsSmemRequest, st>>>(mk, mv, mw, h, s, status);
+    return cudaGetLastError();
+  };
+  if (d == 128) return w_proj ? go(key_states_kernel<128, true>) : go(key_states_kernel<128, false>);
+  return w_proj ? go(key_states_kernel<64, true>) : go(key_states_kernel<64, false>);
 }
 
 cudaError_t launch_reduce_states(const __nv_bfloat16* m01, int ld_m01, const __nv_bfloat16* h,
@@ -484,35 +494,26 @@ cudaError_t launch_reduce_states(const __nv_bfloat16* m01, int ld_m01, const __n
   return cudaGetLastError();
 }
 
-cudaError_t launch_linear_apply(const void* q, const __nv_bfloat16* Hs, const void* w_proj,
-                                float* o_lin, int BH, int d, SeqShape s, int* status, cudaStream_t st) {
-  CUtensorMap mq, mh, mw;
+cudaError_t launch_linear_apply(const void* q, const __nv_bfloat16* Hs, float* o_lin, int BH, int d, SeqShape s,
+                                int* status, cudaStream_t st) {
+  CUtensorMap mq, mh;
   const uint64_t qdims[3] = {(uint64_t)d, (uint64_t)s.n_pad, (uint64_t)BH};
   const uint64_t qstr[2] = {(uint64_t)d * 2, (uint64_t)d * 2 * s.n_pad};
-  const uint32_t qbox[3] = {64, 64, 1};
+  const uint32_t qbox[3] = {64, 128, 1};
   const uint64_t hdims[3] = {(uint64_t)d, (uint64_t)(d + 1), (uint64_t)BH * s.n_blocks};
   const uint64_t hstr[2] = {(uint64_t)d * 2, (uint64_t)d * 2 * (d + 1)};
-  const uint32_t hbox[3] = {64, 128, 1};
+  const uint32_t hbox[3] = {64, (uint32_t)(d + 16), 1};
   if (!make_tile_map(&mq, q, 3, qdims, qstr, qbox) || !make_tile_map(&mh, Hs, 3, hdims, hstr, hbox))
     return cudaErrorInvalidValue;
-  if (w_proj) {
-    const uint64_t wdims[3] = {(uint64_t)d, (uint64_t)d, 1};
-    const uint64_t wstr[2] = {(uint64_t)d * 2, (uint64_t)d * 2 * d};
-    const uint32_t wbox[3] = {64, (uint32_t)d, 1};
-    if (!make_tile_map(&mw, w_proj, 3, wdims, wstr, wbox)) return cudaErrorInvalidValue;
-  } else {
-    mw = mq;
-  }
-  dim3 grid(s.n_blocks, BH);
-  const int has_w = w_proj ? 1 : 0;
+  dim3 grid((s.n_blocks + 1) / 2, BH);
   if (d == 128) {
     cudaError_t e = cudaFuncSetAttribute(linear_apply_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, ApplyLayout<128>::kBytes);
     if (e != cudaSuccess) return e;
-    linear_apply_kernel<128><<<grid, 128, ApplyLayout<128>::kBytes, st>>>(mq, mh, mw, Hs, o_lin, s, has_w, status);
+    linear_apply_kernel<128><<<grid, 128, ApplyLayout<128>::kBytes, st>>>(mq, mh, o_lin, s, status);
   } else {
     cudaError_t e = cudaFuncSetAttribute(linear_apply_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, ApplyLayout<64>::kBytes);
     if (e != cudaSuccess) return e;
-    linear_apply_kernel<64><<<grid, 128, ApplyLayout<64>::kBytes, st>>>(mq, mh, mw, Hs, o_lin, s, has_w, status);
+    linear_apply_kernel<64><<<grid, 128, ApplyLayout<64>::kBytes, st>>>(mq, mh, o_lin, s, status);
   }
   return cudaGetLastError();
 }

@@ -82,7 +82,7 @@ struct AttnArgs {
   const uint32_t* list;                // null = dense
   const int32_t* list_cnt;
   int list_cap, list_per_head;         // list_per_head = 0 when one list serves all heads
-  const float* addend;                 // fp32 [BH][n_pad][d] added to the output, or null
+  const __nv_bfloat16* Hs;             // SLA linear branch: [BH][n_qb][(d+1)][d] rows [H_i'^T ; Z_i], or null
   void* out;                           // bf16 [BH][n_pad][d]
   float* lse;                          // fp32 [BH][n_pad] or null
   int tile3d;                          // 1: blocks are 4x4x4 tiles of raster (F, Hh, Ww)
@@ -94,16 +94,17 @@ struct AttnArgs {
 cudaError_t launch_attention(const AttnArgs& a, cudaStream_t st);
 
 // ------------------------------------------------------------ marginal branch (k_marginal.cu)
-// h[bh][j] = [ (phi(K_j)^T V_j)^T (d rows of d) ; z_j (1 row) ] in bf16, [BH][nb][(d+1)*d].
-cudaError_t launch_key_states(const void* k, const void* v, __nv_bfloat16* h, int BH, int d, SeqShape s,
-                              int* status, cudaStream_t st);
+// h[bh][j] = [ (phi(K_j)^T V_j W)^T (d rows of d) ; z_j (1 row) ] in bf16, [BH][nb][(d+1)*d];
+// W = w_proj (bf16 [d][d]) or the identity when w_proj is null.
+cudaError_t launch_key_states(const void* k, const void* v, const void* w_proj, __nv_bfloat16* h, int BH, int d,
+                              SeqShape s, int* status, cudaStream_t st);
 
 // Hs[bh][i] = sum_j m01[bh][i][j] * h[bh][j]  (bf16 out, fp32 accumulate), [BH][nb][(d+1)*d].
 cudaError_t launch_reduce_states(const __nv_bfloat16* m01, int ld_m01, const __nv_bfloat16* h,
                                  __nv_bfloat16* Hs, int BH, int nb, int d, int* status, cudaStream_t st);
 
-// o_lin[bh][t] = (phi(q_t) H_i / (phi(q_t).Z_i)) [@ W_proj] for every valid token t of block i.
-cudaError_t launch_linear_apply(const void* q, const __nv_bfloat16* Hs, const void* w_proj,
-                                float* o_lin, int BH, int d, SeqShape s, int* status, cudaStream_t st);
+// o_lin[bh][t] = phi(q_t) H_i' / (phi(q_t).Z_i) for every valid token t of block i (0 for pads).
+cudaError_t launch_linear_apply(const void* q, const __nv_bfloat16* Hs, float* o_lin, int BH, int d, SeqShape s,
+                                int* status, cudaStream_t st);
 
 }  // namespace slr

@@ -144,7 +144,6 @@ struct SlaWs {
   int32_t* list_cnt;
   int cap;
   MarginalWs mar;
-  float* olin;
 };
 
 void plan_sla(Carve& c, const Shape& sh, int kc, int kn, bool own_mask, SlaWs& w) {
@@ -160,10 +159,8 @@ void plan_sla(Carve& c, const Shape& sh, int kc, int kn, bool own_mask, SlaWs& w
   w.list_cnt = c.take<int32_t>((size_t)sh.BH * sh.npairs);
   if (sh.nb - kc - kn > 0) {
     plan_marginal(c, sh, w.mar);
-    w.olin = c.take<float>((size_t)sh.BH * sh.n_pad * sh.d);
   } else {
     w.mar.h = w.mar.Hs = nullptr;
-    w.olin = nullptr;
   }
 }
 
@@ -505,9 +502,9 @@ slr_status slr_linear_marginal(const void* q, const void* k, const void* v, cons
   plan_marginal(c, sh, w);
   SLR_TRY(cudaMemsetAsync(status, 0, sizeof(int), s));
   SLR_LAUNCH(kKMaskToM01, s, launch_mask_to_m01(mask, m01, sh.BH, sh.nb, ld_m01(sh.nb), s));
-  SLR_LAUNCH(kKKeyStates, s, launch_key_states(k, v, w.h, sh.BH, sh.d, sh.s, status, s));
+  SLR_LAUNCH(kKKeyStates, s, launch_key_states(k, v, w_proj_opt, w.h, sh.BH, sh.d, sh.s, status, s));
   SLR_LAUNCH(kKReduce, s, launch_reduce_states(m01, ld_m01(sh.nb), w.h, w.Hs, sh.BH, sh.nb, sh.d, status, s));
-  SLR_LAUNCH(kKApply, s, launch_linear_apply(q, w.Hs, w_proj_opt, o_lin, sh.BH, sh.d, sh.s, status, s));
+  SLR_LAUNCH(kKApply, s, launch_linear_apply(q, w.Hs, o_lin, sh.BH, sh.d, sh.s, status, s));
   return SLR_OK;
 }
 
@@ -551,10 +548,9 @@ slr_status slr_sparse_linear_attn(const void* q, const void* k, const void* v, c
   la.list = w.list; la.list_cnt = w.list_cnt; la.status = w.status;
   SLR_LAUNCH(kKLists, s, launch_pair_lists(la, sh.BH, s));
   if (marginal) {
-    SLR_LAUNCH(kKKeyStates, s, launch_key_states(k, v, w.mar.h, sh.BH, sh.d, sh.s, w.status, s));
+    SLR_LAUNCH(kKKeyStates, s, launch_key_states(k, v, w_proj, w.mar.h, sh.BH, sh.d, sh.s, w.status, s));
     SLR_LAUNCH(kKReduce, s, launch_reduce_states(w.cls.m01, ld_m01(sh.nb), w.mar.h, w.mar.Hs, sh.BH, sh.nb, sh.d, w.status, s));
-    SLR_LAUNCH(kKApply, s, launch_linear_apply(q, w.mar.Hs, w_proj, w.olin, sh.BH, sh.d, sh.s, w.status, s));
-    a.addend = w.olin;
+    a.Hs = w.mar.Hs;
   }
   a.list = w.list; a.list_cnt = w.list_cnt; a.list_cap = w.cap; a.list_per_head = 1;
   SLR_LAUNCH(kKAttention, s, launch_attention(a, s));
