@@ -71,8 +71,8 @@ def test_lvsa_sets_rejects_bad_budget(lib):
 def test_workspace_bytes(lib):
     good = slr.make_seq(1, 12, 128, 1, 32760, 32768)
     n = slr.slr_workspace_bytes(slr.SLR_OP_SPARSE_LINEAR, good, slr.SlrFracs(0.05, 0.10))
-    # at least h and H (bf16, (d+1)d per block per head) and the fp32 linear output
-    assert n >= 2 * 12 * 512 * 129 * 128 * 2 + 12 * 32768 * 128 * 4
+    # at least h and H (bf16, (d+1)d per block per head)
+    assert n >= 2 * 12 * 512 * 129 * 128 * 2
     dense = slr.slr_workspace_bytes(slr.SLR_OP_SPARSE_LINEAR, good, slr.SlrFracs(1.0, 0.0))
     assert 0 < dense <= 4096
     for bad in [slr.make_seq(1, 1, 96, 1, 64, 64),          # d unsupported
