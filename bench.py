@@ -135,7 +135,7 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ CPU oracle sample
 
-def cpu_oracle_sample(w, q, k, v, wp, rows_per_head=8, heads=1):
+def cpu_oracle_sample(w, q, k, v, wp, rows_per_head=256, heads=12):
     """Time the fp64 oracle on `heads` heads: full classification + `rows_per_head` query blocks.
 
     Returns (extrapolated ms per full call, description, threads).
@@ -188,13 +188,14 @@ def cpu_oracle_sample(w, q, k, v, wp, rows_per_head=8, heads=1):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="slr", choices=["slr", "reference"])
     ap.add_argument("--workload", default=WORKLOAD.name, choices=sorted(workloads.BY_NAME))
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--oracle-rows", type=int, default=8)
+    ap.add_argument("--oracle-rows", type=int, default=256, help="query blocks per head in the CPU oracle sample")
+    ap.add_argument("--oracle-heads", type=int, default=12, help="heads in the CPU oracle sample")
     args = ap.parse_args()
     w = workloads.BY_NAME[args.workload]
     if w.mode != "sla":
@@ -264,13 +265,13 @@ def main():
     if slr.slr_check_status(ws_sparse, dev) != slr.SLR_OK:
         raise SystemExit("device status error during warm-up")
 
-    # timed region 1: the sparse call (the metric); clocks sampled during it
+    # timed region 1: the sparse call (the metric); clocks are sampled from here
+    # through the dense, profiled and end-to-end regions
     clocks = ClockSampler(local)
     clocks.start()
-    time.sleep(0.3)
+    time.sleep(0.25)
     ms_sparse = timed(call, args.steps)
-    clk = clocks.stop()
-    ms_dense = timed(lambda: call(dense=True), max(3, args.steps // 2))
+    ms_dense = timed(lambda: call(dense=True), max(3, args.steps // 4))
 
     # timed region 2: the same steps with the per-kernel event profiler on
     slr.slr_profile_enable(True)
@@ -312,10 +313,12 @@ def main():
         h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv, hw))
         d2h = ho.numel() * ho.element_size()
         e2e = {"value": round(e2e_ms / world, 4), "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+    clk = clocks.stop()
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cms, desc, threads = cpu_oracle_sample(w, q_h, k_h, v_h, wp_h, rows_per_head=args.oracle_rows)
+        cms, desc, threads = cpu_oracle_sample(w, q_h, k_h, v_h, wp_h, rows_per_head=args.oracle_rows,
+                                               heads=args.oracle_heads)
         cpu = {"value": round(cms, 1), "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc,
                "host_cpus": os.cpu_count()}
 
@@ -367,15 +370,15 @@ def run_reference(args, w, rank, world, warmup):
     """The reference arm: the fp64 oracle on the host cores, bounded samples."""
     if rank != 0:
         return
-    q, k, v = workloads.make_qkv(w, heads=1)
+    q, k, v = workloads.make_qkv(w)
     wp = workloads.make_w_proj(w)
-    rows = max(1, min(args.oracle_rows, 4))
+    rows, heads = args.oracle_rows, args.oracle_heads
     for _ in range(min(warmup, 1)):
-        cpu_oracle_sample(w, q, k, v, wp, rows_per_head=rows)
+        cpu_oracle_sample(w, q, k, v, wp, rows_per_head=rows, heads=heads)
     vals = []
     desc, threads = "", 1
     for _ in range(max(1, min(args.steps, 3))):
-        ms, desc, threads = cpu_oracle_sample(w, q, k, v, wp, rows_per_head=rows)
+        ms, desc, threads = cpu_oracle_sample(w, q, k, v, wp, rows_per_head=rows, heads=heads)
         vals.append(ms)
     val = statistics.median(vals)
     line = {
