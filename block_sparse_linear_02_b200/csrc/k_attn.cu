@@ -57,8 +57,8 @@ struct AttnLayout {
   static constexpr int kQOff = 0;
   static constexpr int kKOff = kQOff + kChunks * kQChunk;
   static constexpr int kVOff = kKOff + kStages * kKVTile;
-  static constexpr int kPOff = kVOff + kStages * kKVTile;
-  static constexpr int kXOff = kPOff + 128 * 128;        // exchange area: 6 x 128 floats
+  static constexpr int kPOff = kVOff + kStages * kKVTile;    // two P buffers of 128 rows x 64 keys
+  static constexpr int kXOff = kPOff + 2 * 128 * 128;    // exchange area: 6 x 128 floats
   static constexpr int kBarOff = kXOff + 6 * 128 * 4;
   static constexpr int kBytes = kBarOff + 256 + 1024;    // + alignment slack
   static_assert(2 * kHsTile <= 2 * kStages * kKVTile, "linear state tiles must fit in the K/V ring");
@@ -130,10 +130,10 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
   uint64_t* k_full = bars + 1;
   uint64_t* v_full = bars + 1 + kStages;
   uint64_t* kv_empty = bars + 1 + 2 * kStages;
-  uint64_t* s_full = bars + 1 + 3 * kStages;     // [2]
-  uint64_t* p_full = s_full + 2;                 // [2]  one per softmax warpgroup
-  uint64_t* o_bar = p_full + 2;                  // [2]
-  uint64_t* loop_done = o_bar + 2;
+  uint64_t* s_full = bars + 1 + 3 * kStages;     // [2]  per S buffer
+  uint64_t* p_full = s_full + 2;                 // [4]  [warpgroup * 2 + P buffer]
+  uint64_t* o_bar = p_full + 4;                  // [4]  [warpgroup * 2 + P buffer]
+  uint64_t* loop_done = o_bar + 4;
   uint64_t* hs_full = loop_done + 1;
   uint64_t* phiq_ready = hs_full + 1;
   uint64_t* lin_done = phiq_ready + 1;
@@ -161,10 +161,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
     for (int s = 0; s < kStages; ++s) { mbar_init(&k_full[s], 1); mbar_init(&v_full[s], 1); mbar_init(&kv_empty[s], 1); }
     mbar_init(&s_full[0], 1);
     mbar_init(&s_full[1], 1);
-    mbar_init(&p_full[0], 128);
-    mbar_init(&p_full[1], 128);
-    mbar_init(&o_bar[0], 1);
-    mbar_init(&o_bar[1], 1);
+    for (int i = 0; i < 4; ++i) { mbar_init(&p_full[i], 128); mbar_init(&o_bar[i], 1); }
     mbar_init(loop_done, 1);
     mbar_init(hs_full, 1);
     mbar_init(phiq_ready, 256);
@@ -251,9 +248,9 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
           mma_bf16_ss(tmem + kColS + sbuf * 64, a, b, idS, kk > 0 ? 1u : 0u);
         }
       };
-      auto issue_pv = [&](int stage, uint32_t col, int kk0, int kk1, bool acc) {
+      auto issue_pv = [&](int stage, int pbuf, uint32_t col, int kk0, int kk1, bool acc) {
         for (int kk = kk0; kk < kk1; ++kk) {
-          uint64_t a = desc_kmajor(p_addr + kk * 32);
+          uint64_t a = desc_kmajor(p_addr + pbuf * 16384 + kk * 32);
           uint64_t b = desc_mnmajor(v_addr + stage * L::kKVTile + kk * 2048, L::kKVChunk);
           mma_bf16_ss(tmem + col, a, b, idO, (acc || kk > kk0) ? 1u : 0u);
         }
@@ -274,22 +271,24 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
           const int s = j % kStages;
           if (!mbar_wait(&v_full[s], (j / kStages) & 1, abort_flag, p.status)) { ok = false; break; }
           const bool far = GATED && j == n_local;
+          const int pb = j & 1;
+          const uint32_t ph = (j >> 1) & 1;
           if (far) {
-            if (!mbar_wait(&p_full[0], j & 1, abort_flag, p.status) ||
-                !mbar_wait(&p_full[1], j & 1, abort_flag, p.status)) { ok = false; break; }
+            if (!mbar_wait(&p_full[pb], ph, abort_flag, p.status) ||
+                !mbar_wait(&p_full[2 + pb], ph, abort_flag, p.status)) { ok = false; break; }
             tc_fence_after();
-            issue_pv(s, kColOf, 0, 4, false);
-            mma_commit(&o_bar[0]);
-            mma_commit(&o_bar[1]);
+            issue_pv(s, pb, kColOf, 0, 4, false);
+            mma_commit(&o_bar[pb]);
+            mma_commit(&o_bar[2 + pb]);
           } else {
-            if (!mbar_wait(&p_full[0], j & 1, abort_flag, p.status)) { ok = false; break; }
+            if (!mbar_wait(&p_full[pb], ph, abort_flag, p.status)) { ok = false; break; }
             tc_fence_after();
-            issue_pv(s, kColO0, 0, 2, j > 0);
-            mma_commit(&o_bar[0]);
-            if (!mbar_wait(&p_full[1], j & 1, abort_flag, p.status)) { ok = false; break; }
+            issue_pv(s, pb, kColO0, 0, 2, j > 0);
+            mma_commit(&o_bar[pb]);
+            if (!mbar_wait(&p_full[2 + pb], ph, abort_flag, p.status)) { ok = false; break; }
             tc_fence_after();
-            issue_pv(s, kColO1, 2, 4, j > 0);
-            mma_commit(&o_bar[1]);
+            issue_pv(s, pb, kColO1, 2, 4, j > 0);
+            mma_commit(&o_bar[2 + pb]);
           }
           mma_commit(&kv_empty[s]);
         }
@@ -414,12 +413,18 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
         rowsum = acc0 + acc1;
       }
       if (far) l_far += rowsum; else l_run += rowsum;
-      // my half of the P buffer and my accumulator are free once P_{j-1} V_{j-1} (my half) has completed
-      if (j > 0) {
-        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&o_bar[wg], (j - 1) & 1, abort_flag, p.status))) { ok = false; break; }
-        tc_fence_after();
+      // P buffer j&1 (my half) is free once P_{j-2} V_{j-2} has completed; my accumulator
+      // may be rescaled once P_{j-1} V_{j-1} has completed
+      const int pb = j & 1;
+      if (j >= 2) {
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&o_bar[wg * 2 + pb], ((j - 2) >> 1) & 1, abort_flag, p.status))) { ok = false; break; }
       }
-      if (!far && j > 0 && __any_sync(0xFFFFFFFFu, need)) {
+      const bool rescale = !far && j > 0 && __any_sync(0xFFFFFFFFu, need);
+      if (rescale) {
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&o_bar[wg * 2 + (pb ^ 1)], ((j - 1) >> 1) & 1, abort_flag, p.status))) { ok = false; break; }
+      }
+      tc_fence_after();
+      if (rescale) {
         #pragma unroll 1
         for (int cc = 0; cc < D / 32; ++cc) {
           uint32_t o[32];
@@ -434,13 +439,14 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
       #pragma unroll
       for (int c8 = 0; c8 < 4; ++c8) {
         uint4 val = make_uint4(packed[4 * c8], packed[4 * c8 + 1], packed[4 * c8 + 2], packed[4 * c8 + 3]);
-        *reinterpret_cast<uint4*>(sP + sw128_offset(r, 4 * wg + c8)) = val;
+        *reinterpret_cast<uint4*>(sP + pb * 16384 + sw128_offset(r, 4 * wg + c8)) = val;
       }
       fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(&p_full[wg]);
+      mbar_arrive(&p_full[wg * 2 + pb]);
     }
-    if (ok && total > 0) ok = __all_sync(0xFFFFFFFFu, mbar_wait(&o_bar[wg], (total - 1) & 1, abort_flag, p.status));
+    if (ok && total > 0)
+      ok = __all_sync(0xFFFFFFFFu, mbar_wait(&o_bar[wg * 2 + ((total - 1) & 1)], ((total - 1) >> 1) & 1, abort_flag, p.status));
     ok = __all_sync(0xFFFFFFFFu, ok);
     tc_fence_after();
 

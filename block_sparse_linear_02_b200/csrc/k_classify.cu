@@ -10,8 +10,10 @@
 //
 // block_logits_kernel: 64x64 output tiles of qbar kbar^T / sqrt(d) (fp64 FMA).
 // classify_rows_kernel: one warp per row; two MSB-first radix selections over
-//   order-preserving 64-bit keys (8 passes of 8-bit digits) find the kc-th
-//   largest and kn-th smallest key; one pass in index order applies the
+//   order-preserving 64-bit keys (8-bit digits, warp-aggregated histogram
+//   counts, stopping once the remaining candidates are exactly the ones
+//   needed) find the kc-th largest and kn-th smallest key; one pass in index
+//   order applies the
 //   thresholds with index tie-breaking and emits the mask row, the ascending
 //   critical list, the marginal indicator row (bf16 1/0 for the tensor-core
 //   contraction) and, on request, P_c in fp32.
@@ -25,23 +27,25 @@
 namespace slr {
 namespace {
 
-__global__ void __launch_bounds__(256)
+// One CTA of 64 threads computes a 64x64 tile; each thread an 8x8 sub-tile, so
+// every pair of shared-memory loads feeds four fp64 FMAs.
+__global__ void __launch_bounds__(64)
 block_logits_kernel(const double* __restrict__ qbar, const double* __restrict__ kbar,
                     double* __restrict__ logits, int nb, int d, double sqrt_d) {
-  __shared__ double As[16][64 + 1];
-  __shared__ double Bs[16][64 + 1];
+  __shared__ double As[16][64];
+  __shared__ double Bs[16][64];
   const int bh = blockIdx.z;
   const int i0 = blockIdx.y * 64, j0 = blockIdx.x * 64;
   const double* A = qbar + (size_t)bh * nb * d;
   const double* B = kbar + (size_t)bh * nb * d;
-  const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
-  double acc[4][4];
+  const int tx = threadIdx.x % 8, ty = threadIdx.x / 8;
+  double acc[8][8];
   #pragma unroll
-  for (int a = 0; a < 4; ++a)
+  for (int a = 0; a < 8; ++a)
     #pragma unroll
-    for (int b = 0; b < 4; ++b) acc[a][b] = 0.0;
+    for (int b = 0; b < 8; ++b) acc[a][b] = 0.0;
   for (int c0 = 0; c0 < d; c0 += 16) {
-    for (int e = threadIdx.x; e < 64 * 16; e += 256) {
+    for (int e = threadIdx.x; e < 64 * 16; e += 64) {
       const int row = e / 16, col = e % 16;
       As[col][row] = (i0 + row < nb) ? A[(size_t)(i0 + row) * d + c0 + col] : 0.0;
       Bs[col][row] = (j0 + row < nb) ? B[(size_t)(j0 + row) * d + c0 + col] : 0.0;
@@ -49,23 +53,23 @@ block_logits_kernel(const double* __restrict__ qbar, const double* __restrict__ 
     __syncthreads();
     #pragma unroll
     for (int c = 0; c < 16; ++c) {
-      double a[4], b[4];
+      double a[8], b[8];
       #pragma unroll
-      for (int u = 0; u < 4; ++u) { a[u] = As[c][ty * 4 + u]; b[u] = Bs[c][tx * 4 + u]; }
+      for (int u = 0; u < 8; ++u) { a[u] = As[c][ty * 8 + u]; b[u] = Bs[c][tx * 8 + u]; }
       #pragma unroll
-      for (int u = 0; u < 4; ++u)
+      for (int u = 0; u < 8; ++u)
         #pragma unroll
-        for (int w = 0; w < 4; ++w) acc[u][w] = fma(a[u], b[w], acc[u][w]);
+        for (int w = 0; w < 8; ++w) acc[u][w] = fma(a[u], b[w], acc[u][w]);
     }
     __syncthreads();
   }
   #pragma unroll
-  for (int u = 0; u < 4; ++u) {
-    const int i = i0 + ty * 4 + u;
+  for (int u = 0; u < 8; ++u) {
+    const int i = i0 + ty * 8 + u;
     if (i >= nb) continue;
     #pragma unroll
-    for (int w = 0; w < 4; ++w) {
-      const int j = j0 + tx * 4 + w;
+    for (int w = 0; w < 8; ++w) {
+      const int j = j0 + tx * 8 + w;
       if (j < nb) logits[((size_t)bh * nb + i) * nb + j] = acc[u][w] / sqrt_d;
     }
   }
@@ -89,18 +93,28 @@ __device__ __forceinline__ int warp_incl_scan(int v, int lane) {
 }
 
 // MSB-first radix selection of the k-th largest (largest=true) or k-th smallest
-// key among keys[0..n).  Returns the key value T, how many of the keys equal to
-// T are taken (take), and how many keys equal T in total (eq_total).
+// key among keys[0..n), 8 bits per pass.  Returns the selection at the level
+// `shift` where it was settled: T (the key's bits above `shift`), how many of
+// the keys whose bits above `shift` equal T are taken (take), and how many such
+// keys there are (eq_total).  The passes stop early once every remaining
+// candidate is needed.
 __device__ void radix_select(const uint64_t* keys, int n, int k, bool largest, unsigned* hist, int lane,
-                             uint64_t& T, int& take, int& eq_total) {
+                             uint64_t& T, int& shift_out, int& take, int& eq_total) {
   uint64_t prefix = 0, pmask = 0;
-  int kk = k, last = 0;
-  for (int shift = 56; shift >= 0; shift -= 8) {
+  int kk = k, last = 0, shift = 56;
+  for (;; shift -= 8) {
     for (int b = lane; b < 256; b += 32) hist[b] = 0;
     __syncwarp();
-    for (int j = lane; j < n; j += 32) {
-      const uint64_t u = keys[j];
-      if ((u & pmask) == prefix) atomicAdd(&hist[(u >> shift) & 255], 1u);
+    for (int j0 = 0; j0 < n; j0 += 32) {
+      const int j = j0 + lane;
+      const uint64_t u = j < n ? keys[j] : 0;
+      const bool cand = j < n && (u & pmask) == prefix;
+      const unsigned bin = (unsigned)((u >> shift) & 255);
+      const unsigned act = __ballot_sync(0xFFFFFFFFu, cand);
+      if (cand) {
+        const unsigned peers = __match_any_sync(act, bin);
+        if ((__ffs(peers) - 1) == lane) atomicAdd(&hist[bin], (unsigned)__popc(peers));
+      }
     }
     __syncwarp();
     int cnt[8], lsum = 0;
@@ -131,8 +145,10 @@ __device__ void radix_select(const uint64_t* keys, int n, int k, bool largest, u
     prefix |= (uint64_t)sel << shift;
     pmask |= (uint64_t)0xFF << shift;
     __syncwarp();
+    if (last == kk || shift == 0) break;      // every remaining candidate is needed, or fully resolved
   }
-  T = prefix;
+  T = prefix >> shift;
+  shift_out = shift;
   take = kk;
   eq_total = last;
 }
@@ -166,24 +182,25 @@ classify_rows_kernel(const double* __restrict__ logits, int rows, int nb, int kc
   }
   __syncwarp();
   uint64_t Tc = 0, Tn = 0;
-  int take_c = 0, eq_c = 0, take_n = 0, eq_n = 0;
-  radix_select(keys, nb, kc, true, hist, lane, Tc, take_c, eq_c);
-  if (kn > 0) radix_select(keys, nb, kn, false, hist, lane, Tn, take_n, eq_n);
+  int sc = 0, sn = 0, take_c = 0, eq_c = 0, take_n = 0, eq_n = 0;
+  radix_select(keys, nb, kc, true, hist, lane, Tc, sc, take_c, eq_c);
+  if (kn > 0) radix_select(keys, nb, kn, false, hist, lane, Tn, sn, take_n, eq_n);
   const unsigned lt_mask = (1u << lane) - 1u;
   int seen_c = 0, seen_n = 0, written = 0;
   for (int base = 0; base < nb; base += 32) {
     const int j = base + lane;
     const bool in = j < nb;
     const uint64_t u = in ? keys[j] : 0;
-    const bool eqc = in && u == Tc;
+    const uint64_t uc = u >> sc, un = u >> sn;
+    const bool eqc = in && uc == Tc;
     const unsigned bc = __ballot_sync(0xFFFFFFFFu, eqc);
-    const bool crit = (in && u > Tc) || (eqc && seen_c + __popc(bc & lt_mask) < take_c);
+    const bool crit = (in && uc > Tc) || (eqc && seen_c + __popc(bc & lt_mask) < take_c);
     seen_c += __popc(bc);
     bool negl = false;
     if (kn > 0) {
-      const bool eqn = in && u == Tn;
+      const bool eqn = in && un == Tn;
       const unsigned bn = __ballot_sync(0xFFFFFFFFu, eqn);
-      negl = (in && u < Tn) || (eqn && seen_n + __popc(bn & lt_mask) >= eq_n - take_n);
+      negl = (in && un < Tn) || (eqn && seen_n + __popc(bn & lt_mask) >= eq_n - take_n);
       seen_n += __popc(bn);
     }
     if (in) {
@@ -217,7 +234,7 @@ __global__ void mask_to_m01_kernel(const int8_t* __restrict__ mask, __nv_bfloat1
 cudaError_t launch_block_logits(const double* qbar, const double* kbar, double* logits,
                                 int BH, int nb, int d, cudaStream_t st) {
   dim3 grid((nb + 63) / 64, (nb + 63) / 64, BH);
-  block_logits_kernel<<<grid, 256, 0, st>>>(qbar, kbar, logits, nb, d, sqrt((double)d));
+  block_logits_kernel<<<grid, 64, 0, st>>>(qbar, kbar, logits, nb, d, sqrt((double)d));
   return cudaGetLastError();
 }
 
