@@ -14,18 +14,22 @@
 //
 // One CTA owns a PAIR of consecutive query blocks (128 query rows = the M of a
 // tcgen05 MMA) and walks the union of their key-block sets; each list entry
-// carries one flag per half, and a half that does not attend a block masks it.
+// carries the block's valid-key count and one flag per half of the pair.  The
+// list is consumed two entries per STEP (128 keys): one 128x128 S tile per step
+// keeps the MMA instruction count and the commits per key low.
 // Warp roles (320 threads):
-//   warp 8     TMA producer: Q once, K_j / V_j into a 3-stage ring, then the
+//   warp 8     TMA producer: Q once, then K_0, V_0, K_1, V_1, ... (each item the
+//              step's two 64-key blocks) into a 5-slot ring, then the
 //              linear-branch state rows;
-//   warp 9     MMA issuer: S_j = Q K_j^T into one of two TMEM S buffers; once a
-//              softmax warpgroup has written its half of P_j to shared memory,
-//              O_w += P_j[:, half w] V_j[half w, :];
-//   warps 0-3  softmax warpgroup 0: key columns 0-31 of every block;
-//   warps 4-7  softmax warpgroup 1: key columns 32-63.
+//   warp 9     MMA issuer: S_j = Q [K_a ; K_b]^T (N = 128) into one of two TMEM
+//              S buffers; once both softmax warpgroups have written P_j back
+//              over S_j (bf16, in TMEM), O_0 += P_j[:, a] V_a and
+//              O_1 += P_j[:, b] V_b with the A operand read from TMEM;
+//   warps 0-3  softmax warpgroup 0: the first block of every step;
+//   warps 4-7  softmax warpgroup 1: the second block.
 // Each warpgroup runs its own online softmax (own running max and sum, own TMEM
-// accumulator O_w) over its half of the keys; the epilogue merges the two
-// halves exactly: O = (2^(m0-M) O_0 + 2^(m1-M) O_1) / (2^(m0-M) l_0 + 2^(m1-M) l_1).
+// accumulator O_w) over its share of the key blocks; the epilogue merges the two
+// shares exactly: O = (2^(m0-M) O_0 + 2^(m1-M) O_1) / (2^(m0-M) l_0 + 2^(m1-M) l_1).
 // The softmax works in the exp2 domain with lazy rescaling (an accumulator is
 // rescaled only when its running max grows by more than 2^8).
 #include <cuda_runtime.h>
@@ -37,31 +41,28 @@
 namespace slr {
 namespace {
 
-constexpr int kStages = 3;
+constexpr int kSlots = 5;           // ring of K/V items, each 128 rows x d
 constexpr int kThreads = 320;
 constexpr uint32_t kColO0 = 0;      // accumulator of warpgroup 0
 constexpr uint32_t kColO1 = 128;    // accumulator of warpgroup 1
-constexpr uint32_t kColS = 256;     // two 64-column S buffers
-constexpr uint32_t kColLin = 256;   // linear branch result (reuses S after the loop)
-constexpr uint32_t kColOf = 384;    // far-field accumulator
+constexpr uint32_t kColS = 256;     // two 128-column S/P buffers: [256, 384) and [384, 512)
+constexpr uint32_t kColLin = 256;   // linear branch result (reuses the S buffers after the loop)
 
 template <int D>
 struct AttnLayout {
   static constexpr int kChunks = D / 64;                 // 64-column (128-byte) chunks
-  static constexpr int kQChunk = 128 * 128;              // bytes of one Q chunk (128 rows)
-  static constexpr int kKVChunk = 64 * 128;              // bytes of one K/V chunk (64 rows)
-  static constexpr int kKVTile = kChunks * kKVChunk;
+  static constexpr int kTile = 128 * 128;                // bytes of one 128-row chunk (Q, or two K/V blocks)
+  static constexpr int kHalf = 64 * 128;                 // bytes of one 64-row block inside a chunk
+  static constexpr int kKV = kChunks * kTile;            // one ring item: K (or V) of one step
   static constexpr int kNL = D + 16;                     // rows of a linear state tile (d + z + zero pad)
   static constexpr int kHsChunk = kNL * 128;
   static constexpr int kHsTile = kChunks * kHsChunk;
   static constexpr int kQOff = 0;
-  static constexpr int kKOff = kQOff + kChunks * kQChunk;
-  static constexpr int kVOff = kKOff + kStages * kKVTile;
-  static constexpr int kPOff = kVOff + kStages * kKVTile;    // two P buffers of 128 rows x 64 keys
-  static constexpr int kXOff = kPOff + 2 * 128 * 128;    // exchange area: 6 x 128 floats
+  static constexpr int kRingOff = kQOff + kChunks * kTile;
+  static constexpr int kXOff = kRingOff + kSlots * kKV;  // exchange area: 6 x 128 floats
   static constexpr int kBarOff = kXOff + 6 * 128 * 4;
   static constexpr int kBytes = kBarOff + 256 + 1024;    // + alignment slack
-  static_assert(2 * kHsTile <= 2 * kStages * kKVTile, "linear state tiles must fit in the K/V ring");
+  static_assert(2 * kHsTile <= kSlots * kKV, "linear state tiles must fit in the K/V ring");
 };
 
 struct AttnKParams {
@@ -101,6 +102,15 @@ __device__ __forceinline__ void tmem_ld1(uint32_t taddr, uint32_t& r) {
   asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(r) : "r"(taddr));
 }
 
+// D[tmem] (+)= A[tmem] * B[smem]^T (A: row m in lane m, two bf16 of K per column).
+__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile("{\n\t.reg .pred p;\n\t"
+               "setp.ne.b32 p, %4, 0;\n\t"
+               "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
+               :: "r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate) : "memory");
+}
+
 // MMA with output lanes masked off (bit i of the 128-bit mask disables TMEM lane i).
 __device__ __forceinline__ void mma_bf16_ss_masked(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                                    uint32_t accumulate, const uint32_t (&mask)[4]) {
@@ -109,6 +119,28 @@ __device__ __forceinline__ void mma_bf16_ss_masked(uint32_t d_tmem, uint64_t a_d
                "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}"
                :: "r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate),
                   "r"(mask[0]), "r"(mask[1]), "r"(mask[2]), "r"(mask[3]) : "memory");
+}
+
+// List entry: key block in bits [0,16), valid keys in bits [16,23), bit 30/31: half 0/1 attends.
+struct Entry {
+  int kb, nvalid;
+  uint32_t flags;
+};
+
+template <bool TILE>
+__device__ __forceinline__ Entry read_entry(const uint32_t* list, int idx, const SeqShape& s) {
+  Entry e;
+  if (list) {
+    const uint32_t w = list[idx];
+    e.kb = (int)(w & 0xFFFFu);
+    e.nvalid = (int)((w >> 16) & 0x7Fu);
+    e.flags = w >> 30;
+  } else {
+    e.kb = idx;
+    e.nvalid = TILE ? 64 : block_valid_count(s, idx);
+    e.flags = 3u;
+  }
+  return e;
 }
 
 template <int D, bool TILE, bool GATED, bool LINEAR>
@@ -121,30 +153,26 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem + L::kQOff;
-  uint8_t* sK = smem + L::kKOff;
-  uint8_t* sV = smem + L::kVOff;
-  uint8_t* sP = smem + L::kPOff;
-  float* xch = reinterpret_cast<float*>(smem + L::kXOff);   // [6][128]: m0 m1 l0 l1 f0 f1
+  uint8_t* sRing = smem + L::kRingOff;
+  float* xch = reinterpret_cast<float*>(smem + L::kXOff);   // [6][128]: m0 m1 l0 l1 far-l spare
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
   uint64_t* q_full = bars + 0;
-  uint64_t* k_full = bars + 1;
-  uint64_t* v_full = bars + 1 + kStages;
-  uint64_t* kv_empty = bars + 1 + 2 * kStages;
-  uint64_t* s_full = bars + 1 + 3 * kStages;     // [2]  per S buffer
-  uint64_t* p_full = s_full + 2;                 // [4]  [warpgroup * 2 + P buffer]
-  uint64_t* o_bar = p_full + 4;                  // [4]  [warpgroup * 2 + P buffer]
-  uint64_t* loop_done = o_bar + 4;
+  uint64_t* slot_full = bars + 1;                // [kSlots] TMA landed in a ring slot
+  uint64_t* s_full = slot_full + kSlots;         // [2] per S buffer
+  uint64_t* p_full = s_full + 2;                 // [2] per S buffer, 256 arrivals
+  uint64_t* pv_done = p_full + 2;                // [4] per step mod 4 (phases cannot alias)
+  uint64_t* loop_done = pv_done + 4;
   uint64_t* hs_full = loop_done + 1;
   uint64_t* phiq_ready = hs_full + 1;
   uint64_t* lin_done = phiq_ready + 1;
-  uint64_t* far_x = lin_done + 1;               // far-field max exchange between the warpgroups
-  uint64_t* drain = far_x + 1;
+  uint64_t* drain = lin_done + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int pair = blockIdx.x, bh = blockIdx.y;
   constexpr uint32_t kTmemCols = 512;
+  const SeqShape seq{p.n_pad, p.seg_len, p.seg_stride, p.n_kb};
 
   const uint32_t* list = nullptr;
   int n_local = p.n_kb;
@@ -153,20 +181,27 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
     list = p.list + off * p.list_cap;
     n_local = p.list_cnt[off];
   }
-  const int total = n_local + (GATED ? 1 : 0);
+  const int local_steps = (n_local + 1) >> 1;
+  const int n_steps = local_steps + (GATED ? 1 : 0);   // the far block is a step of its own
   const bool second_exists = 2 * pair + 1 < p.n_qb;
+  // blocks in step j: 2, except an odd tail (1) and the far step (1, handled by warpgroup 0)
+  auto step_blocks = [&](int j) -> int {
+    if (GATED && j == local_steps) return 1;
+    return (2 * j + 1 < n_local) ? 2 : 1;
+  };
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    for (int s = 0; s < kStages; ++s) { mbar_init(&k_full[s], 1); mbar_init(&v_full[s], 1); mbar_init(&kv_empty[s], 1); }
-    mbar_init(&s_full[0], 1);
-    mbar_init(&s_full[1], 1);
-    for (int i = 0; i < 4; ++i) { mbar_init(&p_full[i], 128); mbar_init(&o_bar[i], 1); }
+    for (int s = 0; s < kSlots; ++s) mbar_init(&slot_full[s], 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&s_full[b], 1);
+      mbar_init(&p_full[b], 256);
+    }
+    for (int b = 0; b < 4; ++b) mbar_init(&pv_done[b], 1);
     mbar_init(loop_done, 1);
     mbar_init(hs_full, 1);
     mbar_init(phiq_ready, 256);
     mbar_init(lin_done, 1);
-    mbar_init(far_x, 256);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -179,118 +214,123 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
 
   if (warp == 8) {
     // ---------------------------------------------------------------- producer
-    if (lane == 0 && total > 0) {
+    if (lane == 0 && n_steps > 0) {
       tma_prefetch_desc(&tmQ); tma_prefetch_desc(&tmK); tma_prefetch_desc(&tmV);
-      mbar_arrive_expect_tx(q_full, L::kChunks * L::kQChunk);
+      mbar_arrive_expect_tx(q_full, L::kChunks * L::kTile);
       if (TILE) {
         for (int half = 0; half < 2; ++half) {
           int tf, th, tw;
           tile_coords(2 * pair + half, p.TF, p.TW, tf, th, tw);
           for (int c = 0; c < L::kChunks; ++c)
-            tma_load_5d(sQ + c * L::kQChunk + half * L::kKVChunk, &tmQ, q_full, c * 64, tw * 4, th * 4, tf * 4, bh);
+            tma_load_5d(sQ + c * L::kTile + half * L::kHalf, &tmQ, q_full, c * 64, tw * 4, th * 4, tf * 4, bh);
         }
       } else {
-        for (int c = 0; c < L::kChunks; ++c) tma_load_3d(sQ + c * L::kQChunk, &tmQ, q_full, c * 64, pair * 128, bh);
+        for (int c = 0; c < L::kChunks; ++c) tma_load_3d(sQ + c * L::kTile, &tmQ, q_full, c * 64, pair * 128, bh);
       }
-      int j = 0;
-      for (; j < total; ++j) {
-        const int s = j % kStages;
-        if (j >= kStages && !mbar_wait(&kv_empty[s], ((j / kStages) - 1) & 1, abort_flag, p.status)) break;
-        const bool far = GATED && j == n_local;
-        const int kb = far ? 0 : (list ? (int)(list[j] & 0x3FFFFFFFu) : j);
-        uint8_t* dK = sK + s * L::kKVTile;
-        uint8_t* dV = sV + s * L::kKVTile;
-        mbar_arrive_expect_tx(&k_full[s], L::kKVTile);
-        mbar_arrive_expect_tx(&v_full[s], L::kKVTile);
-        if (far) {
-          for (int c = 0; c < L::kChunks; ++c) tma_load_3d(dK + c * L::kKVChunk, &tmX1, &k_full[s], c * 64, 0, bh);
-          for (int c = 0; c < L::kChunks; ++c) tma_load_3d(dV + c * L::kKVChunk, &tmX2, &v_full[s], c * 64, 0, bh);
-        } else if (TILE) {
-          int tf, th, tw;
-          tile_coords(kb, p.TF, p.TW, tf, th, tw);
-          for (int c = 0; c < L::kChunks; ++c) tma_load_5d(dK + c * L::kKVChunk, &tmK, &k_full[s], c * 64, tw * 4, th * 4, tf * 4, bh);
-          for (int c = 0; c < L::kChunks; ++c) tma_load_5d(dV + c * L::kKVChunk, &tmV, &v_full[s], c * 64, tw * 4, th * 4, tf * 4, bh);
-        } else {
-          for (int c = 0; c < L::kChunks; ++c) tma_load_3d(dK + c * L::kKVChunk, &tmK, &k_full[s], c * 64, kb * 64, bh);
-          for (int c = 0; c < L::kChunks; ++c) tma_load_3d(dV + c * L::kKVChunk, &tmV, &v_full[s], c * 64, kb * 64, bh);
+      // item i: K (even i) or V (odd i) of step i/2, in slot i % kSlots; the slot's
+      // previous item (i - kSlots) is free once the P.V of its step has completed
+      int i = 0;
+      for (; i < 2 * n_steps; ++i) {
+        const int j = i >> 1, slot = i % kSlots;
+        const bool is_v = i & 1;
+        if (i >= kSlots) {
+          const int q = (i - kSlots) >> 1;
+          if (!mbar_wait(&pv_done[q & 3], (q >> 2) & 1, abort_flag, p.status)) break;
+        }
+        const int nb = step_blocks(j);
+        const bool far = GATED && j == local_steps;
+        mbar_arrive_expect_tx(&slot_full[slot], nb * L::kChunks * L::kHalf);
+        for (int b = 0; b < nb; ++b) {
+          uint8_t* dst = sRing + slot * L::kKV + b * L::kHalf;
+          if (far) {
+            for (int c = 0; c < L::kChunks; ++c)
+              tma_load_3d(dst + c * L::kTile, is_v ? &tmX2 : &tmX1, &slot_full[slot], c * 64, 0, bh);
+          } else {
+            const int kb = list ? (int)(list[2 * j + b] & 0xFFFFu) : 2 * j + b;
+            const CUtensorMap* tm = is_v ? &tmV : &tmK;
+            if (TILE) {
+              int tf, th, tw;
+              tile_coords(kb, p.TF, p.TW, tf, th, tw);
+              for (int c = 0; c < L::kChunks; ++c)
+                tma_load_5d(dst + c * L::kTile, tm, &slot_full[slot], c * 64, tw * 4, th * 4, tf * 4, bh);
+            } else {
+              for (int c = 0; c < L::kChunks; ++c) tma_load_3d(dst + c * L::kTile, tm, &slot_full[slot], c * 64, kb * 64, bh);
+            }
+          }
         }
       }
-      if (LINEAR && j == total && mbar_wait(loop_done, 0, abort_flag, p.status)) {
+      const int j = i >> 1;
+      if (LINEAR && j == n_steps && mbar_wait(loop_done, 0, abort_flag, p.status)) {
         // the K/V ring is free: bring in the [H'^T ; Z] rows of both query blocks
         const int nblk = second_exists ? 2 : 1;
         mbar_arrive_expect_tx(hs_full, nblk * L::kHsTile);
         for (int b = 0; b < nblk; ++b)
           for (int c = 0; c < L::kChunks; ++c)
-            tma_load_3d(sK + b * L::kHsTile + c * L::kHsChunk, &tmX1, hs_full, c * 64, 0,
-                        bh * p.n_qb + 2 * pair + b);
+            tma_load_3d(sRing + b * L::kHsTile + c * L::kHsChunk, &tmX1, hs_full, c * 64, 0, bh * p.n_qb + 2 * pair + b);
       }
       if (*abort_flag) {
-        for (int i = (j - kStages > 0 ? j - kStages : 0); i < j; ++i) {
-          const int s = i % kStages;
+        // let the loads already in flight land before the CTA's shared memory is released
+        for (int it = (i - kSlots > 0 ? i - kSlots : 0); it < i; ++it) {
           const long long t0 = clock64();
-          while (!mbar_try_wait(&k_full[s], (i / kStages) & 1) && clock64() - t0 < kWaitBudgetCycles) {}
-          while (!mbar_try_wait(&v_full[s], (i / kStages) & 1) && clock64() - t0 < kWaitBudgetCycles) {}
+          while (!mbar_try_wait(&slot_full[it % kSlots], (it / kSlots) & 1) && clock64() - t0 < kWaitBudgetCycles) {}
         }
       }
     }
   } else if (warp == 9) {
     // ---------------------------------------------------------------- MMA issuer
-    if (lane == 0 && total > 0) {
-      constexpr uint32_t idS = idesc_bf16(128, 64, false, false);
+    if (lane == 0 && n_steps > 0) {
+      constexpr uint32_t idS = idesc_bf16(128, 128, false, false);
       constexpr uint32_t idO = idesc_bf16(128, D, false, true);
-      const uint32_t q_addr = smem_u32(sQ), k_addr = smem_u32(sK), v_addr = smem_u32(sV), p_addr = smem_u32(sP);
-      auto issue_qk = [&](int stage, int sbuf) {
+      const uint32_t q_addr = smem_u32(sQ), ring_addr = smem_u32(sRing);
+      auto issue_qk = [&](int slot, int sbuf) {
         #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const int c = kk >> 2, sub = kk & 3;
-          uint64_t a = desc_kmajor(q_addr + c * L::kQChunk + sub * 32);
-          uint64_t b = desc_kmajor(k_addr + stage * L::kKVTile + c * L::kKVChunk + sub * 32);
-          mma_bf16_ss(tmem + kColS + sbuf * 64, a, b, idS, kk > 0 ? 1u : 0u);
+          const uint64_t a = desc_kmajor(q_addr + c * L::kTile + sub * 32);
+          const uint64_t b = desc_kmajor(ring_addr + slot * L::kKV + c * L::kTile + sub * 32);
+          mma_bf16_ss(tmem + kColS + sbuf * 128, a, b, idS, kk > 0 ? 1u : 0u);
         }
       };
-      auto issue_pv = [&](int stage, int pbuf, uint32_t col, int kk0, int kk1, bool acc) {
-        for (int kk = kk0; kk < kk1; ++kk) {
-          uint64_t a = desc_kmajor(p_addr + pbuf * 16384 + kk * 32);
-          uint64_t b = desc_mnmajor(v_addr + stage * L::kKVTile + kk * 2048, L::kKVChunk);
-          mma_bf16_ss(tmem + col, a, b, idO, (acc || kk > kk0) ? 1u : 0u);
+      // O_dst (+)= P[:, 64*blk .. +64] V_blk; P lives in TMEM over the step's S buffer
+      auto issue_pv = [&](int slot, int sbuf, int blk, uint32_t col, bool acc) {
+        #pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint32_t a = tmem + kColS + sbuf * 128 + blk * 64 + kk * 8;
+          const uint64_t b = desc_mnmajor(ring_addr + slot * L::kKV + blk * L::kHalf + kk * 2048, L::kTile);
+          mma_bf16_ts(tmem + col, a, b, idO, (acc || kk > 0) ? 1u : 0u);
         }
       };
-      bool ok = mbar_wait(q_full, 0, abort_flag, p.status) && mbar_wait(&k_full[0], 0, abort_flag, p.status);
+      bool ok = mbar_wait(q_full, 0, abort_flag, p.status) && mbar_wait(&slot_full[0], 0, abort_flag, p.status);
+      bool o1_started = false;
       if (ok) {
         tc_fence_after();
         issue_qk(0, 0);
         mma_commit(&s_full[0]);
-        for (int j = 0; j < total && ok; ++j) {
-          if (j + 1 < total) {
-            const int s1 = (j + 1) % kStages;
-            if (!mbar_wait(&k_full[s1], ((j + 1) / kStages) & 1, abort_flag, p.status)) { ok = false; break; }
+        for (int j = 0; j < n_steps && ok; ++j) {
+          const int b = j & 1;
+          if (j + 1 < n_steps) {
+            const int ik = 2 * (j + 1);
+            if (!mbar_wait(&slot_full[ik % kSlots], (ik / kSlots) & 1, abort_flag, p.status)) { ok = false; break; }
             tc_fence_after();
-            issue_qk(s1, (j + 1) & 1);
+            issue_qk(ik % kSlots, (j + 1) & 1);
             mma_commit(&s_full[(j + 1) & 1]);
           }
-          const int s = j % kStages;
-          if (!mbar_wait(&v_full[s], (j / kStages) & 1, abort_flag, p.status)) { ok = false; break; }
-          const bool far = GATED && j == n_local;
-          const int pb = j & 1;
-          const uint32_t ph = (j >> 1) & 1;
+          const int iv = 2 * j + 1;
+          if (!mbar_wait(&slot_full[iv % kSlots], (iv / kSlots) & 1, abort_flag, p.status) ||
+              !mbar_wait(&p_full[b], (j >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
+          tc_fence_after();
+          const bool far = GATED && j == local_steps;
           if (far) {
-            if (!mbar_wait(&p_full[pb], ph, abort_flag, p.status) ||
-                !mbar_wait(&p_full[2 + pb], ph, abort_flag, p.status)) { ok = false; break; }
-            tc_fence_after();
-            issue_pv(s, pb, kColOf, 0, 4, false);
-            mma_commit(&o_bar[pb]);
-            mma_commit(&o_bar[2 + pb]);
+            // the far-field output goes into the other S buffer (its step is done)
+            issue_pv(iv % kSlots, b, 0, kColS + (b ^ 1) * 128, false);
           } else {
-            if (!mbar_wait(&p_full[pb], ph, abort_flag, p.status)) { ok = false; break; }
-            tc_fence_after();
-            issue_pv(s, pb, kColO0, 0, 2, j > 0);
-            mma_commit(&o_bar[pb]);
-            if (!mbar_wait(&p_full[2 + pb], ph, abort_flag, p.status)) { ok = false; break; }
-            tc_fence_after();
-            issue_pv(s, pb, kColO1, 2, 4, j > 0);
-            mma_commit(&o_bar[2 + pb]);
+            issue_pv(iv % kSlots, b, 0, kColO0, j > 0);
+            if (step_blocks(j) == 2) {
+              issue_pv(iv % kSlots, b, 1, kColO1, o1_started);
+              o1_started = true;
+            }
           }
-          mma_commit(&kv_empty[s]);
+          mma_commit(&pv_done[j & 3]);
         }
         if (ok) mma_commit(loop_done);
         if (ok && LINEAR) {
@@ -303,17 +343,17 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
             #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
               const int c = kk >> 2, sub = kk & 3;
-              const uint64_t a = desc_kmajor(q_addr + c * L::kQChunk + sub * 32);
-              const uint64_t b = desc_kmajor(k_addr + c * L::kHsChunk + sub * 32);
-              mma_bf16_ss_masked(tmem + kColLin, a, b, idL, kk > 0 ? 1u : 0u, lo_only);
+              const uint64_t a = desc_kmajor(q_addr + c * L::kTile + sub * 32);
+              const uint64_t bd = desc_kmajor(ring_addr + c * L::kHsChunk + sub * 32);
+              mma_bf16_ss_masked(tmem + kColLin, a, bd, idL, kk > 0 ? 1u : 0u, lo_only);
             }
             if (second_exists) {
               #pragma unroll
               for (int kk = 0; kk < D / 16; ++kk) {
                 const int c = kk >> 2, sub = kk & 3;
-                const uint64_t a = desc_kmajor(q_addr + c * L::kQChunk + sub * 32);
-                const uint64_t b = desc_kmajor(k_addr + L::kHsTile + c * L::kHsChunk + sub * 32);
-                mma_bf16_ss_masked(tmem + kColLin, a, b, idL, kk > 0 ? 1u : 0u, hi_only);
+                const uint64_t a = desc_kmajor(q_addr + c * L::kTile + sub * 32);
+                const uint64_t bd = desc_kmajor(ring_addr + L::kHsTile + c * L::kHsChunk + sub * 32);
+                mma_bf16_ss_masked(tmem + kColLin, a, bd, idL, kk > 0 ? 1u : 0u, hi_only);
               }
             }
             mma_commit(lin_done);
@@ -328,82 +368,79 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
     }
   } else {
     // ---------------------------------------------------------------- softmax + epilogue
-    const int wg = warp >> 2;                  // 0: key columns 0-31, 1: columns 32-63
+    const int wg = warp >> 2;                  // 0: first block of a step, 1: second block
     const int r = threadIdx.x & 127;           // query row of the pair = TMEM lane
     const int half = r >> 6;
     const uint32_t lane_addr = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     const uint32_t my_o = wg ? kColO1 : kColO0;
     const float sl = p.scale_log2;
-    float m_run = -INFINITY, l_run = 0.f, m_far = -INFINITY, l_far = 0.f;
-    const SeqShape seq{p.n_pad, p.seg_len, p.seg_stride, p.n_kb};
-    bool ok = true;
-    for (int j = 0; j < total; ++j) {
-      const bool far = GATED && j == n_local;
-      const int sb = j & 1;
-      if (!__all_sync(0xFFFFFFFFu, mbar_wait(&s_full[sb], (j >> 1) & 1, abort_flag, p.status))) { ok = false; break; }
+    float m_run = -INFINITY, l_run = 0.f, l_far = 0.f;
+    bool ok = true, started = false;
+    for (int j = 0; j < n_steps; ++j) {
+      const int b = j & 1;
+      const bool far = GATED && j == local_steps;
+      const bool mine = wg == 0 || (!far && step_blocks(j) == 2);   // does this warpgroup own a block here
+      Entry e{0, 64, 3u};
+      if (mine && !far) e = read_entry<TILE>(list, 2 * j + wg, seq);
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait(&s_full[b], (j >> 1) & 1, abort_flag, p.status))) { ok = false; break; }
       tc_fence_after();
-      uint32_t sr[32];
-      tmem_ld32(lane_addr + kColS + sb * 64 + wg * 32, sr);
-      int nvalid = 64;
-      bool attend = true;
-      if (!far) {
-        const uint32_t e = list ? list[j] : ((uint32_t)j | 0xC0000000u);
-        attend = (e >> (30 + half)) & 1u;
-        if (!TILE) nvalid = block_valid_count(seq, (int)(e & 0x3FFFFFFFu));
+      if (!mine) {
+        tc_fence_before();
+        mbar_arrive(&p_full[b]);
+        continue;
       }
-      const int lo = wg * 32;
-      const bool none = !attend || nvalid <= lo;
-      const bool full = attend && nvalid >= lo + 32;
+      const uint32_t s_addr = lane_addr + kColS + b * 128 + wg * 64;
+      uint32_t sr[64];
+      tmem_ld32(s_addr, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+      tmem_ld32(s_addr + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+      const bool attend = (e.flags >> half) & 1u;
+      const int nvalid = attend ? e.nvalid : 0;
       tmem_wait_ld();
       float mx = -INFINITY;
-      if (full) {
-        float t[11];
+      if (nvalid == 64) {
+        float t[22];
         #pragma unroll
-        for (int i = 0; i < 10; ++i)
+        for (int i = 0; i < 21; ++i)
           t[i] = max3(__uint_as_float(sr[3 * i]), __uint_as_float(sr[3 * i + 1]), __uint_as_float(sr[3 * i + 2]));
-        t[10] = fmaxf(__uint_as_float(sr[30]), __uint_as_float(sr[31]));
-        const float u0 = max3(t[0], t[1], t[2]), u1 = max3(t[3], t[4], t[5]), u2 = max3(t[6], t[7], t[8]);
-        mx = max3(max3(u0, u1, u2), t[9], t[10]);
-      } else if (!none) {
+        t[21] = __uint_as_float(sr[63]);
+        float u[8];
         #pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          if (lo + c >= nvalid) sr[c] = __float_as_uint(-INFINITY);
+        for (int i = 0; i < 7; ++i) u[i] = max3(t[3 * i], t[3 * i + 1], t[3 * i + 2]);
+        u[7] = t[21];
+        mx = fmaxf(max3(u[0], u[1], u[2]), max3(max3(u[3], u[4], u[5]), u[6], u[7]));
+      } else if (nvalid > 0) {
+        #pragma unroll
+        for (int c = 0; c < 64; ++c) {
+          if (c >= nvalid) sr[c] = __float_as_uint(-INFINITY);
           mx = fmaxf(mx, __uint_as_float(sr[c]));
         }
       }
-      float m_new;
-      if (far) {
-        // both warpgroups share the far block's max so that its P is one consistent row
-        xch[(4 + wg) * 128 + r] = none ? -INFINITY : mx;
-        mbar_arrive(far_x);
-        if (!__all_sync(0xFFFFFFFFu, mbar_wait(far_x, 0, abort_flag, p.status))) { ok = false; break; }
-        const float other = xch[(5 - wg) * 128 + r];
-        m_new = fmaxf(none ? -INFINITY : mx, other) * sl;
-        m_far = m_new;
-      } else {
-        m_new = fmaxf(m_run, mx * sl);
-      }
-      float factor = 1.f;
+      // far step: a fresh softmax of its own; local steps: lazy rescale of the running state
+      float mu;
       bool need = false;
-      if (!far) {
+      float factor = 1.f;
+      if (far) {
+        mu = mx * sl;
+      } else {
+        const float m_new = fmaxf(m_run, mx * sl);
         need = m_new > m_run + 8.f;
         if (need) {
           factor = (m_run == -INFINITY) ? 0.f : ex2(m_run - m_new);
           l_run *= factor;
           m_run = m_new;
         }
+        mu = m_run;
       }
-      const float mcur = far ? m_far : m_run;
-      const float mu = (mcur == -INFINITY) ? 0.f : mcur;
-      uint32_t packed[16];
+      if (mu == -INFINITY) mu = 0.f;
+      uint32_t packed[32];
       float rowsum = 0.f;
-      if (none) {
+      if (nvalid == 0) {
         #pragma unroll
-        for (int c = 0; c < 16; ++c) packed[c] = 0u;
+        for (int c = 0; c < 32; ++c) packed[c] = 0u;
       } else {
         float acc0 = 0.f, acc1 = 0.f;
         #pragma unroll
-        for (int c = 0; c < 32; c += 2) {
+        for (int c = 0; c < 64; c += 2) {
           const float p0 = ex2(fmaf(__uint_as_float(sr[c]), sl, -mu));
           const float p1 = ex2(fmaf(__uint_as_float(sr[c + 1]), sl, -mu));
           acc0 += p0;
@@ -412,19 +449,11 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
         }
         rowsum = acc0 + acc1;
       }
-      if (far) l_far += rowsum; else l_run += rowsum;
-      // P buffer j&1 (my half) is free once P_{j-2} V_{j-2} has completed; my accumulator
-      // may be rescaled once P_{j-1} V_{j-1} has completed
-      const int pb = j & 1;
-      if (j >= 2) {
-        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&o_bar[wg * 2 + pb], ((j - 2) >> 1) & 1, abort_flag, p.status))) { ok = false; break; }
-      }
-      const bool rescale = !far && j > 0 && __any_sync(0xFFFFFFFFu, need);
-      if (rescale) {
-        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&o_bar[wg * 2 + (pb ^ 1)], ((j - 1) >> 1) & 1, abort_flag, p.status))) { ok = false; break; }
-      }
-      tc_fence_after();
-      if (rescale) {
+      if (far) l_far = rowsum; else l_run += rowsum;
+      // rescale my accumulator (once it holds data) after P_{j-1} V_{j-1} has completed
+      if (!far && started && __any_sync(0xFFFFFFFFu, need)) {
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&pv_done[(j - 1) & 3], ((j - 1) >> 2) & 1, abort_flag, p.status))) { ok = false; break; }
+        tc_fence_after();
         #pragma unroll 1
         for (int cc = 0; cc < D / 32; ++cc) {
           uint32_t o[32];
@@ -434,19 +463,15 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
           for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * factor);
           tmem_st32(lane_addr + my_o + cc * 32, o);
         }
-        tmem_wait_st();
       }
-      #pragma unroll
-      for (int c8 = 0; c8 < 4; ++c8) {
-        uint4 val = make_uint4(packed[4 * c8], packed[4 * c8 + 1], packed[4 * c8 + 2], packed[4 * c8 + 3]);
-        *reinterpret_cast<uint4*>(sP + pb * 16384 + sw128_offset(r, 4 * wg + c8)) = val;
-      }
-      fence_proxy_async_smem();
+      tmem_st32(s_addr, packed);          // P (bf16 pairs) over the first 32 columns of my S block
+      tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&p_full[wg * 2 + pb]);
+      mbar_arrive(&p_full[b]);
+      if (!far) started = true;
     }
-    if (ok && total > 0)
-      ok = __all_sync(0xFFFFFFFFu, mbar_wait(&o_bar[wg * 2 + ((total - 1) & 1)], ((total - 1) >> 1) & 1, abort_flag, p.status));
+    if (ok && n_steps > 0)
+      ok = __all_sync(0xFFFFFFFFu, mbar_wait(&pv_done[(n_steps - 1) & 3], ((n_steps - 1) >> 2) & 1, abort_flag, p.status));
     ok = __all_sync(0xFFFFFFFFu, ok);
     tc_fence_after();
 
@@ -468,13 +493,13 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
 
     bool lin_ok = false;
     if (LINEAR) {
-      // phi(Q) in place (the last QK MMA has completed); pad rows -> 0
+      // phi(Q) in place (every QK MMA has completed); pad rows -> 0
       if (ok) {
         constexpr int kGroups = D / 16;                  // 16-byte groups of my row handled by my warpgroup
         #pragma unroll
         for (int g = 0; g < kGroups; ++g) {
           const int gg = wg * kGroups + g;               // 0 .. D/8-1
-          uint4* ptr = reinterpret_cast<uint4*>(sQ + (gg >> 3) * L::kQChunk + sw128_offset(r, gg & 7));
+          uint4* ptr = reinterpret_cast<uint4*>(sQ + (gg >> 3) * L::kTile + sw128_offset(r, gg & 7));
           const uint4 u = *ptr;
           const uint32_t w[4] = {u.x, u.y, u.z, u.w};
           uint32_t o4[4];
@@ -490,10 +515,10 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
       tc_fence_after();
     }
 
-    // ---- merge the two halves
+    // ---- merge the two shares
     xch[wg * 128 + r] = m_run;
     xch[(2 + wg) * 128 + r] = l_run;
-    if (GATED) xch[(4 + wg) * 128 + r] = l_far;
+    if (GATED && wg == 0) xch[512 + r] = l_far;
     softmax_bar();
     const float m0 = xch[r], m1 = xch[128 + r], l0 = xch[256 + r], l1 = xch[384 + r];
     const float M = fmaxf(m0, m1);
@@ -503,9 +528,11 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
     const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
     const float c0 = a0 * inv, c1 = a1 * inv;
     float inv_far = 0.f;
+    uint32_t col_far = 0;
     if (GATED) {
-      const float lf = xch[512 + r] + xch[640 + r];
+      const float lf = xch[512 + r];
       inv_far = lf > 0.f ? 1.f / lf : 0.f;
+      col_far = kColS + ((local_steps & 1) ^ 1) * 128;
     }
     float inv_den = 0.f;
     if (LINEAR && lin_ok) {
@@ -515,25 +542,31 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
       const float den = __uint_as_float(dv);
       inv_den = den > 0.f ? 1.f / den : 0.f;
     }
-    const bool have_o = ok && n_local > 0;         // CTA-uniform
+    const bool have_o0 = ok && n_local > 0;        // CTA-uniform
+    const bool have_o1 = ok && n_local > 1;
     const size_t row_off = ((size_t)bh * p.n_pad + (row_exists ? tok : 0)) * D;
     #pragma unroll 1
     for (int cc = wg * (D / 64); cc < (wg + 1) * (D / 64); ++cc) {
       float v[32];
-      if (have_o) {
-        uint32_t o0[32], o1[32];
+      #pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] = 0.f;
+      if (have_o0) {
+        uint32_t o0[32];
         tmem_ld32(lane_addr + kColO0 + cc * 32, o0);
+        tmem_wait_ld();
+        #pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = c0 * __uint_as_float(o0[i]);
+      }
+      if (have_o1) {
+        uint32_t o1[32];
         tmem_ld32(lane_addr + kColO1 + cc * 32, o1);
         tmem_wait_ld();
         #pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] = c0 * __uint_as_float(o0[i]) + c1 * __uint_as_float(o1[i]);
-      } else {
-        #pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] = 0.f;
+        for (int i = 0; i < 32; ++i) v[i] += c1 * __uint_as_float(o1[i]);
       }
       if (GATED && ok) {
         uint32_t of[32];
-        tmem_ld32(lane_addr + kColOf + cc * 32, of);
+        tmem_ld32(lane_addr + col_far + cc * 32, of);
         tmem_wait_ld();
         #pragma unroll
         for (int i = 0; i < 32; ++i) v[i] = p.gate * v[i] + (1.f - p.gate) * (__uint_as_float(of[i]) * inv_far);

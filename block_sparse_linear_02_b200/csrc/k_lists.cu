@@ -3,7 +3,7 @@
 // The attention kernel handles query blocks in pairs (128 rows = one tcgen05
 // M tile).  pair_lists_kernel turns per-query-block key-block sets into one
 // ascending list per pair: each entry is a key block of the union of the two
-// sets, tagged with which half attends it.  Sets come from
+// sets with its number of valid keys, tagged with which half attends it.  Sets come from
 //   - explicit per-query-block lists (SLA's critical lists or a caller's),
 //   - LVSA frame sets A(t) expanded to the key blocks of each frame (rainbus
 //     page, step 6: all tokens of the attended frames),
@@ -93,8 +93,11 @@ pair_lists_kernel(const ListArgs a) {
       while (u) {
         const int bit = __ffs(u) - 1;
         u &= u - 1u;
-        if (pos < a.cap)
-          out[pos] = (uint32_t)(w * 32 + bit) | (((b0 >> bit) & 1u) << 30) | (((b1 >> bit) & 1u) << 31);
+        if (pos < a.cap) {
+          const int j = w * 32 + bit;
+          const uint32_t nv = a.mode == kListTile3d ? 64u : (uint32_t)block_valid_count(a.s, j);
+          out[pos] = (uint32_t)j | (nv << 16) | (((b0 >> bit) & 1u) << 30) | (((b1 >> bit) & 1u) << 31);
+        }
         ++pos;
       }
       base += __shfl_sync(0xFFFFFFFFu, incl, 31);

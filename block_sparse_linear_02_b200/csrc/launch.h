@@ -45,8 +45,9 @@ cudaError_t launch_mask_to_m01(const int8_t* mask, __nv_bfloat16* m01, int BH, i
                                cudaStream_t st);
 
 // ------------------------------------------------------------ block lists (k_lists.cu)
-// Entries of a pair list: key block index in bits [0,30), bit 30 = the first query
-// block of the pair attends it, bit 31 = the second does.
+// Entries of a pair list: key block index in bits [0,16), its number of valid keys
+// in bits [16,23), bit 30 = the first query block of the pair attends it, bit 31 =
+// the second does.
 enum ListMode { kListExplicit = 0, kListLvsa = 1, kListTile3d = 2 };
 
 struct ListArgs {
@@ -62,6 +63,7 @@ struct ListArgs {
   int set_cap, blocks_per_frame;
   // tile3d: tile grid (TF, TH, TW), tile id = (th*TW + tw)*TF + tf
   int TF, TH, TW, radius;
+  SeqShape s;              // token layout (valid-key counts of linear blocks)
   uint32_t* list;          // [heads][n_pairs][cap]
   int32_t* list_cnt;       // [heads][n_pairs]
   int* status;

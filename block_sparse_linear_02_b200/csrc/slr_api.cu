@@ -476,7 +476,7 @@ slr_status slr_block_sparse_attn(const void* q, const void* k, const void* v, co
     la.mode = kListExplicit;
     la.n_qb = sh.nb; la.n_kb = sh.nb; la.n_pairs = sh.npairs; la.cap = cap;
     la.kv_idx = kv_idx; la.kv_cnt = kv_cnt; la.kv_max = kv_max;
-    la.list = list; la.list_cnt = list_cnt; la.status = status;
+    la.s = sh.s; la.list = list; la.list_cnt = list_cnt; la.status = status;
     SLR_LAUNCH(kKLists, s, launch_pair_lists(la, sh.BH, s));
     a.list = list; a.list_cnt = list_cnt; a.list_cap = cap; a.list_per_head = 1;
   }
@@ -545,7 +545,7 @@ slr_status slr_sparse_linear_attn(const void* q, const void* k, const void* v, c
   la.mode = kListExplicit;
   la.n_qb = sh.nb; la.n_kb = sh.nb; la.n_pairs = sh.npairs; la.cap = w.cap;
   la.kv_idx = w.crit_idx; la.kv_cnt = w.crit_cnt; la.kv_max = kc;
-  la.list = w.list; la.list_cnt = w.list_cnt; la.status = w.status;
+  la.s = sh.s; la.list = w.list; la.list_cnt = w.list_cnt; la.status = w.status;
   SLR_LAUNCH(kKLists, s, launch_pair_lists(la, sh.BH, s));
   if (marginal) {
     SLR_LAUNCH(kKKeyStates, s, launch_key_states(k, v, w_proj, w.mar.h, sh.BH, sh.d, sh.s, w.status, s));
@@ -573,7 +573,7 @@ slr_status slr_frame_mask_attn(const void* q, const void* k, const void* v, cons
   ListArgs la;
   memset(&la, 0, sizeof(la));
   la.n_qb = sh.nb; la.n_kb = sh.nb; la.n_pairs = sh.npairs; la.cap = w.cap;
-  la.list = w.list; la.list_cnt = w.list_cnt; la.status = w.status;
+  la.s = sh.s; la.list = w.list; la.list_cnt = w.list_cnt; la.status = w.status;
   AttnArgs a = attn_base(sh, q, k, v, out, w.status);
   if (m->kind == SLR_MASK_LVSA) {
     SLR_LAUNCH(kKLvsaSets, s, launch_lvsa_sets(m->T, m->C, m->W, m->step, w.sets, w.set_cnt, w.set_cap, s));

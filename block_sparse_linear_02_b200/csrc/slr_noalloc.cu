@@ -94,7 +94,7 @@ extern "C" slr_status slr_block_sparse_attn_noalloc(const void* q, const void* k
     la.mode = kListExplicit;
     la.n_qb = nb; la.n_kb = nb; la.n_pairs = npairs; la.cap = cap;
     la.kv_idx = kv_idx; la.kv_cnt = kv_cnt; la.kv_max = kv_max;
-    la.list = list; la.list_cnt = list_cnt; la.status = status;
+    la.s = a.s; la.list = list; la.list_cnt = list_cnt; la.status = status;
     if (launch_pair_lists(la, (int)bh, s) != cudaSuccess) return SLR_ERR_CUDA;
     a.list = list; a.list_cnt = list_cnt; a.list_cap = cap; a.list_per_head = 1;
   }
