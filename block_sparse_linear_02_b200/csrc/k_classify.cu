@@ -8,7 +8,7 @@
 // first.  Both the logits and the selection are fp64 so that the labels agree
 // with an fp64 evaluation of the same definition.
 //
-// block_logits_kernel: 64x64 output tiles of qbar kbar^T / sqrt(d) (fp64 FMA).
+// block_logits_kernel: 64x64 output tiles of qbar kbar^T on the fp64 tensor cores.
 // classify_rows_kernel: one warp per row; two MSB-first radix selections over
 //   order-preserving 64-bit keys (8-bit digits, warp-aggregated histogram
 //   counts, stopping once the remaining candidates are exactly the ones
@@ -27,50 +27,63 @@
 namespace slr {
 namespace {
 
-// One CTA of 64 threads computes a 64x64 tile; each thread an 8x8 sub-tile, so
-// every pair of shared-memory loads feeds four fp64 FMAs.
-__global__ void __launch_bounds__(64)
+// dots[bh][i][j] = qbar_i . kbar_j in fp64 on the fp64 tensor cores
+// (mma.m8n8k4.f64): one CTA = 4 warps computes a 64x64 tile, each warp a 32x32
+// quarter as 4x4 fragments of 8x8.  The ranking of a row does not depend on the
+// positive scale 1/sqrt(d), so the kernel stores the plain dot products.
+__device__ __forceinline__ void dmma_8x8x4(double (&d)[2], double a, double b) {
+  asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0, %1}, {%2}, {%3}, {%0, %1};"
+               : "+d"(d[0]), "+d"(d[1]) : "d"(a), "d"(b));
+}
+
+__global__ void __launch_bounds__(128)
 block_logits_kernel(const double* __restrict__ qbar, const double* __restrict__ kbar,
-                    double* __restrict__ logits, int nb, int d, double sqrt_d) {
-  __shared__ double As[16][64];
-  __shared__ double Bs[16][64];
+                    double* __restrict__ dots, int nb, int d) {
+  __shared__ double As[64][36];
+  __shared__ double Bs[64][36];
   const int bh = blockIdx.z;
   const int i0 = blockIdx.y * 64, j0 = blockIdx.x * 64;
   const double* A = qbar + (size_t)bh * nb * d;
   const double* B = kbar + (size_t)bh * nb * d;
-  const int tx = threadIdx.x % 8, ty = threadIdx.x / 8;
-  double acc[8][8];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int wy = warp >> 1, wx = warp & 1;
+  double acc[4][4][2];
   #pragma unroll
-  for (int a = 0; a < 8; ++a)
+  for (int a = 0; a < 4; ++a)
     #pragma unroll
-    for (int b = 0; b < 8; ++b) acc[a][b] = 0.0;
-  for (int c0 = 0; c0 < d; c0 += 16) {
-    for (int e = threadIdx.x; e < 64 * 16; e += 64) {
-      const int row = e / 16, col = e % 16;
-      As[col][row] = (i0 + row < nb) ? A[(size_t)(i0 + row) * d + c0 + col] : 0.0;
-      Bs[col][row] = (j0 + row < nb) ? B[(size_t)(j0 + row) * d + c0 + col] : 0.0;
+    for (int b = 0; b < 4; ++b) acc[a][b][0] = acc[a][b][1] = 0.0;
+  for (int c0 = 0; c0 < d; c0 += 32) {
+    for (int e = threadIdx.x; e < 64 * 32; e += 128) {
+      const int row = e >> 5, col = e & 31;
+      As[row][col] = (i0 + row < nb) ? A[(size_t)(i0 + row) * d + c0 + col] : 0.0;
+      Bs[row][col] = (j0 + row < nb) ? B[(size_t)(j0 + row) * d + c0 + col] : 0.0;
     }
     __syncthreads();
     #pragma unroll
-    for (int c = 0; c < 16; ++c) {
-      double a[8], b[8];
+    for (int kk = 0; kk < 32; kk += 4) {
+      double af[4], bf[4];
       #pragma unroll
-      for (int u = 0; u < 8; ++u) { a[u] = As[c][ty * 8 + u]; b[u] = Bs[c][tx * 8 + u]; }
+      for (int t = 0; t < 4; ++t) {
+        af[t] = As[wy * 32 + t * 8 + (lane >> 2)][kk + (lane & 3)];
+        bf[t] = Bs[wx * 32 + t * 8 + (lane >> 2)][kk + (lane & 3)];
+      }
       #pragma unroll
-      for (int u = 0; u < 8; ++u)
+      for (int mt = 0; mt < 4; ++mt)
         #pragma unroll
-        for (int w = 0; w < 8; ++w) acc[u][w] = fma(a[u], b[w], acc[u][w]);
+        for (int nt = 0; nt < 4; ++nt) dmma_8x8x4(acc[mt][nt], af[mt], bf[nt]);
     }
     __syncthreads();
   }
   #pragma unroll
-  for (int u = 0; u < 8; ++u) {
-    const int i = i0 + ty * 8 + u;
+  for (int mt = 0; mt < 4; ++mt) {
+    const int i = i0 + wy * 32 + mt * 8 + (lane >> 2);
     if (i >= nb) continue;
     #pragma unroll
-    for (int w = 0; w < 8; ++w) {
-      const int j = j0 + tx * 8 + w;
-      if (j < nb) logits[((size_t)bh * nb + i) * nb + j] = acc[u][w] / sqrt_d;
+    for (int nt = 0; nt < 4; ++nt) {
+      const int j = j0 + wx * 32 + nt * 8 + 2 * (lane & 3);
+      double* dst = dots + ((size_t)bh * nb + i) * nb + j;
+      if (j < nb) dst[0] = acc[mt][nt][0];
+      if (j + 1 < nb) dst[1] = acc[mt][nt][1];
     }
   }
 }
@@ -158,7 +171,7 @@ constexpr int kRowsPerCta = 4;
 __global__ void __launch_bounds__(128)
 classify_rows_kernel(const double* __restrict__ logits, int rows, int nb, int kc, int kn,
                      int8_t* __restrict__ mask, int32_t* __restrict__ crit_idx, int32_t* __restrict__ crit_cnt,
-                     __nv_bfloat16* __restrict__ m01, int ld_m01, float* __restrict__ scores) {
+                     __nv_bfloat16* __restrict__ m01, int ld_m01, float* __restrict__ scores, double sqrt_d) {
   extern __shared__ uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   uint64_t* keys = reinterpret_cast<uint64_t*>(smem) + (size_t)warp * nb;
@@ -176,7 +189,7 @@ classify_rows_kernel(const double* __restrict__ logits, int rows, int nb, int kc
   for (int o = 16; o > 0; o >>= 1) mx = fmax(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
   double sum = 0.0;
   if (scores) {
-    for (int j = lane; j < nb; j += 32) sum += exp(lg[j] - mx);
+    for (int j = lane; j < nb; j += 32) sum += exp(lg[j] / sqrt_d - mx / sqrt_d);
     #pragma unroll
     for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
   }
@@ -207,7 +220,7 @@ classify_rows_kernel(const double* __restrict__ logits, int rows, int nb, int kc
       const int8_t m = crit ? 1 : (negl ? -1 : 0);
       mask[(size_t)row * nb + j] = m;
       if (m01) m01[(size_t)row * ld_m01 + j] = __float2bfloat16_rn(m == 0 ? 1.f : 0.f);
-      if (scores) scores[(size_t)row * nb + j] = (float)(exp(lg[j] - mx) / sum);
+      if (scores) scores[(size_t)row * nb + j] = (float)(exp(lg[j] / sqrt_d - mx / sqrt_d) / sum);
     }
     const unsigned bcrit = __ballot_sync(0xFFFFFFFFu, crit);
     if (crit) crit_idx[(size_t)row * kc + written + __popc(bcrit & lt_mask)] = j;
@@ -234,11 +247,11 @@ __global__ void mask_to_m01_kernel(const int8_t* __restrict__ mask, __nv_bfloat1
 cudaError_t launch_block_logits(const double* qbar, const double* kbar, double* logits,
                                 int BH, int nb, int d, cudaStream_t st) {
   dim3 grid((nb + 63) / 64, (nb + 63) / 64, BH);
-  block_logits_kernel<<<grid, 64, 0, st>>>(qbar, kbar, logits, nb, d, sqrt((double)d));
+  block_logits_kernel<<<grid, 128, 0, st>>>(qbar, kbar, logits, nb, d);
   return cudaGetLastError();
 }
 
-cudaError_t launch_classify_rows(const double* logits, int BH, int nb, int kc, int kn,
+cudaError_t launch_classify_rows(const double* logits, int BH, int nb, int d, int kc, int kn,
                                  int8_t* mask, int32_t* crit_idx, int32_t* crit_cnt,
                                  __nv_bfloat16* m01, int ld_m01, float* scores, cudaStream_t st) {
   const int rows = BH * nb;
@@ -246,7 +259,7 @@ cudaError_t launch_classify_rows(const double* logits, int BH, int nb, int kc, i
   cudaError_t e = cudaFuncSetAttribute(classify_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   classify_rows_kernel<<<(rows + kRowsPerCta - 1) / kRowsPerCta, 128, smem, st>>>(
-      logits, rows, nb, kc, kn, mask, crit_idx, crit_cnt, m01, ld_m01, scores);
+      logits, rows, nb, kc, kn, mask, crit_idx, crit_cnt, m01, ld_m01, scores, sqrt((double)d));
   return cudaGetLastError();
 }
 

@@ -7,16 +7,17 @@
 // Because linear attention is a normalised weighted sum of value rows,
 // (sum w v / sum w) W = sum w (v W) / sum w, so W_proj is folded into V here.
 //
-//  key_states_kernel    per key block j: (V_j W)^T by one MMA (M=128 channels,
+//  key_states_kernel    persistent over key blocks; per block j: (V_j W)^T by one MMA (M=128 channels,
 //                       N=64 tokens, K=d), then h_j'^T = (V_j W)^T phi(K_j)
 //                       (M=128, N=d, K=64 tokens; phi applied in place in shared
 //                       memory) and z_j = sum_t phi(K_j,t); written as bf16 rows
 //                       [h_j'^T ; z_j] of (d+1)*d elements.  Without W the first
 //                       MMA is skipped and V_j^T is read MN-major from the tile.
-//  reduce_states_kernel per head: Hs = M01 . h, a plain tensor-core GEMM with
-//                       the 0/1 marginal indicator M01 [Nqb x Nkb] (K-major) and
-//                       h [Nkb x (d+1)d] (MN-major), fp32 accumulation in TMEM,
-//                       bf16 out.  Row i of Hs is [H_i'^T ; Z_i].
+//  reduce_states_kernel per head: Hs = M01 . h, a persistent tensor-core GEMM
+//                       with the 0/1 marginal indicator M01 [Nqb x Nkb]
+//                       (K-major) and h [Nkb x (d+1)d] (MN-major), fp32
+//                       accumulation in two TMEM buffers, bf16 out.  Row i of
+//                       Hs is [H_i'^T ; Z_i].
 //  linear_apply_kernel  per pair of query blocks: phi(Q) times the rows
 //                       [H_i'^T ; Z_i] (M=128 tokens, N=d+16), whose column d is
 //                       the denominator phi(q_t).Z_i; fp32 [token][channel] out.
@@ -42,78 +43,115 @@ __device__ __forceinline__ bool cta_wait(uint64_t* bar, uint32_t parity, volatil
 }
 
 // ------------------------------------------------------------------ key states
-// Shared-memory plan (bytes): K/phi(K) 16K | V 16K | W 32K | V'^T 16K | z partials 8K | barriers.
-constexpr int kKsK = 0, kKsV = 16384, kKsW = 32768, kKsVp = 65536, kKsZ = 81920, kKsBar = 81920 + 8192;
-constexpr int kKsSmemRequest = 100 * 1024;   // at most 2 CTAs (2 x 256 TMEM columns) per SM
+// Persistent: each CTA walks key blocks b = blockIdx.x, blockIdx.x + gridDim.x, ...
+// with a 2-stage TMA ring (the next block's K/V load overlaps this block's work)
+// and W_proj loaded once.  Shared memory (bytes): W 32K | 2 x (K 16K, V 16K) | z 4K.
+// (V W)^T is written back over the V stage it was computed from.
+constexpr int kKsW = 0, kKsRing = 32768, kKsStage = 32768, kKsZ = kKsRing + 2 * kKsStage;
+constexpr int kKsBar = kKsZ + 4096;
+constexpr int kKsSmem = kKsBar + 128 + 1024;
 
 template <int D, bool PROJ>
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(128, 2)
 key_states_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-                  const __grid_constant__ CUtensorMap tmW, __nv_bfloat16* __restrict__ h, SeqShape s, int* status) {
+                  const __grid_constant__ CUtensorMap tmW, __nv_bfloat16* __restrict__ h, SeqShape s, int BH,
+                  int* status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
-  uint8_t* sK = smem + kKsK;               // phi(K_j) after the transform, 64 rows (t) x D
-  uint8_t* sV = smem + kKsV;               // V_j, 64 rows (t) x D; chunk 1 zero when D = 64
   uint8_t* sW = smem + kKsW;               // W_proj MN-major: rows c_in, 64 c_out per chunk (chunk stride D*128)
-  uint8_t* sVp = smem + kKsVp;             // (V_j W)^T, K-major: 128 rows (c_out) x 64 t
   float* zred = reinterpret_cast<float*>(smem + kKsZ);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kKsBar);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 4);
+  uint64_t* load = bars;                   // [2]
+  uint64_t* w_bar = bars + 2;
+  uint64_t* mma0 = bars + 3;
+  uint64_t* mma1 = bars + 4;
+  uint64_t* drain = bars + 5;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 6);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  const int blk = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x, warp = tid >> 5;
+  const int tid = threadIdx.x, warp = tid >> 5;
   constexpr uint32_t kColP = 0;            // (V W)^T: 64 columns
   constexpr uint32_t kColH = 64;           // h^T: D columns
+  constexpr int kChunkB = 8192;            // one 64-row x 128-byte chunk
+  const int total = BH * s.n_blocks;
+  auto sK = [&](int st) { return smem + kKsRing + st * kKsStage; };
+  auto sV = [&](int st) { return smem + kKsRing + st * kKsStage + 16384; };
 
   if (tid == 0) {
-    for (int i = 0; i < 4; ++i) mbar_init(&bars[i], 1);
+    mbar_init(&load[0], 1);
+    mbar_init(&load[1], 1);
+    mbar_init(w_bar, 1);
+    mbar_init(mma0, 1);
+    mbar_init(mma1, 1);
+    mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
   if (D == 64) {
-    // upper half of the M = 128 operand must be zero
-    uint4* z = reinterpret_cast<uint4*>(PROJ ? sW + D * 128 : sV + 8192);
-    for (int i = tid; i < 8192 / 16; i += 128) z[i] = make_uint4(0, 0, 0, 0);
+    // upper half of the M = 128 A operand must be zero (W chunk 1, or V's second 8 KB)
+    for (int i = tid; i < 8192 / 16; i += 128) {
+      if (PROJ) reinterpret_cast<uint4*>(sW + D * 128)[i] = make_uint4(0, 0, 0, 0);
+      reinterpret_cast<uint4*>(sV(0) + 8192)[i] = make_uint4(0, 0, 0, 0);
+      reinterpret_cast<uint4*>(sV(1) + 8192)[i] = make_uint4(0, 0, 0, 0);
+    }
   }
   if (warp == 0) { tmem_alloc(tmem_slot, 256); tmem_relinquish(); }
+  fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (tid == 0) {
-    mbar_arrive_expect_tx(&bars[0], 2 * (D / 64) * 8192 + (PROJ ? (D / 64) * D * 128 : 0));
+  auto issue_load = [&](int n, int st) {
+    const int blk_id = blockIdx.x + n * gridDim.x;
+    const int bh = blk_id / s.n_blocks, blk = blk_id % s.n_blocks;
+    mbar_arrive_expect_tx(&load[st], 2 * (D / 64) * kChunkB);
     for (int c = 0; c < D / 64; ++c) {
-      tma_load_3d(sK + c * 8192, &tmK, &bars[0], c * 64, blk * 64, bh);
-      tma_load_3d(sV + c * 8192, &tmV, &bars[0], c * 64, blk * 64, bh);
-      if (PROJ) tma_load_3d(sW + c * D * 128, &tmW, &bars[0], c * 64, 0, 0);
+      tma_load_3d(sK(st) + c * kChunkB, &tmK, &load[st], c * 64, blk * 64, bh);
+      tma_load_3d(sV(st) + c * kChunkB, &tmV, &load[st], c * 64, blk * 64, bh);
     }
-  }
-  bool ok = cta_wait(&bars[0], 0, abort_flag, status);
-  if (PROJ && tid == 0 && ok) {
-    // (V_j W)^T = W^T V_j^T: M = c_out (128), N = t (64), K = c_in (D)
-    tc_fence_after();
-    constexpr uint32_t id = idesc_bf16(128, 64, true, false);
-    #pragma unroll
-    for (int kk = 0; kk < D / 16; ++kk) {
-      const uint64_t a = desc_mnmajor(smem_u32(sW) + kk * 2048, D * 128);
-      const uint64_t b = desc_kmajor(smem_u32(sV) + (kk >> 2) * 8192 + (kk & 3) * 32);
-      mma_bf16_ss(tmem + kColP, a, b, id, kk > 0 ? 1u : 0u);
+  };
+  const int mine = blockIdx.x < total ? (total - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+  if (tid == 0 && mine > 0) {
+    if (PROJ) {
+      mbar_arrive_expect_tx(w_bar, (D / 64) * D * 128);
+      for (int c = 0; c < D / 64; ++c) tma_load_3d(sW + c * D * 128, &tmW, w_bar, c * 64, 0, 0);
     }
-    mma_commit(&bars[1]);
+    issue_load(0, 0);
+    if (mine > 1) issue_load(1, 1);
   }
+  bool ok = true;
+  if (PROJ && mine > 0) ok = cta_wait(w_bar, 0, abort_flag, status);
 
-  // phi in place (pad tokens -> 0) and column sums z
   constexpr int kCPR = D / 8, kRS = 128 / kCPR;
   const int g = tid % kCPR, rs = tid / kCPR;
   const int chunk = g >> 3, q8 = g & 7;
-  const int nvalid = block_valid_count(s, blk);
-  float z[8];
-  #pragma unroll
-  for (int i = 0; i < 8; ++i) z[i] = 0.f;
-  if (ok) {
+  for (int n = 0; n < mine && ok; ++n) {
+    const int st = n & 1;
+    const int blk_id = blockIdx.x + n * gridDim.x;
+    const int bh = blk_id / s.n_blocks, blk = blk_id % s.n_blocks;
+    uint8_t* k_s = sK(st);
+    uint8_t* v_s = sV(st);
+    if (!(ok = cta_wait(&load[st], (n >> 1) & 1, abort_flag, status))) break;
+    if (PROJ && tid == 0) {
+      // (V_j W)^T = W^T V_j^T: M = c_out (128), N = t (64), K = c_in (D)
+      tc_fence_after();
+      constexpr uint32_t id = idesc_bf16(128, 64, true, false);
+      #pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint64_t a = desc_mnmajor(smem_u32(sW) + kk * 2048, D * 128);
+        const uint64_t b = desc_kmajor(smem_u32(v_s) + (kk >> 2) * kChunkB + (kk & 3) * 32);
+        mma_bf16_ss(tmem + kColP, a, b, id, kk > 0 ? 1u : 0u);
+      }
+      mma_commit(mma0);
+    }
+    // phi in place (pad tokens -> 0) and column sums z
+    const int nvalid = block_valid_count(s, blk);
+    float z[8];
+    #pragma unroll
+    for (int i = 0; i < 8; ++i) z[i] = 0.f;
     for (int t = rs; t < 64; t += kRS) {
-      uint4* p = reinterpret_cast<uint4*>(sK + chunk * 8192 + sw128_offset(t, q8));
-      const uint4 u = *p;
+      uint4* pk = reinterpret_cast<uint4*>(k_s + chunk * kChunkB + sw128_offset(t, q8));
+      const uint4 u = *pk;
       const uint32_t w[4] = {u.x, u.y, u.z, u.w};
       uint32_t o[4];
       #pragma unroll
@@ -124,16 +162,14 @@ key_states_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
         z[2 * i + 1] += b;
         o[i] = pack_bf16(a, b);
       }
-      *p = make_uint4(o[0], o[1], o[2], o[3]);
+      *pk = make_uint4(o[0], o[1], o[2], o[3]);
     }
-  }
-  #pragma unroll
-  for (int i = 0; i < 8; ++i) zred[rs * D + g * 8 + i] = z[i];
-  if (PROJ) {
-    // (V W)^T from TMEM into shared memory as the K-major A operand of the next MMA
-    if (ok) ok = cta_wait(&bars[1], 0, abort_flag, status);
-    tc_fence_after();
-    if (ok) {
+    #pragma unroll
+    for (int i = 0; i < 8; ++i) zred[rs * D + g * 8 + i] = z[i];
+    if (PROJ) {
+      // (V W)^T from TMEM over the V stage (V has been consumed): K-major A of the next MMA
+      if (!(ok = cta_wait(mma0, n & 1, abort_flag, status))) break;
+      tc_fence_after();
       uint32_t r[32], r2[32];
       tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + kColP, r);
       tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + kColP + 32, r2);
@@ -142,59 +178,61 @@ key_states_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
       for (int c8 = 0; c8 < 8; ++c8) {
         const uint32_t* src = c8 < 4 ? r : r2;
         const int b = (c8 & 3) * 8;
-        *reinterpret_cast<uint4*>(sVp + sw128_offset(tid, c8)) =
+        *reinterpret_cast<uint4*>(v_s + sw128_offset(tid, c8)) =
             make_uint4(pack_bf16(__uint_as_float(src[b]), __uint_as_float(src[b + 1])),
                        pack_bf16(__uint_as_float(src[b + 2]), __uint_as_float(src[b + 3])),
                        pack_bf16(__uint_as_float(src[b + 4]), __uint_as_float(src[b + 5])),
                        pack_bf16(__uint_as_float(src[b + 6]), __uint_as_float(src[b + 7])));
       }
     }
-  }
-  fence_proxy_async_smem();
-  tc_fence_before();
-  __syncthreads();
-
-  if (tid == 0 && ok) {
-    // h^T = A^T-product: M = c (128), N = a (D), K = t (64)
-    tc_fence_after();
-    constexpr uint32_t id = idesc_bf16(128, D, !PROJ, true);
-    #pragma unroll
-    for (int kk = 0; kk < 4; ++kk) {
-      const uint64_t a = PROJ ? desc_kmajor(smem_u32(sVp) + kk * 32) : desc_mnmajor(smem_u32(sV) + kk * 2048, 8192);
-      const uint64_t b = desc_mnmajor(smem_u32(sK) + kk * 2048, 8192);
-      mma_bf16_ss(tmem + kColH, a, b, id, kk > 0 ? 1u : 0u);
-    }
-    mma_commit(&bars[2]);
-  }
-  __nv_bfloat16* hrow = h + ((size_t)bh * s.n_blocks + blk) * (size_t)(D + 1) * D;
-  for (int a = tid; a < D; a += 128) {
-    float sum = 0.f;
-    #pragma unroll
-    for (int r = 0; r < kRS; ++r) sum += zred[r * D + a];
-    hrow[(size_t)D * D + a] = __float2bfloat16_rn(sum);
-  }
-  if (ok) ok = cta_wait(&bars[2], 0, abort_flag, status);
-  tc_fence_after();
-  if (ok && warp * 32 < D) {
-    const int c = tid;                       // TMEM lane = output row (value channel)
-    #pragma unroll 1
-    for (int cc = 0; cc < D / 32; ++cc) {
-      uint32_t r[32];
-      tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + kColH + cc * 32, r);
-      tmem_wait_ld();
-      uint4* dst = reinterpret_cast<uint4*>(hrow + (size_t)c * D + cc * 32);
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0) {
+      // h^T: M = c (128), N = a (D), K = t (64)
+      tc_fence_after();
+      constexpr uint32_t id = idesc_bf16(128, D, !PROJ, true);
       #pragma unroll
-      for (int i = 0; i < 4; ++i)
-        dst[i] = make_uint4(pack_bf16(__uint_as_float(r[8 * i]), __uint_as_float(r[8 * i + 1])),
-                            pack_bf16(__uint_as_float(r[8 * i + 2]), __uint_as_float(r[8 * i + 3])),
-                            pack_bf16(__uint_as_float(r[8 * i + 4]), __uint_as_float(r[8 * i + 5])),
-                            pack_bf16(__uint_as_float(r[8 * i + 6]), __uint_as_float(r[8 * i + 7])));
+      for (int kk = 0; kk < 4; ++kk) {
+        const uint64_t a = PROJ ? desc_kmajor(smem_u32(v_s) + kk * 32) : desc_mnmajor(smem_u32(v_s) + kk * 2048, kChunkB);
+        const uint64_t b = desc_mnmajor(smem_u32(k_s) + kk * 2048, kChunkB);
+        mma_bf16_ss(tmem + kColH, a, b, id, kk > 0 ? 1u : 0u);
+      }
+      mma_commit(mma1);
     }
+    __nv_bfloat16* hrow = h + ((size_t)bh * s.n_blocks + blk) * (size_t)(D + 1) * D;
+    for (int a = tid; a < D; a += 128) {
+      float sum = 0.f;
+      #pragma unroll
+      for (int r = 0; r < kRS; ++r) sum += zred[r * D + a];
+      hrow[(size_t)D * D + a] = __float2bfloat16_rn(sum);
+    }
+    if (!(ok = cta_wait(mma1, n & 1, abort_flag, status))) break;
+    tc_fence_after();
+    if (warp * 32 < D) {
+      const int c = tid;                     // TMEM lane = output row (value channel)
+      #pragma unroll 1
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t r[32];
+        tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + kColH + cc * 32, r);
+        tmem_wait_ld();
+        uint4* dst = reinterpret_cast<uint4*>(hrow + (size_t)c * D + cc * 32);
+        #pragma unroll
+        for (int i = 0; i < 4; ++i)
+          dst[i] = make_uint4(pack_bf16(__uint_as_float(r[8 * i]), __uint_as_float(r[8 * i + 1])),
+                              pack_bf16(__uint_as_float(r[8 * i + 2]), __uint_as_float(r[8 * i + 3])),
+                              pack_bf16(__uint_as_float(r[8 * i + 4]), __uint_as_float(r[8 * i + 5])),
+                              pack_bf16(__uint_as_float(r[8 * i + 6]), __uint_as_float(r[8 * i + 7])));
+      }
+    }
+    tc_fence_before();
+    __syncthreads();                          // stage st and the TMEM results are no longer read
+    if (tid == 0 && n + 2 < mine) issue_load(n + 2, st);
   }
   if (!ok && tid == 0) {
-    mma_commit(&bars[3]);
+    mma_commit(drain);
     const long long t0 = clock64();
-    while (!mbar_try_wait(&bars[3], 0) && clock64() - t0 < kWaitBudgetCycles) {}
+    while (!mbar_try_wait(drain, 0) && clock64() - t0 < kWaitBudgetCycles) {}
   }
   tc_fence_before();
   __syncthreads();
@@ -202,38 +240,45 @@ key_states_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
 }
 
 // ------------------------------------------------------------------ reduce states (GEMM)
-constexpr int kGemmStages = 2;
+// Persistent: one CTA per SM walks the output tiles (128 query blocks x 256
+// state columns) of every head; a 4-stage TMA ring runs across tile boundaries
+// and two TMEM accumulators let the epilogue of one tile overlap the main loop
+// of the next.  Tiles are ordered M-fastest so the query-block tiles sharing one
+// slab of h run back to back (h is read from HBM about once).
+constexpr int kGemmStages = 4;
 constexpr int kGemmBN = 256;
 constexpr int kGemmABytes = 128 * 128;          // 128 rows x 64 bf16
 constexpr int kGemmBBytes = 4 * 64 * 128;       // 4 chunks of 64 K-rows x 64 bf16
 constexpr int kGemmSmem = kGemmStages * (kGemmABytes + kGemmBBytes) + 256 + 1024;
 
-__global__ void __launch_bounds__(192, 2)
+__global__ void __launch_bounds__(192, 1)
 reduce_states_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                     __nv_bfloat16* __restrict__ Hs, int nb, int ntot, int* status) {
+                     __nv_bfloat16* __restrict__ Hs, int nb, int ntot, int BH, int* status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint8_t* sA = smem;
   uint8_t* sB = smem + kGemmStages * kGemmABytes;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kGemmStages * (kGemmABytes + kGemmBBytes));
-  uint64_t* full = bars;
-  uint64_t* empty = bars + kGemmStages;
-  uint64_t* acc = bars + 2 * kGemmStages;
-  uint64_t* drain = acc + 1;
+  uint64_t* full = bars;                          // [4]
+  uint64_t* empty = bars + kGemmStages;           // [4]
+  uint64_t* acc_full = empty + kGemmStages;       // [2] MMA -> epilogue
+  uint64_t* acc_empty = acc_full + 2;             // [2] epilogue -> MMA (128 arrivals)
+  uint64_t* drain = acc_empty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int m0 = blockIdx.x * 128, n0 = blockIdx.y * kGemmBN, bh = blockIdx.z;
   const int kt_total = (nb + 63) / 64;
+  const int mt = (nb + 127) / 128, nt = (ntot + kGemmBN - 1) / kGemmBN;
+  const int n_tiles = mt * nt * BH;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kGemmStages; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
-    mbar_init(acc, 1);
+    for (int b = 0; b < 2; ++b) { mbar_init(&acc_full[b], 1); mbar_init(&acc_empty[b], 128); }
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 5) { tmem_alloc(tmem_slot, 256); tmem_relinquish(); }
+  if (warp == 5) { tmem_alloc(tmem_slot, 512); tmem_relinquish(); }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -241,17 +286,21 @@ reduce_states_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
 
   if (warp == 4) {
     if (lane == 0) {
-      int kt = 0;
-      for (; kt < kt_total; ++kt) {
-        const int s = kt % kGemmStages;
-        if (kt >= kGemmStages && !mbar_wait(&empty[s], ((kt / kGemmStages) - 1) & 1, abort_flag, status)) break;
-        mbar_arrive_expect_tx(&full[s], kGemmABytes + kGemmBBytes);
-        tma_load_3d(sA + s * kGemmABytes, &tmA, &full[s], kt * 64, m0, bh);
-        for (int c = 0; c < 4; ++c)
-          tma_load_3d(sB + s * kGemmBBytes + c * 8192, &tmB, &full[s], n0 + c * 64, kt * 64, bh);
+      int it = 0;                                 // global k-iteration counter across tiles
+      bool ok = true;
+      for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
+        const int m0 = (t % mt) * 128, n0 = ((t / mt) % nt) * kGemmBN, bh = t / (mt * nt);
+        for (int kt = 0; kt < kt_total; ++kt, ++it) {
+          const int s = it % kGemmStages;
+          if (it >= kGemmStages && !mbar_wait(&empty[s], ((it / kGemmStages) - 1) & 1, abort_flag, status)) { ok = false; break; }
+          mbar_arrive_expect_tx(&full[s], kGemmABytes + kGemmBBytes);
+          tma_load_3d(sA + s * kGemmABytes, &tmA, &full[s], kt * 64, m0, bh);
+          for (int c = 0; c < 4; ++c)
+            tma_load_3d(sB + s * kGemmBBytes + c * 8192, &tmB, &full[s], n0 + c * 64, kt * 64, bh);
+        }
       }
       if (*abort_flag) {
-        for (int i = (kt - kGemmStages > 0 ? kt - kGemmStages : 0); i < kt; ++i) {
+        for (int i = (it - kGemmStages > 0 ? it - kGemmStages : 0); i < it; ++i) {
           const long long t0 = clock64();
           while (!mbar_try_wait(&full[i % kGemmStages], (i / kGemmStages) & 1) && clock64() - t0 < kWaitBudgetCycles) {}
         }
@@ -260,35 +309,46 @@ reduce_states_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
   } else if (warp == 5) {
     if (lane == 0) {
       constexpr uint32_t id = idesc_bf16(128, kGemmBN, false, true);
+      int it = 0, local = 0;
       bool ok = true;
-      for (int kt = 0; kt < kt_total; ++kt) {
-        const int s = kt % kGemmStages;
-        if (!mbar_wait(&full[s], (kt / kGemmStages) & 1, abort_flag, status)) { ok = false; break; }
+      for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++local) {
+        const int ab = local & 1;
+        // the accumulator must have been drained by the epilogue of tile local-2
+        if (local >= 2 && !mbar_wait(&acc_empty[ab], ((local - 2) >> 1) & 1, abort_flag, status)) { ok = false; break; }
         tc_fence_after();
-        #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t a = desc_kmajor(smem_u32(sA + s * kGemmABytes) + kk * 32);
-          const uint64_t b = desc_mnmajor(smem_u32(sB + s * kGemmBBytes) + kk * 2048, 8192);
-          mma_bf16_ss(tmem, a, b, id, (kt > 0 || kk > 0) ? 1u : 0u);
+        for (int kt = 0; kt < kt_total; ++kt, ++it) {
+          const int s = it % kGemmStages;
+          if (!mbar_wait(&full[s], (it / kGemmStages) & 1, abort_flag, status)) { ok = false; break; }
+          tc_fence_after();
+          #pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t a = desc_kmajor(smem_u32(sA + s * kGemmABytes) + kk * 32);
+            const uint64_t b = desc_mnmajor(smem_u32(sB + s * kGemmBBytes) + kk * 2048, 8192);
+            mma_bf16_ss(tmem + ab * kGemmBN, a, b, id, (kt > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(&empty[s]);
         }
-        mma_commit(&empty[s]);
+        if (ok) mma_commit(&acc_full[ab]);
       }
-      mma_commit(ok ? acc : drain);
       if (!ok) {
+        mma_commit(drain);
         const long long t0 = clock64();
         while (!mbar_try_wait(drain, 0) && clock64() - t0 < kWaitBudgetCycles) {}
       }
     }
   } else {
-    const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(acc, 0, abort_flag, status));
-    tc_fence_after();
     const int r = threadIdx.x;
-    const int m = m0 + r;
-    if (ok) {
+    int local = 0;
+    for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++local) {
+      const int ab = local & 1;
+      const int m0 = (t % mt) * 128, n0 = ((t / mt) % nt) * kGemmBN, bh = t / (mt * nt);
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait(&acc_full[ab], (local >> 1) & 1, abort_flag, status))) break;
+      tc_fence_after();
+      const int m = m0 + r;
       #pragma unroll 1
       for (int cc = 0; cc < kGemmBN / 32; ++cc) {
         uint32_t v[32];
-        tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + cc * 32, v);
+        tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + ab * kGemmBN + cc * 32, v);
         tmem_wait_ld();
         const int n = n0 + cc * 32;
         if (m < nb && n < ntot) {
@@ -301,11 +361,13 @@ reduce_states_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
                                 pack_bf16(__uint_as_float(v[8 * i + 6]), __uint_as_float(v[8 * i + 7])));
         }
       }
+      tc_fence_before();
+      mbar_arrive(&acc_empty[ab]);
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) { tc_fence_after(); tmem_dealloc(tmem, 256); }
+  if (warp == 5) { tc_fence_after(); tmem_dealloc(tmem, 512); }
 }
 
 // ------------------------------------------------------------------ linear apply
@@ -464,11 +526,15 @@ cudaError_t launch_key_states(const void* k, const void* v, const void* w_proj, 
   } else {
     mw = mk;
   }
-  dim3 grid(s.n_blocks, BH);
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const long long blocks = (long long)BH * s.n_blocks;
+  const int grid = (int)(blocks < 2LL * sms ? blocks : 2LL * sms);
   auto go = [&](auto kern) -> cudaError_t {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kKsSmemRequest);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kKsSmem);
     if (e != cudaSuccess) return e;
-    kern<<<grid, 128, kKsSmemRequest, st>>>(mk, mv, mw, h, s, status);
+    kern<<<grid, 128, kKsSmem, st>>>(mk, mv, mw, h, s, BH, status);
     return cudaGetLastError();
   };
   if (d == 128) return w_proj ? go(key_states_kernel<128, true>) : go(key_states_kernel<128, false>);
@@ -489,8 +555,12 @@ cudaError_t launch_reduce_states(const __nv_bfloat16* m01, int ld_m01, const __n
     return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(reduce_states_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem);
   if (e != cudaSuccess) return e;
-  dim3 grid((nb + 127) / 128, (ntot + kGemmBN - 1) / kGemmBN, BH);
-  reduce_states_kernel<<<grid, 192, kGemmSmem, st>>>(ma, mb, Hs, nb, ntot, status);
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const long long tiles = (long long)((nb + 127) / 128) * ((ntot + kGemmBN - 1) / kGemmBN) * BH;
+  const int grid = (int)(tiles < sms ? tiles : sms);
+  reduce_states_kernel<<<grid, 192, kGemmSmem, st>>>(ma, mb, Hs, nb, ntot, BH, status);
   return cudaGetLastError();
 }
 

@@ -29,14 +29,14 @@ cudaError_t launch_far_pool(const void* k, const void* v, void* kf, void* vf, in
                             int F, int Hh, int Ww, int cf, int ch, int cw, cudaStream_t st);
 
 // ------------------------------------------------------------ classification (k_classify.cu)
-// logits[bh][i][j] = qbar_i . kbar_j / sqrt(d) in fp64.
+// logits[bh][i][j] = qbar_i . kbar_j in fp64 (the scale 1/sqrt(d) is applied where P_c is formed).
 cudaError_t launch_block_logits(const double* qbar, const double* kbar, double* logits,
                                 int BH, int nb, int d, cudaStream_t st);
 
 // Per row: top kc -> 1, bottom kn -> -1, rest 0; critical list ascending; the
 // marginal indicator m01 (bf16 1/0, row stride ld_m01, pad columns 0); optional
-// P_c in fp32.
-cudaError_t launch_classify_rows(const double* logits, int BH, int nb, int kc, int kn,
+// P_c = softmax(logits / sqrt(d)) in fp32.
+cudaError_t launch_classify_rows(const double* logits, int BH, int nb, int d, int kc, int kn,
                                  int8_t* mask, int32_t* crit_idx, int32_t* crit_cnt,
                                  __nv_bfloat16* m01, int ld_m01, float* scores, cudaStream_t st);
 

@@ -446,7 +446,7 @@ slr_status slr_pool_classify(const void* q, const void* k, const slr_seq* seq, f
   SLR_TRY(cudaMemsetAsync(status, 0, sizeof(int), s));
   SLR_LAUNCH(kKPool, s, launch_pool_means(q, k, w.qbar, w.kbar, sh.BH, sh.d, sh.s, s));
   SLR_LAUNCH(kKLogits, s, launch_block_logits(w.qbar, w.kbar, w.logits, sh.BH, sh.nb, sh.d, s));
-  SLR_LAUNCH(kKClassify, s, launch_classify_rows(w.logits, sh.BH, sh.nb, kc, kn, mask, crit_idx, crit_cnt, w.m01, ld_m01(sh.nb),
+  SLR_LAUNCH(kKClassify, s, launch_classify_rows(w.logits, sh.BH, sh.nb, sh.d, kc, kn, mask, crit_idx, crit_cnt, w.m01, ld_m01(sh.nb),
                                scores_opt, s));
   return SLR_OK;
 }
@@ -538,7 +538,7 @@ slr_status slr_sparse_linear_attn(const void* q, const void* k, const void* v, c
   int8_t* mask = mask_out_opt ? mask_out_opt : w.mask;
   SLR_LAUNCH(kKPool, s, launch_pool_means(q, k, w.cls.qbar, w.cls.kbar, sh.BH, sh.d, sh.s, s));
   SLR_LAUNCH(kKLogits, s, launch_block_logits(w.cls.qbar, w.cls.kbar, w.cls.logits, sh.BH, sh.nb, sh.d, s));
-  SLR_LAUNCH(kKClassify, s, launch_classify_rows(w.cls.logits, sh.BH, sh.nb, kc, kn, mask, w.crit_idx, w.crit_cnt, w.cls.m01,
+  SLR_LAUNCH(kKClassify, s, launch_classify_rows(w.cls.logits, sh.BH, sh.nb, sh.d, kc, kn, mask, w.crit_idx, w.crit_cnt, w.cls.m01,
                                ld_m01(sh.nb), nullptr, s));
   ListArgs la;
   memset(&la, 0, sizeof(la));
