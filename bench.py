@@ -56,6 +56,23 @@ def load_peaks():
     return PEAKS_FALLBACK, "fallback"
 
 
+def measured_traffic(kernel: str):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, or None when
+    the kernel's source has changed since those counters were taken."""
+    import hashlib
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        rec = json.load(f).get(kernel)
+    if not rec:
+        return None
+    with open(os.path.join(ROOT, rec["source"]), "rb") as f:
+        if hashlib.sha256(f.read()).hexdigest() != rec["sha256"]:
+            return None
+    return rec["dram_bytes_per_launch"]
+
+
 def config_dict(w):
     return {
         "workload": (f"{w.name}: SLA layer B={w.batch} H={w.heads} d={w.d} N={w.n_pad} "
@@ -202,17 +219,11 @@ def main():
         raise SystemExit("bench.py times the SLA call; pick an SLA workload")
     warmup = max(3, args.warmup)
 
-    rank = int(os.environ.get("RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    dist = None
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        backend = "nccl" if args.impl == "slr" else "gloo"
-        if args.impl == "slr":
-            torch.cuda.set_device(local)
-        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+    from block_sparse_linear_02_b200 import dist as sdist
+    rank, world, local = sdist.env_ranks()
+    if world > 1 and args.impl == "slr":
+        torch.cuda.set_device(local)
+    dist = sdist.init("nccl" if args.impl == "slr" else "gloo", timeout_s=300)
 
     if args.impl == "reference":
         run_reference(args, w, rank, world, warmup)
@@ -250,12 +261,7 @@ def main():
             fn()
         b.record(stream)
         barrier()
-        ms = a.elapsed_time(b) / steps
-        if dist is not None:
-            t = torch.tensor([ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ms = float(t.item())
-        return ms
+        return sdist.max_over_ranks(a.elapsed_time(b) / steps, device=dev)
 
     # warm-up (both modes)
     for _ in range(warmup):
@@ -312,7 +318,7 @@ def main():
         e2e_ms = timed(e2e_step, max(3, args.steps // 4))
         h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv, hw))
         d2h = ho.numel() * ho.element_size()
-        e2e = {"value": round(e2e_ms / world, 4), "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+        e2e = {"value": round(sdist.aggregate_ms_per_call(e2e_ms, world), 4), "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
     clk = clocks.stop()
 
     cpu = None
@@ -325,7 +331,7 @@ def main():
     if rank == 0:
         line = {
             "metric": METRIC,
-            "value": round(ms_sparse / world, 4),
+            "value": round(sdist.aggregate_ms_per_call(ms_sparse, world), 4),
             "unit": UNIT,
             "n_gpus": world,
             "steps": args.steps,
@@ -349,7 +355,7 @@ def main():
                 "unit": "TFLOP/s",
                 "frac": round(attn_tf / peak_tf, 4),
                 "peak_source": f"{peak_src} bf16 burst",
-                "traffic": None,
+                "traffic": measured_traffic("attention"),
                 "flops_per_launch": crit_fl,
                 "ms_per_launch": round(attn_ms_per, 4),
             },
