@@ -18,9 +18,10 @@
 // list is consumed two entries per STEP (128 keys): one 128x128 S tile per step
 // keeps the MMA instruction count and the commits per key low.
 // Warp roles (320 threads):
-//   warp 8     TMA producer: Q once, then K_0, V_0, K_1, V_1, ... (each item the
-//              step's two 64-key blocks) into a 5-slot ring, then the
-//              linear-branch state rows;
+//   warp 8     TMA producer: Q once (with the Z rows of the linear states), then
+//              K_0, V_0, K_1, V_1, ... (each item the step's two 64-key blocks)
+//              into a 5-slot ring, then the H'^T rows of the linear states as
+//              one more item per query block, so they land during the last steps;
 //   warp 9     MMA issuer: S_j = Q [K_a ; K_b]^T (N = 128) into one of two TMEM
 //              S buffers; once both softmax warpgroups have written P_j back
 //              over S_j (bf16, in TMEM), O_0 += P_j[:, a] V_a and
@@ -47,6 +48,7 @@ constexpr uint32_t kColO0 = 0;      // accumulator of warpgroup 0
 constexpr uint32_t kColO1 = 128;    // accumulator of warpgroup 1
 constexpr uint32_t kColS = 256;     // two 128-column S/P buffers: [256, 384) and [384, 512)
 constexpr uint32_t kColLin = 256;   // linear branch result (reuses the S buffers after the loop)
+constexpr float kLog2e = 1.4426950408889634f;
 
 template <int D>
 struct AttnLayout {
@@ -54,15 +56,18 @@ struct AttnLayout {
   static constexpr int kTile = 128 * 128;                // bytes of one 128-row chunk (Q, or two K/V blocks)
   static constexpr int kHalf = 64 * 128;                 // bytes of one 64-row block inside a chunk
   static constexpr int kKV = kChunks * kTile;            // one ring item: K (or V) of one step
-  static constexpr int kNL = D + 16;                     // rows of a linear state tile (d + z + zero pad)
-  static constexpr int kHsChunk = kNL * 128;
-  static constexpr int kHsTile = kChunks * kHsChunk;
+  static constexpr int kHsChunk = D * 128;               // H'^T rows of one query block: D rows per 64-column chunk
+  static constexpr int kHsTile = kChunks * kHsChunk;     // one ring item
+  static constexpr int kZChunk = 16 * 128;               // [Z ; 15 zero rows] per 64-column chunk
+  static constexpr int kZTile = kChunks * kZChunk;
   static constexpr int kQOff = 0;
   static constexpr int kRingOff = kQOff + kChunks * kTile;
-  static constexpr int kXOff = kRingOff + kSlots * kKV;  // exchange area: 6 x 128 floats
+  static constexpr int kZOff = kRingOff + kSlots * kKV;  // Z tiles of the pair's two query blocks
+  static constexpr int kXOff = kZOff + 2 * kZTile;       // exchange area: 6 x 128 floats
   static constexpr int kBarOff = kXOff + 6 * 128 * 4;
   static constexpr int kBytes = kBarOff + 256 + 1024;    // + alignment slack
-  static_assert(2 * kHsTile <= kSlots * kKV, "linear state tiles must fit in the K/V ring");
+  static_assert(kHsTile <= kKV, "a linear state tile must fit in one ring slot");
+  static_assert(kBytes <= 227 * 1024, "shared memory budget");
 };
 
 struct AttnKParams {
@@ -89,6 +94,9 @@ __device__ __forceinline__ float ex2(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+
+// phi(x) = elu(x) + 1, with exp through the exp2 unit (the result is rounded to bf16)
+__device__ __forceinline__ float phi_fast(float x) { return x > 0.f ? x + 1.f : ex2(x * kLog2e); }
 
 __device__ __forceinline__ float max3(float a, float b, float c) {
   float r;
@@ -148,12 +156,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
             const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmX1,
             const __grid_constant__ CUtensorMap tmX2, const AttnKParams p) {
-  // tmX1/tmX2: far-field K/V maps (GATED) or the linear state map (LINEAR, tmX1).
+  // tmX1/tmX2: far-field K/V maps (GATED), or the linear state maps (LINEAR): tmX1 the
+  // H'^T rows (box D rows), tmX2 the Z row with 15 rows of zero fill (box 16 rows).
   using L = AttnLayout<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem + L::kQOff;
   uint8_t* sRing = smem + L::kRingOff;
+  uint8_t* sZ = smem + L::kZOff;
   float* xch = reinterpret_cast<float*>(smem + L::kXOff);   // [6][128]: m0 m1 l0 l1 far-l spare
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
   uint64_t* q_full = bars + 0;
@@ -161,9 +171,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
   uint64_t* s_full = slot_full + kSlots;         // [2] per S buffer
   uint64_t* p_full = s_full + 2;                 // [2] per S buffer, 256 arrivals
   uint64_t* pv_done = p_full + 2;                // [4] per step mod 4 (phases cannot alias)
-  uint64_t* loop_done = pv_done + 4;
-  uint64_t* hs_full = loop_done + 1;
-  uint64_t* phiq_ready = hs_full + 1;
+  uint64_t* phiq_ready = pv_done + 4;
   uint64_t* lin_done = phiq_ready + 1;
   uint64_t* drain = lin_done + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
@@ -184,6 +192,9 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
   const int local_steps = (n_local + 1) >> 1;
   const int n_steps = local_steps + (GATED ? 1 : 0);   // the far block is a step of its own
   const bool second_exists = 2 * pair + 1 < p.n_qb;
+  const int n_lin = LINEAR ? (second_exists ? 2 : 1) : 0;   // linear state items after the K/V items
+  const int n_items = 2 * n_steps + n_lin;
+  const bool active = n_steps > 0 || LINEAR;
   // blocks in step j: 2, except an odd tail (1) and the far step (1, handled by warpgroup 0)
   auto step_blocks = [&](int j) -> int {
     if (GATED && j == local_steps) return 1;
@@ -198,8 +209,6 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
       mbar_init(&p_full[b], 256);
     }
     for (int b = 0; b < 4; ++b) mbar_init(&pv_done[b], 1);
-    mbar_init(loop_done, 1);
-    mbar_init(hs_full, 1);
     mbar_init(phiq_ready, 256);
     mbar_init(lin_done, 1);
     mbar_init(drain, 1);
@@ -214,9 +223,9 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
 
   if (warp == 8) {
     // ---------------------------------------------------------------- producer
-    if (lane == 0 && n_steps > 0) {
+    if (lane == 0 && active) {
       tma_prefetch_desc(&tmQ); tma_prefetch_desc(&tmK); tma_prefetch_desc(&tmV);
-      mbar_arrive_expect_tx(q_full, L::kChunks * L::kTile);
+      mbar_arrive_expect_tx(q_full, L::kChunks * L::kTile + n_lin * L::kZTile);
       if (TILE) {
         for (int half = 0; half < 2; ++half) {
           int tf, th, tw;
@@ -227,21 +236,34 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
       } else {
         for (int c = 0; c < L::kChunks; ++c) tma_load_3d(sQ + c * L::kTile, &tmQ, q_full, c * 64, pair * 128, bh);
       }
-      // item i: K (even i) or V (odd i) of step i/2, in slot i % kSlots; the slot's
-      // previous item (i - kSlots) is free once the P.V of its step has completed
+      for (int b = 0; b < n_lin; ++b)   // row D of the state (Z) and 15 rows of zero fill
+        for (int c = 0; c < L::kChunks; ++c)
+          tma_load_3d(sZ + b * L::kZTile + c * L::kZChunk, &tmX2, q_full, c * 64, D, bh * p.n_qb + 2 * pair + b);
+      // item i < 2 n_steps: K (even i) or V (odd i) of step i/2; then the H'^T rows of
+      // the query blocks.  Item i lives in slot i % kSlots; the slot's previous item
+      // (i - kSlots, always a K/V item) is free once the P.V of its step has completed.
       int i = 0;
-      for (; i < 2 * n_steps; ++i) {
-        const int j = i >> 1, slot = i % kSlots;
-        const bool is_v = i & 1;
+      for (; i < n_items; ++i) {
+        const int slot = i % kSlots;
         if (i >= kSlots) {
           const int q = (i - kSlots) >> 1;
           if (!mbar_wait(&pv_done[q & 3], (q >> 2) & 1, abort_flag, p.status)) break;
         }
+        uint8_t* dst0 = sRing + slot * L::kKV;
+        if (LINEAR && i >= 2 * n_steps) {
+          const int b = i - 2 * n_steps;
+          mbar_arrive_expect_tx(&slot_full[slot], L::kHsTile);
+          for (int c = 0; c < L::kChunks; ++c)
+            tma_load_3d(dst0 + c * L::kHsChunk, &tmX1, &slot_full[slot], c * 64, 0, bh * p.n_qb + 2 * pair + b);
+          continue;
+        }
+        const int j = i >> 1;
+        const bool is_v = i & 1;
         const int nb = step_blocks(j);
         const bool far = GATED && j == local_steps;
         mbar_arrive_expect_tx(&slot_full[slot], nb * L::kChunks * L::kHalf);
         for (int b = 0; b < nb; ++b) {
-          uint8_t* dst = sRing + slot * L::kKV + b * L::kHalf;
+          uint8_t* dst = dst0 + b * L::kHalf;
           if (far) {
             for (int c = 0; c < L::kChunks; ++c)
               tma_load_3d(dst + c * L::kTile, is_v ? &tmX2 : &tmX1, &slot_full[slot], c * 64, 0, bh);
@@ -259,26 +281,19 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
           }
         }
       }
-      const int j = i >> 1;
-      if (LINEAR && j == n_steps && mbar_wait(loop_done, 0, abort_flag, p.status)) {
-        // the K/V ring is free: bring in the [H'^T ; Z] rows of both query blocks
-        const int nblk = second_exists ? 2 : 1;
-        mbar_arrive_expect_tx(hs_full, nblk * L::kHsTile);
-        for (int b = 0; b < nblk; ++b)
-          for (int c = 0; c < L::kChunks; ++c)
-            tma_load_3d(sRing + b * L::kHsTile + c * L::kHsChunk, &tmX1, hs_full, c * 64, 0, bh * p.n_qb + 2 * pair + b);
-      }
       if (*abort_flag) {
         // let the loads already in flight land before the CTA's shared memory is released
+        long long t0 = clock64();
+        while (!mbar_try_wait(q_full, 0) && clock64() - t0 < kWaitBudgetCycles) {}
         for (int it = (i - kSlots > 0 ? i - kSlots : 0); it < i; ++it) {
-          const long long t0 = clock64();
+          t0 = clock64();
           while (!mbar_try_wait(&slot_full[it % kSlots], (it / kSlots) & 1) && clock64() - t0 < kWaitBudgetCycles) {}
         }
       }
     }
   } else if (warp == 9) {
     // ---------------------------------------------------------------- MMA issuer
-    if (lane == 0 && n_steps > 0) {
+    if (lane == 0 && active) {
       constexpr uint32_t idS = idesc_bf16(128, 128, false, false);
       constexpr uint32_t idO = idesc_bf16(128, D, false, true);
       const uint32_t q_addr = smem_u32(sQ), ring_addr = smem_u32(sRing);
@@ -300,12 +315,15 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
           mma_bf16_ts(tmem + col, a, b, idO, (acc || kk > 0) ? 1u : 0u);
         }
       };
-      bool ok = mbar_wait(q_full, 0, abort_flag, p.status) && mbar_wait(&slot_full[0], 0, abort_flag, p.status);
+      bool ok = mbar_wait(q_full, 0, abort_flag, p.status);
       bool o1_started = false;
-      if (ok) {
-        tc_fence_after();
-        issue_qk(0, 0);
-        mma_commit(&s_full[0]);
+      if (ok && n_steps > 0) {
+        ok = mbar_wait(&slot_full[0], 0, abort_flag, p.status);
+        if (ok) {
+          tc_fence_after();
+          issue_qk(0, 0);
+          mma_commit(&s_full[0]);
+        }
         for (int j = 0; j < n_steps && ok; ++j) {
           const int b = j & 1;
           if (j + 1 < n_steps) {
@@ -332,32 +350,35 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
           }
           mma_commit(&pv_done[j & 3]);
         }
-        if (ok) mma_commit(loop_done);
-        if (ok && LINEAR) {
-          ok = mbar_wait(hs_full, 0, abort_flag, p.status) && mbar_wait(phiq_ready, 0, abort_flag, p.status);
-          if (ok) {
-            tc_fence_after();
-            constexpr uint32_t idL = idesc_bf16(128, L::kNL, false, false);
-            const uint32_t lo_only[4] = {0u, 0u, 0xFFFFFFFFu, 0xFFFFFFFFu};   // write lanes 0-63
-            const uint32_t hi_only[4] = {0xFFFFFFFFu, 0xFFFFFFFFu, 0u, 0u};   // write lanes 64-127
+      }
+      if (ok && LINEAR) {
+        // lin = phi(Q) [H'^T ; Z]^T per query block (lanes of the other block masked off);
+        // column D of the result is the denominator phi(q) . Z
+        ok = mbar_wait(phiq_ready, 0, abort_flag, p.status);
+        for (int b = 0; b < n_lin && ok; ++b) {
+          const int it = 2 * n_steps + b;
+          ok = mbar_wait(&slot_full[it % kSlots], (it / kSlots) & 1, abort_flag, p.status);
+        }
+        if (ok) {
+          tc_fence_after();
+          constexpr uint32_t idH = idesc_bf16(128, D, false, false);
+          constexpr uint32_t idZ = idesc_bf16(128, 16, false, false);
+          const uint32_t z_addr = smem_u32(sZ);
+          const uint32_t lo_only[4] = {0u, 0u, 0xFFFFFFFFu, 0xFFFFFFFFu};   // write lanes 0-63
+          const uint32_t hi_only[4] = {0xFFFFFFFFu, 0xFFFFFFFFu, 0u, 0u};   // write lanes 64-127
+          for (int b = 0; b < n_lin; ++b) {
+            const int slot = (2 * n_steps + b) % kSlots;
             #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
               const int c = kk >> 2, sub = kk & 3;
               const uint64_t a = desc_kmajor(q_addr + c * L::kTile + sub * 32);
-              const uint64_t bd = desc_kmajor(ring_addr + c * L::kHsChunk + sub * 32);
-              mma_bf16_ss_masked(tmem + kColLin, a, bd, idL, kk > 0 ? 1u : 0u, lo_only);
+              const uint64_t bh_ = desc_kmajor(ring_addr + slot * L::kKV + c * L::kHsChunk + sub * 32);
+              const uint64_t bz = desc_kmajor(z_addr + b * L::kZTile + c * L::kZChunk + sub * 32);
+              mma_bf16_ss_masked(tmem + kColLin, a, bh_, idH, kk > 0 ? 1u : 0u, b ? hi_only : lo_only);
+              mma_bf16_ss_masked(tmem + kColLin + D, a, bz, idZ, kk > 0 ? 1u : 0u, b ? hi_only : lo_only);
             }
-            if (second_exists) {
-              #pragma unroll
-              for (int kk = 0; kk < D / 16; ++kk) {
-                const int c = kk >> 2, sub = kk & 3;
-                const uint64_t a = desc_kmajor(q_addr + c * L::kTile + sub * 32);
-                const uint64_t bd = desc_kmajor(ring_addr + L::kHsTile + c * L::kHsChunk + sub * 32);
-                mma_bf16_ss_masked(tmem + kColLin, a, bd, idL, kk > 0 ? 1u : 0u, hi_only);
-              }
-            }
-            mma_commit(lin_done);
           }
+          mma_commit(lin_done);
         }
       }
       if (!ok) {
@@ -470,11 +491,6 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
       mbar_arrive(&p_full[b]);
       if (!far) started = true;
     }
-    if (ok && n_steps > 0)
-      ok = __all_sync(0xFFFFFFFFu, mbar_wait(&pv_done[(n_steps - 1) & 3], ((n_steps - 1) >> 2) & 1, abort_flag, p.status));
-    ok = __all_sync(0xFFFFFFFFu, ok);
-    tc_fence_after();
-
     // ---- token of this row
     int tok;
     bool row_exists;
@@ -493,7 +509,10 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
 
     bool lin_ok = false;
     if (LINEAR) {
-      // phi(Q) in place (every QK MMA has completed); pad rows -> 0
+      // phi(Q) in place: every QK MMA has completed (the last step's S was seen; with no
+      // step at all, Q has landed once q_full completes); pad rows -> 0
+      ok = __all_sync(0xFFFFFFFFu, ok);
+      if (ok && n_steps == 0) ok = __all_sync(0xFFFFFFFFu, mbar_wait(q_full, 0, abort_flag, p.status));
       if (ok) {
         constexpr int kGroups = D / 16;                  // 16-byte groups of my row handled by my warpgroup
         #pragma unroll
@@ -505,12 +524,18 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
           uint32_t o4[4];
           #pragma unroll
           for (int i = 0; i < 4; ++i)
-            o4[i] = valid ? pack_bf16(phi_elu1(bf16_lo(w[i])), phi_elu1(bf16_hi(w[i]))) : 0u;
+            o4[i] = valid ? pack_bf16(phi_fast(bf16_lo(w[i])), phi_fast(bf16_hi(w[i]))) : 0u;
           *ptr = make_uint4(o4[0], o4[1], o4[2], o4[3]);
         }
       }
       fence_proxy_async_smem();
       mbar_arrive(phiq_ready);
+    }
+    if (ok && n_steps > 0)
+      ok = __all_sync(0xFFFFFFFFu, mbar_wait(&pv_done[(n_steps - 1) & 3], ((n_steps - 1) >> 2) & 1, abort_flag, p.status));
+    ok = __all_sync(0xFFFFFFFFu, ok);
+    tc_fence_after();
+    if (LINEAR) {
       if (ok) lin_ok = __all_sync(0xFFFFFFFFu, mbar_wait(lin_done, 0, abort_flag, p.status));
       tc_fence_after();
     }
@@ -660,10 +685,13 @@ cudaError_t launch_attention(const AttnArgs& a, cudaStream_t st) {
     if (!make_tile_map(&maps[3], a.kf, 3, dims, strides, box)) return cudaErrorInvalidValue;
     if (!make_tile_map(&maps[4], a.vf, 3, dims, strides, box)) return cudaErrorInvalidValue;
   } else if (a.Hs) {
+    // [H'^T ; Z] rows of each query block: the D rows of H'^T, and Z with 15 rows of zero fill
     const uint64_t dims[3] = {(uint64_t)D, (uint64_t)(D + 1), (uint64_t)a.BH * a.n_qb};
     const uint64_t strides[2] = {rowb, rowb * (D + 1)};
-    const uint32_t box[3] = {64, (uint32_t)(D + 16), 1};
-    if (!make_tile_map(&maps[3], a.Hs, 3, dims, strides, box)) return cudaErrorInvalidValue;
+    const uint32_t boxh[3] = {64, (uint32_t)D, 1};
+    const uint32_t boxz[3] = {64, 16, 1};
+    if (!make_tile_map(&maps[3], a.Hs, 3, dims, strides, boxh)) return cudaErrorInvalidValue;
+    if (!make_tile_map(&maps[4], a.Hs, 3, dims, strides, boxz)) return cudaErrorInvalidValue;
   }
   AttnKParams kp;
   kp.n_pad = a.s.n_pad; kp.seg_len = a.s.seg_len; kp.seg_stride = a.s.seg_stride;
