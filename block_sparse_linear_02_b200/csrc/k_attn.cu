@@ -18,10 +18,10 @@
 // list is consumed two entries per STEP (128 keys): one 128x128 S tile per step
 // keeps the MMA instruction count and the commits per key low.
 // Warp roles (320 threads):
-//   warp 8     TMA producer: Q once (with the Z rows of the linear states), then
-//              K_0, V_0, K_1, V_1, ... (each item the step's two 64-key blocks)
-//              into a 5-slot ring, then the H'^T rows of the linear states as
-//              one more item per query block, so they land during the last steps;
+//   warp 8     TMA producer: Q once, then K_0, V_0, K_1, V_1, ... (each item the
+//              step's two 64-key blocks) into a 5-slot ring.  With LINEAR the
+//              first three slots first hold the two query blocks' linear states
+//              and phi(Q), and the K/V items start behind them;
 //   warp 9     MMA issuer: S_j = Q [K_a ; K_b]^T (N = 128) into one of two TMEM
 //              S buffers; once both softmax warpgroups have written P_j back
 //              over S_j (bf16, in TMEM), O_0 += P_j[:, a] V_a and
@@ -47,7 +47,6 @@ constexpr int kThreads = 320;
 constexpr uint32_t kColO0 = 0;      // accumulator of warpgroup 0
 constexpr uint32_t kColO1 = 128;    // accumulator of warpgroup 1
 constexpr uint32_t kColS = 256;     // two 128-column S/P buffers: [256, 384) and [384, 512)
-constexpr uint32_t kColLin = 256;   // linear branch result (reuses the S buffers after the loop)
 constexpr float kLog2e = 1.4426950408889634f;
 
 template <int D>
@@ -192,8 +191,11 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
   const int local_steps = (n_local + 1) >> 1;
   const int n_steps = local_steps + (GATED ? 1 : 0);   // the far block is a step of its own
   const bool second_exists = 2 * pair + 1 < p.n_qb;
-  const int n_lin = LINEAR ? (second_exists ? 2 : 1) : 0;   // linear state items after the K/V items
-  const int n_items = 2 * n_steps + n_lin;
+  const int n_lin = LINEAR ? (second_exists ? 2 : 1) : 0;   // linear state tiles
+  // LINEAR: ring slots 0 and 1 first hold the H'^T rows of the two query blocks and
+  // slot 2 holds phi(Q); K/V item i then takes ring position i + kPre
+  constexpr int kPre = LINEAR ? 3 : 0;
+  constexpr uint32_t kColLinOut = kColO0;   // lin (+ denominator at column D) before O_0/O_1 are first written
   const bool active = n_steps > 0 || LINEAR;
   // blocks in step j: 2, except an odd tail (1) and the far step (1, handled by warpgroup 0)
   auto step_blocks = [&](int j) -> int {
@@ -239,24 +241,38 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
       for (int b = 0; b < n_lin; ++b)   // row D of the state (Z) and 15 rows of zero fill
         for (int c = 0; c < L::kChunks; ++c)
           tma_load_3d(sZ + b * L::kZTile + c * L::kZChunk, &tmX2, q_full, c * 64, D, bh * p.n_qb + 2 * pair + b);
-      // item i < 2 n_steps: K (even i) or V (odd i) of step i/2; then the H'^T rows of
-      // the query blocks.  Item i lives in slot i % kSlots; the slot's previous item
-      // (i - kSlots, always a K/V item) is free once the P.V of its step has completed.
+      if (LINEAR) {
+        // the pre-slots complete their barriers' first phase: TMA for the states, a plain
+        // arrive for the phi(Q) slot (and for slot 1 when the pair has one query block)
+        for (int b = 0; b < 2; ++b) {
+          if (b < n_lin) {
+            mbar_arrive_expect_tx(&slot_full[b], L::kHsTile);
+            for (int c = 0; c < L::kChunks; ++c)
+              tma_load_3d(sRing + b * L::kKV + c * L::kHsChunk, &tmX1, &slot_full[b], c * 64, 0, bh * p.n_qb + 2 * pair + b);
+          } else {
+            mbar_arrive(&slot_full[b]);
+          }
+        }
+        mbar_arrive(&slot_full[2]);
+      }
+      // K/V item i: K (even i) or V (odd i) of step i/2, at ring position g = i + kPre
+      // (slot g % kSlots).  The slot's previous occupant is position g - kSlots: a K/V
+      // item, free once the P.V of its step has completed, or a pre-slot, free once the
+      // linear-branch MMAs have completed.
       int i = 0;
-      for (; i < n_items; ++i) {
-        const int slot = i % kSlots;
-        if (i >= kSlots) {
-          const int q = (i - kSlots) >> 1;
-          if (!mbar_wait(&pv_done[q & 3], (q >> 2) & 1, abort_flag, p.status)) break;
+      for (; i < 2 * n_steps; ++i) {
+        const int g = i + kPre, slot = g % kSlots;
+        if (g >= kSlots) {
+          bool freed;
+          if (LINEAR && g - kSlots < kPre) {
+            freed = mbar_wait(lin_done, 0, abort_flag, p.status);
+          } else {
+            const int q = (i - kSlots) >> 1;
+            freed = mbar_wait(&pv_done[q & 3], (q >> 2) & 1, abort_flag, p.status);
+          }
+          if (!freed) break;
         }
         uint8_t* dst0 = sRing + slot * L::kKV;
-        if (LINEAR && i >= 2 * n_steps) {
-          const int b = i - 2 * n_steps;
-          mbar_arrive_expect_tx(&slot_full[slot], L::kHsTile);
-          for (int c = 0; c < L::kChunks; ++c)
-            tma_load_3d(dst0 + c * L::kHsChunk, &tmX1, &slot_full[slot], c * 64, 0, bh * p.n_qb + 2 * pair + b);
-          continue;
-        }
         const int j = i >> 1;
         const bool is_v = i & 1;
         const int nb = step_blocks(j);
@@ -285,9 +301,9 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
         // let the loads already in flight land before the CTA's shared memory is released
         long long t0 = clock64();
         while (!mbar_try_wait(q_full, 0) && clock64() - t0 < kWaitBudgetCycles) {}
-        for (int it = (i - kSlots > 0 ? i - kSlots : 0); it < i; ++it) {
+        for (int g = (i + kPre - kSlots > 0 ? i + kPre - kSlots : 0); g < i + kPre; ++g) {
           t0 = clock64();
-          while (!mbar_try_wait(&slot_full[it % kSlots], (it / kSlots) & 1) && clock64() - t0 < kWaitBudgetCycles) {}
+          while (!mbar_try_wait(&slot_full[g % kSlots], (g / kSlots) & 1) && clock64() - t0 < kWaitBudgetCycles) {}
         }
       }
     }
@@ -315,70 +331,71 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
           mma_bf16_ts(tmem + col, a, b, idO, (acc || kk > 0) ? 1u : 0u);
         }
       };
+      // lin = phi(Q) [H'^T ; Z]^T per query block (lanes of the other block masked off)
+      // into the O columns, before any P.V; column D of the result is phi(q) . Z
+      auto issue_lin = [&]() {
+        constexpr uint32_t idH = idesc_bf16(128, D, false, false);
+        constexpr uint32_t idZ = idesc_bf16(128, 16, false, false);
+        const uint32_t z_addr = smem_u32(sZ), phq_addr = ring_addr + 2 * L::kKV;
+        const uint32_t lo_only[4] = {0u, 0u, 0xFFFFFFFFu, 0xFFFFFFFFu};   // write lanes 0-63
+        const uint32_t hi_only[4] = {0xFFFFFFFFu, 0xFFFFFFFFu, 0u, 0u};   // write lanes 64-127
+        for (int b = 0; b < n_lin; ++b) {
+          #pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const int c = kk >> 2, sub = kk & 3;
+            const uint64_t a = desc_kmajor(phq_addr + c * L::kTile + sub * 32);
+            const uint64_t bh_ = desc_kmajor(ring_addr + b * L::kKV + c * L::kHsChunk + sub * 32);
+            const uint64_t bz = desc_kmajor(z_addr + b * L::kZTile + c * L::kZChunk + sub * 32);
+            mma_bf16_ss_masked(tmem + kColLinOut, a, bh_, idH, kk > 0 ? 1u : 0u, b ? hi_only : lo_only);
+            mma_bf16_ss_masked(tmem + kColLinOut + D, a, bz, idZ, kk > 0 ? 1u : 0u, b ? hi_only : lo_only);
+          }
+        }
+        mma_commit(lin_done);
+      };
       bool ok = mbar_wait(q_full, 0, abort_flag, p.status);
       bool o1_started = false;
       if (ok && n_steps > 0) {
-        ok = mbar_wait(&slot_full[0], 0, abort_flag, p.status);
+        ok = mbar_wait(&slot_full[kPre % kSlots], (kPre / kSlots) & 1, abort_flag, p.status);
         if (ok) {
           tc_fence_after();
-          issue_qk(0, 0);
+          issue_qk(kPre % kSlots, 0);
           mma_commit(&s_full[0]);
         }
+      }
+      if (ok && LINEAR) {
+        ok = mbar_wait(phiq_ready, 0, abort_flag, p.status) && mbar_wait(&slot_full[0], 0, abort_flag, p.status) &&
+             mbar_wait(&slot_full[1], 0, abort_flag, p.status);
+        if (ok) {
+          tc_fence_after();
+          issue_lin();
+        }
+      }
+      if (ok && n_steps > 0) {
         for (int j = 0; j < n_steps && ok; ++j) {
           const int b = j & 1;
           if (j + 1 < n_steps) {
-            const int ik = 2 * (j + 1);
-            if (!mbar_wait(&slot_full[ik % kSlots], (ik / kSlots) & 1, abort_flag, p.status)) { ok = false; break; }
+            const int gk = 2 * (j + 1) + kPre;
+            if (!mbar_wait(&slot_full[gk % kSlots], (gk / kSlots) & 1, abort_flag, p.status)) { ok = false; break; }
             tc_fence_after();
-            issue_qk(ik % kSlots, (j + 1) & 1);
+            issue_qk(gk % kSlots, (j + 1) & 1);
             mma_commit(&s_full[(j + 1) & 1]);
           }
-          const int iv = 2 * j + 1;
-          if (!mbar_wait(&slot_full[iv % kSlots], (iv / kSlots) & 1, abort_flag, p.status) ||
+          const int gv = 2 * j + 1 + kPre;
+          if (!mbar_wait(&slot_full[gv % kSlots], (gv / kSlots) & 1, abort_flag, p.status) ||
               !mbar_wait(&p_full[b], (j >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
           tc_fence_after();
           const bool far = GATED && j == local_steps;
           if (far) {
             // the far-field output goes into the other S buffer (its step is done)
-            issue_pv(iv % kSlots, b, 0, kColS + (b ^ 1) * 128, false);
+            issue_pv(gv % kSlots, b, 0, kColS + (b ^ 1) * 128, false);
           } else {
-            issue_pv(iv % kSlots, b, 0, kColO0, j > 0);
+            issue_pv(gv % kSlots, b, 0, kColO0, j > 0);
             if (step_blocks(j) == 2) {
-              issue_pv(iv % kSlots, b, 1, kColO1, o1_started);
+              issue_pv(gv % kSlots, b, 1, kColO1, o1_started);
               o1_started = true;
             }
           }
           mma_commit(&pv_done[j & 3]);
-        }
-      }
-      if (ok && LINEAR) {
-        // lin = phi(Q) [H'^T ; Z]^T per query block (lanes of the other block masked off);
-        // column D of the result is the denominator phi(q) . Z
-        ok = mbar_wait(phiq_ready, 0, abort_flag, p.status);
-        for (int b = 0; b < n_lin && ok; ++b) {
-          const int it = 2 * n_steps + b;
-          ok = mbar_wait(&slot_full[it % kSlots], (it / kSlots) & 1, abort_flag, p.status);
-        }
-        if (ok) {
-          tc_fence_after();
-          constexpr uint32_t idH = idesc_bf16(128, D, false, false);
-          constexpr uint32_t idZ = idesc_bf16(128, 16, false, false);
-          const uint32_t z_addr = smem_u32(sZ);
-          const uint32_t lo_only[4] = {0u, 0u, 0xFFFFFFFFu, 0xFFFFFFFFu};   // write lanes 0-63
-          const uint32_t hi_only[4] = {0xFFFFFFFFu, 0xFFFFFFFFu, 0u, 0u};   // write lanes 64-127
-          for (int b = 0; b < n_lin; ++b) {
-            const int slot = (2 * n_steps + b) % kSlots;
-            #pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-              const int c = kk >> 2, sub = kk & 3;
-              const uint64_t a = desc_kmajor(q_addr + c * L::kTile + sub * 32);
-              const uint64_t bh_ = desc_kmajor(ring_addr + slot * L::kKV + c * L::kHsChunk + sub * 32);
-              const uint64_t bz = desc_kmajor(z_addr + b * L::kZTile + c * L::kZChunk + sub * 32);
-              mma_bf16_ss_masked(tmem + kColLin, a, bh_, idH, kk > 0 ? 1u : 0u, b ? hi_only : lo_only);
-              mma_bf16_ss_masked(tmem + kColLin + D, a, bz, idZ, kk > 0 ? 1u : 0u, b ? hi_only : lo_only);
-            }
-          }
-          mma_commit(lin_done);
         }
       }
       if (!ok) {
@@ -397,7 +414,70 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
     const float sl = p.scale_log2;
     float m_run = -INFINITY, l_run = 0.f, l_far = 0.f;
     bool ok = true, started = false;
-    for (int j = 0; j < n_steps; ++j) {
+    // ---- token of this row
+    int tok;
+    bool row_exists;
+    if (TILE) {
+      const int tile = 2 * pair + half;
+      row_exists = tile < p.n_qb;
+      int tf, th, tw;
+      tile_coords(tile, p.TF, p.TW, tf, th, tw);
+      const int rr = r & 63;
+      tok = ((tf * 4 + (rr >> 4)) * p.Hh + th * 4 + ((rr >> 2) & 3)) * p.Ww + tw * 4 + (rr & 3);
+    } else {
+      tok = pair * 128 + r;
+      row_exists = tok < p.n_pad;
+    }
+    const bool valid = row_exists && (TILE || token_valid(seq, tok));
+
+    // ---- linear branch first (LINEAR): phi(Q) into ring slot 2 (pad rows -> 0; Q stays in
+    // place for the QK MMAs), then the MMA warp's lin = phi(Q) [H'^T ; Z]^T lands in the O
+    // columns; my half of the row, divided by its denominator, is kept in registers as
+    // bf16 pairs (the output is rounded to bf16 in the end as well)
+    uint32_t lin[D / 4];
+    #pragma unroll
+    for (int i = 0; i < D / 4; ++i) lin[i] = 0u;
+    if (LINEAR) {
+      ok = __all_sync(0xFFFFFFFFu, mbar_wait(q_full, 0, abort_flag, p.status));
+      if (ok) {
+        uint8_t* sPhi = sRing + 2 * L::kKV;
+        constexpr int kGroups = D / 16;                  // 16-byte groups of my row handled by my warpgroup
+        #pragma unroll
+        for (int g = 0; g < kGroups; ++g) {
+          const int gg = wg * kGroups + g;               // 0 .. D/8-1
+          const int off = (gg >> 3) * L::kTile + sw128_offset(r, gg & 7);
+          const uint4 u = *reinterpret_cast<const uint4*>(sQ + off);
+          const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+          uint32_t o4[4];
+          #pragma unroll
+          for (int i = 0; i < 4; ++i)
+            o4[i] = valid ? pack_bf16(phi_fast(bf16_lo(w[i])), phi_fast(bf16_hi(w[i]))) : 0u;
+          *reinterpret_cast<uint4*>(sPhi + off) = make_uint4(o4[0], o4[1], o4[2], o4[3]);
+        }
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(phiq_ready);
+      if (ok) ok = __all_sync(0xFFFFFFFFu, mbar_wait(lin_done, 0, abort_flag, p.status));
+      tc_fence_after();
+      if (ok) {
+        uint32_t dv;
+        tmem_ld1(lane_addr + kColLinOut + D, dv);
+        tmem_wait_ld();
+        const float den = __uint_as_float(dv);
+        const float inv_den = den > 0.f ? 1.f / den : 0.f;
+        #pragma unroll
+        for (int k = 0; k < D / 64; ++k) {
+          uint32_t t[32];
+          tmem_ld32(lane_addr + kColLinOut + wg * (D / 2) + k * 32, t);
+          tmem_wait_ld();
+          #pragma unroll
+          for (int i = 0; i < 16; ++i)
+            lin[k * 16 + i] = pack_bf16(__uint_as_float(t[2 * i]) * inv_den, __uint_as_float(t[2 * i + 1]) * inv_den);
+        }
+      }
+      tc_fence_before();   // the first P.V overwrites these columns after p_full
+    }
+    for (int j = 0; j < n_steps && ok; ++j) {
       const int b = j & 1;
       const bool far = GATED && j == local_steps;
       const bool mine = wg == 0 || (!far && step_blocks(j) == 2);   // does this warpgroup own a block here
@@ -491,54 +571,10 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
       mbar_arrive(&p_full[b]);
       if (!far) started = true;
     }
-    // ---- token of this row
-    int tok;
-    bool row_exists;
-    if (TILE) {
-      const int tile = 2 * pair + half;
-      row_exists = tile < p.n_qb;
-      int tf, th, tw;
-      tile_coords(tile, p.TF, p.TW, tf, th, tw);
-      const int rr = r & 63;
-      tok = ((tf * 4 + (rr >> 4)) * p.Hh + th * 4 + ((rr >> 2) & 3)) * p.Ww + tw * 4 + (rr & 3);
-    } else {
-      tok = pair * 128 + r;
-      row_exists = tok < p.n_pad;
-    }
-    const bool valid = row_exists && (TILE || token_valid(seq, tok));
-
-    bool lin_ok = false;
-    if (LINEAR) {
-      // phi(Q) in place: every QK MMA has completed (the last step's S was seen; with no
-      // step at all, Q has landed once q_full completes); pad rows -> 0
-      ok = __all_sync(0xFFFFFFFFu, ok);
-      if (ok && n_steps == 0) ok = __all_sync(0xFFFFFFFFu, mbar_wait(q_full, 0, abort_flag, p.status));
-      if (ok) {
-        constexpr int kGroups = D / 16;                  // 16-byte groups of my row handled by my warpgroup
-        #pragma unroll
-        for (int g = 0; g < kGroups; ++g) {
-          const int gg = wg * kGroups + g;               // 0 .. D/8-1
-          uint4* ptr = reinterpret_cast<uint4*>(sQ + (gg >> 3) * L::kTile + sw128_offset(r, gg & 7));
-          const uint4 u = *ptr;
-          const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-          uint32_t o4[4];
-          #pragma unroll
-          for (int i = 0; i < 4; ++i)
-            o4[i] = valid ? pack_bf16(phi_fast(bf16_lo(w[i])), phi_fast(bf16_hi(w[i]))) : 0u;
-          *ptr = make_uint4(o4[0], o4[1], o4[2], o4[3]);
-        }
-      }
-      fence_proxy_async_smem();
-      mbar_arrive(phiq_ready);
-    }
     if (ok && n_steps > 0)
       ok = __all_sync(0xFFFFFFFFu, mbar_wait(&pv_done[(n_steps - 1) & 3], ((n_steps - 1) >> 2) & 1, abort_flag, p.status));
     ok = __all_sync(0xFFFFFFFFu, ok);
     tc_fence_after();
-    if (LINEAR) {
-      if (ok) lin_ok = __all_sync(0xFFFFFFFFu, mbar_wait(lin_done, 0, abort_flag, p.status));
-      tc_fence_after();
-    }
 
     // ---- merge the two shares
     xch[wg * 128 + r] = m_run;
@@ -559,19 +595,12 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
       inv_far = lf > 0.f ? 1.f / lf : 0.f;
       col_far = kColS + ((local_steps & 1) ^ 1) * 128;
     }
-    float inv_den = 0.f;
-    if (LINEAR && lin_ok) {
-      uint32_t dv;
-      tmem_ld1(lane_addr + kColLin + D, dv);
-      tmem_wait_ld();
-      const float den = __uint_as_float(dv);
-      inv_den = den > 0.f ? 1.f / den : 0.f;
-    }
     const bool have_o0 = ok && n_local > 0;        // CTA-uniform
     const bool have_o1 = ok && n_local > 1;
     const size_t row_off = ((size_t)bh * p.n_pad + (row_exists ? tok : 0)) * D;
-    #pragma unroll 1
-    for (int cc = wg * (D / 64); cc < (wg + 1) * (D / 64); ++cc) {
+    #pragma unroll
+    for (int k = 0; k < D / 64; ++k) {
+      const int cc = wg * (D / 64) + k;          // my 32-column chunks
       float v[32];
       #pragma unroll
       for (int i = 0; i < 32; ++i) v[i] = 0.f;
@@ -596,12 +625,12 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
         #pragma unroll
         for (int i = 0; i < 32; ++i) v[i] = p.gate * v[i] + (1.f - p.gate) * (__uint_as_float(of[i]) * inv_far);
       }
-      if (LINEAR && lin_ok) {
-        uint32_t ol[32];
-        tmem_ld32(lane_addr + kColLin + cc * 32, ol);
-        tmem_wait_ld();
+      if (LINEAR) {
         #pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] += __uint_as_float(ol[i]) * inv_den;
+        for (int i = 0; i < 16; ++i) {
+          v[2 * i] += bf16_lo(lin[k * 16 + i]);
+          v[2 * i + 1] += bf16_hi(lin[k * 16 + i]);
+        }
       }
       if (!row_exists) continue;
       uint4* dst = reinterpret_cast<uint4*>(p.out + row_off + cc * 32);
