@@ -30,6 +30,7 @@ import math
 import os
 import statistics
 import subprocess
+import tempfile
 import sys
 import time
 
@@ -87,7 +88,7 @@ def config_dict(w):
 
 
 def sla_flops(w, kc, kn):
-    """Algorithmic FLOPs of one call on computed blocks (the SURVEY's count)."""
+    """Algorithmic FLOPs of one call on computed blocks."""
     nb = w.n_blocks
     BH = w.batch * w.heads
     d = w.d
@@ -109,11 +110,13 @@ class ClockSampler:
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{gpu_index}.csv")
+        # the raw samples go to $SLR_CLOCKS_CSV when set, else to the temp directory
+        self.path = os.environ.get("SLR_CLOCKS_CSV") or os.path.join(tempfile.gettempdir(),
+                                                                      f"slr_clocks_rank{gpu_index}.csv")
 
     def start(self):
         try:
-            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            os.makedirs(os.path.dirname(os.path.abspath(self.path)), exist_ok=True)
             self.f = open(self.path, "w")
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
                                           "--format=csv,noheader,nounits", "-lms", "200"],

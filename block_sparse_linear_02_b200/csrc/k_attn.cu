@@ -1,9 +1,9 @@
 // k_attn.cu -- block-sparse flash attention on tcgen05 (sm_100a).
 //
 // Computes, for every 64-token query block i, exact softmax attention over the
-// valid keys of a set of 64-token key blocks (SLA page section 3, critical
-// branch: "精确的稀疏FlashAttention"; the LVSA page's step-6 formula is the same
-// normalised sum).  Two fused epilogues:
+// valid keys of a set of 64-token key blocks (SLA page section 3, the critical
+// branch, which runs block-sparse FlashAttention; the LVSA page's step-6 formula
+// is the same normalised sum).  Two fused epilogues:
 //   LINEAR  (SLA): the linear-attention branch of the same query block is added,
 //           O = O_s + phi(Q_i) H_i' / (phi(Q_i) . Z_i) with H_i' = sum of
 //           phi(K_j)^T V_j W_proj over its marginal blocks -- one more MMA of

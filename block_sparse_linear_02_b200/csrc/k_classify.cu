@@ -1,22 +1,28 @@
-// k_classify.cu -- SLA's compressed scores and percentile classification.
+// k_classify.cu -- SLA's compressed scores, percentile classification and the
+// critical pair lists.
 //
 // SLA page section 3: the pooled Q and K give a compressed attention-weight
 // matrix P_c = softmax(pool(Q) pool(K)^T / sqrt(d)); within each query-block row
 // the top 5 % positions are labelled critical (1), the bottom 10 % negligible
 // (-1), the rest marginal (0).  Softmax is strictly increasing along a row, so
-// the labels are taken on the fp64 logits; ties rank the lower key-block index
-// first.  Both the logits and the selection are fp64 so that the labels agree
-// with an fp64 evaluation of the same definition.
+// the labels are taken on the logits qbar_i . kbar_j; ties rank the lower
+// key-block index first.
 //
-// block_logits_kernel: 64x64 output tiles of qbar kbar^T on the fp64 tensor cores.
-// classify_rows_kernel: one warp per row; two MSB-first radix selections over
-//   order-preserving 64-bit keys (8-bit digits, warp-aggregated histogram
-//   counts, stopping once the remaining candidates are exactly the ones
-//   needed) find the kc-th largest and kn-th smallest key; one pass in index
-//   order applies the
-//   thresholds with index tie-breaking and emits the mask row, the ascending
-//   critical list, the marginal indicator row (bf16 1/0 for the tensor-core
-//   contraction) and, on request, P_c in fp32.
+// logits_kernel: one CTA per 128 x 128 tile of one head's logit matrix on the
+//   tensor cores.  The pooling kernel writes each mean as a bf16 pair hi + lo,
+//   query rows as [qh | qh | ql] and key rows as [kh | kl | kh], so one bf16
+//   GEMM over K = 3d with fp32 accumulation gives qh.kh + qh.kl + ql.kh: the
+//   logit up to the ql.kl term, about 2^-16 of it.  The tile is stored as
+//   order-preserving 32-bit keys (pad columns 0).
+// classify_kernel: one warp per pair of query blocks.  For both rows, the kc-th
+//   largest and the kn-th smallest key by bisection (one comparison per key and
+//   one warp sum per bit); then one pass in index order applies the thresholds
+//   with index tie-breaking and writes what the caller asked for: the mask row,
+//   the ascending critical list, the marginal indicator m01 (bf16 1/0, the
+//   operand of the tensor-core contraction), P_c in fp32, and the pair's union
+//   list for the attention kernel.
+// Against an exact evaluation the logits' error moves P_c by ~1e-8, so a label
+// can differ only for a pair whose score is that close to its row's threshold.
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 #include <math.h>
@@ -27,208 +33,245 @@
 namespace slr {
 namespace {
 
-// dots[bh][i][j] = qbar_i . kbar_j in fp64 on the fp64 tensor cores
-// (mma.m8n8k4.f64): one CTA = 4 warps computes a 64x64 tile, each warp a 32x32
-// quarter as 4x4 fragments of 8x8.  The ranking of a row does not depend on the
-// positive scale 1/sqrt(d), so the kernel stores the plain dot products.
-__device__ __forceinline__ void dmma_8x8x4(double (&d)[2], double a, double b) {
-  asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0, %1}, {%2}, {%3}, {%0, %1};"
-               : "+d"(d[0]), "+d"(d[1]) : "d"(a), "d"(b));
+// Order-preserving map of an fp32 value onto uint32 (larger value -> larger key);
+// -0 is folded onto +0 so that equal values give equal keys.  A finite value
+// never maps to 0, which marks padding.
+__device__ __forceinline__ uint32_t okey(float x) {
+  if (x == 0.f) x = 0.f;
+  const uint32_t b = __float_as_uint(x);
+  return (b >> 31) ? ~b : (b | 0x80000000u);
+}
+__device__ __forceinline__ float okey_value(uint32_t k) {
+  return __uint_as_float((k >> 31) ? (k & 0x7FFFFFFFu) : ~k);
 }
 
-__global__ void __launch_bounds__(128)
-block_logits_kernel(const double* __restrict__ qbar, const double* __restrict__ kbar,
-                    double* __restrict__ dots, int nb, int d) {
-  __shared__ double As[64][36];
-  __shared__ double Bs[64][36];
-  const int bh = blockIdx.z;
-  const int i0 = blockIdx.y * 64, j0 = blockIdx.x * 64;
-  const double* A = qbar + (size_t)bh * nb * d;
-  const double* B = kbar + (size_t)bh * nb * d;
+__device__ __forceinline__ int warp_sum(int v) { return (int)__reduce_add_sync(0xFFFFFFFFu, (unsigned)v); }
+
+// ------------------------------------------------------------------ logits GEMM
+template <int D>
+struct LgLayout {
+  static constexpr int kChunks = 3 * D / 64;          // K = 3d in chunks of 64
+  static constexpr int kTile = 128 * 128;             // 128 rows x 64 bf16
+  static constexpr int kBOff = kChunks * kTile;
+  static constexpr int kBarOff = 2 * kChunks * kTile;
+  static constexpr int kBytes = kBarOff + 256 + 1024; // + alignment slack
+};
+
+template <int D>
+__global__ void __launch_bounds__(128, 1)
+logits_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+              uint32_t* __restrict__ keys, int nb, int nbp, int* status) {
+  using L = LgLayout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBarOff);   // [kChunks]
+  uint64_t* done = full + L::kChunks;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  const int n0 = blockIdx.x * 128, m0 = blockIdx.y * 128, bh = blockIdx.z;
+  const int warp = threadIdx.x >> 5;
+  if (threadIdx.x == 0) {
+    for (int c = 0; c < L::kChunks; ++c) mbar_init(&full[c], 1);
+    mbar_init(done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) { tmem_alloc(tmem_slot, 128); tmem_relinquish(); }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (threadIdx.x == 0) {
+    for (int c = 0; c < L::kChunks; ++c) {
+      mbar_arrive_expect_tx(&full[c], 2 * L::kTile);
+      tma_load_3d(smem + c * L::kTile, &tmA, &full[c], c * 64, m0, bh);
+      tma_load_3d(smem + L::kBOff + c * L::kTile, &tmB, &full[c], c * 64, n0, bh);
+    }
+    constexpr uint32_t id = idesc_bf16(128, 128, false, false);
+    bool ok = true;
+    for (int c = 0; c < L::kChunks && ok; ++c) {
+      ok = mbar_wait(&full[c], 0, abort_flag, status);
+      if (!ok) break;
+      tc_fence_after();
+      #pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        const uint64_t a = desc_kmajor(smem_u32(smem + c * L::kTile) + kk * 32);
+        const uint64_t b = desc_kmajor(smem_u32(smem + L::kBOff + c * L::kTile) + kk * 32);
+        mma_bf16_ss(tmem, a, b, id, (c > 0 || kk > 0) ? 1u : 0u);
+      }
+    }
+    mma_commit(done);   // also when aborting: the MMAs already issued complete before the CTA exits
+    if (!ok) {
+      // let the loads in flight land before the shared memory is released
+      for (int c = 0; c < L::kChunks; ++c) {
+        const long long t0 = clock64();
+        while (!mbar_try_wait(&full[c], 0) && clock64() - t0 < kWaitBudgetCycles) {}
+      }
+    }
+  }
+  const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(done, 0, abort_flag, status)) && !*abort_flag;
+  tc_fence_after();
+  const int m = m0 + threadIdx.x;          // my row = my TMEM lane
+  if (ok) {                                // warp-uniform: the TMEM loads are warp-collective
+    uint32_t* dst = keys + ((size_t)bh * nb + (m < nb ? m : 0)) * nbp + n0;
+    #pragma unroll 1
+    for (int cc = 0; cc < 4; ++cc) {
+      uint32_t v[32];
+      tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + cc * 32, v);
+      tmem_wait_ld();
+      if (m >= nb) continue;
+      #pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] = n0 + cc * 32 + i < nb ? okey(__uint_as_float(v[i])) : 0u;
+      uint4* d4 = reinterpret_cast<uint4*>(dst + cc * 32);
+      #pragma unroll
+      for (int i = 0; i < 8; ++i) d4[i] = make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) { tc_fence_after(); tmem_dealloc(tmem, 128); }
+}
+
+// ------------------------------------------------------------------ classification
+struct ClsArgs {
+  const uint32_t* keys;    // [BH][nb][nbp] order keys of the logits, pads 0
+  int nb, nbp, kc, kn, n_pairs;
+  float inv_sqrt_d;
+  int8_t* mask;
+  int32_t* crit_idx;
+  int32_t* crit_cnt;
+  __nv_bfloat16* m01;
+  int ld_m01;
+  float* scores;
+  uint32_t* list;
+  int32_t* list_cnt;
+  int list_cap;
+  SeqShape s;
+  int* status;
+};
+
+constexpr int kClsWarps = 4;
+
+__global__ void __launch_bounds__(kClsWarps * 32)
+classify_kernel(const ClsArgs a) {
+  extern __shared__ __align__(16) uint32_t skeys[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int wy = warp >> 1, wx = warp & 1;
-  double acc[4][4][2];
-  #pragma unroll
-  for (int a = 0; a < 4; ++a)
-    #pragma unroll
-    for (int b = 0; b < 4; ++b) acc[a][b][0] = acc[a][b][1] = 0.0;
-  for (int c0 = 0; c0 < d; c0 += 32) {
-    for (int e = threadIdx.x; e < 64 * 32; e += 128) {
-      const int row = e >> 5, col = e & 31;
-      As[row][col] = (i0 + row < nb) ? A[(size_t)(i0 + row) * d + c0 + col] : 0.0;
-      Bs[row][col] = (j0 + row < nb) ? B[(size_t)(j0 + row) * d + c0 + col] : 0.0;
-    }
-    __syncthreads();
-    #pragma unroll
-    for (int kk = 0; kk < 32; kk += 4) {
-      double af[4], bf[4];
-      #pragma unroll
-      for (int t = 0; t < 4; ++t) {
-        af[t] = As[wy * 32 + t * 8 + (lane >> 2)][kk + (lane & 3)];
-        bf[t] = Bs[wx * 32 + t * 8 + (lane >> 2)][kk + (lane & 3)];
-      }
-      #pragma unroll
-      for (int mt = 0; mt < 4; ++mt)
-        #pragma unroll
-        for (int nt = 0; nt < 4; ++nt) dmma_8x8x4(acc[mt][nt], af[mt], bf[nt]);
-    }
-    __syncthreads();
-  }
-  #pragma unroll
-  for (int mt = 0; mt < 4; ++mt) {
-    const int i = i0 + wy * 32 + mt * 8 + (lane >> 2);
-    if (i >= nb) continue;
-    #pragma unroll
-    for (int nt = 0; nt < 4; ++nt) {
-      const int j = j0 + wx * 32 + nt * 8 + 2 * (lane & 3);
-      double* dst = dots + ((size_t)bh * nb + i) * nb + j;
-      if (j < nb) dst[0] = acc[mt][nt][0];
-      if (j + 1 < nb) dst[1] = acc[mt][nt][1];
-    }
-  }
-}
-
-// Order-preserving map of an fp64 value onto uint64 (larger value -> larger key);
-// -0 is folded onto +0 so that equal values give equal keys.
-__device__ __forceinline__ uint64_t order_key(double x) {
-  if (x == 0.0) x = 0.0;
-  const uint64_t b = (uint64_t)__double_as_longlong(x);
-  return (b >> 63) ? ~b : (b | 0x8000000000000000ull);
-}
-
-__device__ __forceinline__ int warp_incl_scan(int v, int lane) {
-  #pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int y = __shfl_up_sync(0xFFFFFFFFu, v, o);
-    if (lane >= o) v += y;
-  }
-  return v;
-}
-
-// MSB-first radix selection of the k-th largest (largest=true) or k-th smallest
-// key among keys[0..n), 8 bits per pass.  Returns the selection at the level
-// `shift` where it was settled: T (the key's bits above `shift`), how many of
-// the keys whose bits above `shift` equal T are taken (take), and how many such
-// keys there are (eq_total).  The passes stop early once every remaining
-// candidate is needed.
-__device__ void radix_select(const uint64_t* keys, int n, int k, bool largest, unsigned* hist, int lane,
-                             uint64_t& T, int& shift_out, int& take, int& eq_total) {
-  uint64_t prefix = 0, pmask = 0;
-  int kk = k, last = 0, shift = 56;
-  for (;; shift -= 8) {
-    for (int b = lane; b < 256; b += 32) hist[b] = 0;
-    __syncwarp();
-    for (int j0 = 0; j0 < n; j0 += 32) {
-      const int j = j0 + lane;
-      const uint64_t u = j < n ? keys[j] : 0;
-      const bool cand = j < n && (u & pmask) == prefix;
-      const unsigned bin = (unsigned)((u >> shift) & 255);
-      const unsigned act = __ballot_sync(0xFFFFFFFFu, cand);
-      if (cand) {
-        const unsigned peers = __match_any_sync(act, bin);
-        if ((__ffs(peers) - 1) == lane) atomicAdd(&hist[bin], (unsigned)__popc(peers));
-      }
-    }
-    __syncwarp();
-    int cnt[8], lsum = 0;
-    #pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      const int bin = largest ? 255 - (lane * 8 + q) : lane * 8 + q;
-      cnt[q] = (int)hist[bin];
-      lsum += cnt[q];
-    }
-    const int incl = warp_incl_scan(lsum, lane);
-    const int excl = incl - lsum;
-    const bool has = excl < kk && incl >= kk;
-    const unsigned bal = __ballot_sync(0xFFFFFFFFu, has);
-    const int src = __ffs(bal) - 1;
-    int sel = 0, before = 0;
-    if (lane == src) {
-      int acc = excl;
-      #pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        if (acc + cnt[q] >= kk) { sel = largest ? 255 - (lane * 8 + q) : lane * 8 + q; before = acc; break; }
-        acc += cnt[q];
-      }
-    }
-    sel = __shfl_sync(0xFFFFFFFFu, sel, src);
-    before = __shfl_sync(0xFFFFFFFFu, before, src);
-    kk -= before;
-    last = (int)hist[sel];
-    prefix |= (uint64_t)sel << shift;
-    pmask |= (uint64_t)0xFF << shift;
-    __syncwarp();
-    if (last == kk || shift == 0) break;      // every remaining candidate is needed, or fully resolved
-  }
-  T = prefix >> shift;
-  shift_out = shift;
-  take = kk;
-  eq_total = last;
-}
-
-constexpr int kRowsPerCta = 4;
-
-__global__ void __launch_bounds__(128)
-classify_rows_kernel(const double* __restrict__ logits, int rows, int nb, int kc, int kn,
-                     int8_t* __restrict__ mask, int32_t* __restrict__ crit_idx, int32_t* __restrict__ crit_cnt,
-                     __nv_bfloat16* __restrict__ m01, int ld_m01, float* __restrict__ scores, double sqrt_d) {
-  extern __shared__ uint8_t smem[];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  uint64_t* keys = reinterpret_cast<uint64_t*>(smem) + (size_t)warp * nb;
-  unsigned* hist = reinterpret_cast<unsigned*>(reinterpret_cast<uint64_t*>(smem) + (size_t)kRowsPerCta * nb) + warp * 256;
-  const int row = blockIdx.x * kRowsPerCta + warp;
-  if (row >= rows) return;
-  const double* lg = logits + (size_t)row * nb;
-  double mx = -INFINITY;
-  for (int j = lane; j < nb; j += 32) {
-    const double x = lg[j];
-    keys[j] = order_key(x);
-    mx = fmax(mx, x);
-  }
-  #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) mx = fmax(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
-  double sum = 0.0;
-  if (scores) {
-    for (int j = lane; j < nb; j += 32) sum += exp(lg[j] / sqrt_d - mx / sqrt_d);
-    #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
+  const int bh = blockIdx.y, pair = blockIdx.x * kClsWarps + warp;
+  const int nb = a.nb, nbp = a.nbp;
+  const int qb0 = 2 * pair;
+  if (qb0 >= nb) return;
+  const int nrows = qb0 + 1 < nb ? 2 : 1;
+  uint32_t* rowk[2] = {skeys + (size_t)(2 * warp) * nbp, skeys + (size_t)(2 * warp + 1) * nbp};
+  for (int r = 0; r < nrows; ++r) {
+    const uint4* src = reinterpret_cast<const uint4*>(a.keys + ((size_t)bh * nb + qb0 + r) * nbp);
+    for (int e = lane; e < nbp / 4; e += 32) reinterpret_cast<uint4*>(rowk[r])[e] = src[e];
   }
   __syncwarp();
-  uint64_t Tc = 0, Tn = 0;
-  int sc = 0, sn = 0, take_c = 0, eq_c = 0, take_n = 0, eq_n = 0;
-  radix_select(keys, nb, kc, true, hist, lane, Tc, sc, take_c, eq_c);
-  if (kn > 0) radix_select(keys, nb, kn, false, hist, lane, Tn, sn, take_n, eq_n);
-  const unsigned lt_mask = (1u << lane) - 1u;
-  int seen_c = 0, seen_n = 0, written = 0;
-  for (int base = 0; base < nb; base += 32) {
-    const int j = base + lane;
-    const bool in = j < nb;
-    const uint64_t u = in ? keys[j] : 0;
-    const uint64_t uc = u >> sc, un = u >> sn;
-    const bool eqc = in && uc == Tc;
-    const unsigned bc = __ballot_sync(0xFFFFFFFFu, eqc);
-    const bool crit = (in && uc > Tc) || (eqc && seen_c + __popc(bc & lt_mask) < take_c);
-    seen_c += __popc(bc);
-    bool negl = false;
-    if (kn > 0) {
-      const bool eqn = in && un == Tn;
-      const unsigned bn = __ballot_sync(0xFFFFFFFFu, eqn);
-      negl = (in && un < Tn) || (eqn && seen_n + __popc(bn & lt_mask) >= eq_n - take_n);
-      seen_n += __popc(bn);
+  const int npad = nbp - nb;
+
+  // ---- thresholds: Tc = kc-th largest key, Tn = kn-th smallest
+  uint32_t Tc[2] = {0u, 0u}, Tn[2] = {0xFFFFFFFFu, 0xFFFFFFFFu};
+  for (int bit = 31; bit >= 0; --bit) {
+    #pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      if (r >= nrows) break;                      // warp-uniform
+      const uint32_t cc = Tc[r] | (1u << bit), cn = Tn[r] & ~(1u << bit);
+      int nc = 0, nn = 0;
+      for (int j = lane * 4; j < nbp; j += 128) {
+        const uint4 k4 = *reinterpret_cast<const uint4*>(rowk[r] + j);
+        nc += (k4.x >= cc) + (k4.y >= cc) + (k4.z >= cc) + (k4.w >= cc);
+        nn += (k4.x <= cn) + (k4.y <= cn) + (k4.z <= cn) + (k4.w <= cn);
+      }
+      if (warp_sum(nc) >= a.kc) Tc[r] = cc;
+      if (warp_sum(nn) - npad >= a.kn) Tn[r] = cn;   // pads (key 0) always count as <=
     }
-    if (in) {
-      const int8_t m = crit ? 1 : (negl ? -1 : 0);
-      mask[(size_t)row * nb + j] = m;
-      if (m01) m01[(size_t)row * ld_m01 + j] = __float2bfloat16_rn(m == 0 ? 1.f : 0.f);
-      if (scores) scores[(size_t)row * nb + j] = (float)(exp(lg[j] / sqrt_d - mx / sqrt_d) / sum);
-    }
-    const unsigned bcrit = __ballot_sync(0xFFFFFFFFu, crit);
-    if (crit) crit_idx[(size_t)row * kc + written + __popc(bcrit & lt_mask)] = j;
-    written += __popc(bcrit);
   }
-  if (m01)
-    for (int j = nb + lane; j < ld_m01; j += 32) m01[(size_t)row * ld_m01 + j] = __float2bfloat16_rn(0.f);
-  if (lane == 0) crit_cnt[row] = kc;
+  // keys above the critical threshold, below the negligible one, equal to it; the row max
+  int gt_c[2] = {0, 0}, lt_n[2] = {0, 0}, eq_n[2] = {0, 0};
+  float row_max[2] = {0.f, 0.f}, row_sum[2] = {1.f, 1.f};
+  #pragma unroll
+  for (int r = 0; r < 2; ++r) {
+    if (r >= nrows) break;
+    uint32_t kmax = 0u;
+    for (int j = lane * 4; j < nbp; j += 128) {
+      const uint4 k4 = *reinterpret_cast<const uint4*>(rowk[r] + j);
+      const uint32_t kk[4] = {k4.x, k4.y, k4.z, k4.w};
+      #pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        gt_c[r] += kk[i] > Tc[r];
+        lt_n[r] += kk[i] != 0u && kk[i] < Tn[r];
+        eq_n[r] += kk[i] == Tn[r];
+        kmax = kk[i] > kmax ? kk[i] : kmax;
+      }
+    }
+    gt_c[r] = warp_sum(gt_c[r]);
+    lt_n[r] = warp_sum(lt_n[r]);
+    eq_n[r] = warp_sum(eq_n[r]);
+    row_max[r] = okey_value(__reduce_max_sync(0xFFFFFFFFu, kmax));
+    if (a.scores) {
+      float sum = 0.f;
+      for (int j = lane; j < nb; j += 32) sum += expf((okey_value(rowk[r][j]) - row_max[r]) * a.inv_sqrt_d);
+      #pragma unroll
+      for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
+      row_sum[r] = sum;
+    }
+  }
+
+  // ---- labels in index order and the outputs
+  const unsigned lt_mask = (1u << lane) - 1u;
+  int seen_c[2] = {0, 0}, seen_n[2] = {0, 0}, written[2] = {0, 0}, listed = 0;
+  uint32_t* lst = a.list ? a.list + ((size_t)bh * a.n_pairs + pair) * a.list_cap : nullptr;
+  for (int j0 = 0; j0 < nb; j0 += 32) {
+    const int j = j0 + lane;
+    const bool in = j < nb;
+    bool crit[2] = {false, false};
+    #pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      if (r >= nrows) break;
+      const uint32_t k = in ? rowk[r][j] : 0u;
+      const bool eqc = in && k == Tc[r];
+      const unsigned bc = __ballot_sync(0xFFFFFFFFu, eqc);
+      crit[r] = (in && k > Tc[r]) || (eqc && seen_c[r] + __popc(bc & lt_mask) < a.kc - gt_c[r]);
+      seen_c[r] += __popc(bc);
+      bool negl = false;
+      if (a.kn > 0) {
+        const bool eqn = in && k == Tn[r];
+        const unsigned bn = __ballot_sync(0xFFFFFFFFu, eqn);
+        negl = (in && k < Tn[r]) || (eqn && seen_n[r] + __popc(bn & lt_mask) >= eq_n[r] - (a.kn - lt_n[r]));
+        seen_n[r] += __popc(bn);
+      }
+      const size_t row = (size_t)bh * nb + qb0 + r;
+      if (in) {
+        const int8_t m = crit[r] ? 1 : (negl ? -1 : 0);
+        if (a.mask) a.mask[row * nb + j] = m;
+        if (a.m01) a.m01[row * a.ld_m01 + j] = __float2bfloat16_rn(m == 0 ? 1.f : 0.f);
+        if (a.scores) a.scores[row * nb + j] = expf((okey_value(k) - row_max[r]) * a.inv_sqrt_d) / row_sum[r];
+      }
+      const unsigned bcrit = __ballot_sync(0xFFFFFFFFu, crit[r]);
+      if (a.crit_idx && crit[r]) a.crit_idx[row * a.kc + written[r] + __popc(bcrit & lt_mask)] = j;
+      written[r] += __popc(bcrit);
+    }
+    if (lst) {
+      const bool u = crit[0] || crit[1];
+      const unsigned bu = __ballot_sync(0xFFFFFFFFu, u);
+      const int pos = listed + __popc(bu & lt_mask);
+      if (u && pos < a.list_cap)
+        lst[pos] = (uint32_t)j | ((uint32_t)block_valid_count(a.s, j) << 16) | ((uint32_t)crit[0] << 30) |
+                   ((uint32_t)crit[1] << 31);
+      listed += __popc(bu);
+    }
+  }
+  for (int r = 0; r < nrows; ++r) {
+    const size_t row = (size_t)bh * nb + qb0 + r;
+    if (a.m01)
+      for (int j = nb + lane; j < a.ld_m01; j += 32) a.m01[row * a.ld_m01 + j] = __float2bfloat16_rn(0.f);
+    if (lane == 0 && a.crit_cnt) a.crit_cnt[row] = a.kc;
+  }
+  if (lst && lane == 0) {
+    if (listed > a.list_cap) { atomicCAS(a.status, 0, kErrIndex); listed = a.list_cap; }
+    a.list_cnt[(size_t)bh * a.n_pairs + pair] = listed;
+  }
 }
 
 __global__ void mask_to_m01_kernel(const int8_t* __restrict__ mask, __nv_bfloat16* __restrict__ m01,
@@ -242,24 +285,54 @@ __global__ void mask_to_m01_kernel(const int8_t* __restrict__ mask, __nv_bfloat1
   }
 }
 
-}  // namespace
-
-cudaError_t launch_block_logits(const double* qbar, const double* kbar, double* logits,
-                                int BH, int nb, int d, cudaStream_t st) {
-  dim3 grid((nb + 63) / 64, (nb + 63) / 64, BH);
-  block_logits_kernel<<<grid, 128, 0, st>>>(qbar, kbar, logits, nb, d);
+template <int D>
+cudaError_t launch_logits_d(const void* qsplit, const void* ksplit, uint32_t* keys, int BH, int nb, int nbp,
+                            int* status, cudaStream_t st) {
+  using L = LgLayout<D>;
+  CUtensorMap ma, mb;
+  const uint64_t dims[3] = {(uint64_t)(3 * D), (uint64_t)nb, (uint64_t)BH};
+  const uint64_t strides[2] = {(uint64_t)(3 * D) * 2, (uint64_t)(3 * D) * 2 * nb};
+  const uint32_t box[3] = {64, 128, 1};
+  if (!make_tile_map(&ma, qsplit, 3, dims, strides, box)) return cudaErrorInvalidValue;
+  if (!make_tile_map(&mb, ksplit, 3, dims, strides, box)) return cudaErrorInvalidValue;
+  static unsigned long long attr_set = 0;        // one bit per device
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 64 || !(attr_set & (1ull << dev))) {
+    cudaError_t e = cudaFuncSetAttribute(logits_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes);
+    if (e != cudaSuccess) return e;
+    if (dev < 64) attr_set |= 1ull << dev;
+  }
+  dim3 grid(nbp / 128, nbp / 128, BH);
+  logits_kernel<D><<<grid, 128, L::kBytes, st>>>(ma, mb, keys, nb, nbp, status);
   return cudaGetLastError();
 }
 
-cudaError_t launch_classify_rows(const double* logits, int BH, int nb, int d, int kc, int kn,
-                                 int8_t* mask, int32_t* crit_idx, int32_t* crit_cnt,
-                                 __nv_bfloat16* m01, int ld_m01, float* scores, cudaStream_t st) {
-  const int rows = BH * nb;
-  const size_t smem = (size_t)kRowsPerCta * nb * sizeof(uint64_t) + (size_t)kRowsPerCta * 256 * sizeof(unsigned);
-  cudaError_t e = cudaFuncSetAttribute(classify_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+}  // namespace
+
+int logits_row_stride(int nb) { return (nb + 127) / 128 * 128; }
+
+cudaError_t launch_logits(const void* qsplit, const void* ksplit, uint32_t* keys, int BH, int nb, int d,
+                          int* status, cudaStream_t st) {
+  const int nbp = logits_row_stride(nb);
+  return d == 128 ? launch_logits_d<128>(qsplit, ksplit, keys, BH, nb, nbp, status, st)
+                  : launch_logits_d<64>(qsplit, ksplit, keys, BH, nb, nbp, status, st);
+}
+
+cudaError_t launch_classify(const uint32_t* keys, int BH, int nb, int d, int kc, int kn,
+                            int8_t* mask, int32_t* crit_idx, int32_t* crit_cnt, __nv_bfloat16* m01, int ld_m01,
+                            float* scores, uint32_t* list, int32_t* list_cnt, int list_cap, SeqShape s,
+                            int* status, cudaStream_t st) {
+  ClsArgs a;
+  a.keys = keys; a.nb = nb; a.nbp = logits_row_stride(nb); a.kc = kc; a.kn = kn; a.n_pairs = (nb + 1) / 2;
+  a.inv_sqrt_d = (float)(1.0 / sqrt((double)d));
+  a.mask = mask; a.crit_idx = crit_idx; a.crit_cnt = crit_cnt; a.m01 = m01; a.ld_m01 = ld_m01;
+  a.scores = scores; a.list = list; a.list_cnt = list_cnt; a.list_cap = list_cap; a.s = s; a.status = status;
+  const size_t smem = (size_t)2 * kClsWarps * a.nbp * sizeof(uint32_t);
+  cudaError_t e = cudaFuncSetAttribute(classify_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  classify_rows_kernel<<<(rows + kRowsPerCta - 1) / kRowsPerCta, 128, smem, st>>>(
-      logits, rows, nb, kc, kn, mask, crit_idx, crit_cnt, m01, ld_m01, scores, sqrt((double)d));
+  dim3 grid((a.n_pairs + kClsWarps - 1) / kClsWarps, BH);
+  classify_kernel<<<grid, kClsWarps * 32, smem, st>>>(a);
   return cudaGetLastError();
 }
 

@@ -1,8 +1,8 @@
 // k_marginal.cu -- the linear-attention branch of SLA on tcgen05 (sm_100a).
 //
-// SLA page section 3 ("边缘权重 ... 线性注意力"): for marginal block pairs the
-// attention is replaced by linear attention with feature map phi, evaluated as
-// "K^T V first, then apply Q"; its output passes through the learnable
+// SLA page section 3 (the marginal-weight branch): for marginal block pairs the
+// attention is replaced by linear attention with feature map phi, evaluated by
+// forming K^T V first and applying Q afterwards; its output passes through the learnable
 // projection W_proj before it is added (same section, projection paragraph).
 // Because linear attention is a normalised weighted sum of value rows,
 // (sum w v / sum w) W = sum w (v W) / sum w, so W_proj is folded into V here.

@@ -1,10 +1,12 @@
 // k_pool.cu -- bandwidth-bound pooling kernels.
 //
-// pool_means_kernel: the block mean-pooling of Q and K that feeds SLA's
-// compressed score matrix (SLA page section 3: "对查询（Q）和键（K）矩阵进行平均
-// 池化").  One CTA reads one 64-token block (16-byte vector loads, valid tokens
-// only) and writes its mean in fp64.  Sums of at most 64 bf16 values are exact
-// in fp64, so the pooled means do not depend on summation order.
+// pool_means_kernel: the per-block mean of Q and of K that feeds SLA's
+// compressed score matrix (SLA page, section 3: both Q and K are averaged over
+// each token block first).  One CTA reads one 64-token block (16-byte vector
+// loads, valid tokens only).  Sums of at most 64 bf16 values are exact in fp64,
+// so the mean does not depend on summation order.  It is written as a bf16 pair
+// hi + lo (hi = bf16(mean), lo = bf16(mean - hi), 16 significant bits together)
+// in the row layout the tensor-core logits GEMM consumes.
 //
 // far_pool_kernel: the far field of the RoPeSLR gated mode -- K and V averaged
 // over cells of (cf, ch, cw) raster tokens (aixinbiao page: K and V compressed
@@ -22,13 +24,14 @@ namespace {
 template <int D>
 __global__ void __launch_bounds__(128)
 pool_means_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
-                  double* __restrict__ qbar, double* __restrict__ kbar, SeqShape s) {
+                  __nv_bfloat16* __restrict__ qsplit, __nv_bfloat16* __restrict__ ksplit, SeqShape s) {
   constexpr int kCPR = D / 8;          // 16-byte chunks per row
   constexpr int kRG = 128 / kCPR;      // row groups
   __shared__ double red[kRG][D];
   const int blk = blockIdx.x, bh = blockIdx.y;
-  const __nv_bfloat16* x = (blockIdx.z == 0 ? q : k) + ((size_t)bh * s.n_pad + (size_t)blk * kBlock) * D;
-  double* out = (blockIdx.z == 0 ? qbar : kbar) + ((size_t)bh * s.n_blocks + blk) * D;
+  const bool is_q = blockIdx.z == 0;
+  const __nv_bfloat16* x = (is_q ? q : k) + ((size_t)bh * s.n_pad + (size_t)blk * kBlock) * D;
+  __nv_bfloat16* out = (is_q ? qsplit : ksplit) + ((size_t)bh * s.n_blocks + blk) * 3 * D;
   const int chunk = threadIdx.x % kCPR, rg = threadIdx.x / kCPR;
   const int nvalid = block_valid_count(s, blk);   // valid tokens form a prefix of the block
   double acc[8];
@@ -50,7 +53,14 @@ pool_means_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
     double sum = 0.0;
     #pragma unroll
     for (int g = 0; g < kRG; ++g) sum += red[g][c];
-    out[c] = sum / (double)nvalid;
+    const double mean = sum / (double)nvalid;
+    const __nv_bfloat16 hi = __double2bfloat16(mean);
+    const __nv_bfloat16 lo = __double2bfloat16(mean - (double)__bfloat162float(hi));
+    // Q rows [hi | hi | lo], K rows [hi | lo | hi]: their dot product is
+    // qh.kh + qh.kl + ql.kh, the pooled logit up to the tiny ql.kl term
+    out[c] = hi;
+    out[D + c] = is_q ? hi : lo;
+    out[2 * D + c] = is_q ? lo : hi;
   }
 }
 
@@ -97,13 +107,15 @@ far_pool_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __rest
 
 }  // namespace
 
-cudaError_t launch_pool_means(const void* q, const void* k, double* qbar, double* kbar,
+cudaError_t launch_pool_means(const void* q, const void* k, void* qsplit, void* ksplit,
                               int BH, int d, SeqShape s, cudaStream_t st) {
   dim3 grid(s.n_blocks, BH, 2);
+  auto* qs = static_cast<__nv_bfloat16*>(qsplit);
+  auto* ks = static_cast<__nv_bfloat16*>(ksplit);
   if (d == 128)
-    pool_means_kernel<128><<<grid, 128, 0, st>>>((const __nv_bfloat16*)q, (const __nv_bfloat16*)k, qbar, kbar, s);
+    pool_means_kernel<128><<<grid, 128, 0, st>>>((const __nv_bfloat16*)q, (const __nv_bfloat16*)k, qs, ks, s);
   else
-    pool_means_kernel<64><<<grid, 128, 0, st>>>((const __nv_bfloat16*)q, (const __nv_bfloat16*)k, qbar, kbar, s);
+    pool_means_kernel<64><<<grid, 128, 0, st>>>((const __nv_bfloat16*)q, (const __nv_bfloat16*)k, qs, ks, s);
   return cudaGetLastError();
 }
 

@@ -19,8 +19,9 @@ bool make_tile_map(CUtensorMap* map, const void* base, int rank, const uint64_t*
                    const uint64_t* strides_bytes, const uint32_t* box);
 
 // ------------------------------------------------------------ pooling (k_pool.cu)
-// Means of the valid tokens of every 64-token block of q and k, fp64 [BH][Nb][d].
-cudaError_t launch_pool_means(const void* q, const void* k, double* qbar, double* kbar,
+// Means of the valid tokens of every 64-token block of q and k, each written as a
+// bf16 pair hi + lo: rows [BH][Nb][3d], [qh | qh | ql] for q and [kh | kl | kh] for k.
+cudaError_t launch_pool_means(const void* q, const void* k, void* qsplit, void* ksplit,
                               int BH, int d, SeqShape s, cudaStream_t st);
 
 // Far-field K/V: means over cells of (cf, ch, cw) tokens of the raster (F, Hh, Ww),
@@ -29,16 +30,25 @@ cudaError_t launch_far_pool(const void* k, const void* v, void* kf, void* vf, in
                             int F, int Hh, int Ww, int cf, int ch, int cw, cudaStream_t st);
 
 // ------------------------------------------------------------ classification (k_classify.cu)
-// logits[bh][i][j] = qbar_i . kbar_j in fp64 (the scale 1/sqrt(d) is applied where P_c is formed).
-cudaError_t launch_block_logits(const double* qbar, const double* kbar, double* logits,
-                                int BH, int nb, int d, cudaStream_t st);
+// Row stride (entries) of the logit-key matrix: Nb rounded up to 128.
+int logits_row_stride(int nb);
 
-// Per row: top kc -> 1, bottom kn -> -1, rest 0; critical list ascending; the
-// marginal indicator m01 (bf16 1/0, row stride ld_m01, pad columns 0); optional
-// P_c = softmax(logits / sqrt(d)) in fp32.
-cudaError_t launch_classify_rows(const double* logits, int BH, int nb, int d, int kc, int kn,
-                                 int8_t* mask, int32_t* crit_idx, int32_t* crit_cnt,
-                                 __nv_bfloat16* m01, int ld_m01, float* scores, cudaStream_t st);
+// keys[bh][i][j] = order-preserving uint32 key of the logit qbar_i . kbar_j (from the
+// split rows of launch_pool_means), row stride logits_row_stride(nb), pad entries 0.
+cudaError_t launch_logits(const void* qsplit, const void* ksplit, uint32_t* keys, int BH, int nb, int d,
+                          int* status, cudaStream_t st);
+
+// Labels per row from the logit keys (top kc -> 1, bottom kn -> -1, rest 0, ties to
+// the lower index) and the outputs, each optional (nullptr = skip): mask
+// [BH][nb][nb]; crit_idx [BH][nb][kc] ascending and crit_cnt [BH][nb]; the marginal
+// indicator m01 (bf16 1/0, row stride ld_m01, pad columns 0); P_c =
+// softmax(logits / sqrt(d)) in fp32; pair lists [BH][(nb+1)/2][list_cap] of the
+// union of the critical sets of query blocks 2p and 2p+1 (entry layout below) with
+// counts list_cnt [BH][(nb+1)/2].
+cudaError_t launch_classify(const uint32_t* keys, int BH, int nb, int d, int kc, int kn,
+                            int8_t* mask, int32_t* crit_idx, int32_t* crit_cnt, __nv_bfloat16* m01, int ld_m01,
+                            float* scores, uint32_t* list, int32_t* list_cnt, int list_cap, SeqShape s,
+                            int* status, cudaStream_t st);
 
 // m01 = (mask == 0) as bf16 with row stride ld_m01 (pad columns zeroed).
 cudaError_t launch_mask_to_m01(const int8_t* mask, __nv_bfloat16* m01, int BH, int nb, int ld_m01,

@@ -114,15 +114,16 @@ int ld_m01(int nb) { return (nb + 63) / 64 * 64; }
 // ---------------------------------------------------------------- workspace plans
 
 struct ClassifyWs {
-  double *qbar, *kbar, *logits;
+  __nv_bfloat16 *qsplit, *ksplit;
+  uint32_t* keys;
   __nv_bfloat16* m01;
 };
 
-void plan_classify(Carve& c, const Shape& sh, ClassifyWs& w) {
-  w.qbar = c.take<double>((size_t)sh.BH * sh.nb * sh.d);
-  w.kbar = c.take<double>((size_t)sh.BH * sh.nb * sh.d);
-  w.logits = c.take<double>((size_t)sh.BH * sh.nb * sh.nb);
-  w.m01 = c.take<__nv_bfloat16>((size_t)sh.BH * sh.nb * ld_m01(sh.nb));
+void plan_classify(Carve& c, const Shape& sh, bool m01, ClassifyWs& w) {
+  w.qsplit = c.take<__nv_bfloat16>((size_t)sh.BH * sh.nb * 3 * sh.d);
+  w.ksplit = c.take<__nv_bfloat16>((size_t)sh.BH * sh.nb * 3 * sh.d);
+  w.keys = c.take<uint32_t>((size_t)sh.BH * sh.nb * logits_row_stride(sh.nb));
+  w.m01 = m01 ? c.take<__nv_bfloat16>((size_t)sh.BH * sh.nb * ld_m01(sh.nb)) : nullptr;
 }
 
 struct MarginalWs {
@@ -138,23 +139,18 @@ void plan_marginal(Carve& c, const Shape& sh, MarginalWs& w) {
 struct SlaWs {
   int* status;
   ClassifyWs cls;
-  int8_t* mask;
-  int32_t *crit_idx, *crit_cnt;
   uint32_t* list;
   int32_t* list_cnt;
   int cap;
   MarginalWs mar;
 };
 
-void plan_sla(Carve& c, const Shape& sh, int kc, int kn, bool own_mask, SlaWs& w) {
+void plan_sla(Carve& c, const Shape& sh, int kc, int kn, SlaWs& w) {
   w.status = c.take<int>(64);
   const bool dense = kc == sh.nb;
   w.cap = dense ? 0 : (2 * kc < sh.nb ? 2 * kc : sh.nb);
   if (dense) return;
-  plan_classify(c, sh, w.cls);
-  w.mask = own_mask ? c.take<int8_t>((size_t)sh.BH * sh.nb * sh.nb) : nullptr;
-  w.crit_idx = c.take<int32_t>((size_t)sh.BH * sh.nb * kc);
-  w.crit_cnt = c.take<int32_t>((size_t)sh.BH * sh.nb);
+  plan_classify(c, sh, sh.nb - kc - kn > 0, w.cls);
   w.list = c.take<uint32_t>((size_t)sh.BH * sh.npairs * w.cap);
   w.list_cnt = c.take<int32_t>((size_t)sh.BH * sh.npairs);
   if (sh.nb - kc - kn > 0) {
@@ -238,7 +234,7 @@ enum KernelKind {
   kKFarPool, kKMaskToM01, kKNumKinds
 };
 const char* const kKindNames[kKNumKinds] = {
-    "pool_means", "block_logits", "classify_rows", "pair_lists", "key_states", "reduce_states",
+    "pool_means", "logits", "classify", "pair_lists", "key_states", "reduce_states",
     "linear_apply", "attention", "lvsa_sets", "far_pool", "mask_to_m01"};
 
 struct ProfRec {
@@ -377,7 +373,7 @@ size_t slr_workspace_bytes(int op, const slr_seq* seq, const void* params) {
       if (sh.nb > kMaxClassifyBlocks || !params) return 0;
       c.take<int>(64);
       ClassifyWs w;
-      plan_classify(c, sh, w);
+      plan_classify(c, sh, false, w);
       return c.off;
     }
     case SLR_OP_BLOCK_SPARSE: {
@@ -402,7 +398,7 @@ size_t slr_workspace_bytes(int op, const slr_seq* seq, const void* params) {
       if (counts(sh.nb, f->crit_frac, f->negl_frac, &kc, &kn) != SLR_OK) return 0;
       if (kc != sh.nb && sh.nb > kMaxClassifyBlocks) return 0;
       SlaWs w;
-      plan_sla(c, sh, kc, kn, true, w);
+      plan_sla(c, sh, kc, kn, w);
       return c.off;
     }
     case SLR_OP_FRAME_MASK: {
@@ -442,12 +438,12 @@ slr_status slr_pool_classify(const void* q, const void* k, const slr_seq* seq, f
   Carve c(ws);
   int* status = c.take<int>(64);
   ClassifyWs w;
-  plan_classify(c, sh, w);
+  plan_classify(c, sh, false, w);
   SLR_TRY(cudaMemsetAsync(status, 0, sizeof(int), s));
-  SLR_LAUNCH(kKPool, s, launch_pool_means(q, k, w.qbar, w.kbar, sh.BH, sh.d, sh.s, s));
-  SLR_LAUNCH(kKLogits, s, launch_block_logits(w.qbar, w.kbar, w.logits, sh.BH, sh.nb, sh.d, s));
-  SLR_LAUNCH(kKClassify, s, launch_classify_rows(w.logits, sh.BH, sh.nb, sh.d, kc, kn, mask, crit_idx, crit_cnt, w.m01, ld_m01(sh.nb),
-                               scores_opt, s));
+  SLR_LAUNCH(kKPool, s, launch_pool_means(q, k, w.qsplit, w.ksplit, sh.BH, sh.d, sh.s, s));
+  SLR_LAUNCH(kKLogits, s, launch_logits(w.qsplit, w.ksplit, w.keys, sh.BH, sh.nb, sh.d, status, s));
+  SLR_LAUNCH(kKClassify, s, launch_classify(w.keys, sh.BH, sh.nb, sh.d, kc, kn, mask, crit_idx, crit_cnt,
+                                            nullptr, 0, scores_opt, nullptr, nullptr, 0, sh.s, status, s));
   return SLR_OK;
 }
 
@@ -527,7 +523,7 @@ slr_status slr_sparse_linear_attn(const void* q, const void* k, const void* v, c
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   Carve c(ws);
   SlaWs w;
-  plan_sla(c, sh, kc, kn, true, w);
+  plan_sla(c, sh, kc, kn, w);
   SLR_TRY(cudaMemsetAsync(w.status, 0, sizeof(int), s));
   AttnArgs a = attn_base(sh, q, k, v, out, w.status);
   if (dense) {
@@ -535,18 +531,11 @@ slr_status slr_sparse_linear_attn(const void* q, const void* k, const void* v, c
     SLR_LAUNCH(kKAttention, s, launch_attention(a, s));
     return SLR_OK;
   }
-  int8_t* mask = mask_out_opt ? mask_out_opt : w.mask;
-  SLR_LAUNCH(kKPool, s, launch_pool_means(q, k, w.cls.qbar, w.cls.kbar, sh.BH, sh.d, sh.s, s));
-  SLR_LAUNCH(kKLogits, s, launch_block_logits(w.cls.qbar, w.cls.kbar, w.cls.logits, sh.BH, sh.nb, sh.d, s));
-  SLR_LAUNCH(kKClassify, s, launch_classify_rows(w.cls.logits, sh.BH, sh.nb, sh.d, kc, kn, mask, w.crit_idx, w.crit_cnt, w.cls.m01,
-                               ld_m01(sh.nb), nullptr, s));
-  ListArgs la;
-  memset(&la, 0, sizeof(la));
-  la.mode = kListExplicit;
-  la.n_qb = sh.nb; la.n_kb = sh.nb; la.n_pairs = sh.npairs; la.cap = w.cap;
-  la.kv_idx = w.crit_idx; la.kv_cnt = w.crit_cnt; la.kv_max = kc;
-  la.s = sh.s; la.list = w.list; la.list_cnt = w.list_cnt; la.status = w.status;
-  SLR_LAUNCH(kKLists, s, launch_pair_lists(la, sh.BH, s));
+  SLR_LAUNCH(kKPool, s, launch_pool_means(q, k, w.cls.qsplit, w.cls.ksplit, sh.BH, sh.d, sh.s, s));
+  SLR_LAUNCH(kKLogits, s, launch_logits(w.cls.qsplit, w.cls.ksplit, w.cls.keys, sh.BH, sh.nb, sh.d, w.status, s));
+  SLR_LAUNCH(kKClassify, s, launch_classify(w.cls.keys, sh.BH, sh.nb, sh.d, kc, kn, mask_out_opt, nullptr,
+                                            nullptr, w.cls.m01, ld_m01(sh.nb), nullptr, w.list, w.list_cnt, w.cap,
+                                            sh.s, w.status, s));
   if (marginal) {
     SLR_LAUNCH(kKKeyStates, s, launch_key_states(k, v, w_proj, w.mar.h, sh.BH, sh.d, sh.s, w.status, s));
     SLR_LAUNCH(kKReduce, s, launch_reduce_states(w.cls.m01, ld_m01(sh.nb), w.mar.h, w.mar.Hs, sh.BH, sh.nb, sh.d, w.status, s));

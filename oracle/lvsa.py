@@ -16,7 +16,7 @@ Source: rainbus paper-digest page "LVSAï¼šé¢å‘é•¿è§†é¢‘æ‰©æ•£æ¨¡åž‹çš„æ— è®­ç»
 * A(t) = G_s u W(t), and every query token of frame t attends, with one exact
   softmax, every key token of the frames in A(t) (step 6 formula).
 
-Readings where the page is silent (also listed in the design doc):
+Readings where the page is silent:
 
 * "the side with the most room": room_lo = w_lo frames to the left, room_hi =
   T - 1 - w_hi to the right; grow w_hi when room_hi >= room_lo (a tie grows the

@@ -8,13 +8,13 @@ section 3 "SLA方法的核心机制":
 * each position of P_c is labelled critical (1, top 5 %), negligible (-1,
   bottom 10 %) or marginal (0, the rest);
 * critical pairs get exact softmax (FlashAttention-style) attention;
-* marginal pairs get linear attention with a feature map phi, evaluated as
-  "K^T V first, then apply Q";
+* marginal pairs get linear attention with a feature map phi, evaluated by
+  forming K^T V first and multiplying by Q afterwards;
 * negligible pairs are skipped;
 * a learnable projection is applied to the linear-attention output before it
-  is added to the sparse output (same section, the "可学习的投影层" paragraph).
+  is added to the sparse output (same section, the paragraph on the projection layer).
 
-Readings where the page is silent (each is also listed in the design doc):
+Readings where the page is silent:
 
 1. Percentiles are taken per query-block row of P_c.
 2. kc = max(1, ceil(p_c * Nkb)), kn = floor(p_n * Nkb), capped so that

@@ -10,7 +10,7 @@ Source: aixinbiao blog page "RoPeSLR æŠŠè§†é¢‘æ‰©æ•£é‡Œçš„ attention ç äº†ä¸€å
 * the two outputs are fused by a gate: g * local + (1 - g) * global
   (g = 0.55 at convergence on that page).
 
-Readings (also listed in the design doc):
+Readings:
 
 * the neighbourhood is taken at tile granularity: tokens are grouped in
   4x4x4 tiles of the (frame, h, w) raster; a query attends every token of the
