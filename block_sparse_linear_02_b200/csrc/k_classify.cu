@@ -139,6 +139,7 @@ struct ClsArgs {
   int nb, nbp, kc, kn, n_pairs;
   float inv_sqrt_d;
   int8_t* mask;
+  bool mask_vec;           // rows of the mask can take 4-byte stores (nb % 4 == 0, 4-byte aligned base)
   int32_t* crit_idx;
   int32_t* crit_cnt;
   __nv_bfloat16* m01;
@@ -152,64 +153,167 @@ struct ClsArgs {
 };
 
 constexpr int kClsWarps = 4;
+constexpr int kPrefixBits = 12;      // thresholds are first located to the top 12 key bits
+constexpr int kMaxCand = 32;         // candidates resolved exactly by ranking
 
+__device__ __forceinline__ int warp_excl_scan(int v, int lane) {
+  int x = v;
+  #pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xFFFFFFFFu, x, o);
+    if (lane >= o) x += y;
+  }
+  return x - v;
+}
+
+// One warp per pair of query blocks.  Each row's keys sit in shared memory; lane l
+// owns keys 128 g + 4 l .. +3 of every 128-key group g (one 16-byte load).
+//   1. Bisection over the top kPrefixBits key bits: Tc = prefix of the kc-th
+//      largest key, Tn = prefix of the kn-th smallest.
+//   2. The keys sharing the threshold prefix (a handful, since the prefix fixes
+//      sign, exponent and 3 mantissa bits) are collected and ranked exactly; if
+//      more than kMaxCand share a prefix the bisection continues over the
+//      remaining bits instead.
+//   3. One pass in index order writes the labels and outputs; ties at a threshold
+//      go to the lower index (critical) or leave the higher index marginal
+//      (negligible), via warp prefix counts of the tied keys.
 __global__ void __launch_bounds__(kClsWarps * 32)
 classify_kernel(const ClsArgs a) {
   extern __shared__ __align__(16) uint32_t skeys[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int bh = blockIdx.y, pair = blockIdx.x * kClsWarps + warp;
-  const int nb = a.nb, nbp = a.nbp;
+  const int nb = a.nb, nbp = a.nbp, ng = nbp / 128;
   const int qb0 = 2 * pair;
   if (qb0 >= nb) return;
   const int nrows = qb0 + 1 < nb ? 2 : 1;
   uint32_t* rowk[2] = {skeys + (size_t)(2 * warp) * nbp, skeys + (size_t)(2 * warp + 1) * nbp};
+  uint32_t* cand = skeys + (size_t)kClsWarps * 2 * nbp + warp * (4 * kMaxCand + 4);   // [4][kMaxCand]
+  int* ccount = reinterpret_cast<int*>(cand + 4 * kMaxCand);                            // [4]
   for (int r = 0; r < nrows; ++r) {
     const uint4* src = reinterpret_cast<const uint4*>(a.keys + ((size_t)bh * nb + qb0 + r) * nbp);
     for (int e = lane; e < nbp / 4; e += 32) reinterpret_cast<uint4*>(rowk[r])[e] = src[e];
   }
+  if (lane < 4) ccount[lane] = 0;
   __syncwarp();
   const int npad = nbp - nb;
 
-  // ---- thresholds: Tc = kc-th largest key, Tn = kn-th smallest
+  // ---- 1. thresholds to kPrefixBits bits (pads are key 0: never >= a candidate
+  // top threshold, always <= a candidate bottom one)
   uint32_t Tc[2] = {0u, 0u}, Tn[2] = {0xFFFFFFFFu, 0xFFFFFFFFu};
-  for (int bit = 31; bit >= 0; --bit) {
-    #pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      if (r >= nrows) break;                      // warp-uniform
-      const uint32_t cc = Tc[r] | (1u << bit), cn = Tn[r] & ~(1u << bit);
-      int nc = 0, nn = 0;
-      for (int j = lane * 4; j < nbp; j += 128) {
-        const uint4 k4 = *reinterpret_cast<const uint4*>(rowk[r] + j);
-        nc += (k4.x >= cc) + (k4.y >= cc) + (k4.z >= cc) + (k4.w >= cc);
-        nn += (k4.x <= cn) + (k4.y <= cn) + (k4.z <= cn) + (k4.w <= cn);
+  auto bisect = [&](int hi, int lo) {
+    for (int bit = hi; bit >= lo; --bit) {
+      #pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        if (r >= nrows) break;                    // warp-uniform
+        const uint32_t cc = Tc[r] | (1u << bit), cn = Tn[r] & ~(1u << bit);
+        int nc = 0, nn = 0;
+        for (int g = 0; g < ng; ++g) {
+          const uint4 k4 = *reinterpret_cast<const uint4*>(rowk[r] + g * 128 + lane * 4);
+          nc += (k4.x >= cc) + (k4.y >= cc) + (k4.z >= cc) + (k4.w >= cc);
+          nn += (k4.x <= cn) + (k4.y <= cn) + (k4.z <= cn) + (k4.w <= cn);
+        }
+        if (warp_sum(nc) >= a.kc) Tc[r] = cc;
+        if (warp_sum(nn) - npad >= a.kn) Tn[r] = cn;
       }
-      if (warp_sum(nc) >= a.kc) Tc[r] = cc;
-      if (warp_sum(nn) - npad >= a.kn) Tn[r] = cn;   // pads (key 0) always count as <=
     }
-  }
-  // keys above the critical threshold, below the negligible one, equal to it; the row max
+  };
+  bisect(31, 32 - kPrefixBits);
+
+  // ---- 2. exact thresholds: collect the keys that share each threshold prefix
+  constexpr int kSh = 32 - kPrefixBits;
   int gt_c[2] = {0, 0}, lt_n[2] = {0, 0}, eq_n[2] = {0, 0};
-  float row_max[2] = {0.f, 0.f}, row_sum[2] = {1.f, 1.f};
   #pragma unroll
   for (int r = 0; r < 2; ++r) {
     if (r >= nrows) break;
-    uint32_t kmax = 0u;
-    for (int j = lane * 4; j < nbp; j += 128) {
-      const uint4 k4 = *reinterpret_cast<const uint4*>(rowk[r] + j);
+    const uint32_t pc = Tc[r] >> kSh, pn = Tn[r] >> kSh;
+    int gt = 0, lt = 0;
+    for (int g = 0; g < ng; ++g) {
+      const uint4 k4 = *reinterpret_cast<const uint4*>(rowk[r] + g * 128 + lane * 4);
       const uint32_t kk[4] = {k4.x, k4.y, k4.z, k4.w};
       #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        gt_c[r] += kk[i] > Tc[r];
-        lt_n[r] += kk[i] != 0u && kk[i] < Tn[r];
-        eq_n[r] += kk[i] == Tn[r];
-        kmax = kk[i] > kmax ? kk[i] : kmax;
+        const uint32_t pk = kk[i] >> kSh;
+        gt += pk > pc;
+        lt += kk[i] != 0u && pk < pn;
+        if (pk == pc) { const int at = atomicAdd(&ccount[2 * r], 1); if (at < kMaxCand) cand[(2 * r) * kMaxCand + at] = kk[i]; }
+        if (kk[i] != 0u && pk == pn) { const int at = atomicAdd(&ccount[2 * r + 1], 1); if (at < kMaxCand) cand[(2 * r + 1) * kMaxCand + at] = kk[i]; }
       }
     }
-    gt_c[r] = warp_sum(gt_c[r]);
-    lt_n[r] = warp_sum(lt_n[r]);
-    eq_n[r] = warp_sum(eq_n[r]);
-    row_max[r] = okey_value(__reduce_max_sync(0xFFFFFFFFu, kmax));
-    if (a.scores) {
+    gt_c[r] = warp_sum(gt);
+    lt_n[r] = warp_sum(lt);
+  }
+  __syncwarp();
+  bool fits = true;
+  for (int r = 0; r < nrows; ++r) fits = fits && ccount[2 * r] <= kMaxCand && (a.kn == 0 || ccount[2 * r + 1] <= kMaxCand);
+  if (fits) {
+    #pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      if (r >= nrows) break;
+      // top: the (kc - gt)-th largest candidate; lane l ranks candidate l
+      {
+        const int n = ccount[2 * r], need = a.kc - gt_c[r];
+        const uint32_t c = lane < n ? cand[(2 * r) * kMaxCand + lane] : 0u;
+        int above = 0, atleast = 0;
+        for (int m = 0; m < n; ++m) {
+          const uint32_t o = cand[(2 * r) * kMaxCand + m];
+          above += o > c;
+          atleast += o >= c;
+        }
+        const bool is_t = lane < n && above < need && need <= atleast;
+        const unsigned bt = __ballot_sync(0xFFFFFFFFu, is_t);
+        const int src = __ffs(bt) - 1;
+        Tc[r] = __shfl_sync(0xFFFFFFFFu, c, src);
+        gt_c[r] += __shfl_sync(0xFFFFFFFFu, above, src);
+      }
+      if (a.kn > 0) {
+        const int n = ccount[2 * r + 1], need = a.kn - lt_n[r];
+        const uint32_t c = lane < n ? cand[(2 * r + 1) * kMaxCand + lane] : 0xFFFFFFFFu;
+        int below = 0, atmost = 0;
+        for (int m = 0; m < n; ++m) {
+          const uint32_t o = cand[(2 * r + 1) * kMaxCand + m];
+          below += o < c;
+          atmost += o <= c;
+        }
+        const bool is_t = lane < n && below < need && need <= atmost;
+        const unsigned bt = __ballot_sync(0xFFFFFFFFu, is_t);
+        const int src = __ffs(bt) - 1;
+        Tn[r] = __shfl_sync(0xFFFFFFFFu, c, src);
+        lt_n[r] += __shfl_sync(0xFFFFFFFFu, below, src);
+        eq_n[r] = __shfl_sync(0xFFFFFFFFu, atmost - below, src);
+      }
+    }
+  } else {
+    // many keys share a prefix (e.g. tied rows): finish the bisection and count
+    bisect(31 - kPrefixBits, 0);
+    #pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      if (r >= nrows) break;
+      int gt = 0, lt = 0, eq = 0;
+      for (int g = 0; g < ng; ++g) {
+        const uint4 k4 = *reinterpret_cast<const uint4*>(rowk[r] + g * 128 + lane * 4);
+        const uint32_t kk[4] = {k4.x, k4.y, k4.z, k4.w};
+        #pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          gt += kk[i] > Tc[r];
+          lt += kk[i] != 0u && kk[i] < Tn[r];
+          eq += kk[i] == Tn[r];
+        }
+      }
+      gt_c[r] = warp_sum(gt);
+      lt_n[r] = warp_sum(lt);
+      eq_n[r] = warp_sum(eq);
+    }
+  }
+
+  // ---- P_c normaliser (only when scores are requested)
+  float row_max[2] = {0.f, 0.f}, row_sum[2] = {1.f, 1.f};
+  if (a.scores) {
+    #pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      if (r >= nrows) break;
+      uint32_t kmax = 0u;
+      for (int j = lane; j < nb; j += 32) kmax = rowk[r][j] > kmax ? rowk[r][j] : kmax;
+      row_max[r] = okey_value(__reduce_max_sync(0xFFFFFFFFu, kmax));
       float sum = 0.f;
       for (int j = lane; j < nb; j += 32) sum += expf((okey_value(rowk[r][j]) - row_max[r]) * a.inv_sqrt_d);
       #pragma unroll
@@ -218,48 +322,95 @@ classify_kernel(const ClsArgs a) {
     }
   }
 
-  // ---- labels in index order and the outputs
-  const unsigned lt_mask = (1u << lane) - 1u;
+  // ---- 3. labels in index order and the outputs
   int seen_c[2] = {0, 0}, seen_n[2] = {0, 0}, written[2] = {0, 0}, listed = 0;
   uint32_t* lst = a.list ? a.list + ((size_t)bh * a.n_pairs + pair) * a.list_cap : nullptr;
-  for (int j0 = 0; j0 < nb; j0 += 32) {
-    const int j = j0 + lane;
-    const bool in = j < nb;
-    bool crit[2] = {false, false};
+  for (int g = 0; g < ng; ++g) {
+    const int j0 = g * 128 + lane * 4;           // my 4 keys: j0 .. j0+3
+    uint32_t crit_bits[2] = {0u, 0u};
     #pragma unroll
     for (int r = 0; r < 2; ++r) {
       if (r >= nrows) break;
-      const uint32_t k = in ? rowk[r][j] : 0u;
-      const bool eqc = in && k == Tc[r];
-      const unsigned bc = __ballot_sync(0xFFFFFFFFu, eqc);
-      crit[r] = (in && k > Tc[r]) || (eqc && seen_c[r] + __popc(bc & lt_mask) < a.kc - gt_c[r]);
-      seen_c[r] += __popc(bc);
-      bool negl = false;
+      const uint4 k4 = *reinterpret_cast<const uint4*>(rowk[r] + g * 128 + lane * 4);
+      const uint32_t kk[4] = {k4.x, k4.y, k4.z, k4.w};
+      uint32_t gtb = 0, eqcb = 0, ltb = 0, eqnb = 0;
+      #pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const bool in = j0 + i < nb;
+        gtb |= (uint32_t)(in && kk[i] > Tc[r]) << i;
+        eqcb |= (uint32_t)(in && kk[i] == Tc[r]) << i;
+        ltb |= (uint32_t)(in && kk[i] < Tn[r]) << i;
+        eqnb |= (uint32_t)(in && kk[i] == Tn[r]) << i;
+      }
+      // critical: all above Tc, plus the first (kc - gt_c) keys equal to Tc in index order
+      uint32_t cb = gtb;
+      if (__any_sync(0xFFFFFFFFu, eqcb != 0u)) {
+        const int ne = __popc(eqcb);
+        int rank = seen_c[r] + warp_excl_scan(ne, lane);
+        for (int i = 0; i < 4; ++i)
+          if ((eqcb >> i) & 1u) { if (rank < a.kc - gt_c[r]) cb |= 1u << i; ++rank; }
+        seen_c[r] += warp_sum(ne);
+      }
+      // negligible: all below Tn, plus the last (kn - lt_n) keys equal to Tn
+      uint32_t nbm = 0u;
       if (a.kn > 0) {
-        const bool eqn = in && k == Tn[r];
-        const unsigned bn = __ballot_sync(0xFFFFFFFFu, eqn);
-        negl = (in && k < Tn[r]) || (eqn && seen_n[r] + __popc(bn & lt_mask) >= eq_n[r] - (a.kn - lt_n[r]));
-        seen_n[r] += __popc(bn);
+        nbm = ltb;
+        if (__any_sync(0xFFFFFFFFu, eqnb != 0u)) {
+          const int ne = __popc(eqnb);
+          int rank = seen_n[r] + warp_excl_scan(ne, lane);
+          for (int i = 0; i < 4; ++i)
+            if ((eqnb >> i) & 1u) { if (rank >= eq_n[r] - (a.kn - lt_n[r])) nbm |= 1u << i; ++rank; }
+          seen_n[r] += warp_sum(ne);
+        }
       }
+      crit_bits[r] = cb;
       const size_t row = (size_t)bh * nb + qb0 + r;
-      if (in) {
-        const int8_t m = crit[r] ? 1 : (negl ? -1 : 0);
-        if (a.mask) a.mask[row * nb + j] = m;
-        if (a.m01) a.m01[row * a.ld_m01 + j] = __float2bfloat16_rn(m == 0 ? 1.f : 0.f);
-        if (a.scores) a.scores[row * nb + j] = expf((okey_value(k) - row_max[r]) * a.inv_sqrt_d) / row_sum[r];
+      if (j0 < nb) {
+        int8_t m[4];
+        #pragma unroll
+        for (int i = 0; i < 4; ++i) m[i] = ((cb >> i) & 1u) ? 1 : (((nbm >> i) & 1u) ? -1 : 0);
+        if (j0 + 3 < nb) {
+          if (a.mask) {
+            const uint32_t w = (uint32_t)(uint8_t)m[0] | ((uint32_t)(uint8_t)m[1] << 8) |
+                               ((uint32_t)(uint8_t)m[2] << 16) | ((uint32_t)(uint8_t)m[3] << 24);
+            if (a.mask_vec) *reinterpret_cast<uint32_t*>(a.mask + row * nb + j0) = w;
+            else for (int i = 0; i < 4; ++i) a.mask[row * nb + j0 + i] = m[i];
+          }
+          if (a.m01)
+            *reinterpret_cast<uint2*>(a.m01 + row * a.ld_m01 + j0) =
+                make_uint2(pack_bf16(m[0] == 0 ? 1.f : 0.f, m[1] == 0 ? 1.f : 0.f),
+                           pack_bf16(m[2] == 0 ? 1.f : 0.f, m[3] == 0 ? 1.f : 0.f));
+        } else {
+          for (int i = 0; i < 4 && j0 + i < nb; ++i) {
+            if (a.mask) a.mask[row * nb + j0 + i] = m[i];
+            if (a.m01) a.m01[row * a.ld_m01 + j0 + i] = __float2bfloat16_rn(m[i] == 0 ? 1.f : 0.f);
+          }
+        }
+        if (a.scores)
+          for (int i = 0; i < 4 && j0 + i < nb; ++i)
+            a.scores[row * nb + j0 + i] = expf((okey_value(kk[i]) - row_max[r]) * a.inv_sqrt_d) / row_sum[r];
       }
-      const unsigned bcrit = __ballot_sync(0xFFFFFFFFu, crit[r]);
-      if (a.crit_idx && crit[r]) a.crit_idx[row * a.kc + written[r] + __popc(bcrit & lt_mask)] = j;
-      written[r] += __popc(bcrit);
+      if (a.crit_idx) {
+        const int nc = __popc(cb);
+        int pos = written[r] + warp_excl_scan(nc, lane);
+        for (int i = 0; i < 4; ++i)
+          if ((cb >> i) & 1u) a.crit_idx[row * a.kc + pos++] = j0 + i;
+        written[r] += warp_sum(nc);
+      }
     }
     if (lst) {
-      const bool u = crit[0] || crit[1];
-      const unsigned bu = __ballot_sync(0xFFFFFFFFu, u);
-      const int pos = listed + __popc(bu & lt_mask);
-      if (u && pos < a.list_cap)
-        lst[pos] = (uint32_t)j | ((uint32_t)block_valid_count(a.s, j) << 16) | ((uint32_t)crit[0] << 30) |
-                   ((uint32_t)crit[1] << 31);
-      listed += __popc(bu);
+      const uint32_t u = crit_bits[0] | crit_bits[1];
+      const int nu = __popc(u);
+      int pos = listed + warp_excl_scan(nu, lane);
+      for (int i = 0; i < 4; ++i)
+        if ((u >> i) & 1u) {
+          const int j = j0 + i;
+          if (pos < a.list_cap)
+            lst[pos] = (uint32_t)j | ((uint32_t)block_valid_count(a.s, j) << 16) |
+                       (((crit_bits[0] >> i) & 1u) << 30) | (((crit_bits[1] >> i) & 1u) << 31);
+          ++pos;
+        }
+      listed += warp_sum(nu);
     }
   }
   for (int r = 0; r < nrows; ++r) {
@@ -326,9 +477,9 @@ cudaError_t launch_classify(const uint32_t* keys, int BH, int nb, int d, int kc,
   ClsArgs a;
   a.keys = keys; a.nb = nb; a.nbp = logits_row_stride(nb); a.kc = kc; a.kn = kn; a.n_pairs = (nb + 1) / 2;
   a.inv_sqrt_d = (float)(1.0 / sqrt((double)d));
-  a.mask = mask; a.crit_idx = crit_idx; a.crit_cnt = crit_cnt; a.m01 = m01; a.ld_m01 = ld_m01;
+  a.mask = mask; a.mask_vec = (nb % 4 == 0) && (reinterpret_cast<uintptr_t>(mask) % 4 == 0); a.crit_idx = crit_idx; a.crit_cnt = crit_cnt; a.m01 = m01; a.ld_m01 = ld_m01;
   a.scores = scores; a.list = list; a.list_cnt = list_cnt; a.list_cap = list_cap; a.s = s; a.status = status;
-  const size_t smem = (size_t)2 * kClsWarps * a.nbp * sizeof(uint32_t);
+  const size_t smem = ((size_t)2 * kClsWarps * a.nbp + kClsWarps * (4 * kMaxCand + 4)) * sizeof(uint32_t);
   cudaError_t e = cudaFuncSetAttribute(classify_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid((a.n_pairs + kClsWarps - 1) / kClsWarps, BH);

@@ -239,6 +239,279 @@ key_states_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
   if (warp == 0) { tc_fence_after(); tmem_dealloc(tmem, 256); }
 }
 
+// ------------------------------------------------------------------ key states, d = 128
+// Warp-specialised and persistent (one CTA per SM): warp 0 streams K_j, V_j into a
+// 3-stage ring, warp 1 issues the MMAs, warps 2-5 (128 threads) apply phi in place,
+// form the column sums z_j, move (V_j W)^T from TMEM into the operand layout of the
+// second MMA, and drain h_j'^T from TMEM into a swizzled staging tile that two TMA
+// stores write out.  TMEM holds two (V W)^T and two h^T accumulators, so block n's
+// drain overlaps block n+1's MMAs.
+constexpr int kKpStages = 3;
+struct KpLayout {
+  static constexpr int kW = 0;                               // W_proj MN-major, 2 chunks x 16 KB
+  static constexpr int kRing = 32768;                        // stages: K 16 KB | V 16 KB
+  static constexpr int kStage = 32768;
+  static constexpr int kOut = kRing + kKpStages * kStage;    // h^T staging: 2 boxes of 64 columns
+  static constexpr int kZ = kOut + 32768;                    // z partials [2][8][128] floats
+  static constexpr int kBar = kZ + 2 * 8 * 128 * 4;
+  static constexpr int kBytes = kBar + 256 + 1024;
+};
+
+__device__ __forceinline__ float phi_exp2(float x) {
+  // elu(x) + 1; exp through the exp2 unit (the result is rounded to bf16)
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x * 1.4426950408889634f));
+  return x > 0.f ? x + 1.f : y;
+}
+
+
+template <bool PROJ>
+__global__ void __launch_bounds__(192, 1)
+key_states_pipe_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                       const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmH,
+                       __nv_bfloat16* __restrict__ h, SeqShape s, int BH, int* status) {
+  constexpr int D = 128;
+  using L = KpLayout;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint8_t* sW = smem + L::kW;
+  uint8_t* sOut = smem + L::kOut;
+  float* zbuf = reinterpret_cast<float*>(smem + L::kZ);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
+  uint64_t* full = bars;                          // [3] stage loaded
+  uint64_t* empty = full + kKpStages;             // [3] stage consumed by the second MMA
+  uint64_t* w_bar = empty + kKpStages;
+  uint64_t* p_full = w_bar + 1;                   // [2] (V W)^T in TMEM
+  uint64_t* conv_done = p_full + 2;               // [2] operands of the second MMA ready (128 arrivals)
+  uint64_t* h_full = conv_done + 2;               // [2] h^T in TMEM
+  uint64_t* h_free = h_full + 2;                  // [2] h^T drained (128 arrivals)
+  uint64_t* out_free = h_free + 2;                // staging tile read by the previous stores
+  uint64_t* out_full = out_free + 1;              // staging tile written (128 arrivals)
+  uint64_t* drain = out_full + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  constexpr int kChunkB = 8192;                   // 64 rows x 128 bytes
+  constexpr uint32_t kColP = 0;                   // P[b] at b * 64
+  constexpr uint32_t kColH = 128;                 // H[b] at 128 + b * 128
+  const int total = BH * s.n_blocks;
+  const int mine = blockIdx.x < total ? (total - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+  auto sK = [&](int st) { return smem + L::kRing + st * L::kStage; };
+  auto sV = [&](int st) { return smem + L::kRing + st * L::kStage + 16384; };
+
+  if (tid == 0) {
+    for (int i = 0; i < kKpStages; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
+    mbar_init(w_bar, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&p_full[b], 1);
+      mbar_init(&conv_done[b], 128);
+      mbar_init(&h_full[b], 1);
+      mbar_init(&h_free[b], 128);
+    }
+    mbar_init(out_free, 1);
+    mbar_init(out_full, 128);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) { tmem_alloc(tmem_slot, 512); tmem_relinquish(); }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- producer
+    if (lane == 0 && mine > 0) {
+      tma_prefetch_desc(&tmK); tma_prefetch_desc(&tmV);
+      if (PROJ) {
+        mbar_arrive_expect_tx(w_bar, 2 * D * 128);
+        for (int c = 0; c < 2; ++c) tma_load_3d(sW + c * D * 128, &tmW, w_bar, c * 64, 0, 0);
+      }
+      int n = 0;
+      for (; n < mine; ++n) {
+        const int st = n % kKpStages;
+        if (n >= kKpStages && !mbar_wait(&empty[st], ((n / kKpStages) - 1) & 1, abort_flag, status)) break;
+        const int blk_id = blockIdx.x + n * gridDim.x;
+        const int bh = blk_id / s.n_blocks, blk = blk_id % s.n_blocks;
+        mbar_arrive_expect_tx(&full[st], 2 * 2 * kChunkB);
+        for (int c = 0; c < 2; ++c) {
+          tma_load_3d(sK(st) + c * kChunkB, &tmK, &full[st], c * 64, blk * 64, bh);
+          tma_load_3d(sV(st) + c * kChunkB, &tmV, &full[st], c * 64, blk * 64, bh);
+        }
+      }
+      if (*abort_flag) {
+        long long t0 = clock64();
+        if (PROJ) while (!mbar_try_wait(w_bar, 0) && clock64() - t0 < kWaitBudgetCycles) {}
+        for (int i = (n - kKpStages > 0 ? n - kKpStages : 0); i < n; ++i) {
+          t0 = clock64();
+          while (!mbar_try_wait(&full[i % kKpStages], (i / kKpStages) & 1) && clock64() - t0 < kWaitBudgetCycles) {}
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0 && mine > 0) {
+      bool ok = !PROJ || mbar_wait(w_bar, 0, abort_flag, status);
+      for (int n = 0; n < mine && ok; ++n) {
+        const int st = n % kKpStages, b = n & 1;
+        if (!(ok = mbar_wait(&full[st], (n / kKpStages) & 1, abort_flag, status))) break;
+        tc_fence_after();
+        if (PROJ) {
+          // (V_j W)^T = W^T V_j^T: M = c_out, N = t (64), K = c_in
+          constexpr uint32_t id = idesc_bf16(128, 64, true, false);
+          #pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t a = desc_mnmajor(smem_u32(sW) + kk * 2048, D * 128);
+            const uint64_t bd = desc_kmajor(smem_u32(sV(st)) + (kk >> 2) * kChunkB + (kk & 3) * 32);
+            mma_bf16_ss(tmem + kColP + b * 64, a, bd, id, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(&p_full[b]);
+        }
+        if (!(ok = mbar_wait(&conv_done[b], (n >> 1) & 1, abort_flag, status))) break;
+        if (n >= 2 && !(ok = mbar_wait(&h_free[b], ((n - 2) >> 1) & 1, abort_flag, status))) break;
+        tc_fence_after();
+        // h^T: M = c (value channel), N = a (key feature), K = t (64 tokens)
+        constexpr uint32_t id = idesc_bf16(128, D, !PROJ, true);
+        #pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint64_t a = PROJ ? desc_kmajor(smem_u32(sV(st)) + kk * 32)
+                                  : desc_mnmajor(smem_u32(sV(st)) + kk * 2048, kChunkB);
+          const uint64_t bd = desc_mnmajor(smem_u32(sK(st)) + kk * 2048, kChunkB);
+          mma_bf16_ss(tmem + kColH + b * 128, a, bd, id, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(&h_full[b]);
+        mma_commit(&empty[st]);
+      }
+      if (!ok) {
+        mma_commit(drain);
+        const long long t0 = clock64();
+        while (!mbar_try_wait(drain, 0) && clock64() - t0 < kWaitBudgetCycles) {}
+      }
+    }
+  } else {
+    // ---------------------------------------------------------------- math warps
+    const int mt = tid - 64;                       // 0..127
+    const int c = (warp & 3) * 32 + lane;          // my TMEM lane = output row
+    const uint32_t lane_addr = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+    constexpr int kCPR = D / 8, kRS = 128 / kCPR;  // 16 chunks of 8 channels, 8 row sets
+    const int g = mt % kCPR, rs = mt / kCPR;
+    const int chunk = g >> 3, q8 = g & 7;
+    bool ok = true;
+    // Drain of block m: h^T from TMEM into the staging tile, z_j from the partial sums,
+    // then two TMA stores.  Every hand-off between the 128 math threads goes through an
+    // mbarrier with a bounded wait (no named barriers), so an abort cannot strand a warp.
+    auto epilogue = [&](int m) {
+      const int b = m & 1;
+      const int blk_id = blockIdx.x + m * gridDim.x;
+      const int bh = blk_id / s.n_blocks, blk = blk_id % s.n_blocks;
+      const size_t row0 = ((size_t)bh * s.n_blocks + blk) * (D + 1);
+      // conv_done(m) completed after every math thread wrote its z partials of block m
+      bool okl = mbar_wait(&conv_done[b], (m >> 1) & 1, abort_flag, status) &&
+                 mbar_wait(&h_full[b], (m >> 1) & 1, abort_flag, status);
+      if (mt == 0 && okl) {
+        bulk_wait_read_all();                      // the previous block's stores have read the tile
+        mbar_arrive(out_free);
+      }
+      okl = okl && mbar_wait(out_free, m & 1, abort_flag, status);
+      if (!(ok = __all_sync(0xFFFFFFFFu, okl))) return;
+      tc_fence_after();
+      #pragma unroll
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t r[32];
+        tmem_ld32(lane_addr + kColH + b * 128 + cc * 32, r);
+        tmem_wait_ld();
+        uint8_t* box = sOut + (cc >> 1) * 16384;
+        #pragma unroll
+        for (int i = 0; i < 4; ++i)
+          *reinterpret_cast<uint4*>(box + sw128_offset(c, (cc & 1) * 4 + i)) =
+              make_uint4(pack_bf16(__uint_as_float(r[8 * i]), __uint_as_float(r[8 * i + 1])),
+                         pack_bf16(__uint_as_float(r[8 * i + 2]), __uint_as_float(r[8 * i + 3])),
+                         pack_bf16(__uint_as_float(r[8 * i + 4]), __uint_as_float(r[8 * i + 5])),
+                         pack_bf16(__uint_as_float(r[8 * i + 6]), __uint_as_float(r[8 * i + 7])));
+      }
+      tc_fence_before();
+      mbar_arrive(&h_free[b]);
+      {
+        float sum = 0.f;                           // z_j[a], a = mt
+        #pragma unroll
+        for (int r = 0; r < kRS; ++r) sum += zbuf[(b * kRS + r) * D + mt];
+        h[(row0 + D) * D + mt] = __float2bfloat16_rn(sum);
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(out_full);
+      if (mt == 0) {
+        if (!(ok = mbar_wait(out_full, m & 1, abort_flag, status))) return;
+        tma_store_2d(&tmH, sOut, 0, (int)row0);
+        tma_store_2d(&tmH, sOut + 16384, 64, (int)row0);
+        bulk_commit();
+      }
+    };
+    for (int n = 0; n < mine && ok; ++n) {
+      const int st = n % kKpStages, b = n & 1;
+      const int blk_id = blockIdx.x + n * gridDim.x;
+      const int blk = blk_id % s.n_blocks;
+      if (!(ok = __all_sync(0xFFFFFFFFu, mbar_wait(&full[st], (n / kKpStages) & 1, abort_flag, status)))) break;
+      // phi in place (pad tokens -> 0) and partial column sums
+      const int nvalid = block_valid_count(s, blk);
+      float z[8];
+      #pragma unroll
+      for (int i = 0; i < 8; ++i) z[i] = 0.f;
+      uint8_t* k_s = sK(st);
+      #pragma unroll 2
+      for (int t = rs; t < 64; t += kRS) {
+        uint4* pk = reinterpret_cast<uint4*>(k_s + chunk * kChunkB + sw128_offset(t, q8));
+        const uint4 u = *pk;
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+        uint32_t o[4];
+        #pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float x0 = t < nvalid ? phi_exp2(bf16_lo(w[i])) : 0.f;
+          const float x1 = t < nvalid ? phi_exp2(bf16_hi(w[i])) : 0.f;
+          z[2 * i] += x0;
+          z[2 * i + 1] += x1;
+          o[i] = pack_bf16(x0, x1);
+        }
+        *pk = make_uint4(o[0], o[1], o[2], o[3]);
+      }
+      #pragma unroll
+      for (int i = 0; i < 8; ++i) zbuf[(b * kRS + rs) * D + g * 8 + i] = z[i];
+      if (PROJ) {
+        // (V W)^T from TMEM over the V stage (V has been consumed): K-major A operand
+        if (!(ok = __all_sync(0xFFFFFFFFu, mbar_wait(&p_full[b], (n >> 1) & 1, abort_flag, status)))) break;
+        tc_fence_after();
+        uint32_t r[32], r2[32];
+        tmem_ld32(lane_addr + kColP + b * 64, r);
+        tmem_ld32(lane_addr + kColP + b * 64 + 32, r2);
+        tmem_wait_ld();
+        uint8_t* v_s = sV(st);
+        #pragma unroll
+        for (int c8 = 0; c8 < 8; ++c8) {
+          const uint32_t* src = c8 < 4 ? r : r2;
+          const int o = (c8 & 3) * 8;
+          *reinterpret_cast<uint4*>(v_s + sw128_offset(c, c8)) =
+              make_uint4(pack_bf16(__uint_as_float(src[o]), __uint_as_float(src[o + 1])),
+                         pack_bf16(__uint_as_float(src[o + 2]), __uint_as_float(src[o + 3])),
+                         pack_bf16(__uint_as_float(src[o + 4]), __uint_as_float(src[o + 5])),
+                         pack_bf16(__uint_as_float(src[o + 6]), __uint_as_float(src[o + 7])));
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(&conv_done[b]);
+      if (n >= 1) {
+        epilogue(n - 1);
+        if (!ok) break;
+      }
+    }
+    if (ok && mine > 0) epilogue(mine - 1);
+    if (mt == 0) bulk_wait_all();
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) { tc_fence_after(); tmem_dealloc(tmem, 512); }
+}
+
 // ------------------------------------------------------------------ reduce states (GEMM)
 // Persistent: one CTA per SM walks the output tiles (128 query blocks x 256
 // state columns) of every head; a 4-stage TMA ring runs across tile boundaries
@@ -537,7 +810,22 @@ cudaError_t launch_key_states(const void* k, const void* v, const void* w_proj, 
     kern<<<grid, 128, kKsSmem, st>>>(mk, mv, mw, h, s, BH, status);
     return cudaGetLastError();
   };
-  if (d == 128) return w_proj ? go(key_states_kernel<128, true>) : go(key_states_kernel<128, false>);
+  if (d == 128) {
+    // h viewed as rows of d values: [BH * Nb * (d + 1)][d]; the store boxes cover rows 0..d-1 of a block
+    CUtensorMap mh;
+    const uint64_t hdims[2] = {(uint64_t)d, (uint64_t)BH * s.n_blocks * (d + 1)};
+    const uint64_t hstr[1] = {(uint64_t)d * 2};
+    const uint32_t hbox[2] = {64, 128};
+    if (!make_tile_map(&mh, h, 2, hdims, hstr, hbox)) return cudaErrorInvalidValue;
+    const int pgrid = (int)(blocks < sms ? blocks : sms);
+    auto pipe = [&](auto kern) -> cudaError_t {
+      cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, KpLayout::kBytes);
+      if (e != cudaSuccess) return e;
+      kern<<<pgrid, 192, KpLayout::kBytes, st>>>(mk, mv, mw, mh, h, s, BH, status);
+      return cudaGetLastError();
+    };
+    return w_proj ? pipe(key_states_pipe_kernel<true>) : pipe(key_states_pipe_kernel<false>);
+  }
   return w_proj ? go(key_states_kernel<64, true>) : go(key_states_kernel<64, false>);
 }
 

@@ -113,6 +113,17 @@ __device__ __forceinline__ void tma_load_5d(void* dst, const void* desc, uint64_
       : "memory");
 }
 
+// TMA tile store from shared memory (tensor map in param space), tracked by bulk groups.
+__device__ __forceinline__ void tma_store_2d(const void* desc, const void* src, int c0, int c1) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];"
+               :: "l"(desc), "r"(smem_u32(src)), "r"(c0), "r"(c1) : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// the shared-memory sources of every committed store have been read
+__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// every committed store has completed
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 // ------------------------------------------------------------------ tcgen05
 
 // TMEM allocation: executed by one full warp; the base address lands in *slot.
