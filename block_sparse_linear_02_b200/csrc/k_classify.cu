@@ -177,7 +177,7 @@ __device__ __forceinline__ int warp_excl_scan(int v, int lane) {
 //   3. One pass in index order writes the labels and outputs; ties at a threshold
 //      go to the lower index (critical) or leave the higher index marginal
 //      (negligible), via warp prefix counts of the tied keys.
-__global__ void __launch_bounds__(kClsWarps * 32)
+__global__ void __launch_bounds__(kClsWarps * 32, 6)
 classify_kernel(const ClsArgs a) {
   extern __shared__ __align__(16) uint32_t skeys[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -187,13 +187,13 @@ classify_kernel(const ClsArgs a) {
   if (qb0 >= nb) return;
   const int nrows = qb0 + 1 < nb ? 2 : 1;
   uint32_t* rowk[2] = {skeys + (size_t)(2 * warp) * nbp, skeys + (size_t)(2 * warp + 1) * nbp};
-  uint32_t* cand = skeys + (size_t)kClsWarps * 2 * nbp + warp * (4 * kMaxCand + 4);   // [4][kMaxCand]
-  int* ccount = reinterpret_cast<int*>(cand + 4 * kMaxCand);                            // [4]
+  uint32_t* cand = skeys + (size_t)kClsWarps * 2 * nbp + warp * (4 * kMaxCand);   // [4][kMaxCand]
+  int ccount[4] = {0, 0, 0, 0};
+  const unsigned lt_mask = (1u << lane) - 1u;
   for (int r = 0; r < nrows; ++r) {
     const uint4* src = reinterpret_cast<const uint4*>(a.keys + ((size_t)bh * nb + qb0 + r) * nbp);
     for (int e = lane; e < nbp / 4; e += 32) reinterpret_cast<uint4*>(rowk[r])[e] = src[e];
   }
-  if (lane < 4) ccount[lane] = 0;
   __syncwarp();
   const int npad = nbp - nb;
 
@@ -235,8 +235,19 @@ classify_kernel(const ClsArgs a) {
         const uint32_t pk = kk[i] >> kSh;
         gt += pk > pc;
         lt += kk[i] != 0u && pk < pn;
-        if (pk == pc) { const int at = atomicAdd(&ccount[2 * r], 1); if (at < kMaxCand) cand[(2 * r) * kMaxCand + at] = kk[i]; }
-        if (kk[i] != 0u && pk == pn) { const int at = atomicAdd(&ccount[2 * r + 1], 1); if (at < kMaxCand) cand[(2 * r + 1) * kMaxCand + at] = kk[i]; }
+        // keys sharing a threshold prefix, appended in ballot order (their order is irrelevant)
+        const unsigned mc = __ballot_sync(0xFFFFFFFFu, pk == pc);
+        if (mc) {
+          const int at = ccount[2 * r] + __popc(mc & lt_mask);
+          if (pk == pc && at < kMaxCand) cand[(2 * r) * kMaxCand + at] = kk[i];
+          ccount[2 * r] += __popc(mc);
+        }
+        const unsigned mn = __ballot_sync(0xFFFFFFFFu, kk[i] != 0u && pk == pn);
+        if (mn) {
+          const int at = ccount[2 * r + 1] + __popc(mn & lt_mask);
+          if (kk[i] != 0u && pk == pn && at < kMaxCand) cand[(2 * r + 1) * kMaxCand + at] = kk[i];
+          ccount[2 * r + 1] += __popc(mn);
+        }
       }
     }
     gt_c[r] = warp_sum(gt);
@@ -324,6 +335,7 @@ classify_kernel(const ClsArgs a) {
 
   // ---- 3. labels in index order and the outputs
   int seen_c[2] = {0, 0}, seen_n[2] = {0, 0}, written[2] = {0, 0}, listed = 0;
+  (void)lt_mask;
   uint32_t* lst = a.list ? a.list + ((size_t)bh * a.n_pairs + pair) * a.list_cap : nullptr;
   for (int g = 0; g < ng; ++g) {
     const int j0 = g * 128 + lane * 4;           // my 4 keys: j0 .. j0+3
@@ -479,7 +491,7 @@ cudaError_t launch_classify(const uint32_t* keys, int BH, int nb, int d, int kc,
   a.inv_sqrt_d = (float)(1.0 / sqrt((double)d));
   a.mask = mask; a.mask_vec = (nb % 4 == 0) && (reinterpret_cast<uintptr_t>(mask) % 4 == 0); a.crit_idx = crit_idx; a.crit_cnt = crit_cnt; a.m01 = m01; a.ld_m01 = ld_m01;
   a.scores = scores; a.list = list; a.list_cnt = list_cnt; a.list_cap = list_cap; a.s = s; a.status = status;
-  const size_t smem = ((size_t)2 * kClsWarps * a.nbp + kClsWarps * (4 * kMaxCand + 4)) * sizeof(uint32_t);
+  const size_t smem = ((size_t)2 * kClsWarps * a.nbp + kClsWarps * 4 * kMaxCand) * sizeof(uint32_t);
   cudaError_t e = cudaFuncSetAttribute(classify_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid((a.n_pairs + kClsWarps - 1) / kClsWarps, BH);

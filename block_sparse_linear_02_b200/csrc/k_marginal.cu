@@ -240,12 +240,12 @@ key_states_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
 }
 
 // ------------------------------------------------------------------ key states, d = 128
-// Warp-specialised and persistent (one CTA per SM): warp 0 streams K_j, V_j into a
-// 3-stage ring, warp 1 issues the MMAs, warps 2-5 (128 threads) apply phi in place,
-// form the column sums z_j, move (V_j W)^T from TMEM into the operand layout of the
-// second MMA, and drain h_j'^T from TMEM into a swizzled staging tile that two TMA
-// stores write out.  TMEM holds two (V W)^T and two h^T accumulators, so block n's
-// drain overlaps block n+1's MMAs.
+// Warp-specialised and persistent (one CTA per SM, 320 threads): warp 0 streams K_j,
+// V_j into a 3-stage ring; warp 1 issues the MMAs; warps 2-5 apply phi in place, form
+// z_j and move (V_j W)^T from TMEM into the operand layout of the second MMA; warps 6-9
+// drain h_j'^T from TMEM into a swizzled staging tile that two TMA stores write out.
+// TMEM holds two (V W)^T and two h^T accumulators, so block n's drain overlaps block
+// n+1's phi and MMAs.  Every hand-off goes through an mbarrier with a bounded wait.
 constexpr int kKpStages = 3;
 struct KpLayout {
   static constexpr int kW = 0;                               // W_proj MN-major, 2 chunks x 16 KB
@@ -266,7 +266,7 @@ __device__ __forceinline__ float phi_exp2(float x) {
 
 
 template <bool PROJ>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
 key_states_pipe_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                        const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmH,
                        __nv_bfloat16* __restrict__ h, SeqShape s, int BH, int* status) {
@@ -287,7 +287,8 @@ key_states_pipe_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_con
   uint64_t* h_free = h_full + 2;                  // [2] h^T drained (128 arrivals)
   uint64_t* out_free = h_free + 2;                // staging tile read by the previous stores
   uint64_t* out_full = out_free + 1;              // staging tile written (128 arrivals)
-  uint64_t* drain = out_full + 1;
+  uint64_t* z_ready = out_full + 1;               // [2] z partials of a block written (128 arrivals)
+  uint64_t* drain = z_ready + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -310,6 +311,8 @@ key_states_pipe_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_con
     }
     mbar_init(out_free, 1);
     mbar_init(out_full, 128);
+    mbar_init(&z_ready[0], 128);
+    mbar_init(&z_ready[1], 128);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -389,68 +392,19 @@ key_states_pipe_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_con
         while (!mbar_try_wait(drain, 0) && clock64() - t0 < kWaitBudgetCycles) {}
       }
     }
-  } else {
-    // ---------------------------------------------------------------- math warps
-    const int mt = tid - 64;                       // 0..127
-    const int c = (warp & 3) * 32 + lane;          // my TMEM lane = output row
+  } else if (warp < 6) {
+    // ---------------------------------------------------------------- phi warps
+    const int pt = tid - 64;                       // 0..127
+    const int c = (warp & 3) * 32 + lane;          // my TMEM lane = row of (V W)^T
     const uint32_t lane_addr = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     constexpr int kCPR = D / 8, kRS = 128 / kCPR;  // 16 chunks of 8 channels, 8 row sets
-    const int g = mt % kCPR, rs = mt / kCPR;
+    const int g = pt % kCPR, rs = pt / kCPR;
     const int chunk = g >> 3, q8 = g & 7;
     bool ok = true;
-    // Drain of block m: h^T from TMEM into the staging tile, z_j from the partial sums,
-    // then two TMA stores.  Every hand-off between the 128 math threads goes through an
-    // mbarrier with a bounded wait (no named barriers), so an abort cannot strand a warp.
-    auto epilogue = [&](int m) {
-      const int b = m & 1;
-      const int blk_id = blockIdx.x + m * gridDim.x;
-      const int bh = blk_id / s.n_blocks, blk = blk_id % s.n_blocks;
-      const size_t row0 = ((size_t)bh * s.n_blocks + blk) * (D + 1);
-      // conv_done(m) completed after every math thread wrote its z partials of block m
-      bool okl = mbar_wait(&conv_done[b], (m >> 1) & 1, abort_flag, status) &&
-                 mbar_wait(&h_full[b], (m >> 1) & 1, abort_flag, status);
-      if (mt == 0 && okl) {
-        bulk_wait_read_all();                      // the previous block's stores have read the tile
-        mbar_arrive(out_free);
-      }
-      okl = okl && mbar_wait(out_free, m & 1, abort_flag, status);
-      if (!(ok = __all_sync(0xFFFFFFFFu, okl))) return;
-      tc_fence_after();
-      #pragma unroll
-      for (int cc = 0; cc < D / 32; ++cc) {
-        uint32_t r[32];
-        tmem_ld32(lane_addr + kColH + b * 128 + cc * 32, r);
-        tmem_wait_ld();
-        uint8_t* box = sOut + (cc >> 1) * 16384;
-        #pragma unroll
-        for (int i = 0; i < 4; ++i)
-          *reinterpret_cast<uint4*>(box + sw128_offset(c, (cc & 1) * 4 + i)) =
-              make_uint4(pack_bf16(__uint_as_float(r[8 * i]), __uint_as_float(r[8 * i + 1])),
-                         pack_bf16(__uint_as_float(r[8 * i + 2]), __uint_as_float(r[8 * i + 3])),
-                         pack_bf16(__uint_as_float(r[8 * i + 4]), __uint_as_float(r[8 * i + 5])),
-                         pack_bf16(__uint_as_float(r[8 * i + 6]), __uint_as_float(r[8 * i + 7])));
-      }
-      tc_fence_before();
-      mbar_arrive(&h_free[b]);
-      {
-        float sum = 0.f;                           // z_j[a], a = mt
-        #pragma unroll
-        for (int r = 0; r < kRS; ++r) sum += zbuf[(b * kRS + r) * D + mt];
-        h[(row0 + D) * D + mt] = __float2bfloat16_rn(sum);
-      }
-      fence_proxy_async_smem();
-      mbar_arrive(out_full);
-      if (mt == 0) {
-        if (!(ok = mbar_wait(out_full, m & 1, abort_flag, status))) return;
-        tma_store_2d(&tmH, sOut, 0, (int)row0);
-        tma_store_2d(&tmH, sOut + 16384, 64, (int)row0);
-        bulk_commit();
-      }
-    };
     for (int n = 0; n < mine && ok; ++n) {
       const int st = n % kKpStages, b = n & 1;
       const int blk_id = blockIdx.x + n * gridDim.x;
-      const int blk = blk_id % s.n_blocks;
+      const int bh = blk_id / s.n_blocks, blk = blk_id % s.n_blocks;
       if (!(ok = __all_sync(0xFFFFFFFFu, mbar_wait(&full[st], (n / kKpStages) & 1, abort_flag, status)))) break;
       // phi in place (pad tokens -> 0) and partial column sums
       const int nvalid = block_valid_count(s, blk);
@@ -458,8 +412,9 @@ key_states_pipe_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_con
       #pragma unroll
       for (int i = 0; i < 8; ++i) z[i] = 0.f;
       uint8_t* k_s = sK(st);
-      #pragma unroll 2
-      for (int t = rs; t < 64; t += kRS) {
+      #pragma unroll
+      for (int tt = 0; tt < 64 / kRS; ++tt) {
+        const int t = rs + tt * kRS;
         uint4* pk = reinterpret_cast<uint4*>(k_s + chunk * kChunkB + sw128_offset(t, q8));
         const uint4 u = *pk;
         const uint32_t w[4] = {u.x, u.y, u.z, u.w};
@@ -476,6 +431,7 @@ key_states_pipe_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_con
       }
       #pragma unroll
       for (int i = 0; i < 8; ++i) zbuf[(b * kRS + rs) * D + g * 8 + i] = z[i];
+      mbar_arrive(&z_ready[b]);
       if (PROJ) {
         // (V W)^T from TMEM over the V stage (V has been consumed): K-major A operand
         if (!(ok = __all_sync(0xFFFFFFFFu, mbar_wait(&p_full[b], (n >> 1) & 1, abort_flag, status)))) break;
@@ -499,13 +455,58 @@ key_states_pipe_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_con
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&conv_done[b]);
-      if (n >= 1) {
-        epilogue(n - 1);
-        if (!ok) break;
+      // z_j[a], a = pt, once every phi thread has written its partials
+      if (!(ok = mbar_wait(&z_ready[b], (n >> 1) & 1, abort_flag, status))) break;
+      float sum = 0.f;
+      #pragma unroll
+      for (int r = 0; r < kRS; ++r) sum += zbuf[(b * kRS + r) * D + pt];
+      h[(((size_t)bh * s.n_blocks + blk) * (D + 1) + D) * D + pt] = __float2bfloat16_rn(sum);
+    }
+  } else {
+    // ---------------------------------------------------------------- drain warps
+    const int dt = tid - 192;                      // 0..127
+    const int c = (warp & 3) * 32 + lane;          // my TMEM lane = row of h^T
+    const uint32_t lane_addr = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+    bool ok = true;
+    for (int m = 0; m < mine && ok; ++m) {
+      const int b = m & 1;
+      const int blk_id = blockIdx.x + m * gridDim.x;
+      const int bh = blk_id / s.n_blocks, blk = blk_id % s.n_blocks;
+      const int row0 = (int)(((size_t)bh * s.n_blocks + blk) * (D + 1));
+      bool okl = mbar_wait(&h_full[b], (m >> 1) & 1, abort_flag, status);
+      if (dt == 0 && okl) {
+        bulk_wait_read_all();                      // the previous block's stores have read the tile
+        mbar_arrive(out_free);
+      }
+      okl = okl && mbar_wait(out_free, m & 1, abort_flag, status);
+      if (!(ok = __all_sync(0xFFFFFFFFu, okl))) break;
+      tc_fence_after();
+      #pragma unroll
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t r[32];
+        tmem_ld32(lane_addr + kColH + b * 128 + cc * 32, r);
+        tmem_wait_ld();
+        uint8_t* box = sOut + (cc >> 1) * 16384;
+        #pragma unroll
+        for (int i = 0; i < 4; ++i)
+          *reinterpret_cast<uint4*>(box + sw128_offset(c, (cc & 1) * 4 + i)) =
+              make_uint4(pack_bf16(__uint_as_float(r[8 * i]), __uint_as_float(r[8 * i + 1])),
+                         pack_bf16(__uint_as_float(r[8 * i + 2]), __uint_as_float(r[8 * i + 3])),
+                         pack_bf16(__uint_as_float(r[8 * i + 4]), __uint_as_float(r[8 * i + 5])),
+                         pack_bf16(__uint_as_float(r[8 * i + 6]), __uint_as_float(r[8 * i + 7])));
+      }
+      tc_fence_before();
+      mbar_arrive(&h_free[b]);
+      fence_proxy_async_smem();
+      mbar_arrive(out_full);
+      if (dt == 0) {
+        if (!(ok = mbar_wait(out_full, m & 1, abort_flag, status))) break;
+        tma_store_2d(&tmH, sOut, 0, row0);
+        tma_store_2d(&tmH, sOut + 16384, 64, row0);
+        bulk_commit();
       }
     }
-    if (ok && mine > 0) epilogue(mine - 1);
-    if (mt == 0) bulk_wait_all();
+    if (dt == 0) bulk_wait_all();
   }
   tc_fence_before();
   __syncthreads();
@@ -821,7 +822,7 @@ cudaError_t launch_key_states(const void* k, const void* v, const void* w_proj, 
     auto pipe = [&](auto kern) -> cudaError_t {
       cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, KpLayout::kBytes);
       if (e != cudaSuccess) return e;
-      kern<<<pgrid, 192, KpLayout::kBytes, st>>>(mk, mv, mw, mh, h, s, BH, status);
+      kern<<<pgrid, 320, KpLayout::kBytes, st>>>(mk, mv, mw, mh, h, s, BH, status);
       return cudaGetLastError();
     };
     return w_proj ? pipe(key_states_pipe_kernel<true>) : pipe(key_states_pipe_kernel<false>);
