@@ -240,10 +240,11 @@ key_states_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
 }
 
 // ------------------------------------------------------------------ key states, d = 128
-// Warp-specialised and persistent (one CTA per SM, 320 threads): warp 0 streams K_j,
-// V_j into a 3-stage ring; warp 1 issues the MMAs; warps 2-5 apply phi in place, form
-// z_j and move (V_j W)^T from TMEM into the operand layout of the second MMA; warps 6-9
-// drain h_j'^T from TMEM into a swizzled staging tile that two TMA stores write out.
+// Warp-specialised and persistent (one CTA per SM, 448 threads): warp 0 streams K_j,
+// V_j into a 3-stage ring; warp 1 issues the MMAs; warps 2-9 apply phi in place and
+// form z_j, warps 2-5 also move (V_j W)^T from TMEM into the operand layout of the
+// second MMA; warps 10-13 drain h_j'^T from TMEM into a swizzled staging tile that two
+// TMA stores write out.
 // TMEM holds two (V W)^T and two h^T accumulators, so block n's drain overlaps block
 // n+1's phi and MMAs.  Every hand-off goes through an mbarrier with a bounded wait.
 constexpr int kKpStages = 3;
@@ -252,21 +253,22 @@ struct KpLayout {
   static constexpr int kRing = 32768;                        // stages: K 16 KB | V 16 KB
   static constexpr int kStage = 32768;
   static constexpr int kOut = kRing + kKpStages * kStage;    // h^T staging: 2 boxes of 64 columns
-  static constexpr int kZ = kOut + 32768;                    // z partials [2][8][128] floats
-  static constexpr int kBar = kZ + 2 * 8 * 128 * 4;
+  static constexpr int kZ = kOut + 32768;                    // z partials [2][16][128] floats
+  static constexpr int kBar = kZ + 2 * 16 * 128 * 4;
   static constexpr int kBytes = kBar + 256 + 1024;
 };
 
 __device__ __forceinline__ float phi_exp2(float x) {
-  // elu(x) + 1; exp through the exp2 unit (the result is rounded to bf16)
+  // elu(x) + 1 = exp(min(x, 0)) + max(x, 0), branch-free; exp through the exp2 unit
+  // (the result is rounded to bf16)
   float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x * 1.4426950408889634f));
-  return x > 0.f ? x + 1.f : y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(fminf(x, 0.f) * 1.4426950408889634f));
+  return y + fmaxf(x, 0.f);
 }
 
 
 template <bool PROJ>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(448, 1)
 key_states_pipe_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                        const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmH,
                        __nv_bfloat16* __restrict__ h, SeqShape s, int BH, int* status) {
@@ -282,12 +284,12 @@ key_states_pipe_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_con
   uint64_t* empty = full + kKpStages;             // [3] stage consumed by the second MMA
   uint64_t* w_bar = empty + kKpStages;
   uint64_t* p_full = w_bar + 1;                   // [2] (V W)^T in TMEM
-  uint64_t* conv_done = p_full + 2;               // [2] operands of the second MMA ready (128 arrivals)
+  uint64_t* conv_done = p_full + 2;               // [2] operands of the second MMA ready (256 arrivals)
   uint64_t* h_full = conv_done + 2;               // [2] h^T in TMEM
   uint64_t* h_free = h_full + 2;                  // [2] h^T drained (128 arrivals)
   uint64_t* out_free = h_free + 2;                // staging tile read by the previous stores
   uint64_t* out_full = out_free + 1;              // staging tile written (128 arrivals)
-  uint64_t* z_ready = out_full + 1;               // [2] z partials of a block written (128 arrivals)
+  uint64_t* z_ready = out_full + 1;               // [2] z partials of a block written (256 arrivals)
   uint64_t* drain = z_ready + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -305,14 +307,14 @@ key_states_pipe_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_con
     mbar_init(w_bar, 1);
     for (int b = 0; b < 2; ++b) {
       mbar_init(&p_full[b], 1);
-      mbar_init(&conv_done[b], 128);
+      mbar_init(&conv_done[b], 256);
       mbar_init(&h_full[b], 1);
       mbar_init(&h_free[b], 128);
     }
     mbar_init(out_free, 1);
     mbar_init(out_full, 128);
-    mbar_init(&z_ready[0], 128);
-    mbar_init(&z_ready[1], 128);
+    mbar_init(&z_ready[0], 256);
+    mbar_init(&z_ready[1], 256);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -392,12 +394,13 @@ key_states_pipe_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_con
         while (!mbar_try_wait(drain, 0) && clock64() - t0 < kWaitBudgetCycles) {}
       }
     }
-  } else if (warp < 6) {
+  } else if (warp < 10) {
     // ---------------------------------------------------------------- phi warps
-    const int pt = tid - 64;                       // 0..127
+    const int pt = tid - 64;                       // 0..255
+    const bool conv = warp < 6;                    // warps 2-5 also move (V W)^T
     const int c = (warp & 3) * 32 + lane;          // my TMEM lane = row of (V W)^T
     const uint32_t lane_addr = tmem + ((uint32_t)((warp & 3) * 32) << 16);
-    constexpr int kCPR = D / 8, kRS = 128 / kCPR;  // 16 chunks of 8 channels, 8 row sets
+    constexpr int kCPR = D / 8, kRS = 256 / kCPR;  // 16 chunks of 8 channels, 16 row sets
     const int g = pt % kCPR, rs = pt / kCPR;
     const int chunk = g >> 3, q8 = g & 7;
     bool ok = true;
@@ -432,7 +435,7 @@ key_states_pipe_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_con
       #pragma unroll
       for (int i = 0; i < 8; ++i) zbuf[(b * kRS + rs) * D + g * 8 + i] = z[i];
       mbar_arrive(&z_ready[b]);
-      if (PROJ) {
+      if (PROJ && conv) {
         // (V W)^T from TMEM over the V stage (V has been consumed): K-major A operand
         if (!(ok = __all_sync(0xFFFFFFFFu, mbar_wait(&p_full[b], (n >> 1) & 1, abort_flag, status)))) break;
         tc_fence_after();
@@ -457,14 +460,16 @@ key_states_pipe_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_con
       mbar_arrive(&conv_done[b]);
       // z_j[a], a = pt, once every phi thread has written its partials
       if (!(ok = mbar_wait(&z_ready[b], (n >> 1) & 1, abort_flag, status))) break;
-      float sum = 0.f;
-      #pragma unroll
-      for (int r = 0; r < kRS; ++r) sum += zbuf[(b * kRS + r) * D + pt];
-      h[(((size_t)bh * s.n_blocks + blk) * (D + 1) + D) * D + pt] = __float2bfloat16_rn(sum);
+      if (pt < D) {
+        float sum = 0.f;
+        #pragma unroll
+        for (int r = 0; r < kRS; ++r) sum += zbuf[(b * kRS + r) * D + pt];
+        h[(((size_t)bh * s.n_blocks + blk) * (D + 1) + D) * D + pt] = __float2bfloat16_rn(sum);
+      }
     }
   } else {
     // ---------------------------------------------------------------- drain warps
-    const int dt = tid - 192;                      // 0..127
+    const int dt = tid - 320;                      // 0..127
     const int c = (warp & 3) * 32 + lane;          // my TMEM lane = row of h^T
     const uint32_t lane_addr = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     bool ok = true;
@@ -822,7 +827,7 @@ cudaError_t launch_key_states(const void* k, const void* v, const void* w_proj, 
     auto pipe = [&](auto kern) -> cudaError_t {
       cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, KpLayout::kBytes);
       if (e != cudaSuccess) return e;
-      kern<<<pgrid, 320, KpLayout::kBytes, st>>>(mk, mv, mw, mh, h, s, BH, status);
+      kern<<<pgrid, 448, KpLayout::kBytes, st>>>(mk, mv, mw, mh, h, s, BH, status);
       return cudaGetLastError();
     };
     return w_proj ? pipe(key_states_pipe_kernel<true>) : pipe(key_states_pipe_kernel<false>);
