@@ -94,8 +94,9 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-// phi(x) = elu(x) + 1, with exp through the exp2 unit (the result is rounded to bf16)
-__device__ __forceinline__ float phi_fast(float x) { return x > 0.f ? x + 1.f : ex2(x * kLog2e); }
+// phi(x) = elu(x) + 1 = exp(min(x, 0)) + max(x, 0), branch-free, exp through the exp2
+// unit (the result is rounded to bf16)
+__device__ __forceinline__ float phi_fast(float x) { return ex2(fminf(x, 0.f) * kLog2e) + fmaxf(x, 0.f); }
 
 __device__ __forceinline__ float max3(float a, float b, float c) {
   float r;
@@ -432,8 +433,9 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
 
     // ---- linear branch first (LINEAR): phi(Q) into ring slot 2 (pad rows -> 0; Q stays in
     // place for the QK MMAs), then the MMA warp's lin = phi(Q) [H'^T ; Z]^T lands in the O
-    // columns; my half of the row, divided by its denominator, is kept in registers as
-    // bf16 pairs (the output is rounded to bf16 in the end as well)
+    // columns; my half of the row, divided by its denominator, is read during the first
+    // step (before its P is handed over, since the first P.V overwrites those columns) and
+    // kept in registers as bf16 pairs (the output is rounded to bf16 in the end as well)
     uint32_t lin[D / 4];
     #pragma unroll
     for (int i = 0; i < D / 4; ++i) lin[i] = 0u;
@@ -457,26 +459,28 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
       }
       fence_proxy_async_smem();
       mbar_arrive(phiq_ready);
+    }
+    bool lin_pending = LINEAR;
+    auto read_lin = [&]() {
+      lin_pending = false;
       if (ok) ok = __all_sync(0xFFFFFFFFu, mbar_wait(lin_done, 0, abort_flag, p.status));
       tc_fence_after();
-      if (ok) {
-        uint32_t dv;
-        tmem_ld1(lane_addr + kColLinOut + D, dv);
+      if (!ok) return;
+      uint32_t dv;
+      tmem_ld1(lane_addr + kColLinOut + D, dv);
+      tmem_wait_ld();
+      const float den = __uint_as_float(dv);
+      const float inv_den = den > 0.f ? 1.f / den : 0.f;
+      #pragma unroll
+      for (int k = 0; k < D / 64; ++k) {
+        uint32_t t[32];
+        tmem_ld32(lane_addr + kColLinOut + wg * (D / 2) + k * 32, t);
         tmem_wait_ld();
-        const float den = __uint_as_float(dv);
-        const float inv_den = den > 0.f ? 1.f / den : 0.f;
         #pragma unroll
-        for (int k = 0; k < D / 64; ++k) {
-          uint32_t t[32];
-          tmem_ld32(lane_addr + kColLinOut + wg * (D / 2) + k * 32, t);
-          tmem_wait_ld();
-          #pragma unroll
-          for (int i = 0; i < 16; ++i)
-            lin[k * 16 + i] = pack_bf16(__uint_as_float(t[2 * i]) * inv_den, __uint_as_float(t[2 * i + 1]) * inv_den);
-        }
+        for (int i = 0; i < 16; ++i)
+          lin[k * 16 + i] = pack_bf16(__uint_as_float(t[2 * i]) * inv_den, __uint_as_float(t[2 * i + 1]) * inv_den);
       }
-      tc_fence_before();   // the first P.V overwrites these columns after p_full
-    }
+    };
     for (int j = 0; j < n_steps && ok; ++j) {
       const int b = j & 1;
       const bool far = GATED && j == local_steps;
@@ -486,6 +490,10 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
       if (!__all_sync(0xFFFFFFFFu, mbar_wait(&s_full[b], (j >> 1) & 1, abort_flag, p.status))) { ok = false; break; }
       tc_fence_after();
       if (!mine) {
+        if (LINEAR && j == 0) {
+          read_lin();
+          if (!ok) break;
+        }
         tc_fence_before();
         mbar_arrive(&p_full[b]);
         continue;
@@ -565,12 +573,17 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
           tmem_st32(lane_addr + my_o + cc * 32, o);
         }
       }
+      if (LINEAR && j == 0) {
+        read_lin();
+        if (!ok) break;
+      }
       tmem_st32(s_addr, packed);          // P (bf16 pairs) over the first 32 columns of my S block
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&p_full[b]);
       if (!far) started = true;
     }
+    if (LINEAR && lin_pending) read_lin();         // no step read it
     if (ok && n_steps > 0)
       ok = __all_sync(0xFFFFFFFFu, mbar_wait(&pv_done[(n_steps - 1) & 3], ((n_steps - 1) >> 2) & 1, abort_flag, p.status));
     ok = __all_sync(0xFFFFFFFFu, ok);
