@@ -504,32 +504,6 @@ slr_status slr_linear_marginal(const void* q, const void* k, const void* v, cons
   return SLR_OK;
 }
 
-// A second stream per host thread and device on which the SLA call runs the key-block
-// states (they depend on K, V and W_proj only) beside the pooling and classification
-// chain.  The call forks it from the caller's stream with an event and joins it back
-// before the states are reduced, so the caller's stream order is kept and the call
-// stays capturable into a CUDA graph.  Thread-local, so concurrent host threads never
-// share the events.
-struct SideStream {
-  cudaStream_t s = nullptr;
-  cudaEvent_t fork = nullptr, join = nullptr;
-};
-constexpr int kMaxSideDevices = 64;
-thread_local SideStream t_side[kMaxSideDevices];
-
-SideStream* side_stream() {
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxSideDevices) return nullptr;
-  SideStream& ss = t_side[dev];
-  if (!ss.s) {
-    if (cudaStreamCreateWithFlags(&ss.s, cudaStreamNonBlocking) != cudaSuccess) { ss.s = nullptr; return nullptr; }
-    if (cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming) != cudaSuccess ||
-        cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming) != cudaSuccess)
-      return nullptr;
-  }
-  return &ss;
-}
-
 slr_status slr_sparse_linear_attn(const void* q, const void* k, const void* v, const void* w_proj,
                                   const slr_seq* seq, float crit_frac, float negl_frac, int phi,
                                   void* out, int8_t* mask_out_opt, void* ws, size_t ws_bytes, void* stream) {
@@ -559,22 +533,11 @@ slr_status slr_sparse_linear_attn(const void* q, const void* k, const void* v, c
   }
   SLR_LAUNCH(kKPool, s, launch_pool_means(q, k, w.cls.qsplit, w.cls.ksplit, sh.BH, sh.d, sh.s, s));
   SLR_LAUNCH(kKLogits, s, launch_logits(w.cls.qsplit, w.cls.ksplit, w.cls.keys, sh.BH, sh.nb, sh.d, w.status, s));
-  // the key states run beside the classification kernel (which fits next to them on an
-  // SM; the logits GEMM does not, so the fork comes after it)
-  SideStream* side = nullptr;
-  if (marginal) {
-    side = side_stream();
-    if (!side) return SLR_ERR_CUDA;
-    SLR_TRY(cudaEventRecord(side->fork, s));
-    SLR_TRY(cudaStreamWaitEvent(side->s, side->fork, 0));
-    SLR_LAUNCH(kKKeyStates, side->s, launch_key_states(k, v, w_proj, w.mar.h, sh.BH, sh.d, sh.s, w.status, side->s));
-    SLR_TRY(cudaEventRecord(side->join, side->s));
-  }
   SLR_LAUNCH(kKClassify, s, launch_classify(w.cls.keys, sh.BH, sh.nb, sh.d, kc, kn, mask_out_opt, nullptr,
                                             nullptr, w.cls.m01, ld_m01(sh.nb), nullptr, w.list, w.list_cnt, w.cap,
                                             sh.s, w.status, s));
   if (marginal) {
-    SLR_TRY(cudaStreamWaitEvent(s, side->join, 0));
+    SLR_LAUNCH(kKKeyStates, s, launch_key_states(k, v, w_proj, w.mar.h, sh.BH, sh.d, sh.s, w.status, s));
     SLR_LAUNCH(kKReduce, s, launch_reduce_states(w.cls.m01, ld_m01(sh.nb), w.mar.h, w.mar.Hs, sh.BH, sh.nb, sh.d, w.status, s));
     a.Hs = w.mar.Hs;
   }
