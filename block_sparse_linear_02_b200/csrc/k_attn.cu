@@ -62,8 +62,8 @@ struct AttnLayout {
   static constexpr int kQOff = 0;
   static constexpr int kRingOff = kQOff + kChunks * kTile;
   static constexpr int kZOff = kRingOff + kSlots * kKV;  // Z tiles of the pair's two query blocks
-  static constexpr int kXOff = kZOff + 2 * kZTile;       // exchange area: 6 x 128 floats
-  static constexpr int kBarOff = kXOff + 6 * 128 * 4;
+  static constexpr int kXOff = kZOff + 2 * kZTile;       // exchange area: [2 shares][2 tiles][3][128] floats
+  static constexpr int kBarOff = kXOff + 12 * 128 * 4;
   static constexpr int kBytes = kBarOff + 256 + 1024;    // + alignment slack
   static_assert(kHsTile <= kKV, "a linear state tile must fit in one ring slot");
   static_assert(kBytes <= 227 * 1024, "shared memory budget");
@@ -79,7 +79,11 @@ struct AttnKParams {
   int F, Hh, Ww, TF, TH, TW;
   float gate, scale_log2;
   int* status;
+  int n_tiles;            // heads x pairs
+  int* tile_counter;      // global tile queue, zero at launch
 };
+
+constexpr int kTq = 4;    // tile-index slots between the producer and the other roles
 
 __device__ __forceinline__ void tile_coords(int tile, int TF, int TW, int& tf, int& th, int& tw) {
   tf = tile % TF;
@@ -103,8 +107,6 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
   asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
   return r;
 }
-
-__device__ __forceinline__ void softmax_bar() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 
 __device__ __forceinline__ void tmem_ld1(uint32_t taddr, uint32_t& r) {
   asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(r) : "r"(taddr));
@@ -151,6 +153,38 @@ __device__ __forceinline__ Entry read_entry(const uint32_t* list, int idx, const
   return e;
 }
 
+// Per-tile quantities every role derives from the tile index.
+struct TileInfo {
+  int bh, pair;
+  const uint32_t* list;            // null = every key block (dense)
+  int n_local, local_steps, n_steps, n_lin;
+  bool second_exists;
+};
+
+template <bool GATED, bool LINEAR>
+__device__ __forceinline__ TileInfo tile_info(int t, const AttnKParams& p) {
+  TileInfo ti;
+  ti.bh = t / p.n_pairs;
+  ti.pair = t % p.n_pairs;
+  ti.list = nullptr;
+  ti.n_local = p.n_kb;
+  if (p.list) {
+    const size_t off = (p.list_per_head ? (size_t)ti.bh * p.n_pairs : 0) + ti.pair;
+    ti.list = p.list + off * p.list_cap;
+    ti.n_local = p.list_cnt[off];
+  }
+  ti.local_steps = (ti.n_local + 1) >> 1;
+  ti.n_steps = ti.local_steps + (GATED ? 1 : 0);   // the far block is a step of its own
+  ti.second_exists = 2 * ti.pair + 1 < p.n_qb;
+  ti.n_lin = LINEAR ? (ti.second_exists ? 2 : 1) : 0;
+  return ti;
+}
+
+// Persistent: one CTA per SM takes tiles (head, pair of query blocks) from a global
+// queue.  The producer fetches the next tile index as soon as it has issued the current
+// tile's loads and hands it to the other roles through a small ring of tile slots, so
+// the next tile's Q, linear states and first K/V blocks load while the current tile
+// finishes.  Ring positions, step counters and the per-tile barriers run on across tiles.
 template <int D, bool TILE, bool GATED, bool LINEAR>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -164,48 +198,36 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
   uint8_t* sQ = smem + L::kQOff;
   uint8_t* sRing = smem + L::kRingOff;
   uint8_t* sZ = smem + L::kZOff;
-  float* xch = reinterpret_cast<float*>(smem + L::kXOff);   // [6][128]: m0 m1 l0 l1 far-l spare
+  float* xch = reinterpret_cast<float*>(smem + L::kXOff);   // [2 tiles][3][128]: m, l, far-l per warpgroup share
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
-  uint64_t* q_full = bars + 0;
-  uint64_t* slot_full = bars + 1;                // [kSlots] TMA landed in a ring slot
+  uint64_t* q_full = bars + 0;                   // Q (and Z) of the current tile landed
+  uint64_t* q_free = q_full + 1;                 // every MMA reading Q / Z of a tile has completed
+  uint64_t* slot_full = q_free + 1;              // [kSlots] ring slot filled (TMA, or freed for phi(Q))
   uint64_t* s_full = slot_full + kSlots;         // [2] per S buffer
   uint64_t* p_full = s_full + 2;                 // [2] per S buffer, 256 arrivals
   uint64_t* pv_done = p_full + 2;                // [4] per step mod 4 (phases cannot alias)
-  uint64_t* phiq_ready = pv_done + 4;
+  uint64_t* phiq_ready = pv_done + 4;            // 256 arrivals per tile
   uint64_t* lin_done = phiq_ready + 1;
-  uint64_t* drain = lin_done + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* o_free = lin_done + 1;               // the epilogue has read O_0/O_1 (256 arrivals per tile)
+  uint64_t* xch_bar = o_free + 1;                // both shares of every row published (256 arrivals per tile)
+  uint64_t* tq_full = xch_bar + 1;               // [kTq] tile slot written
+  uint64_t* tq_empty = tq_full + kTq;            // [kTq] tile slot read (MMA thread + one lane per softmax warp)
+  uint64_t* drain = tq_empty + kTq;
+  int* tq = reinterpret_cast<int*>(drain + 1);   // [kTq] tile indices
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tq + kTq);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int pair = blockIdx.x, bh = blockIdx.y;
   constexpr uint32_t kTmemCols = 512;
   const SeqShape seq{p.n_pad, p.seg_len, p.seg_stride, p.n_kb};
-
-  const uint32_t* list = nullptr;
-  int n_local = p.n_kb;
-  if (p.list) {
-    size_t off = (p.list_per_head ? (size_t)bh * p.n_pairs : 0) + pair;
-    list = p.list + off * p.list_cap;
-    n_local = p.list_cnt[off];
-  }
-  const int local_steps = (n_local + 1) >> 1;
-  const int n_steps = local_steps + (GATED ? 1 : 0);   // the far block is a step of its own
-  const bool second_exists = 2 * pair + 1 < p.n_qb;
-  const int n_lin = LINEAR ? (second_exists ? 2 : 1) : 0;   // linear state tiles
-  // LINEAR: ring slots 0 and 1 first hold the H'^T rows of the two query blocks and
-  // slot 2 holds phi(Q); K/V item i then takes ring position i + kPre
+  // LINEAR: a tile's first three ring positions hold the H'^T rows of its two query
+  // blocks and phi(Q); its K/V items follow
   constexpr int kPre = LINEAR ? 3 : 0;
   constexpr uint32_t kColLinOut = kColO0;   // lin (+ denominator at column D) before O_0/O_1 are first written
-  const bool active = n_steps > 0 || LINEAR;
-  // blocks in step j: 2, except an odd tail (1) and the far step (1, handled by warpgroup 0)
-  auto step_blocks = [&](int j) -> int {
-    if (GATED && j == local_steps) return 1;
-    return (2 * j + 1 < n_local) ? 2 : 1;
-  };
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
+    mbar_init(q_free, 1);
     for (int s = 0; s < kSlots; ++s) mbar_init(&slot_full[s], 1);
     for (int b = 0; b < 2; ++b) {
       mbar_init(&s_full[b], 1);
@@ -214,6 +236,9 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
     for (int b = 0; b < 4; ++b) mbar_init(&pv_done[b], 1);
     mbar_init(phiq_ready, 256);
     mbar_init(lin_done, 1);
+    mbar_init(o_free, 256);
+    mbar_init(xch_bar, 256);
+    for (int e = 0; e < kTq; ++e) { mbar_init(&tq_full[e], 1); mbar_init(&tq_empty[e], 9); }
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -226,91 +251,119 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
 
   if (warp == 8) {
     // ---------------------------------------------------------------- producer
-    if (lane == 0 && active) {
+    if (lane == 0) {
       tma_prefetch_desc(&tmQ); tma_prefetch_desc(&tmK); tma_prefetch_desc(&tmV);
-      mbar_arrive_expect_tx(q_full, L::kChunks * L::kTile + n_lin * L::kZTile);
-      if (TILE) {
-        for (int half = 0; half < 2; ++half) {
-          int tf, th, tw;
-          tile_coords(2 * pair + half, p.TF, p.TW, tf, th, tw);
+      // how the current occupant of each ring slot is released: kind 0 = the P.V of
+      // global step idx, kind 1 = the linear-branch MMAs of local tile idx, -1 = free
+      int rel_kind[kSlots], rel_idx[kSlots];
+      #pragma unroll
+      for (int s = 0; s < kSlots; ++s) { rel_kind[s] = -1; rel_idx[s] = 0; }
+      auto slot_released = [&](int slot) -> bool {
+        if (rel_kind[slot] == 0) {
+          const int q = rel_idx[slot];
+          return mbar_wait(&pv_done[q & 3], (q >> 2) & 1, abort_flag, p.status);
+        }
+        if (rel_kind[slot] == 1) return mbar_wait(lin_done, rel_idx[slot] & 1, abort_flag, p.status);
+        return true;
+      };
+      int i = 0, J = 0, g = 0, q_loaded = -1;
+      bool ok = true;
+      while (ok) {
+        int t = atomicAdd(p.tile_counter, 1);
+        if (t > p.n_tiles) t = p.n_tiles;              // sentinel: no more tiles
+        const int e = i % kTq;
+        if (i >= kTq && !(ok = mbar_wait(&tq_empty[e], ((i / kTq) - 1) & 1, abort_flag, p.status))) break;
+        tq[e] = t;
+        mbar_arrive(&tq_full[e]);
+        if (t >= p.n_tiles) break;
+        const TileInfo ti = tile_info<GATED, LINEAR>(t, p);
+        auto step_blocks = [&](int j) -> int {
+          if (GATED && j == ti.local_steps) return 1;
+          return (2 * j + 1 < ti.n_local) ? 2 : 1;
+        };
+        // Q (and Z) of this tile once every MMA of the previous tile that reads them is done
+        if (i > 0 && !(ok = mbar_wait(q_free, (i - 1) & 1, abort_flag, p.status))) break;
+        mbar_arrive_expect_tx(q_full, L::kChunks * L::kTile + ti.n_lin * L::kZTile);
+        q_loaded = i;
+        if (TILE) {
+          for (int half = 0; half < 2; ++half) {
+            int tf, th, tw;
+            tile_coords(2 * ti.pair + half, p.TF, p.TW, tf, th, tw);
+            for (int c = 0; c < L::kChunks; ++c)
+              tma_load_5d(sQ + c * L::kTile + half * L::kHalf, &tmQ, q_full, c * 64, tw * 4, th * 4, tf * 4, ti.bh);
+          }
+        } else {
+          for (int c = 0; c < L::kChunks; ++c) tma_load_3d(sQ + c * L::kTile, &tmQ, q_full, c * 64, ti.pair * 128, ti.bh);
+        }
+        for (int b = 0; b < ti.n_lin; ++b)   // row D of the state (Z) and 15 rows of zero fill
           for (int c = 0; c < L::kChunks; ++c)
-            tma_load_5d(sQ + c * L::kTile + half * L::kHalf, &tmQ, q_full, c * 64, tw * 4, th * 4, tf * 4, bh);
-        }
-      } else {
-        for (int c = 0; c < L::kChunks; ++c) tma_load_3d(sQ + c * L::kTile, &tmQ, q_full, c * 64, pair * 128, bh);
-      }
-      for (int b = 0; b < n_lin; ++b)   // row D of the state (Z) and 15 rows of zero fill
-        for (int c = 0; c < L::kChunks; ++c)
-          tma_load_3d(sZ + b * L::kZTile + c * L::kZChunk, &tmX2, q_full, c * 64, D, bh * p.n_qb + 2 * pair + b);
-      if (LINEAR) {
-        // the pre-slots complete their barriers' first phase: TMA for the states, a plain
-        // arrive for the phi(Q) slot (and for slot 1 when the pair has one query block)
-        for (int b = 0; b < 2; ++b) {
-          if (b < n_lin) {
-            mbar_arrive_expect_tx(&slot_full[b], L::kHsTile);
-            for (int c = 0; c < L::kChunks; ++c)
-              tma_load_3d(sRing + b * L::kKV + c * L::kHsChunk, &tmX1, &slot_full[b], c * 64, 0, bh * p.n_qb + 2 * pair + b);
-          } else {
-            mbar_arrive(&slot_full[b]);
-          }
-        }
-        mbar_arrive(&slot_full[2]);
-      }
-      // K/V item i: K (even i) or V (odd i) of step i/2, at ring position g = i + kPre
-      // (slot g % kSlots).  The slot's previous occupant is position g - kSlots: a K/V
-      // item, free once the P.V of its step has completed, or a pre-slot, free once the
-      // linear-branch MMAs have completed.
-      int i = 0;
-      for (; i < 2 * n_steps; ++i) {
-        const int g = i + kPre, slot = g % kSlots;
-        if (g >= kSlots) {
-          bool freed;
-          if (LINEAR && g - kSlots < kPre) {
-            freed = mbar_wait(lin_done, 0, abort_flag, p.status);
-          } else {
-            const int q = (i - kSlots) >> 1;
-            freed = mbar_wait(&pv_done[q & 3], (q >> 2) & 1, abort_flag, p.status);
-          }
-          if (!freed) break;
-        }
-        uint8_t* dst0 = sRing + slot * L::kKV;
-        const int j = i >> 1;
-        const bool is_v = i & 1;
-        const int nb = step_blocks(j);
-        const bool far = GATED && j == local_steps;
-        mbar_arrive_expect_tx(&slot_full[slot], nb * L::kChunks * L::kHalf);
-        for (int b = 0; b < nb; ++b) {
-          uint8_t* dst = dst0 + b * L::kHalf;
-          if (far) {
-            for (int c = 0; c < L::kChunks; ++c)
-              tma_load_3d(dst + c * L::kTile, is_v ? &tmX2 : &tmX1, &slot_full[slot], c * 64, 0, bh);
-          } else {
-            const int kb = list ? (int)(list[2 * j + b] & 0xFFFFu) : 2 * j + b;
-            const CUtensorMap* tm = is_v ? &tmV : &tmK;
-            if (TILE) {
-              int tf, th, tw;
-              tile_coords(kb, p.TF, p.TW, tf, th, tw);
+            tma_load_3d(sZ + b * L::kZTile + c * L::kZChunk, &tmX2, q_full, c * 64, D, ti.bh * p.n_qb + 2 * ti.pair + b);
+        if (LINEAR) {
+          // pre-slots: the states by TMA; the phi(Q) slot is handed to the softmax warps
+          // (plain arrive) once its previous occupant is released; a missing second
+          // query block's slot completes its phase with a plain arrive too
+          for (int pr = 0; pr < 3 && ok; ++pr, ++g) {
+            const int slot = g % kSlots;
+            if (!(ok = slot_released(slot))) break;
+            if (pr < ti.n_lin) {
+              mbar_arrive_expect_tx(&slot_full[slot], L::kHsTile);
               for (int c = 0; c < L::kChunks; ++c)
-                tma_load_5d(dst + c * L::kTile, tm, &slot_full[slot], c * 64, tw * 4, th * 4, tf * 4, bh);
+                tma_load_3d(sRing + slot * L::kKV + c * L::kHsChunk, &tmX1, &slot_full[slot], c * 64, 0,
+                            ti.bh * p.n_qb + 2 * ti.pair + pr);
             } else {
-              for (int c = 0; c < L::kChunks; ++c) tma_load_3d(dst + c * L::kTile, tm, &slot_full[slot], c * 64, kb * 64, bh);
+              mbar_arrive(&slot_full[slot]);
+            }
+            rel_kind[slot] = 1;
+            rel_idx[slot] = i;
+          }
+        }
+        // K/V items: K (even it) or V (odd it) of step it/2
+        for (int it = 0; it < 2 * ti.n_steps && ok; ++it, ++g) {
+          const int slot = g % kSlots;
+          if (!(ok = slot_released(slot))) break;
+          const int j = it >> 1;
+          const bool is_v = it & 1;
+          const int nb = step_blocks(j);
+          const bool far = GATED && j == ti.local_steps;
+          mbar_arrive_expect_tx(&slot_full[slot], nb * L::kChunks * L::kHalf);
+          for (int b = 0; b < nb; ++b) {
+            uint8_t* dst = sRing + slot * L::kKV + b * L::kHalf;
+            if (far) {
+              for (int c = 0; c < L::kChunks; ++c)
+                tma_load_3d(dst + c * L::kTile, is_v ? &tmX2 : &tmX1, &slot_full[slot], c * 64, 0, ti.bh);
+            } else {
+              const int kb = ti.list ? (int)(ti.list[2 * j + b] & 0xFFFFu) : 2 * j + b;
+              const CUtensorMap* tm = is_v ? &tmV : &tmK;
+              if (TILE) {
+                int tf, th, tw;
+                tile_coords(kb, p.TF, p.TW, tf, th, tw);
+                for (int c = 0; c < L::kChunks; ++c)
+                  tma_load_5d(dst + c * L::kTile, tm, &slot_full[slot], c * 64, tw * 4, th * 4, tf * 4, ti.bh);
+              } else {
+                for (int c = 0; c < L::kChunks; ++c)
+                  tma_load_3d(dst + c * L::kTile, tm, &slot_full[slot], c * 64, kb * 64, ti.bh);
+              }
             }
           }
+          rel_kind[slot] = 0;
+          rel_idx[slot] = J + j;
         }
+        J += ti.n_steps;
+        ++i;
       }
       if (*abort_flag) {
         // let the loads already in flight land before the CTA's shared memory is released
         long long t0 = clock64();
-        while (!mbar_try_wait(q_full, 0) && clock64() - t0 < kWaitBudgetCycles) {}
-        for (int g = (i + kPre - kSlots > 0 ? i + kPre - kSlots : 0); g < i + kPre; ++g) {
+        if (q_loaded >= 0) while (!mbar_try_wait(q_full, q_loaded & 1) && clock64() - t0 < kWaitBudgetCycles) {}
+        for (int gg = (g - kSlots > 0 ? g - kSlots : 0); gg < g; ++gg) {
           t0 = clock64();
-          while (!mbar_try_wait(&slot_full[g % kSlots], (g / kSlots) & 1) && clock64() - t0 < kWaitBudgetCycles) {}
+          while (!mbar_try_wait(&slot_full[gg % kSlots], (gg / kSlots) & 1) && clock64() - t0 < kWaitBudgetCycles) {}
         }
       }
     }
   } else if (warp == 9) {
     // ---------------------------------------------------------------- MMA issuer
-    if (lane == 0 && active) {
+    if (lane == 0) {
       constexpr uint32_t idS = idesc_bf16(128, 128, false, false);
       constexpr uint32_t idO = idesc_bf16(128, D, false, true);
       const uint32_t q_addr = smem_u32(sQ), ring_addr = smem_u32(sRing);
@@ -334,18 +387,19 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
       };
       // lin = phi(Q) [H'^T ; Z]^T per query block (lanes of the other block masked off)
       // into the O columns, before any P.V; column D of the result is phi(q) . Z
-      auto issue_lin = [&]() {
+      auto issue_lin = [&](int g0, int n_lin) {
         constexpr uint32_t idH = idesc_bf16(128, D, false, false);
         constexpr uint32_t idZ = idesc_bf16(128, 16, false, false);
-        const uint32_t z_addr = smem_u32(sZ), phq_addr = ring_addr + 2 * L::kKV;
+        const uint32_t z_addr = smem_u32(sZ), phq_addr = ring_addr + ((g0 + 2) % kSlots) * L::kKV;
         const uint32_t lo_only[4] = {0u, 0u, 0xFFFFFFFFu, 0xFFFFFFFFu};   // write lanes 0-63
         const uint32_t hi_only[4] = {0xFFFFFFFFu, 0xFFFFFFFFu, 0u, 0u};   // write lanes 64-127
         for (int b = 0; b < n_lin; ++b) {
+          const uint32_t hs_addr = ring_addr + ((g0 + b) % kSlots) * L::kKV;
           #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const int c = kk >> 2, sub = kk & 3;
             const uint64_t a = desc_kmajor(phq_addr + c * L::kTile + sub * 32);
-            const uint64_t bh_ = desc_kmajor(ring_addr + b * L::kKV + c * L::kHsChunk + sub * 32);
+            const uint64_t bh_ = desc_kmajor(hs_addr + c * L::kHsChunk + sub * 32);
             const uint64_t bz = desc_kmajor(z_addr + b * L::kZTile + c * L::kZChunk + sub * 32);
             mma_bf16_ss_masked(tmem + kColLinOut, a, bh_, idH, kk > 0 ? 1u : 0u, b ? hi_only : lo_only);
             mma_bf16_ss_masked(tmem + kColLinOut + D, a, bz, idZ, kk > 0 ? 1u : 0u, b ? hi_only : lo_only);
@@ -353,39 +407,56 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
         }
         mma_commit(lin_done);
       };
-      bool ok = mbar_wait(q_full, 0, abort_flag, p.status);
-      bool o1_started = false;
-      if (ok && n_steps > 0) {
-        ok = mbar_wait(&slot_full[kPre % kSlots], (kPre / kSlots) & 1, abort_flag, p.status);
-        if (ok) {
+      int i = 0, J = 0, g = 0;
+      bool ok = true;
+      while (ok) {
+        const int e = i % kTq;
+        if (!(ok = mbar_wait(&tq_full[e], (i / kTq) & 1, abort_flag, p.status))) break;
+        const int t = tq[e];
+        mbar_arrive(&tq_empty[e]);
+        if (t >= p.n_tiles) break;
+        const TileInfo ti = tile_info<GATED, LINEAR>(t, p);
+        auto step_blocks = [&](int j) -> int {
+          if (GATED && j == ti.local_steps) return 1;
+          return (2 * j + 1 < ti.n_local) ? 2 : 1;
+        };
+        const int gkv = g + kPre;                  // ring position of this tile's K_0
+        if (!(ok = mbar_wait(q_full, i & 1, abort_flag, p.status))) break;
+        // GATED: the previous tile's far-field output sits in the S buffer this tile's
+        // first QK writes, so wait until its epilogue has read it
+        if (GATED && i > 0 && !(ok = mbar_wait(o_free, (i - 1) & 1, abort_flag, p.status))) break;
+        if (ti.n_steps > 0) {
+          if (!(ok = mbar_wait(&slot_full[gkv % kSlots], (gkv / kSlots) & 1, abort_flag, p.status))) break;
           tc_fence_after();
-          issue_qk(kPre % kSlots, 0);
-          mma_commit(&s_full[0]);
+          issue_qk(gkv % kSlots, J & 1);
+          mma_commit(&s_full[J & 1]);
         }
-      }
-      if (ok && LINEAR) {
-        ok = mbar_wait(phiq_ready, 0, abort_flag, p.status) && mbar_wait(&slot_full[0], 0, abort_flag, p.status) &&
-             mbar_wait(&slot_full[1], 0, abort_flag, p.status);
-        if (ok) {
+        if (LINEAR) {
+          ok = mbar_wait(phiq_ready, i & 1, abort_flag, p.status) &&
+               mbar_wait(&slot_full[g % kSlots], (g / kSlots) & 1, abort_flag, p.status) &&
+               mbar_wait(&slot_full[(g + 1) % kSlots], ((g + 1) / kSlots) & 1, abort_flag, p.status) &&
+               (i == 0 || mbar_wait(o_free, (i - 1) & 1, abort_flag, p.status));
+          if (!ok) break;
           tc_fence_after();
-          issue_lin();
+          issue_lin(g, ti.n_lin);
         }
-      }
-      if (ok && n_steps > 0) {
-        for (int j = 0; j < n_steps && ok; ++j) {
-          const int b = j & 1;
-          if (j + 1 < n_steps) {
-            const int gk = 2 * (j + 1) + kPre;
-            if (!mbar_wait(&slot_full[gk % kSlots], (gk / kSlots) & 1, abort_flag, p.status)) { ok = false; break; }
+        if (ti.n_steps <= 1) mma_commit(q_free);   // the last MMA reading Q (and Z) has been issued
+        bool o1_started = false;
+        for (int j = 0; j < ti.n_steps && ok; ++j) {
+          const int Jj = J + j, b = Jj & 1;
+          if (j + 1 < ti.n_steps) {
+            const int gk = gkv + 2 * (j + 1);
+            if (!(ok = mbar_wait(&slot_full[gk % kSlots], (gk / kSlots) & 1, abort_flag, p.status))) break;
             tc_fence_after();
-            issue_qk(gk % kSlots, (j + 1) & 1);
-            mma_commit(&s_full[(j + 1) & 1]);
+            issue_qk(gk % kSlots, (Jj + 1) & 1);
+            mma_commit(&s_full[(Jj + 1) & 1]);
+            if (j + 2 == ti.n_steps) mma_commit(q_free);
           }
-          const int gv = 2 * j + 1 + kPre;
+          const int gv = gkv + 2 * j + 1;
           if (!mbar_wait(&slot_full[gv % kSlots], (gv / kSlots) & 1, abort_flag, p.status) ||
-              !mbar_wait(&p_full[b], (j >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
+              !mbar_wait(&p_full[b], (Jj >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
           tc_fence_after();
-          const bool far = GATED && j == local_steps;
+          const bool far = GATED && j == ti.local_steps;
           if (far) {
             // the far-field output goes into the other S buffer (its step is done)
             issue_pv(gv % kSlots, b, 0, kColS + (b ^ 1) * 128, false);
@@ -396,8 +467,11 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
               o1_started = true;
             }
           }
-          mma_commit(&pv_done[j & 3]);
+          mma_commit(&pv_done[Jj & 3]);
         }
+        g += kPre + 2 * ti.n_steps;
+        J += ti.n_steps;
+        ++i;
       }
       if (!ok) {
         mma_commit(drain);
@@ -413,253 +487,285 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
     const uint32_t lane_addr = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     const uint32_t my_o = wg ? kColO1 : kColO0;
     const float sl = p.scale_log2;
-    float m_run = -INFINITY, l_run = 0.f, l_far = 0.f;
-    bool ok = true, started = false;
-    // ---- token of this row
-    int tok;
-    bool row_exists;
-    if (TILE) {
-      const int tile = 2 * pair + half;
-      row_exists = tile < p.n_qb;
-      int tf, th, tw;
-      tile_coords(tile, p.TF, p.TW, tf, th, tw);
-      const int rr = r & 63;
-      tok = ((tf * 4 + (rr >> 4)) * p.Hh + th * 4 + ((rr >> 2) & 3)) * p.Ww + tw * 4 + (rr & 3);
-    } else {
-      tok = pair * 128 + r;
-      row_exists = tok < p.n_pad;
-    }
-    const bool valid = row_exists && (TILE || token_valid(seq, tok));
+    int i = 0, J = 0, g = 0;
+    bool ok = true;
+    while (ok) {
+      const int e = i % kTq;
+      ok = __all_sync(0xFFFFFFFFu, mbar_wait(&tq_full[e], (i / kTq) & 1, abort_flag, p.status));
+      if (!ok) break;
+      const int t = tq[e];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tq_empty[e]);
+      if (t >= p.n_tiles) break;
+      const TileInfo ti = tile_info<GATED, LINEAR>(t, p);
+      const int local_steps = ti.local_steps, n_steps = ti.n_steps, n_local = ti.n_local;
+      auto step_blocks = [&](int j) -> int {
+        if (GATED && j == local_steps) return 1;
+        return (2 * j + 1 < n_local) ? 2 : 1;
+      };
+      float m_run = -INFINITY, l_run = 0.f, l_far = 0.f;
+      bool started = false;
 
-    // ---- linear branch first (LINEAR): phi(Q) into ring slot 2 (pad rows -> 0; Q stays in
-    // place for the QK MMAs), then the MMA warp's lin = phi(Q) [H'^T ; Z]^T lands in the O
-    // columns; my half of the row, divided by its denominator, is read during the first
-    // step (before its P is handed over, since the first P.V overwrites those columns) and
-    // kept in registers as bf16 pairs (the output is rounded to bf16 in the end as well)
-    uint32_t lin[D / 4];
-    #pragma unroll
-    for (int i = 0; i < D / 4; ++i) lin[i] = 0u;
-    if (LINEAR) {
-      ok = __all_sync(0xFFFFFFFFu, mbar_wait(q_full, 0, abort_flag, p.status));
-      if (ok) {
-        uint8_t* sPhi = sRing + 2 * L::kKV;
-        constexpr int kGroups = D / 16;                  // 16-byte groups of my row handled by my warpgroup
-        #pragma unroll
-        for (int g = 0; g < kGroups; ++g) {
-          const int gg = wg * kGroups + g;               // 0 .. D/8-1
-          const int off = (gg >> 3) * L::kTile + sw128_offset(r, gg & 7);
-          const uint4 u = *reinterpret_cast<const uint4*>(sQ + off);
-          const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-          uint32_t o4[4];
-          #pragma unroll
-          for (int i = 0; i < 4; ++i)
-            o4[i] = valid ? pack_bf16(phi_fast(bf16_lo(w[i])), phi_fast(bf16_hi(w[i]))) : 0u;
-          *reinterpret_cast<uint4*>(sPhi + off) = make_uint4(o4[0], o4[1], o4[2], o4[3]);
-        }
+      // ---- token of this row
+      int tok;
+      bool row_exists;
+      if (TILE) {
+        const int tile = 2 * ti.pair + half;
+        row_exists = tile < p.n_qb;
+        int tf, th, tw;
+        tile_coords(tile, p.TF, p.TW, tf, th, tw);
+        const int rr = r & 63;
+        tok = ((tf * 4 + (rr >> 4)) * p.Hh + th * 4 + ((rr >> 2) & 3)) * p.Ww + tw * 4 + (rr & 3);
+      } else {
+        tok = ti.pair * 128 + r;
+        row_exists = tok < p.n_pad;
       }
-      fence_proxy_async_smem();
-      mbar_arrive(phiq_ready);
-    }
-    bool lin_pending = LINEAR;
-    auto read_lin = [&]() {
-      lin_pending = false;
-      if (ok) ok = __all_sync(0xFFFFFFFFu, mbar_wait(lin_done, 0, abort_flag, p.status));
-      tc_fence_after();
-      if (!ok) return;
-      uint32_t dv;
-      tmem_ld1(lane_addr + kColLinOut + D, dv);
-      tmem_wait_ld();
-      const float den = __uint_as_float(dv);
-      const float inv_den = den > 0.f ? 1.f / den : 0.f;
+      const bool valid = row_exists && (TILE || token_valid(seq, tok));
+
+      // ---- linear branch first (LINEAR): phi(Q) into the tile's third pre-slot (pad rows
+      // -> 0; Q stays in place for the QK MMAs), then the MMA warp's lin = phi(Q) [H'^T ; Z]^T
+      // lands in the O columns; my half of the row, divided by its denominator, is read
+      // during the first step (before its P is handed over, since the first P.V overwrites
+      // those columns) and kept in registers as bf16 pairs (the output is rounded to bf16
+      // in the end as well)
+      uint32_t lin[D / 4];
       #pragma unroll
-      for (int k = 0; k < D / 64; ++k) {
-        uint32_t t[32];
-        tmem_ld32(lane_addr + kColLinOut + wg * (D / 2) + k * 32, t);
-        tmem_wait_ld();
-        #pragma unroll
-        for (int i = 0; i < 16; ++i)
-          lin[k * 16 + i] = pack_bf16(__uint_as_float(t[2 * i]) * inv_den, __uint_as_float(t[2 * i + 1]) * inv_den);
+      for (int k = 0; k < D / 4; ++k) lin[k] = 0u;
+      if (LINEAR) {
+        const int gphi = g + 2;
+        ok = __all_sync(0xFFFFFFFFu, mbar_wait(q_full, i & 1, abort_flag, p.status) &&
+                                         mbar_wait(&slot_full[gphi % kSlots], (gphi / kSlots) & 1, abort_flag, p.status));
+        if (ok) {
+          uint8_t* sPhi = sRing + (gphi % kSlots) * L::kKV;
+          constexpr int kGroups = D / 16;                  // 16-byte groups of my row handled by my warpgroup
+          #pragma unroll
+          for (int gr = 0; gr < kGroups; ++gr) {
+            const int gg = wg * kGroups + gr;              // 0 .. D/8-1
+            const int off = (gg >> 3) * L::kTile + sw128_offset(r, gg & 7);
+            const uint4 u = *reinterpret_cast<const uint4*>(sQ + off);
+            const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+            uint32_t o4[4];
+            #pragma unroll
+            for (int k = 0; k < 4; ++k)
+              o4[k] = valid ? pack_bf16(phi_fast(bf16_lo(w[k])), phi_fast(bf16_hi(w[k]))) : 0u;
+            *reinterpret_cast<uint4*>(sPhi + off) = make_uint4(o4[0], o4[1], o4[2], o4[3]);
+          }
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(phiq_ready);
       }
-    };
-    for (int j = 0; j < n_steps && ok; ++j) {
-      const int b = j & 1;
-      const bool far = GATED && j == local_steps;
-      const bool mine = wg == 0 || (!far && step_blocks(j) == 2);   // does this warpgroup own a block here
-      Entry e{0, 64, 3u};
-      if (mine && !far) e = read_entry<TILE>(list, 2 * j + wg, seq);
-      if (!__all_sync(0xFFFFFFFFu, mbar_wait(&s_full[b], (j >> 1) & 1, abort_flag, p.status))) { ok = false; break; }
-      tc_fence_after();
-      if (!mine) {
+      bool lin_pending = LINEAR;
+      auto read_lin = [&]() {
+        lin_pending = false;
+        if (ok) ok = __all_sync(0xFFFFFFFFu, mbar_wait(lin_done, i & 1, abort_flag, p.status));
+        tc_fence_after();
+        if (!ok) return;
+        uint32_t dv;
+        tmem_ld1(lane_addr + kColLinOut + D, dv);
+        tmem_wait_ld();
+        const float den = __uint_as_float(dv);
+        const float inv_den = den > 0.f ? 1.f / den : 0.f;
+        #pragma unroll
+        for (int k = 0; k < D / 64; ++k) {
+          uint32_t tv[32];
+          tmem_ld32(lane_addr + kColLinOut + wg * (D / 2) + k * 32, tv);
+          tmem_wait_ld();
+          #pragma unroll
+          for (int m = 0; m < 16; ++m)
+            lin[k * 16 + m] = pack_bf16(__uint_as_float(tv[2 * m]) * inv_den, __uint_as_float(tv[2 * m + 1]) * inv_den);
+        }
+      };
+
+      for (int j = 0; j < n_steps && ok; ++j) {
+        const int Jj = J + j, b = Jj & 1;
+        const bool far = GATED && j == local_steps;
+        const bool mine = wg == 0 || (!far && step_blocks(j) == 2);   // does this warpgroup own a block here
+        Entry en{0, 64, 3u};
+        if (mine && !far) en = read_entry<TILE>(ti.list, 2 * j + wg, seq);
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&s_full[b], (Jj >> 1) & 1, abort_flag, p.status))) { ok = false; break; }
+        tc_fence_after();
+        if (!mine) {
+          if (LINEAR && j == 0) {
+            read_lin();
+            if (!ok) break;
+          }
+          tc_fence_before();
+          mbar_arrive(&p_full[b]);
+          continue;
+        }
+        const uint32_t s_addr = lane_addr + kColS + b * 128 + wg * 64;
+        uint32_t sr[64];
+        tmem_ld32(s_addr, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+        tmem_ld32(s_addr + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+        const bool attend = (en.flags >> half) & 1u;
+        const int nvalid = attend ? en.nvalid : 0;
+        tmem_wait_ld();
+        float mx = -INFINITY;
+        if (nvalid == 64) {
+          float t3[22];
+          #pragma unroll
+          for (int k = 0; k < 21; ++k)
+            t3[k] = max3(__uint_as_float(sr[3 * k]), __uint_as_float(sr[3 * k + 1]), __uint_as_float(sr[3 * k + 2]));
+          t3[21] = __uint_as_float(sr[63]);
+          float u[8];
+          #pragma unroll
+          for (int k = 0; k < 7; ++k) u[k] = max3(t3[3 * k], t3[3 * k + 1], t3[3 * k + 2]);
+          u[7] = t3[21];
+          mx = fmaxf(max3(u[0], u[1], u[2]), max3(max3(u[3], u[4], u[5]), u[6], u[7]));
+        } else if (nvalid > 0) {
+          #pragma unroll
+          for (int c = 0; c < 64; ++c) {
+            if (c >= nvalid) sr[c] = __float_as_uint(-INFINITY);
+            mx = fmaxf(mx, __uint_as_float(sr[c]));
+          }
+        }
+        // far step: a fresh softmax of its own; local steps: lazy rescale of the running state
+        float mu;
+        bool need = false;
+        float factor = 1.f;
+        if (far) {
+          mu = mx * sl;
+        } else {
+          const float m_new = fmaxf(m_run, mx * sl);
+          need = m_new > m_run + 8.f;
+          if (need) {
+            factor = (m_run == -INFINITY) ? 0.f : ex2(m_run - m_new);
+            l_run *= factor;
+            m_run = m_new;
+          }
+          mu = m_run;
+        }
+        if (mu == -INFINITY) mu = 0.f;
+        uint32_t packed[32];
+        float rowsum = 0.f;
+        if (nvalid == 0) {
+          #pragma unroll
+          for (int c = 0; c < 32; ++c) packed[c] = 0u;
+        } else {
+          float acc0 = 0.f, acc1 = 0.f;
+          #pragma unroll
+          for (int c = 0; c < 64; c += 2) {
+            const float p0 = ex2(fmaf(__uint_as_float(sr[c]), sl, -mu));
+            const float p1 = ex2(fmaf(__uint_as_float(sr[c + 1]), sl, -mu));
+            acc0 += p0;
+            acc1 += p1;
+            packed[c >> 1] = pack_bf16(p0, p1);
+          }
+          rowsum = acc0 + acc1;
+        }
+        if (far) l_far = rowsum; else l_run += rowsum;
+        // rescale my accumulator (once it holds data) after the previous P.V has completed
+        if (!far && started && __any_sync(0xFFFFFFFFu, need)) {
+          if (!__all_sync(0xFFFFFFFFu, mbar_wait(&pv_done[(Jj - 1) & 3], ((Jj - 1) >> 2) & 1, abort_flag, p.status))) { ok = false; break; }
+          tc_fence_after();
+          #pragma unroll 1
+          for (int cc = 0; cc < D / 32; ++cc) {
+            uint32_t o[32];
+            tmem_ld32(lane_addr + my_o + cc * 32, o);
+            tmem_wait_ld();
+            #pragma unroll
+            for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * factor);
+            tmem_st32(lane_addr + my_o + cc * 32, o);
+          }
+        }
         if (LINEAR && j == 0) {
           read_lin();
           if (!ok) break;
         }
+        tmem_st32(s_addr, packed);          // P (bf16 pairs) over the first 32 columns of my S block
+        tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&p_full[b]);
-        continue;
+        if (!far) started = true;
       }
-      const uint32_t s_addr = lane_addr + kColS + b * 128 + wg * 64;
-      uint32_t sr[64];
-      tmem_ld32(s_addr, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-      tmem_ld32(s_addr + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
-      const bool attend = (e.flags >> half) & 1u;
-      const int nvalid = attend ? e.nvalid : 0;
-      tmem_wait_ld();
-      float mx = -INFINITY;
-      if (nvalid == 64) {
-        float t[22];
-        #pragma unroll
-        for (int i = 0; i < 21; ++i)
-          t[i] = max3(__uint_as_float(sr[3 * i]), __uint_as_float(sr[3 * i + 1]), __uint_as_float(sr[3 * i + 2]));
-        t[21] = __uint_as_float(sr[63]);
-        float u[8];
-        #pragma unroll
-        for (int i = 0; i < 7; ++i) u[i] = max3(t[3 * i], t[3 * i + 1], t[3 * i + 2]);
-        u[7] = t[21];
-        mx = fmaxf(max3(u[0], u[1], u[2]), max3(max3(u[3], u[4], u[5]), u[6], u[7]));
-      } else if (nvalid > 0) {
-        #pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          if (c >= nvalid) sr[c] = __float_as_uint(-INFINITY);
-          mx = fmaxf(mx, __uint_as_float(sr[c]));
-        }
+      if (LINEAR && lin_pending) read_lin();         // no step read it
+      if (ok && n_steps > 0) {
+        const int Jl = J + n_steps - 1;
+        ok = __all_sync(0xFFFFFFFFu, mbar_wait(&pv_done[Jl & 3], (Jl >> 2) & 1, abort_flag, p.status));
       }
-      // far step: a fresh softmax of its own; local steps: lazy rescale of the running state
-      float mu;
-      bool need = false;
-      float factor = 1.f;
-      if (far) {
-        mu = mx * sl;
-      } else {
-        const float m_new = fmaxf(m_run, mx * sl);
-        need = m_new > m_run + 8.f;
-        if (need) {
-          factor = (m_run == -INFINITY) ? 0.f : ex2(m_run - m_new);
-          l_run *= factor;
-          m_run = m_new;
-        }
-        mu = m_run;
+      ok = __all_sync(0xFFFFFFFFu, ok);
+      tc_fence_after();
+
+      // ---- merge the two shares (published through shared memory, double-buffered by tile)
+      float* xb = xch + (i & 1) * (3 * 128);
+      if (wg == 0) { xb[r] = m_run; xb[128 + r] = l_run; }
+      float* xo = xch + 2 * (3 * 128) + (i & 1) * (3 * 128);   // the second warpgroup's share
+      if (wg == 1) { xo[r] = m_run; xo[128 + r] = l_run; }
+      if (GATED && wg == 0) xb[256 + r] = l_far;
+      mbar_arrive(xch_bar);
+      if (ok) ok = __all_sync(0xFFFFFFFFu, mbar_wait(xch_bar, i & 1, abort_flag, p.status));
+      const float m0 = xb[r], l0 = xb[128 + r], m1 = xo[r], l1 = xo[128 + r];
+      const float M = fmaxf(m0, m1);
+      const float a0 = (m0 == -INFINITY) ? 0.f : ex2(m0 - M);
+      const float a1 = (m1 == -INFINITY) ? 0.f : ex2(m1 - M);
+      const float Lsum = a0 * l0 + a1 * l1;
+      const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
+      const float c0 = a0 * inv, c1 = a1 * inv;
+      float inv_far = 0.f;
+      uint32_t col_far = 0;
+      if (GATED) {
+        const float lf = xb[256 + r];
+        inv_far = lf > 0.f ? 1.f / lf : 0.f;
+        col_far = kColS + (((J + local_steps) & 1) ^ 1) * 128;
       }
-      if (mu == -INFINITY) mu = 0.f;
-      uint32_t packed[32];
-      float rowsum = 0.f;
-      if (nvalid == 0) {
+      const bool have_o0 = ok && n_local > 0;        // uniform over the softmax warps
+      const bool have_o1 = ok && n_local > 1;
+      const size_t row_off = ((size_t)ti.bh * p.n_pad + (row_exists ? tok : 0)) * D;
+      #pragma unroll
+      for (int k = 0; k < D / 64; ++k) {
+        const int cc = wg * (D / 64) + k;          // my 32-column chunks
+        float v[32];
         #pragma unroll
-        for (int c = 0; c < 32; ++c) packed[c] = 0u;
-      } else {
-        float acc0 = 0.f, acc1 = 0.f;
-        #pragma unroll
-        for (int c = 0; c < 64; c += 2) {
-          const float p0 = ex2(fmaf(__uint_as_float(sr[c]), sl, -mu));
-          const float p1 = ex2(fmaf(__uint_as_float(sr[c + 1]), sl, -mu));
-          acc0 += p0;
-          acc1 += p1;
-          packed[c >> 1] = pack_bf16(p0, p1);
-        }
-        rowsum = acc0 + acc1;
-      }
-      if (far) l_far = rowsum; else l_run += rowsum;
-      // rescale my accumulator (once it holds data) after P_{j-1} V_{j-1} has completed
-      if (!far && started && __any_sync(0xFFFFFFFFu, need)) {
-        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&pv_done[(j - 1) & 3], ((j - 1) >> 2) & 1, abort_flag, p.status))) { ok = false; break; }
-        tc_fence_after();
-        #pragma unroll 1
-        for (int cc = 0; cc < D / 32; ++cc) {
-          uint32_t o[32];
-          tmem_ld32(lane_addr + my_o + cc * 32, o);
+        for (int m = 0; m < 32; ++m) v[m] = 0.f;
+        if (have_o0) {
+          uint32_t o0[32];
+          tmem_ld32(lane_addr + kColO0 + cc * 32, o0);
           tmem_wait_ld();
           #pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * factor);
-          tmem_st32(lane_addr + my_o + cc * 32, o);
+          for (int m = 0; m < 32; ++m) v[m] = c0 * __uint_as_float(o0[m]);
+        }
+        if (have_o1) {
+          uint32_t o1[32];
+          tmem_ld32(lane_addr + kColO1 + cc * 32, o1);
+          tmem_wait_ld();
+          #pragma unroll
+          for (int m = 0; m < 32; ++m) v[m] += c1 * __uint_as_float(o1[m]);
+        }
+        if (GATED && ok) {
+          uint32_t of[32];
+          tmem_ld32(lane_addr + col_far + cc * 32, of);
+          tmem_wait_ld();
+          #pragma unroll
+          for (int m = 0; m < 32; ++m) v[m] = p.gate * v[m] + (1.f - p.gate) * (__uint_as_float(of[m]) * inv_far);
+        }
+        if (LINEAR) {
+          #pragma unroll
+          for (int m = 0; m < 16; ++m) {
+            v[2 * m] += bf16_lo(lin[k * 16 + m]);
+            v[2 * m + 1] += bf16_hi(lin[k * 16 + m]);
+          }
+        }
+        if (!row_exists) continue;
+        uint4* dst = reinterpret_cast<uint4*>(p.out + row_off + cc * 32);
+        #pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          uint4 w4 = make_uint4(0, 0, 0, 0);
+          if (valid)
+            w4 = make_uint4(pack_bf16(v[8 * m], v[8 * m + 1]), pack_bf16(v[8 * m + 2], v[8 * m + 3]),
+                            pack_bf16(v[8 * m + 4], v[8 * m + 5]), pack_bf16(v[8 * m + 6], v[8 * m + 7]));
+          dst[m] = w4;
         }
       }
-      if (LINEAR && j == 0) {
-        read_lin();
-        if (!ok) break;
-      }
-      tmem_st32(s_addr, packed);          // P (bf16 pairs) over the first 32 columns of my S block
-      tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&p_full[b]);
-      if (!far) started = true;
-    }
-    if (LINEAR && lin_pending) read_lin();         // no step read it
-    if (ok && n_steps > 0)
-      ok = __all_sync(0xFFFFFFFFu, mbar_wait(&pv_done[(n_steps - 1) & 3], ((n_steps - 1) >> 2) & 1, abort_flag, p.status));
-    ok = __all_sync(0xFFFFFFFFu, ok);
-    tc_fence_after();
-
-    // ---- merge the two shares
-    xch[wg * 128 + r] = m_run;
-    xch[(2 + wg) * 128 + r] = l_run;
-    if (GATED && wg == 0) xch[512 + r] = l_far;
-    softmax_bar();
-    const float m0 = xch[r], m1 = xch[128 + r], l0 = xch[256 + r], l1 = xch[384 + r];
-    const float M = fmaxf(m0, m1);
-    const float a0 = (m0 == -INFINITY) ? 0.f : ex2(m0 - M);
-    const float a1 = (m1 == -INFINITY) ? 0.f : ex2(m1 - M);
-    const float Lsum = a0 * l0 + a1 * l1;
-    const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
-    const float c0 = a0 * inv, c1 = a1 * inv;
-    float inv_far = 0.f;
-    uint32_t col_far = 0;
-    if (GATED) {
-      const float lf = xch[512 + r];
-      inv_far = lf > 0.f ? 1.f / lf : 0.f;
-      col_far = kColS + ((local_steps & 1) ^ 1) * 128;
-    }
-    const bool have_o0 = ok && n_local > 0;        // CTA-uniform
-    const bool have_o1 = ok && n_local > 1;
-    const size_t row_off = ((size_t)bh * p.n_pad + (row_exists ? tok : 0)) * D;
-    #pragma unroll
-    for (int k = 0; k < D / 64; ++k) {
-      const int cc = wg * (D / 64) + k;          // my 32-column chunks
-      float v[32];
-      #pragma unroll
-      for (int i = 0; i < 32; ++i) v[i] = 0.f;
-      if (have_o0) {
-        uint32_t o0[32];
-        tmem_ld32(lane_addr + kColO0 + cc * 32, o0);
-        tmem_wait_ld();
-        #pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] = c0 * __uint_as_float(o0[i]);
+      mbar_arrive(o_free);                        // O_0/O_1 (and the far output) have been read
+      if (p.lse && row_exists && wg == 0) {
+        float val = 0.f;
+        if (valid) val = (Lsum > 0.f) ? (M + log2f(Lsum)) * 0.69314718055994531f : -INFINITY;
+        p.lse[(size_t)ti.bh * p.n_pad + tok] = val;
       }
-      if (have_o1) {
-        uint32_t o1[32];
-        tmem_ld32(lane_addr + kColO1 + cc * 32, o1);
-        tmem_wait_ld();
-        #pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] += c1 * __uint_as_float(o1[i]);
-      }
-      if (GATED && ok) {
-        uint32_t of[32];
-        tmem_ld32(lane_addr + col_far + cc * 32, of);
-        tmem_wait_ld();
-        #pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] = p.gate * v[i] + (1.f - p.gate) * (__uint_as_float(of[i]) * inv_far);
-      }
-      if (LINEAR) {
-        #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          v[2 * i] += bf16_lo(lin[k * 16 + i]);
-          v[2 * i + 1] += bf16_hi(lin[k * 16 + i]);
-        }
-      }
-      if (!row_exists) continue;
-      uint4* dst = reinterpret_cast<uint4*>(p.out + row_off + cc * 32);
-      #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        uint4 w4 = make_uint4(0, 0, 0, 0);
-        if (valid)
-          w4 = make_uint4(pack_bf16(v[8 * i], v[8 * i + 1]), pack_bf16(v[8 * i + 2], v[8 * i + 3]),
-                          pack_bf16(v[8 * i + 4], v[8 * i + 5]), pack_bf16(v[8 * i + 6], v[8 * i + 7]));
-        dst[i] = w4;
-      }
-    }
-    if (p.lse && row_exists && wg == 0) {
-      float val = 0.f;
-      if (valid) val = (Lsum > 0.f) ? (M + log2f(Lsum)) * 0.69314718055994531f : -INFINITY;
-      p.lse[(size_t)bh * p.n_pad + tok] = val;
+      g += kPre + 2 * n_steps;
+      J += n_steps;
+      ++i;
     }
   }
 
@@ -683,7 +789,10 @@ cudaError_t launch_variant(const AttnArgs& a, const CUtensorMap* maps, const Att
     if (e != cudaSuccess) return e;
     if (dev < 64) attr_set |= 1ull << dev;
   }
-  dim3 grid(a.n_pairs, a.BH);
+  int sms = 148;
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int grid = kp.n_tiles < sms ? kp.n_tiles : sms;
+  if (grid < 1) return cudaSuccess;
   kern<<<grid, kThreads, L::kBytes, st>>>(maps[0], maps[1], maps[2], maps[3], maps[4], kp);
   return cudaGetLastError();
 }
@@ -745,6 +854,10 @@ cudaError_t launch_attention(const AttnArgs& a, cudaStream_t st) {
   kp.gate = a.gate;
   kp.scale_log2 = (float)(1.4426950408889634 / sqrt((double)D));
   kp.status = a.status;
+  kp.n_tiles = a.n_pairs * a.BH;
+  kp.tile_counter = a.tile_counter;
+  if (!a.tile_counter) return cudaErrorInvalidValue;
+  if (cudaMemsetAsync(a.tile_counter, 0, sizeof(int), st) != cudaSuccess) return cudaErrorInvalidValue;
   return D == 128 ? launch_d<128>(a, maps, kp, st) : launch_d<64>(a, maps, kp, st);
 }
 

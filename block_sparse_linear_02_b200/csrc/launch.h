@@ -102,6 +102,7 @@ struct AttnArgs {
   int gated;                           // 1: add the far-field branch and gate
   float gate;
   int* status;
+  int* tile_counter;                   // one int of scratch, zeroed by launch_attention on the stream
 };
 cudaError_t launch_attention(const AttnArgs& a, cudaStream_t st);
 

@@ -304,6 +304,7 @@ AttnArgs attn_base(const Shape& sh, const void* q, const void* k, const void* v,
   a.n_qb = sh.nb; a.n_kb = sh.nb; a.n_pairs = sh.npairs;
   a.out = out;
   a.status = status;
+  a.tile_counter = status + 1;   // the status area holds 64 ints
   a.gate = 1.f;
   return a;
 }

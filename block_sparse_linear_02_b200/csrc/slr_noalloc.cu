@@ -85,6 +85,7 @@ extern "C" slr_status slr_block_sparse_attn_noalloc(const void* q, const void* k
   AttnArgs a;
   memset(&a, 0, sizeof(a));
   a.q = q; a.k = k; a.v = v; a.out = o; a.lse = lse_opt; a.status = status;
+  a.tile_counter = reinterpret_cast<int*>(scratch) + 1;   // inside the status area of the scratch
   a.BH = (int)bh; a.d = seq->d;
   a.s = SeqShape{(int)n_pad, seq->seg_len, seq->seg_stride, nb};
   a.n_qb = nb; a.n_kb = nb; a.n_pairs = npairs; a.gate = 1.f;
