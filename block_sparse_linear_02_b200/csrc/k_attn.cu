@@ -268,9 +268,11 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
       };
       int i = 0, J = 0, g = 0, q_loaded = -1;
       bool ok = true;
+      int t_next = atomicAdd(p.tile_counter, 1);       // the queue is read one tile ahead
       while (ok) {
-        int t = atomicAdd(p.tile_counter, 1);
+        int t = t_next;
         if (t > p.n_tiles) t = p.n_tiles;              // sentinel: no more tiles
+        if (t < p.n_tiles) t_next = atomicAdd(p.tile_counter, 1);
         const int e = i % kTq;
         if (i >= kTq && !(ok = mbar_wait(&tq_empty[e], ((i / kTq) - 1) & 1, abort_flag, p.status))) break;
         tq[e] = t;
@@ -385,12 +387,12 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
           mma_bf16_ts(tmem + col, a, b, idO, (acc || kk > 0) ? 1u : 0u);
         }
       };
-      // lin = phi(Q) [H'^T ; Z]^T per query block (lanes of the other block masked off)
-      // into the O columns, before any P.V; column D of the result is phi(q) . Z
+      // lin = phi(Q) H'_b per query block b (lanes of the other block masked off) into the
+      // O columns, before any P.V; the denominators phi(q) . Z_b are dot products the
+      // softmax warps form while they compute phi(Q)
       auto issue_lin = [&](int g0, int n_lin) {
         constexpr uint32_t idH = idesc_bf16(128, D, false, false);
-        constexpr uint32_t idZ = idesc_bf16(128, 16, false, false);
-        const uint32_t z_addr = smem_u32(sZ), phq_addr = ring_addr + ((g0 + 2) % kSlots) * L::kKV;
+        const uint32_t phq_addr = ring_addr + ((g0 + 2) % kSlots) * L::kKV;
         const uint32_t lo_only[4] = {0u, 0u, 0xFFFFFFFFu, 0xFFFFFFFFu};   // write lanes 0-63
         const uint32_t hi_only[4] = {0xFFFFFFFFu, 0xFFFFFFFFu, 0u, 0u};   // write lanes 64-127
         for (int b = 0; b < n_lin; ++b) {
@@ -400,9 +402,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
             const int c = kk >> 2, sub = kk & 3;
             const uint64_t a = desc_kmajor(phq_addr + c * L::kTile + sub * 32);
             const uint64_t bh_ = desc_kmajor(hs_addr + c * L::kHsChunk + sub * 32);
-            const uint64_t bz = desc_kmajor(z_addr + b * L::kZTile + c * L::kZChunk + sub * 32);
             mma_bf16_ss_masked(tmem + kColLinOut, a, bh_, idH, kk > 0 ? 1u : 0u, b ? hi_only : lo_only);
-            mma_bf16_ss_masked(tmem + kColLinOut + D, a, bz, idZ, kk > 0 ? 1u : 0u, b ? hi_only : lo_only);
           }
         }
         mma_commit(lin_done);
@@ -531,23 +531,31 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
       uint32_t lin[D / 4];
       #pragma unroll
       for (int k = 0; k < D / 4; ++k) lin[k] = 0u;
+      float den_part = 0.f;                       // phi(q) . Z over my half of the channels
       if (LINEAR) {
         const int gphi = g + 2;
         ok = __all_sync(0xFFFFFFFFu, mbar_wait(q_full, i & 1, abort_flag, p.status) &&
                                          mbar_wait(&slot_full[gphi % kSlots], (gphi / kSlots) & 1, abort_flag, p.status));
         if (ok) {
           uint8_t* sPhi = sRing + (gphi % kSlots) * L::kKV;
+          const uint8_t* zrow = sZ + half * L::kZTile;     // Z of my query block: row 0 of its Z tile
           constexpr int kGroups = D / 16;                  // 16-byte groups of my row handled by my warpgroup
           #pragma unroll
           for (int gr = 0; gr < kGroups; ++gr) {
             const int gg = wg * kGroups + gr;              // 0 .. D/8-1
             const int off = (gg >> 3) * L::kTile + sw128_offset(r, gg & 7);
             const uint4 u = *reinterpret_cast<const uint4*>(sQ + off);
+            const uint4 zu = *reinterpret_cast<const uint4*>(zrow + (gg >> 3) * L::kZChunk + (gg & 7) * 16);
             const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+            const uint32_t zw[4] = {zu.x, zu.y, zu.z, zu.w};
             uint32_t o4[4];
             #pragma unroll
-            for (int k = 0; k < 4; ++k)
+            for (int k = 0; k < 4; ++k) {
               o4[k] = valid ? pack_bf16(phi_fast(bf16_lo(w[k])), phi_fast(bf16_hi(w[k]))) : 0u;
+              // the denominator uses the same bf16 phi values the MMA multiplies
+              den_part = fmaf(bf16_lo(o4[k]), bf16_lo(zw[k]), den_part);
+              den_part = fmaf(bf16_hi(o4[k]), bf16_hi(zw[k]), den_part);
+            }
             *reinterpret_cast<uint4*>(sPhi + off) = make_uint4(o4[0], o4[1], o4[2], o4[3]);
           }
         }
@@ -560,19 +568,13 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
         if (ok) ok = __all_sync(0xFFFFFFFFu, mbar_wait(lin_done, i & 1, abort_flag, p.status));
         tc_fence_after();
         if (!ok) return;
-        uint32_t dv;
-        tmem_ld1(lane_addr + kColLinOut + D, dv);
-        tmem_wait_ld();
-        const float den = __uint_as_float(dv);
-        const float inv_den = den > 0.f ? 1.f / den : 0.f;
         #pragma unroll
         for (int k = 0; k < D / 64; ++k) {
           uint32_t tv[32];
           tmem_ld32(lane_addr + kColLinOut + wg * (D / 2) + k * 32, tv);
           tmem_wait_ld();
           #pragma unroll
-          for (int m = 0; m < 16; ++m)
-            lin[k * 16 + m] = pack_bf16(__uint_as_float(tv[2 * m]) * inv_den, __uint_as_float(tv[2 * m + 1]) * inv_den);
+          for (int m = 0; m < 16; ++m) lin[k * 16 + m] = pack_bf16(__uint_as_float(tv[2 * m]), __uint_as_float(tv[2 * m + 1]));
         }
       };
 
@@ -692,6 +694,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
       float* xo = xch + 2 * (3 * 128) + (i & 1) * (3 * 128);   // the second warpgroup's share
       if (wg == 1) { xo[r] = m_run; xo[128 + r] = l_run; }
       if (GATED && wg == 0) xb[256 + r] = l_far;
+      if (LINEAR) (wg ? xo : xb)[256 + r] = den_part;
       mbar_arrive(xch_bar);
       if (ok) ok = __all_sync(0xFFFFFFFFu, mbar_wait(xch_bar, i & 1, abort_flag, p.status));
       const float m0 = xb[r], l0 = xb[128 + r], m1 = xo[r], l1 = xo[128 + r];
@@ -701,6 +704,11 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
       const float Lsum = a0 * l0 + a1 * l1;
       const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
       const float c0 = a0 * inv, c1 = a1 * inv;
+      float inv_den = 0.f;
+      if (LINEAR) {
+        const float den = xb[256 + r] + xo[256 + r];
+        inv_den = den > 0.f ? 1.f / den : 0.f;
+      }
       float inv_far = 0.f;
       uint32_t col_far = 0;
       if (GATED) {
@@ -741,8 +749,8 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
         if (LINEAR) {
           #pragma unroll
           for (int m = 0; m < 16; ++m) {
-            v[2 * m] += bf16_lo(lin[k * 16 + m]);
-            v[2 * m + 1] += bf16_hi(lin[k * 16 + m]);
+            v[2 * m] = fmaf(bf16_lo(lin[k * 16 + m]), inv_den, v[2 * m]);
+            v[2 * m + 1] = fmaf(bf16_hi(lin[k * 16 + m]), inv_den, v[2 * m + 1]);
           }
         }
         if (!row_exists) continue;
