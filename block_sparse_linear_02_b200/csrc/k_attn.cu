@@ -98,10 +98,6 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-// phi(x) = elu(x) + 1 = exp(min(x, 0)) + max(x, 0), branch-free, exp through the exp2
-// unit (the result is rounded to bf16)
-__device__ __forceinline__ float phi_fast(float x) { return ex2(fminf(x, 0.f) * kLog2e) + fmaxf(x, 0.f); }
-
 __device__ __forceinline__ float max3(float a, float b, float c) {
   float r;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
@@ -189,9 +185,11 @@ template <int D, bool TILE, bool GATED, bool LINEAR>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
             const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmX1,
-            const __grid_constant__ CUtensorMap tmX2, const AttnKParams p) {
+            const __grid_constant__ CUtensorMap tmX2, const __grid_constant__ CUtensorMap tmX3,
+            const AttnKParams p) {
   // tmX1/tmX2: far-field K/V maps (GATED), or the linear state maps (LINEAR): tmX1 the
-  // H'^T rows (box D rows), tmX2 the Z row with 15 rows of zero fill (box 16 rows).
+  // H'^T rows (box D rows), tmX2 the Z row with 15 rows of zero fill (box 16 rows);
+  // tmX3: phi(Q) (LINEAR, same boxes as Q).
   using L = AttnLayout<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -206,8 +204,8 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
   uint64_t* s_full = slot_full + kSlots;         // [2] per S buffer
   uint64_t* p_full = s_full + 2;                 // [2] per S buffer, 256 arrivals
   uint64_t* pv_done = p_full + 2;                // [4] per step mod 4 (phases cannot alias)
-  uint64_t* phiq_ready = pv_done + 4;            // 256 arrivals per tile
-  uint64_t* lin_done = phiq_ready + 1;
+  uint64_t* den_done = pv_done + 4;              // the tile's phi(Q) slot has been read (256 arrivals per tile)
+  uint64_t* lin_done = den_done + 1;
   uint64_t* o_free = lin_done + 1;               // the epilogue has read O_0/O_1 (256 arrivals per tile)
   uint64_t* xch_bar = o_free + 1;                // both shares of every row published (256 arrivals per tile)
   uint64_t* tq_full = xch_bar + 1;               // [kTq] tile slot written
@@ -234,7 +232,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
       mbar_init(&p_full[b], 256);
     }
     for (int b = 0; b < 4; ++b) mbar_init(&pv_done[b], 1);
-    mbar_init(phiq_ready, 256);
+    mbar_init(den_done, 256);
     mbar_init(lin_done, 1);
     mbar_init(o_free, 256);
     mbar_init(xch_bar, 256);
@@ -254,7 +252,8 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
     if (lane == 0) {
       tma_prefetch_desc(&tmQ); tma_prefetch_desc(&tmK); tma_prefetch_desc(&tmV);
       // how the current occupant of each ring slot is released: kind 0 = the P.V of
-      // global step idx, kind 1 = the linear-branch MMAs of local tile idx, -1 = free
+      // global step idx, kind 1 = the linear-branch MMAs of local tile idx, kind 2 = those
+      // MMAs and the softmax warps' denominator reads of local tile idx, -1 = free
       int rel_kind[kSlots], rel_idx[kSlots];
       #pragma unroll
       for (int s = 0; s < kSlots; ++s) { rel_kind[s] = -1; rel_idx[s] = 0; }
@@ -263,7 +262,10 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
           const int q = rel_idx[slot];
           return mbar_wait(&pv_done[q & 3], (q >> 2) & 1, abort_flag, p.status);
         }
-        if (rel_kind[slot] == 1) return mbar_wait(lin_done, rel_idx[slot] & 1, abort_flag, p.status);
+        if (rel_kind[slot] >= 1) {
+          if (!mbar_wait(lin_done, rel_idx[slot] & 1, abort_flag, p.status)) return false;
+          if (rel_kind[slot] == 2) return mbar_wait(den_done, rel_idx[slot] & 1, abort_flag, p.status);
+        }
         return true;
       };
       int i = 0, J = 0, g = 0, q_loaded = -1;
@@ -301,13 +303,16 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
           for (int c = 0; c < L::kChunks; ++c)
             tma_load_3d(sZ + b * L::kZTile + c * L::kZChunk, &tmX2, q_full, c * 64, D, ti.bh * p.n_qb + 2 * ti.pair + b);
         if (LINEAR) {
-          // pre-slots: the states by TMA; the phi(Q) slot is handed to the softmax warps
-          // (plain arrive) once its previous occupant is released; a missing second
-          // query block's slot completes its phase with a plain arrive too
+          // pre-slots by TMA: the states of the two query blocks, then phi(Q); a missing
+          // second query block's slot completes its phase with a plain arrive
           for (int pr = 0; pr < 3 && ok; ++pr, ++g) {
             const int slot = g % kSlots;
             if (!(ok = slot_released(slot))) break;
-            if (pr < ti.n_lin) {
+            if (pr == 2) {
+              mbar_arrive_expect_tx(&slot_full[slot], L::kChunks * L::kTile);
+              for (int c = 0; c < L::kChunks; ++c)
+                tma_load_3d(sRing + slot * L::kKV + c * L::kTile, &tmX3, &slot_full[slot], c * 64, ti.pair * 128, ti.bh);
+            } else if (pr < ti.n_lin) {
               mbar_arrive_expect_tx(&slot_full[slot], L::kHsTile);
               for (int c = 0; c < L::kChunks; ++c)
                 tma_load_3d(sRing + slot * L::kKV + c * L::kHsChunk, &tmX1, &slot_full[slot], c * 64, 0,
@@ -315,7 +320,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
             } else {
               mbar_arrive(&slot_full[slot]);
             }
-            rel_kind[slot] = 1;
+            rel_kind[slot] = pr == 2 ? 2 : 1;
             rel_idx[slot] = i;
           }
         }
@@ -432,7 +437,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
           mma_commit(&s_full[J & 1]);
         }
         if (LINEAR) {
-          ok = mbar_wait(phiq_ready, i & 1, abort_flag, p.status) &&
+          ok = mbar_wait(&slot_full[(g + 2) % kSlots], ((g + 2) / kSlots) & 1, abort_flag, p.status) &&
                mbar_wait(&slot_full[g % kSlots], (g / kSlots) & 1, abort_flag, p.status) &&
                mbar_wait(&slot_full[(g + 1) % kSlots], ((g + 1) / kSlots) & 1, abort_flag, p.status) &&
                (i == 0 || mbar_wait(o_free, (i - 1) & 1, abort_flag, p.status));
@@ -522,45 +527,40 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
       }
       const bool valid = row_exists && (TILE || token_valid(seq, tok));
 
-      // ---- linear branch first (LINEAR): phi(Q) into the tile's third pre-slot (pad rows
-      // -> 0; Q stays in place for the QK MMAs), then the MMA warp's lin = phi(Q) [H'^T ; Z]^T
-      // lands in the O columns; my half of the row, divided by its denominator, is read
+      // ---- linear branch (LINEAR): phi(Q) arrives by TMA in the tile's third pre-slot, and
+      // the MMA warp's lin = phi(Q) H'_b lands in the O columns; my half of the row is read
       // during the first step (before its P is handed over, since the first P.V overwrites
       // those columns) and kept in registers as bf16 pairs (the output is rounded to bf16
-      // in the end as well)
+      // in the end as well).  The denominator phi(q) . Z_b is a dot product over the same
+      // bf16 phi values, my half of the channels here, summed with the other half in the
+      // epilogue.
       uint32_t lin[D / 4];
       #pragma unroll
       for (int k = 0; k < D / 4; ++k) lin[k] = 0u;
-      float den_part = 0.f;                       // phi(q) . Z over my half of the channels
+      float den_part = 0.f;
       if (LINEAR) {
         const int gphi = g + 2;
         ok = __all_sync(0xFFFFFFFFu, mbar_wait(q_full, i & 1, abort_flag, p.status) &&
                                          mbar_wait(&slot_full[gphi % kSlots], (gphi / kSlots) & 1, abort_flag, p.status));
         if (ok) {
-          uint8_t* sPhi = sRing + (gphi % kSlots) * L::kKV;
+          const uint8_t* sPhi = sRing + (gphi % kSlots) * L::kKV;
           const uint8_t* zrow = sZ + half * L::kZTile;     // Z of my query block: row 0 of its Z tile
           constexpr int kGroups = D / 16;                  // 16-byte groups of my row handled by my warpgroup
           #pragma unroll
           for (int gr = 0; gr < kGroups; ++gr) {
             const int gg = wg * kGroups + gr;              // 0 .. D/8-1
-            const int off = (gg >> 3) * L::kTile + sw128_offset(r, gg & 7);
-            const uint4 u = *reinterpret_cast<const uint4*>(sQ + off);
+            const uint4 u = *reinterpret_cast<const uint4*>(sPhi + (gg >> 3) * L::kTile + sw128_offset(r, gg & 7));
             const uint4 zu = *reinterpret_cast<const uint4*>(zrow + (gg >> 3) * L::kZChunk + (gg & 7) * 16);
             const uint32_t w[4] = {u.x, u.y, u.z, u.w};
             const uint32_t zw[4] = {zu.x, zu.y, zu.z, zu.w};
-            uint32_t o4[4];
             #pragma unroll
             for (int k = 0; k < 4; ++k) {
-              o4[k] = valid ? pack_bf16(phi_fast(bf16_lo(w[k])), phi_fast(bf16_hi(w[k]))) : 0u;
-              // the denominator uses the same bf16 phi values the MMA multiplies
-              den_part = fmaf(bf16_lo(o4[k]), bf16_lo(zw[k]), den_part);
-              den_part = fmaf(bf16_hi(o4[k]), bf16_hi(zw[k]), den_part);
+              den_part = fmaf(bf16_lo(w[k]), bf16_lo(zw[k]), den_part);
+              den_part = fmaf(bf16_hi(w[k]), bf16_hi(zw[k]), den_part);
             }
-            *reinterpret_cast<uint4*>(sPhi + off) = make_uint4(o4[0], o4[1], o4[2], o4[3]);
           }
         }
-        fence_proxy_async_smem();
-        mbar_arrive(phiq_ready);
+        mbar_arrive(den_done);
       }
       bool lin_pending = LINEAR;
       auto read_lin = [&]() {
@@ -801,7 +801,7 @@ cudaError_t launch_variant(const AttnArgs& a, const CUtensorMap* maps, const Att
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int grid = kp.n_tiles < sms ? kp.n_tiles : sms;
   if (grid < 1) return cudaSuccess;
-  kern<<<grid, kThreads, L::kBytes, st>>>(maps[0], maps[1], maps[2], maps[3], maps[4], kp);
+  kern<<<grid, kThreads, L::kBytes, st>>>(maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], kp);
   return cudaGetLastError();
 }
 
@@ -817,7 +817,7 @@ cudaError_t launch_d(const AttnArgs& a, const CUtensorMap* maps, const AttnKPara
 cudaError_t launch_attention(const AttnArgs& a, cudaStream_t st) {
   const int D = a.d;
   if (a.tile3d && !a.gated) return cudaErrorInvalidValue;
-  CUtensorMap maps[5];
+  CUtensorMap maps[6];
   const uint64_t rowb = (uint64_t)D * 2;
   if (a.tile3d) {
     const uint64_t dims[5] = {(uint64_t)D, (uint64_t)a.Ww, (uint64_t)a.Hh, (uint64_t)a.F, (uint64_t)a.BH};
@@ -837,6 +837,7 @@ cudaError_t launch_attention(const AttnArgs& a, cudaStream_t st) {
   }
   maps[3] = maps[1];
   maps[4] = maps[2];
+  maps[5] = maps[0];
   if (a.gated) {
     const uint64_t dims[3] = {(uint64_t)D, 64, (uint64_t)a.BH};
     const uint64_t strides[2] = {rowb, rowb * 64};
@@ -851,6 +852,11 @@ cudaError_t launch_attention(const AttnArgs& a, cudaStream_t st) {
     const uint32_t boxz[3] = {64, 16, 1};
     if (!make_tile_map(&maps[3], a.Hs, 3, dims, strides, boxh)) return cudaErrorInvalidValue;
     if (!make_tile_map(&maps[4], a.Hs, 3, dims, strides, boxz)) return cudaErrorInvalidValue;
+    if (!a.phi_q) return cudaErrorInvalidValue;
+    const uint64_t qdims[3] = {(uint64_t)D, (uint64_t)a.s.n_pad, (uint64_t)a.BH};
+    const uint64_t qstrides[2] = {rowb, rowb * a.s.n_pad};
+    const uint32_t boxq[3] = {64, 128, 1};
+    if (!make_tile_map(&maps[5], a.phi_q, 3, qdims, qstrides, boxq)) return cudaErrorInvalidValue;
   }
   AttnKParams kp;
   kp.n_pad = a.s.n_pad; kp.seg_len = a.s.seg_len; kp.seg_stride = a.s.seg_stride;

@@ -6,7 +6,9 @@
 // loads, valid tokens only).  Sums of at most 64 bf16 values are exact in fp64,
 // so the mean does not depend on summation order.  It is written as a bf16 pair
 // hi + lo (hi = bf16(mean), lo = bf16(mean - hi), 16 significant bits together)
-// in the row layout the tensor-core logits GEMM consumes.
+// in the row layout the tensor-core logits GEMM consumes.  With phi_q given, the Q
+// pass also writes phi(Q) = elu(Q) + 1 for every token of the block (0 for pad
+// tokens), the operand of the linear branch the attention kernel applies.
 //
 // far_pool_kernel: the far field of the RoPeSLR gated mode -- K and V averaged
 // over cells of (cf, ch, cw) raster tokens (aixinbiao page: K and V compressed
@@ -21,10 +23,18 @@
 namespace slr {
 namespace {
 
+__device__ __forceinline__ float phi_elu1_ex2(float x) {
+  // elu(x) + 1 = exp(min(x, 0)) + max(x, 0); exp through the exp2 unit (rounded to bf16 after)
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(fminf(x, 0.f) * 1.4426950408889634f));
+  return y + fmaxf(x, 0.f);
+}
+
 template <int D>
 __global__ void __launch_bounds__(128)
 pool_means_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
-                  __nv_bfloat16* __restrict__ qsplit, __nv_bfloat16* __restrict__ ksplit, SeqShape s) {
+                  __nv_bfloat16* __restrict__ qsplit, __nv_bfloat16* __restrict__ ksplit,
+                  __nv_bfloat16* __restrict__ phi_q, SeqShape s) {
   constexpr int kCPR = D / 8;          // 16-byte chunks per row
   constexpr int kRG = 128 / kCPR;      // row groups
   __shared__ double red[kRG][D];
@@ -34,12 +44,33 @@ pool_means_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
   __nv_bfloat16* out = (is_q ? qsplit : ksplit) + ((size_t)bh * s.n_blocks + blk) * 3 * D;
   const int chunk = threadIdx.x % kCPR, rg = threadIdx.x / kCPR;
   const int nvalid = block_valid_count(s, blk);   // valid tokens form a prefix of the block
+  // all of a thread's rows are loaded before any is summed (64 / kRG 16-byte loads in flight)
+  constexpr int kRows = kBlock / kRG;
+  uint4 u[kRows];
+  #pragma unroll
+  for (int k = 0; k < kRows; ++k) {
+    const int r = rg + k * kRG;
+    u[k] = r < nvalid ? __ldg(reinterpret_cast<const uint4*>(x + (size_t)r * D + chunk * 8)) : make_uint4(0, 0, 0, 0);
+  }
+  if (is_q && phi_q) {
+    uint4* dst = reinterpret_cast<uint4*>(phi_q + ((size_t)bh * s.n_pad + (size_t)blk * kBlock) * D);
+    #pragma unroll
+    for (int k = 0; k < kRows; ++k) {
+      const int r = rg + k * kRG;
+      const uint32_t w[4] = {u[k].x, u[k].y, u[k].z, u[k].w};
+      uint32_t o[4];
+      #pragma unroll
+      for (int i = 0; i < 4; ++i)
+        o[i] = r < nvalid ? pack_bf16(phi_elu1_ex2(bf16_lo(w[i])), phi_elu1_ex2(bf16_hi(w[i]))) : 0u;
+      dst[(size_t)r * (D / 8) + chunk] = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+  }
   double acc[8];
   #pragma unroll
   for (int i = 0; i < 8; ++i) acc[i] = 0.0;
-  for (int r = rg; r < nvalid; r += kRG) {
-    const uint4 u = __ldg(reinterpret_cast<const uint4*>(x + (size_t)r * D + chunk * 8));
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+  #pragma unroll
+  for (int k = 0; k < kRows; ++k) {
+    const uint32_t w[4] = {u[k].x, u[k].y, u[k].z, u[k].w};
     #pragma unroll
     for (int i = 0; i < 4; ++i) {
       acc[2 * i] += (double)bf16_lo(w[i]);
@@ -107,15 +138,16 @@ far_pool_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __rest
 
 }  // namespace
 
-cudaError_t launch_pool_means(const void* q, const void* k, void* qsplit, void* ksplit,
+cudaError_t launch_pool_means(const void* q, const void* k, void* qsplit, void* ksplit, void* phi_q,
                               int BH, int d, SeqShape s, cudaStream_t st) {
   dim3 grid(s.n_blocks, BH, 2);
   auto* qs = static_cast<__nv_bfloat16*>(qsplit);
   auto* ks = static_cast<__nv_bfloat16*>(ksplit);
+  auto* pq = static_cast<__nv_bfloat16*>(phi_q);
   if (d == 128)
-    pool_means_kernel<128><<<grid, 128, 0, st>>>((const __nv_bfloat16*)q, (const __nv_bfloat16*)k, qs, ks, s);
+    pool_means_kernel<128><<<grid, 128, 0, st>>>((const __nv_bfloat16*)q, (const __nv_bfloat16*)k, qs, ks, pq, s);
   else
-    pool_means_kernel<64><<<grid, 128, 0, st>>>((const __nv_bfloat16*)q, (const __nv_bfloat16*)k, qs, ks, s);
+    pool_means_kernel<64><<<grid, 128, 0, st>>>((const __nv_bfloat16*)q, (const __nv_bfloat16*)k, qs, ks, pq, s);
   return cudaGetLastError();
 }
 

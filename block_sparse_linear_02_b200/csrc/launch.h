@@ -21,7 +21,8 @@ bool make_tile_map(CUtensorMap* map, const void* base, int rank, const uint64_t*
 // ------------------------------------------------------------ pooling (k_pool.cu)
 // Means of the valid tokens of every 64-token block of q and k, each written as a
 // bf16 pair hi + lo: rows [BH][Nb][3d], [qh | qh | ql] for q and [kh | kl | kh] for k.
-cudaError_t launch_pool_means(const void* q, const void* k, void* qsplit, void* ksplit,
+// With phi_q non-null, also phi(q) = elu(q) + 1 in bf16 [BH][N_pad][d] (pad tokens 0).
+cudaError_t launch_pool_means(const void* q, const void* k, void* qsplit, void* ksplit, void* phi_q,
                               int BH, int d, SeqShape s, cudaStream_t st);
 
 // Far-field K/V: means over cells of (cf, ch, cw) tokens of the raster (F, Hh, Ww),
@@ -95,6 +96,7 @@ struct AttnArgs {
   const int32_t* list_cnt;
   int list_cap, list_per_head;         // list_per_head = 0 when one list serves all heads
   const __nv_bfloat16* Hs;             // SLA linear branch: [BH][n_qb][(d+1)][d] rows [H_i'^T ; Z_i], or null
+  const void* phi_q;                   // SLA linear branch: phi(q) bf16 [BH][n_pad][d] (with Hs)
   void* out;                           // bf16 [BH][n_pad][d]
   float* lse;                          // fp32 [BH][n_pad] or null
   int tile3d;                          // 1: blocks are 4x4x4 tiles of raster (F, Hh, Ww)

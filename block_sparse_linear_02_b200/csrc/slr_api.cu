@@ -117,6 +117,7 @@ struct ClassifyWs {
   __nv_bfloat16 *qsplit, *ksplit;
   uint32_t* keys;
   __nv_bfloat16* m01;
+  __nv_bfloat16* phi_q;                // phi(q) for the linear branch (SLA with marginal blocks)
 };
 
 void plan_classify(Carve& c, const Shape& sh, bool m01, ClassifyWs& w) {
@@ -124,6 +125,7 @@ void plan_classify(Carve& c, const Shape& sh, bool m01, ClassifyWs& w) {
   w.ksplit = c.take<__nv_bfloat16>((size_t)sh.BH * sh.nb * 3 * sh.d);
   w.keys = c.take<uint32_t>((size_t)sh.BH * sh.nb * logits_row_stride(sh.nb));
   w.m01 = m01 ? c.take<__nv_bfloat16>((size_t)sh.BH * sh.nb * ld_m01(sh.nb)) : nullptr;
+  w.phi_q = m01 ? c.take<__nv_bfloat16>((size_t)sh.BH * sh.s.n_pad * sh.d) : nullptr;
 }
 
 struct MarginalWs {
@@ -441,7 +443,7 @@ slr_status slr_pool_classify(const void* q, const void* k, const slr_seq* seq, f
   ClassifyWs w;
   plan_classify(c, sh, false, w);
   SLR_TRY(cudaMemsetAsync(status, 0, sizeof(int), s));
-  SLR_LAUNCH(kKPool, s, launch_pool_means(q, k, w.qsplit, w.ksplit, sh.BH, sh.d, sh.s, s));
+  SLR_LAUNCH(kKPool, s, launch_pool_means(q, k, w.qsplit, w.ksplit, nullptr, sh.BH, sh.d, sh.s, s));
   SLR_LAUNCH(kKLogits, s, launch_logits(w.qsplit, w.ksplit, w.keys, sh.BH, sh.nb, sh.d, status, s));
   SLR_LAUNCH(kKClassify, s, launch_classify(w.keys, sh.BH, sh.nb, sh.d, kc, kn, mask, crit_idx, crit_cnt,
                                             nullptr, 0, scores_opt, nullptr, nullptr, 0, sh.s, status, s));
@@ -532,7 +534,7 @@ slr_status slr_sparse_linear_attn(const void* q, const void* k, const void* v, c
     SLR_LAUNCH(kKAttention, s, launch_attention(a, s));
     return SLR_OK;
   }
-  SLR_LAUNCH(kKPool, s, launch_pool_means(q, k, w.cls.qsplit, w.cls.ksplit, sh.BH, sh.d, sh.s, s));
+  SLR_LAUNCH(kKPool, s, launch_pool_means(q, k, w.cls.qsplit, w.cls.ksplit, w.cls.phi_q, sh.BH, sh.d, sh.s, s));
   SLR_LAUNCH(kKLogits, s, launch_logits(w.cls.qsplit, w.cls.ksplit, w.cls.keys, sh.BH, sh.nb, sh.d, w.status, s));
   SLR_LAUNCH(kKClassify, s, launch_classify(w.cls.keys, sh.BH, sh.nb, sh.d, kc, kn, mask_out_opt, nullptr,
                                             nullptr, w.cls.m01, ld_m01(sh.nb), nullptr, w.list, w.list_cnt, w.cap,
@@ -541,6 +543,7 @@ slr_status slr_sparse_linear_attn(const void* q, const void* k, const void* v, c
     SLR_LAUNCH(kKKeyStates, s, launch_key_states(k, v, w_proj, w.mar.h, sh.BH, sh.d, sh.s, w.status, s));
     SLR_LAUNCH(kKReduce, s, launch_reduce_states(w.cls.m01, ld_m01(sh.nb), w.mar.h, w.mar.Hs, sh.BH, sh.nb, sh.d, w.status, s));
     a.Hs = w.mar.Hs;
+    a.phi_q = w.cls.phi_q;
   }
   a.list = w.list; a.list_cnt = w.list_cnt; a.list_cap = w.cap; a.list_per_head = 1;
   SLR_LAUNCH(kKAttention, s, launch_attention(a, s));
