@@ -578,12 +578,20 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
         }
       };
 
+      // my list entry of step j, read one step ahead
+      auto entry_of = [&](int j) -> Entry {
+        Entry e{0, 64, 3u};
+        const bool far_j = GATED && j == local_steps;
+        if (j < n_steps && !far_j && (wg == 0 || step_blocks(j) == 2)) e = read_entry<TILE>(ti.list, 2 * j + wg, seq);
+        return e;
+      };
+      Entry en_next = entry_of(0);
       for (int j = 0; j < n_steps && ok; ++j) {
         const int Jj = J + j, b = Jj & 1;
         const bool far = GATED && j == local_steps;
         const bool mine = wg == 0 || (!far && step_blocks(j) == 2);   // does this warpgroup own a block here
-        Entry en{0, 64, 3u};
-        if (mine && !far) en = read_entry<TILE>(ti.list, 2 * j + wg, seq);
+        const Entry en = en_next;
+        en_next = entry_of(j + 1);
         if (!__all_sync(0xFFFFFFFFu, mbar_wait(&s_full[b], (Jj >> 1) & 1, abort_flag, p.status))) { ok = false; break; }
         tc_fence_after();
         if (!mine) {
@@ -725,19 +733,19 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
         float v[32];
         #pragma unroll
         for (int m = 0; m < 32; ++m) v[m] = 0.f;
-        if (have_o0) {
+        if (have_o1) {                             // both accumulators, one wait
+          uint32_t o0[32], o1[32];
+          tmem_ld32(lane_addr + kColO0 + cc * 32, o0);
+          tmem_ld32(lane_addr + kColO1 + cc * 32, o1);
+          tmem_wait_ld();
+          #pragma unroll
+          for (int m = 0; m < 32; ++m) v[m] = fmaf(c1, __uint_as_float(o1[m]), c0 * __uint_as_float(o0[m]));
+        } else if (have_o0) {
           uint32_t o0[32];
           tmem_ld32(lane_addr + kColO0 + cc * 32, o0);
           tmem_wait_ld();
           #pragma unroll
           for (int m = 0; m < 32; ++m) v[m] = c0 * __uint_as_float(o0[m]);
-        }
-        if (have_o1) {
-          uint32_t o1[32];
-          tmem_ld32(lane_addr + kColO1 + cc * 32, o1);
-          tmem_wait_ld();
-          #pragma unroll
-          for (int m = 0; m < 32; ++m) v[m] += c1 * __uint_as_float(o1[m]);
         }
         if (GATED && ok) {
           uint32_t of[32];
