@@ -610,8 +610,33 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
         const bool attend = (en.flags >> half) & 1u;
         const int nvalid = attend ? en.nvalid : 0;
         tmem_wait_ld();
+        // A full block against a running max already set: exponentials against that max
+        // with the row max taken in the same pass; only a row whose max then rises past
+        // the lazy-rescale threshold repeats the pass (the same P as with the max first).
+        // Not in the LINEAR variant, which holds the linear result in registers and ran
+        // slower with the fused pass.
+        const bool spec = !LINEAR && !far && nvalid == 64 && m_run != -INFINITY;
         float mx = -INFINITY;
-        if (nvalid == 64) {
+        uint32_t packed[32];
+        float rowsum = 0.f;
+        if (spec) {
+          float acc0 = 0.f, acc1 = 0.f, mx0 = -INFINITY, mx1 = -INFINITY;
+          #pragma unroll
+          for (int c = 0; c < 64; c += 4) {
+            const float s0 = __uint_as_float(sr[c]), s1 = __uint_as_float(sr[c + 1]);
+            const float s2 = __uint_as_float(sr[c + 2]), s3 = __uint_as_float(sr[c + 3]);
+            const float p0 = ex2(fmaf(s0, sl, -m_run)), p1 = ex2(fmaf(s1, sl, -m_run));
+            const float p2 = ex2(fmaf(s2, sl, -m_run)), p3 = ex2(fmaf(s3, sl, -m_run));
+            acc0 += p0 + p2;
+            acc1 += p1 + p3;
+            packed[c >> 1] = pack_bf16(p0, p1);
+            packed[(c >> 1) + 1] = pack_bf16(p2, p3);
+            mx0 = max3(mx0, s0, s1);
+            mx1 = max3(mx1, s2, s3);
+          }
+          rowsum = acc0 + acc1;
+          mx = fmaxf(mx0, mx1);
+        } else if (nvalid == 64) {
           float t3[22];
           #pragma unroll
           for (int k = 0; k < 21; ++k)
@@ -646,22 +671,23 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
           mu = m_run;
         }
         if (mu == -INFINITY) mu = 0.f;
-        uint32_t packed[32];
-        float rowsum = 0.f;
-        if (nvalid == 0) {
-          #pragma unroll
-          for (int c = 0; c < 32; ++c) packed[c] = 0u;
-        } else {
-          float acc0 = 0.f, acc1 = 0.f;
-          #pragma unroll
-          for (int c = 0; c < 64; c += 2) {
-            const float p0 = ex2(fmaf(__uint_as_float(sr[c]), sl, -mu));
-            const float p1 = ex2(fmaf(__uint_as_float(sr[c + 1]), sl, -mu));
-            acc0 += p0;
-            acc1 += p1;
-            packed[c >> 1] = pack_bf16(p0, p1);
+        if (!spec || need) {
+          rowsum = 0.f;
+          if (nvalid == 0) {
+            #pragma unroll
+            for (int c = 0; c < 32; ++c) packed[c] = 0u;
+          } else {
+            float acc0 = 0.f, acc1 = 0.f;
+            #pragma unroll
+            for (int c = 0; c < 64; c += 2) {
+              const float p0 = ex2(fmaf(__uint_as_float(sr[c]), sl, -mu));
+              const float p1 = ex2(fmaf(__uint_as_float(sr[c + 1]), sl, -mu));
+              acc0 += p0;
+              acc1 += p1;
+              packed[c >> 1] = pack_bf16(p0, p1);
+            }
+            rowsum = acc0 + acc1;
           }
-          rowsum = acc0 + acc1;
         }
         if (far) l_far = rowsum; else l_run += rowsum;
         // rescale my accumulator (once it holds data) after the previous P.V has completed
