@@ -98,6 +98,25 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// Paired fp32 arithmetic: one instruction does the work of two, rounded as the scalar forms.
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+
 __device__ __forceinline__ float max3(float a, float b, float c) {
   float r;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
@@ -127,27 +146,12 @@ __device__ __forceinline__ void mma_bf16_ss_masked(uint32_t d_tmem, uint64_t a_d
                   "r"(mask[0]), "r"(mask[1]), "r"(mask[2]), "r"(mask[3]) : "memory");
 }
 
-// List entry: key block in bits [0,16), valid keys in bits [16,23), bit 30/31: half 0/1 attends.
+// List word: key block in bits [0,16), valid keys in bits [16,23), bit 30/31: half 0/1
+// attends.  The softmax side needs the valid-key count and the two attend bits.
 struct Entry {
-  int kb, nvalid;
+  int nvalid;
   uint32_t flags;
 };
-
-template <bool TILE>
-__device__ __forceinline__ Entry read_entry(const uint32_t* list, int idx, const SeqShape& s) {
-  Entry e;
-  if (list) {
-    const uint32_t w = list[idx];
-    e.kb = (int)(w & 0xFFFFu);
-    e.nvalid = (int)((w >> 16) & 0x7Fu);
-    e.flags = w >> 30;
-  } else {
-    e.kb = idx;
-    e.nvalid = TILE ? 64 : block_valid_count(s, idx);
-    e.flags = 3u;
-  }
-  return e;
-}
 
 // Per-tile quantities every role derives from the tile index.
 struct TileInfo {
@@ -374,23 +378,27 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
       constexpr uint32_t idS = idesc_bf16(128, 128, false, false);
       constexpr uint32_t idO = idesc_bf16(128, D, false, true);
       const uint32_t q_addr = smem_u32(sQ), ring_addr = smem_u32(sRing);
+      // Shared-memory descriptors: the start-address field is (address >> 4) in the low 14
+      // bits and every operand lies below 256 KB, so an operand's descriptor is a base
+      // descriptor plus its byte offset >> 4.
+      const uint64_t dQ = desc_kmajor(q_addr);
+      const uint64_t dK = desc_kmajor(ring_addr);
+      const uint64_t dV = desc_mnmajor(ring_addr, L::kTile);
       auto issue_qk = [&](int slot, int sbuf) {
+        const uint64_t db = dK + (uint32_t)((slot * L::kKV) >> 4);
         #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const int c = kk >> 2, sub = kk & 3;
-          const uint64_t a = desc_kmajor(q_addr + c * L::kTile + sub * 32);
-          const uint64_t b = desc_kmajor(ring_addr + slot * L::kKV + c * L::kTile + sub * 32);
-          mma_bf16_ss(tmem + kColS + sbuf * 128, a, b, idS, kk > 0 ? 1u : 0u);
+          const uint32_t off = (uint32_t)(((kk >> 2) * L::kTile + (kk & 3) * 32) >> 4);
+          mma_bf16_ss(tmem + kColS + sbuf * 128, dQ + off, db + off, idS, kk > 0 ? 1u : 0u);
         }
       };
       // O_dst (+)= P[:, 64*blk .. +64] V_blk; P lives in TMEM over the step's S buffer
       auto issue_pv = [&](int slot, int sbuf, int blk, uint32_t col, bool acc) {
+        const uint64_t db = dV + (uint32_t)((slot * L::kKV + blk * L::kHalf) >> 4);
+        const uint32_t a = tmem + kColS + sbuf * 128 + blk * 64;
         #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          const uint32_t a = tmem + kColS + sbuf * 128 + blk * 64 + kk * 8;
-          const uint64_t b = desc_mnmajor(ring_addr + slot * L::kKV + blk * L::kHalf + kk * 2048, L::kTile);
-          mma_bf16_ts(tmem + col, a, b, idO, (acc || kk > 0) ? 1u : 0u);
-        }
+        for (int kk = 0; kk < 4; ++kk)
+          mma_bf16_ts(tmem + col, a + kk * 8, db + (uint32_t)(kk * 2048 >> 4), idO, (acc || kk > 0) ? 1u : 0u);
       };
       // lin = phi(Q) H'_b per query block b (lanes of the other block masked off) into the
       // O columns, before any P.V; the denominators phi(q) . Z_b are dot products the
@@ -578,20 +586,20 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
         }
       };
 
-      // my list entry of step j, read one step ahead
-      auto entry_of = [&](int j) -> Entry {
-        Entry e{0, 64, 3u};
+      // my list word of step j, loaded one step ahead and decoded only where it is used, so
+      // that the load's latency is not waited for at the top of the step
+      auto word_of = [&](int j) -> uint32_t {
         const bool far_j = GATED && j == local_steps;
-        if (j < n_steps && !far_j && (wg == 0 || step_blocks(j) == 2)) e = read_entry<TILE>(ti.list, 2 * j + wg, seq);
-        return e;
+        if (ti.list && j < n_steps && !far_j && (wg == 0 || step_blocks(j) == 2)) return ti.list[2 * j + wg];
+        return 0u;
       };
-      Entry en_next = entry_of(0);
+      uint32_t w_next = word_of(0);
       for (int j = 0; j < n_steps && ok; ++j) {
         const int Jj = J + j, b = Jj & 1;
         const bool far = GATED && j == local_steps;
         const bool mine = wg == 0 || (!far && step_blocks(j) == 2);   // does this warpgroup own a block here
-        const Entry en = en_next;
-        en_next = entry_of(j + 1);
+        const uint32_t w_cur = w_next;
+        w_next = word_of(j + 1);
         if (!__all_sync(0xFFFFFFFFu, mbar_wait(&s_full[b], (Jj >> 1) & 1, abort_flag, p.status))) { ok = false; break; }
         tc_fence_after();
         if (!mine) {
@@ -607,6 +615,15 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
         uint32_t sr[64];
         tmem_ld32(s_addr, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
         tmem_ld32(s_addr + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+        Entry en{64, 3u};
+        if (!far) {
+          if (ti.list) {
+            en.nvalid = (int)((w_cur >> 16) & 0x7Fu);
+            en.flags = w_cur >> 30;
+          } else if (!TILE) {
+            en.nvalid = block_valid_count(seq, 2 * j + wg);
+          }
+        }
         const bool attend = (en.flags >> half) & 1u;
         const int nvalid = attend ? en.nvalid : 0;
         tmem_wait_ld();
@@ -620,21 +637,22 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
         uint32_t packed[32];
         float rowsum = 0.f;
         if (spec) {
-          float acc0 = 0.f, acc1 = 0.f, mx0 = -INFINITY, mx1 = -INFINITY;
+          const float2 sl2 = make_float2(sl, sl), nm2 = make_float2(-m_run, -m_run);
+          float2 acc = make_float2(0.f, 0.f);
+          float mx0 = -INFINITY, mx1 = -INFINITY;
           #pragma unroll
           for (int c = 0; c < 64; c += 4) {
             const float s0 = __uint_as_float(sr[c]), s1 = __uint_as_float(sr[c + 1]);
             const float s2 = __uint_as_float(sr[c + 2]), s3 = __uint_as_float(sr[c + 3]);
-            const float p0 = ex2(fmaf(s0, sl, -m_run)), p1 = ex2(fmaf(s1, sl, -m_run));
-            const float p2 = ex2(fmaf(s2, sl, -m_run)), p3 = ex2(fmaf(s3, sl, -m_run));
-            acc0 += p0 + p2;
-            acc1 += p1 + p3;
+            const float2 x01 = fma2(make_float2(s0, s1), sl2, nm2), x23 = fma2(make_float2(s2, s3), sl2, nm2);
+            const float p0 = ex2(x01.x), p1 = ex2(x01.y), p2 = ex2(x23.x), p3 = ex2(x23.y);
+            acc = add2(acc, add2(make_float2(p0, p1), make_float2(p2, p3)));
             packed[c >> 1] = pack_bf16(p0, p1);
             packed[(c >> 1) + 1] = pack_bf16(p2, p3);
             mx0 = max3(mx0, s0, s1);
             mx1 = max3(mx1, s2, s3);
           }
-          rowsum = acc0 + acc1;
+          rowsum = acc.x + acc.y;
           mx = fmaxf(mx0, mx1);
         } else if (nvalid == 64) {
           float t3[22];
@@ -677,16 +695,16 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
             #pragma unroll
             for (int c = 0; c < 32; ++c) packed[c] = 0u;
           } else {
-            float acc0 = 0.f, acc1 = 0.f;
+            const float2 sl2 = make_float2(sl, sl), nm2 = make_float2(-mu, -mu);
+            float2 acc = make_float2(0.f, 0.f);
             #pragma unroll
             for (int c = 0; c < 64; c += 2) {
-              const float p0 = ex2(fmaf(__uint_as_float(sr[c]), sl, -mu));
-              const float p1 = ex2(fmaf(__uint_as_float(sr[c + 1]), sl, -mu));
-              acc0 += p0;
-              acc1 += p1;
+              const float2 x = fma2(make_float2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), sl2, nm2);
+              const float p0 = ex2(x.x), p1 = ex2(x.y);
+              acc = add2(acc, make_float2(p0, p1));
               packed[c >> 1] = pack_bf16(p0, p1);
             }
-            rowsum = acc0 + acc1;
+            rowsum = acc.x + acc.y;
           }
         }
         if (far) l_far = rowsum; else l_run += rowsum;
