@@ -523,21 +523,28 @@ key_states_pipe_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_con
 // state columns) of every head; a 4-stage TMA ring runs across tile boundaries
 // and two TMEM accumulators let the epilogue of one tile overlap the main loop
 // of the next.  Tiles are ordered M-fastest so the query-block tiles sharing one
-// slab of h run back to back (h is read from HBM about once).
+// slab of h run back to back (h is read from HBM about once).  Each epilogue warp
+// stages its 32 rows x 64 columns per chunk in a 128B-swizzled tile and writes it
+// with a TMA tensor store (whole 128-byte row segments instead of 16-byte pieces
+// of 32 different rows).
 constexpr int kGemmStages = 4;
 constexpr int kGemmBN = 256;
 constexpr int kGemmABytes = 128 * 128;          // 128 rows x 64 bf16
 constexpr int kGemmBBytes = 4 * 64 * 128;       // 4 chunks of 64 K-rows x 64 bf16
-constexpr int kGemmSmem = kGemmStages * (kGemmABytes + kGemmBBytes) + 256 + 1024;
+constexpr int kGemmOutBytes = 32 * 128;         // one warp's staged chunk: 32 rows x 64 bf16
+constexpr int kGemmOutOff = kGemmStages * (kGemmABytes + kGemmBBytes);   // [4 warps][2 buffers]
+constexpr int kGemmBarOff = kGemmOutOff + 4 * 2 * kGemmOutBytes;
+constexpr int kGemmSmem = kGemmBarOff + 256 + 1024;
+static_assert(kGemmSmem <= 227 * 1024, "shared memory budget");
 
 __global__ void __launch_bounds__(192, 1)
 reduce_states_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                     __nv_bfloat16* __restrict__ Hs, int nb, int ntot, int BH, int* status) {
+                     const __grid_constant__ CUtensorMap tmHs, int nb, int ntot, int BH, int* status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint8_t* sA = smem;
   uint8_t* sB = smem + kGemmStages * kGemmABytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kGemmStages * (kGemmABytes + kGemmBBytes));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kGemmBarOff);
   uint64_t* full = bars;                          // [4]
   uint64_t* empty = bars + kGemmStages;           // [4]
   uint64_t* acc_full = empty + kGemmStages;       // [2] MMA -> epilogue
@@ -616,33 +623,47 @@ reduce_states_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
       }
     }
   } else {
-    const int r = threadIdx.x;
-    int local = 0;
+    // epilogue warps 0-3: TMEM lanes 32*warp.. = output rows m0 + 32*warp ..
+    uint8_t* sOut = smem + kGemmOutOff + warp * 2 * kGemmOutBytes;
+    int local = 0, chunk = 0;                     // chunk: this warp's store count, for the 2 staging buffers
     for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++local) {
       const int ab = local & 1;
       const int m0 = (t % mt) * 128, n0 = ((t / mt) % nt) * kGemmBN, bh = t / (mt * nt);
       if (!__all_sync(0xFFFFFFFFu, mbar_wait(&acc_full[ab], (local >> 1) & 1, abort_flag, status))) break;
       tc_fence_after();
-      const int m = m0 + r;
       #pragma unroll 1
-      for (int cc = 0; cc < kGemmBN / 32; ++cc) {
-        uint32_t v[32];
-        tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + ab * kGemmBN + cc * 32, v);
+      for (int q = 0; q < kGemmBN / 64; ++q) {
+        const int n = n0 + q * 64;
+        if (n >= ntot) break;                      // uniform: the columns past the end have nothing to store
+        uint32_t v[64];
+        tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + ab * kGemmBN + q * 64, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+        tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + ab * kGemmBN + q * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+        uint8_t* buf = sOut + (chunk & 1) * kGemmOutBytes;
+        if (lane == 0) bulk_wait_read_1();         // the store issued from this buffer two chunks ago has read it
+        __syncwarp();
         tmem_wait_ld();
-        const int n = n0 + cc * 32;
-        if (m < nb && n < ntot) {
-          uint4* dst = reinterpret_cast<uint4*>(Hs + ((size_t)bh * nb + m) * ntot + n);
-          #pragma unroll
-          for (int i = 0; i < 4; ++i)
-            dst[i] = make_uint4(pack_bf16(__uint_as_float(v[8 * i]), __uint_as_float(v[8 * i + 1])),
-                                pack_bf16(__uint_as_float(v[8 * i + 2]), __uint_as_float(v[8 * i + 3])),
-                                pack_bf16(__uint_as_float(v[8 * i + 4]), __uint_as_float(v[8 * i + 5])),
-                                pack_bf16(__uint_as_float(v[8 * i + 6]), __uint_as_float(v[8 * i + 7])));
+        #pragma unroll
+        for (int i = 0; i < 8; ++i)
+          *reinterpret_cast<uint4*>(buf + sw128_offset(lane, i)) =
+              make_uint4(pack_bf16(__uint_as_float(v[8 * i]), __uint_as_float(v[8 * i + 1])),
+                         pack_bf16(__uint_as_float(v[8 * i + 2]), __uint_as_float(v[8 * i + 3])),
+                         pack_bf16(__uint_as_float(v[8 * i + 4]), __uint_as_float(v[8 * i + 5])),
+                         pack_bf16(__uint_as_float(v[8 * i + 6]), __uint_as_float(v[8 * i + 7])));
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          // rows past nb inside the box are clipped by the tensor map; a box wholly past
+          // nb is not stored, but its (empty) group is still committed so that the
+          // two-buffer wait above stays counted per chunk
+          if (m0 + warp * 32 < nb) tma_store_3d(&tmHs, buf, n, m0 + warp * 32, bh);
+          bulk_commit();
         }
+        ++chunk;
       }
       tc_fence_before();
       mbar_arrive(&acc_empty[ab]);
     }
+    if (lane == 0) bulk_wait_all();
   }
   tc_fence_before();
   __syncthreads();
@@ -838,14 +859,16 @@ cudaError_t launch_key_states(const void* k, const void* v, const void* w_proj, 
 cudaError_t launch_reduce_states(const __nv_bfloat16* m01, int ld_m01, const __nv_bfloat16* h,
                                  __nv_bfloat16* Hs, int BH, int nb, int d, int* status, cudaStream_t st) {
   const int ntot = (d + 1) * d;
-  CUtensorMap ma, mb;
+  CUtensorMap ma, mb, mo;
   const uint64_t adims[3] = {(uint64_t)ld_m01, (uint64_t)nb, (uint64_t)BH};
   const uint64_t astr[2] = {(uint64_t)ld_m01 * 2, (uint64_t)ld_m01 * 2 * nb};
   const uint32_t abox[3] = {64, 128, 1};
   const uint64_t bdims[3] = {(uint64_t)ntot, (uint64_t)nb, (uint64_t)BH};
   const uint64_t bstr[2] = {(uint64_t)ntot * 2, (uint64_t)ntot * 2 * nb};
   const uint32_t bbox[3] = {64, 64, 1};
-  if (!make_tile_map(&ma, m01, 3, adims, astr, abox) || !make_tile_map(&mb, h, 3, bdims, bstr, bbox))
+  const uint32_t obox[3] = {64, 32, 1};           // Hs [BH][nb][ntot]: one warp's 32 rows x 64 columns
+  if (!make_tile_map(&ma, m01, 3, adims, astr, abox) || !make_tile_map(&mb, h, 3, bdims, bstr, bbox) ||
+      !make_tile_map(&mo, Hs, 3, bdims, bstr, obox))
     return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(reduce_states_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem);
   if (e != cudaSuccess) return e;
@@ -854,7 +877,7 @@ cudaError_t launch_reduce_states(const __nv_bfloat16* m01, int ld_m01, const __n
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const long long tiles = (long long)((nb + 127) / 128) * ((ntot + kGemmBN - 1) / kGemmBN) * BH;
   const int grid = (int)(tiles < sms ? tiles : sms);
-  reduce_states_kernel<<<grid, 192, kGemmSmem, st>>>(ma, mb, Hs, nb, ntot, BH, status);
+  reduce_states_kernel<<<grid, 192, kGemmSmem, st>>>(ma, mb, mo, nb, ntot, BH, status);
   return cudaGetLastError();
 }
 
