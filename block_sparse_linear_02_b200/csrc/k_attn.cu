@@ -64,7 +64,11 @@ struct AttnLayout {
   static constexpr int kZOff = kRingOff + kSlots * kKV;  // Z tiles of the pair's two query blocks
   static constexpr int kXOff = kZOff + 2 * kZTile;       // exchange area: [2 shares][2 tiles][3][128] floats
   static constexpr int kBarOff = kXOff + 12 * 128 * 4;
-  static constexpr int kBytes = kBarOff + 256 + 1024;    // + alignment slack
+  // output staging (non-tile layouts): per softmax warp one 32-row x 32-column bf16
+  // chunk (64-byte rows, 64-byte swizzle), written to HBM by TMA tensor stores
+  static constexpr int kOutChunk = 32 * 64;
+  static constexpr int kOutOff = (kBarOff + 256 + 1023) / 1024 * 1024;
+  static constexpr int kBytes = kOutOff + 8 * kOutChunk + 1024;   // + alignment slack
   static_assert(kHsTile <= kKV, "a linear state tile must fit in one ring slot");
   static_assert(kBytes <= 227 * 1024, "shared memory budget");
 };
@@ -190,10 +194,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
             const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmX1,
             const __grid_constant__ CUtensorMap tmX2, const __grid_constant__ CUtensorMap tmX3,
-            const AttnKParams p) {
+            const __grid_constant__ CUtensorMap tmO, const AttnKParams p) {
   // tmX1/tmX2: far-field K/V maps (GATED), or the linear state maps (LINEAR): tmX1 the
   // H'^T rows (box D rows), tmX2 the Z row with 15 rows of zero fill (box 16 rows);
-  // tmX3: phi(Q) (LINEAR, same boxes as Q).
+  // tmX3: phi(Q) (LINEAR, same boxes as Q).  tmO: the output, boxes of 32 rows x 32
+  // columns with 64-byte swizzle (not used by the tile layout).
   using L = AttnLayout<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -201,6 +206,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
   uint8_t* sRing = smem + L::kRingOff;
   uint8_t* sZ = smem + L::kZOff;
   float* xch = reinterpret_cast<float*>(smem + L::kXOff);   // [2 tiles][3][128]: m, l, far-l per warpgroup share
+  uint8_t* sOut = smem + L::kOutOff;                         // [8 softmax warps] output staging chunks
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
   uint64_t* q_full = bars + 0;                   // Q (and Z) of the current tile landed
   uint64_t* q_free = q_full + 1;                 // every MMA reading Q / Z of a tile has completed
@@ -805,15 +811,39 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
             v[2 * m + 1] = fmaf(bf16_hi(lin[k * 16 + m]), inv_den, v[2 * m + 1]);
           }
         }
-        if (!row_exists) continue;
-        uint4* dst = reinterpret_cast<uint4*>(p.out + row_off + cc * 32);
-        #pragma unroll
-        for (int m = 0; m < 4; ++m) {
-          uint4 w4 = make_uint4(0, 0, 0, 0);
-          if (valid)
-            w4 = make_uint4(pack_bf16(v[8 * m], v[8 * m + 1]), pack_bf16(v[8 * m + 2], v[8 * m + 3]),
-                            pack_bf16(v[8 * m + 4], v[8 * m + 5]), pack_bf16(v[8 * m + 6], v[8 * m + 7]));
-          dst[m] = w4;
+        if (TILE) {
+          if (!row_exists) continue;
+          uint4* dst = reinterpret_cast<uint4*>(p.out + row_off + cc * 32);
+          #pragma unroll
+          for (int m = 0; m < 4; ++m) {
+            uint4 w4 = make_uint4(0, 0, 0, 0);
+            if (valid)
+              w4 = make_uint4(pack_bf16(v[8 * m], v[8 * m + 1]), pack_bf16(v[8 * m + 2], v[8 * m + 3]),
+                              pack_bf16(v[8 * m + 4], v[8 * m + 5]), pack_bf16(v[8 * m + 6], v[8 * m + 7]));
+            dst[m] = w4;
+          }
+        } else {
+          // my row's 32 columns into the warp's staging chunk (64-byte swizzle: 16-byte piece
+          // m of row r sits at piece m ^ ((r >> 1) & 3)), then one TMA store of 32 rows; the
+          // rows past the sequence end are clipped by the tensor map
+          uint8_t* stg = sOut + warp * L::kOutChunk;
+          if (lane == 0) bulk_wait_read_all();     // the last store from this chunk has read it
+          __syncwarp();
+          #pragma unroll
+          for (int m = 0; m < 4; ++m) {
+            uint4 w4 = make_uint4(0, 0, 0, 0);
+            if (valid)
+              w4 = make_uint4(pack_bf16(v[8 * m], v[8 * m + 1]), pack_bf16(v[8 * m + 2], v[8 * m + 3]),
+                              pack_bf16(v[8 * m + 4], v[8 * m + 5]), pack_bf16(v[8 * m + 6], v[8 * m + 7]));
+            *reinterpret_cast<uint4*>(stg + lane * 64 + ((m ^ ((lane >> 1) & 3)) << 4)) = w4;
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            const int row0 = ti.pair * 128 + (warp & 3) * 32;
+            if (row0 < p.n_pad) tma_store_3d(&tmO, stg, cc * 32, row0, ti.bh);
+            bulk_commit();
+          }
         }
       }
       tc_fence_before();
@@ -829,6 +859,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
     }
   }
 
+  if (!TILE && warp < 8 && lane == 0) bulk_wait_all();   // output stores complete
   tc_fence_before();
   __syncthreads();
   if (warp == 9) {
@@ -853,7 +884,7 @@ cudaError_t launch_variant(const AttnArgs& a, const CUtensorMap* maps, const Att
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int grid = kp.n_tiles < sms ? kp.n_tiles : sms;
   if (grid < 1) return cudaSuccess;
-  kern<<<grid, kThreads, L::kBytes, st>>>(maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], kp);
+  kern<<<grid, kThreads, L::kBytes, st>>>(maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], maps[6], kp);
   return cudaGetLastError();
 }
 
@@ -869,7 +900,7 @@ cudaError_t launch_d(const AttnArgs& a, const CUtensorMap* maps, const AttnKPara
 cudaError_t launch_attention(const AttnArgs& a, cudaStream_t st) {
   const int D = a.d;
   if (a.tile3d && !a.gated) return cudaErrorInvalidValue;
-  CUtensorMap maps[6];
+  CUtensorMap maps[7];
   const uint64_t rowb = (uint64_t)D * 2;
   if (a.tile3d) {
     const uint64_t dims[5] = {(uint64_t)D, (uint64_t)a.Ww, (uint64_t)a.Hh, (uint64_t)a.F, (uint64_t)a.BH};
@@ -890,6 +921,13 @@ cudaError_t launch_attention(const AttnArgs& a, cudaStream_t st) {
   maps[3] = maps[1];
   maps[4] = maps[2];
   maps[5] = maps[0];
+  maps[6] = maps[0];
+  if (!a.tile3d) {
+    const uint64_t dims[3] = {(uint64_t)D, (uint64_t)a.s.n_pad, (uint64_t)a.BH};
+    const uint64_t strides[2] = {rowb, rowb * a.s.n_pad};
+    const uint32_t boxo[3] = {32, 32, 1};
+    if (!make_tile_map(&maps[6], a.out, 3, dims, strides, boxo, 64)) return cudaErrorInvalidValue;
+  }
   if (a.gated) {
     const uint64_t dims[3] = {(uint64_t)D, 64, (uint64_t)a.BH};
     const uint64_t strides[2] = {rowb, rowb * 64};

@@ -15,8 +15,10 @@ namespace slr {
 // ------------------------------------------------------------ tensor maps
 // A tile map over a bf16 tensor whose innermost dimension is contiguous.
 // dims[0] is the innermost extent (elements), strides are in bytes for dims 1..rank-1.
+// swizzle_bytes: 128 (the default), 64, 32 or 0 (none); the box's inner extent in
+// bytes must not exceed it when it is not 0.
 bool make_tile_map(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
-                   const uint64_t* strides_bytes, const uint32_t* box);
+                   const uint64_t* strides_bytes, const uint32_t* box, int swizzle_bytes = 128);
 
 // ------------------------------------------------------------ pooling (k_pool.cu)
 // Means of the valid tokens of every 64-token block of q and k, each written as a
