@@ -7,13 +7,14 @@
 //   LINEAR  (SLA): the linear-attention branch of the same query block is added,
 //           O = O_s + phi(Q_i) H_i' / (phi(Q_i) . Z_i) with H_i' = sum of
 //           phi(K_j)^T V_j W_proj over its marginal blocks -- one more MMA of
-//           phi(Q) against the [H_i'^T ; Z_i] rows (the last row gives the
-//           denominator as an extra output column);
+//           phi(Q) against the H_i'^T rows, and the denominator as a dot product
+//           of phi(q) with Z_i in the softmax warps;
 //   GATED   (RoPeSLR page): a far-field block of 64 pooled tokens with its own
 //           softmax, combined as g*local + (1-g)*far.
 //
-// One CTA owns a PAIR of consecutive query blocks (128 query rows = the M of a
-// tcgen05 MMA) and walks the union of their key-block sets; each list entry
+// A tile is a PAIR of consecutive query blocks (128 query rows = the M of a
+// tcgen05 MMA); the kernel is persistent (one CTA per SM takes tiles from a global
+// queue) and a tile walks the union of its key-block sets; each list entry
 // carries the block's valid-key count and one flag per half of the pair.  The
 // list is consumed two entries per STEP (128 keys): one 128x128 S tile per step
 // keeps the MMA instruction count and the commits per key low.
@@ -32,7 +33,9 @@
 // accumulator O_w) over its share of the key blocks; the epilogue merges the two
 // shares exactly: O = (2^(m0-M) O_0 + 2^(m1-M) O_1) / (2^(m0-M) l_0 + 2^(m1-M) l_1).
 // The softmax works in the exp2 domain with lazy rescaling (an accumulator is
-// rescaled only when its running max grows by more than 2^8).
+// rescaled only when its running max grows by more than 2^8).  In the row-major
+// layouts the output leaves through shared memory: each softmax warp stages its 32
+// rows x 32 columns and one TMA tensor store writes them.
 #include <cuda_runtime.h>
 #include <math.h>
 
@@ -47,7 +50,6 @@ constexpr int kThreads = 320;
 constexpr uint32_t kColO0 = 0;      // accumulator of warpgroup 0
 constexpr uint32_t kColO1 = 128;    // accumulator of warpgroup 1
 constexpr uint32_t kColS = 256;     // two 128-column S/P buffers: [256, 384) and [384, 512)
-constexpr float kLog2e = 1.4426950408889634f;
 
 template <int D>
 struct AttnLayout {
@@ -125,10 +127,6 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
   float r;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
   return r;
-}
-
-__device__ __forceinline__ void tmem_ld1(uint32_t taddr, uint32_t& r) {
-  asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(r) : "r"(taddr));
 }
 
 // D[tmem] (+)= A[tmem] * B[smem]^T (A: row m in lane m, two bf16 of K per column).
