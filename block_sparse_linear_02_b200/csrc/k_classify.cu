@@ -48,30 +48,39 @@ __device__ __forceinline__ float okey_value(uint32_t k) {
 __device__ __forceinline__ int warp_sum(int v) { return (int)__reduce_add_sync(0xFFFFFFFFu, (unsigned)v); }
 
 // ------------------------------------------------------------------ logits GEMM
+// One 128x128 logit tile per CTA, K = 3d streamed through a 3-stage ring of (A, B)
+// 64-column chunks, so that two CTAs fit on an SM and the tiles of a head run in one
+// wave.  Roles: thread 0 loads, thread 32 issues the MMAs; then every warp turns its
+// 32 rows into keys, stages them 128B-swizzled in the (then idle) ring and writes
+// them with TMA tensor stores.
 template <int D>
 struct LgLayout {
   static constexpr int kChunks = 3 * D / 64;          // K = 3d in chunks of 64
   static constexpr int kTile = 128 * 128;             // 128 rows x 64 bf16
-  static constexpr int kBOff = kChunks * kTile;
-  static constexpr int kBarOff = 2 * kChunks * kTile;
+  static constexpr int kStages = 3;
+  static constexpr int kStage = 2 * kTile;            // A chunk, then B chunk
+  static constexpr int kOutChunk = 32 * 128;          // one warp's 32 rows x 32 keys
+  static constexpr int kBarOff = kStages * kStage;
   static constexpr int kBytes = kBarOff + 256 + 1024; // + alignment slack
+  static_assert(16 * kOutChunk <= kStages * kStage, "key staging reuses the ring");
 };
 
 template <int D>
-__global__ void __launch_bounds__(128, 1)
+__global__ void __launch_bounds__(128, 2)
 logits_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-              uint32_t* __restrict__ keys, int nb, int nbp, int* status) {
+              const __grid_constant__ CUtensorMap tmKeys, int nb, int nbp, int* status) {
   using L = LgLayout<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBarOff);   // [kChunks]
-  uint64_t* done = full + L::kChunks;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBarOff);   // [kStages]
+  uint64_t* empty = full + L::kStages;                              // [kStages]
+  uint64_t* done = empty + L::kStages;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   const int n0 = blockIdx.x * 128, m0 = blockIdx.y * 128, bh = blockIdx.z;
-  const int warp = threadIdx.x >> 5;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    for (int c = 0; c < L::kChunks; ++c) mbar_init(&full[c], 1);
+    for (int s = 0; s < L::kStages; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
     mbar_init(done, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -83,50 +92,64 @@ logits_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
   const uint32_t tmem = *tmem_slot;
 
   if (threadIdx.x == 0) {
+    // ---- loads
+    int issued = 0;
     for (int c = 0; c < L::kChunks; ++c) {
-      mbar_arrive_expect_tx(&full[c], 2 * L::kTile);
-      tma_load_3d(smem + c * L::kTile, &tmA, &full[c], c * 64, m0, bh);
-      tma_load_3d(smem + L::kBOff + c * L::kTile, &tmB, &full[c], c * 64, n0, bh);
+      const int s = c % L::kStages;
+      if (c >= L::kStages && !mbar_wait(&empty[s], ((c / L::kStages) - 1) & 1, abort_flag, status)) break;
+      mbar_arrive_expect_tx(&full[s], L::kStage);
+      tma_load_3d(smem + s * L::kStage, &tmA, &full[s], c * 64, m0, bh);
+      tma_load_3d(smem + s * L::kStage + L::kTile, &tmB, &full[s], c * 64, n0, bh);
+      ++issued;
     }
-    constexpr uint32_t id = idesc_bf16(128, 128, false, false);
-    bool ok = true;
-    for (int c = 0; c < L::kChunks && ok; ++c) {
-      ok = mbar_wait(&full[c], 0, abort_flag, status);
-      if (!ok) break;
-      tc_fence_after();
-      #pragma unroll
-      for (int kk = 0; kk < 4; ++kk) {
-        const uint64_t a = desc_kmajor(smem_u32(smem + c * L::kTile) + kk * 32);
-        const uint64_t b = desc_kmajor(smem_u32(smem + L::kBOff + c * L::kTile) + kk * 32);
-        mma_bf16_ss(tmem, a, b, id, (c > 0 || kk > 0) ? 1u : 0u);
+    if (*abort_flag) {
+      // let the loads in flight land before the shared memory is released
+      for (int c = (issued > L::kStages ? issued - L::kStages : 0); c < issued; ++c) {
+        const long long t0 = clock64();
+        while (!mbar_try_wait(&full[c % L::kStages], (c / L::kStages) & 1) && clock64() - t0 < kWaitBudgetCycles) {}
       }
+    }
+  } else if (threadIdx.x == 32) {
+    // ---- MMAs
+    constexpr uint32_t id = idesc_bf16(128, 128, false, false);
+    for (int c = 0; c < L::kChunks; ++c) {
+      const int s = c % L::kStages;
+      if (!mbar_wait(&full[s], (c / L::kStages) & 1, abort_flag, status)) break;
+      tc_fence_after();
+      const uint32_t base = smem_u32(smem + s * L::kStage);
+      #pragma unroll
+      for (int kk = 0; kk < 4; ++kk)
+        mma_bf16_ss(tmem, desc_kmajor(base + kk * 32), desc_kmajor(base + L::kTile + kk * 32), id,
+                    (c > 0 || kk > 0) ? 1u : 0u);
+      mma_commit(&empty[s]);
     }
     mma_commit(done);   // also when aborting: the MMAs already issued complete before the CTA exits
-    if (!ok) {
-      // let the loads in flight land before the shared memory is released
-      for (int c = 0; c < L::kChunks; ++c) {
-        const long long t0 = clock64();
-        while (!mbar_try_wait(&full[c], 0) && clock64() - t0 < kWaitBudgetCycles) {}
-      }
-    }
   }
   const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(done, 0, abort_flag, status)) && !*abort_flag;
   tc_fence_after();
-  const int m = m0 + threadIdx.x;          // my row = my TMEM lane
-  if (ok) {                                // warp-uniform: the TMEM loads are warp-collective
-    uint32_t* dst = keys + ((size_t)bh * nb + (m < nb ? m : 0)) * nbp + n0;
+  __syncthreads();                          // every role is past the ring before it is reused
+  if (ok) {                                 // warp-uniform: the TMEM loads are warp-collective
+    const int row0 = m0 + warp * 32;
     #pragma unroll 1
     for (int cc = 0; cc < 4; ++cc) {
       uint32_t v[32];
       tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + cc * 32, v);
       tmem_wait_ld();
-      if (m >= nb) continue;
       #pragma unroll
       for (int i = 0; i < 32; ++i) v[i] = n0 + cc * 32 + i < nb ? okey(__uint_as_float(v[i])) : 0u;
-      uint4* d4 = reinterpret_cast<uint4*>(dst + cc * 32);
+      uint8_t* buf = smem + (warp * 4 + cc) * L::kOutChunk;
       #pragma unroll
-      for (int i = 0; i < 8; ++i) d4[i] = make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+      for (int i = 0; i < 8; ++i)
+        *reinterpret_cast<uint4*>(buf + sw128_offset(lane, i)) = make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+      fence_proxy_async_smem();
+      __syncwarp();
+      // the keys moved as bf16 pairs: 32 keys = 64 elements; rows past nb are clipped
+      if (lane == 0 && row0 < nb) {
+        tma_store_3d(&tmKeys, buf, 2 * (n0 + cc * 32), row0, bh);
+        bulk_commit();
+      }
     }
+    if (lane == 0) bulk_wait_all();
   }
   tc_fence_before();
   __syncthreads();
@@ -458,6 +481,11 @@ cudaError_t launch_logits_d(const void* qsplit, const void* ksplit, uint32_t* ke
   const uint32_t box[3] = {64, 128, 1};
   if (!make_tile_map(&ma, qsplit, 3, dims, strides, box)) return cudaErrorInvalidValue;
   if (!make_tile_map(&mb, ksplit, 3, dims, strides, box)) return cudaErrorInvalidValue;
+  CUtensorMap mk;                                // keys [BH][nb][nbp] uint32, moved as bf16 pairs
+  const uint64_t kdims[3] = {(uint64_t)(2 * nbp), (uint64_t)nb, (uint64_t)BH};
+  const uint64_t kstrides[2] = {(uint64_t)nbp * 4, (uint64_t)nbp * 4 * nb};
+  const uint32_t kbox[3] = {64, 32, 1};
+  if (!make_tile_map(&mk, keys, 3, kdims, kstrides, kbox)) return cudaErrorInvalidValue;
   static unsigned long long attr_set = 0;        // one bit per device
   int dev = 0;
   cudaGetDevice(&dev);
@@ -467,7 +495,7 @@ cudaError_t launch_logits_d(const void* qsplit, const void* ksplit, uint32_t* ke
     if (dev < 64) attr_set |= 1ull << dev;
   }
   dim3 grid(nbp / 128, nbp / 128, BH);
-  logits_kernel<D><<<grid, 128, L::kBytes, st>>>(ma, mb, keys, nb, nbp, status);
+  logits_kernel<D><<<grid, 128, L::kBytes, st>>>(ma, mb, mk, nb, nbp, status);
   return cudaGetLastError();
 }
 
