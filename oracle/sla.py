@@ -26,6 +26,12 @@ Readings where the page is silent:
 4. Linear attention is normalised: O_l = phi(q) H / (phi(q) . Z) with
    H = sum phi(k)^T v, Z = sum phi(k) over the marginal keys; phi = elu + 1;
    a row with no marginal key gives O_l = 0.
+4b. The page also reports (the paragraph on the linear branch's activation
+   function) that a softmax feature map worked better than elu + 1 or ReLU,
+   without defining it.  The plainest reading, available here as
+   ``phi="softmax"``: each q and k row is mapped by a softmax over its d
+   channels, applied to Q and K separately; the rest of the branch is
+   unchanged.  (Not on the library's path yet: its feature map is elu + 1.)
 5. The projection is a right product O_l @ W_proj with W_proj [d, d], no bias.
 6. Pad tokens (past ``seg_len`` in a segment) are excluded from every sum; pad
    query rows give 0.  Pooled means use valid tokens only.
@@ -162,7 +168,17 @@ def phi_elu1(x: np.ndarray) -> np.ndarray:
     return np.where(x > 0, x + 1.0, np.exp(np.minimum(x, 0.0)))
 
 
-def key_block_states(k, v, valid, block: int = BLOCK):
+def phi_softmax(x: np.ndarray) -> np.ndarray:
+    """phi(x) = softmax of each row over its channels (reading 4b); shifted by the
+    row max before the exponential, which does not change the result."""
+    e = np.exp(x - x.max(axis=-1, keepdims=True))
+    return e / e.sum(axis=-1, keepdims=True)
+
+
+FEATURE_MAPS = {"elu1": phi_elu1, "softmax": phi_softmax}
+
+
+def key_block_states(k, v, valid, block: int = BLOCK, phi: str = "elu1"):
     """Per key block j: h_j = phi(K_j)^T V_j [d, dv] and z_j = sum_t phi(K_j,t) [d].
 
     The linear branch is evaluated "K^T V first, then Q" (SLA page sec. 3);
@@ -176,13 +192,13 @@ def key_block_states(k, v, valid, block: int = BLOCK):
     for j in range(nb):
         r = np.arange(j * block, (j + 1) * block)
         r = r[valid[r]]
-        fk = phi_elu1(k[r])
+        fk = FEATURE_MAPS[phi](k[r])
         h[j] = fk.T @ v[r]
         z[j] = fk.sum(axis=0)
     return h, z
 
 
-def linear_attention(q, k, v, valid, marginal, rows=None, block: int = BLOCK):
+def linear_attention(q, k, v, valid, marginal, rows=None, block: int = BLOCK, phi: str = "elu1"):
     """Linear attention of every query block over its marginal key blocks.
 
     ``marginal`` is a boolean [Nqb, Nkb] selector.  For query block i,
@@ -192,7 +208,7 @@ def linear_attention(q, k, v, valid, marginal, rows=None, block: int = BLOCK):
     """
     n, d = q.shape
     nb = n // block
-    h, z = key_block_states(k, v, valid, block)
+    h, z = key_block_states(k, v, valid, block, phi)
     sel = np.asarray(marginal, dtype=np.float64)
     out = np.zeros((n, v.shape[1]))
     rows = range(nb) if rows is None else rows
@@ -203,12 +219,12 @@ def linear_attention(q, k, v, valid, marginal, rows=None, block: int = BLOCK):
         Z = sel[i] @ z
         t = np.arange(i * block, (i + 1) * block)
         t = t[valid[t]]
-        fq = phi_elu1(q[t])
+        fq = FEATURE_MAPS[phi](q[t])
         out[t] = (fq @ H) / (fq @ Z)[:, None]
     return out
 
 
-def sla_head(q, k, v, w_proj, valid, crit_frac, negl_frac, rows=None, block: int = BLOCK):
+def sla_head(q, k, v, w_proj, valid, crit_frac, negl_frac, rows=None, block: int = BLOCK, phi: str = "elu1"):
     """The SLA forward of one head: O = O_s + O_l @ W_proj (SLA page sec. 3 and 5).
 
     Returns a dict with the pooled means, logits, P_c, the mask, the per-row
@@ -221,19 +237,19 @@ def sla_head(q, k, v, w_proj, valid, crit_frac, negl_frac, rows=None, block: int
     kc, kn = block_counts(kbar.shape[0], crit_frac, negl_frac)
     mask = classify(logits, kc, kn)
     o_s = block_sparse_attention(q, k, v, valid, lists_from_mask(mask, 1), rows, block)
-    o_l = linear_attention(q, k, v, valid, mask == 0, rows, block)
+    o_l = linear_attention(q, k, v, valid, mask == 0, rows, block, phi)
     o = o_s + o_l @ np.asarray(w_proj, dtype=np.float64)
     tau_c, tau_n = threshold_band(p, mask)
     return dict(qbar=qbar, kbar=kbar, logits=logits, p=p, mask=mask, kc=kc, kn=kn,
                 tau_c=tau_c, tau_n=tau_n, o_s=o_s, o_l=o_l, o=o)
 
 
-def sla(q, k, v, w_proj, n_seg, seg_len, seg_stride, crit_frac, negl_frac, rows=None):
+def sla(q, k, v, w_proj, n_seg, seg_len, seg_stride, crit_frac, negl_frac, rows=None, phi: str = "elu1"):
     """SLA over [B, H, N, d] fp64 arrays; returns a list (over b, h) of ``sla_head`` dicts."""
     valid = valid_tokens(n_seg, seg_len, seg_stride)
     res = []
     for b in range(q.shape[0]):
         for h in range(q.shape[1]):
             res.append(sla_head(q[b, h], k[b, h], v[b, h], w_proj, valid,
-                                crit_frac, negl_frac, rows))
+                                crit_frac, negl_frac, rows, phi=phi))
     return res

@@ -191,6 +191,38 @@ def test_all_marginal_equals_quadratic_linear_attention():
     np.testing.assert_allclose(out, ref, rtol=1e-12, atol=1e-13)
 
 
+def test_phi_softmax_is_a_row_distribution_and_shift_invariant():
+    rng = _rng(21)
+    x = rng.standard_normal((7, 16)) * 4
+    f = sla.phi_softmax(x)
+    assert (f > 0).all()
+    np.testing.assert_allclose(f.sum(axis=1), 1.0, rtol=0, atol=1e-15)
+    np.testing.assert_allclose(sla.phi_softmax(x + rng.standard_normal((7, 1)) * 30), f, rtol=1e-12, atol=0)
+    np.testing.assert_array_equal(sla.phi_softmax(np.full((2, 8), 3.25)), np.full((2, 8), 1 / 8))
+    # against the library routine
+    np.testing.assert_allclose(f, torch.softmax(torch.tensor(x), dim=-1).numpy(), rtol=1e-13, atol=0)
+
+
+def test_all_marginal_softmax_feature_map_equals_quadratic_form():
+    rng = _rng(22)
+    n, d = 192, 12
+    q, k, v = (rng.standard_normal((n, d)) for _ in range(3))
+    valid = sla.valid_tokens(1, 170, 192)
+    q[~valid] = k[~valid] = v[~valid] = 0
+    nb = n // 64
+    out = sla.linear_attention(q, k, v, valid, np.ones((nb, nb), bool), phi="softmax")
+    # quadratic form with the features from the library softmax: weights phi(q).phi(k)
+    # over valid keys, normalised per row
+    fq = torch.softmax(torch.tensor(q), dim=-1).numpy()
+    fk = torch.softmax(torch.tensor(k), dim=-1).numpy()
+    w = (fq @ fk.T) * valid[None, :]
+    ref = (w @ v) / w.sum(axis=1, keepdims=True)
+    ref[~valid] = 0
+    np.testing.assert_allclose(out, ref, rtol=1e-12, atol=1e-13)
+    # and the two feature maps give different outputs (the switch is live)
+    assert np.abs(out - sla.linear_attention(q, k, v, valid, np.ones((nb, nb), bool))).max() > 1e-3
+
+
 def test_linear_constant_values_reproduced():
     rng = _rng(10)
     n, d = 128, 6
