@@ -1,0 +1,73 @@
+"""Host-side pieces of bench.py: the DRAM-traffic record lookup, the clock-log
+parser and the algorithmic FLOP count (no GPU needed)."""
+import hashlib
+import json
+import os
+
+import bench
+import workloads
+
+
+def test_traffic_record_used_only_while_the_source_hash_matches(tmp_path, monkeypatch):
+    src = tmp_path / "k.cu"
+    src.write_text("kernel source\n")
+    (tmp_path / "profiles").mkdir()
+    rec = {"attention": {"source": "k.cu", "sha256": hashlib.sha256(src.read_bytes()).hexdigest(),
+                         "dram_bytes_per_launch": 123456}}
+    (tmp_path / "profiles" / "traffic.json").write_text(json.dumps(rec))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.measured_traffic("attention") == 123456
+    assert bench.measured_traffic("pool_means") is None
+    src.write_text("kernel source, changed\n")
+    assert bench.measured_traffic("attention") is None
+
+
+def test_traffic_record_missing_file(tmp_path, monkeypatch):
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.measured_traffic("attention") is None
+
+
+class _FakeProc:
+    def terminate(self):
+        pass
+
+    def wait(self, timeout=None):
+        return 0
+
+
+def test_clock_log_parsing(tmp_path):
+    path = tmp_path / "clocks.csv"
+    lines = [
+        "0, 1965, 1965, 700.1, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active",
+        "0, 1950, 1965, 990.0, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+        "0, 1900, 1965, 995.0, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+        "garbage line",
+    ]
+    s = bench.ClockSampler(0)
+    s.path = str(path)
+    s.f = open(path, "w")
+    s.f.write("\n".join(lines) + "\n")
+    s.proc = _FakeProc()
+    r = s.stop()
+    assert r == {"sm_mhz": 1950.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"], "samples": 3}
+
+
+def test_clock_sampler_without_nvidia_smi_reports_nothing():
+    s = bench.ClockSampler(0)
+    s.proc = None
+    assert s.stop() is None
+
+
+def test_critical_flops_of_the_32k_workload():
+    # 4 * 64 * 64 * d FLOP per critical (query block, key block) pair, 26 of 512 key
+    # blocks per row, 512 rows, 12 heads, d = 128: 0.335 TFLOP per call
+    w = workloads.WAN
+    crit, _ = bench.sla_flops(w, 26, 51)
+    assert crit == 4 * 64 * 64 * 128 * 512 * 26 * 12
+    assert abs(crit / 1e12 - 0.335) < 5e-4
+
+
+def test_config_names_the_workload():
+    c = bench.config_dict(workloads.WAN)
+    assert c["seq_len"] == 32768 and c["heads"] == 12 and c["head_dim"] == 128 and c["global_batch"] == 1
+    assert "32760 valid" in c["workload"] and "5% critical / 10% negligible" in c["workload"]
