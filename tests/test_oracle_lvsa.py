@@ -25,8 +25,10 @@ def _constants(golden_dir):
 def test_printed_constants(golden_dir):
     for kind, vals in _constants(golden_dir):
         if kind == "wan_budget":
-            frames, temporal_stride, budget = vals
+            frames, temporal_stride, budget, T, W = vals
             assert (frames - 1) // temporal_stride + 1 == budget
+            for s in range(4):
+                assert {len(A) for A in lvsa.attention_sets(T, budget, W, s)} == {budget}
         elif kind == "period":
             T, C, W, tper = vals
             assert lvsa.global_period(T, C, W) == tper

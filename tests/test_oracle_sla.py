@@ -345,3 +345,73 @@ def test_lse_matches_scipy_logsumexp():
         else:
             ref = logsumexp([q[t] @ k[u] / math.sqrt(d) for u in keys])
             assert abs(lse[t] - ref) < 1e-12
+
+
+# ---------------------------------------------------------------- compressed scores (P_c)
+
+def _pc_golden(golden_dir):
+    blocks = {"q": {}, "k": {}}
+    logits, pc, mask = {}, {}, {}
+    e = math.e
+    with open(os.path.join(golden_dir, "compressed_scores.txt")) as f:
+        for line in f:
+            if line.startswith("#") or not line.strip():
+                continue
+            kind, rest = line.split(None, 1)
+            if kind in ("q", "k"):
+                head, pads = rest.split("pad")
+                a, b = head.split("|")
+                blk, nvalid, *a_vals = a.split()
+                blocks[kind][int(blk)] = (int(nvalid), [float(x) for x in a_vals], [float(x) for x in b.split()],
+                                          [float(x) for x in pads.split()])
+            elif kind == "logit":
+                row, *vals = rest.split()
+                logits[int(row)] = [float(x) for x in vals]
+            elif kind == "pc":
+                row, *exprs = rest.split()
+                pc[int(row)] = [eval(x, {"__builtins__": {}}, {"e": e}) for x in exprs]
+            elif kind == "mask":
+                row, *vals = rest.split()
+                mask[int(row)] = [int(x) for x in vals]
+    return blocks, logits, pc, mask
+
+
+def _golden_tokens(spec):
+    nb = len(spec)
+    x = np.zeros((nb * 64, 4))
+    valid = np.zeros(nb * 64, bool)
+    for j, (nvalid, a, b, pad) in spec.items():
+        for t in range(64):
+            x[j * 64 + t] = (a if t % 2 == 0 else b) if t < nvalid else pad
+            valid[j * 64 + t] = t < nvalid
+    return x, valid
+
+
+def test_compressed_scores_hand_example(golden_dir):
+    """P_c = softmax(pool(Q) pool(K)^T / sqrt(d)) on the hand-worked 2 x 3 example: the
+    pooled means (pads excluded), the 1/sqrt(d) scale, the row softmax and the labels."""
+    blocks, logits, pc, mask = _pc_golden(golden_dir)
+    q, vq = _golden_tokens(blocks["q"])
+    k, vk = _golden_tokens(blocks["k"])
+    qbar, kbar = sla.pool_blocks(q, vq), sla.pool_blocks(k, vk)
+    np.testing.assert_array_equal(qbar, [[2, 0, 0, 0], [0, 2, 0, 0]])
+    np.testing.assert_array_equal(kbar, [[0, 0, 5, 5], [1, 1, 0, 0], [2, -2, 0, 0]])
+    lg = sla.block_logits(qbar, kbar)
+    np.testing.assert_array_equal(lg, [logits[0], logits[1]])
+    np.testing.assert_allclose(sla.compressed_scores(qbar, kbar), [pc[0], pc[1]], rtol=1e-14, atol=0)
+    np.testing.assert_array_equal(sla.classify(lg, 1, 1), [mask[0], mask[1]])
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_compressed_scores_match_torch_pool_and_softmax(d):
+    """Library routines: avg_pool1d over 64-token windows, then torch.softmax of the
+    pooled products scaled by 1/sqrt(d) (full blocks, no pads)."""
+    rng = _rng(20 + d)
+    q = _bf16ish(rng.standard_normal((640, d)))
+    k = _bf16ish(rng.standard_normal((640, d)) + 0.3 * rng.standard_normal(d))
+    valid = np.ones(640, bool)
+    qbar = torch.nn.functional.avg_pool1d(torch.tensor(q).T[None], 64, 64)[0].T
+    kbar = torch.nn.functional.avg_pool1d(torch.tensor(k).T[None], 64, 64)[0].T
+    ref = torch.softmax(qbar @ kbar.T / math.sqrt(d), dim=-1).numpy()
+    got = sla.compressed_scores(sla.pool_blocks(q, valid), sla.pool_blocks(k, valid))
+    np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-15)
