@@ -231,6 +231,16 @@ def _check_qkv(*ts):
             raise ValueError("q, k, v must be contiguous bf16 CUDA tensors [B, H, N_pad, d]")
 
 
+def slr_check_noalloc_status(device=None) -> int:
+    """Synchronise and return (and clear) the status word that
+    slr_block_sparse_attn_noalloc writes into its static scratch when it is given
+    no status tensor: slr_check_status(NULL, stream) in the C ABI."""
+    import torch
+    device = device or torch.device("cuda", torch.cuda.current_device())
+    with torch.cuda.device(device):
+        return lib().slr_check_status(None, ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream))
+
+
 def slr_check_status(ws=None, device=None) -> int:
     """Synchronise and return the device status word of the default workspace."""
     import torch
@@ -332,8 +342,10 @@ def slr_block_sparse_attn_noalloc(q, k, v, seq: SlrSeq, kv_idx=None, kv_cnt=None
                                   status=None):
     """slr_block_sparse_attn without a workspace (static device scratch); returns (o, lse).
 
-    ``status``: optional int32 CUDA tensor of one element that receives the device status.
-    Outputs are allocated here only when not given; the library call itself allocates nothing.
+    ``status``: optional int32 CUDA tensor of one element that receives the device status;
+    without it the status lands in the static scratch and slr_check_noalloc_status()
+    reads it.  Outputs are allocated here only when not given; the library call itself
+    allocates nothing.
     """
     import torch
     _check_qkv(q, k, v)

@@ -121,6 +121,10 @@ cudaError_t launch_reduce_states(const __nv_bfloat16* m01, int ld_m01, const __n
                                  __nv_bfloat16* Hs, int BH, int nb, int d, int* status, cudaStream_t st);
 
 // o_lin[bh][t] = phi(q_t) H_i' / (phi(q_t).Z_i) for every valid token t of block i (0 for pads).
+// ------------------------------------------------------------ no-workspace call (slr_noalloc.cu)
+// Reads and clears the status word of the static scratch on the current device.
+int noalloc_check_status(void* stream);   // an slr_status value
+
 cudaError_t launch_linear_apply(const void* q, const __nv_bfloat16* Hs, float* o_lin, int BH, int d, SeqShape s,
                                 int* status, cudaStream_t st);
 

@@ -390,7 +390,7 @@ size_t slr_workspace_bytes(int op, const slr_seq* seq, const void* params) {
     case SLR_OP_BLOCK_SPARSE: {
       c.take<int>(64);
       const int kv_max = params ? *static_cast<const int*>(params) : sh.nb;
-      const int cap = 2 * kv_max < sh.nb ? 2 * kv_max : sh.nb;
+      const int cap = (int)(2LL * kv_max < sh.nb ? 2LL * kv_max : sh.nb);
       c.take<uint32_t>((size_t)sh.BH * sh.npairs * (cap > 0 ? cap : 1));
       c.take<int32_t>((size_t)sh.BH * sh.npairs);
       return c.off;
@@ -425,7 +425,7 @@ size_t slr_workspace_bytes(int op, const slr_seq* seq, const void* params) {
 }
 
 slr_status slr_check_status(void* ws, void* stream) {
-  if (!ws) return SLR_ERR_ARG;
+  if (!ws) return noalloc_check_status(stream);
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return SLR_ERR_CUDA;
   int code = 0;
   if (cudaMemcpy(&code, ws, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return SLR_ERR_CUDA;
@@ -471,7 +471,7 @@ slr_status slr_block_sparse_attn(const void* q, const void* k, const void* v, co
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   Carve c(ws);
   int* status = c.take<int>(64);
-  const int cap = 2 * km < sh.nb ? 2 * km : sh.nb;
+  const int cap = (int)(2LL * km < sh.nb ? 2LL * km : sh.nb);
   uint32_t* list = c.take<uint32_t>((size_t)sh.BH * sh.npairs * cap);
   int32_t* list_cnt = c.take<int32_t>((size_t)sh.BH * sh.npairs);
   SLR_TRY(cudaMemsetAsync(status, 0, sizeof(int), s));

@@ -48,6 +48,24 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 }  // namespace
 
+namespace slr {
+
+// slr_check_status(NULL, stream): the status word the no-workspace call writes into
+// word 0 of the static scratch when its caller passes no status pointer.  Synchronises
+// the stream, reads the word on the current device and clears it.
+int noalloc_check_status(void* stream) {
+  void* base = nullptr;
+  slr_status st = scratch_address(&base);
+  if (st != SLR_OK) return st;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return SLR_ERR_CUDA;
+  int code = 0;
+  if (cudaMemcpy(&code, base, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return SLR_ERR_CUDA;
+  if (cudaMemset(base, 0, sizeof(int)) != cudaSuccess) return SLR_ERR_CUDA;
+  return code == 0 ? SLR_OK : -code;
+}
+
+}  // namespace slr
+
 extern "C" slr_status slr_block_sparse_attn_noalloc(const void* q, const void* k, const void* v,
                                                     const slr_seq* seq, const int32_t* kv_idx,
                                                     const int32_t* kv_cnt, int kv_max, void* o,
@@ -67,7 +85,7 @@ extern "C" slr_status slr_block_sparse_attn_noalloc(const void* q, const void* k
   if (kv_idx && (!kv_cnt || kv_max < 1)) return SLR_ERR_ARG;
 
   const int nb = (int)(n_pad / kBlock), npairs = (nb + 1) / 2;
-  const int cap = kv_idx ? (2 * kv_max < nb ? 2 * kv_max : nb) : 0;
+  const int cap = kv_idx ? (int)(2LL * kv_max < nb ? 2LL * kv_max : nb) : 0;
   const size_t list_bytes = kv_idx ? align256((size_t)bh * npairs * cap * sizeof(uint32_t)) : 0;
   const size_t cnt_bytes = kv_idx ? align256((size_t)bh * npairs * sizeof(int32_t)) : 0;
   if (kStatusBytes + list_bytes + cnt_bytes > kNoallocScratchBytes) return SLR_ERR_WORKSPACE;

@@ -99,7 +99,15 @@ typedef struct {
  * each key block of a row critical (1, the kc highest), negligible (-1, the kn
  * lowest) or marginal (0), ranking by score descending then index ascending.
  * kc = max(1, ceil(crit_frac*Nkb)), kn = floor(negl_frac*Nkb), kc+kn <= Nkb
- * (see slr_block_counts).  Pooling and scores are computed in fp64.
+ * (see slr_block_counts).
+ * Precision: each block sum is exact (fp64 over at most 64 bf16 values) and the
+ * mean is kept as a bf16 pair hi + lo (16 significant bits); the logits are
+ * formed on the tensor cores from those pairs (the products hi.hi, hi.lo and
+ * lo.hi in bf16 with fp32 accumulation; lo.lo, ~2^-16 relative, is dropped).
+ * P_c is then within ~1e-8 of its fp64 value (the tests bound it by 1e-6), so
+ * a label can differ from an exact-arithmetic ranking only for a pair whose
+ * P_c lies that close to its row's threshold; row counts are always exact and
+ * exact ties go to the lower key-block index.
  *
  *   q, k       bf16 [B][H][N_pad][d] device, read only
  *   mask       int8 [B][H][Nb][Nb] device, written
@@ -195,13 +203,16 @@ slr_status slr_frame_mask_attn(const void* q, const void* k, const void* v, cons
  * plug-in whose interface passes only input and output tensors.
  *
  * It computes exactly what slr_block_sparse_attn computes, with the same
- * arguments except `ws`/`ws_bytes`.  Its scratch (the per-pair key-block lists
- * and, when status_opt is NULL, the status word) lives in one static device
- * array of SLR_NOALLOC_SCRATCH_BYTES that every GPU which loads the library
- * holds until the process exits; the call allocates nothing.
+ * arguments except `ws`/`ws_bytes`.  Its scratch (the status word, the
+ * attention kernel's tile-queue counter and the per-pair key-block lists)
+ * lives in one static device array of SLR_NOALLOC_SCRATCH_BYTES that every GPU
+ * which loads the library holds until the process exits; the call allocates
+ * nothing.
  *   status_opt  int device pointer or NULL: zeroed by the call, then receives
  *               the device status (0, or 5 / 6 for a timeout / an out-of-range
- *               index: the negated SLR_ERR_TIMEOUT / SLR_ERR_INDEX).
+ *               index: the negated SLR_ERR_TIMEOUT / SLR_ERR_INDEX).  With NULL
+ *               the status goes to the static array's status word (zeroed by
+ *               the call as well), which slr_check_status(NULL, stream) reads.
  * Returns SLR_ERR_WORKSPACE when the lists of this shape need more than the
  * static scratch: 256 + B*H*ceil(Nb/2)*(min(Nb, 2*kv_max) + 1)*4 bytes (each
  * part rounded up to 256) must fit in SLR_NOALLOC_SCRATCH_BYTES; the dense mode
@@ -211,7 +222,9 @@ slr_status slr_frame_mask_attn(const void* q, const void* k, const void* v, cons
  * that first call before any stream capture.  All calls in the process share
  * the one array, which keeps the last call's lists: calls that can overlap on
  * the GPU (different streams, or different host threads on one device) race on
- * it and must be serialised by the caller.
+ * it -- on the lists, on the status word and, in every mode including the
+ * dense one, on the tile-queue counter, so that an overlapping call can skip or
+ * repeat tiles -- and must be serialised by the caller.
  */
 #define SLR_NOALLOC_SCRATCH_BYTES (4u << 20)
 slr_status slr_block_sparse_attn_noalloc(const void* q, const void* k, const void* v, const slr_seq* seq,
@@ -224,7 +237,10 @@ slr_status slr_block_sparse_attn_noalloc(const void* q, const void* k, const voi
 size_t slr_workspace_bytes(int op, const slr_seq* seq, const void* params);
 
 /* Synchronises `stream`, returns the status word that the device wrote into
- * `ws` since the last call started (SLR_OK if none), and clears it. */
+ * `ws` since the last call started (SLR_OK if none), and clears it.  ws == NULL
+ * reads (and clears) instead the status word of slr_block_sparse_attn_noalloc's
+ * static scratch on the current device, where that call reports when it is
+ * given no status pointer. */
 slr_status slr_check_status(void* ws, void* stream);
 
 /* Host-only: kc and kn for a row of n_kb key blocks (rule in slr_pool_classify). */

@@ -89,6 +89,15 @@ def test_workspace_bytes(lib):
     assert slr.slr_workspace_bytes(slr.SLR_OP_FRAME_MASK, slr.make_seq(1, 16, 128, 1, 32768, 32768), t3bad) == 0
 
 
+def test_block_sparse_list_cap_clamps_without_overflow(lib):
+    # the pair lists hold min(Nb, 2 kv_max) entries; 2 kv_max must not overflow int for huge kv_max
+    seq = slr.make_seq(1, 2, 64, 1, 64 * 40, 64 * 40)
+    full = slr.slr_workspace_bytes(slr.SLR_OP_BLOCK_SPARSE, seq, ctypes.c_int(40))
+    for km in (2 ** 30 + 1, 2 ** 31 - 1):
+        assert slr.slr_workspace_bytes(slr.SLR_OP_BLOCK_SPARSE, seq, ctypes.c_int(km)) == full
+    assert 0 < slr.slr_workspace_bytes(slr.SLR_OP_BLOCK_SPARSE, seq, ctypes.c_int(3)) < full
+
+
 def test_invalid_arguments_rejected_before_cuda(lib):
     seq = slr.make_seq(1, 1, 64, 1, 256, 256)
     vp = ctypes.c_void_p

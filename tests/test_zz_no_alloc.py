@@ -6,14 +6,18 @@ inputs and outputs).  Its scratch is a static device array inside libslr.
 Checked through the C ABI against the workspace entry point
 slr_block_sparse_attn on two calls in a row (different shapes, so stale lists
 left in the shared scratch by the first call would show in the second), plus
-the dense mode and the size limit.  Collected last so that a failure here
-cannot hide the other GPU tests."""
+the dense mode, the size limit, one direct comparison with the fp64 oracle and
+the status word read through slr_check_status(NULL) when no status tensor is
+passed.  Every call here runs after the previous one on one stream: calls that
+overlap on the GPU race on the shared array and are not exercised.  Collected
+last so that a failure here cannot hide the other GPU tests."""
 import numpy as np
 import pytest
 import torch
 
 import block_sparse_linear_02_b200 as slr
-from gpu_common import MAX_ABS, RMS_REL, assert_close, cuda, make_inputs, to64
+from gpu_common import MAX_ABS, RMS_REL, assert_close, cuda, make_inputs, to64, valid_np
+from oracle import sla as osla
 
 pytestmark = pytest.mark.gpu
 
@@ -61,3 +65,43 @@ def test_noalloc_rejects_shapes_beyond_the_static_scratch():
     with pytest.raises(slr.SlrError) as e:
         slr.slr_block_sparse_attn_noalloc(q, q, q, seq, idx, cnt)
     assert e.value.code == slr.SLR_ERR_WORKSPACE
+
+
+def test_noalloc_matches_oracle_directly():
+    """The no-workspace call against the fp64 oracle itself (ragged segments, duplicates in a set)."""
+    H, d, n_seg, seg_len, stride = 2, 128, 2, 500, 512
+    q, k, v = make_inputs(1, H, d, n_seg, seg_len, stride, seed=74)
+    seq = slr.make_seq(1, H, d, n_seg, seg_len, stride)
+    nb = n_seg * stride // 64
+    idx_np = np.random.default_rng(74).integers(0, nb, (1, H, nb, 6)).astype(np.int32)
+    cnt_np = np.random.default_rng(75).integers(0, 7, (1, H, nb)).astype(np.int32)
+    idx_np[0, 0, 3, :3] = 5                      # a duplicated entry counts once
+    cnt_np[0, 0, 3] = 3
+    o, _ = slr.slr_block_sparse_attn_noalloc(cuda(q), cuda(k), cuda(v), seq, cuda(torch.from_numpy(idx_np)),
+                                             cuda(torch.from_numpy(cnt_np)))
+    assert slr.slr_check_noalloc_status() == slr.SLR_OK
+    valid = valid_np(n_seg, seg_len, stride)
+    for h in range(H):
+        sets = [idx_np[0, h, i, :cnt_np[0, h, i]].tolist() for i in range(nb)]
+        ref = osla.block_sparse_attention(to64(q[0, h]), to64(k[0, h]), to64(v[0, h]), valid, sets)
+        assert_close(to64(o[0, h]), ref, f"noalloc vs oracle head {h}")
+
+
+def test_noalloc_status_without_status_tensor():
+    """An out-of-range entry, with no status tensor passed: the error lands in the static
+    scratch's status word and slr_check_status(NULL) (slr_check_noalloc_status) reports it."""
+    H, d, n = 1, 64, 256
+    q, k, v = (cuda(x) for x in make_inputs(1, H, d, 1, n, n, seed=76))
+    seq = slr.make_seq(1, H, d, 1, n, n)
+    idx = cuda(torch.tensor([[[[0, 4], [1, 2], [3, -1], [2, 2]]]], dtype=torch.int32))
+    cnt = cuda(torch.full((1, H, 4), 2, dtype=torch.int32))
+    o, _ = slr.slr_block_sparse_attn_noalloc(q, k, v, seq, idx, cnt)
+    assert slr.slr_check_noalloc_status() == slr.SLR_ERR_INDEX
+    assert slr.slr_check_noalloc_status() == slr.SLR_OK            # read and cleared
+    ref = osla.block_sparse_attention(to64(q[0, 0]), to64(k[0, 0]), to64(v[0, 0]), np.ones(n, bool),
+                                      [[0], [1, 2], [3], [2]])
+    assert_close(to64(o[0, 0]), ref, "valid entries still attended")
+    # the next call starts from a cleared word
+    good = cuda(torch.tensor([[[[0, 1], [1, 2], [3, 0], [2, 2]]]], dtype=torch.int32))
+    slr.slr_block_sparse_attn_noalloc(q, k, v, seq, good, cnt)
+    assert slr.slr_check_noalloc_status() == slr.SLR_OK
