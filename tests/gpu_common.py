@@ -14,6 +14,10 @@ MAX_ABS = 2e-2
 RMS_REL = 5e-3
 BAND = 1e-5
 
+# (test id, what, max-abs, rms-rel) of every output comparison, printed at the end of
+# the session (tests/conftest.py) so that the margin to the tolerances is visible.
+ERRORS: list = []
+
 
 def to64(t: torch.Tensor) -> np.ndarray:
     return t.detach().to("cpu", torch.float32).double().numpy()
@@ -32,6 +36,8 @@ def assert_close(out: np.ndarray, ref: np.ndarray, what: str = "", max_abs: floa
     ma = float(np.abs(err).max()) if err.size else 0.0
     denom = float(np.sqrt(np.mean(ref * ref))) if ref.size else 1.0
     rr = float(np.sqrt(np.mean(err * err)) / max(denom, 1e-30)) if err.size else 0.0
+    import os
+    ERRORS.append((os.environ.get("PYTEST_CURRENT_TEST", "?").split(" ")[0], what, ma, rr))
     assert ma <= max_abs, f"{what}: max-abs {ma:.3e} > {max_abs}"
     assert rr <= rms_rel, f"{what}: rms-rel {rr:.3e} > {rms_rel}"
     return ma, rr

@@ -71,3 +71,20 @@ def test_config_names_the_workload():
     c = bench.config_dict(workloads.WAN)
     assert c["seq_len"] == 32768 and c["heads"] == 12 and c["head_dim"] == 128 and c["global_batch"] == 1
     assert "32760 valid" in c["workload"] and "5% critical / 10% negligible" in c["workload"]
+
+
+def test_tile3d_pair_count_of_the_rope_workload():
+    # 2 x 16 x 16 tiles; clipped 3-neighbourhoods: 2*2 along frames, 2*2 + 14*3 = 46 along each
+    # spatial axis -> 4 * 46 * 46 = 8464 local pairs per head, plus one far block per tile
+    f, pairs = bench.tile3d_flops(workloads.ROPESLR)
+    assert pairs == 8464
+    assert f == 4 * 64 * 64 * 128 * (8464 + 512) * 16
+
+
+def test_lvsa_flops_counts_attended_frame_blocks():
+    from oracle import lvsa as olvsa
+    w = workloads.LVSA
+    sets = olvsa.attention_sets(w.frames, w.lvsa_C, w.lvsa_W, 0)
+    # every frame attends C = 21 frames of 25 blocks: 121 * 25 * 21 * 25 block pairs
+    assert bench.lvsa_flops(w, sets) == 4 * 64 * 64 * 128 * 121 * 25 * 21 * 25 * 12
+    assert abs(bench.lvsa_flops(w, sets) / 1e12 - 39.97) < 0.01

@@ -50,6 +50,27 @@ def test_explicit_lists_ragged(d):
         assert np.abs(got[fin] - ref_lse[fin]).max() < 1e-3
 
 
+def test_explicit_lists_two_batch_entries():
+    # B = 2: lists, valid-key counts and TMA coordinates are indexed by b * H + h
+    B, H, d, n_seg, seg_len, stride, kv_max = 2, 3, 128, 2, 450, 512, 9
+    q, k, v = make_inputs(B, H, d, n_seg, seg_len, stride, seed=11)
+    nb = n_seg * stride // 64
+    idx, cnt = _random_lists(B * H, nb, kv_max, seed=12)
+    seq = slr.make_seq(B, H, d, n_seg, seg_len, stride)
+    o, _ = slr.slr_block_sparse_attn(cuda(q), cuda(k), cuda(v), seq,
+                                     cuda(torch.from_numpy(idx).reshape(B, H, nb, kv_max)),
+                                     cuda(torch.from_numpy(cnt).reshape(B, H, nb)))
+    status_ok()
+    valid = valid_np(n_seg, seg_len, stride)
+    outs, refs = [], []
+    for b in range(B):
+        for h in range(H):
+            lists = [list(idx[b * H + h, i, :cnt[b * H + h, i]]) for i in range(nb)]
+            refs.append(osla.block_sparse_attention(to64(q[b, h]), to64(k[b, h]), to64(v[b, h]), valid, lists))
+            outs.append(to64(o[b, h]))
+    assert_close(np.concatenate(outs), np.concatenate(refs), "explicit lists B=2")
+
+
 @pytest.mark.parametrize("d", [64, 128])
 def test_dense_odd_block_count(d):
     H, seg_len, stride = 2, 300, 320           # 5 blocks -> the last pair has one block

@@ -1,7 +1,9 @@
 """GPU parity of slr_frame_mask_attn against the fp64 oracle: LVSA frame masks
-(small case in full for four denoising steps, the 121-frame workload on sampled
-query blocks) and the gated tile neighbourhood + far field (small grids in
-full, including an odd tile count, and the 8x64x64 workload on sampled tiles)."""
+(small case in full for four denoising steps and with two batch entries, the
+121-frame workload on 64 sampled query blocks of every head, including the
+first and last blocks and frame tails) and the gated tile neighbourhood + far
+field (small grids in full, including an odd tile count and two batch entries,
+and the 8x64x64 workload on sampled tokens)."""
 import numpy as np
 import pytest
 import torch
@@ -28,6 +30,22 @@ def test_lvsa_small_full(step):
         assert_close(to64(out[0, h]), ref, f"step {step} head {h}")
 
 
+def test_lvsa_two_batch_entries():
+    B, T, C, W, seg_len, stride, H, d = 2, 9, 6, 1, 150, 192, 2, 128
+    q, k, v = make_inputs(B, H, d, T, seg_len, stride, seed=43)
+    seq = slr.make_seq(B, H, d, T, seg_len, stride)
+    out = slr.slr_frame_mask_attn(cuda(q), cuda(k), cuda(v), seq, slr.lvsa_mask(T, C, W, 2))
+    status_ok()
+    sets = olvsa.attention_sets(T, C, W, 2)
+    outs, refs = [], []
+    for b in range(B):
+        for h in range(H):
+            outs.append(to64(out[b, h]))
+            refs.append(olvsa.frame_mask_attention(to64(q[b, h]), to64(k[b, h]), to64(v[b, h]), T, seg_len, stride,
+                                                   sets))
+    assert_close(np.concatenate(outs), np.concatenate(refs), "lvsa B=2")
+
+
 @pytest.mark.parametrize("step", [0, 3])
 def test_lvsa_workload_sampled(step):
     w = workloads.LVSA
@@ -37,10 +55,12 @@ def test_lvsa_workload_sampled(step):
     status_ok()
     sets = olvsa.attention_sets(w.frames, w.lvsa_C, w.lvsa_W, step)
     bpf = w.seg_stride // 64
-    rows = [0, 24, 25, 60 * bpf + 7, 120 * bpf + 24, w.n_blocks - 1]
-    sel = rows_of_blocks(rows)
     outs, refs = [], []
     for h in range(w.heads):
+        rng = np.random.default_rng(100 * step + h)
+        rows = sorted(set([0, 24, 25, 60 * bpf + 7, 120 * bpf + 24, w.n_blocks - 1] +
+                          rng.choice(w.n_blocks, 58, replace=False).tolist()))
+        sel = rows_of_blocks(rows)
         ref = olvsa.frame_mask_attention(to64(q[0, h]), to64(k[0, h]), to64(v[0, h]), w.n_seg, w.seg_len,
                                          w.seg_stride, sets, rows=rows)
         outs.append(to64(out[0, h])[sel])
@@ -62,6 +82,22 @@ def test_tile3d_small_full(F, Hh, Ww, cell, gate):
     for h in range(H):
         r = otile.gated_head(to64(q[0, h]), to64(k[0, h]), to64(v[0, h]), F, Hh, Ww, cell=cell, gate=gate)
         assert_close(to64(out[0, h]), r["o"], f"tile3d head {h}")
+
+
+def test_tile3d_two_batch_entries():
+    B, H, d, F, Hh, Ww, cell = 2, 2, 128, 8, 8, 16, (2, 2, 4)
+    n = F * Hh * Ww
+    q, k, v = make_inputs(B, H, d, 1, n, n, seed=53)
+    seq = slr.make_seq(B, H, d, 1, n, n)
+    out = slr.slr_frame_mask_attn(cuda(q), cuda(k), cuda(v), seq, slr.tile3d_mask(F, Hh, Ww, 1, cell, 0.55))
+    status_ok()
+    outs, refs = [], []
+    for b in range(B):
+        for h in range(H):
+            r = otile.gated_head(to64(q[b, h]), to64(k[b, h]), to64(v[b, h]), F, Hh, Ww, cell=cell, gate=0.55)
+            outs.append(to64(out[b, h]))
+            refs.append(r["o"])
+    assert_close(np.concatenate(outs), np.concatenate(refs), "tile3d B=2")
 
 
 def test_tile3d_workload_sampled():
