@@ -69,7 +69,7 @@ struct AttnLayout {
   // output staging (non-tile layouts): per softmax warp one 32-row x 32-column bf16
   // chunk (64-byte rows, 64-byte swizzle), written to HBM by TMA tensor stores
   static constexpr int kOutChunk = 32 * 64;
-  static constexpr int kOutOff = (kBarOff + 256 + 1023) / 1024 * 1024;
+  static constexpr int kOutOff = (kBarOff + 512 + 1023) / 1024 * 1024;
   static constexpr int kBytes = kOutOff + 8 * kOutChunk + 1024;   // + alignment slack
   static_assert(kHsTile <= kKV, "a linear state tile must fit in one ring slot");
   static_assert(kBytes <= 227 * 1024, "shared memory budget");
@@ -209,12 +209,13 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
   uint64_t* q_full = bars + 0;                   // Q (and Z) of the current tile landed
   uint64_t* q_free = q_full + 1;                 // every MMA reading Q / Z of a tile has completed
   uint64_t* slot_full = q_free + 1;              // [kSlots] ring slot filled (TMA, or freed for phi(Q))
-  uint64_t* s_full = slot_full + kSlots;         // [2] per S buffer
-  uint64_t* p_full = s_full + 2;                 // [2] per S buffer, 256 arrivals
+  uint64_t* s_full = slot_full + kSlots;         // [4] per step mod 4: S_j written (the step's K item is free)
+  uint64_t* p_full = s_full + 4;                 // [2] per S buffer, 256 arrivals
   uint64_t* pv_done = p_full + 2;                // [4] per step mod 4 (phases cannot alias)
   uint64_t* den_done = pv_done + 4;              // the tile's phi(Q) slot has been read (256 arrivals per tile)
   uint64_t* lin_done = den_done + 1;
-  uint64_t* o_free = lin_done + 1;               // the epilogue has read O_0/O_1 (256 arrivals per tile)
+  uint64_t* lin_read = lin_done + 1;             // the tile's linear result has been read (256 arrivals per tile)
+  uint64_t* o_free = lin_read + 1;               // the epilogue has read O_0/O_1 (256 arrivals per tile)
   uint64_t* xch_bar = o_free + 1;                // both shares of every row published (256 arrivals per tile)
   uint64_t* tq_full = xch_bar + 1;               // [kTq] tile slot written
   uint64_t* tq_empty = tq_full + kTq;            // [kTq] tile slot read (MMA thread + one lane per softmax warp)
@@ -229,19 +230,19 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
   // LINEAR: a tile's first three ring positions hold the H'^T rows of its two query
   // blocks and phi(Q); its K/V items follow
   constexpr int kPre = LINEAR ? 3 : 0;
-  constexpr uint32_t kColLinOut = kColO0;   // lin (+ denominator at column D) before O_0/O_1 are first written
+  // LINEAR: the tile's lin = phi(Q) H'_b (D columns) is written into the S buffer that step 1
+  // of the tile will use, so it waits neither for the previous tile's epilogue nor for O
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
     mbar_init(q_free, 1);
     for (int s = 0; s < kSlots; ++s) mbar_init(&slot_full[s], 1);
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&s_full[b], 1);
-      mbar_init(&p_full[b], 256);
-    }
+    for (int b = 0; b < 4; ++b) mbar_init(&s_full[b], 1);
+    for (int b = 0; b < 2; ++b) mbar_init(&p_full[b], 256);
     for (int b = 0; b < 4; ++b) mbar_init(&pv_done[b], 1);
     mbar_init(den_done, 256);
     mbar_init(lin_done, 1);
+    mbar_init(lin_read, 256);
     mbar_init(o_free, 256);
     mbar_init(xch_bar, 256);
     for (int e = 0; e < kTq; ++e) { mbar_init(&tq_full[e], 1); mbar_init(&tq_empty[e], 9); }
@@ -260,8 +261,11 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
     if (lane == 0) {
       tma_prefetch_desc(&tmQ); tma_prefetch_desc(&tmK); tma_prefetch_desc(&tmV);
       // how the current occupant of each ring slot is released: kind 0 = the P.V of
-      // global step idx, kind 1 = the linear-branch MMAs of local tile idx, kind 2 = those
-      // MMAs and the softmax warps' denominator reads of local tile idx, -1 = free
+      // global step idx (a V item), kind 3 = the QK of global step idx (a K item: only QK
+      // reads it, so its slot turns over a step earlier, which lets the next tile's first
+      // K load while the current tile still runs), kind 1 = the linear-branch MMAs of
+      // local tile idx, kind 2 = those MMAs and the softmax warps' denominator reads of
+      // local tile idx, -1 = free
       int rel_kind[kSlots], rel_idx[kSlots];
       #pragma unroll
       for (int s = 0; s < kSlots; ++s) { rel_kind[s] = -1; rel_idx[s] = 0; }
@@ -269,6 +273,10 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
         if (rel_kind[slot] == 0) {
           const int q = rel_idx[slot];
           return mbar_wait(&pv_done[q & 3], (q >> 2) & 1, abort_flag, p.status);
+        }
+        if (rel_kind[slot] == 3) {
+          const int q = rel_idx[slot];
+          return mbar_wait(&s_full[q & 3], (q >> 2) & 1, abort_flag, p.status);
         }
         if (rel_kind[slot] >= 1) {
           if (!mbar_wait(lin_done, rel_idx[slot] & 1, abort_flag, p.status)) return false;
@@ -360,7 +368,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
               }
             }
           }
-          rel_kind[slot] = 0;
+          rel_kind[slot] = is_v ? 0 : 3;
           rel_idx[slot] = J + j;
         }
         J += ti.n_steps;
@@ -405,9 +413,9 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
           mma_bf16_ts(tmem + col, a + kk * 8, db + (uint32_t)(kk * 2048 >> 4), idO, (acc || kk > 0) ? 1u : 0u);
       };
       // lin = phi(Q) H'_b per query block b (lanes of the other block masked off) into the
-      // O columns, before any P.V; the denominators phi(q) . Z_b are dot products the
-      // softmax warps form while they compute phi(Q)
-      auto issue_lin = [&](int g0, int n_lin) {
+      // TMEM columns col (the S buffer of the tile's step 1); the denominators phi(q) . Z_b
+      // are dot products the softmax warps form from phi(Q) in shared memory
+      auto issue_lin = [&](int g0, int n_lin, uint32_t col) {
         constexpr uint32_t idH = idesc_bf16(128, D, false, false);
         const uint32_t phq_addr = ring_addr + ((g0 + 2) % kSlots) * L::kKV;
         const uint32_t lo_only[4] = {0u, 0u, 0xFFFFFFFFu, 0xFFFFFFFFu};   // write lanes 0-63
@@ -419,10 +427,19 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
             const int c = kk >> 2, sub = kk & 3;
             const uint64_t a = desc_kmajor(phq_addr + c * L::kTile + sub * 32);
             const uint64_t bh_ = desc_kmajor(hs_addr + c * L::kHsChunk + sub * 32);
-            mma_bf16_ss_masked(tmem + kColLinOut, a, bh_, idH, kk > 0 ? 1u : 0u, b ? hi_only : lo_only);
+            mma_bf16_ss_masked(tmem + col, a, bh_, idH, kk > 0 ? 1u : 0u, b ? hi_only : lo_only);
           }
         }
         mma_commit(lin_done);
+      };
+      // LINEAR: the local tile whose linear result the softmax warps may still be reading
+      // from an S buffer; any MMA that writes an S buffer first waits for that read
+      int lin_tile = -1;
+      auto settle_lin = [&]() -> bool {
+        if (!LINEAR || lin_tile < 0) return true;
+        const int tl = lin_tile;
+        lin_tile = -1;
+        return mbar_wait(lin_read, tl & 1, abort_flag, p.status);
       };
       int i = 0, J = 0, g = 0;
       bool ok = true;
@@ -438,6 +455,19 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
           return (2 * j + 1 < ti.n_local) ? 2 : 1;
         };
         const int gkv = g + kPre;                  // ring position of this tile's K_0
+        if (LINEAR) {
+          // lin first: it needs only the pre-slots (loaded ahead of K_0), and the softmax
+          // warps read it while QK_0 runs.  Its S buffer was last read by the P.V of the
+          // previous tile's last step, issued earlier from this thread (MMAs run in order).
+          ok = mbar_wait(&slot_full[(g + 2) % kSlots], ((g + 2) / kSlots) & 1, abort_flag, p.status) &&
+               mbar_wait(&slot_full[g % kSlots], (g / kSlots) & 1, abort_flag, p.status) &&
+               mbar_wait(&slot_full[(g + 1) % kSlots], ((g + 1) / kSlots) & 1, abort_flag, p.status) &&
+               settle_lin();
+          if (!ok) break;
+          tc_fence_after();
+          issue_lin(g, ti.n_lin, kColS + ((J + 1) & 1) * 128);
+          lin_tile = i;
+        }
         if (!(ok = mbar_wait(q_full, i & 1, abort_flag, p.status))) break;
         // GATED: the previous tile's far-field output sits in the S buffer this tile's
         // first QK writes, so wait until its epilogue has read it
@@ -445,17 +475,8 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
         if (ti.n_steps > 0) {
           if (!(ok = mbar_wait(&slot_full[gkv % kSlots], (gkv / kSlots) & 1, abort_flag, p.status))) break;
           tc_fence_after();
-          issue_qk(gkv % kSlots, J & 1);
-          mma_commit(&s_full[J & 1]);
-        }
-        if (LINEAR) {
-          ok = mbar_wait(&slot_full[(g + 2) % kSlots], ((g + 2) / kSlots) & 1, abort_flag, p.status) &&
-               mbar_wait(&slot_full[g % kSlots], (g / kSlots) & 1, abort_flag, p.status) &&
-               mbar_wait(&slot_full[(g + 1) % kSlots], ((g + 1) / kSlots) & 1, abort_flag, p.status) &&
-               (i == 0 || mbar_wait(o_free, (i - 1) & 1, abort_flag, p.status));
-          if (!ok) break;
-          tc_fence_after();
-          issue_lin(g, ti.n_lin);
+          issue_qk(gkv % kSlots, J & 1);           // S buffer J & 1: never the tile's lin buffer
+          mma_commit(&s_full[J & 3]);
         }
         if (ti.n_steps <= 1) mma_commit(q_free);   // the last MMA reading Q (and Z) has been issued
         bool o1_started = false;
@@ -463,10 +484,11 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
           const int Jj = J + j, b = Jj & 1;
           if (j + 1 < ti.n_steps) {
             const int gk = gkv + 2 * (j + 1);
-            if (!(ok = mbar_wait(&slot_full[gk % kSlots], (gk / kSlots) & 1, abort_flag, p.status))) break;
+            if (!(ok = mbar_wait(&slot_full[gk % kSlots], (gk / kSlots) & 1, abort_flag, p.status) &&
+                       settle_lin())) break;
             tc_fence_after();
             issue_qk(gk % kSlots, (Jj + 1) & 1);
-            mma_commit(&s_full[(Jj + 1) & 1]);
+            mma_commit(&s_full[(Jj + 1) & 3]);
             if (j + 2 == ti.n_steps) mma_commit(q_free);
           }
           const int gv = gkv + 2 * j + 1;
@@ -540,12 +562,11 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
       const bool valid = row_exists && (TILE || token_valid(seq, tok));
 
       // ---- linear branch (LINEAR): phi(Q) arrives by TMA in the tile's third pre-slot, and
-      // the MMA warp's lin = phi(Q) H'_b lands in the O columns; my half of the row is read
-      // during the first step (before its P is handed over, since the first P.V overwrites
-      // those columns) and kept in registers as bf16 pairs (the output is rounded to bf16
-      // in the end as well).  The denominator phi(q) . Z_b is a dot product over the same
-      // bf16 phi values, my half of the channels here, summed with the other half in the
-      // epilogue.
+      // the MMA warp's lin = phi(Q) H'_b lands in the S buffer of the tile's step 1; my half
+      // of the row is read before the first step (the QK of step 1 waits for that read) and
+      // kept in registers as bf16 pairs (the output is rounded to bf16 in the end as well).
+      // The denominator phi(q) . Z_b is a dot product over the same bf16 phi values, my half
+      // of the channels here, summed with the other half in the epilogue.
       uint32_t lin[D / 4];
       #pragma unroll
       for (int k = 0; k < D / 4; ++k) lin[k] = 0u;
@@ -573,22 +594,22 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
           }
         }
         mbar_arrive(den_done);
-      }
-      bool lin_pending = LINEAR;
-      auto read_lin = [&]() {
-        lin_pending = false;
         if (ok) ok = __all_sync(0xFFFFFFFFu, mbar_wait(lin_done, i & 1, abort_flag, p.status));
         tc_fence_after();
-        if (!ok) return;
-        #pragma unroll
-        for (int k = 0; k < D / 64; ++k) {
-          uint32_t tv[32];
-          tmem_ld32(lane_addr + kColLinOut + wg * (D / 2) + k * 32, tv);
-          tmem_wait_ld();
+        if (ok) {
+          const uint32_t lin_addr = lane_addr + kColS + ((J + 1) & 1) * 128 + wg * (D / 2);
           #pragma unroll
-          for (int m = 0; m < 16; ++m) lin[k * 16 + m] = pack_bf16(__uint_as_float(tv[2 * m]), __uint_as_float(tv[2 * m + 1]));
+          for (int k = 0; k < D / 64; ++k) {
+            uint32_t tv[32];
+            tmem_ld32(lin_addr + k * 32, tv);
+            tmem_wait_ld();
+            #pragma unroll
+            for (int m = 0; m < 16; ++m) lin[k * 16 + m] = pack_bf16(__uint_as_float(tv[2 * m]), __uint_as_float(tv[2 * m + 1]));
+          }
+          tc_fence_before();
+          mbar_arrive(lin_read);
         }
-      };
+      }
 
       // my list word of step j, loaded one step ahead and decoded only where it is used, so
       // that the load's latency is not waited for at the top of the step
@@ -604,13 +625,9 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
         const bool mine = wg == 0 || (!far && step_blocks(j) == 2);   // does this warpgroup own a block here
         const uint32_t w_cur = w_next;
         w_next = word_of(j + 1);
-        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&s_full[b], (Jj >> 1) & 1, abort_flag, p.status))) { ok = false; break; }
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&s_full[Jj & 3], (Jj >> 2) & 1, abort_flag, p.status))) { ok = false; break; }
         tc_fence_after();
         if (!mine) {
-          if (LINEAR && j == 0) {
-            read_lin();
-            if (!ok) break;
-          }
           tc_fence_before();
           mbar_arrive(&p_full[b]);
           continue;
@@ -726,17 +743,12 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
             tmem_st32(lane_addr + my_o + cc * 32, o);
           }
         }
-        if (LINEAR && j == 0) {
-          read_lin();
-          if (!ok) break;
-        }
         tmem_st32(s_addr, packed);          // P (bf16 pairs) over the first 32 columns of my S block
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&p_full[b]);
         if (!far) started = true;
       }
-      if (LINEAR && lin_pending) read_lin();         // no step read it
       if (ok && n_steps > 0) {
         const int Jl = J + n_steps - 1;
         ok = __all_sync(0xFFFFFFFFu, mbar_wait(&pv_done[Jl & 3], (Jl >> 2) & 1, abort_flag, p.status));
