@@ -85,11 +85,12 @@ def measured_traffic(kernel: str, workload: str = "wan"):
     return rec["dram_bytes_per_launch"]
 
 
-def config_dict(w):
+def config_dict(w, phi="elu1"):
     if w.mode == "sla":
         desc = (f"{w.name}: SLA layer B={w.batch} H={w.heads} d={w.d} N={w.n_pad} "
                 f"({w.n_valid} valid, {w.frames} frames of {w.fh}x{w.fw}), block 64, "
-                f"{int(w.crit_frac * 100)}% critical / {int(w.negl_frac * 100)}% negligible, phi=elu+1")
+                f"{int(w.crit_frac * 100)}% critical / {int(w.negl_frac * 100)}% negligible, "
+                + ("phi=elu+1" if phi == "elu1" else "phi=softmax over the channels"))
     elif w.mode == "lvsa":
         desc = (f"{w.name}: LVSA frame mask B={w.batch} H={w.heads} d={w.d} T={w.frames} frames of "
                 f"{w.fh}x{w.fw}={w.seg_len} tokens padded to {w.seg_stride} (N={w.n_pad}), C={w.lvsa_C}, "
@@ -217,7 +218,7 @@ def _blas_threads():
         return 1
 
 
-def cpu_oracle_sample(w, q, k, v, wp, rows_per_head=256, heads=12):
+def cpu_oracle_sample(w, q, k, v, wp, rows_per_head=256, heads=12, phi="elu1"):
     """Time the fp64 oracle on a bounded sample of workload `w` and extrapolate to a
     full call.  Only oracle functions run inside the timed spans.
 
@@ -250,7 +251,7 @@ def cpu_oracle_sample(w, q, k, v, wp, rows_per_head=256, heads=12):
             mask = osla.classify(lg, kc, kn)
             t1 = time.perf_counter()
             o_s = osla.block_sparse_attention(qh, kh, vh, valid, osla.lists_from_mask(mask, 1), rows=rows)
-            o_l = osla.linear_attention(qh, kh, vh, valid, mask == 0, rows=rows)
+            o_l = osla.linear_attention(qh, kh, vh, valid, mask == 0, rows=rows, phi=phi)
             o_s + o_l @ wp64
             t2 = time.perf_counter()
             fixed += t1 - t0
@@ -290,8 +291,9 @@ def cpu_oracle_sample(w, q, k, v, wp, rows_per_head=256, heads=12):
 class Runner:
     """Inputs, calls and timing of one workload on this rank's GPU."""
 
-    def __init__(self, w, slr, dev, dist, sdist, world):
+    def __init__(self, w, slr, dev, dist, sdist, world, phi="elu1"):
         self.w, self.slr, self.dev, self.dist, self.sdist, self.world = w, slr, dev, dist, sdist, world
+        self.phi = slr.SLR_PHI_SOFTMAX if phi == "softmax" else slr.SLR_PHI_ELU1
         self.q_h, self.k_h, self.v_h = workloads.make_qkv(w)
         self.wp_h = workloads.make_w_proj(w)
         self.q, self.k, self.v, self.wp = (x.to(dev) for x in (self.q_h, self.k_h, self.v_h, self.wp_h))
@@ -314,7 +316,7 @@ class Runner:
         ws = self.ws if ws is None else ws
         if w.mode == "sla":
             slr.slr_sparse_linear_attn(q, k, v, self.wp if wp is None else wp, self.seq, w.crit_frac, w.negl_frac,
-                                       out=o, ws=ws)
+                                       out=o, ws=ws, phi=self.phi)
         else:
             slr.slr_frame_mask_attn(q, k, v, self.seq, self.masks[i % len(self.masks)], out=o, ws=ws)
 
@@ -466,6 +468,8 @@ def main():
     ap.add_argument("--workload", default=WORKLOAD.name, choices=sorted(workloads.BY_NAME))
     ap.add_argument("--others", default="auto", choices=["auto", "none"],
                     help="auto: at one GPU also measure the other workloads under other_configs")
+    ap.add_argument("--phi", default="elu1", choices=["elu1", "softmax"],
+                    help="feature map of the linear branch of the SLA workloads")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--oracle-rows", type=int, default=256, help="query blocks per head in the CPU oracle sample")
@@ -494,7 +498,7 @@ def main():
     # SM clocks are sampled only while a workload's GPU regions run (not while the
     # host generates inputs or runs the oracle)
     clocks = ClockSampler(local)
-    r = Runner(w, slr, dev, dist, sdist, world)
+    r = Runner(w, slr, dev, dist, sdist, world, phi=args.phi)
     clocks.start()
     time.sleep(0.25)
     res = r.measure(args.steps, warmup, peaks, peak_src, with_e2e=not args.no_e2e)
@@ -506,12 +510,12 @@ def main():
         for ow in OTHER_WORKLOADS:
             if ow.name == w.name:
                 continue
-            ro = Runner(ow, slr, dev, dist, sdist, world)
+            ro = Runner(ow, slr, dev, dist, sdist, world, phi=args.phi)
             clocks.start(append=True)
             time.sleep(0.25)
             o = ro.measure(args.steps, warmup, peaks, peak_src, with_e2e=False)
             clocks.pause()
-            others.append((ow, {"config": config_dict(ow), **o}))
+            others.append((ow, {"config": config_dict(ow, args.phi), **o}))
             ro.release()
             del ro
     clk = clocks.stop()
@@ -520,7 +524,7 @@ def main():
             rows = {"hunyuan": 16, "lvsa": 8, "ropeslr": 8}.get(ow.name, 16)
             qo, ko, vo = workloads.make_qkv(ow, heads=2)
             cms, desc, threads = cpu_oracle_sample(ow, qo, ko, vo, workloads.make_w_proj(ow), rows_per_head=rows,
-                                                   heads=2)
+                                                   heads=2, phi=args.phi)
             o["cpu_baseline"] = {"value": round(cms, 1), "unit": UNIT, "cores": threads, "kind": "oracle",
                                  "sample": desc, "extrapolated": True}
     others = [o for _, o in others]
@@ -528,7 +532,7 @@ def main():
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cms, desc, threads = cpu_oracle_sample(w, q_h, k_h, v_h, wp_h, rows_per_head=args.oracle_rows,
-                                               heads=args.oracle_heads)
+                                               heads=args.oracle_heads, phi=args.phi)
         cpu = {"value": round(cms, 1), "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc,
                "extrapolated": True, "host_cpus": os.cpu_count()}
 
@@ -548,7 +552,7 @@ def main():
             "vs_baseline": None,
             "dtype": "bf16",
             "data": "synthetic (seeded bf16; frame-correlated for the SLA workloads)",
-            "config": config_dict(w),
+            "config": config_dict(w, args.phi),
             **{k_: res[k_] for k_ in ("tflops_computed_blocks", "tflops_pct_bf16_peak", "dense_ms_per_call",
                                       "dense_ms_median", "speedup_vs_dense", "speedup_vs_dense_median",
                                       "roofline", "work", "kernels", "profiled_ms_per_step", "gpu_launches")},
@@ -571,18 +575,18 @@ def run_reference(args, w, rank, world, warmup):
     wp = workloads.make_w_proj(w)
     rows, heads = args.oracle_rows, args.oracle_heads
     for _ in range(min(warmup, 1)):
-        cpu_oracle_sample(w, q, k, v, wp, rows_per_head=rows, heads=heads)
+        cpu_oracle_sample(w, q, k, v, wp, rows_per_head=rows, heads=heads, phi=args.phi)
     vals = []
     desc, threads = "", 1
     for _ in range(max(1, min(args.steps, 3))):
-        ms, desc, threads = cpu_oracle_sample(w, q, k, v, wp, rows_per_head=rows, heads=heads)
+        ms, desc, threads = cpu_oracle_sample(w, q, k, v, wp, rows_per_head=rows, heads=heads, phi=args.phi)
         vals.append(ms)
     val = statistics.median(vals)
     line = {
         "metric": METRIC, "value": round(val, 1), "unit": UNIT, "n_gpus": world, "steps": len(vals),
         "warmup": warmup, "ms_per_step": round(val, 1), "higher_is_better": False, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded bf16; frame-correlated for the SLA workloads)",
-        "config": config_dict(w), "impl": "reference",
+        "config": config_dict(w, args.phi), "impl": "reference",
         "cpu_baseline": {"value": round(val, 1), "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc,
                          "extrapolated": True},
         "e2e": {"value": round(val, 1), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},

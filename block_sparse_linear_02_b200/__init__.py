@@ -28,6 +28,7 @@ SLR_ERR_TIMEOUT = -5
 SLR_ERR_INDEX = -6
 
 SLR_PHI_ELU1 = 0
+SLR_PHI_SOFTMAX = 1
 SLR_MASK_LVSA = 1
 SLR_MASK_TILE3D = 2
 
@@ -292,7 +293,7 @@ def slr_block_sparse_attn(q, k, v, seq: SlrSeq, kv_idx=None, kv_cnt=None, out=No
     return o, l
 
 
-def slr_linear_marginal(q, k, v, seq: SlrSeq, mask, w_proj=None, out=None, ws=None):
+def slr_linear_marginal(q, k, v, seq: SlrSeq, mask, w_proj=None, out=None, ws=None, phi: int = SLR_PHI_ELU1):
     """Linear attention over the marginal (mask == 0) key blocks, optionally times W_proj; fp32 output."""
     import torch
     _check_qkv(q, k, v)
@@ -303,13 +304,13 @@ def slr_linear_marginal(q, k, v, seq: SlrSeq, mask, w_proj=None, out=None, ws=No
     need = slr_workspace_bytes(SLR_OP_LINEAR_MARGINAL, seq, None)
     wp, wn = _ws(ws, dev).get(need, dev)
     _check(lib().slr_linear_marginal(_ptr(q), _ptr(k), _ptr(v), ctypes.byref(seq), _ptr(mask.contiguous()),
-                                     SLR_PHI_ELU1, _ptr(w_proj), _ptr(o), wp, wn, _stream(q)),
+                                     phi, _ptr(w_proj), _ptr(o), wp, wn, _stream(q)),
            "slr_linear_marginal")
     return o
 
 
 def slr_sparse_linear_attn(q, k, v, w_proj, seq: SlrSeq, crit_frac: float, negl_frac: float,
-                           out=None, mask_out: bool = False, ws=None):
+                           out=None, mask_out: bool = False, ws=None, phi: int = SLR_PHI_ELU1):
     """The full SLA forward; returns (out bf16, mask int8 or None)."""
     import torch
     _check_qkv(q, k, v)
@@ -320,7 +321,7 @@ def slr_sparse_linear_attn(q, k, v, w_proj, seq: SlrSeq, crit_frac: float, negl_
     need = slr_workspace_bytes(SLR_OP_SPARSE_LINEAR, seq, SlrFracs(crit_frac, negl_frac))
     wp, wn = _ws(ws, dev).get(need, dev)
     _check(lib().slr_sparse_linear_attn(_ptr(q), _ptr(k), _ptr(v), _ptr(w_proj), ctypes.byref(seq), crit_frac,
-                                        negl_frac, SLR_PHI_ELU1, _ptr(o), _ptr(m), wp, wn, _stream(q)),
+                                        negl_frac, phi, _ptr(o), _ptr(m), wp, wn, _stream(q)),
            "slr_sparse_linear_attn")
     return o, m
 

@@ -55,7 +55,7 @@ template <int D, bool PROJ>
 __global__ void __launch_bounds__(128, 2)
 key_states_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                   const __grid_constant__ CUtensorMap tmW, __nv_bfloat16* __restrict__ h, SeqShape s, int BH,
-                  int* status) {
+                  int phi, int* status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint8_t* sW = smem + kKsW;               // W_proj MN-major: rows c_in, 64 c_out per chunk (chunk stride D*128)
@@ -149,15 +149,27 @@ key_states_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
     float z[8];
     #pragma unroll
     for (int i = 0; i < 8; ++i) z[i] = 0.f;
-    for (int t = rs; t < 64; t += kRS) {
+    for (int t = rs; t < 64; t += kRS) {       // the same trip count in every lane
       uint4* pk = reinterpret_cast<uint4*>(k_s + chunk * kChunkB + sw128_offset(t, q8));
       const uint4 u = *pk;
       const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+      float f[8];
+      #pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        f[2 * i] = bf16_lo(w[i]);
+        f[2 * i + 1] = bf16_hi(w[i]);
+      }
+      if (phi == SLR_PHI_SOFTMAX) {
+        row_softmax8<kCPR>(f);                 // the kCPR lanes of row t
+      } else {
+        #pragma unroll
+        for (int i = 0; i < 8; ++i) f[i] = phi_elu1(f[i]);
+      }
       uint32_t o[4];
       #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const float a = t < nvalid ? phi_elu1(bf16_lo(w[i])) : 0.f;
-        const float b = t < nvalid ? phi_elu1(bf16_hi(w[i])) : 0.f;
+        const float a = t < nvalid ? f[2 * i] : 0.f;
+        const float b = t < nvalid ? f[2 * i + 1] : 0.f;
         z[2 * i] += a;
         z[2 * i + 1] += b;
         o[i] = pack_bf16(a, b);
@@ -271,7 +283,7 @@ template <bool PROJ>
 __global__ void __launch_bounds__(448, 1)
 key_states_pipe_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                        const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmH,
-                       __nv_bfloat16* __restrict__ h, SeqShape s, int BH, int* status) {
+                       __nv_bfloat16* __restrict__ h, SeqShape s, int BH, int phi, int* status) {
   constexpr int D = 128;
   using L = KpLayout;
   extern __shared__ uint8_t smem_raw[];
@@ -421,11 +433,23 @@ key_states_pipe_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_con
         uint4* pk = reinterpret_cast<uint4*>(k_s + chunk * kChunkB + sw128_offset(t, q8));
         const uint4 u = *pk;
         const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+        float f[8];
+        #pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          f[2 * i] = bf16_lo(w[i]);
+          f[2 * i + 1] = bf16_hi(w[i]);
+        }
+        if (phi == SLR_PHI_SOFTMAX) {
+          row_softmax8<kCPR>(f);               // the kCPR lanes of row t (a half warp)
+        } else {
+          #pragma unroll
+          for (int i = 0; i < 8; ++i) f[i] = phi_exp2(f[i]);
+        }
         uint32_t o[4];
         #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          const float x0 = t < nvalid ? phi_exp2(bf16_lo(w[i])) : 0.f;
-          const float x1 = t < nvalid ? phi_exp2(bf16_hi(w[i])) : 0.f;
+          const float x0 = t < nvalid ? f[2 * i] : 0.f;
+          const float x1 = t < nvalid ? f[2 * i + 1] : 0.f;
           z[2 * i] += x0;
           z[2 * i + 1] += x1;
           o[i] = pack_bf16(x0, x1);
@@ -696,7 +720,7 @@ __device__ __forceinline__ void mma_masked(uint32_t d_tmem, uint64_t a, uint64_t
 template <int D>
 __global__ void __launch_bounds__(128)
 linear_apply_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmH,
-                    float* __restrict__ o_lin, SeqShape s, int* status) {
+                    float* __restrict__ o_lin, SeqShape s, int phi, int* status) {
   using L = ApplyLayout<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
@@ -729,11 +753,32 @@ linear_apply_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     }
   }
   bool ok = cta_wait(&bars[0], 0, abort_flag, status);
-  // phi(Q) in place, one row per thread; pad rows -> 0
+  // phi(Q) in place, one row per thread; pad rows -> 0.  The softmax map takes the
+  // row max in a first pass over the row and the sum of exponentials in a second.
   const int r = tid;
   const int tok = pair * 128 + r;
   const bool valid = tok < s.n_pad && token_valid(s, tok);
   if (ok) {
+    float m = -INFINITY, inv = 1.f;
+    if (phi == SLR_PHI_SOFTMAX) {
+      #pragma unroll
+      for (int gg = 0; gg < D / 8; ++gg) {
+        const uint4 u = *reinterpret_cast<const uint4*>(sQ + (gg >> 3) * 16384 + sw128_offset(r, gg & 7));
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+        #pragma unroll
+        for (int i = 0; i < 4; ++i) m = fmaxf(m, fmaxf(bf16_lo(w[i]), bf16_hi(w[i])));
+      }
+      float sum = 0.f;
+      #pragma unroll
+      for (int gg = 0; gg < D / 8; ++gg) {
+        const uint4 u = *reinterpret_cast<const uint4*>(sQ + (gg >> 3) * 16384 + sw128_offset(r, gg & 7));
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+        #pragma unroll
+        for (int i = 0; i < 4; ++i)
+          sum += exp2f((bf16_lo(w[i]) - m) * 1.4426950408889634f) + exp2f((bf16_hi(w[i]) - m) * 1.4426950408889634f);
+      }
+      inv = 1.f / sum;
+    }
     #pragma unroll
     for (int gg = 0; gg < D / 8; ++gg) {
       uint4* ptr = reinterpret_cast<uint4*>(sQ + (gg >> 3) * 16384 + sw128_offset(r, gg & 7));
@@ -741,7 +786,17 @@ linear_apply_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
       const uint32_t w[4] = {u.x, u.y, u.z, u.w};
       uint32_t o4[4];
       #pragma unroll
-      for (int i = 0; i < 4; ++i) o4[i] = valid ? pack_bf16(phi_elu1(bf16_lo(w[i])), phi_elu1(bf16_hi(w[i]))) : 0u;
+      for (int i = 0; i < 4; ++i) {
+        float a = bf16_lo(w[i]), b = bf16_hi(w[i]);
+        if (phi == SLR_PHI_SOFTMAX) {
+          a = exp2f((a - m) * 1.4426950408889634f) * inv;
+          b = exp2f((b - m) * 1.4426950408889634f) * inv;
+        } else {
+          a = phi_elu1(a);
+          b = phi_elu1(b);
+        }
+        o4[i] = valid ? pack_bf16(a, b) : 0u;
+      }
       *ptr = make_uint4(o4[0], o4[1], o4[2], o4[3]);
     }
   }
@@ -810,8 +865,8 @@ linear_apply_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
 
 }  // namespace
 
-cudaError_t launch_key_states(const void* k, const void* v, const void* w_proj, __nv_bfloat16* h, int BH, int d,
-                              SeqShape s, int* status, cudaStream_t st) {
+cudaError_t launch_key_states(const void* k, const void* v, const void* w_proj, __nv_bfloat16* h, int phi, int BH,
+                              int d, SeqShape s, int* status, cudaStream_t st) {
   CUtensorMap mk, mv, mw;
   const uint64_t dims[3] = {(uint64_t)d, (uint64_t)s.n_pad, (uint64_t)BH};
   const uint64_t strides[2] = {(uint64_t)d * 2, (uint64_t)d * 2 * s.n_pad};
@@ -834,7 +889,7 @@ cudaError_t launch_key_states(const void* k, const void* v, const void* w_proj, 
   auto go = [&](auto kern) -> cudaError_t {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kKsSmem);
     if (e != cudaSuccess) return e;
-    kern<<<grid, 128, kKsSmem, st>>>(mk, mv, mw, h, s, BH, status);
+    kern<<<grid, 128, kKsSmem, st>>>(mk, mv, mw, h, s, BH, phi, status);
     return cudaGetLastError();
   };
   if (d == 128) {
@@ -848,7 +903,7 @@ cudaError_t launch_key_states(const void* k, const void* v, const void* w_proj, 
     auto pipe = [&](auto kern) -> cudaError_t {
       cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, KpLayout::kBytes);
       if (e != cudaSuccess) return e;
-      kern<<<pgrid, 448, KpLayout::kBytes, st>>>(mk, mv, mw, mh, h, s, BH, status);
+      kern<<<pgrid, 448, KpLayout::kBytes, st>>>(mk, mv, mw, mh, h, s, BH, phi, status);
       return cudaGetLastError();
     };
     return w_proj ? pipe(key_states_pipe_kernel<true>) : pipe(key_states_pipe_kernel<false>);
@@ -881,8 +936,8 @@ cudaError_t launch_reduce_states(const __nv_bfloat16* m01, int ld_m01, const __n
   return cudaGetLastError();
 }
 
-cudaError_t launch_linear_apply(const void* q, const __nv_bfloat16* Hs, float* o_lin, int BH, int d, SeqShape s,
-                                int* status, cudaStream_t st) {
+cudaError_t launch_linear_apply(const void* q, const __nv_bfloat16* Hs, float* o_lin, int phi, int BH, int d,
+                                SeqShape s, int* status, cudaStream_t st) {
   CUtensorMap mq, mh;
   const uint64_t qdims[3] = {(uint64_t)d, (uint64_t)s.n_pad, (uint64_t)BH};
   const uint64_t qstr[2] = {(uint64_t)d * 2, (uint64_t)d * 2 * s.n_pad};
@@ -896,11 +951,11 @@ cudaError_t launch_linear_apply(const void* q, const __nv_bfloat16* Hs, float* o
   if (d == 128) {
     cudaError_t e = cudaFuncSetAttribute(linear_apply_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, ApplyLayout<128>::kBytes);
     if (e != cudaSuccess) return e;
-    linear_apply_kernel<128><<<grid, 128, ApplyLayout<128>::kBytes, st>>>(mq, mh, o_lin, s, status);
+    linear_apply_kernel<128><<<grid, 128, ApplyLayout<128>::kBytes, st>>>(mq, mh, o_lin, s, phi, status);
   } else {
     cudaError_t e = cudaFuncSetAttribute(linear_apply_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, ApplyLayout<64>::kBytes);
     if (e != cudaSuccess) return e;
-    linear_apply_kernel<64><<<grid, 128, ApplyLayout<64>::kBytes, st>>>(mq, mh, o_lin, s, status);
+    linear_apply_kernel<64><<<grid, 128, ApplyLayout<64>::kBytes, st>>>(mq, mh, o_lin, s, phi, status);
   }
   return cudaGetLastError();
 }

@@ -34,7 +34,7 @@ template <int D>
 __global__ void __launch_bounds__(128)
 pool_means_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
                   __nv_bfloat16* __restrict__ qsplit, __nv_bfloat16* __restrict__ ksplit,
-                  __nv_bfloat16* __restrict__ phi_q, SeqShape s) {
+                  __nv_bfloat16* __restrict__ phi_q, int phi, SeqShape s) {
   constexpr int kCPR = D / 8;          // 16-byte chunks per row
   constexpr int kRG = 128 / kCPR;      // row groups
   __shared__ double red[kRG][D];
@@ -58,10 +58,21 @@ pool_means_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
     for (int k = 0; k < kRows; ++k) {
       const int r = rg + k * kRG;
       const uint32_t w[4] = {u[k].x, u[k].y, u[k].z, u[k].w};
+      float f[8];
+      #pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        f[2 * i] = bf16_lo(w[i]);
+        f[2 * i + 1] = bf16_hi(w[i]);
+      }
+      if (phi == SLR_PHI_SOFTMAX) {
+        row_softmax8<kCPR>(f);                   // the kCPR lanes of row r (uniform: phi is per launch)
+      } else {
+        #pragma unroll
+        for (int i = 0; i < 8; ++i) f[i] = phi_elu1_ex2(f[i]);
+      }
       uint32_t o[4];
       #pragma unroll
-      for (int i = 0; i < 4; ++i)
-        o[i] = r < nvalid ? pack_bf16(phi_elu1_ex2(bf16_lo(w[i])), phi_elu1_ex2(bf16_hi(w[i]))) : 0u;
+      for (int i = 0; i < 4; ++i) o[i] = r < nvalid ? pack_bf16(f[2 * i], f[2 * i + 1]) : 0u;
       dst[(size_t)r * (D / 8) + chunk] = make_uint4(o[0], o[1], o[2], o[3]);
     }
   }
@@ -138,16 +149,16 @@ far_pool_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __rest
 
 }  // namespace
 
-cudaError_t launch_pool_means(const void* q, const void* k, void* qsplit, void* ksplit, void* phi_q,
+cudaError_t launch_pool_means(const void* q, const void* k, void* qsplit, void* ksplit, void* phi_q, int phi,
                               int BH, int d, SeqShape s, cudaStream_t st) {
   dim3 grid(s.n_blocks, BH, 2);
   auto* qs = static_cast<__nv_bfloat16*>(qsplit);
   auto* ks = static_cast<__nv_bfloat16*>(ksplit);
   auto* pq = static_cast<__nv_bfloat16*>(phi_q);
   if (d == 128)
-    pool_means_kernel<128><<<grid, 128, 0, st>>>((const __nv_bfloat16*)q, (const __nv_bfloat16*)k, qs, ks, pq, s);
+    pool_means_kernel<128><<<grid, 128, 0, st>>>((const __nv_bfloat16*)q, (const __nv_bfloat16*)k, qs, ks, pq, phi, s);
   else
-    pool_means_kernel<64><<<grid, 128, 0, st>>>((const __nv_bfloat16*)q, (const __nv_bfloat16*)k, qs, ks, pq, s);
+    pool_means_kernel<64><<<grid, 128, 0, st>>>((const __nv_bfloat16*)q, (const __nv_bfloat16*)k, qs, ks, pq, phi, s);
   return cudaGetLastError();
 }
 

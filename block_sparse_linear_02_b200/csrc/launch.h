@@ -5,6 +5,8 @@
 
 #include <cuda_runtime.h>
 #include <cuda.h>
+
+#include "../../include/slr.h"   // the SLR_PHI_* feature-map codes the kernels take
 #include <cuda_bf16.h>
 #include <stdint.h>
 
@@ -23,8 +25,9 @@ bool make_tile_map(CUtensorMap* map, const void* base, int rank, const uint64_t*
 // ------------------------------------------------------------ pooling (k_pool.cu)
 // Means of the valid tokens of every 64-token block of q and k, each written as a
 // bf16 pair hi + lo: rows [BH][Nb][3d], [qh | qh | ql] for q and [kh | kl | kh] for k.
-// With phi_q non-null, also phi(q) = elu(q) + 1 in bf16 [BH][N_pad][d] (pad tokens 0).
-cudaError_t launch_pool_means(const void* q, const void* k, void* qsplit, void* ksplit, void* phi_q,
+// With phi_q non-null, also phi(q) in bf16 [BH][N_pad][d] (pad tokens 0); phi is
+// SLR_PHI_ELU1 (elu(q) + 1) or SLR_PHI_SOFTMAX (softmax of each row over its d channels).
+cudaError_t launch_pool_means(const void* q, const void* k, void* qsplit, void* ksplit, void* phi_q, int phi,
                               int BH, int d, SeqShape s, cudaStream_t st);
 
 // Far-field K/V: means over cells of (cf, ch, cw) tokens of the raster (F, Hh, Ww),
@@ -113,8 +116,8 @@ cudaError_t launch_attention(const AttnArgs& a, cudaStream_t st);
 // ------------------------------------------------------------ marginal branch (k_marginal.cu)
 // h[bh][j] = [ (phi(K_j)^T V_j W)^T (d rows of d) ; z_j (1 row) ] in bf16, [BH][nb][(d+1)*d];
 // W = w_proj (bf16 [d][d]) or the identity when w_proj is null.
-cudaError_t launch_key_states(const void* k, const void* v, const void* w_proj, __nv_bfloat16* h, int BH, int d,
-                              SeqShape s, int* status, cudaStream_t st);
+cudaError_t launch_key_states(const void* k, const void* v, const void* w_proj, __nv_bfloat16* h, int phi, int BH,
+                              int d, SeqShape s, int* status, cudaStream_t st);
 
 // Hs[bh][i] = sum_j m01[bh][i][j] * h[bh][j]  (bf16 out, fp32 accumulate), [BH][nb][(d+1)*d].
 cudaError_t launch_reduce_states(const __nv_bfloat16* m01, int ld_m01, const __nv_bfloat16* h,
@@ -125,7 +128,7 @@ cudaError_t launch_reduce_states(const __nv_bfloat16* m01, int ld_m01, const __n
 // Reads and clears the status word of the static scratch on the current device.
 int noalloc_check_status(void* stream);   // an slr_status value
 
-cudaError_t launch_linear_apply(const void* q, const __nv_bfloat16* Hs, float* o_lin, int BH, int d, SeqShape s,
-                                int* status, cudaStream_t st);
+cudaError_t launch_linear_apply(const void* q, const __nv_bfloat16* Hs, float* o_lin, int phi, int BH, int d,
+                                SeqShape s, int* status, cudaStream_t st);
 
 }  // namespace slr

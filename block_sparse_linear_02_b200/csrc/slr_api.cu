@@ -451,7 +451,7 @@ slr_status slr_pool_classify(const void* q, const void* k, const slr_seq* seq, f
   ClassifyWs w;
   plan_classify(c, sh, false, w);
   SLR_TRY(cudaMemsetAsync(status, 0, sizeof(int), s));
-  SLR_LAUNCH(kKPool, s, launch_pool_means(q, k, w.qsplit, w.ksplit, nullptr, sh.BH, sh.d, sh.s, s));
+  SLR_LAUNCH(kKPool, s, launch_pool_means(q, k, w.qsplit, w.ksplit, nullptr, SLR_PHI_ELU1, sh.BH, sh.d, sh.s, s));
   SLR_LAUNCH(kKLogits, s, launch_logits(w.qsplit, w.ksplit, w.keys, sh.BH, sh.nb, sh.d, status, s));
   SLR_LAUNCH(kKClassify, s, launch_classify(w.keys, sh.BH, sh.nb, sh.d, kc, kn, mask, crit_idx, crit_cnt,
                                             nullptr, 0, scores_opt, nullptr, nullptr, 0, sh.s, status, s));
@@ -499,7 +499,7 @@ slr_status slr_linear_marginal(const void* q, const void* k, const void* v, cons
   if (st != SLR_OK) return st;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !mask || !aligned16(o_lin)) return SLR_ERR_ARG;
   if (w_proj_opt && !aligned16(w_proj_opt)) return SLR_ERR_ARG;
-  if (phi != SLR_PHI_ELU1) return SLR_ERR_UNSUPPORTED;
+  if (phi != SLR_PHI_ELU1 && phi != SLR_PHI_SOFTMAX) return SLR_ERR_UNSUPPORTED;
   if ((st = ws_check(ws, ws_bytes, slr_workspace_bytes(SLR_OP_LINEAR_MARGINAL, seq, nullptr))) != SLR_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   Carve c(ws);
@@ -509,9 +509,9 @@ slr_status slr_linear_marginal(const void* q, const void* k, const void* v, cons
   plan_marginal(c, sh, w);
   SLR_TRY(cudaMemsetAsync(status, 0, sizeof(int), s));
   SLR_LAUNCH(kKMaskToM01, s, launch_mask_to_m01(mask, m01, sh.BH, sh.nb, ld_m01(sh.nb), s));
-  SLR_LAUNCH(kKKeyStates, s, launch_key_states(k, v, w_proj_opt, w.h, sh.BH, sh.d, sh.s, status, s));
+  SLR_LAUNCH(kKKeyStates, s, launch_key_states(k, v, w_proj_opt, w.h, phi, sh.BH, sh.d, sh.s, status, s));
   SLR_LAUNCH(kKReduce, s, launch_reduce_states(m01, ld_m01(sh.nb), w.h, w.Hs, sh.BH, sh.nb, sh.d, status, s));
-  SLR_LAUNCH(kKApply, s, launch_linear_apply(q, w.Hs, o_lin, sh.BH, sh.d, sh.s, status, s));
+  SLR_LAUNCH(kKApply, s, launch_linear_apply(q, w.Hs, o_lin, phi, sh.BH, sh.d, sh.s, status, s));
   return SLR_OK;
 }
 
@@ -522,7 +522,7 @@ slr_status slr_sparse_linear_attn(const void* q, const void* k, const void* v, c
   slr_status st = check_seq(seq, sh);
   if (st != SLR_OK) return st;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return SLR_ERR_ARG;
-  if (phi != SLR_PHI_ELU1) return SLR_ERR_UNSUPPORTED;
+  if (phi != SLR_PHI_ELU1 && phi != SLR_PHI_SOFTMAX) return SLR_ERR_UNSUPPORTED;
   int kc, kn;
   if ((st = counts(sh.nb, crit_frac, negl_frac, &kc, &kn)) != SLR_OK) return st;
   const bool dense = kc == sh.nb;
@@ -542,13 +542,13 @@ slr_status slr_sparse_linear_attn(const void* q, const void* k, const void* v, c
     SLR_LAUNCH(kKAttention, s, launch_attention(a, s));
     return SLR_OK;
   }
-  SLR_LAUNCH(kKPool, s, launch_pool_means(q, k, w.cls.qsplit, w.cls.ksplit, w.cls.phi_q, sh.BH, sh.d, sh.s, s));
+  SLR_LAUNCH(kKPool, s, launch_pool_means(q, k, w.cls.qsplit, w.cls.ksplit, w.cls.phi_q, phi, sh.BH, sh.d, sh.s, s));
   SLR_LAUNCH(kKLogits, s, launch_logits(w.cls.qsplit, w.cls.ksplit, w.cls.keys, sh.BH, sh.nb, sh.d, w.status, s));
   SLR_LAUNCH(kKClassify, s, launch_classify(w.cls.keys, sh.BH, sh.nb, sh.d, kc, kn, mask_out_opt, nullptr,
                                             nullptr, w.cls.m01, ld_m01(sh.nb), nullptr, w.list, w.list_cnt, w.cap,
                                             sh.s, w.status, s));
   if (marginal) {
-    SLR_LAUNCH(kKKeyStates, s, launch_key_states(k, v, w_proj, w.mar.h, sh.BH, sh.d, sh.s, w.status, s));
+    SLR_LAUNCH(kKKeyStates, s, launch_key_states(k, v, w_proj, w.mar.h, phi, sh.BH, sh.d, sh.s, w.status, s));
     SLR_LAUNCH(kKReduce, s, launch_reduce_states(w.cls.m01, ld_m01(sh.nb), w.mar.h, w.mar.Hs, sh.BH, sh.nb, sh.d, w.status, s));
     a.Hs = w.mar.Hs;
     a.phi_q = w.cls.phi_q;

@@ -250,4 +250,27 @@ __device__ __forceinline__ float bf16_hi(uint32_t u) { return __uint_as_float(u 
 // phi(x) = elu(x) + 1
 __device__ __forceinline__ float phi_elu1(float x) { return x > 0.f ? x + 1.f : expf(x); }
 
+// The softmax feature map: one row of channels, spread over a group of kLanes
+// consecutive lanes that hold 8 channels each, is replaced by its softmax.  Every
+// lane of the warp takes part (the reductions are warp shuffles).
+template <int kLanes>
+__device__ __forceinline__ void row_softmax8(float (&x)[8]) {
+  float m = x[0];
+  #pragma unroll
+  for (int i = 1; i < 8; ++i) m = fmaxf(m, x[i]);
+  #pragma unroll
+  for (int off = kLanes / 2; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, off));
+  float sum = 0.f;
+  #pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    x[i] = exp2f((x[i] - m) * 1.4426950408889634f);
+    sum += x[i];
+  }
+  #pragma unroll
+  for (int off = kLanes / 2; off > 0; off >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, off);
+  const float inv = 1.f / sum;
+  #pragma unroll
+  for (int i = 0; i < 8; ++i) x[i] *= inv;
+}
+
 }  // namespace slr

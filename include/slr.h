@@ -59,8 +59,11 @@ typedef struct {
 } slr_seq;
 
 /* Feature map of the linear branch; SLA page section 3 names phi, and the
- * plainest reading used here is phi(x) = elu(x) + 1. */
+ * plainest reading used here is phi(x) = elu(x) + 1.  The page later reports that
+ * a softmax activation works better there; SLR_PHI_SOFTMAX reads it as the softmax
+ * of each q and k row over its d channels. */
 #define SLR_PHI_ELU1 0
+#define SLR_PHI_SOFTMAX 1
 
 /* External block masks for slr_frame_mask_attn. */
 #define SLR_MASK_LVSA   1
@@ -151,7 +154,7 @@ slr_status slr_block_sparse_attn(const void* q, const void* k, const void* v, co
  * optionally multiplied on the right by W_proj (SLA page, projection paragraph).
  *
  *   mask       int8 [B][H][Nb][Nb] device: 0 = marginal, anything else = not
- *   phi        SLR_PHI_ELU1
+ *   phi        SLR_PHI_ELU1 or SLR_PHI_SOFTMAX
  *   w_proj_opt bf16 [d][d] device or NULL (NULL = no projection)
  *   o_lin      float [B][H][N_pad][d] device, written
  */

@@ -26,7 +26,7 @@ def _seq(w):
     return slr.make_seq(w.batch, w.heads, w.d, w.n_seg, w.seg_len, w.seg_stride)
 
 
-def _compare(q, k, v, wp, seq, crit, negl, out, mask, heads, sample=None, seed=0, batches=(0,)):
+def _compare(q, k, v, wp, seq, crit, negl, out, mask, heads, sample=None, seed=0, batches=(0,), phi="elu1"):
     """Masks of every listed (b, h) in full; outputs on all or `sample` query blocks.
     Returns the number of query blocks whose label row differed (checked on the
     library's labels)."""
@@ -42,7 +42,7 @@ def _compare(q, k, v, wp, seq, crit, negl, out, mask, heads, sample=None, seed=0
                 rng = np.random.default_rng(seed + 100 * b + h)
                 rows = sorted(set([0, nb - 1] + list(rng.choice(nb, sample, replace=False))))
             q64, k64, v64 = to64(q[b, h]), to64(k[b, h]), to64(v[b, h])
-            r = osla.sla_head(q64, k64, v64, w64, valid, crit, negl, rows=rows)
+            r = osla.sla_head(q64, k64, v64, w64, valid, crit, negl, rows=rows, phi=phi)
             gm = mask[b, h].cpu().numpy()
             check_mask(gm, r["mask"], r["p"], r["tau_c"], r["tau_n"], r["kc"], r["kn"])
             rows = list(range(nb)) if rows is None else rows
@@ -51,7 +51,7 @@ def _compare(q, k, v, wp, seq, crit, negl, out, mask, heads, sample=None, seed=0
             if moved:
                 # the oracle's forward on the library's labels for those query blocks
                 o_s = osla.block_sparse_attention(q64, k64, v64, valid, osla.lists_from_mask(gm, 1), rows=moved)
-                o_l = osla.linear_attention(q64, k64, v64, valid, gm == 0, rows=moved)
+                o_l = osla.linear_attention(q64, k64, v64, valid, gm == 0, rows=moved, phi=phi)
                 sel = rows_of_blocks(moved)
                 o_ref = o_ref.copy()
                 o_ref[sel] = (o_s + o_l @ w64)[sel]
@@ -85,6 +85,39 @@ def test_ragged_full(d):
     # pad query rows are zero
     pad = ~valid_np(n_seg, seg_len, stride)
     assert torch.count_nonzero(out[0, :, torch.from_numpy(pad)]).item() == 0
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_softmax_feature_map_ragged_full(d):
+    # the linear branch with phi = softmax over each q and k row's channels
+    H, n_seg, seg_len, stride = 2, 3, 600, 640
+    q, k, v = make_inputs(1, H, d, n_seg, seg_len, stride, seed=41 + d)
+    wp = random_bf16((d, d), 8, 1.0 / np.sqrt(d))
+    seq = slr.make_seq(1, H, d, n_seg, seg_len, stride)
+    out, mask = slr.slr_sparse_linear_attn(cuda(q), cuda(k), cuda(v), cuda(wp), seq, 0.1, 0.2, mask_out=True,
+                                           phi=slr.SLR_PHI_SOFTMAX)
+    status_ok()
+    assert _compare(q, k, v, wp, seq, 0.1, 0.2, out, mask, range(H), phi="softmax") == 0
+
+
+def test_softmax_feature_map_tiny_and_wan_sampled():
+    # the tiny workload in full and the 32k-token workload on 16 sampled blocks of 4 heads
+    w = workloads.TINY
+    q, k, v = workloads.make_qkv(w)
+    wp = workloads.make_w_proj(w)
+    out, mask = slr.slr_sparse_linear_attn(cuda(q), cuda(k), cuda(v), cuda(wp), _seq(w), w.crit_frac,
+                                           w.negl_frac, mask_out=True, phi=slr.SLR_PHI_SOFTMAX)
+    status_ok()
+    assert _compare(q, k, v, wp, _seq(w), w.crit_frac, w.negl_frac, out, mask, range(w.heads), phi="softmax") == 0
+    w = workloads.WAN
+    q, k, v = workloads.make_qkv(w)
+    wp = workloads.make_w_proj(w)
+    out, mask = slr.slr_sparse_linear_attn(cuda(q), cuda(k), cuda(v), cuda(wp), _seq(w), w.crit_frac,
+                                           w.negl_frac, mask_out=True, phi=slr.SLR_PHI_SOFTMAX)
+    status_ok()
+    flipped = _compare(q, k, v, wp, _seq(w), w.crit_frac, w.negl_frac, out, mask, [0, 5, 6, 11], sample=16,
+                       phi="softmax")
+    assert flipped <= 2
 
 
 def test_two_batch_entries_full():
