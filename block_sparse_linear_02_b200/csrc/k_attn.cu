@@ -33,9 +33,9 @@
 // accumulator O_w) over its share of the key blocks; the epilogue merges the two
 // shares exactly: O = (2^(m0-M) O_0 + 2^(m1-M) O_1) / (2^(m0-M) l_0 + 2^(m1-M) l_1).
 // The softmax works in the exp2 domain with lazy rescaling (an accumulator is
-// rescaled only when its running max grows by more than 2^8).  In the row-major
-// layouts the output leaves through shared memory: each softmax warp stages its 32
-// rows x 32 columns and one TMA tensor store writes them.
+// rescaled only when its running max grows by more than 2^8).  The output leaves
+// through shared memory: each softmax warp stages its 32 rows x 32 columns and one TMA
+// tensor store writes them (in the tile layout the 32 rows are a 2 x 4 x 4 brick).
 #include <cuda_runtime.h>
 #include <math.h>
 
@@ -66,8 +66,8 @@ struct AttnLayout {
   static constexpr int kZOff = kRingOff + kSlots * kKV;  // Z tiles of the pair's two query blocks
   static constexpr int kXOff = kZOff + 2 * kZTile;       // exchange area: [2 shares][2 tiles][3][128] floats
   static constexpr int kBarOff = kXOff + 12 * 128 * 4;
-  // output staging (non-tile layouts): per softmax warp one 32-row x 32-column bf16
-  // chunk (64-byte rows, 64-byte swizzle), written to HBM by TMA tensor stores
+  // output staging: per softmax warp one 32-row x 32-column bf16 chunk (64-byte rows,
+  // 64-byte swizzle), written to HBM by TMA tensor stores
   static constexpr int kOutChunk = 32 * 64;
   static constexpr int kOutOff = (kBarOff + 512 + 1023) / 1024 * 1024;
   static constexpr int kBytes = kOutOff + 8 * kOutChunk + 1024;   // + alignment slack
@@ -196,7 +196,8 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
   // tmX1/tmX2: far-field K/V maps (GATED), or the linear state maps (LINEAR): tmX1 the
   // H'^T rows (box D rows), tmX2 the Z row with 15 rows of zero fill (box 16 rows);
   // tmX3: phi(Q) (LINEAR, same boxes as Q).  tmO: the output, boxes of 32 rows x 32
-  // columns with 64-byte swizzle (not used by the tile layout).
+  // columns with 64-byte swizzle; in the tile layout the 32 rows are a 2 x 4 x 4
+  // (frame, height, width) brick of one 4 x 4 x 4 tile.
   using L = AttnLayout<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -786,7 +787,6 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
       }
       const bool have_o0 = ok && n_local > 0;        // uniform over the softmax warps
       const bool have_o1 = ok && n_local > 1;
-      const size_t row_off = ((size_t)ti.bh * p.n_pad + (row_exists ? tok : 0)) * D;
       #pragma unroll
       for (int k = 0; k < D / 64; ++k) {
         const int cc = wg * (D / 64) + k;          // my 32-column chunks
@@ -821,39 +821,37 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
             v[2 * m + 1] = fmaf(bf16_hi(lin[k * 16 + m]), inv_den, v[2 * m + 1]);
           }
         }
-        if (TILE) {
-          if (!row_exists) continue;
-          uint4* dst = reinterpret_cast<uint4*>(p.out + row_off + cc * 32);
-          #pragma unroll
-          for (int m = 0; m < 4; ++m) {
-            uint4 w4 = make_uint4(0, 0, 0, 0);
-            if (valid)
-              w4 = make_uint4(pack_bf16(v[8 * m], v[8 * m + 1]), pack_bf16(v[8 * m + 2], v[8 * m + 3]),
-                              pack_bf16(v[8 * m + 4], v[8 * m + 5]), pack_bf16(v[8 * m + 6], v[8 * m + 7]));
-            dst[m] = w4;
-          }
-        } else {
-          // my row's 32 columns into the warp's staging chunk (64-byte swizzle: 16-byte piece
-          // m of row r sits at piece m ^ ((r >> 1) & 3)), then one TMA store of 32 rows; the
-          // rows past the sequence end are clipped by the tensor map
-          uint8_t* stg = sOut + warp * L::kOutChunk;
-          if (lane == 0) bulk_wait_read_all();     // the last store from this chunk has read it
-          __syncwarp();
-          #pragma unroll
-          for (int m = 0; m < 4; ++m) {
-            uint4 w4 = make_uint4(0, 0, 0, 0);
-            if (valid)
-              w4 = make_uint4(pack_bf16(v[8 * m], v[8 * m + 1]), pack_bf16(v[8 * m + 2], v[8 * m + 3]),
-                              pack_bf16(v[8 * m + 4], v[8 * m + 5]), pack_bf16(v[8 * m + 6], v[8 * m + 7]));
-            *reinterpret_cast<uint4*>(stg + lane * 64 + ((m ^ ((lane >> 1) & 3)) << 4)) = w4;
-          }
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) {
+        // my row's 32 columns into the warp's staging chunk (64-byte swizzle: 16-byte piece
+        // m of row r sits at piece m ^ ((r >> 1) & 3)), then one TMA store of the warp's 32
+        // rows; rows past the sequence end are clipped by the tensor map
+        uint8_t* stg = sOut + warp * L::kOutChunk;
+        if (lane == 0) bulk_wait_read_all();       // the last store from this chunk has read it
+        __syncwarp();
+        #pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          uint4 w4 = make_uint4(0, 0, 0, 0);
+          if (valid)
+            w4 = make_uint4(pack_bf16(v[8 * m], v[8 * m + 1]), pack_bf16(v[8 * m + 2], v[8 * m + 3]),
+                            pack_bf16(v[8 * m + 4], v[8 * m + 5]), pack_bf16(v[8 * m + 6], v[8 * m + 7]));
+          *reinterpret_cast<uint4*>(stg + lane * 64 + ((m ^ ((lane >> 1) & 3)) << 4)) = w4;
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          if (TILE) {
+            // warps 0-1 hold the first tile of the pair, 2-3 the second; each covers two of
+            // the tile's four frames (row = 16 f + 4 h + w inside the tile)
+            const int tile = 2 * ti.pair + ((warp & 3) >> 1);
+            if (tile < p.n_qb) {
+              int tf, th, tw;
+              tile_coords(tile, p.TF, p.TW, tf, th, tw);
+              tma_store_5d(&tmO, stg, cc * 32, tw * 4, th * 4, tf * 4 + 2 * (warp & 1), ti.bh);
+            }
+          } else {
             const int row0 = ti.pair * 128 + (warp & 3) * 32;
             if (row0 < p.n_pad) tma_store_3d(&tmO, stg, cc * 32, row0, ti.bh);
-            bulk_commit();
           }
+          bulk_commit();
         }
       }
       tc_fence_before();
@@ -869,7 +867,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
     }
   }
 
-  if (!TILE && warp < 8 && lane == 0) bulk_wait_all();   // output stores complete
+  if (warp < 8 && lane == 0) bulk_wait_all();   // output stores complete
   tc_fence_before();
   __syncthreads();
   if (warp == 9) {
@@ -931,8 +929,12 @@ cudaError_t launch_attention(const AttnArgs& a, cudaStream_t st) {
   maps[3] = maps[1];
   maps[4] = maps[2];
   maps[5] = maps[0];
-  maps[6] = maps[0];
-  if (!a.tile3d) {
+  if (a.tile3d) {
+    const uint64_t dims[5] = {(uint64_t)D, (uint64_t)a.Ww, (uint64_t)a.Hh, (uint64_t)a.F, (uint64_t)a.BH};
+    const uint64_t strides[4] = {rowb, rowb * a.Ww, rowb * a.Ww * a.Hh, rowb * a.Ww * a.Hh * a.F};
+    const uint32_t boxo[5] = {32, 4, 4, 2, 1};
+    if (!make_tile_map(&maps[6], a.out, 5, dims, strides, boxo, 64)) return cudaErrorInvalidValue;
+  } else {
     const uint64_t dims[3] = {(uint64_t)D, (uint64_t)a.s.n_pad, (uint64_t)a.BH};
     const uint64_t strides[2] = {rowb, rowb * a.s.n_pad};
     const uint32_t boxo[3] = {32, 32, 1};
