@@ -20,12 +20,24 @@ Readings:
   giving 64 pooled tokens for an 8x64x64 latent; the page's pyramid text is
   garbled (2k + 128 tokens cannot make rank 64), so the single pool is used;
 * the far-field branch has its own softmax over the pooled tokens;
-* RoPE is applied upstream: q and k arrive already rotated;
-* the gate multiplies the two normalised outputs.
+* the gate multiplies the two normalised outputs;
+* RoPE (the page: the neighbourhood branch "encodes relative position with
+  RoPE") is optional here (``rope=True``) and reads as the usual 3-D rotary
+  embedding: the d channels of q and k split into three contiguous groups for
+  the frame, height and width axes -- with P = d/2 channel pairs, the height
+  and width groups take floor(P/3) pairs each and the frame group the rest
+  (d = 128: 44, 42, 42 channels) -- and pair i of a group of n pairs (channels
+  2i, 2i+1 inside the group) is rotated by the angle pos * base^(-i/n), pos the
+  token's coordinate on that axis, base 10000.  It is applied to q and k of the
+  neighbourhood branch only; the far field (pooled tokens, no position) uses the
+  unrotated q and the pooled unrotated K and V.
 
 Parity status: every function is pinned (tests/test_oracle_tile3d.py): g = 1
 and g = 0 special cases, a tile grid of at most 2 per dimension (local equals
-dense attention), one pooling cell (global equals mean of V).
+dense attention), one pooling cell (global equals mean of V); the rotary
+embedding by hand-worked rotations, norm preservation, the identity at the
+origin and the invariance of rotated dot products under a common shift of
+both positions.
 """
 from __future__ import annotations
 
@@ -99,9 +111,40 @@ def global_attention(q, kbar, vbar, rows=None):
     return out
 
 
-def gated_head(q, k, v, F, Hh, Ww, tile=(4, 4, 4), radius=1, cell=(2, 16, 16), gate=0.55, rows=None):
-    """O = g * local + (1 - g) * global for one head (RoPeSLR page)."""
-    loc = local_attention(q, k, v, F, Hh, Ww, tile, radius, rows)
+def rope_split(d: int) -> tuple[int, int, int]:
+    """Channel pairs of the (frame, height, width) groups of the rotary embedding."""
+    pairs = d // 2
+    n_hw = pairs // 3
+    return pairs - 2 * n_hw, n_hw, n_hw
+
+
+def rope_3d(x, F, Hh, Ww, base: float = 10000.0):
+    """The 3-D rotary embedding of one head's rows x [F*Hh*Ww, d] in raster order.
+
+    Pair i of an axis group with n pairs is rotated by pos * base^(-i/n), pos the
+    token's coordinate on that axis: (a, b) -> (a cos - b sin, a sin + b cos).
+    """
+    n, d = x.shape
+    f, h, w = np.meshgrid(np.arange(F), np.arange(Hh), np.arange(Ww), indexing="ij")
+    pos = [f.reshape(-1).astype(np.float64), h.reshape(-1).astype(np.float64), w.reshape(-1).astype(np.float64)]
+    out = np.array(x, dtype=np.float64, copy=True)
+    c0 = 0
+    for axis, n_pairs in enumerate(rope_split(d)):
+        for i in range(n_pairs):
+            ang = pos[axis] * base ** (-i / n_pairs)
+            a, b = x[:, c0 + 2 * i], x[:, c0 + 2 * i + 1]
+            out[:, c0 + 2 * i] = a * np.cos(ang) - b * np.sin(ang)
+            out[:, c0 + 2 * i + 1] = a * np.sin(ang) + b * np.cos(ang)
+        c0 += 2 * n_pairs
+    return out
+
+
+def gated_head(q, k, v, F, Hh, Ww, tile=(4, 4, 4), radius=1, cell=(2, 16, 16), gate=0.55, rows=None,
+               rope: bool = False):
+    """O = g * local + (1 - g) * global for one head (RoPeSLR page); with ``rope`` the
+    neighbourhood branch sees rotated q and k."""
+    ql, kl = (rope_3d(q, F, Hh, Ww), rope_3d(k, F, Hh, Ww)) if rope else (q, k)
+    loc = local_attention(ql, kl, v, F, Hh, Ww, tile, radius, rows)
     kbar, vbar = far_field(k, v, F, Hh, Ww, cell)
     glob = global_attention(q, kbar, vbar, rows)
     return dict(local=loc, glob=glob, kbar=kbar, vbar=vbar, o=gate * loc + (1.0 - gate) * glob)

@@ -70,3 +70,69 @@ def test_local_neighbourhood_brute_force():
         p = np.exp(lg - lg.max())
         p /= p.sum()
         np.testing.assert_allclose(loc[t], p @ v[keys], rtol=1e-12, atol=1e-13)
+
+
+# ---------------------------------------------------------------- rotary embedding
+
+def test_rope_split_of_the_head_sizes():
+    assert tile3d.rope_split(128) == (22, 21, 21)       # 44 + 42 + 42 channels
+    assert tile3d.rope_split(64) == (12, 10, 10)
+
+
+def test_rope_hand_rotations():
+    # d = 12: 6 pairs -> frame 2, height 2, width 2 pairs; pair 0 of a group has angle = pos
+    F, Hh, Ww, d = 2, 3, 4, 12
+    x = np.zeros((F * Hh * Ww, d))
+    t = (1 * Hh + 2) * Ww + 3                      # token (f, h, w) = (1, 2, 3)
+    x[t, 0] = 1.0                                 # frame pair 0 (channels 0, 1): (1, 0)
+    x[t, 2] = 1.0                                 # frame pair 1 (channels 2, 3): (1, 0), angle 10000^(-1/2)
+    x[t, 4] = 2.0                                 # height pair 0 (channels 4, 5): (2, 1)
+    x[t, 5] = 1.0
+    x[t, 9] = -1.0                                # width pair 0 (channels 8, 9): (0, -1)
+    r = tile3d.rope_3d(x, F, Hh, Ww)
+    # frame pair 0 rotated by 1
+    assert np.allclose(r[t, 0:2], [math.cos(1.0), math.sin(1.0)], atol=1e-15)
+    # frame pair 1: f = 1 times 10000^(-1/2) = 0.01
+    assert np.allclose(r[t, 2:4], [math.cos(0.01), math.sin(0.01)], atol=1e-15)
+    # height pair 0 = (2, 1), angle 2
+    a, b = 2.0, 1.0
+    assert np.allclose(r[t, 4:6], [a * math.cos(2) - b * math.sin(2), a * math.sin(2) + b * math.cos(2)], atol=1e-14)
+    # width pair 0 = channels 8, 9 = (0, -1), angle 3
+    assert np.allclose(r[t, 8:10], [math.sin(3.0), -math.cos(3.0)], atol=1e-14)
+
+
+def test_rope_identity_at_origin_and_norm_preserved():
+    q, _, _ = _qkv(11, 2 * 8 * 8, 64)
+    r = tile3d.rope_3d(q, 2, 8, 8)
+    assert np.allclose(r[0], q[0], atol=0)        # token (0, 0, 0) is not rotated
+    pair_norm = lambda x: x[:, 0::2] ** 2 + x[:, 1::2] ** 2  # noqa: E731
+    assert np.allclose(pair_norm(r), pair_norm(q), rtol=1e-12, atol=1e-12)
+
+
+def test_rope_dot_products_depend_on_relative_position_only():
+    # the same q at (1, 2, 3) and k at (0, 5, 1), and both shifted by (2, 1, 4): equal dot products
+    F, Hh, Ww, d = 4, 8, 8, 128
+    rng = np.random.default_rng(12)
+    qv, kv = rng.standard_normal(d), rng.standard_normal(d)
+    tok = lambda f, h, w: (f * Hh + h) * Ww + w  # noqa: E731
+    x = np.zeros((F * Hh * Ww, d))
+    y = np.zeros((F * Hh * Ww, d))
+    x[tok(1, 2, 3)] = qv
+    x[tok(3, 3, 7)] = qv
+    y[tok(0, 5, 1)] = kv
+    y[tok(2, 6, 5)] = kv
+    rq, rk = tile3d.rope_3d(x, F, Hh, Ww), tile3d.rope_3d(y, F, Hh, Ww)
+    a = rq[tok(1, 2, 3)] @ rk[tok(0, 5, 1)]
+    b = rq[tok(3, 3, 7)] @ rk[tok(2, 6, 5)]
+    assert abs(a - b) < 1e-10 * (1 + abs(a))
+    assert abs(a - qv @ kv) > 1e-3                 # and the rotation did change it
+
+
+def test_gated_head_with_rope_rotates_the_local_branch_only():
+    F, Hh, Ww, d = 4, 8, 8, 32
+    q, k, v = _qkv(13, F * Hh * Ww, d)
+    r = tile3d.gated_head(q, k, v, F, Hh, Ww, cell=(2, 4, 4), gate=0.55, rope=True)
+    loc = tile3d.local_attention(tile3d.rope_3d(q, F, Hh, Ww), tile3d.rope_3d(k, F, Hh, Ww), v, F, Hh, Ww)
+    kb, vb = tile3d.far_field(k, v, F, Hh, Ww, (2, 4, 4))
+    glob = tile3d.global_attention(q, kb, vb)
+    assert np.allclose(r["o"], 0.55 * loc + 0.45 * glob, rtol=1e-12, atol=1e-12)
