@@ -28,9 +28,11 @@ Readings:
   and width groups take floor(P/3) pairs each and the frame group the rest
   (d = 128: 44, 42, 42 channels) -- and pair i of a group of n pairs (channels
   2i, 2i+1 inside the group) is rotated by the angle pos * base^(-i/n), pos the
-  token's coordinate on that axis, base 10000.  It is applied to q and k of the
-  neighbourhood branch only; the far field (pooled tokens, no position) uses the
-  unrotated q and the pooled unrotated K and V.
+  token's coordinate on that axis, base 10000.  As in a video transformer that
+  rotates q and k at the start of its attention block, the rotation is applied
+  to q and k before both branches: the neighbourhood sees rotated q and k, and
+  the far field pools the rotated K (and V as it is).  With ``rope=False`` q and
+  k are taken as given (rotated upstream, or not at all).
 
 Parity status: every function is pinned (tests/test_oracle_tile3d.py): g = 1
 and g = 0 special cases, a tile grid of at most 2 per dimension (local equals
@@ -141,10 +143,11 @@ def rope_3d(x, F, Hh, Ww, base: float = 10000.0):
 
 def gated_head(q, k, v, F, Hh, Ww, tile=(4, 4, 4), radius=1, cell=(2, 16, 16), gate=0.55, rows=None,
                rope: bool = False):
-    """O = g * local + (1 - g) * global for one head (RoPeSLR page); with ``rope`` the
-    neighbourhood branch sees rotated q and k."""
-    ql, kl = (rope_3d(q, F, Hh, Ww), rope_3d(k, F, Hh, Ww)) if rope else (q, k)
-    loc = local_attention(ql, kl, v, F, Hh, Ww, tile, radius, rows)
+    """O = g * local + (1 - g) * global for one head (RoPeSLR page); with ``rope`` q and
+    k are first rotated by the 3-D rotary embedding."""
+    if rope:
+        q, k = rope_3d(q, F, Hh, Ww), rope_3d(k, F, Hh, Ww)
+    loc = local_attention(q, k, v, F, Hh, Ww, tile, radius, rows)
     kbar, vbar = far_field(k, v, F, Hh, Ww, cell)
     glob = global_attention(q, kbar, vbar, rows)
     return dict(local=loc, glob=glob, kbar=kbar, vbar=vbar, o=gate * loc + (1.0 - gate) * glob)

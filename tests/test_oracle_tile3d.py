@@ -128,11 +128,13 @@ def test_rope_dot_products_depend_on_relative_position_only():
     assert abs(a - qv @ kv) > 1e-3                 # and the rotation did change it
 
 
-def test_gated_head_with_rope_rotates_the_local_branch_only():
+def test_gated_head_with_rope_equals_rotating_q_and_k_first():
     F, Hh, Ww, d = 4, 8, 8, 32
     q, k, v = _qkv(13, F * Hh * Ww, d)
     r = tile3d.gated_head(q, k, v, F, Hh, Ww, cell=(2, 4, 4), gate=0.55, rope=True)
-    loc = tile3d.local_attention(tile3d.rope_3d(q, F, Hh, Ww), tile3d.rope_3d(k, F, Hh, Ww), v, F, Hh, Ww)
-    kb, vb = tile3d.far_field(k, v, F, Hh, Ww, (2, 4, 4))
-    glob = tile3d.global_attention(q, kb, vb)
-    assert np.allclose(r["o"], 0.55 * loc + 0.45 * glob, rtol=1e-12, atol=1e-12)
+    qr, kr = tile3d.rope_3d(q, F, Hh, Ww), tile3d.rope_3d(k, F, Hh, Ww)
+    ref = tile3d.gated_head(qr, kr, v, F, Hh, Ww, cell=(2, 4, 4), gate=0.55)
+    assert np.allclose(r["o"], ref["o"], rtol=1e-12, atol=1e-12)
+    # the far field pools the rotated keys
+    kb, _ = tile3d.far_field(kr, v, F, Hh, Ww, (2, 4, 4))
+    assert np.allclose(r["kbar"], kb)
