@@ -98,7 +98,8 @@ def config_dict(w, phi="elu1"):
     else:
         desc = (f"{w.name}: gated tile neighbourhood + far field B={w.batch} H={w.heads} d={w.d} "
                 f"{w.frames}x{w.fh}x{w.fw}={w.n_pad} tokens, 4x4x4 tiles, 3x3x3 tile neighbourhood, "
-                f"64 far tokens from {w.cell[0]}x{w.cell[1]}x{w.cell[2]} cells, gate {w.gate}")
+                f"64 far tokens from {w.cell[0]}x{w.cell[1]}x{w.cell[2]} cells, gate {w.gate}"
+                + (", 3-D RoPE on q and k" if w.rope else ""))
     bytes_in = w.n_pad * w.d * 2 * w.heads * w.batch
     return {
         "workload": desc,
@@ -276,9 +277,14 @@ def cpu_oracle_sample(w, q, k, v, wp, rows_per_head=256, heads=12, phi="elu1"):
         for h in range(heads):
             qh, kh, vh = (f64(x[0, h]) for x in (q, k, v))
             t0 = time.perf_counter()
+            if w.rope:      # the rotation covers every token whatever the sample
+                qh, kh = otile.rope_3d(qh, w.frames, w.fh, w.fw), otile.rope_3d(kh, w.frames, w.fh, w.fw)
+            t1 = time.perf_counter()
             otile.gated_head(qh, kh, vh, w.frames, w.fh, w.fw, w.tile, w.radius, w.cell, w.gate, rows=toks)
-            per_rows += time.perf_counter() - t0
-        what = (f"gated_head (far-field pooling in full) for {rows_per_head * 64} of {w.n_pad} query tokens")
+            fixed += t1 - t0
+            per_rows += time.perf_counter() - t1
+        what = ((f"rope_3d of q and k in full, then " if w.rope else "")
+                + f"gated_head (far-field pooling in full) for {rows_per_head * 64} of {w.n_pad} query tokens")
     per_head = fixed / heads + (per_rows / heads) * (nb / rows_per_head)
     total_ms = per_head * w.heads * w.batch * 1e3
     desc = (f"{heads} of {w.heads} heads: {what}; extrapolated linearly to {w.heads} heads x {nb} blocks "
@@ -307,7 +313,7 @@ class Runner:
         if w.mode == "lvsa":
             self.masks = [slr.lvsa_mask(w.frames, w.lvsa_C, w.lvsa_W, s) for s in w.lvsa_steps]
         elif w.mode == "tile3d":
-            self.masks = [slr.tile3d_mask(w.frames, w.fh, w.fw, w.radius, w.cell, w.gate)]
+            self.masks = [slr.tile3d_mask(w.frames, w.fh, w.fw, w.radius, w.cell, w.gate, rope=w.rope)]
 
     def call(self, i=0, o=None, q=None, k=None, v=None, wp=None, ws=None):
         slr, w = self.slr, self.w

@@ -61,7 +61,7 @@ class SlrMaskDesc(ctypes.Structure):
     _fields_ = [("kind", ctypes.c_int), ("T", ctypes.c_int), ("C", ctypes.c_int), ("W", ctypes.c_int),
                 ("step", ctypes.c_int), ("F", ctypes.c_int), ("Hh", ctypes.c_int), ("Ww", ctypes.c_int),
                 ("tile", ctypes.c_int * 3), ("radius", ctypes.c_int), ("cell", ctypes.c_int * 3),
-                ("gate", ctypes.c_float)]
+                ("gate", ctypes.c_float), ("rope", ctypes.c_int)]
 
 
 class SlrFracs(ctypes.Structure):
@@ -142,9 +142,11 @@ def lvsa_mask(T: int, C: int, W: int, step: int) -> SlrMaskDesc:
     return m
 
 
-def tile3d_mask(F: int, Hh: int, Ww: int, radius: int = 1, cell=(2, 16, 16), gate: float = 0.55) -> SlrMaskDesc:
+def tile3d_mask(F: int, Hh: int, Ww: int, radius: int = 1, cell=(2, 16, 16), gate: float = 0.55,
+                rope: bool = False) -> SlrMaskDesc:
     m = SlrMaskDesc()
     m.kind, m.F, m.Hh, m.Ww, m.radius, m.gate = SLR_MASK_TILE3D, F, Hh, Ww, radius, gate
+    m.rope = 1 if rope else 0
     m.tile[:] = [4, 4, 4]
     m.cell[:] = list(cell)
     return m

@@ -31,9 +31,16 @@ cudaError_t launch_pool_means(const void* q, const void* k, void* qsplit, void* 
                               int BH, int d, SeqShape s, cudaStream_t st);
 
 // Far-field K/V: means over cells of (cf, ch, cw) tokens of the raster (F, Hh, Ww),
-// bf16 [BH][ncells][d], cells in raster order of the cell grid.
-cudaError_t launch_far_pool(const void* k, const void* v, void* kf, void* vf, int BH, int d,
-                            int F, int Hh, int Ww, int cf, int ch, int cw, cudaStream_t st);
+// bf16 [BH][ncells][d], cells in raster order of the cell grid.  With rope = 1 the same
+// pass writes q and k rotated by the 3-D rotary embedding (base 10000, channel pairs
+// split frame / height / width) into qr and kr (bf16 [BH][F*Hh*Ww][d]), and the K means
+// are those of the rotated keys; the cos / sin table of a cell takes
+// far_pool_table_bytes(d, cf, ch, cw) of shared memory, at most kFarPoolTableMax.
+constexpr size_t kFarPoolTableMax = 48 * 1024;
+size_t far_pool_table_bytes(int d, int cf, int ch, int cw);
+cudaError_t launch_far_pool(const void* q, const void* k, const void* v, void* qr, void* kr, void* kf, void* vf,
+                            int BH, int d, int F, int Hh, int Ww, int cf, int ch, int cw, int rope,
+                            cudaStream_t st);
 
 // ------------------------------------------------------------ classification (k_classify.cu)
 // Row stride (entries) of the logit-key matrix: Nb rounded up to 128.

@@ -178,12 +178,14 @@ struct FrameWs {
   int32_t* list_cnt;
   int cap;
   void *kf, *vf;
+  void *qr, *kr;     // rotated q and k (TILE3D with rope)
 };
 
 slr_status check_mask(const slr_mask_desc* m, const Shape& sh) {
   if (!m) return SLR_ERR_ARG;
   if (m->kind == SLR_MASK_LVSA) {
     if (m->T != sh.n_seg || m->W < 0 || m->step < 0 || m->C <= 2 * m->W + 1) return SLR_ERR_ARG;
+    if (m->rope != 0) return SLR_ERR_UNSUPPORTED;
     return SLR_OK;
   }
   if (m->kind == SLR_MASK_TILE3D) {
@@ -197,6 +199,8 @@ slr_status check_mask(const slr_mask_desc* m, const Shape& sh) {
     if (c[0] < 1 || c[1] < 1 || c[2] < 1 || m->F % c[0] || m->Hh % c[1] || m->Ww % c[2]) return SLR_ERR_ARG;
     if ((m->F / c[0]) * (m->Hh / c[1]) * (m->Ww / c[2]) != 64) return SLR_ERR_UNSUPPORTED;
     if (!(m->gate >= 0.f && m->gate <= 1.f)) return SLR_ERR_ARG;
+    if (m->rope != 0 && m->rope != 1) return SLR_ERR_ARG;
+    if (m->rope && far_pool_table_bytes(sh.d, c[0], c[1], c[2]) > kFarPoolTableMax) return SLR_ERR_UNSUPPORTED;
     return SLR_OK;
   }
   return SLR_ERR_ARG;
@@ -206,6 +210,7 @@ void plan_frame(Carve& c, const Shape& sh, const slr_mask_desc* m, FrameWs& w) {
   w.status = c.take<int>(64);
   w.sets = w.set_cnt = nullptr;
   w.kf = w.vf = nullptr;
+  w.qr = w.kr = nullptr;
   if (m->kind == SLR_MASK_LVSA) {
     const LvsaGlobals g = lvsa_globals(m->T, m->C, m->W, m->step);
     const int win = (2 * m->W + 1 < m->T - g.count) ? 2 * m->W + 1 : m->T - g.count;
@@ -222,6 +227,10 @@ void plan_frame(Carve& c, const Shape& sh, const slr_mask_desc* m, FrameWs& w) {
     w.kf = c.take<__nv_bfloat16>((size_t)sh.BH * 64 * sh.d);
     w.vf = c.take<__nv_bfloat16>((size_t)sh.BH * 64 * sh.d);
     w.set_cap = 0;
+    if (m->rope) {
+      w.qr = c.take<__nv_bfloat16>((size_t)sh.BH * sh.n_pad * sh.d);
+      w.kr = c.take<__nv_bfloat16>((size_t)sh.BH * sh.n_pad * sh.d);
+    }
   }
   w.list = c.take<uint32_t>((size_t)sh.npairs * w.cap);
   w.list_cnt = c.take<int32_t>((size_t)sh.npairs);
@@ -584,7 +593,14 @@ slr_status slr_frame_mask_attn(const void* q, const void* k, const void* v, cons
   } else {
     la.mode = kListTile3d;
     la.TF = m->F / 4; la.TH = m->Hh / 4; la.TW = m->Ww / 4; la.radius = m->radius;
-    SLR_LAUNCH(kKFarPool, s, launch_far_pool(k, v, w.kf, w.vf, sh.BH, sh.d, m->F, m->Hh, m->Ww, m->cell[0], m->cell[1], m->cell[2], s));
+    // with the rotary embedding the pooling pass also rotates q and k (once, for both
+    // branches: the far field pools the rotated K) and the attention reads the rotated copies
+    SLR_LAUNCH(kKFarPool, s, launch_far_pool(q, k, v, w.qr, w.kr, w.kf, w.vf, sh.BH, sh.d, m->F, m->Hh, m->Ww,
+                                             m->cell[0], m->cell[1], m->cell[2], m->rope, s));
+    if (m->rope) {
+      a.q = w.qr;
+      a.k = w.kr;
+    }
     a.tile3d = 1; a.F = m->F; a.Hh = m->Hh; a.Ww = m->Ww;
     a.gated = 1; a.gate = m->gate; a.kf = w.kf; a.vf = w.vf;
   }

@@ -78,6 +78,9 @@ typedef struct {
     int radius;               /* Chebyshev tile radius of the local neighbourhood (1 -> 3x3x3)  */
     int cell[3];              /* far-field pooling cell; the cell grid must hold 64 cells       */
     float gate;               /* g in g*local + (1-g)*global                                    */
+    int rope;                 /* TILE3D: 1 = rotate q and k by the 3-D rotary embedding first
+                                 (aixinbiao page: the neighbourhood branch encodes relative
+                                 position with RoPE); 0 = take q and k as given.  LVSA: 0    */
 } slr_mask_desc;
 
 /* Percentile parameters for the classifying calls (params of slr_workspace_bytes). */
@@ -190,7 +193,13 @@ slr_status slr_sparse_linear_attn(const void* q, const void* k, const void* v, c
  *    within Chebyshev tile distance `radius` of its own tile (clipped at the
  *    borders), and separately, with its own softmax, 64 far-field tokens made
  *    by mean-pooling K and V over `cell`-sized cells; the output is
- *    gate*local + (1-gate)*far.
+ *    gate*local + (1-gate)*far.  With rope = 1, q and k are first rotated by the
+ *    3-D rotary embedding (base 10000; with P = d/2 channel pairs, the height and
+ *    width axes take floor(P/3) consecutive pairs each after the frame axis's
+ *    P - 2 floor(P/3); pair i of an axis group of n pairs turns by
+ *    coordinate * 10000^(-i/n)), for both branches: the far field pools the
+ *    rotated K.  The rotated q and k are kept in the workspace (2 x B*H*N_pad*d
+ *    bf16 more).
  *   out  bf16 [B][H][N_pad][d] device, written
  */
 slr_status slr_frame_mask_attn(const void* q, const void* k, const void* v, const slr_seq* seq,

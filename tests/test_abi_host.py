@@ -87,6 +87,14 @@ def test_workspace_bytes(lib):
     assert slr.slr_workspace_bytes(slr.SLR_OP_FRAME_MASK, slr.make_seq(1, 16, 128, 1, 32768, 32768), t3) > 0
     t3bad = slr.tile3d_mask(8, 64, 64, cell=(2, 8, 8))      # 256 cells, not 64
     assert slr.slr_workspace_bytes(slr.SLR_OP_FRAME_MASK, slr.make_seq(1, 16, 128, 1, 32768, 32768), t3bad) == 0
+    # with the rotary embedding the rotated q and k (bf16 [B*H][N][d] each) live in the workspace too
+    seq3 = slr.make_seq(1, 16, 128, 1, 32768, 32768)
+    plain = slr.slr_workspace_bytes(slr.SLR_OP_FRAME_MASK, seq3, t3)
+    roped = slr.slr_workspace_bytes(slr.SLR_OP_FRAME_MASK, seq3, slr.tile3d_mask(8, 64, 64, rope=True))
+    assert roped - plain >= 2 * 16 * 32768 * 128 * 2
+    t3bad = slr.tile3d_mask(8, 64, 64)
+    t3bad.rope = 2
+    assert slr.slr_workspace_bytes(slr.SLR_OP_FRAME_MASK, seq3, t3bad) == 0
 
 
 def test_block_sparse_list_cap_clamps_without_overflow(lib):
@@ -133,6 +141,11 @@ def test_invalid_arguments_rejected_before_cuda(lib):
     m = slr.lvsa_mask(5, 6, 1, 0)
     assert lib.slr_frame_mask_attn(fake, fake, fake, ctypes.byref(seq), ctypes.byref(m), fake, ws, 1 << 20,
                                    None) == slr.SLR_ERR_ARG
+    # the rotary embedding is defined for the tile neighbourhood only
+    m = slr.lvsa_mask(1, 6, 1, 0)
+    m.rope = 1
+    assert lib.slr_frame_mask_attn(fake, fake, fake, ctypes.byref(seq), ctypes.byref(m), fake, ws, 1 << 20,
+                                   None) == slr.SLR_ERR_UNSUPPORTED
     # linear branch needs a mask
     assert lib.slr_linear_marginal(fake, fake, fake, ctypes.byref(seq), None, 0, None, fake, ws, 1 << 20,
                                    None) == slr.SLR_ERR_ARG

@@ -3,7 +3,8 @@
 121-frame workload on 64 sampled query blocks of every head, including the
 first and last blocks and frame tails) and the gated tile neighbourhood + far
 field (small grids in full, including an odd tile count and two batch entries,
-and the 8x64x64 workload on sampled tokens)."""
+and the 8x64x64 workload on sampled tokens), with and without the 3-D rotary
+embedding of q and k."""
 import numpy as np
 import pytest
 import torch
@@ -116,3 +117,60 @@ def test_tile3d_workload_sampled():
         outs.append(to64(out[0, h])[toks])
         refs.append(r["o"][toks])
     assert_close(np.concatenate(outs), np.concatenate(refs), "tile3d workload")
+
+
+@pytest.mark.parametrize("F,Hh,Ww,cell,d", [(8, 16, 16, (2, 4, 4), 128), (12, 8, 8, (3, 2, 2), 64),
+                                            (4, 16, 32, (1, 4, 8), 128)])
+def test_tile3d_rope_small_full(F, Hh, Ww, cell, d):
+    H, n = 2, F * Hh * Ww
+    q, k, v = make_inputs(1, H, d, 1, n, n, seed=57)
+    seq = slr.make_seq(1, H, d, 1, n, n)
+    out = slr.slr_frame_mask_attn(cuda(q), cuda(k), cuda(v), seq,
+                                  slr.tile3d_mask(F, Hh, Ww, 1, cell, 0.55, rope=True))
+    status_ok()
+    for h in range(H):
+        r = otile.gated_head(to64(q[0, h]), to64(k[0, h]), to64(v[0, h]), F, Hh, Ww, cell=cell, gate=0.55,
+                             rope=True)
+        assert_close(to64(out[0, h]), r["o"], f"tile3d rope head {h}")
+    # the rotation changes the result: the same call without it is far from the rotated oracle
+    plain = slr.slr_frame_mask_attn(cuda(q), cuda(k), cuda(v), seq, slr.tile3d_mask(F, Hh, Ww, 1, cell, 0.55))
+    r = otile.gated_head(to64(q[0, 0]), to64(k[0, 0]), to64(v[0, 0]), F, Hh, Ww, cell=cell, gate=0.55, rope=True)
+    assert np.abs(to64(plain[0, 0]) - r["o"]).max() > 0.05
+
+
+def test_tile3d_rope_two_batch_entries():
+    B, H, d, F, Hh, Ww, cell = 2, 2, 128, 8, 8, 16, (2, 2, 4)
+    n = F * Hh * Ww
+    q, k, v = make_inputs(B, H, d, 1, n, n, seed=59)
+    seq = slr.make_seq(B, H, d, 1, n, n)
+    out = slr.slr_frame_mask_attn(cuda(q), cuda(k), cuda(v), seq,
+                                  slr.tile3d_mask(F, Hh, Ww, 1, cell, 0.3, rope=True))
+    status_ok()
+    outs, refs = [], []
+    for b in range(B):
+        for h in range(H):
+            r = otile.gated_head(to64(q[b, h]), to64(k[b, h]), to64(v[b, h]), F, Hh, Ww, cell=cell, gate=0.3,
+                                 rope=True)
+            outs.append(to64(out[b, h]))
+            refs.append(r["o"])
+    assert_close(np.concatenate(outs), np.concatenate(refs), "tile3d rope B=2")
+
+
+def test_tile3d_rope_workload_sampled():
+    w = workloads.ROPESLR
+    q, k, v = workloads.make_qkv(w)
+    seq = slr.make_seq(1, w.heads, w.d, 1, w.seg_len, w.seg_stride)
+    out = slr.slr_frame_mask_attn(cuda(q), cuda(k), cuda(v), seq,
+                                  slr.tile3d_mask(w.frames, w.fh, w.fw, w.radius, w.cell, w.gate, rope=True))
+    status_ok()
+    rng = np.random.default_rng(7)
+    # sampled tokens plus the raster's corners, where the height and width angles are largest
+    toks = sorted(set(rng.choice(w.n_pad, 300, replace=False).tolist()
+                      + [0, w.fw - 1, w.fh * w.fw - 1, w.n_pad - 1]))
+    outs, refs = [], []
+    for h in range(1, w.heads, 4):
+        r = otile.gated_head(to64(q[0, h]), to64(k[0, h]), to64(v[0, h]), w.frames, w.fh, w.fw,
+                             w.tile, w.radius, w.cell, w.gate, rows=toks, rope=True)
+        outs.append(to64(out[0, h])[toks])
+        refs.append(r["o"][toks])
+    assert_close(np.concatenate(outs), np.concatenate(refs), "tile3d rope workload")

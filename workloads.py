@@ -61,6 +61,7 @@ class Workload:
     radius: int = 1
     cell: tuple = (2, 16, 16)
     gate: float = 0.55
+    rope: bool = False  # 3-D rotary embedding of q and k before both branches
     batch: int = 1
 
     @property
@@ -91,7 +92,7 @@ LVSA = Workload("lvsa", 4, heads=12, d=128, frames=121, fh=30, fw=52,
                 seg_stride=1600, n_seg=121, seg_len=1560, mode="lvsa", correlated=False,
                 lvsa_C=21, lvsa_W=3, lvsa_steps=(0, 1, 2, 3))
 ROPESLR = Workload("ropeslr", 5, heads=16, d=128, frames=8, fh=64, fw=64,
-                   seg_stride=32768, n_seg=1, seg_len=32768, mode="tile3d", correlated=False)
+                   seg_stride=32768, n_seg=1, seg_len=32768, mode="tile3d", correlated=False, rope=True)
 
 ALL = (TINY, WAN, HUNYUAN, LVSA, ROPESLR)
 BY_NAME = {w.name: w for w in ALL}
