@@ -19,6 +19,9 @@ three source write-ups define:
                        aixinbiao blog page, section "稀疏邻域加低秩远场": a
                        3x3x3 local neighbourhood, a pooled low-rank far field
                        and the gate g*local + (1-g)*global.
+* ``oracle.sta``    -- the 3-D sliding tile attention mask of VORTA (arXiv
+                       2505.18809), as described on the zhaoyang97 paper-notes
+                       page, section "方法详解", design 1, and attention over it.
 
 It shares no code with the CUDA library and imports nothing from it.  Only the
 tests, ``__graft_entry__.smoke()`` and the CPU-baseline leg of ``bench.py`` may
@@ -28,4 +31,4 @@ All arithmetic is fp64.  Parity status of every function is listed in each
 module's header; every function is pinned by a test in ``tests/test_oracle_*.py``
 against closed forms, special cases, library routines or hand-worked examples.
 """
-from . import sla, lvsa, tile3d  # noqa: F401
+from . import sla, lvsa, tile3d, sta  # noqa: F401
