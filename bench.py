@@ -95,6 +95,10 @@ def config_dict(w, phi="elu1"):
         desc = (f"{w.name}: LVSA frame mask B={w.batch} H={w.heads} d={w.d} T={w.frames} frames of "
                 f"{w.fh}x{w.fw}={w.seg_len} tokens padded to {w.seg_stride} (N={w.n_pad}), C={w.lvsa_C}, "
                 f"W={w.lvsa_W}, denoising steps {list(w.lvsa_steps)} in turn, no linear branch")
+    elif w.mode == "sta":
+        desc = (f"{w.name}: sliding tile attention B={w.batch} H={w.heads} d={w.d} "
+                f"{w.frames}x{w.fh}x{w.fw}={w.n_pad} tokens, 4x4x4 tiles, window "
+                f"{w.window[0]}x{w.window[1]}x{w.window[2]} tokens")
     else:
         desc = (f"{w.name}: gated tile neighbourhood + far field B={w.batch} H={w.heads} d={w.d} "
                 f"{w.frames}x{w.fh}x{w.fw}={w.n_pad} tokens, 4x4x4 tiles, 3x3x3 tile neighbourhood, "
@@ -143,6 +147,16 @@ def tile3d_flops(w):
     pairs = extent_sum(tf) * extent_sum(th) * extent_sum(tw)
     far = tf * th * tw
     return 4.0 * 64 * 64 * w.d * (pairs + far) * w.heads * w.batch, pairs
+
+
+def sta_flops(w):
+    """FLOPs of one sliding tile call: 4*64*64*d per (query tile, key tile) pair of the
+    clipped window, the tile radius on each axis being (window / 4 - 1) / 2."""
+    def extent_sum(n_tiles, r):
+        return sum(min(t + r, n_tiles - 1) - max(t - r, 0) + 1 for t in range(n_tiles))
+    rad = [(x // 4 - 1) // 2 for x in w.window]
+    pairs = (extent_sum(w.frames // 4, rad[0]) * extent_sum(w.fh // 4, rad[1]) * extent_sum(w.fw // 4, rad[2]))
+    return 4.0 * 64 * 64 * w.d * pairs * w.heads * w.batch, pairs
 
 
 # ------------------------------------------------------------------ clocks
@@ -230,6 +244,7 @@ def cpu_oracle_sample(w, q, k, v, wp, rows_per_head=256, heads=12, phi="elu1"):
     """
     from oracle import lvsa as olvsa
     from oracle import sla as osla
+    from oracle import sta as osta
     from oracle import tile3d as otile
     heads = min(heads, w.heads)
     nb = w.n_blocks
@@ -272,6 +287,14 @@ def cpu_oracle_sample(w, q, k, v, wp, rows_per_head=256, heads=12, phi="elu1"):
             per_rows += t2 - t1
         what = (f"attention_sets in full, then frame_mask_attention for {rows_per_head} of {nb} query "
                 f"blocks (step {step})")
+    elif w.mode == "sta":
+        toks = sorted(rng.choice(w.n_pad, rows_per_head * 64, replace=False).tolist())
+        for h in range(heads):
+            qh, kh, vh = (f64(x[0, h]) for x in (q, k, v))
+            t0 = time.perf_counter()
+            osta.sliding_tile_attention(qh, kh, vh, w.frames, w.fh, w.fw, window=w.window, rows=toks)
+            per_rows += time.perf_counter() - t0
+        what = f"sliding_tile_attention for {rows_per_head * 64} of {w.n_pad} query tokens"
     else:
         toks = sorted(rng.choice(w.n_pad, rows_per_head * 64, replace=False).tolist())
         for h in range(heads):
@@ -314,6 +337,8 @@ class Runner:
             self.masks = [slr.lvsa_mask(w.frames, w.lvsa_C, w.lvsa_W, s) for s in w.lvsa_steps]
         elif w.mode == "tile3d":
             self.masks = [slr.tile3d_mask(w.frames, w.fh, w.fw, w.radius, w.cell, w.gate, rope=w.rope)]
+        elif w.mode == "sta":
+            self.masks = [slr.sta_mask(w.frames, w.fh, w.fw, w.window)]
 
     def call(self, i=0, o=None, q=None, k=None, v=None, wp=None, ws=None):
         slr, w = self.slr, self.w
@@ -376,6 +401,9 @@ class Runner:
             fl = [lvsa_flops(w, slr.slr_lvsa_attention_sets(w.frames, w.lvsa_C, w.lvsa_W, s)) for s in w.lvsa_steps]
             f = sum(fl) / len(fl)
             return f, f, {"computed_tflop_per_step": [x / 1e12 for x in fl]}
+        if w.mode == "sta":
+            f, pairs = sta_flops(w)
+            return f, f, {"tile_pairs_per_head": pairs, "computed_tflop": f / 1e12}
         f, pairs = tile3d_flops(w)
         return f, f, {"local_tile_pairs_per_head": pairs, "computed_tflop": f / 1e12}
 

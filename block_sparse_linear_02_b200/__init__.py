@@ -31,6 +31,7 @@ SLR_PHI_ELU1 = 0
 SLR_PHI_SOFTMAX = 1
 SLR_MASK_LVSA = 1
 SLR_MASK_TILE3D = 2
+SLR_MASK_STA = 3
 
 SLR_OP_POOL_CLASSIFY = 1
 SLR_OP_BLOCK_SPARSE = 2
@@ -61,7 +62,7 @@ class SlrMaskDesc(ctypes.Structure):
     _fields_ = [("kind", ctypes.c_int), ("T", ctypes.c_int), ("C", ctypes.c_int), ("W", ctypes.c_int),
                 ("step", ctypes.c_int), ("F", ctypes.c_int), ("Hh", ctypes.c_int), ("Ww", ctypes.c_int),
                 ("tile", ctypes.c_int * 3), ("radius", ctypes.c_int), ("cell", ctypes.c_int * 3),
-                ("gate", ctypes.c_float), ("rope", ctypes.c_int)]
+                ("gate", ctypes.c_float), ("rope", ctypes.c_int), ("window", ctypes.c_int * 3)]
 
 
 class SlrFracs(ctypes.Structure):
@@ -149,6 +150,15 @@ def tile3d_mask(F: int, Hh: int, Ww: int, radius: int = 1, cell=(2, 16, 16), gat
     m.rope = 1 if rope else 0
     m.tile[:] = [4, 4, 4]
     m.cell[:] = list(cell)
+    return m
+
+
+def sta_mask(F: int, Hh: int, Ww: int, window=(12, 12, 12)) -> SlrMaskDesc:
+    """Sliding tile attention over 4x4x4 tiles; window in tokens per axis (odd multiples of 4)."""
+    m = SlrMaskDesc()
+    m.kind, m.F, m.Hh, m.Ww = SLR_MASK_STA, F, Hh, Ww
+    m.tile[:] = [4, 4, 4]
+    m.window[:] = list(window)
     return m
 
 

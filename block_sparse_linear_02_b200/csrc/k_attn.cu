@@ -898,7 +898,8 @@ cudaError_t launch_variant(const AttnArgs& a, const CUtensorMap* maps, const Att
 
 template <int D>
 cudaError_t launch_d(const AttnArgs& a, const CUtensorMap* maps, const AttnKParams& kp, cudaStream_t st) {
-  if (a.tile3d) return launch_variant<D, true, true, false>(a, maps, kp, st);
+  if (a.tile3d) return a.gated ? launch_variant<D, true, true, false>(a, maps, kp, st)
+                               : launch_variant<D, true, false, false>(a, maps, kp, st);
   if (a.Hs) return launch_variant<D, false, false, true>(a, maps, kp, st);
   return launch_variant<D, false, false, false>(a, maps, kp, st);
 }
@@ -907,7 +908,6 @@ cudaError_t launch_d(const AttnArgs& a, const CUtensorMap* maps, const AttnKPara
 
 cudaError_t launch_attention(const AttnArgs& a, cudaStream_t st) {
   const int D = a.d;
-  if (a.tile3d && !a.gated) return cudaErrorInvalidValue;
   CUtensorMap maps[7];
   const uint64_t rowb = (uint64_t)D * 2;
   if (a.tile3d) {

@@ -61,11 +61,11 @@ pair_lists_kernel(const ListArgs a) {
       }
     } else {  // tile neighbourhood
       const int tf = qb % a.TF, tw = (qb / a.TF) % a.TW, th = (qb / a.TF) / a.TW;
-      const int side = 2 * a.radius + 1;
-      for (int e = threadIdx.x; e < side * side * side; e += blockDim.x) {
-        const int nf = tf + e / (side * side) - a.radius;
-        const int nh = th + (e / side) % side - a.radius;
-        const int nw = tw + e % side - a.radius;
+      const int sf = 2 * a.rad[0] + 1, sh = 2 * a.rad[1] + 1, sw = 2 * a.rad[2] + 1;
+      for (int e = threadIdx.x; e < sf * sh * sw; e += blockDim.x) {
+        const int nf = tf + e / (sh * sw) - a.rad[0];
+        const int nh = th + (e / sw) % sh - a.rad[1];
+        const int nw = tw + e % sw - a.rad[2];
         if (nf < 0 || nf >= a.TF || nh < 0 || nh >= a.TH || nw < 0 || nw >= a.TW) continue;
         const int j = (nh * a.TW + nw) * a.TF + nf;
         atomicOr(&bm[half][j >> 5], 1u << (j & 31));

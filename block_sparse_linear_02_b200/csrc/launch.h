@@ -84,8 +84,10 @@ struct ListArgs {
   const int32_t* sets;     // [T][set_cap]
   const int32_t* set_cnt;  // [T]
   int set_cap, blocks_per_frame;
-  // tile3d: tile grid (TF, TH, TW), tile id = (th*TW + tw)*TF + tf
-  int TF, TH, TW, radius;
+  // tile3d: tile grid (TF, TH, TW), tile id = (th*TW + tw)*TF + tf; a key tile is a
+  // neighbour when it is within rad[0] / rad[1] / rad[2] tiles on the frame / height /
+  // width axis
+  int TF, TH, TW, rad[3];
   SeqShape s;              // token layout (valid-key counts of linear blocks)
   uint32_t* list;          // [heads][n_pairs][cap]
   int32_t* list_cnt;       // [heads][n_pairs]

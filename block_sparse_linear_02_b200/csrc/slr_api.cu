@@ -203,7 +203,24 @@ slr_status check_mask(const slr_mask_desc* m, const Shape& sh) {
     if (m->rope && far_pool_table_bytes(sh.d, c[0], c[1], c[2]) > kFarPoolTableMax) return SLR_ERR_UNSUPPORTED;
     return SLR_OK;
   }
+  if (m->kind == SLR_MASK_STA) {
+    if (sh.n_seg != 1 || sh.seg_len != sh.seg_stride) return SLR_ERR_UNSUPPORTED;
+    if (m->F < 1 || m->Hh < 1 || m->Ww < 1) return SLR_ERR_ARG;
+    if ((long long)m->F * m->Hh * m->Ww != sh.n_pad) return SLR_ERR_ARG;
+    if (m->tile[0] != 4 || m->tile[1] != 4 || m->tile[2] != 4) return SLR_ERR_UNSUPPORTED;
+    if (m->F % 4 || m->Hh % 4 || m->Ww % 4) return SLR_ERR_UNSUPPORTED;
+    for (int a = 0; a < 3; ++a)            // an odd number of whole tiles
+      if (m->window[a] < 4 || m->window[a] % 4 || (m->window[a] / 4) % 2 == 0) return SLR_ERR_ARG;
+    if (m->rope != 0) return SLR_ERR_UNSUPPORTED;
+    return SLR_OK;
+  }
   return SLR_ERR_ARG;
+}
+
+// Tile radius per axis of a TILE3D or STA mask: a window of (2r+1) tiles keeps the tiles
+// whose centres lie within half a window of the query tile's centre, i.e. within r tiles
+void mask_radii(const slr_mask_desc* m, int rad[3]) {
+  for (int a = 0; a < 3; ++a) rad[a] = m->kind == SLR_MASK_STA ? (m->window[a] / 4 - 1) / 2 : m->radius;
 }
 
 void plan_frame(Carve& c, const Shape& sh, const slr_mask_desc* m, FrameWs& w) {
@@ -221,12 +238,15 @@ void plan_frame(Carve& c, const Shape& sh, const slr_mask_desc* m, FrameWs& w) {
     const long long cap = 2LL * w.set_cap * bpf;
     w.cap = cap < sh.nb ? (int)cap : sh.nb;
   } else {
-    const int side = 2 * m->radius + 1;
-    const long long cap = 2LL * side * side * side;
+    int rad[3];
+    mask_radii(m, rad);
+    const long long cap = 2LL * (2 * rad[0] + 1) * (2 * rad[1] + 1) * (2 * rad[2] + 1);
     w.cap = cap < sh.nb ? (int)cap : sh.nb;
-    w.kf = c.take<__nv_bfloat16>((size_t)sh.BH * 64 * sh.d);
-    w.vf = c.take<__nv_bfloat16>((size_t)sh.BH * 64 * sh.d);
     w.set_cap = 0;
+    if (m->kind == SLR_MASK_TILE3D) {
+      w.kf = c.take<__nv_bfloat16>((size_t)sh.BH * 64 * sh.d);
+      w.vf = c.take<__nv_bfloat16>((size_t)sh.BH * 64 * sh.d);
+    }
     if (m->rope) {
       w.qr = c.take<__nv_bfloat16>((size_t)sh.BH * sh.n_pad * sh.d);
       w.kr = c.take<__nv_bfloat16>((size_t)sh.BH * sh.n_pad * sh.d);
@@ -592,7 +612,11 @@ slr_status slr_frame_mask_attn(const void* q, const void* k, const void* v, cons
     la.blocks_per_frame = sh.seg_stride / kBlock;
   } else {
     la.mode = kListTile3d;
-    la.TF = m->F / 4; la.TH = m->Hh / 4; la.TW = m->Ww / 4; la.radius = m->radius;
+    la.TF = m->F / 4; la.TH = m->Hh / 4; la.TW = m->Ww / 4;
+    mask_radii(m, la.rad);
+    a.tile3d = 1; a.F = m->F; a.Hh = m->Hh; a.Ww = m->Ww;
+  }
+  if (m->kind == SLR_MASK_TILE3D) {
     // with the rotary embedding the pooling pass also rotates q and k (once, for both
     // branches: the far field pools the rotated K) and the attention reads the rotated copies
     SLR_LAUNCH(kKFarPool, s, launch_far_pool(q, k, v, w.qr, w.kr, w.kf, w.vf, sh.BH, sh.d, m->F, m->Hh, m->Ww,
@@ -601,7 +625,6 @@ slr_status slr_frame_mask_attn(const void* q, const void* k, const void* v, cons
       a.q = w.qr;
       a.k = w.kr;
     }
-    a.tile3d = 1; a.F = m->F; a.Hh = m->Hh; a.Ww = m->Ww;
     a.gated = 1; a.gate = m->gate; a.kf = w.kf; a.vf = w.vf;
   }
   SLR_LAUNCH(kKLists, s, launch_pair_lists(la, 1, s));

@@ -68,11 +68,13 @@ typedef struct {
 /* External block masks for slr_frame_mask_attn. */
 #define SLR_MASK_LVSA   1
 #define SLR_MASK_TILE3D 2
+#define SLR_MASK_STA    3
 typedef struct {
-    int kind;                 /* SLR_MASK_LVSA or SLR_MASK_TILE3D                              */
+    int kind;                 /* SLR_MASK_LVSA, SLR_MASK_TILE3D or SLR_MASK_STA                */
     /* LVSA (rainbus page, "方法步骤详情" steps 1-6): frames are the n_seg segments, T == n_seg */
     int T, C, W, step;        /* frames, budget, window half-width, denoising step s            */
-    /* TILE3D (aixinbiao page): raster (F, Hh, Ww) tokens, F*Hh*Ww == N_pad, n_seg == 1         */
+    /* TILE3D (aixinbiao page) and STA (VORTA page): raster (F, Hh, Ww) tokens,
+       F*Hh*Ww == N_pad, n_seg == 1                                                            */
     int F, Hh, Ww;
     int tile[3];              /* token tile, must be {4, 4, 4}                                  */
     int radius;               /* Chebyshev tile radius of the local neighbourhood (1 -> 3x3x3)  */
@@ -80,7 +82,9 @@ typedef struct {
     float gate;               /* g in g*local + (1-g)*global                                    */
     int rope;                 /* TILE3D: 1 = rotate q and k by the 3-D rotary embedding first
                                  (aixinbiao page: the neighbourhood branch encodes relative
-                                 position with RoPE); 0 = take q and k as given.  LVSA: 0    */
+                                 position with RoPE); 0 = take q and k as given.  LVSA, STA: 0 */
+    int window[3];            /* STA: window (frame, height, width) in tokens, each an odd
+                                 multiple of the tile size 4                                   */
 } slr_mask_desc;
 
 /* Percentile parameters for the classifying calls (params of slr_workspace_bytes). */
@@ -200,6 +204,13 @@ slr_status slr_sparse_linear_attn(const void* q, const void* k, const void* v, c
  *    coordinate * 10000^(-i/n)), for both branches: the far field pools the
  *    rotated K.  The rotated q and k are kept in the workspace (2 x B*H*N_pad*d
  *    bf16 more).
+ *  SLR_MASK_STA (VORTA paper notes, section 方法详解, design 1: 3-D sliding tile
+ *    attention, M = {j in (tau(i) - w, tau(i) + w]} with tau the centre of the
+ *    position's tile): q, k, v are in raster (F, Hh, Ww) order, tiles are
+ *    4x4x4 tokens, and a query attends, with one softmax, every key whose tile
+ *    centre lies, on every axis, in (tau(query) - W/2, tau(query) + W/2] for
+ *    that axis's window W = `window` -- with W = (2r+1)*4 the tiles within r
+ *    tiles of the query's tile, clipped at the borders.  No far field, no gate.
  *   out  bf16 [B][H][N_pad][d] device, written
  */
 slr_status slr_frame_mask_attn(const void* q, const void* k, const void* v, const slr_seq* seq,

@@ -95,6 +95,14 @@ def test_workspace_bytes(lib):
     t3bad = slr.tile3d_mask(8, 64, 64)
     t3bad.rope = 2
     assert slr.slr_workspace_bytes(slr.SLR_OP_FRAME_MASK, seq3, t3bad) == 0
+    # sliding tile mask: lists only (no far field); windows must be odd numbers of 4-token tiles
+    sta = slr.slr_workspace_bytes(slr.SLR_OP_FRAME_MASK, seq3, slr.sta_mask(8, 64, 64, (12, 20, 28)))
+    assert 0 < sta < plain
+    for bad in [(12, 16, 12), (10, 12, 12), (0, 12, 12), (12, 12, -4)]:
+        assert slr.slr_workspace_bytes(slr.SLR_OP_FRAME_MASK, seq3, slr.sta_mask(8, 64, 64, bad)) == 0
+    sta_rope = slr.sta_mask(8, 64, 64)
+    sta_rope.rope = 1
+    assert slr.slr_workspace_bytes(slr.SLR_OP_FRAME_MASK, seq3, sta_rope) == 0
 
 
 def test_block_sparse_list_cap_clamps_without_overflow(lib):

@@ -4,7 +4,8 @@
 first and last blocks and frame tails) and the gated tile neighbourhood + far
 field (small grids in full, including an odd tile count and two batch entries,
 and the 8x64x64 workload on sampled tokens), with and without the 3-D rotary
-embedding of q and k."""
+embedding of q and k; the sliding tile mask (small grids in full with windows of
+one to seven tiles per axis, two batch entries, 8x64x64 on sampled tokens)."""
 import numpy as np
 import pytest
 import torch
@@ -13,6 +14,7 @@ import block_sparse_linear_02_b200 as slr
 import workloads
 from gpu_common import assert_close, cuda, make_inputs, rows_of_blocks, status_ok, to64, valid_np
 from oracle import lvsa as olvsa
+from oracle import sta as osta
 from oracle import tile3d as otile
 
 pytestmark = pytest.mark.gpu
@@ -174,3 +176,50 @@ def test_tile3d_rope_workload_sampled():
         outs.append(to64(out[0, h])[toks])
         refs.append(r["o"][toks])
     assert_close(np.concatenate(outs), np.concatenate(refs), "tile3d rope workload")
+
+
+@pytest.mark.parametrize("F,Hh,Ww,window,d", [(8, 16, 16, (12, 12, 12), 128), (8, 16, 24, (4, 20, 12), 128),
+                                              (12, 8, 32, (20, 4, 28), 64), (4, 16, 16, (4, 4, 4), 128)])
+def test_sta_small_full(F, Hh, Ww, window, d):
+    H, n = 2, F * Hh * Ww
+    q, k, v = make_inputs(1, H, d, 1, n, n, seed=61)
+    seq = slr.make_seq(1, H, d, 1, n, n)
+    out = slr.slr_frame_mask_attn(cuda(q), cuda(k), cuda(v), seq, slr.sta_mask(F, Hh, Ww, window))
+    status_ok()
+    for h in range(H):
+        ref = osta.sliding_tile_attention(to64(q[0, h]), to64(k[0, h]), to64(v[0, h]), F, Hh, Ww, window=window)
+        assert_close(to64(out[0, h]), ref, f"sta head {h}")
+
+
+def test_sta_two_batch_entries():
+    B, H, d, F, Hh, Ww, window = 2, 2, 128, 8, 8, 16, (12, 4, 20)
+    n = F * Hh * Ww
+    q, k, v = make_inputs(B, H, d, 1, n, n, seed=63)
+    seq = slr.make_seq(B, H, d, 1, n, n)
+    out = slr.slr_frame_mask_attn(cuda(q), cuda(k), cuda(v), seq, slr.sta_mask(F, Hh, Ww, window))
+    status_ok()
+    outs, refs = [], []
+    for b in range(B):
+        for h in range(H):
+            refs.append(osta.sliding_tile_attention(to64(q[b, h]), to64(k[b, h]), to64(v[b, h]), F, Hh, Ww,
+                                                    window=window))
+            outs.append(to64(out[b, h]))
+    assert_close(np.concatenate(outs), np.concatenate(refs), "sta B=2")
+
+
+def test_sta_workload_sampled():
+    w = workloads.STA
+    q, k, v = workloads.make_qkv(w)
+    seq = slr.make_seq(1, w.heads, w.d, 1, w.seg_len, w.seg_stride)
+    out = slr.slr_frame_mask_attn(cuda(q), cuda(k), cuda(v), seq, slr.sta_mask(w.frames, w.fh, w.fw, w.window))
+    status_ok()
+    rng = np.random.default_rng(9)
+    toks = sorted(set(rng.choice(w.n_pad, 300, replace=False).tolist()
+                      + [0, w.fw - 1, w.fh * w.fw - 1, w.n_pad - 1]))
+    outs, refs = [], []
+    for h in range(0, w.heads, 5):
+        ref = osta.sliding_tile_attention(to64(q[0, h]), to64(k[0, h]), to64(v[0, h]), w.frames, w.fh, w.fw,
+                                          window=w.window, rows=toks)
+        outs.append(to64(out[0, h])[toks])
+        refs.append(ref[toks])
+    assert_close(np.concatenate(outs), np.concatenate(refs), "sta workload")

@@ -48,7 +48,7 @@ class Workload:
     seg_stride: int     # padded tokens per segment
     n_seg: int          # number of padded segments
     seg_len: int        # valid tokens per segment
-    mode: str           # "sla", "lvsa" or "tile3d"
+    mode: str           # "sla", "lvsa", "tile3d" or "sta"
     correlated: bool
     crit_frac: float = 0.05
     negl_frac: float = 0.10
@@ -62,6 +62,8 @@ class Workload:
     cell: tuple = (2, 16, 16)
     gate: float = 0.55
     rope: bool = False  # 3-D rotary embedding of q and k before both branches
+    # STA: sliding tile window in tokens per axis (odd multiples of the 4-token tile)
+    window: tuple = (12, 12, 12)
     batch: int = 1
 
     @property
@@ -94,7 +96,12 @@ LVSA = Workload("lvsa", 4, heads=12, d=128, frames=121, fh=30, fw=52,
 ROPESLR = Workload("ropeslr", 5, heads=16, d=128, frames=8, fh=64, fw=64,
                    seg_stride=32768, n_seg=1, seg_len=32768, mode="tile3d", correlated=False, rope=True)
 
-ALL = (TINY, WAN, HUNYUAN, LVSA, ROPESLR)
+# VORTA's local heads: 3-D sliding tile attention on the same 8x64x64 latent, windows of
+# 3 x 7 x 5 tiles (12 x 28 x 20 tokens, ~14 % of the keys); not one of the quoted configurations
+STA = Workload("sta", 6, heads=16, d=128, frames=8, fh=64, fw=64,
+               seg_stride=32768, n_seg=1, seg_len=32768, mode="sta", correlated=False, window=(12, 28, 20))
+
+ALL = (TINY, WAN, HUNYUAN, LVSA, ROPESLR, STA)
 BY_NAME = {w.name: w for w in ALL}
 
 
