@@ -356,17 +356,12 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
               for (int c = 0; c < L::kChunks; ++c)
                 tma_load_3d(dst + c * L::kTile, is_v ? &tmX2 : &tmX1, &slot_full[slot], c * 64, 0, ti.bh);
             } else {
+              // key block kb: rows [64 kb, 64 kb + 64) (in the tile layout K and V are in
+              // tile-major order, so a 4x4x4 tile is one such block)
               const int kb = ti.list ? (int)(ti.list[2 * j + b] & 0xFFFFu) : 2 * j + b;
               const CUtensorMap* tm = is_v ? &tmV : &tmK;
-              if (TILE) {
-                int tf, th, tw;
-                tile_coords(kb, p.TF, p.TW, tf, th, tw);
-                for (int c = 0; c < L::kChunks; ++c)
-                  tma_load_5d(dst + c * L::kTile, tm, &slot_full[slot], c * 64, tw * 4, th * 4, tf * 4, ti.bh);
-              } else {
-                for (int c = 0; c < L::kChunks; ++c)
-                  tma_load_3d(dst + c * L::kTile, tm, &slot_full[slot], c * 64, kb * 64, ti.bh);
-              }
+              for (int c = 0; c < L::kChunks; ++c)
+                tma_load_3d(dst + c * L::kTile, tm, &slot_full[slot], c * 64, kb * 64, ti.bh);
             }
           }
           rel_kind[slot] = is_v ? 0 : 3;
@@ -911,12 +906,16 @@ cudaError_t launch_attention(const AttnArgs& a, cudaStream_t st) {
   CUtensorMap maps[7];
   const uint64_t rowb = (uint64_t)D * 2;
   if (a.tile3d) {
+    // Q (raster) by 4x4x4 tile boxes; K and V arrive in tile-major order, a tile = 64 rows
     const uint64_t dims[5] = {(uint64_t)D, (uint64_t)a.Ww, (uint64_t)a.Hh, (uint64_t)a.F, (uint64_t)a.BH};
     const uint64_t strides[4] = {rowb, rowb * a.Ww, rowb * a.Ww * a.Hh, rowb * a.Ww * a.Hh * a.F};
     const uint32_t box[5] = {64, 4, 4, 4, 1};
     if (!make_tile_map(&maps[0], a.q, 5, dims, strides, box)) return cudaErrorInvalidValue;
-    if (!make_tile_map(&maps[1], a.k, 5, dims, strides, box)) return cudaErrorInvalidValue;
-    if (!make_tile_map(&maps[2], a.v, 5, dims, strides, box)) return cudaErrorInvalidValue;
+    const uint64_t kdims[3] = {(uint64_t)D, (uint64_t)a.s.n_pad, (uint64_t)a.BH};
+    const uint64_t kstrides[2] = {rowb, rowb * a.s.n_pad};
+    const uint32_t boxkv[3] = {64, 64, 1};
+    if (!make_tile_map(&maps[1], a.k, 3, kdims, kstrides, boxkv)) return cudaErrorInvalidValue;
+    if (!make_tile_map(&maps[2], a.v, 3, kdims, kstrides, boxkv)) return cudaErrorInvalidValue;
   } else {
     const uint64_t dims[3] = {(uint64_t)D, (uint64_t)a.s.n_pad, (uint64_t)a.BH};
     const uint64_t strides[2] = {rowb, rowb * a.s.n_pad};

@@ -14,7 +14,8 @@
 // over cells of (cf, ch, cw) raster tokens (aixinbiao page: K and V compressed
 // by token mean-pooling into a small low-rank set), rounded to bf16 because
 // they are tensor-core operands of the attention kernel; with the 3-D rotary
-// embedding the same pass rotates Q and K, so each is read from HBM once.
+// embedding the same pass rotates Q and K, so each is read from HBM once.  The same pass
+// writes K (rotated) and V in the tile-major order the tile attention kernel loads.
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 
@@ -107,6 +108,34 @@ pool_means_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
   }
 }
 
+// Row of raster token (f, h, w) in the tile-major order of 4x4x4 tiles: tile
+// (th * TW + tw) * TF + tf, and inside it (f % 4, h % 4, w % 4) in raster order.
+__device__ __forceinline__ int tile_major_row(int f, int h, int w, int TF, int TW) {
+  return ((((h >> 2) * TW + (w >> 2)) * TF + (f >> 2)) << 6) + ((f & 3) << 4) + ((h & 3) << 2) + (w & 3);
+}
+
+// K and V of a raster (F, Hh, Ww) sequence copied into tile-major order, so that the
+// attention kernel loads each 4x4x4 key tile as 64 consecutive rows (one 16 KB box per
+// 64 channels) instead of gathering 16 runs of 4 tokens.  One CTA per (raster row (f, h),
+// head, tensor); the row's Ww tokens are 4-token runs of Ww / 4 tiles.
+template <int D>
+__global__ void __launch_bounds__(256)
+tile_major_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
+                  __nv_bfloat16* __restrict__ kt, __nv_bfloat16* __restrict__ vt, int F, int Hh, int Ww) {
+  constexpr int kCPR = D / 8;              // 16-byte chunks per token
+  const int row = blockIdx.x, bh = blockIdx.y;
+  const int f = row / Hh, h = row % Hh;
+  const size_t n = (size_t)F * Hh * Ww;
+  const __nv_bfloat16* x = (blockIdx.z == 0 ? k : v) + ((size_t)bh * n + (size_t)row * Ww) * D;
+  __nv_bfloat16* y = (blockIdx.z == 0 ? kt : vt) + (size_t)bh * n * D;
+  const int TF = F >> 2, TW = Ww >> 2;
+  for (int i = threadIdx.x; i < Ww * kCPR; i += blockDim.x) {
+    const int w = i / kCPR, c = i % kCPR;
+    const uint4 u = __ldg(reinterpret_cast<const uint4*>(x + (size_t)w * D + c * 8));
+    *reinterpret_cast<uint4*>(y + (size_t)tile_major_row(f, h, w, TF, TW) * D + c * 8) = u;
+  }
+}
+
 // Channel pairs of the 3-D rotary embedding: with P = D/2 pairs the frame axis takes the
 // first P - 2 floor(P/3), the height and width axes floor(P/3) each.
 template <int D>
@@ -125,7 +154,7 @@ template <int D>
 __global__ void __launch_bounds__(128)
 far_pool_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
                 const __nv_bfloat16* __restrict__ v, __nv_bfloat16* __restrict__ qr,
-                __nv_bfloat16* __restrict__ kr, __nv_bfloat16* __restrict__ kf,
+                __nv_bfloat16* __restrict__ kt, __nv_bfloat16* __restrict__ vt, __nv_bfloat16* __restrict__ kf,
                 __nv_bfloat16* __restrict__ vf, int F, int Hh, int Ww, int cf, int ch, int cw, int rope) {
   using R = RopeSplit<D>;
   constexpr int kCPR = D / 8;              // 16-byte chunks per row = 4 channel pairs each
@@ -139,7 +168,9 @@ far_pool_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __rest
   const __nv_bfloat16* x = (z == 0 ? k : z == 1 ? v : q) + (size_t)bh * n * D;
   const bool rotate = rope && z != 1;
   const bool pool = z != 2;
-  __nv_bfloat16* xr = rotate ? (z == 0 ? kr : qr) + (size_t)bh * n * D : nullptr;
+  // K and V (rotated K) leave in tile-major order, rotated Q in raster order
+  __nv_bfloat16* xo = (z == 0 ? kt : z == 1 ? vt : qr) + (size_t)bh * n * D;
+  const int TF = F >> 2, TW = Ww >> 2;
   const int chunk = threadIdx.x % kCPR, rg = threadIdx.x / kCPR;
   const int per_cell = cf * ch * cw;
   int tab_off[4] = {0, 0, 0, 0}, tab_stride[4] = {0, 0, 0, 0}, axis[4] = {0, 0, 0, 0};
@@ -175,11 +206,13 @@ far_pool_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __rest
   for (int r0 = rg; r0 < per_cell; r0 += kBatch * kRG) {
     uint4 u[kBatch];
     int pos[kBatch][3];
-    size_t off[kBatch];
+    size_t off[kBatch], dst[kBatch];
     #pragma unroll
     for (int b = 0; b < kBatch; ++b) {
       pos[b][0] = df; pos[b][1] = dh; pos[b][2] = dw;
-      off[b] = (((size_t)(c_f * cf + df) * Hh + (c_h * ch + dh)) * Ww + (c_w * cw + dw)) * D + chunk * 8;
+      const int f = c_f * cf + df, h = c_h * ch + dh, w = c_w * cw + dw;
+      off[b] = (((size_t)f * Hh + h) * Ww + w) * D + chunk * 8;
+      dst[b] = z == 2 ? off[b] : (size_t)tile_major_row(f, h, w, TF, TW) * D + chunk * 8;
       u[b] = r0 + b * kRG < per_cell ? __ldg(reinterpret_cast<const uint4*>(x + off[b])) : make_uint4(0, 0, 0, 0);
       dw += kRG;
       while (dw >= cw) {
@@ -190,15 +223,17 @@ far_pool_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __rest
     #pragma unroll
     for (int b = 0; b < kBatch; ++b) {
       uint32_t w[4] = {u[b].x, u[b].y, u[b].z, u[b].w};
-      if (rotate && r0 + b * kRG < per_cell) {
-        #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int pe = axis[e] == 0 ? pos[b][0] : axis[e] == 1 ? pos[b][1] : pos[b][2];
-          const float2 c = cs_tab[tab_off[e] + pe * tab_stride[e]];
-          const float a = bf16_lo(w[e]), bb = bf16_hi(w[e]);
-          w[e] = pack_bf16(a * c.x - bb * c.y, a * c.y + bb * c.x);
+      if (r0 + b * kRG < per_cell) {
+        if (rotate) {
+          #pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int pe = axis[e] == 0 ? pos[b][0] : axis[e] == 1 ? pos[b][1] : pos[b][2];
+            const float2 c = cs_tab[tab_off[e] + pe * tab_stride[e]];
+            const float a = bf16_lo(w[e]), bb = bf16_hi(w[e]);
+            w[e] = pack_bf16(a * c.x - bb * c.y, a * c.y + bb * c.x);
+          }
         }
-        *reinterpret_cast<uint4*>(xr + off[b]) = make_uint4(w[0], w[1], w[2], w[3]);
+        *reinterpret_cast<uint4*>(xo + dst[b]) = make_uint4(w[0], w[1], w[2], w[3]);
       }
       if (pool) {                          // rows past the cell loaded as zeros
         #pragma unroll
@@ -242,8 +277,20 @@ size_t far_pool_table_bytes(int d, int cf, int ch, int cw) {
   return (size_t)((size_t)cf * (pairs - 2 * hw) + ((size_t)ch + cw) * hw) * sizeof(float2);
 }
 
-cudaError_t launch_far_pool(const void* q, const void* k, const void* v, void* qr, void* kr, void* kf, void* vf,
-                            int BH, int d, int F, int Hh, int Ww, int cf, int ch, int cw, int rope,
+cudaError_t launch_tile_major(const void* k, const void* v, void* kt, void* vt, int BH, int d, int F, int Hh,
+                              int Ww, cudaStream_t st) {
+  dim3 grid(F * Hh, BH, 2);
+  auto* k_ = static_cast<const __nv_bfloat16*>(k);
+  auto* v_ = static_cast<const __nv_bfloat16*>(v);
+  auto* kt_ = static_cast<__nv_bfloat16*>(kt);
+  auto* vt_ = static_cast<__nv_bfloat16*>(vt);
+  if (d == 128) tile_major_kernel<128><<<grid, 256, 0, st>>>(k_, v_, kt_, vt_, F, Hh, Ww);
+  else tile_major_kernel<64><<<grid, 256, 0, st>>>(k_, v_, kt_, vt_, F, Hh, Ww);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_far_pool(const void* q, const void* k, const void* v, void* qr, void* kt, void* vt, void* kf,
+                            void* vf, int BH, int d, int F, int Hh, int Ww, int cf, int ch, int cw, int rope,
                             cudaStream_t st) {
   const int ncells = (F / cf) * (Hh / ch) * (Ww / cw);
   dim3 grid(ncells, BH, rope ? 3 : 2);
@@ -253,13 +300,14 @@ cudaError_t launch_far_pool(const void* q, const void* k, const void* v, void* q
   auto* k_ = static_cast<const __nv_bfloat16*>(k);
   auto* v_ = static_cast<const __nv_bfloat16*>(v);
   auto* qr_ = static_cast<__nv_bfloat16*>(qr);
-  auto* kr_ = static_cast<__nv_bfloat16*>(kr);
+  auto* kt_ = static_cast<__nv_bfloat16*>(kt);
+  auto* vt_ = static_cast<__nv_bfloat16*>(vt);
   auto* kf_ = static_cast<__nv_bfloat16*>(kf);
   auto* vf_ = static_cast<__nv_bfloat16*>(vf);
   if (d == 128)
-    far_pool_kernel<128><<<grid, 128, tab, st>>>(q_, k_, v_, qr_, kr_, kf_, vf_, F, Hh, Ww, cf, ch, cw, rope);
+    far_pool_kernel<128><<<grid, 128, tab, st>>>(q_, k_, v_, qr_, kt_, vt_, kf_, vf_, F, Hh, Ww, cf, ch, cw, rope);
   else
-    far_pool_kernel<64><<<grid, 128, tab, st>>>(q_, k_, v_, qr_, kr_, kf_, vf_, F, Hh, Ww, cf, ch, cw, rope);
+    far_pool_kernel<64><<<grid, 128, tab, st>>>(q_, k_, v_, qr_, kt_, vt_, kf_, vf_, F, Hh, Ww, cf, ch, cw, rope);
   return cudaGetLastError();
 }
 

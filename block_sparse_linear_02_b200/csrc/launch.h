@@ -30,16 +30,23 @@ bool make_tile_map(CUtensorMap* map, const void* base, int rank, const uint64_t*
 cudaError_t launch_pool_means(const void* q, const void* k, void* qsplit, void* ksplit, void* phi_q, int phi,
                               int BH, int d, SeqShape s, cudaStream_t st);
 
+// Tile-major order of a raster (F, Hh, Ww) sequence (F, Hh, Ww multiples of 4): 4x4x4
+// tile (th * TW + tw) * TF + tf takes rows [64 tile, 64 tile + 64), its tokens in (f, h, w)
+// raster order inside the tile.  launch_tile_major copies K and V into that order
+// (bf16 [BH][F*Hh*Ww][d] each).
+cudaError_t launch_tile_major(const void* k, const void* v, void* kt, void* vt, int BH, int d, int F, int Hh,
+                              int Ww, cudaStream_t st);
+
 // Far-field K/V: means over cells of (cf, ch, cw) tokens of the raster (F, Hh, Ww),
-// bf16 [BH][ncells][d], cells in raster order of the cell grid.  With rope = 1 the same
-// pass writes q and k rotated by the 3-D rotary embedding (base 10000, channel pairs
-// split frame / height / width) into qr and kr (bf16 [BH][F*Hh*Ww][d]), and the K means
-// are those of the rotated keys; the cos / sin table of a cell takes
-// far_pool_table_bytes(d, cf, ch, cw) of shared memory, at most kFarPoolTableMax.
+// bf16 [BH][ncells][d], cells in raster order of the cell grid.  The same pass writes K and
+// V in tile-major order into kt and vt.  With rope = 1 it also writes q rotated by the 3-D
+// rotary embedding (base 10000, channel pairs split frame / height / width) into qr (raster
+// order), K is rotated before it is written and pooled, and the cos / sin table of a cell
+// takes far_pool_table_bytes(d, cf, ch, cw) of shared memory, at most kFarPoolTableMax.
 constexpr size_t kFarPoolTableMax = 48 * 1024;
 size_t far_pool_table_bytes(int d, int cf, int ch, int cw);
-cudaError_t launch_far_pool(const void* q, const void* k, const void* v, void* qr, void* kr, void* kf, void* vf,
-                            int BH, int d, int F, int Hh, int Ww, int cf, int ch, int cw, int rope,
+cudaError_t launch_far_pool(const void* q, const void* k, const void* v, void* qr, void* kt, void* vt, void* kf,
+                            void* vf, int BH, int d, int F, int Hh, int Ww, int cf, int ch, int cw, int rope,
                             cudaStream_t st);
 
 // ------------------------------------------------------------ classification (k_classify.cu)

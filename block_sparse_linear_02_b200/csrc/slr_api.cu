@@ -178,7 +178,8 @@ struct FrameWs {
   int32_t* list_cnt;
   int cap;
   void *kf, *vf;
-  void *qr, *kr;     // rotated q and k (TILE3D with rope)
+  void* qr;          // rotated q, raster order (TILE3D with rope)
+  void *kt, *vt;     // K (rotated with rope) and V in tile-major order (TILE3D, STA)
 };
 
 slr_status check_mask(const slr_mask_desc* m, const Shape& sh) {
@@ -227,7 +228,7 @@ void plan_frame(Carve& c, const Shape& sh, const slr_mask_desc* m, FrameWs& w) {
   w.status = c.take<int>(64);
   w.sets = w.set_cnt = nullptr;
   w.kf = w.vf = nullptr;
-  w.qr = w.kr = nullptr;
+  w.qr = w.kt = w.vt = nullptr;
   if (m->kind == SLR_MASK_LVSA) {
     const LvsaGlobals g = lvsa_globals(m->T, m->C, m->W, m->step);
     const int win = (2 * m->W + 1 < m->T - g.count) ? 2 * m->W + 1 : m->T - g.count;
@@ -247,10 +248,9 @@ void plan_frame(Carve& c, const Shape& sh, const slr_mask_desc* m, FrameWs& w) {
       w.kf = c.take<__nv_bfloat16>((size_t)sh.BH * 64 * sh.d);
       w.vf = c.take<__nv_bfloat16>((size_t)sh.BH * 64 * sh.d);
     }
-    if (m->rope) {
-      w.qr = c.take<__nv_bfloat16>((size_t)sh.BH * sh.n_pad * sh.d);
-      w.kr = c.take<__nv_bfloat16>((size_t)sh.BH * sh.n_pad * sh.d);
-    }
+    w.kt = c.take<__nv_bfloat16>((size_t)sh.BH * sh.n_pad * sh.d);
+    w.vt = c.take<__nv_bfloat16>((size_t)sh.BH * sh.n_pad * sh.d);
+    if (m->rope) w.qr = c.take<__nv_bfloat16>((size_t)sh.BH * sh.n_pad * sh.d);
   }
   w.list = c.take<uint32_t>((size_t)sh.npairs * w.cap);
   w.list_cnt = c.take<int32_t>((size_t)sh.npairs);
@@ -270,11 +270,11 @@ slr_status ws_check(void* ws, size_t have, size_t need) {
 // ---------------------------------------------------------------- per-kernel profiler
 enum KernelKind {
   kKPool, kKLogits, kKClassify, kKLists, kKKeyStates, kKReduce, kKApply, kKAttention, kKLvsaSets,
-  kKFarPool, kKMaskToM01, kKNumKinds
+  kKFarPool, kKMaskToM01, kKTileMajor, kKNumKinds
 };
 const char* const kKindNames[kKNumKinds] = {
     "pool_means", "logits", "classify", "pair_lists", "key_states", "reduce_states",
-    "linear_apply", "attention", "lvsa_sets", "far_pool", "mask_to_m01"};
+    "linear_apply", "attention", "lvsa_sets", "far_pool", "mask_to_m01", "tile_major"};
 
 struct ProfRec {
   int kind;
@@ -615,16 +615,18 @@ slr_status slr_frame_mask_attn(const void* q, const void* k, const void* v, cons
     la.TF = m->F / 4; la.TH = m->Hh / 4; la.TW = m->Ww / 4;
     mask_radii(m, la.rad);
     a.tile3d = 1; a.F = m->F; a.Hh = m->Hh; a.Ww = m->Ww;
+    // the attention loads every key tile as 64 consecutive rows of tile-major K and V
+    a.k = w.kt;
+    a.v = w.vt;
   }
-  if (m->kind == SLR_MASK_TILE3D) {
-    // with the rotary embedding the pooling pass also rotates q and k (once, for both
-    // branches: the far field pools the rotated K) and the attention reads the rotated copies
-    SLR_LAUNCH(kKFarPool, s, launch_far_pool(q, k, v, w.qr, w.kr, w.kf, w.vf, sh.BH, sh.d, m->F, m->Hh, m->Ww,
-                                             m->cell[0], m->cell[1], m->cell[2], m->rope, s));
-    if (m->rope) {
-      a.q = w.qr;
-      a.k = w.kr;
-    }
+  if (m->kind == SLR_MASK_STA) {
+    SLR_LAUNCH(kKTileMajor, s, launch_tile_major(k, v, w.kt, w.vt, sh.BH, sh.d, m->F, m->Hh, m->Ww, s));
+  } else if (m->kind == SLR_MASK_TILE3D) {
+    // the pooling pass writes tile-major K and V, and with the rotary embedding it also
+    // rotates q and k (once, for both branches: the far field pools the rotated K)
+    SLR_LAUNCH(kKFarPool, s, launch_far_pool(q, k, v, w.qr, w.kt, w.vt, w.kf, w.vf, sh.BH, sh.d, m->F, m->Hh,
+                                             m->Ww, m->cell[0], m->cell[1], m->cell[2], m->rope, s));
+    if (m->rope) a.q = w.qr;
     a.gated = 1; a.gate = m->gate; a.kf = w.kf; a.vf = w.vf;
   }
   SLR_LAUNCH(kKLists, s, launch_pair_lists(la, 1, s));

@@ -202,8 +202,7 @@ slr_status slr_sparse_linear_attn(const void* q, const void* k, const void* v, c
  *    width axes take floor(P/3) consecutive pairs each after the frame axis's
  *    P - 2 floor(P/3); pair i of an axis group of n pairs turns by
  *    coordinate * 10000^(-i/n)), for both branches: the far field pools the
- *    rotated K.  The rotated q and k are kept in the workspace (2 x B*H*N_pad*d
- *    bf16 more).
+ *    rotated K; the rotated q is kept in the workspace (B*H*N_pad*d bf16).
  *  SLR_MASK_STA (VORTA paper notes, section 方法详解, design 1: 3-D sliding tile
  *    attention, M = {j in (tau(i) - w, tau(i) + w]} with tau the centre of the
  *    position's tile): q, k, v are in raster (F, Hh, Ww) order, tiles are
@@ -211,6 +210,9 @@ slr_status slr_sparse_linear_attn(const void* q, const void* k, const void* v, c
  *    centre lies, on every axis, in (tau(query) - W/2, tau(query) + W/2] for
  *    that axis's window W = `window` -- with W = (2r+1)*4 the tiles within r
  *    tiles of the query's tile, clipped at the borders.  No far field, no gate.
+ *  TILE3D and STA keep copies of K (rotated with rope) and V in the workspace in
+ *    tile-major order (2 x B*H*N_pad*d bf16), so that the attention loads each
+ *    4x4x4 key tile as one run of 64 rows; q, k, v and out stay in raster order.
  *   out  bf16 [B][H][N_pad][d] device, written
  */
 slr_status slr_frame_mask_attn(const void* q, const void* k, const void* v, const slr_seq* seq,
