@@ -76,8 +76,9 @@ def measured_traffic(kernel: str, workload: str = "wan"):
     if not os.path.exists(p):
         return None
     with open(p) as f:
-        rec = json.load(f).get(kernel)
-    if not rec or rec.get("workload", "wan") != workload:
+        recs = json.load(f)
+    rec = recs.get(f"{kernel}:{workload}")            # records are keyed kernel:workload
+    if not rec or rec.get("workload") != workload:
         return None
     with open(os.path.join(ROOT, rec["source"]), "rb") as f:
         if hashlib.sha256(f.read()).hexdigest() != rec["sha256"]:

@@ -30,6 +30,7 @@ bool make_tile_map(CUtensorMap* map, const void* base, int rank, const uint64_t*
 cudaError_t launch_pool_means(const void* q, const void* k, void* qsplit, void* ksplit, void* phi_q, int phi,
                               int BH, int d, SeqShape s, cudaStream_t st);
 
+// ------------------------------------------------------------ tile layouts (k_far.cu)
 // Tile-major order of a raster (F, Hh, Ww) sequence (F, Hh, Ww multiples of 4): 4x4x4
 // tile (th * TW + tw) * TF + tf takes rows [64 tile, 64 tile + 64), its tokens in (f, h, w)
 // raster order inside the tile.  launch_tile_major copies K and V into that order
@@ -37,17 +38,19 @@ cudaError_t launch_pool_means(const void* q, const void* k, void* qsplit, void* 
 cudaError_t launch_tile_major(const void* k, const void* v, void* kt, void* vt, int BH, int d, int F, int Hh,
                               int Ww, cudaStream_t st);
 
-// Far-field K/V: means over cells of (cf, ch, cw) tokens of the raster (F, Hh, Ww),
-// bf16 [BH][ncells][d], cells in raster order of the cell grid.  The same pass writes K and
-// V in tile-major order into kt and vt.  With rope = 1 it also writes q rotated by the 3-D
-// rotary embedding (base 10000, channel pairs split frame / height / width) into qr (raster
-// order), K is rotated before it is written and pooled, and the cos / sin table of a cell
-// takes far_pool_table_bytes(d, cf, ch, cw) of shared memory, at most kFarPoolTableMax.
-constexpr size_t kFarPoolTableMax = 48 * 1024;
-size_t far_pool_table_bytes(int d, int cf, int ch, int cw);
-cudaError_t launch_far_pool(const void* q, const void* k, const void* v, void* qr, void* kt, void* vt, void* kf,
-                            void* vf, int BH, int d, int F, int Hh, int Ww, int cf, int ch, int cw, int rope,
-                            cudaStream_t st);
+// The RoPeSLR far-field pass: K and V written in tile-major order into kt and vt, and
+// their means over cells of (cf, ch, cw) tokens into kf and vf (bf16 [BH][ncells][d], cells
+// in raster order of the cell grid), through fp32 row sums in `part`
+// (far_partial_bytes).  With rope = 1, q and k are first rotated by the 3-D rotary
+// embedding (base 10000, channel pairs split frame / height / width; the cos / sin table
+// in `tab`, far_rope_table_bytes) and the rotated q is written, in raster order, into qr.
+// A raster row of Ww tokens passes through shared memory: Ww * d * 2 <= kFarRowBytesMax.
+constexpr size_t kFarRowBytesMax = 96 * 1024;
+size_t far_rope_table_bytes(int d, int F, int Hh, int Ww);
+size_t far_partial_bytes(int BH, int d, int F, int Hh, int Ww, int cw);
+cudaError_t launch_far_field(const void* q, const void* k, const void* v, void* qr, void* kt, void* vt, void* kf,
+                             void* vf, void* tab, void* part, int BH, int d, int F, int Hh, int Ww, int cf, int ch,
+                             int cw, int rope, cudaStream_t st);
 
 // ------------------------------------------------------------ classification (k_classify.cu)
 // Row stride (entries) of the logit-key matrix: Nb rounded up to 128.

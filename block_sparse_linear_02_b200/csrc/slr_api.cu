@@ -180,6 +180,7 @@ struct FrameWs {
   void *kf, *vf;
   void* qr;          // rotated q, raster order (TILE3D with rope)
   void *kt, *vt;     // K (rotated with rope) and V in tile-major order (TILE3D, STA)
+  void *tab, *part;  // TILE3D: RoPE cos / sin table, far-field row sums
 };
 
 slr_status check_mask(const slr_mask_desc* m, const Shape& sh) {
@@ -201,7 +202,7 @@ slr_status check_mask(const slr_mask_desc* m, const Shape& sh) {
     if ((m->F / c[0]) * (m->Hh / c[1]) * (m->Ww / c[2]) != 64) return SLR_ERR_UNSUPPORTED;
     if (!(m->gate >= 0.f && m->gate <= 1.f)) return SLR_ERR_ARG;
     if (m->rope != 0 && m->rope != 1) return SLR_ERR_ARG;
-    if (m->rope && far_pool_table_bytes(sh.d, c[0], c[1], c[2]) > kFarPoolTableMax) return SLR_ERR_UNSUPPORTED;
+    if ((size_t)m->Ww * sh.d * 2 > kFarRowBytesMax) return SLR_ERR_UNSUPPORTED;
     return SLR_OK;
   }
   if (m->kind == SLR_MASK_STA) {
@@ -228,7 +229,7 @@ void plan_frame(Carve& c, const Shape& sh, const slr_mask_desc* m, FrameWs& w) {
   w.status = c.take<int>(64);
   w.sets = w.set_cnt = nullptr;
   w.kf = w.vf = nullptr;
-  w.qr = w.kt = w.vt = nullptr;
+  w.qr = w.kt = w.vt = w.tab = w.part = nullptr;
   if (m->kind == SLR_MASK_LVSA) {
     const LvsaGlobals g = lvsa_globals(m->T, m->C, m->W, m->step);
     const int win = (2 * m->W + 1 < m->T - g.count) ? 2 * m->W + 1 : m->T - g.count;
@@ -247,6 +248,8 @@ void plan_frame(Carve& c, const Shape& sh, const slr_mask_desc* m, FrameWs& w) {
     if (m->kind == SLR_MASK_TILE3D) {
       w.kf = c.take<__nv_bfloat16>((size_t)sh.BH * 64 * sh.d);
       w.vf = c.take<__nv_bfloat16>((size_t)sh.BH * 64 * sh.d);
+      w.part = c.take<uint8_t>(far_partial_bytes(sh.BH, sh.d, m->F, m->Hh, m->Ww, m->cell[2]));
+      if (m->rope) w.tab = c.take<uint8_t>(far_rope_table_bytes(sh.d, m->F, m->Hh, m->Ww));
     }
     w.kt = c.take<__nv_bfloat16>((size_t)sh.BH * sh.n_pad * sh.d);
     w.vt = c.take<__nv_bfloat16>((size_t)sh.BH * sh.n_pad * sh.d);
@@ -624,8 +627,8 @@ slr_status slr_frame_mask_attn(const void* q, const void* k, const void* v, cons
   } else if (m->kind == SLR_MASK_TILE3D) {
     // the pooling pass writes tile-major K and V, and with the rotary embedding it also
     // rotates q and k (once, for both branches: the far field pools the rotated K)
-    SLR_LAUNCH(kKFarPool, s, launch_far_pool(q, k, v, w.qr, w.kt, w.vt, w.kf, w.vf, sh.BH, sh.d, m->F, m->Hh,
-                                             m->Ww, m->cell[0], m->cell[1], m->cell[2], m->rope, s));
+    SLR_LAUNCH(kKFarPool, s, launch_far_field(q, k, v, w.qr, w.kt, w.vt, w.kf, w.vf, w.tab, w.part, sh.BH, sh.d,
+                                              m->F, m->Hh, m->Ww, m->cell[0], m->cell[1], m->cell[2], m->rope, s));
     if (m->rope) a.q = w.qr;
     a.gated = 1; a.gate = m->gate; a.kf = w.kf; a.vf = w.vf;
   }

@@ -210,6 +210,8 @@ slr_status slr_sparse_linear_attn(const void* q, const void* k, const void* v, c
  *    centre lies, on every axis, in (tau(query) - W/2, tau(query) + W/2] for
  *    that axis's window W = `window` -- with W = (2r+1)*4 the tiles within r
  *    tiles of the query's tile, clipped at the borders.  No far field, no gate.
+ *  TILE3D needs Ww * d * 2 <= 96 KB (a raster row of K or V passes through
+ *    shared memory in the far-field pass), else SLR_ERR_UNSUPPORTED.
  *  TILE3D and STA keep copies of K (rotated with rope) and V in the workspace in
  *    tile-major order (2 x B*H*N_pad*d bf16), so that the attention loads each
  *    4x4x4 key tile as one run of 64 rows; q, k, v and out stay in raster order.

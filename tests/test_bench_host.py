@@ -12,11 +12,15 @@ def test_traffic_record_used_only_while_the_source_hash_matches(tmp_path, monkey
     src = tmp_path / "k.cu"
     src.write_text("kernel source\n")
     (tmp_path / "profiles").mkdir()
-    rec = {"attention": {"source": "k.cu", "sha256": hashlib.sha256(src.read_bytes()).hexdigest(),
-                         "dram_bytes_per_launch": 123456}}
+    sha = hashlib.sha256(src.read_bytes()).hexdigest()
+    rec = {"attention:wan": {"workload": "wan", "source": "k.cu", "sha256": sha, "dram_bytes_per_launch": 123456},
+           "attention:ropeslr": {"workload": "ropeslr", "source": "k.cu", "sha256": sha,
+                                 "dram_bytes_per_launch": 654321}}
     (tmp_path / "profiles" / "traffic.json").write_text(json.dumps(rec))
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     assert bench.measured_traffic("attention") == 123456
+    assert bench.measured_traffic("attention", "ropeslr") == 654321
+    assert bench.measured_traffic("attention", "lvsa") is None
     assert bench.measured_traffic("pool_means") is None
     src.write_text("kernel source, changed\n")
     assert bench.measured_traffic("attention") is None
