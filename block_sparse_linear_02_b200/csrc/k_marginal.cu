@@ -543,17 +543,21 @@ key_states_pipe_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_con
 }
 
 // ------------------------------------------------------------------ reduce states (GEMM)
-// Persistent: one CTA per SM walks the output tiles (128 query blocks x 256
-// state columns) of every head; a 4-stage TMA ring runs across tile boundaries
-// and two TMEM accumulators let the epilogue of one tile overlap the main loop
-// of the next.  Tiles are ordered M-fastest so the query-block tiles sharing one
-// slab of h run back to back (h is read from HBM about once).  Each epilogue warp
-// stages its 32 rows x 64 columns per chunk in a 128B-swizzled tile and writes it
-// with a TMA tensor store (whole 128-byte row segments instead of 16-byte pieces
-// of 32 different rows).
-constexpr int kGemmStages = 4;
+// Persistent: one CTA per SM walks the output tiles (256 query blocks x 256 state
+// columns) of every head.  A tile is two M = 128 halves that share every B stage (the
+// 64 K-rows x 256 columns of h), so each h slab crosses from L2 into shared memory half
+// as often per output as with 128-row tiles.  A 3-stage TMA ring of 64 KB stages runs
+// across tile boundaries; the two halves' accumulators fill TMEM (2 x 256 columns), so
+// the epilogue hands each half back as soon as it has read it and the next tile's first
+// stage starts on half 0 while half 1 drains.  Tiles are ordered M-fastest so the tiles
+// sharing one slab of h run back to back (h is read from HBM about once).  Each epilogue
+// warp stages its 32 rows x 64 columns per chunk in a 128B-swizzled tile and writes it
+// with a TMA tensor store.
+constexpr int kGemmStages = 3;
+constexpr int kGemmBM = 256;
 constexpr int kGemmBN = 256;
-constexpr int kGemmABytes = 128 * 128;          // 128 rows x 64 bf16
+constexpr int kGemmAHalf = 128 * 128;           // 128 rows x 64 bf16
+constexpr int kGemmABytes = 2 * kGemmAHalf;
 constexpr int kGemmBBytes = 4 * 64 * 128;       // 4 chunks of 64 K-rows x 64 bf16
 constexpr int kGemmOutBytes = 32 * 128;         // one warp's staged chunk: 32 rows x 64 bf16
 constexpr int kGemmOutOff = kGemmStages * (kGemmABytes + kGemmBBytes);   // [4 warps][2 buffers]
@@ -569,21 +573,22 @@ reduce_states_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
   uint8_t* sA = smem;
   uint8_t* sB = smem + kGemmStages * kGemmABytes;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kGemmBarOff);
-  uint64_t* full = bars;                          // [4]
-  uint64_t* empty = bars + kGemmStages;           // [4]
-  uint64_t* acc_full = empty + kGemmStages;       // [2] MMA -> epilogue
-  uint64_t* acc_empty = acc_full + 2;             // [2] epilogue -> MMA (128 arrivals)
+  uint64_t* full = bars;                          // [3]
+  uint64_t* empty = bars + kGemmStages;           // [3]
+  uint64_t* acc_full = empty + kGemmStages;       // MMA -> epilogue, one phase per tile
+  uint64_t* acc_empty = acc_full + 1;             // [2] per half: epilogue -> MMA (128 arrivals)
   uint64_t* drain = acc_empty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int kt_total = (nb + 63) / 64;
-  const int mt = (nb + 127) / 128, nt = (ntot + kGemmBN - 1) / kGemmBN;
+  const int mt = (nb + kGemmBM - 1) / kGemmBM, nt = (ntot + kGemmBN - 1) / kGemmBN;
   const int n_tiles = mt * nt * BH;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kGemmStages; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
-    for (int b = 0; b < 2; ++b) { mbar_init(&acc_full[b], 1); mbar_init(&acc_empty[b], 128); }
+    mbar_init(acc_full, 1);
+    for (int b = 0; b < 2; ++b) mbar_init(&acc_empty[b], 128);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -599,12 +604,14 @@ reduce_states_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
       int it = 0;                                 // global k-iteration counter across tiles
       bool ok = true;
       for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
-        const int m0 = (t % mt) * 128, n0 = ((t / mt) % nt) * kGemmBN, bh = t / (mt * nt);
+        const int m0 = (t % mt) * kGemmBM, n0 = ((t / mt) % nt) * kGemmBN, bh = t / (mt * nt);
         for (int kt = 0; kt < kt_total; ++kt, ++it) {
           const int s = it % kGemmStages;
           if (it >= kGemmStages && !mbar_wait(&empty[s], ((it / kGemmStages) - 1) & 1, abort_flag, status)) { ok = false; break; }
           mbar_arrive_expect_tx(&full[s], kGemmABytes + kGemmBBytes);
+          // rows past nb (the second half of the last M tile) arrive as zero fill
           tma_load_3d(sA + s * kGemmABytes, &tmA, &full[s], kt * 64, m0, bh);
+          tma_load_3d(sA + s * kGemmABytes + kGemmAHalf, &tmA, &full[s], kt * 64, m0 + 128, bh);
           for (int c = 0; c < 4; ++c)
             tma_load_3d(sB + s * kGemmBBytes + c * 8192, &tmB, &full[s], n0 + c * 64, kt * 64, bh);
         }
@@ -622,23 +629,27 @@ reduce_states_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
       int it = 0, local = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++local) {
-        const int ab = local & 1;
-        // the accumulator must have been drained by the epilogue of tile local-2
-        if (local >= 2 && !mbar_wait(&acc_empty[ab], ((local - 2) >> 1) & 1, abort_flag, status)) { ok = false; break; }
-        tc_fence_after();
         for (int kt = 0; kt < kt_total; ++kt, ++it) {
           const int s = it % kGemmStages;
           if (!mbar_wait(&full[s], (it / kGemmStages) & 1, abort_flag, status)) { ok = false; break; }
-          tc_fence_after();
+          const uint32_t a_base = smem_u32(sA + s * kGemmABytes);
+          const uint64_t b0 = desc_mnmajor(smem_u32(sB + s * kGemmBBytes), 8192);
           #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t a = desc_kmajor(smem_u32(sA + s * kGemmABytes) + kk * 32);
-            const uint64_t b = desc_mnmajor(smem_u32(sB + s * kGemmBBytes) + kk * 2048, 8192);
-            mma_bf16_ss(tmem + ab * kGemmBN, a, b, id, (kt > 0 || kk > 0) ? 1u : 0u);
+          for (int half = 0; half < 2; ++half) {
+            // half h of the accumulator must have been read by the epilogue of tile local-1
+            if (kt == 0 && local >= 1 &&
+                !mbar_wait(&acc_empty[half], (local - 1) & 1, abort_flag, status)) { ok = false; break; }
+            tc_fence_after();
+            #pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint64_t a = desc_kmajor(a_base + half * kGemmAHalf + kk * 32);
+              mma_bf16_ss(tmem + half * kGemmBN, a, b0 + (uint32_t)((kk * 2048) >> 4), id, (kt > 0 || kk > 0) ? 1u : 0u);
+            }
           }
+          if (!ok) break;
           mma_commit(&empty[s]);
         }
-        if (ok) mma_commit(&acc_full[ab]);
+        if (ok) mma_commit(acc_full);
       }
       if (!ok) {
         mma_commit(drain);
@@ -647,45 +658,48 @@ reduce_states_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
       }
     }
   } else {
-    // epilogue warps 0-3: TMEM lanes 32*warp.. = output rows m0 + 32*warp ..
+    // epilogue warps 0-3: TMEM lanes 32*warp.. = rows m0 + 128*half + 32*warp ..
     uint8_t* sOut = smem + kGemmOutOff + warp * 2 * kGemmOutBytes;
     int local = 0, chunk = 0;                     // chunk: this warp's store count, for the 2 staging buffers
     for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++local) {
-      const int ab = local & 1;
-      const int m0 = (t % mt) * 128, n0 = ((t / mt) % nt) * kGemmBN, bh = t / (mt * nt);
-      if (!__all_sync(0xFFFFFFFFu, mbar_wait(&acc_full[ab], (local >> 1) & 1, abort_flag, status))) break;
+      const int m0 = (t % mt) * kGemmBM, n0 = ((t / mt) % nt) * kGemmBN, bh = t / (mt * nt);
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait(acc_full, local & 1, abort_flag, status))) break;
       tc_fence_after();
-      #pragma unroll 1
-      for (int q = 0; q < kGemmBN / 64; ++q) {
-        const int n = n0 + q * 64;
-        if (n >= ntot) break;                      // uniform: the columns past the end have nothing to store
-        uint32_t v[64];
-        tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + ab * kGemmBN + q * 64, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
-        tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + ab * kGemmBN + q * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
-        uint8_t* buf = sOut + (chunk & 1) * kGemmOutBytes;
-        if (lane == 0) bulk_wait_read_1();         // the store issued from this buffer two chunks ago has read it
-        __syncwarp();
-        tmem_wait_ld();
-        #pragma unroll
-        for (int i = 0; i < 8; ++i)
-          *reinterpret_cast<uint4*>(buf + sw128_offset(lane, i)) =
-              make_uint4(pack_bf16(__uint_as_float(v[8 * i]), __uint_as_float(v[8 * i + 1])),
-                         pack_bf16(__uint_as_float(v[8 * i + 2]), __uint_as_float(v[8 * i + 3])),
-                         pack_bf16(__uint_as_float(v[8 * i + 4]), __uint_as_float(v[8 * i + 5])),
-                         pack_bf16(__uint_as_float(v[8 * i + 6]), __uint_as_float(v[8 * i + 7])));
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          // rows past nb inside the box are clipped by the tensor map; a box wholly past
-          // nb is not stored, but its (empty) group is still committed so that the
-          // two-buffer wait above stays counted per chunk
-          if (m0 + warp * 32 < nb) tma_store_3d(&tmHs, buf, n, m0 + warp * 32, bh);
-          bulk_commit();
+      for (int half = 0; half < 2; ++half) {
+        const int r0 = m0 + half * 128 + warp * 32;
+        #pragma unroll 1
+        for (int q = 0; q < kGemmBN / 64; ++q) {
+          const int n = n0 + q * 64;
+          if (n >= ntot) break;                    // uniform: the columns past the end have nothing to store
+          uint32_t v[64];
+          const uint32_t col = tmem + ((uint32_t)(warp * 32) << 16) + half * kGemmBN + q * 64;
+          tmem_ld32(col, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+          tmem_ld32(col + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+          uint8_t* buf = sOut + (chunk & 1) * kGemmOutBytes;
+          if (lane == 0) bulk_wait_read_1();       // the store issued from this buffer two chunks ago has read it
+          __syncwarp();
+          tmem_wait_ld();
+          #pragma unroll
+          for (int i = 0; i < 8; ++i)
+            *reinterpret_cast<uint4*>(buf + sw128_offset(lane, i)) =
+                make_uint4(pack_bf16(__uint_as_float(v[8 * i]), __uint_as_float(v[8 * i + 1])),
+                           pack_bf16(__uint_as_float(v[8 * i + 2]), __uint_as_float(v[8 * i + 3])),
+                           pack_bf16(__uint_as_float(v[8 * i + 4]), __uint_as_float(v[8 * i + 5])),
+                           pack_bf16(__uint_as_float(v[8 * i + 6]), __uint_as_float(v[8 * i + 7])));
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            // rows past nb inside the box are clipped by the tensor map; a box wholly past
+            // nb is not stored, but its (empty) group is still committed so that the
+            // two-buffer wait above stays counted per chunk
+            if (r0 < nb) tma_store_3d(&tmHs, buf, n, r0, bh);
+            bulk_commit();
+          }
+          ++chunk;
         }
-        ++chunk;
+        tc_fence_before();
+        mbar_arrive(&acc_empty[half]);
       }
-      tc_fence_before();
-      mbar_arrive(&acc_empty[ab]);
     }
     if (lane == 0) bulk_wait_all();
   }
@@ -930,7 +944,7 @@ cudaError_t launch_reduce_states(const __nv_bfloat16* m01, int ld_m01, const __n
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const long long tiles = (long long)((nb + 127) / 128) * ((ntot + kGemmBN - 1) / kGemmBN) * BH;
+  const long long tiles = (long long)((nb + kGemmBM - 1) / kGemmBM) * ((ntot + kGemmBN - 1) / kGemmBN) * BH;
   const int grid = (int)(tiles < sms ? tiles : sms);
   reduce_states_kernel<<<grid, 192, kGemmSmem, st>>>(ma, mb, mo, nb, ntot, BH, status);
   return cudaGetLastError();
