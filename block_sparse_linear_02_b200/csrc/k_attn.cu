@@ -22,7 +22,8 @@
 //   warp 8     TMA producer: Q once, then K_0, V_0, K_1, V_1, ... (each item the
 //              step's two 64-key blocks) into a 5-slot ring.  With LINEAR the
 //              first three slots first hold the two query blocks' linear states
-//              and phi(Q), and the K/V items start behind them;
+//              and phi(Q), and the K/V items start behind them; without it V_j and
+//              K_{j+1} complete one barrier per step;
 //   warp 9     MMA issuer: S_j = Q [K_a ; K_b]^T (N = 128) into one of two TMEM
 //              S buffers; once both softmax warpgroups have written P_j back
 //              over S_j (bf16, in TMEM), O_0 += P_j[:, a] V_a and
@@ -221,7 +222,8 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
   uint64_t* tq_full = xch_bar + 1;               // [kTq] tile slot written
   uint64_t* tq_empty = tq_full + kTq;            // [kTq] tile slot read (MMA thread + one lane per softmax warp)
   uint64_t* drain = tq_empty + kTq;
-  int* tq = reinterpret_cast<int*>(drain + 1);   // [kTq] tile indices
+  uint64_t* kv_step = drain + 1;                 // [4] per step mod 4: V_j and K_{j+1} landed (non-LINEAR)
+  int* tq = reinterpret_cast<int*>(kv_step + 4); // [kTq] tile indices
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tq + kTq);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -231,6 +233,12 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
   // LINEAR: a tile's first three ring positions hold the H'^T rows of its two query
   // blocks and phi(Q); its K/V items follow
   constexpr int kPre = LINEAR ? 3 : 0;
+  // Without the linear pre-slots the ring positions of a tile's items are regular, and
+  // V_j and K_{j+1} (consecutive positions) complete one step barrier together, so the MMA
+  // thread polls once per step for both.  Their slots are freed by step j-2 (K_{j-2}'s QK,
+  // V_{j-2}'s P.V), so waiting for both before issuing either delays only V_j, which is not
+  // needed before P.V_j.
+  constexpr bool KVSTEP = !LINEAR;
   // LINEAR: the tile's lin = phi(Q) H'_b (D columns) is written into the S buffer that step 1
   // of the tile will use, so it waits neither for the previous tile's epilogue nor for O
 
@@ -248,6 +256,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
     mbar_init(xch_bar, 256);
     for (int e = 0; e < kTq; ++e) { mbar_init(&tq_full[e], 1); mbar_init(&tq_empty[e], 9); }
     mbar_init(drain, 1);
+    for (int q = 0; q < 4; ++q) mbar_init(&kv_step[q], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -285,7 +294,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
         }
         return true;
       };
-      int i = 0, J = 0, g = 0, q_loaded = -1;
+      int i = 0, J = 0, g = 0, q_loaded = -1, kv_armed = -1;   // kv_armed: last step barrier armed
       bool ok = true;
       int t_next = atomicAdd(p.tile_counter, 1);       // the queue is read one tile ahead
       while (ok) {
@@ -341,31 +350,72 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
             rel_idx[slot] = i;
           }
         }
-        // K/V items: K (even it) or V (odd it) of step it/2
-        for (int it = 0; it < 2 * ti.n_steps && ok; ++it, ++g) {
-          const int slot = g % kSlots;
-          if (!(ok = slot_released(slot))) break;
-          const int j = it >> 1;
-          const bool is_v = it & 1;
+        // one K or V item of step j into a ring slot, its TMA completing on barrier `bar`
+        auto load_item = [&](int slot, int j, bool is_v, uint64_t* bar) {
           const int nb = step_blocks(j);
           const bool far = GATED && j == ti.local_steps;
-          mbar_arrive_expect_tx(&slot_full[slot], nb * L::kChunks * L::kHalf);
           for (int b = 0; b < nb; ++b) {
             uint8_t* dst = sRing + slot * L::kKV + b * L::kHalf;
             if (far) {
               for (int c = 0; c < L::kChunks; ++c)
-                tma_load_3d(dst + c * L::kTile, is_v ? &tmX2 : &tmX1, &slot_full[slot], c * 64, 0, ti.bh);
+                tma_load_3d(dst + c * L::kTile, is_v ? &tmX2 : &tmX1, bar, c * 64, 0, ti.bh);
             } else {
               // key block kb: rows [64 kb, 64 kb + 64) (in the tile layout K and V are in
               // tile-major order, so a 4x4x4 tile is one such block)
               const int kb = ti.list ? (int)(ti.list[2 * j + b] & 0xFFFFu) : 2 * j + b;
               const CUtensorMap* tm = is_v ? &tmV : &tmK;
               for (int c = 0; c < L::kChunks; ++c)
-                tma_load_3d(dst + c * L::kTile, tm, &slot_full[slot], c * 64, kb * 64, ti.bh);
+                tma_load_3d(dst + c * L::kTile, tm, bar, c * 64, kb * 64, ti.bh);
             }
           }
-          rel_kind[slot] = is_v ? 0 : 3;
-          rel_idx[slot] = J + j;
+        };
+        auto item_bytes = [&](int j) -> uint32_t { return (uint32_t)(step_blocks(j) * L::kChunks * L::kHalf); };
+        if (KVSTEP) {
+          // K_0 on its slot barrier; then per step j, V_j and K_{j+1} on kv_step[j]; their slot
+          // barriers get a plain arrive, so every use of a slot still advances its phase once
+          if (ti.n_steps > 0 && ok) {
+            const int slot = g % kSlots;
+            if ((ok = slot_released(slot))) {
+              mbar_arrive_expect_tx(&slot_full[slot], item_bytes(0));
+              load_item(slot, 0, false, &slot_full[slot]);
+              rel_kind[slot] = 3;
+              rel_idx[slot] = J;
+              ++g;
+            }
+          }
+          for (int j = 0; j < ti.n_steps && ok; ++j) {
+            const bool has_k = j + 1 < ti.n_steps;
+            const int sv = g % kSlots, sk = (g + 1) % kSlots;
+            if (!(ok = slot_released(sv))) break;
+            if (has_k && !(ok = slot_released(sk))) break;
+            uint64_t* bar = &kv_step[(J + j) & 3];
+            mbar_arrive_expect_tx(bar, item_bytes(j) + (has_k ? item_bytes(j + 1) : 0u));
+            load_item(sv, j, true, bar);
+            mbar_arrive(&slot_full[sv]);
+            rel_kind[sv] = 0;
+            rel_idx[sv] = J + j;
+            ++g;
+            if (has_k) {
+              load_item(sk, j + 1, false, bar);
+              mbar_arrive(&slot_full[sk]);
+              rel_kind[sk] = 3;
+              rel_idx[sk] = J + j + 1;
+              ++g;
+            }
+            kv_armed = J + j;
+          }
+        } else {
+          // K/V items: K (even it) or V (odd it) of step it/2
+          for (int it = 0; it < 2 * ti.n_steps && ok; ++it, ++g) {
+            const int slot = g % kSlots;
+            if (!(ok = slot_released(slot))) break;
+            const int j = it >> 1;
+            const bool is_v = it & 1;
+            mbar_arrive_expect_tx(&slot_full[slot], item_bytes(j));
+            load_item(slot, j, is_v, &slot_full[slot]);
+            rel_kind[slot] = is_v ? 0 : 3;
+            rel_idx[slot] = J + j;
+          }
         }
         J += ti.n_steps;
         ++i;
@@ -377,6 +427,11 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
         for (int gg = (g - kSlots > 0 ? g - kSlots : 0); gg < g; ++gg) {
           t0 = clock64();
           while (!mbar_try_wait(&slot_full[gg % kSlots], (gg / kSlots) & 1) && clock64() - t0 < kWaitBudgetCycles) {}
+        }
+        // the step barriers whose loads may still be in flight (the ring holds at most 3 steps)
+        for (int q = (kv_armed - 3 > 0 ? kv_armed - 3 : 0); q <= kv_armed; ++q) {
+          t0 = clock64();
+          while (!mbar_try_wait(&kv_step[q & 3], (q >> 2) & 1) && clock64() - t0 < kWaitBudgetCycles) {}
         }
       }
     }
@@ -478,17 +533,21 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
         bool o1_started = false;
         for (int j = 0; j < ti.n_steps && ok; ++j) {
           const int Jj = J + j, b = Jj & 1;
+          if (KVSTEP) {                            // V_j and K_{j+1} have landed (one barrier for both)
+            if (!(ok = mbar_wait(&kv_step[Jj & 3], (Jj >> 2) & 1, abort_flag, p.status))) break;
+            tc_fence_after();
+          }
           if (j + 1 < ti.n_steps) {
             const int gk = gkv + 2 * (j + 1);
-            if (!(ok = mbar_wait(&slot_full[gk % kSlots], (gk / kSlots) & 1, abort_flag, p.status) &&
-                       settle_lin())) break;
+            ok = KVSTEP || mbar_wait(&slot_full[gk % kSlots], (gk / kSlots) & 1, abort_flag, p.status);
+            if (!(ok = ok && settle_lin())) break;
             tc_fence_after();
             issue_qk(gk % kSlots, (Jj + 1) & 1);
             mma_commit(&s_full[(Jj + 1) & 3]);
             if (j + 2 == ti.n_steps) mma_commit(q_free);
           }
           const int gv = gkv + 2 * j + 1;
-          if (!mbar_wait(&slot_full[gv % kSlots], (gv / kSlots) & 1, abort_flag, p.status) ||
+          if ((!KVSTEP && !mbar_wait(&slot_full[gv % kSlots], (gv / kSlots) & 1, abort_flag, p.status)) ||
               !mbar_wait(&p_full[b], (Jj >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
           tc_fence_after();
           const bool far = GATED && j == ti.local_steps;
