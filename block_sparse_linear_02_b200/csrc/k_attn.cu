@@ -60,12 +60,12 @@ struct AttnLayout {
   static constexpr int kKV = kChunks * kTile;            // one ring item: K (or V) of one step
   static constexpr int kHsChunk = D * 128;               // H'^T rows of one query block: D rows per 64-column chunk
   static constexpr int kHsTile = kChunks * kHsChunk;     // one ring item
-  static constexpr int kZChunk = 16 * 128;               // [Z ; 15 zero rows] per 64-column chunk
+  static constexpr int kZChunk = 128;                    // the Z row, one 64-column chunk
   static constexpr int kZTile = kChunks * kZChunk;
   static constexpr int kQOff = 0;
   static constexpr int kRingOff = kQOff + kChunks * kTile;
-  static constexpr int kZOff = kRingOff + kSlots * kKV;  // Z tiles of the pair's two query blocks
-  static constexpr int kXOff = kZOff + 2 * kZTile;       // exchange area: [2 shares][2 tiles][3][128] floats
+  static constexpr int kZOff = kRingOff + kSlots * kKV;  // [2 tile parities][2 query blocks] Z rows
+  static constexpr int kXOff = kZOff + 4 * kZTile;       // exchange area: [2 shares][2 tiles][3][128] floats
   static constexpr int kBarOff = kXOff + 12 * 128 * 4;
   // output staging: per softmax warp one 32-row x 32-column bf16 chunk (64-byte rows,
   // 64-byte swizzle), written to HBM by TMA tensor stores
@@ -208,8 +208,8 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
   float* xch = reinterpret_cast<float*>(smem + L::kXOff);   // [2 tiles][3][128]: m, l, far-l per warpgroup share
   uint8_t* sOut = smem + L::kOutOff;                         // [8 softmax warps] output staging chunks
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
-  uint64_t* q_full = bars + 0;                   // Q (and Z) of the current tile landed
-  uint64_t* q_free = q_full + 1;                 // every MMA reading Q / Z of a tile has completed
+  uint64_t* q_full = bars + 0;                   // Q of the current tile landed
+  uint64_t* q_free = q_full + 1;                 // every MMA reading Q of a tile has completed
   uint64_t* slot_full = q_free + 1;              // [kSlots] ring slot filled (TMA, or freed for phi(Q))
   uint64_t* s_full = slot_full + kSlots;         // [4] per step mod 4: S_j written (the step's K item is free)
   uint64_t* p_full = s_full + 4;                 // [2] per S buffer, 256 arrivals
@@ -223,7 +223,8 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
   uint64_t* tq_empty = tq_full + kTq;            // [kTq] tile slot read (MMA thread + one lane per softmax warp)
   uint64_t* drain = tq_empty + kTq;
   uint64_t* kv_step = drain + 1;                 // [4] per step mod 4: V_j and K_{j+1} landed (non-LINEAR)
-  int* tq = reinterpret_cast<int*>(kv_step + 4); // [kTq] tile indices
+  uint64_t* z_full = kv_step + 4;                // [2] per tile parity: the tile's Z rows landed (LINEAR)
+  int* tq = reinterpret_cast<int*>(z_full + 2);  // [kTq] tile indices
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tq + kTq);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -257,6 +258,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
     for (int e = 0; e < kTq; ++e) { mbar_init(&tq_full[e], 1); mbar_init(&tq_empty[e], 9); }
     mbar_init(drain, 1);
     for (int q = 0; q < 4; ++q) mbar_init(&kv_step[q], 1);
+    for (int q = 0; q < 2; ++q) mbar_init(&z_full[q], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -311,9 +313,9 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
           if (GATED && j == ti.local_steps) return 1;
           return (2 * j + 1 < ti.n_local) ? 2 : 1;
         };
-        // Q (and Z) of this tile once every MMA of the previous tile that reads them is done
+        // Q of this tile once every MMA of the previous tile that reads it is done
         if (i > 0 && !(ok = mbar_wait(q_free, (i - 1) & 1, abort_flag, p.status))) break;
-        mbar_arrive_expect_tx(q_full, L::kChunks * L::kTile + ti.n_lin * L::kZTile);
+        mbar_arrive_expect_tx(q_full, L::kChunks * L::kTile);
         q_loaded = i;
         if (TILE) {
           for (int half = 0; half < 2; ++half) {
@@ -325,9 +327,17 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
         } else {
           for (int c = 0; c < L::kChunks; ++c) tma_load_3d(sQ + c * L::kTile, &tmQ, q_full, c * 64, ti.pair * 128, ti.bh);
         }
-        for (int b = 0; b < ti.n_lin; ++b)   // row D of the state (Z) and 15 rows of zero fill
-          for (int c = 0; c < L::kChunks; ++c)
-            tma_load_3d(sZ + b * L::kZTile + c * L::kZChunk, &tmX2, q_full, c * 64, D, ti.bh * p.n_qb + 2 * ti.pair + b);
+        if (LINEAR) {
+          // row D of the state (Z) of each query block, into this tile parity's buffer and on the
+          // parity's own barrier: the softmax warps read it at the tile start, which can come
+          // after the next tile's Q has landed (a one-step tile releases Q after its only QK),
+          // so neither the buffer nor q_full's phase may be shared with the next tile
+          mbar_arrive_expect_tx(&z_full[i & 1], ti.n_lin * L::kZTile);
+          for (int b = 0; b < ti.n_lin; ++b)
+            for (int c = 0; c < L::kChunks; ++c)
+              tma_load_3d(sZ + ((i & 1) * 2 + b) * L::kZTile + c * L::kZChunk, &tmX2, &z_full[i & 1], c * 64, D,
+                          ti.bh * p.n_qb + 2 * ti.pair + b);
+        }
         if (LINEAR) {
           // pre-slots by TMA: the states of the two query blocks, then phi(Q); a missing
           // second query block's slot completes its phase with a plain arrive
@@ -424,6 +434,10 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
         // let the loads already in flight land before the CTA's shared memory is released
         long long t0 = clock64();
         if (q_loaded >= 0) while (!mbar_try_wait(q_full, q_loaded & 1) && clock64() - t0 < kWaitBudgetCycles) {}
+        if (LINEAR && q_loaded >= 0) {
+          t0 = clock64();
+          while (!mbar_try_wait(&z_full[q_loaded & 1], (q_loaded >> 1) & 1) && clock64() - t0 < kWaitBudgetCycles) {}
+        }
         for (int gg = (g - kSlots > 0 ? g - kSlots : 0); gg < g; ++gg) {
           t0 = clock64();
           while (!mbar_try_wait(&slot_full[gg % kSlots], (gg / kSlots) & 1) && clock64() - t0 < kWaitBudgetCycles) {}
@@ -529,7 +543,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
           issue_qk(gkv % kSlots, J & 1);           // S buffer J & 1: never the tile's lin buffer
           mma_commit(&s_full[J & 3]);
         }
-        if (ti.n_steps <= 1) mma_commit(q_free);   // the last MMA reading Q (and Z) has been issued
+        if (ti.n_steps <= 1) mma_commit(q_free);   // the last MMA reading Q has been issued
         bool o1_started = false;
         for (int j = 0; j < ti.n_steps && ok; ++j) {
           const int Jj = J + j, b = Jj & 1;
@@ -628,11 +642,11 @@ attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
       float den_part = 0.f;
       if (LINEAR) {
         const int gphi = g + 2;
-        ok = __all_sync(0xFFFFFFFFu, mbar_wait(q_full, i & 1, abort_flag, p.status) &&
+        ok = __all_sync(0xFFFFFFFFu, mbar_wait(&z_full[i & 1], (i >> 1) & 1, abort_flag, p.status) &&
                                          mbar_wait(&slot_full[gphi % kSlots], (gphi / kSlots) & 1, abort_flag, p.status));
         if (ok) {
           const uint8_t* sPhi = sRing + (gphi % kSlots) * L::kKV;
-          const uint8_t* zrow = sZ + half * L::kZTile;     // Z of my query block: row 0 of its Z tile
+          const uint8_t* zrow = sZ + ((i & 1) * 2 + half) * L::kZTile;   // Z of my query block, this tile parity
           constexpr int kGroups = D / 16;                  // 16-byte groups of my row handled by my warpgroup
           #pragma unroll
           for (int gr = 0; gr < kGroups; ++gr) {
@@ -1005,13 +1019,13 @@ cudaError_t launch_attention(const AttnArgs& a, cudaStream_t st) {
     if (!make_tile_map(&maps[3], a.kf, 3, dims, strides, box)) return cudaErrorInvalidValue;
     if (!make_tile_map(&maps[4], a.vf, 3, dims, strides, box)) return cudaErrorInvalidValue;
   } else if (a.Hs) {
-    // [H'^T ; Z] rows of each query block: the D rows of H'^T, and Z with 15 rows of zero fill
+    // [H'^T ; Z] rows of each query block: the D rows of H'^T, and the Z row
     const uint64_t dims[3] = {(uint64_t)D, (uint64_t)(D + 1), (uint64_t)a.BH * a.n_qb};
     const uint64_t strides[2] = {rowb, rowb * (D + 1)};
     const uint32_t boxh[3] = {64, (uint32_t)D, 1};
-    const uint32_t boxz[3] = {64, 16, 1};
+    const uint32_t boxz[3] = {64, 1, 1};
     if (!make_tile_map(&maps[3], a.Hs, 3, dims, strides, boxh)) return cudaErrorInvalidValue;
-    if (!make_tile_map(&maps[4], a.Hs, 3, dims, strides, boxz)) return cudaErrorInvalidValue;
+    if (!make_tile_map(&maps[4], a.Hs, 3, dims, strides, boxz, 0)) return cudaErrorInvalidValue;   // read as a plain row
     if (!a.phi_q) return cudaErrorInvalidValue;
     const uint64_t qdims[3] = {(uint64_t)D, (uint64_t)a.s.n_pad, (uint64_t)a.BH};
     const uint64_t qstrides[2] = {rowb, rowb * a.s.n_pad};

@@ -2,8 +2,9 @@
 oracle: the tiny workload and ragged cases in full (one with two batch
 entries), the 32k-token workload at full size (all masks of all heads, outputs
 on 64 sampled query blocks of every head), the 115k-token workload (all masks
-of all 24 heads, outputs on 64 sampled query blocks of every head) and the
-dense mode.
+of all 24 heads, outputs on 64 sampled query blocks of every head), the 32k
+workload with one or two critical blocks per query block (one- and two-step
+tiles, many per CTA) and the dense mode.
 
 Where the library's label row differs from the oracle's (only inside the 1e-5
 threshold band, which check_mask enforces), that query block's output is
@@ -151,6 +152,23 @@ def test_hunyuan_workload_sampled():
     status_ok()
     flipped = _compare(q, k, v, wp, _seq(w), w.crit_frac, w.negl_frac, out, mask, range(w.heads), sample=64)
     assert flipped <= 4
+
+
+@pytest.mark.parametrize("crit", [0.001, 0.003])
+def test_one_and_two_step_tiles_many_per_cta(crit):
+    # one or two critical blocks per query block: every pair's tile walks one or two steps,
+    # and each CTA takes ~21 such tiles in a row (a short tile hands its Q buffer back after
+    # its only QK, so the next tile's Q and Z can land before this tile's softmax starts)
+    w = workloads.WAN
+    q, k, v = workloads.make_qkv(w)
+    wp = workloads.make_w_proj(w)
+    kc, kn = slr.slr_block_counts(w.n_blocks, crit, w.negl_frac)
+    assert kc == (1 if crit == 0.001 else 2)
+    out, mask = slr.slr_sparse_linear_attn(cuda(q), cuda(k), cuda(v), cuda(wp), _seq(w), crit, w.negl_frac,
+                                           mask_out=True)
+    status_ok()
+    flipped = _compare(q, k, v, wp, _seq(w), crit, w.negl_frac, out, mask, [0, 5, 11], sample=32, seed=7)
+    assert flipped <= 2
 
 
 @pytest.mark.parametrize("name", ["tiny", "wan"])
