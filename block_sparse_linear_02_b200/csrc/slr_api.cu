@@ -221,8 +221,13 @@ slr_status check_mask(const slr_mask_desc* m, const Shape& sh) {
 
 // Tile radius per axis of a TILE3D or STA mask: a window of (2r+1) tiles keeps the tiles
 // whose centres lie within half a window of the query tile's centre, i.e. within r tiles
+// A radius past the grid adds no tile, so it is clamped to the grid's extent on that axis.
 void mask_radii(const slr_mask_desc* m, int rad[3]) {
-  for (int a = 0; a < 3; ++a) rad[a] = m->kind == SLR_MASK_STA ? (m->window[a] / 4 - 1) / 2 : m->radius;
+  const int extent[3] = {m->F / 4, m->Hh / 4, m->Ww / 4};
+  for (int a = 0; a < 3; ++a) {
+    const int r = m->kind == SLR_MASK_STA ? (m->window[a] / 4 - 1) / 2 : m->radius;
+    rad[a] = r < extent[a] - 1 ? r : extent[a] - 1;
+  }
 }
 
 void plan_frame(Carve& c, const Shape& sh, const slr_mask_desc* m, FrameWs& w) {
