@@ -5,7 +5,8 @@ first and last blocks and frame tails) and the gated tile neighbourhood + far
 field (small grids in full, including an odd tile count and two batch entries,
 and the 8x64x64 workload on sampled tokens), with and without the 3-D rotary
 embedding of q and k; the sliding tile mask (small grids in full with windows of
-one to seven tiles per axis, two batch entries, 8x64x64 on sampled tokens)."""
+one to seven tiles per axis, two batch entries, 8x64x64 on sampled tokens, and a
+window covering the grid against the dense call)."""
 import numpy as np
 import pytest
 import torch
@@ -223,3 +224,20 @@ def test_sta_workload_sampled():
         outs.append(to64(out[0, h])[toks])
         refs.append(ref[toks])
     assert_close(np.concatenate(outs), np.concatenate(refs), "sta workload")
+
+
+def test_sta_window_covering_the_grid_is_dense_attention():
+    # every tile within reach on every axis: the sliding tile call equals the library's dense
+    # block-sparse call on the same (raster) tokens, and both equal plain softmax attention
+    H, d, F, Hh, Ww = 2, 128, 8, 16, 16
+    n = F * Hh * Ww
+    q, k, v = make_inputs(1, H, d, 1, n, n, seed=67)
+    seq = slr.make_seq(1, H, d, 1, n, n)
+    out = slr.slr_frame_mask_attn(cuda(q), cuda(k), cuda(v), seq, slr.sta_mask(F, Hh, Ww, (12, 28, 28)))
+    status_ok()
+    dense, _ = slr.slr_block_sparse_attn(cuda(q), cuda(k), cuda(v), seq)
+    status_ok()
+    for h in range(H):
+        ref = osta.sliding_tile_attention(to64(q[0, h]), to64(k[0, h]), to64(v[0, h]), F, Hh, Ww, window=(12, 28, 28))
+        assert_close(to64(out[0, h]), ref, f"sta covering head {h}")
+        assert_close(to64(dense[0, h]), ref, f"dense head {h}")
