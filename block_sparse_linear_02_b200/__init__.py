@@ -32,6 +32,7 @@ SLR_PHI_SOFTMAX = 1
 SLR_MASK_LVSA = 1
 SLR_MASK_TILE3D = 2
 SLR_MASK_STA = 3
+ABI_VERSION = 200          # include/slr.h SLR_ABI_VERSION
 
 SLR_OP_POOL_CLASSIFY = 1
 SLR_OP_BLOCK_SPARSE = 2
@@ -105,6 +106,9 @@ def lib() -> ctypes.CDLL:
                      "slr_sparse_linear_attn", "slr_frame_mask_attn", "slr_check_status",
                      "slr_block_counts", "slr_lvsa_attention_sets", "slr_version"):
             getattr(L, name).restype = i
+        if L.slr_version() != ABI_VERSION:
+            # the structs above mirror include/slr.h of this version; an older build would read them wrongly
+            raise RuntimeError(f"{LIB_PATH} has ABI {L.slr_version()}, this binding expects {ABI_VERSION}; rebuild it")
         _lib = L
     return _lib
 

@@ -360,7 +360,7 @@ AttnArgs attn_base(const Shape& sh, const void* q, const void* k, const void* v,
 
 extern "C" {
 
-int slr_version(void) { return 100; }
+int slr_version(void) { return SLR_ABI_VERSION; }
 
 slr_status slr_profile_enable(int on) {
   g_prof = on != 0;

@@ -296,6 +296,9 @@ slr_status slr_profile_enable(int on);
 int slr_profile_collect(const char** names, int* launches, double* total_ms, int max);
 
 const char* slr_status_string(slr_status s);
+/* ABI version, 100 * major + minor.  200: slr_mask_desc gained `rope` and `window` (and the
+ * SLR_MASK_STA kind), so a caller built against an earlier header passes a shorter struct. */
+#define SLR_ABI_VERSION 200
 int slr_version(void);
 
 #ifdef __cplusplus
