@@ -22,6 +22,10 @@ three source write-ups define:
 * ``oracle.sta``    -- the 3-D sliding tile attention mask of VORTA (arXiv
                        2505.18809), as described on the zhaoyang97 paper-notes
                        page, section "方法详解", design 1, and attention over it.
+* ``oracle.svoo``   -- SVOO (arXiv 2603.18636), as described on the gist.science
+                       summary, section 3, stage 2: bidirectional Q-K
+                       co-clustering from sampled anchors, and attention over
+                       the top block pairs of the co-clustered order.
 
 It shares no code with the CUDA library and imports nothing from it.  Only the
 tests, ``__graft_entry__.smoke()`` and the CPU-baseline leg of ``bench.py`` may
@@ -31,4 +35,4 @@ All arithmetic is fp64.  Parity status of every function is listed in each
 module's header; every function is pinned by a test in ``tests/test_oracle_*.py``
 against closed forms, special cases, library routines or hand-worked examples.
 """
-from . import sla, lvsa, tile3d, sta  # noqa: F401
+from . import sla, lvsa, tile3d, sta, svoo  # noqa: F401

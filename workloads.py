@@ -6,7 +6,7 @@ attention arithmetic.  Every tensor is drawn in fp32 from a seeded
 the fp64 oracle receive identical bf16 bits.  Pad tokens (the tail of every
 segment past ``seg_len``) are zero.
 
-The five workloads follow the shapes the source pages talk about:
+The workloads follow the shapes the source pages talk about:
 
 * ``tiny``    -- 2 heads, d=64, 4 frames of 8x8 tokens (256 tokens), SLA with
                  25 % critical / 25 % negligible.
@@ -21,6 +21,11 @@ The five workloads follow the shapes the source pages talk about:
 * ``ropeslr`` -- RoPeSLR-shaped gated local + far field: 16 heads, d=128,
                  8x64x64 = 32,768 tokens; N(0,1); 4x4x4 tiles, 3x3x3 tile
                  neighbourhood, 2x16x16 pooling cells, gate g=0.55.
+* ``sta``     -- VORTA's sliding tile attention on the same 8x64x64 latent,
+                 windows of 12x28x20 tokens.
+* ``svoo``    -- SVOO's co-clustered block-sparse attention on the wan layer:
+                 64 query and 64 key clusters from sampled anchors
+                 (``make_anchors``), 2 iterations, 20 % of the key blocks kept.
 
 Frame-correlated recipe (wan, hunyuan): for head h, frame f, position p and
 channel c, ``x = sqrt(0.5)*s[h,f,c] + sqrt(0.5)*e[h,f,p,c]`` with s, e ~ N(0,1),
@@ -48,7 +53,7 @@ class Workload:
     seg_stride: int     # padded tokens per segment
     n_seg: int          # number of padded segments
     seg_len: int        # valid tokens per segment
-    mode: str           # "sla", "lvsa", "tile3d" or "sta"
+    mode: str           # "sla", "lvsa", "tile3d", "sta" or "svoo"
     correlated: bool
     crit_frac: float = 0.05
     negl_frac: float = 0.10
@@ -64,6 +69,10 @@ class Workload:
     rope: bool = False  # 3-D rotary embedding of q and k before both branches
     # STA: sliding tile window in tokens per axis (odd multiples of the 4-token tile)
     window: tuple = (12, 12, 12)
+    # SVOO: query and key cluster counts, co-clustering iterations, kept fraction of key blocks
+    clusters: tuple = (64, 64)
+    iters: int = 2
+    keep_frac: float = 0.2
     batch: int = 1
 
     @property
@@ -101,7 +110,15 @@ ROPESLR = Workload("ropeslr", 5, heads=16, d=128, frames=8, fh=64, fw=64,
 STA = Workload("sta", 6, heads=16, d=128, frames=8, fh=64, fw=64,
                seg_stride=32768, n_seg=1, seg_len=32768, mode="sta", correlated=False, window=(12, 28, 20))
 
-ALL = (TINY, WAN, HUNYUAN, LVSA, ROPESLR, STA)
+# SVOO's co-clustered block-sparse attention on the Wan2.1-1.3B-shaped layer (the model the
+# SVOO summary reports first): 64 query and 64 key clusters, 2 iterations, 20 % of the key
+# blocks kept per query block (the summary's example of a robust layer that loses 80 % of
+# its attention); not one of the quoted configurations
+SVOO = Workload("svoo", 7, heads=12, d=128, frames=21, fh=30, fw=52,
+                seg_stride=32768, n_seg=1, seg_len=32760, mode="svoo", correlated=True,
+                clusters=(64, 64), iters=2, keep_frac=0.2)
+
+ALL = (TINY, WAN, HUNYUAN, LVSA, ROPESLR, STA, SVOO)
 BY_NAME = {w.name: w for w in ALL}
 
 
@@ -158,3 +175,33 @@ def small_variant(w: Workload, **changes) -> Workload:
 def random_bf16(shape, seed: int, scale: float = 1.0) -> torch.Tensor:
     gen = torch.Generator().manual_seed(seed)
     return (torch.randn(*shape, generator=gen, dtype=torch.float32) * scale).to(torch.bfloat16)
+
+
+def make_anchors(w: Workload, which: str, heads: int | None = None) -> torch.Tensor:
+    """SVOO anchor tokens: int32 [B, H, C], C distinct valid tokens per (b, h) drawn
+    uniformly without replacement (C = clusters[0] for "q", clusters[1] for "k")."""
+    C = w.clusters[0] if which == "q" else w.clusters[1]
+    seed = {"q": 5000, "k": 6000}[which] + w.index
+    H = w.heads if heads is None else heads
+    valid = torch.nonzero(_valid_rows(w.n_seg, w.seg_len, w.seg_stride)).reshape(-1)
+    out = torch.zeros(w.batch, H, C, dtype=torch.int32)
+    for b in range(w.batch):
+        for h in range(H):
+            gen = torch.Generator().manual_seed(seed * 1_000_003 + b * 1009 + h)
+            out[b, h] = valid[torch.randperm(valid.numel(), generator=gen)[:C]].to(torch.int32)
+    return out
+
+
+def make_mixture(n: int, d: int, n_comp: int, seed: int, spread: float = 0.05):
+    """Well-separated Gaussian mixture: (x bf16 [n, d], component [n] int64, anchors [n_comp]).
+
+    Component means ~ N(0, 1)^d, each token = its component's mean + spread * N(0, 1)^d.
+    Every component holds at least one token; anchors[m] is the first token of component m.
+    """
+    gen = torch.Generator().manual_seed(seed)
+    mu = torch.randn(n_comp, d, generator=gen, dtype=torch.float32)
+    comp = torch.randint(n_comp, (n,), generator=gen)
+    comp[torch.randperm(n, generator=gen)[:n_comp]] = torch.arange(n_comp)
+    x = mu[comp] + spread * torch.randn(n, d, generator=gen, dtype=torch.float32)
+    anchors = torch.tensor([int(torch.nonzero(comp == m)[0]) for m in range(n_comp)], dtype=torch.int64)
+    return x.to(torch.bfloat16), comp, anchors
