@@ -100,6 +100,11 @@ def config_dict(w, phi="elu1"):
         desc = (f"{w.name}: sliding tile attention B={w.batch} H={w.heads} d={w.d} "
                 f"{w.frames}x{w.fh}x{w.fw}={w.n_pad} tokens, 4x4x4 tiles, window "
                 f"{w.window[0]}x{w.window[1]}x{w.window[2]} tokens")
+    elif w.mode == "svoo":
+        desc = (f"{w.name}: SVOO co-clustered block-sparse attention B={w.batch} H={w.heads} d={w.d} "
+                f"N={w.n_pad} ({w.n_valid} valid, {w.frames} frames of {w.fh}x{w.fw}), {w.clusters[0]} query + "
+                f"{w.clusters[1]} key clusters from sampled anchors, {w.iters} iterations, top "
+                f"{int(round(w.keep_frac * 100))}% key blocks per query block; one call = co-clustering + attention")
     else:
         desc = (f"{w.name}: gated tile neighbourhood + far field B={w.batch} H={w.heads} d={w.d} "
                 f"{w.frames}x{w.fh}x{w.fw}={w.n_pad} tokens, 4x4x4 tiles, 3x3x3 tile neighbourhood, "
@@ -148,6 +153,12 @@ def tile3d_flops(w):
     pairs = extent_sum(tf) * extent_sum(th) * extent_sum(tw)
     far = tf * th * tw
     return 4.0 * 64 * 64 * w.d * (pairs + far) * w.heads * w.batch, pairs
+
+
+def svoo_flops(w, kc):
+    """FLOPs of one SVOO attention on computed blocks: 4*64*64*d per kept (query block,
+    key block) pair, kc pairs per query block."""
+    return 4.0 * 64 * 64 * w.d * w.n_blocks * kc * w.heads * w.batch
 
 
 def sta_flops(w):
@@ -246,6 +257,7 @@ def cpu_oracle_sample(w, q, k, v, wp, rows_per_head=256, heads=12, phi="elu1"):
     from oracle import lvsa as olvsa
     from oracle import sla as osla
     from oracle import sta as osta
+    from oracle import svoo as osvoo
     from oracle import tile3d as otile
     heads = min(heads, w.heads)
     nb = w.n_blocks
@@ -288,6 +300,22 @@ def cpu_oracle_sample(w, q, k, v, wp, rows_per_head=256, heads=12, phi="elu1"):
             per_rows += t2 - t1
         what = (f"attention_sets in full, then frame_mask_attention for {rows_per_head} of {nb} query "
                 f"blocks (step {step})")
+    elif w.mode == "svoo":
+        valid = osla.valid_tokens(w.n_seg, w.seg_len, w.seg_stride)
+        qa, ka = workloads.make_anchors(w, "q", heads), workloads.make_anchors(w, "k", heads)
+        for h in range(heads):
+            qh, kh, vh = (f64(x[0, h]) for x in (q, k, v))
+            t0 = time.perf_counter()
+            ql, kl = osvoo.co_cluster(qh, kh, qa[0, h].numpy(), ka[0, h].numpy(), iters=w.iters, valid=valid)
+            qp, kp = osvoo.cluster_order(ql, w.clusters[0]), osvoo.cluster_order(kl, w.clusters[1])
+            mask, _ = osvoo.block_selection(qh[qp], kh[kp], valid, w.keep_frac)
+            t1 = time.perf_counter()
+            osvoo.svoo_attention(qh, kh, vh, qp, kp, w.keep_frac, valid=valid, rows=rows, mask=mask)
+            t2 = time.perf_counter()
+            fixed += t1 - t0
+            per_rows += t2 - t1
+        what = (f"co_cluster ({w.iters} iterations), cluster_order and block_selection in full, then "
+                f"svoo_attention for {rows_per_head} of {nb} query blocks")
     elif w.mode == "sta":
         toks = sorted(rng.choice(w.n_pad, rows_per_head * 64, replace=False).tolist())
         for h in range(heads):
@@ -340,8 +368,12 @@ class Runner:
             self.masks = [slr.tile3d_mask(w.frames, w.fh, w.fw, w.radius, w.cell, w.gate, rope=w.rope)]
         elif w.mode == "sta":
             self.masks = [slr.sta_mask(w.frames, w.fh, w.fw, w.window)]
+        elif w.mode == "svoo":
+            self.qa_h, self.ka_h = workloads.make_anchors(w, "q"), workloads.make_anchors(w, "k")
+            self.qa, self.ka = self.qa_h.to(dev), self.ka_h.to(dev)
+            self.ws_cl = slr.Workspace(dev)
 
-    def call(self, i=0, o=None, q=None, k=None, v=None, wp=None, ws=None):
+    def call(self, i=0, o=None, q=None, k=None, v=None, wp=None, ws=None, anchors=None):
         slr, w = self.slr, self.w
         o = self.out if o is None else o
         q, k, v = (self.q if q is None else q), (self.k if k is None else k), (self.v if v is None else v)
@@ -349,6 +381,10 @@ class Runner:
         if w.mode == "sla":
             slr.slr_sparse_linear_attn(q, k, v, self.wp if wp is None else wp, self.seq, w.crit_frac, w.negl_frac,
                                        out=o, ws=ws, phi=self.phi)
+        elif w.mode == "svoo":
+            qa, ka = (self.qa, self.ka) if anchors is None else anchors
+            _, _, qp, kp = slr.slr_svoo_cocluster(q, k, self.seq, qa, ka, iters=w.iters, ws=self.ws_cl)
+            slr.slr_svoo_attn(q, k, v, self.seq, qp, kp, w.keep_frac, out=o, ws=ws)
         else:
             slr.slr_frame_mask_attn(q, k, v, self.seq, self.masks[i % len(self.masks)], out=o, ws=ws)
 
@@ -388,7 +424,10 @@ class Runner:
         return self.sdist.max_over_ranks(total, device=self.dev), statistics.median(ts), min(ts)
 
     def status_ok(self):
-        return self.slr.slr_check_status(self.ws, self.dev) == self.slr.SLR_OK
+        ok = self.slr.slr_check_status(self.ws, self.dev) == self.slr.SLR_OK
+        if self.w.mode == "svoo":
+            ok = ok and self.slr.slr_check_status(self.ws_cl, self.dev) == self.slr.SLR_OK
+        return ok
 
     def work(self):
         """(FLOPs of the dominant kernel per call, all FLOPs on computed blocks, details)."""
@@ -405,6 +444,10 @@ class Runner:
         if w.mode == "sta":
             f, pairs = sta_flops(w)
             return f, f, {"tile_pairs_per_head": pairs, "computed_tflop": f / 1e12}
+        if w.mode == "svoo":
+            kc, _ = slr.slr_block_counts(w.n_blocks, w.keep_frac, 0.0)
+            f = svoo_flops(w, kc)
+            return f, f, {"kc": kc, "computed_tflop": f / 1e12, "clusters": list(w.clusters), "iters": w.iters}
         f, pairs = tile3d_flops(w)
         return f, f, {"local_tile_pairs_per_head": pairs, "computed_tflop": f / 1e12}
 
@@ -468,6 +511,10 @@ class Runner:
         dq, dk, dv, dw, do = (torch.empty_like(x, device=self.dev) for x in (self.q_h, self.k_h, self.v_h,
                                                                                self.wp_h, self.out))
         sla = self.w.mode == "sla"
+        svoo = self.w.mode == "svoo"
+        if svoo:     # the sampled anchor tokens are inputs of the call too
+            hqa, hka = self.qa_h.pin_memory(), self.ka_h.pin_memory()
+            dqa, dka = torch.empty_like(hqa, device=self.dev), torch.empty_like(hka, device=self.dev)
 
         def step(i):
             dq.copy_(hq, non_blocking=True)
@@ -475,19 +522,24 @@ class Runner:
             dv.copy_(hv, non_blocking=True)
             if sla:
                 dw.copy_(hw, non_blocking=True)
-            self.call(i, o=do, q=dq, k=dk, v=dv, wp=dw)
+            if svoo:
+                dqa.copy_(hqa, non_blocking=True)
+                dka.copy_(hka, non_blocking=True)
+            self.call(i, o=do, q=dq, k=dk, v=dv, wp=dw, anchors=(dqa, dka) if svoo else None)
             ho.copy_(do, non_blocking=True)
 
         for i in range(2):
             step(i)
         ms, _, _ = self.timed(step, max(3, steps // 4))
         h2d = sum(x.numel() * x.element_size() for x in ((hq, hk, hv, hw) if sla else (hq, hk, hv)))
+        if svoo:
+            h2d += sum(x.numel() * x.element_size() for x in (hqa, hka))
         d2h = ho.numel() * ho.element_size()
         return {"value": round(self.sdist.aggregate_ms_per_call(ms, self.world), 4), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
     def release(self):
-        for name in ("q", "k", "v", "wp", "out", "flush", "ws", "ws_dense"):
+        for name in ("q", "k", "v", "wp", "out", "flush", "ws", "ws_dense", "ws_cl", "qa", "ka"):
             setattr(self, name, None)
         torch.cuda.empty_cache()
 
@@ -507,10 +559,15 @@ def main():
                     help="feature map of the linear branch of the SLA workloads")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--oracle-rows", type=int, default=256, help="query blocks per head in the CPU oracle sample")
-    ap.add_argument("--oracle-heads", type=int, default=12, help="heads in the CPU oracle sample")
+    ap.add_argument("--oracle-rows", type=int, default=None,
+                    help="query blocks per head in the CPU oracle sample (default 256; 64 for svoo)")
+    ap.add_argument("--oracle-heads", type=int, default=None,
+                    help="heads in the CPU oracle sample (default 12; 2 for svoo, whose co-clustering runs in full)")
     args = ap.parse_args()
     w = workloads.BY_NAME[args.workload]
+    small = w.mode == "svoo"
+    args.oracle_rows = args.oracle_rows or (64 if small else 256)
+    args.oracle_heads = args.oracle_heads or (2 if small else 12)
     warmup = max(3, args.warmup)
 
     from block_sparse_linear_02_b200 import dist as sdist

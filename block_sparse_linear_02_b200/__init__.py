@@ -7,8 +7,8 @@ arithmetic happens in the library's kernels; there is no fallback path, and a
 missing ``libslr.so`` raises immediately.
 
 Function names match the C entry points: ``slr_pool_classify``,
-``slr_block_sparse_attn``, ``slr_linear_marginal``, ``slr_sparse_linear_attn``
-and ``slr_frame_mask_attn``; host helpers ``slr_block_counts``,
+``slr_block_sparse_attn``, ``slr_linear_marginal``, ``slr_sparse_linear_attn``,
+``slr_frame_mask_attn``, ``slr_svoo_cocluster`` and ``slr_svoo_attn``; host helpers ``slr_block_counts``,
 ``slr_lvsa_attention_sets``, ``slr_workspace_bytes`` and ``slr_check_status``.
 """
 from __future__ import annotations
@@ -32,19 +32,21 @@ SLR_PHI_SOFTMAX = 1
 SLR_MASK_LVSA = 1
 SLR_MASK_TILE3D = 2
 SLR_MASK_STA = 3
-ABI_VERSION = 200          # include/slr.h SLR_ABI_VERSION
+ABI_VERSION = 201          # include/slr.h SLR_ABI_VERSION
 
 SLR_OP_POOL_CLASSIFY = 1
 SLR_OP_BLOCK_SPARSE = 2
 SLR_OP_LINEAR_MARGINAL = 3
 SLR_OP_SPARSE_LINEAR = 4
 SLR_OP_FRAME_MASK = 5
+SLR_OP_SVOO_COCLUSTER = 6
+SLR_OP_SVOO_ATTN = 7
 
 EXPORTS = (
     "slr_pool_classify", "slr_block_sparse_attn", "slr_linear_marginal", "slr_sparse_linear_attn",
     "slr_frame_mask_attn", "slr_workspace_bytes", "slr_check_status", "slr_block_counts",
     "slr_lvsa_attention_sets", "slr_status_string", "slr_version", "slr_profile_enable",
-    "slr_profile_collect", "slr_block_sparse_attn_noalloc",
+    "slr_profile_collect", "slr_block_sparse_attn_noalloc", "slr_svoo_cocluster", "slr_svoo_attn",
 )
 
 
@@ -89,6 +91,8 @@ def lib() -> ctypes.CDLL:
         L.slr_frame_mask_attn.argtypes = [vp, vp, vp, seqp, maskp, vp, vp, sz, vp]
         L.slr_block_sparse_attn_noalloc.argtypes = [vp, vp, vp, seqp, vp, vp, i, vp, vp, vp, vp]
         L.slr_block_sparse_attn_noalloc.restype = i
+        L.slr_svoo_cocluster.argtypes = [vp, vp, seqp, i, i, i, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.slr_svoo_attn.argtypes = [vp, vp, vp, seqp, vp, vp, f, vp, vp, vp, sz, vp]
         L.slr_workspace_bytes.argtypes = [i, seqp, vp]
         L.slr_workspace_bytes.restype = sz
         L.slr_check_status.argtypes = [vp, vp]
@@ -104,7 +108,8 @@ def lib() -> ctypes.CDLL:
         L.slr_profile_collect.restype = i
         for name in ("slr_pool_classify", "slr_block_sparse_attn", "slr_linear_marginal",
                      "slr_sparse_linear_attn", "slr_frame_mask_attn", "slr_check_status",
-                     "slr_block_counts", "slr_lvsa_attention_sets", "slr_version"):
+                     "slr_block_counts", "slr_lvsa_attention_sets", "slr_version", "slr_svoo_cocluster",
+                     "slr_svoo_attn"):
             getattr(L, name).restype = i
         if L.slr_version() != ABI_VERSION:
             # the structs above mirror include/slr.h of this version; an older build would read them wrongly
@@ -376,3 +381,45 @@ def slr_block_sparse_attn_noalloc(q, k, v, seq: SlrSeq, kv_idx=None, kv_cnt=None
                                                _ptr(kv_cnt), kv_max, _ptr(o), _ptr(l), _ptr(status), _stream(q)),
            "slr_block_sparse_attn_noalloc")
     return o, l
+
+
+def slr_svoo_cocluster(q, k, seq: SlrSeq, q_anchor, k_anchor, iters: int = 2, ws=None):
+    """SVOO's bidirectional co-clustering from anchor tokens (int32 [B, H, n_qc] and
+    [B, H, n_kc]); returns (q_label, k_label, q_perm, k_perm), each int32 [B, H, N_pad]."""
+    import torch
+    _check_qkv(q, k)
+    for a in (q_anchor, k_anchor):
+        if a.dtype != torch.int32 or not a.is_cuda or a.dim() != 3 or tuple(a.shape[:2]) != (seq.B, seq.H):
+            raise ValueError("anchors must be int32 CUDA tensors [B, H, clusters]")
+    q_anchor, k_anchor = q_anchor.contiguous(), k_anchor.contiguous()
+    n_qc, n_kc = q_anchor.shape[-1], k_anchor.shape[-1]
+    dev = q.device
+    shape = (seq.B, seq.H, seq.n_seg * seq.seg_stride)
+    ql, kl, qp, kp = (torch.empty(shape, dtype=torch.int32, device=dev) for _ in range(4))
+    need = slr_workspace_bytes(SLR_OP_SVOO_COCLUSTER, seq, (ctypes.c_int * 2)(n_qc, n_kc))
+    wp, wn = _ws(ws, dev).get(need, dev)
+    _check(lib().slr_svoo_cocluster(_ptr(q), _ptr(k), ctypes.byref(seq), n_qc, n_kc, iters, _ptr(q_anchor),
+                                    _ptr(k_anchor), _ptr(ql), _ptr(kl), _ptr(qp), _ptr(kp), wp, wn, _stream(q)),
+           "slr_svoo_cocluster")
+    return ql, kl, qp, kp
+
+
+def slr_svoo_attn(q, k, v, seq: SlrSeq, q_perm, k_perm, keep_frac: float, out=None, mask_out: bool = False,
+                  ws=None):
+    """Attention over the top keep_frac of the key blocks of the co-clustered orders
+    (int32 [B, H, N_pad] permutations); returns (out bf16 in token order, mask int8 or None)."""
+    import torch
+    _check_qkv(q, k, v)
+    for p_ in (q_perm, k_perm):
+        if p_.dtype != torch.int32 or not p_.is_cuda or tuple(p_.shape) != tuple(q.shape[:3]):
+            raise ValueError("permutations must be int32 CUDA tensors [B, H, N_pad]")
+    q_perm, k_perm = q_perm.contiguous(), k_perm.contiguous()
+    dev = q.device
+    o = torch.empty_like(q) if out is None else out
+    nb = seq.n_seg * seq.seg_stride // 64
+    m = torch.empty(seq.B, seq.H, nb, nb, dtype=torch.int8, device=dev) if mask_out else None
+    need = slr_workspace_bytes(SLR_OP_SVOO_ATTN, seq, ctypes.c_float(keep_frac))
+    wp, wn = _ws(ws, dev).get(need, dev)
+    _check(lib().slr_svoo_attn(_ptr(q), _ptr(k), _ptr(v), ctypes.byref(seq), _ptr(q_perm), _ptr(k_perm),
+                               keep_frac, _ptr(o), _ptr(m), wp, wn, _stream(q)), "slr_svoo_attn")
+    return o, m

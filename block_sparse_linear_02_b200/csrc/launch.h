@@ -143,6 +143,37 @@ cudaError_t launch_reduce_states(const __nv_bfloat16* m01, int ld_m01, const __n
                                  __nv_bfloat16* Hs, int BH, int nb, int d, int* status, cudaStream_t st);
 
 // o_lin[bh][t] = phi(q_t) H_i' / (phi(q_t).Z_i) for every valid token t of block i (0 for pads).
+// ------------------------------------------------------------ SVOO co-clustering (k_svoo.cu)
+// Cluster counts are padded to Cp = the power of two >= max(C, 32); C <= kSvooMaxClusters.
+// Centres are fp32 [BH][Cp][d]; ub bf16 [BH][Cp][3d] and bias fp32 [BH][Cp] hold the metric
+// of the assigning side; labels and perm are int32 [BH][n_pad]; counts and offs int32
+// [BH][svoo_sort_chunks(n_pad)][C + 1] (counts zero before the first assignment; the sort
+// clears them again); start int32 [BH][C + 2].
+constexpr int kSvooMaxClusters = 128;
+int svoo_padded_clusters(int C);
+int svoo_sort_chunks(int n_pad);
+// centres[n] = x[anchor[n]] (an anchor that is not a valid token sets SLR_ERR_INDEX)
+cudaError_t launch_svoo_anchors(const void* x, const int32_t* anchor, float* centres, int C, int BH, int d,
+                                SeqShape s, int* status, cudaStream_t st);
+// labels of the tokens of x: the own centre (of C_own) whose affinity vector against the
+// C_other centres of the other side is nearest (pads: C_own); label histogram into counts
+cudaError_t launch_svoo_assign(const void* x, const float* other, int C_other, float* own, int C_own,
+                               __nv_bfloat16* ub, float* bias, int32_t* labels, int32_t* counts, int BH, int d,
+                               SeqShape s, int* status, cudaStream_t st);
+// the stable order of the labels: perm (position -> token) and the cluster starts
+cudaError_t launch_svoo_sort(const int32_t* labels, int32_t* counts, int32_t* offs, int32_t* start, int32_t* perm,
+                             int C, int BH, SeqShape s, cudaStream_t st);
+// centres = means of their tokens (an empty cluster keeps its centre)
+cudaError_t launch_svoo_update(const void* x, const int32_t* perm, const int32_t* start, float* centres, int C,
+                               int BH, int d, SeqShape s, cudaStream_t st);
+// qp[p] = q[q_perm[p]], kp[p] = k[k_perm[p]], vp[p] = v[k_perm[p]] (bf16 rows of d)
+cudaError_t launch_svoo_gather(const void* q, const void* k, const void* v, const int32_t* q_perm,
+                               const int32_t* k_perm, void* qp, void* kp, void* vp, int BH, int d, int n_pad,
+                               int* status, cudaStream_t st);
+// out[q_perm[p]] = src[p]
+cudaError_t launch_svoo_scatter_rows(const void* src, const int32_t* q_perm, void* out, int BH, int d, int n_pad,
+                                     int* status, cudaStream_t st);
+
 // ------------------------------------------------------------ no-workspace call (slr_noalloc.cu)
 // Reads and clears the status word of the static scratch on the current device.
 int noalloc_check_status(void* stream);   // an slr_status value

@@ -264,6 +264,56 @@ void plan_frame(Carve& c, const Shape& sh, const slr_mask_desc* m, FrameWs& w) {
   w.list_cnt = c.take<int32_t>((size_t)sh.npairs);
 }
 
+struct SvooClusterWs {
+  int* status;
+  float *cq, *ck;                      // centres [BH][Cp][d]
+  __nv_bfloat16* ub;                   // metric of the assigning side [BH][Cp][3d]
+  float* bias;                         // [BH][Cp]
+  int32_t *counts, *offs, *start;      // counting sort
+};
+
+void plan_svoo_cluster(Carve& c, const Shape& sh, int n_qc, int n_kc, SvooClusterWs& w) {
+  const int cpq = svoo_padded_clusters(n_qc), cpk = svoo_padded_clusters(n_kc);
+  const int cpm = cpq > cpk ? cpq : cpk, cm = n_qc > n_kc ? n_qc : n_kc;
+  const size_t nch = (size_t)svoo_sort_chunks(sh.n_pad);
+  w.status = c.take<int>(64);
+  w.cq = c.take<float>((size_t)sh.BH * cpq * sh.d);
+  w.ck = c.take<float>((size_t)sh.BH * cpk * sh.d);
+  w.ub = c.take<__nv_bfloat16>((size_t)sh.BH * cpm * 3 * sh.d);
+  w.bias = c.take<float>((size_t)sh.BH * cpm);
+  w.counts = c.take<int32_t>((size_t)sh.BH * nch * (cm + 1));
+  w.offs = c.take<int32_t>((size_t)sh.BH * nch * (cm + 1));
+  w.start = c.take<int32_t>((size_t)sh.BH * (cm + 2));
+}
+
+struct SvooAttnWs {
+  int* status;
+  ClassifyWs cls;
+  uint32_t* list;
+  int32_t* list_cnt;
+  int cap;
+  void *qp, *kp, *vp, *op;             // the reordered q, k, v and the output in that order
+};
+
+void plan_svoo_attn(Carve& c, const Shape& sh, int kc, SvooAttnWs& w) {
+  w.status = c.take<int>(64);
+  const bool dense = kc == sh.nb;
+  w.cap = dense ? 0 : (2 * kc < sh.nb ? 2 * kc : sh.nb);
+  if (!dense) {
+    plan_classify(c, sh, false, w.cls);
+    w.list = c.take<uint32_t>((size_t)sh.BH * sh.npairs * w.cap);
+    w.list_cnt = c.take<int32_t>((size_t)sh.BH * sh.npairs);
+  } else {
+    w.list = nullptr;
+    w.list_cnt = nullptr;
+  }
+  const size_t rows = (size_t)sh.BH * sh.n_pad * sh.d;
+  w.qp = c.take<__nv_bfloat16>(rows);
+  w.kp = c.take<__nv_bfloat16>(rows);
+  w.vp = c.take<__nv_bfloat16>(rows);
+  w.op = c.take<__nv_bfloat16>(rows);
+}
+
 slr_status ws_check(void* ws, size_t have, size_t need) {
   if (!ws || (reinterpret_cast<uintptr_t>(ws) & (kAlign - 1))) return SLR_ERR_WORKSPACE;
   if (have < need) return SLR_ERR_WORKSPACE;
@@ -278,11 +328,13 @@ slr_status ws_check(void* ws, size_t have, size_t need) {
 // ---------------------------------------------------------------- per-kernel profiler
 enum KernelKind {
   kKPool, kKLogits, kKClassify, kKLists, kKKeyStates, kKReduce, kKApply, kKAttention, kKLvsaSets,
-  kKFarPool, kKMaskToM01, kKTileMajor, kKNumKinds
+  kKFarPool, kKMaskToM01, kKTileMajor, kKSvooAnchors, kKSvooAssign, kKSvooSort, kKSvooUpdate, kKSvooGather,
+  kKSvooScatter, kKNumKinds
 };
 const char* const kKindNames[kKNumKinds] = {
     "pool_means", "logits", "classify", "pair_lists", "key_states", "reduce_states",
-    "linear_apply", "attention", "lvsa_sets", "far_pool", "mask_to_m01", "tile_major"};
+    "linear_apply", "attention", "lvsa_sets", "far_pool", "mask_to_m01", "tile_major",
+    "svoo_anchors", "svoo_assign", "svoo_sort", "svoo_update", "svoo_gather", "svoo_scatter"};
 
 struct ProfRec {
   int kind;
@@ -454,6 +506,24 @@ size_t slr_workspace_bytes(int op, const slr_seq* seq, const void* params) {
       if (check_mask(m, sh) != SLR_OK) return 0;
       FrameWs w;
       plan_frame(c, sh, m, w);
+      return c.off;
+    }
+    case SLR_OP_SVOO_COCLUSTER: {
+      const int* cl = static_cast<const int*>(params);
+      if (!cl || sh.n_seg != 1) return 0;
+      if (cl[0] < 2 || cl[0] > kSvooMaxClusters || cl[1] < 2 || cl[1] > kSvooMaxClusters) return 0;
+      SvooClusterWs w;
+      plan_svoo_cluster(c, sh, cl[0], cl[1], w);
+      return c.off;
+    }
+    case SLR_OP_SVOO_ATTN: {
+      const float* keep = static_cast<const float*>(params);
+      if (!keep || sh.n_seg != 1) return 0;
+      int kc, kn;
+      if (!(*keep > 0.f) || counts(sh.nb, *keep, 0.f, &kc, &kn) != SLR_OK) return 0;
+      if (kc != sh.nb && sh.nb > kMaxClassifyBlocks) return 0;
+      SvooAttnWs w;
+      plan_svoo_attn(c, sh, kc, w);
       return c.off;
     }
     default:
@@ -640,6 +710,80 @@ slr_status slr_frame_mask_attn(const void* q, const void* k, const void* v, cons
   SLR_LAUNCH(kKLists, s, launch_pair_lists(la, 1, s));
   a.list = w.list; a.list_cnt = w.list_cnt; a.list_cap = w.cap; a.list_per_head = 0;
   SLR_LAUNCH(kKAttention, s, launch_attention(a, s));
+  return SLR_OK;
+}
+
+slr_status slr_svoo_cocluster(const void* q, const void* k, const slr_seq* seq, int n_qc, int n_kc, int iters,
+                              const int32_t* q_anchor, const int32_t* k_anchor, int32_t* q_label, int32_t* k_label,
+                              int32_t* q_perm, int32_t* k_perm, void* ws, size_t ws_bytes, void* stream) {
+  Shape sh;
+  slr_status st = check_seq(seq, sh);
+  if (st != SLR_OK) return st;
+  if (sh.n_seg != 1) return SLR_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !q_anchor || !k_anchor || !q_label || !k_label || !q_perm || !k_perm)
+    return SLR_ERR_ARG;
+  if (n_qc < 2 || n_qc > kSvooMaxClusters || n_kc < 2 || n_kc > kSvooMaxClusters || iters < 1) return SLR_ERR_ARG;
+  const int cl[2] = {n_qc, n_kc};
+  if ((st = ws_check(ws, ws_bytes, slr_workspace_bytes(SLR_OP_SVOO_COCLUSTER, seq, cl))) != SLR_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  Carve c(ws);
+  SvooClusterWs w;
+  plan_svoo_cluster(c, sh, n_qc, n_kc, w);
+  const int cm = n_qc > n_kc ? n_qc : n_kc;
+  SLR_TRY(cudaMemsetAsync(w.status, 0, sizeof(int), s));
+  SLR_TRY(cudaMemsetAsync(w.counts, 0, (size_t)sh.BH * svoo_sort_chunks(sh.n_pad) * (cm + 1) * sizeof(int32_t), s));
+  SLR_LAUNCH(kKSvooAnchors, s, launch_svoo_anchors(q, q_anchor, w.cq, n_qc, sh.BH, sh.d, sh.s, w.status, s));
+  SLR_LAUNCH(kKSvooAnchors, s, launch_svoo_anchors(k, k_anchor, w.ck, n_kc, sh.BH, sh.d, sh.s, w.status, s));
+  for (int it = 0; it < iters; ++it) {
+    // step A: the keys against the query centres, then the key centres move
+    SLR_LAUNCH(kKSvooAssign, s, launch_svoo_assign(k, w.cq, n_qc, w.ck, n_kc, w.ub, w.bias, k_label, w.counts,
+                                                   sh.BH, sh.d, sh.s, w.status, s));
+    SLR_LAUNCH(kKSvooSort, s, launch_svoo_sort(k_label, w.counts, w.offs, w.start, k_perm, n_kc, sh.BH, sh.s, s));
+    SLR_LAUNCH(kKSvooUpdate, s, launch_svoo_update(k, k_perm, w.start, w.ck, n_kc, sh.BH, sh.d, sh.s, s));
+    // step B: the queries against the updated key centres
+    SLR_LAUNCH(kKSvooAssign, s, launch_svoo_assign(q, w.ck, n_kc, w.cq, n_qc, w.ub, w.bias, q_label, w.counts,
+                                                   sh.BH, sh.d, sh.s, w.status, s));
+    SLR_LAUNCH(kKSvooSort, s, launch_svoo_sort(q_label, w.counts, w.offs, w.start, q_perm, n_qc, sh.BH, sh.s, s));
+    if (it + 1 < iters)
+      SLR_LAUNCH(kKSvooUpdate, s, launch_svoo_update(q, q_perm, w.start, w.cq, n_qc, sh.BH, sh.d, sh.s, s));
+  }
+  return SLR_OK;
+}
+
+slr_status slr_svoo_attn(const void* q, const void* k, const void* v, const slr_seq* seq, const int32_t* q_perm,
+                         const int32_t* k_perm, float keep_frac, void* out, int8_t* mask_out_opt, void* ws,
+                         size_t ws_bytes, void* stream) {
+  Shape sh;
+  slr_status st = check_seq(seq, sh);
+  if (st != SLR_OK) return st;
+  if (sh.n_seg != 1) return SLR_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !q_perm || !k_perm) return SLR_ERR_ARG;
+  if (!(keep_frac > 0.f && keep_frac <= 1.f)) return SLR_ERR_ARG;
+  int kc, kn;
+  if ((st = counts(sh.nb, keep_frac, 0.f, &kc, &kn)) != SLR_OK) return st;
+  const bool dense = kc == sh.nb;
+  if (!dense && sh.nb > kMaxClassifyBlocks) return SLR_ERR_UNSUPPORTED;
+  if ((st = ws_check(ws, ws_bytes, slr_workspace_bytes(SLR_OP_SVOO_ATTN, seq, &keep_frac))) != SLR_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  Carve c(ws);
+  SvooAttnWs w;
+  plan_svoo_attn(c, sh, kc, w);
+  SLR_TRY(cudaMemsetAsync(w.status, 0, sizeof(int), s));
+  SLR_LAUNCH(kKSvooGather, s, launch_svoo_gather(q, k, v, q_perm, k_perm, w.qp, w.kp, w.vp, sh.BH, sh.d, sh.n_pad,
+                                                 w.status, s));
+  AttnArgs a = attn_base(sh, w.qp, w.kp, w.vp, w.op, w.status);
+  if (dense) {
+    if (mask_out_opt) SLR_TRY(cudaMemsetAsync(mask_out_opt, 1, (size_t)sh.BH * sh.nb * sh.nb, s));
+  } else {
+    SLR_LAUNCH(kKPool, s, launch_pool_means(w.qp, w.kp, w.cls.qsplit, w.cls.ksplit, nullptr, SLR_PHI_ELU1, sh.BH,
+                                            sh.d, sh.s, s));
+    SLR_LAUNCH(kKLogits, s, launch_logits(w.cls.qsplit, w.cls.ksplit, w.cls.keys, sh.BH, sh.nb, sh.d, w.status, s));
+    SLR_LAUNCH(kKClassify, s, launch_classify(w.cls.keys, sh.BH, sh.nb, sh.d, kc, 0, mask_out_opt, nullptr, nullptr,
+                                              nullptr, 0, nullptr, w.list, w.list_cnt, w.cap, sh.s, w.status, s));
+    a.list = w.list; a.list_cnt = w.list_cnt; a.list_cap = w.cap; a.list_per_head = 1;
+  }
+  SLR_LAUNCH(kKAttention, s, launch_attention(a, s));
+  SLR_LAUNCH(kKSvooScatter, s, launch_svoo_scatter_rows(w.op, q_perm, out, sh.BH, sh.d, sh.n_pad, w.status, s));
   return SLR_OK;
 }
 

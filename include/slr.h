@@ -3,12 +3,14 @@
  * (frame x height x width) token sequence of a video diffusion transformer,
  * hand-written for NVIDIA B200 (sm_100a).
  *
- * The operations follow three source write-ups:
+ * The operations follow these source write-ups:
  *  - SLA (Sparse-Linear Attention, arXiv 2509.24006), techwalker page
  *    "清华大学破解视频生成卡顿难题", section 3 "SLA方法的核心机制";
  *  - LVSA (arXiv 2605.31057), rainbus paper digest, sections "核心方法" and
  *    "方法步骤详情";
- *  - RoPeSLR (arXiv 2605.20659), aixinbiao blog, section "稀疏邻域加低秩远场".
+ *  - RoPeSLR (arXiv 2605.20659), aixinbiao blog, section "稀疏邻域加低秩远场";
+ *  - VORTA (arXiv 2505.18809), zhaoyang97 paper notes, section "方法详解";
+ *  - SVOO (arXiv 2603.18636), gist.science summary, section 3.
  *
  * Conventions shared by every compute entry point
  * ------------------------------------------------
@@ -99,6 +101,8 @@ typedef struct {
 #define SLR_OP_LINEAR_MARGINAL 3   /* params: unused (NULL)                        */
 #define SLR_OP_SPARSE_LINEAR   4   /* params: const slr_fracs*                     */
 #define SLR_OP_FRAME_MASK      5   /* params: const slr_mask_desc*                 */
+#define SLR_OP_SVOO_COCLUSTER  6   /* params: const int[2] {n_qc, n_kc}            */
+#define SLR_OP_SVOO_ATTN       7   /* params: const float* keep_frac               */
 
 /* ------------------------------------------------------------------ compute */
 
@@ -222,6 +226,71 @@ slr_status slr_frame_mask_attn(const void* q, const void* k, const void* v, cons
                                void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * slr_svoo_cocluster -- SVOO's online bidirectional co-clustering (gist.science
+ * summary of SVOO, arXiv 2603.18636, section 3, stage 2).  Per (b, h): query
+ * centres start at the anchor queries and key centres at the anchor keys; then
+ * `iters` times
+ *   step A: every valid key gets the label of the key centre whose affinity
+ *           vector (its dot products with the query centres) is nearest in
+ *           Euclidean distance to the key's own affinity vector (ties: the lower
+ *           centre); each key centre moves to the mean of its keys (a centre
+ *           with no key stays);
+ *   step B: the same for every valid query against the key centres of step A,
+ *           and the query centres move to their means.
+ * Pad tokens get the label n_qc (queries) or n_kc (keys).  The permutations list
+ * the tokens by ascending label, in token order within a label (a stable sort),
+ * so that pads end them: they are the orders slr_svoo_attn takes.
+ * Precision: the centres and their metric are formed in fp64 and kept in fp32;
+ * the distances of the tokens to the centres come from the tensor cores with the
+ * metric split into three bf16 terms (24 significant bits) and fp32
+ * accumulation, so a label can differ from an exact evaluation only for a token
+ * whose two nearest centres are within ~1e-6 (relative) of each other.  The call
+ * is deterministic: the same inputs give the same outputs.
+ *
+ *   q, k        bf16 [B][H][N_pad][d] device, read only
+ *   n_qc, n_kc  cluster counts, 2..128
+ *   iters       iterations, >= 1 (the summary: about 2)
+ *   q_anchor    int32 [B][H][n_qc] device: a valid query token per query centre
+ *   k_anchor    int32 [B][H][n_kc] device: a valid key token per key centre
+ *   q_label, k_label  int32 [B][H][N_pad] device, written
+ *   q_perm, k_perm    int32 [B][H][N_pad] device, written: position -> token
+ * Requires n_seg == 1 (one padded segment).  An anchor that is not a valid token
+ * sets SLR_ERR_INDEX in the status word (its centre starts at 0).
+ */
+slr_status slr_svoo_cocluster(const void* q, const void* k, const slr_seq* seq, int n_qc, int n_kc, int iters,
+                              const int32_t* q_anchor, const int32_t* k_anchor,
+                              int32_t* q_label, int32_t* k_label, int32_t* q_perm, int32_t* k_perm,
+                              void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * slr_svoo_attn -- softmax attention over the top block pairs of a co-clustered
+ * order (SVOO summary, section 3, stage 2, block selection).  The rows of q are
+ * taken in the order q_perm and those of k and v in the order k_perm; blocks are
+ * 64 consecutive rows of those orders.  Within every query block the key blocks
+ * are ranked by the SLA compressed score (as slr_pool_classify: block means,
+ * softmax(pool(Q) pool(K)^T / sqrt(d)), ties to the lower index) and the top
+ * kc = max(1, ceil(keep_frac * Nb)) are computed with exact softmax attention,
+ * scale 1/sqrt(d); the others are skipped.  keep_frac = 1 computes every block
+ * (the dense attention of the sequence, whatever the orders).  The output is
+ * written back in the original token order.
+ *
+ *   q_perm, k_perm  int32 [B][H][N_pad] device: permutations of the tokens whose
+ *                   first seg_len positions are the valid tokens (as
+ *                   slr_svoo_cocluster writes them); an entry outside [0, N_pad)
+ *                   sets SLR_ERR_INDEX; entries that repeat a token leave some
+ *                   output rows unwritten
+ *   keep_frac       in (0, 1]
+ *   out             bf16 [B][H][N_pad][d] device, written (pad rows 0)
+ *   mask_out_opt    int8 [B][H][Nb][Nb] device or NULL: 1 = computed pair, 0 =
+ *                   skipped, over the blocks of the two orders
+ * Requires n_seg == 1 and Nb <= 4096.  The workspace holds the reordered q, k, v
+ * and output (4 x B*H*N_pad*d bf16).
+ */
+slr_status slr_svoo_attn(const void* q, const void* k, const void* v, const slr_seq* seq,
+                         const int32_t* q_perm, const int32_t* k_perm, float keep_frac,
+                         void* out, int8_t* mask_out_opt, void* ws, size_t ws_bytes, void* stream);
+
+/*
  * slr_block_sparse_attn_noalloc -- slr_block_sparse_attn without a workspace.
  * The source pages have no counterpart to this call; it exists for callers
  * that cannot allocate device memory for the library: a host application that
@@ -297,8 +366,9 @@ int slr_profile_collect(const char** names, int* launches, double* total_ms, int
 
 const char* slr_status_string(slr_status s);
 /* ABI version, 100 * major + minor.  200: slr_mask_desc gained `rope` and `window` (and the
- * SLR_MASK_STA kind), so a caller built against an earlier header passes a shorter struct. */
-#define SLR_ABI_VERSION 200
+ * SLR_MASK_STA kind), so a caller built against an earlier header passes a shorter struct.
+ * 201: the SVOO calls slr_svoo_cocluster and slr_svoo_attn. */
+#define SLR_ABI_VERSION 201
 int slr_version(void);
 
 #ifdef __cplusplus

@@ -38,7 +38,7 @@ def test_exports_every_declared_symbol(lib):
 
 
 def test_version_and_strings(lib):
-    assert lib.slr_version() == 200            # slr_mask_desc with rope and window
+    assert lib.slr_version() == 201            # the SVOO calls
     for code in range(0, -7, -1):
         assert slr.status_string(code) not in ("", "unknown status")
 
@@ -159,3 +159,42 @@ def test_invalid_arguments_rejected_before_cuda(lib):
     # linear branch needs a mask
     assert lib.slr_linear_marginal(fake, fake, fake, ctypes.byref(seq), None, 0, None, fake, ws, 1 << 20,
                                    None) == slr.SLR_ERR_ARG
+
+
+def test_svoo_workspace_and_arguments(lib):
+    seq = slr.make_seq(1, 12, 128, 1, 32760, 32768)
+    cl = lambda a, b: (ctypes.c_int * 2)(a, b)
+    n = slr.slr_workspace_bytes(slr.SLR_OP_SVOO_COCLUSTER, seq, cl(64, 64))
+    # centres (fp32) and the metric (bf16, 3 terms) of up to 64 clusters, the sort counts
+    assert 2 * 12 * 64 * 128 * 4 < n < 8 << 20
+    for a, b in ((1, 64), (64, 129), (0, 0)):
+        assert slr.slr_workspace_bytes(slr.SLR_OP_SVOO_COCLUSTER, seq, cl(a, b)) == 0
+    two = slr.make_seq(1, 12, 128, 2, 16380, 16384)
+    assert slr.slr_workspace_bytes(slr.SLR_OP_SVOO_COCLUSTER, two, cl(64, 64)) == 0
+    rows = 12 * 32768 * 128 * 2
+    dense = slr.slr_workspace_bytes(slr.SLR_OP_SVOO_ATTN, seq, ctypes.c_float(1.0))
+    assert 4 * rows <= dense < 4 * rows + 4096          # the reordered q, k, v and output
+    sparse = slr.slr_workspace_bytes(slr.SLR_OP_SVOO_ATTN, seq, ctypes.c_float(0.2))
+    assert sparse > dense                                 # plus the classification and the lists
+    for bad in (0.0, -0.5, 1.5, float("nan")):
+        assert slr.slr_workspace_bytes(slr.SLR_OP_SVOO_ATTN, seq, ctypes.c_float(bad)) == 0
+    vp = ctypes.c_void_p
+    fake, ws = vp(0x1000), vp(0x100000)
+    small = slr.make_seq(1, 1, 64, 1, 256, 256)
+    args = lambda nq, nk, it, anc: (fake, fake, ctypes.byref(small), nq, nk, it, anc, anc, fake, fake, fake, fake,
+                                    ws, 1 << 30, None)
+    assert lib.slr_svoo_cocluster(*args(1, 4, 2, fake)) == slr.SLR_ERR_ARG
+    assert lib.slr_svoo_cocluster(*args(4, 200, 2, fake)) == slr.SLR_ERR_ARG
+    assert lib.slr_svoo_cocluster(*args(4, 4, 0, fake)) == slr.SLR_ERR_ARG
+    assert lib.slr_svoo_cocluster(*args(4, 4, 2, None)) == slr.SLR_ERR_ARG
+    assert lib.slr_svoo_cocluster(*args(4, 4, 2, fake)[:13], 16, None) == slr.SLR_ERR_WORKSPACE
+    segs = slr.make_seq(1, 1, 64, 2, 128, 128)
+    assert lib.slr_svoo_cocluster(fake, fake, ctypes.byref(segs), 4, 4, 2, fake, fake, fake, fake, fake, fake, ws,
+                                  1 << 30, None) == slr.SLR_ERR_UNSUPPORTED
+    for keep in (0.0, 1.25):
+        assert lib.slr_svoo_attn(fake, fake, fake, ctypes.byref(small), fake, fake, keep, fake, None, ws, 1 << 30,
+                                 None) == slr.SLR_ERR_ARG
+    assert lib.slr_svoo_attn(fake, fake, fake, ctypes.byref(small), None, fake, 0.5, fake, None, ws, 1 << 30,
+                             None) == slr.SLR_ERR_ARG
+    assert lib.slr_svoo_attn(fake, fake, fake, ctypes.byref(segs), fake, fake, 0.5, fake, None, ws, 1 << 30,
+                             None) == slr.SLR_ERR_UNSUPPORTED
