@@ -13,8 +13,10 @@ At one GPU the same run also measures the other workloads, each with its own
 dense-mode comparison, roofline and bounded CPU-oracle sample, under
 ``other_configs``: the HunyuanVideo-shaped SLA layer (24 heads, 115,200
 tokens), the LVSA frame mask (121 frames x 1,600 tokens, 12 heads, denoising
-steps 0..3 in turn) and the RoPeSLR-shaped gated tile neighbourhood + far field
-(16 heads, 8 x 64 x 64 tokens).  ``--workload NAME`` makes that workload the
+steps 0..3 in turn), the RoPeSLR-shaped gated tile neighbourhood + far field
+(16 heads, 8 x 64 x 64 tokens), VORTA's sliding tile attention on the same
+latent, and SVOO's co-clustering + attention over the top 20 % co-clustered block
+pairs on the Wan-shaped layer.  ``--workload NAME`` makes that workload the
 headline instead.
 
 Printed (rank 0, one JSON line): the device-timed ms per call (inputs resident
@@ -53,7 +55,7 @@ import torch  # noqa: E402
 import workloads  # noqa: E402
 
 WORKLOAD = workloads.WAN
-OTHER_WORKLOADS = (workloads.HUNYUAN, workloads.LVSA, workloads.ROPESLR)
+OTHER_WORKLOADS = (workloads.HUNYUAN, workloads.LVSA, workloads.ROPESLR, workloads.STA, workloads.SVOO)
 METRIC = "ms per sparse attn call & TFLOPS on computed blocks (% BF16 peak); speedup vs dense"
 UNIT = "ms/call"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -613,7 +615,7 @@ def main():
     clk = clocks.stop()
     if rank == 0 and not args.no_cpu_baseline:
         for ow, o in others:
-            rows = {"hunyuan": 16, "lvsa": 8, "ropeslr": 8}.get(ow.name, 16)
+            rows = {"hunyuan": 16, "lvsa": 8, "ropeslr": 8, "sta": 8, "svoo": 16}.get(ow.name, 16)
             qo, ko, vo = workloads.make_qkv(ow, heads=2)
             cms, desc, threads = cpu_oracle_sample(ow, qo, ko, vo, workloads.make_w_proj(ow), rows_per_head=rows,
                                                    heads=2, phi=args.phi)

@@ -16,13 +16,15 @@
 //   svoo_assign_kernel   the scores b_n - 2 x . u_n of 128 tokens against every centre
 //                        as one tcgen05 GEMM (M = 128 tokens, N = centres, K = 3d over
 //                        the three terms, fp32 accumulation in TMEM), then the argmin of
-//                        each row (ties to the lower centre) and a per-1024-token
-//                        histogram of the labels
+//                        each row (ties to the lower centre) and the label histogram of
+//                        each 1024-token chunk (one CTA per chunk: a ring of token tiles,
+//                        scores double-buffered in TMEM)
 //   svoo_scan_kernel     bucket offsets of every 1024-token chunk (exclusive scan)
 //   svoo_scatter_kernel  the stable order: position -> token, by ascending label and
 //                        then token index (the counting sort's second pass)
-//   svoo_update_kernel   each centre becomes the fp64 mean of its tokens, read in that
-//                        order; an empty cluster keeps its centre
+//   svoo_piece_kernel    fp64 sums of pieces of 256 consecutive positions of one cluster
+//   svoo_finalize_kernel each centre becomes the mean of its tokens (its pieces added in
+//                        order); an empty cluster keeps its centre
 // Every kernel is deterministic (no floating-point atomics), so a call repeated on the
 // same inputs returns the same labels.  Pad tokens take the label C and end the order.
 //
@@ -105,95 +107,99 @@ __global__ void __launch_bounds__(128) svoo_metric_kernel(const float* __restric
 }
 
 // ------------------------------------------------------------------ assignment
-// Shared memory of one CTA (offsets from a 1024-byte aligned base):
-//   A  D/64 chunks of 128 token rows x 64 bf16 (16 KB each), 128-byte swizzled
-//   B  3D/64 chunks of Cp centre rows x 64 bf16: the hi chunks, the mid chunks, the lo chunks
-//   then the Cp biases, the label histogram, two mbarriers, the TMEM slot and the abort flag
+// One CTA per 1024-token chunk of one head (8 tiles of 128 tokens), one CTA per SM.
+// Shared memory (offsets from a 1024-byte aligned base):
+//   X  a ring of kXStages token tiles, each D/64 chunks of 128 rows x 64 bf16 (16 KB),
+//      128-byte swizzled
+//   U  3D/64 chunks of Cp centre rows x 64 bf16: the hi chunks, the mid chunks, the lo
+//      chunks (loaded once: the chunk's head has one metric)
+//   then the Cp biases, the label histogram, the mbarriers, the TMEM slot, the abort flag
+// Thread 0 loads and issues the MMAs; tile i's scores go to TMEM columns (i & 1) * Cp, so
+// that the four warps' argmin of tile i - 1 overlaps the MMAs of tile i, and the load of
+// tile i + kXStages - 1 is issued as soon as the MMAs of tile i - 1 have read their stage.
 constexpr int kMaxClusters = 128;
 constexpr int kHistSlots = 160;       // >= kMaxClusters + 1 buckets
+constexpr int kAsgTiles = kSortChunk / kAsgRows;
+constexpr int kXStages = 3;
 template <int D>
 struct AsgLayout {
   static constexpr int kAChunks = D / 64;
   static constexpr int kBChunks = 3 * D / 64;
   static constexpr int kAChunkBytes = kAsgRows * 128;
+  static constexpr int kXBytes = kAChunks * kAChunkBytes;
   __host__ __device__ static size_t b_chunk_bytes(int Cp) { return (size_t)Cp * 128; }
-  __host__ __device__ static size_t bias_off(int Cp) { return (size_t)kAChunks * kAChunkBytes + kBChunks * b_chunk_bytes(Cp); }
-  __host__ __device__ static size_t bytes(int Cp) { return bias_off(Cp) + kMaxClusters * 4 + kHistSlots * 4 + 32 + 1024; }
+  __host__ __device__ static size_t u_off() { return (size_t)kXStages * kXBytes; }
+  __host__ __device__ static size_t bias_off(int Cp) { return u_off() + kBChunks * b_chunk_bytes(Cp); }
+  __host__ __device__ static size_t bytes(int Cp) { return bias_off(Cp) + kMaxClusters * 4 + kHistSlots * 4 + 128 + 1024; }
 };
 
 template <int D>
-__global__ void __launch_bounds__(128) svoo_assign_kernel(const __grid_constant__ CUtensorMap tmX,
-                                                          const __grid_constant__ CUtensorMap tmU,
-                                                          const float* __restrict__ bias, int C, int Cp,
-                                                          int32_t* __restrict__ labels, int32_t* __restrict__ counts,
-                                                          int n_chunks, SeqShape s, int* status) {
+__global__ void __launch_bounds__(128, 1) svoo_assign_kernel(const __grid_constant__ CUtensorMap tmX,
+                                                             const __grid_constant__ CUtensorMap tmU,
+                                                             const float* __restrict__ bias, int C, int Cp,
+                                                             int32_t* __restrict__ labels,
+                                                             int32_t* __restrict__ counts, int n_chunks, SeqShape s,
+                                                             int* status) {
   using L = AsgLayout<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t b_chunk = (uint32_t)L::b_chunk_bytes(Cp);
-  uint8_t* sA = smem;
-  uint8_t* sB = smem + L::kAChunks * L::kAChunkBytes;
+  uint8_t* sX = smem;
+  uint8_t* sU = smem + L::u_off();
   float* sbias = reinterpret_cast<float*>(smem + L::bias_off(Cp));
   int* hist = reinterpret_cast<int*>(sbias + kMaxClusters);
-  uint64_t* full = reinterpret_cast<uint64_t*>(hist + kHistSlots);
-  uint64_t* done = full + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  uint64_t* x_full = reinterpret_cast<uint64_t*>(hist + kHistSlots);   // [kXStages]
+  uint64_t* u_full = x_full + kXStages;
+  uint64_t* mma_done = u_full + 1;                                     // [2]
+  uint64_t* drain = mma_done + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  const int m0 = blockIdx.x * kAsgRows, bh = blockIdx.y;
+  const int chunk = blockIdx.x, bh = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m_base = chunk * kSortChunk;
+  int tiles = (s.n_pad - m_base + kAsgRows - 1) / kAsgRows;
+  if (tiles > kAsgTiles) tiles = kAsgTiles;
   if (threadIdx.x == 0) {
-    mbar_init(full, 1);
-    mbar_init(done, 1);
+    for (int i = 0; i < kXStages; ++i) mbar_init(&x_full[i], 1);
+    mbar_init(u_full, 1);
+    mbar_init(&mma_done[0], 1);
+    mbar_init(&mma_done[1], 1);
+    mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
   for (int i = threadIdx.x; i < Cp; i += blockDim.x) sbias[i] = bias[(size_t)bh * Cp + i];
   for (int i = threadIdx.x; i <= C; i += blockDim.x) hist[i] = 0;
-  if (warp == 0) { tmem_alloc(tmem_slot, (uint32_t)Cp); tmem_relinquish(); }
+  if (warp == 0) { tmem_alloc(tmem_slot, (uint32_t)(2 * Cp)); tmem_relinquish(); }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-
+  const uint32_t id = idesc_bf16(kAsgRows, Cp, false, false);
+  int issued = 0, landed = 0;              // thread 0: token tiles loaded / waited for
+  auto load_x = [&](int i) {
+    uint64_t* bar = &x_full[i % kXStages];
+    mbar_arrive_expect_tx(bar, (uint32_t)L::kXBytes);
+    #pragma unroll
+    for (int c = 0; c < L::kAChunks; ++c)
+      tma_load_3d(sX + (i % kXStages) * L::kXBytes + c * L::kAChunkBytes, &tmX, bar, c * 64,
+                  m_base + i * kAsgRows, bh);
+    ++issued;
+  };
   if (threadIdx.x == 0) {
-    // one transaction barrier for the token tile and the three terms of every centre
-    mbar_arrive_expect_tx(full, (uint32_t)(L::kAChunks * L::kAChunkBytes + L::kBChunks * b_chunk));
+    mbar_arrive_expect_tx(u_full, (uint32_t)(L::kBChunks * b_chunk));
     #pragma unroll
-    for (int c = 0; c < L::kAChunks; ++c) tma_load_3d(sA + c * L::kAChunkBytes, &tmX, full, c * 64, m0, bh);
-    #pragma unroll
-    for (int c = 0; c < L::kBChunks; ++c) tma_load_3d(sB + c * b_chunk, &tmU, full, c * 64, 0, bh);
-    if (mbar_wait(full, 0, abort_flag, status)) {
-      tc_fence_after();
-      const uint32_t id = idesc_bf16(kAsgRows, Cp, false, false);
-      uint32_t acc = 0;
-      #pragma unroll
-      for (int part = 0; part < 3; ++part) {
-        #pragma unroll
-        for (int c = 0; c < L::kAChunks; ++c) {
-          const uint32_t a = smem_u32(sA + c * L::kAChunkBytes);
-          const uint32_t b = smem_u32(sB + (part * L::kAChunks + c) * b_chunk);
-          #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            mma_bf16_ss(tmem, desc_kmajor(a + kk * 32), desc_kmajor(b + kk * 32), id, acc);
-            acc = 1;
-          }
-        }
-      }
-    } else {
-      // let the loads in flight land before the shared memory is released
-      const long long t0 = clock64();
-      while (!mbar_try_wait(full, 0) && clock64() - t0 < kWaitBudgetCycles) {}
-    }
-    mma_commit(done);   // also when aborting: arrives once the MMAs issued so far are done
+    for (int c = 0; c < L::kBChunks; ++c) tma_load_3d(sU + c * b_chunk, &tmU, u_full, c * 64, 0, bh);
+    for (int i = 0; i < kXStages - 1 && i < tiles; ++i) load_x(i);
   }
-  const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(done, 0, abort_flag, status)) && !*abort_flag;
-  tc_fence_after();
-  if (ok) {                                 // warp-uniform: the TMEM loads are warp-collective
+
+  // labels of tile j from TMEM buffer j & 1 (all four warps, one row each)
+  auto epilogue = [&](int j) {
     float best_v = __int_as_float(0x7F800000);
     int best = 0;
     for (int cc = 0; cc < Cp / 32; ++cc) {
       uint32_t v[32];
-      tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + cc * 32, v);
+      tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)((j & 1) * Cp + cc * 32), v);
       tmem_wait_ld();
       #pragma unroll
       for (int i = 0; i < 32; ++i) {
@@ -202,29 +208,89 @@ __global__ void __launch_bounds__(128) svoo_assign_kernel(const __grid_constant_
         if (n < C && sc < best_v) { best_v = sc; best = n; }
       }
     }
-    const int t = m0 + warp * 32 + lane;
+    const int t = m_base + j * kAsgRows + warp * 32 + lane;
     if (t < s.n_pad) {
       const int lab = token_valid(s, t) ? best : C;
       labels[(size_t)bh * s.n_pad + t] = lab;
       atomicAdd(&hist[lab], 1);
     }
+  };
+
+  for (int i = 0; i <= tiles; ++i) {
+    if (*abort_flag) break;                 // uniform: read after the barrier that ends each pass
+    if (i < tiles && threadIdx.x == 0) {
+      bool ok = (i > 0 || mbar_wait(u_full, 0, abort_flag, status)) &&
+                mbar_wait(&x_full[i % kXStages], (uint32_t)(i / kXStages) & 1u, abort_flag, status);
+      if (ok) {
+        ++landed;
+        tc_fence_after();
+        const uint32_t d = tmem + (uint32_t)((i & 1) * Cp);
+        uint32_t acc = 0;
+        #pragma unroll
+        for (int part = 0; part < 3; ++part) {
+          #pragma unroll
+          for (int c = 0; c < L::kAChunks; ++c) {
+            const uint32_t a = smem_u32(sX + (i % kXStages) * L::kXBytes + c * L::kAChunkBytes);
+            const uint32_t b = smem_u32(sU + (part * L::kAChunks + c) * b_chunk);
+            #pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              mma_bf16_ss(d, desc_kmajor(a + kk * 32), desc_kmajor(b + kk * 32), id, acc);
+              acc = 1;
+            }
+          }
+        }
+        mma_commit(&mma_done[i & 1]);
+        // the stage of tile i - 1 is free once its MMAs are done: load tile i + kXStages - 1 into it
+        if (i + kXStages - 1 < tiles &&
+            (i == 0 || mbar_wait(&mma_done[(i - 1) & 1], (uint32_t)((i - 1) >> 1) & 1u, abort_flag, status)))
+          load_x(i + kXStages - 1);
+      }
+    }
+    if (i > 0) {
+      const int j = i - 1;
+      const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(&mma_done[j & 1], (uint32_t)(j >> 1) & 1u, abort_flag,
+                                                        status));
+      tc_fence_after();
+      if (ok) epilogue(j);
+    }
+    tc_fence_before();
+    __syncthreads();                        // TMEM buffer (i - 1) & 1 is read before tile i + 1 reuses it
+    tc_fence_after();
   }
-  tc_fence_before();
+  if (threadIdx.x == 0) {
+    // loads still in flight land before the shared memory is released; the MMAs issued
+    // so far are done before TMEM is released
+    for (int i = landed; i < issued; ++i) {
+      const long long t0 = clock64();
+      while (!mbar_try_wait(&x_full[i % kXStages], (uint32_t)(i / kXStages) & 1u) &&
+             clock64() - t0 < kWaitBudgetCycles) {}
+    }
+    mma_commit(drain);
+  }
+  {
+    const long long t0 = clock64();
+    while (!mbar_try_wait(drain, 0) && clock64() - t0 < kWaitBudgetCycles) {}
+  }
+  tc_fence_after();
   __syncthreads();
-  if (ok) {
-    int32_t* cnt = counts + ((size_t)bh * n_chunks + m0 / kSortChunk) * (C + 1);
+  if (!*abort_flag) {
+    int32_t* cnt = counts + ((size_t)bh * n_chunks + chunk) * (C + 1);
     for (int i = threadIdx.x; i <= C; i += blockDim.x)
       if (hist[i]) atomicAdd(&cnt[i], hist[i]);
   }
-  if (warp == 0) { tc_fence_after(); tmem_dealloc(tmem, (uint32_t)Cp); }
+  if (warp == 0) { tc_fence_after(); tmem_dealloc(tmem, (uint32_t)(2 * Cp)); }
 }
 
 // ------------------------------------------------------------------ counting sort
 // Exclusive offsets of every (chunk, bucket): the tokens of bucket b in chunk ch start at
 // offs[ch][b] = start[b] + (tokens of bucket b in chunks before ch).  The counts are
-// cleared on the way, ready for the next step's histogram.
+// cleared on the way, ready for the next step's histogram.  Also the piece offsets of the
+// centre update: cluster n (< C) is cut into ceil(size / kPiece) pieces of consecutive
+// positions, the first of which is piece poff[n]; poff[C] = the number of pieces.
+constexpr int kPiece = 256;
 __global__ void __launch_bounds__(256) svoo_scan_kernel(int32_t* __restrict__ counts, int32_t* __restrict__ offs,
-                                                        int32_t* __restrict__ start, int n_chunks, int C) {
+                                                        int32_t* __restrict__ start, int32_t* __restrict__ poff,
+                                                        int n_chunks, int C) {
   __shared__ int total[kHistSlots];
   __shared__ int base[kHistSlots + 1];
   const int bh = blockIdx.x, b = threadIdx.x, nbk = C + 1;
@@ -232,19 +298,28 @@ __global__ void __launch_bounds__(256) svoo_scan_kernel(int32_t* __restrict__ co
   int32_t* off = offs + (size_t)bh * n_chunks * nbk;
   if (b < nbk) {
     int run = 0;
-    for (int ch = 0; ch < n_chunks; ++ch) {
-      const int v = cnt[(size_t)ch * nbk + b];
-      off[(size_t)ch * nbk + b] = run;
-      cnt[(size_t)ch * nbk + b] = 0;
-      run += v;
+    for (int c0 = 0; c0 < n_chunks; c0 += 8) {
+      int v[8];
+      #pragma unroll
+      for (int j = 0; j < 8; ++j) v[j] = c0 + j < n_chunks ? cnt[(size_t)(c0 + j) * nbk + b] : 0;
+      #pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (c0 + j < n_chunks) {
+          off[(size_t)(c0 + j) * nbk + b] = run;
+          cnt[(size_t)(c0 + j) * nbk + b] = 0;
+        }
+        run += v[j];
+      }
     }
     total[b] = run;
   }
   __syncthreads();
   if (b == 0) {
-    int r = 0;
+    int r = 0, pr = 0;
     for (int i = 0; i < nbk; ++i) { base[i] = r; r += total[i]; }
     base[nbk] = r;
+    for (int i = 0; i < C; ++i) { poff[(size_t)bh * (C + 1) + i] = pr; pr += (total[i] + kPiece - 1) / kPiece; }
+    poff[(size_t)bh * (C + 1) + C] = pr;
   }
   __syncthreads();
   if (b < nbk)
@@ -292,54 +367,80 @@ __global__ void __launch_bounds__(kScatterThreads) svoo_scatter_kernel(const int
 }
 
 // ------------------------------------------------------------------ centre update
-// Centre n = mean of the tokens at positions [start[n], start[n+1]) of the order, in
-// fp64.  The positions are taken 256 at a time (their token indices staged in shared
-// memory); warp w sums rows w, w + 8, ... of each group of 256, lane l owning channels
-// [l D/32, (l+1) D/32), and the eight warp sums are added in warp order.
+// Centre n = mean of the tokens at positions [start[n], start[n+1]) of the order, in fp64,
+// in two deterministic passes.  svoo_piece_kernel: one CTA per piece of kPiece consecutive
+// positions of one cluster (their token indices staged in shared memory); warp w sums rows
+// w, w + 8, ... of the piece, lane l owning channels [l D/32, (l+1) D/32), and the eight warp
+// sums are added in warp order into part[piece].  svoo_finalize_kernel: the pieces of each
+// cluster are added in order and divided by its size; an empty cluster keeps its centre.
 template <int D>
-__global__ void __launch_bounds__(256) svoo_update_kernel(const __nv_bfloat16* __restrict__ x,
-                                                          const int32_t* __restrict__ perm,
-                                                          const int32_t* __restrict__ start,
-                                                          float* __restrict__ centres, int C, int Cp, int n_pad) {
+__global__ void __launch_bounds__(256) svoo_piece_kernel(const __nv_bfloat16* __restrict__ x,
+                                                         const int32_t* __restrict__ perm,
+                                                         const int32_t* __restrict__ start,
+                                                         const int32_t* __restrict__ poff,
+                                                         double* __restrict__ part, int C, int n_pad,
+                                                         int max_pieces) {
   constexpr int kPer = D / 32;              // channels per lane: 4 (d = 128) or 2 (d = 64)
-  __shared__ int sp[256];
+  __shared__ int sp[kPiece];
   __shared__ double red[8][D];
-  const int n = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int b0 = start[(size_t)bh * (C + 2) + n], b1 = start[(size_t)bh * (C + 2) + n + 1];
-  const int32_t* pr = perm + (size_t)bh * n_pad;
+  __shared__ int s_n;
+  const int p = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int32_t* po = poff + (size_t)bh * (C + 1);
+  if (p >= po[C]) return;                   // uniform: fewer pieces than the bound
+  if (tid == 0) {                           // the cluster of this piece: the last n with poff[n] <= p
+    int lo = 0, hi = C - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (po[mid] <= p) lo = mid; else hi = mid - 1;
+    }
+    s_n = lo;
+  }
+  __syncthreads();
+  const int n = s_n;
+  const int p0 = start[(size_t)bh * (C + 2) + n] + (p - po[n]) * kPiece;
+  const int p1 = min(start[(size_t)bh * (C + 2) + n + 1], p0 + kPiece);
+  const int cnt = p1 - p0;
+  if (tid < cnt) sp[tid] = perm[(size_t)bh * n_pad + p0 + tid];
+  __syncthreads();
   const __nv_bfloat16* xb = x + (size_t)bh * n_pad * D;
   double acc[kPer];
   #pragma unroll
   for (int i = 0; i < kPer; ++i) acc[i] = 0.0;
-  for (int p0 = b0; p0 < b1; p0 += 256) {
-    const int cnt = min(256, b1 - p0);
-    __syncthreads();                        // the previous group's indices are consumed
-    if (tid < cnt) sp[tid] = pr[p0 + tid];
-    __syncthreads();
-    #pragma unroll 8
-    for (int j = warp; j < cnt; j += 8) {
-      const int t = sp[j];
-      if ((unsigned)t >= (unsigned)n_pad) continue;   // only after an aborted assignment
-      const __nv_bfloat16* row = xb + (size_t)t * D + lane * kPer;
-      if constexpr (kPer == 4) {
-        const uint2 w = *reinterpret_cast<const uint2*>(row);
-        acc[0] += (double)bf16_lo(w.x); acc[1] += (double)bf16_hi(w.x);
-        acc[2] += (double)bf16_lo(w.y); acc[3] += (double)bf16_hi(w.y);
-      } else {
-        const uint32_t w = *reinterpret_cast<const uint32_t*>(row);
-        acc[0] += (double)bf16_lo(w); acc[1] += (double)bf16_hi(w);
-      }
+  #pragma unroll 8
+  for (int j = warp; j < cnt; j += 8) {
+    const int t = sp[j];
+    if ((unsigned)t >= (unsigned)n_pad) continue;     // only after an aborted assignment
+    const __nv_bfloat16* row = xb + (size_t)t * D + lane * kPer;
+    if constexpr (kPer == 4) {
+      const uint2 w = *reinterpret_cast<const uint2*>(row);
+      acc[0] += (double)bf16_lo(w.x); acc[1] += (double)bf16_hi(w.x);
+      acc[2] += (double)bf16_lo(w.y); acc[3] += (double)bf16_hi(w.y);
+    } else {
+      const uint32_t w = *reinterpret_cast<const uint32_t*>(row);
+      acc[0] += (double)bf16_lo(w); acc[1] += (double)bf16_hi(w);
     }
   }
   #pragma unroll
   for (int i = 0; i < kPer; ++i) red[warp][lane * kPer + i] = acc[i];
   __syncthreads();
-  if (tid < D && b1 > b0) {
+  if (tid < D) {
     double sum = 0.0;
     #pragma unroll
     for (int w = 0; w < 8; ++w) sum += red[w][tid];
-    centres[((size_t)bh * Cp + n) * D + tid] = (float)(sum / (double)(b1 - b0));
+    part[((size_t)bh * max_pieces + p) * D + tid] = sum;
   }
+}
+
+__global__ void svoo_finalize_kernel(const double* __restrict__ part, const int32_t* __restrict__ start,
+                                     const int32_t* __restrict__ poff, float* __restrict__ centres, int C, int Cp,
+                                     int d, int max_pieces) {
+  const int n = blockIdx.x, bh = blockIdx.y, c = threadIdx.x;
+  const int size = start[(size_t)bh * (C + 2) + n + 1] - start[(size_t)bh * (C + 2) + n];
+  if (size <= 0) return;
+  const int q0 = poff[(size_t)bh * (C + 1) + n], q1 = poff[(size_t)bh * (C + 1) + n + 1];
+  double sum = 0.0;
+  for (int q = q0; q < q1; ++q) sum += part[((size_t)bh * max_pieces + q) * d + c];
+  centres[((size_t)bh * Cp + n) * d + c] = (float)(sum / (double)size);
 }
 
 // ------------------------------------------------------------------ row gather / scatter
@@ -441,7 +542,7 @@ cudaError_t launch_assign_d(const void* x, const __nv_bfloat16* ub, const float*
   const size_t smem = L::bytes(Cp);
   cudaError_t e = cudaFuncSetAttribute(svoo_assign_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  dim3 grid((s.n_pad + kAsgRows - 1) / kAsgRows, BH);
+  dim3 grid(svoo_sort_chunks(s.n_pad), BH);
   svoo_assign_kernel<D><<<grid, 128, smem, st>>>(mx, mu, bias, C, Cp, labels, counts, svoo_sort_chunks(s.n_pad), s,
                                                  status);
   return cudaGetLastError();
@@ -458,24 +559,30 @@ cudaError_t launch_svoo_assign(const void* x, const float* other, int C_other, f
                   : launch_assign_d<64>(x, ub, bias, C_own, Cp, labels, counts, BH, s, status, st);
 }
 
-cudaError_t launch_svoo_sort(const int32_t* labels, int32_t* counts, int32_t* offs, int32_t* start, int32_t* perm,
-                             int C, int BH, SeqShape s, cudaStream_t st) {
+cudaError_t launch_svoo_sort(const int32_t* labels, int32_t* counts, int32_t* offs, int32_t* start, int32_t* poff,
+                             int32_t* perm, int C, int BH, SeqShape s, cudaStream_t st) {
   const int nch = svoo_sort_chunks(s.n_pad);
-  svoo_scan_kernel<<<BH, 256, 0, st>>>(counts, offs, start, nch, C);
+  svoo_scan_kernel<<<BH, 256, 0, st>>>(counts, offs, start, poff, nch, C);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   svoo_scatter_kernel<<<dim3(nch, BH), kScatterThreads, 0, st>>>(labels, offs, perm, nch, C, s.n_pad);
   return cudaGetLastError();
 }
 
-cudaError_t launch_svoo_update(const void* x, const int32_t* perm, const int32_t* start, float* centres, int C,
-                               int BH, int d, SeqShape s, cudaStream_t st) {
+int svoo_max_pieces(int n_pad, int C) { return (n_pad + kPiece - 1) / kPiece + C; }
+
+cudaError_t launch_svoo_update(const void* x, const int32_t* perm, const int32_t* start, const int32_t* poff,
+                               double* part, float* centres, int C, int BH, int d, SeqShape s, cudaStream_t st) {
   const int Cp = svoo_padded_clusters(C);
+  const int mp = svoo_max_pieces(s.n_pad, C);
   const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
   if (d == 128)
-    svoo_update_kernel<128><<<dim3(C, BH), 256, 0, st>>>(xb, perm, start, centres, C, Cp, s.n_pad);
+    svoo_piece_kernel<128><<<dim3(mp, BH), 256, 0, st>>>(xb, perm, start, poff, part, C, s.n_pad, mp);
   else
-    svoo_update_kernel<64><<<dim3(C, BH), 256, 0, st>>>(xb, perm, start, centres, C, Cp, s.n_pad);
+    svoo_piece_kernel<64><<<dim3(mp, BH), 256, 0, st>>>(xb, perm, start, poff, part, C, s.n_pad, mp);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  svoo_finalize_kernel<<<dim3(C, BH), d, 0, st>>>(part, start, poff, centres, C, Cp, d, mp);
   return cudaGetLastError();
 }
 

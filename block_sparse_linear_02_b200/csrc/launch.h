@@ -160,12 +160,15 @@ cudaError_t launch_svoo_anchors(const void* x, const int32_t* anchor, float* cen
 cudaError_t launch_svoo_assign(const void* x, const float* other, int C_other, float* own, int C_own,
                                __nv_bfloat16* ub, float* bias, int32_t* labels, int32_t* counts, int BH, int d,
                                SeqShape s, int* status, cudaStream_t st);
-// the stable order of the labels: perm (position -> token) and the cluster starts
-cudaError_t launch_svoo_sort(const int32_t* labels, int32_t* counts, int32_t* offs, int32_t* start, int32_t* perm,
-                             int C, int BH, SeqShape s, cudaStream_t st);
-// centres = means of their tokens (an empty cluster keeps its centre)
-cudaError_t launch_svoo_update(const void* x, const int32_t* perm, const int32_t* start, float* centres, int C,
-                               int BH, int d, SeqShape s, cudaStream_t st);
+// the stable order of the labels: perm (position -> token), the cluster starts and the
+// piece offsets of the update (poff int32 [BH][C + 1])
+cudaError_t launch_svoo_sort(const int32_t* labels, int32_t* counts, int32_t* offs, int32_t* start, int32_t* poff,
+                             int32_t* perm, int C, int BH, SeqShape s, cudaStream_t st);
+// centres = means of their tokens (an empty cluster keeps its centre), through fp64 piece
+// sums part [BH][svoo_max_pieces(n_pad, C)][d]
+int svoo_max_pieces(int n_pad, int C);
+cudaError_t launch_svoo_update(const void* x, const int32_t* perm, const int32_t* start, const int32_t* poff,
+                               double* part, float* centres, int C, int BH, int d, SeqShape s, cudaStream_t st);
 // qp[p] = q[q_perm[p]], kp[p] = k[k_perm[p]], vp[p] = v[k_perm[p]] (bf16 rows of d)
 cudaError_t launch_svoo_gather(const void* q, const void* k, const void* v, const int32_t* q_perm,
                                const int32_t* k_perm, void* qp, void* kp, void* vp, int BH, int d, int n_pad,

@@ -270,6 +270,8 @@ struct SvooClusterWs {
   __nv_bfloat16* ub;                   // metric of the assigning side [BH][Cp][3d]
   float* bias;                         // [BH][Cp]
   int32_t *counts, *offs, *start;      // counting sort
+  int32_t* poff;                       // piece offsets of the centre update
+  double* part;                        // fp64 piece sums of the centre update
 };
 
 void plan_svoo_cluster(Carve& c, const Shape& sh, int n_qc, int n_kc, SvooClusterWs& w) {
@@ -284,6 +286,8 @@ void plan_svoo_cluster(Carve& c, const Shape& sh, int n_qc, int n_kc, SvooCluste
   w.counts = c.take<int32_t>((size_t)sh.BH * nch * (cm + 1));
   w.offs = c.take<int32_t>((size_t)sh.BH * nch * (cm + 1));
   w.start = c.take<int32_t>((size_t)sh.BH * (cm + 2));
+  w.poff = c.take<int32_t>((size_t)sh.BH * (cm + 1));
+  w.part = c.take<double>((size_t)sh.BH * svoo_max_pieces(sh.n_pad, cm) * sh.d);
 }
 
 struct SvooAttnWs {
@@ -738,14 +742,18 @@ slr_status slr_svoo_cocluster(const void* q, const void* k, const slr_seq* seq, 
     // step A: the keys against the query centres, then the key centres move
     SLR_LAUNCH(kKSvooAssign, s, launch_svoo_assign(k, w.cq, n_qc, w.ck, n_kc, w.ub, w.bias, k_label, w.counts,
                                                    sh.BH, sh.d, sh.s, w.status, s));
-    SLR_LAUNCH(kKSvooSort, s, launch_svoo_sort(k_label, w.counts, w.offs, w.start, k_perm, n_kc, sh.BH, sh.s, s));
-    SLR_LAUNCH(kKSvooUpdate, s, launch_svoo_update(k, k_perm, w.start, w.ck, n_kc, sh.BH, sh.d, sh.s, s));
+    SLR_LAUNCH(kKSvooSort, s, launch_svoo_sort(k_label, w.counts, w.offs, w.start, w.poff, k_perm, n_kc, sh.BH,
+                                               sh.s, s));
+    SLR_LAUNCH(kKSvooUpdate, s, launch_svoo_update(k, k_perm, w.start, w.poff, w.part, w.ck, n_kc, sh.BH, sh.d,
+                                                   sh.s, s));
     // step B: the queries against the updated key centres
     SLR_LAUNCH(kKSvooAssign, s, launch_svoo_assign(q, w.ck, n_kc, w.cq, n_qc, w.ub, w.bias, q_label, w.counts,
                                                    sh.BH, sh.d, sh.s, w.status, s));
-    SLR_LAUNCH(kKSvooSort, s, launch_svoo_sort(q_label, w.counts, w.offs, w.start, q_perm, n_qc, sh.BH, sh.s, s));
+    SLR_LAUNCH(kKSvooSort, s, launch_svoo_sort(q_label, w.counts, w.offs, w.start, w.poff, q_perm, n_qc, sh.BH,
+                                               sh.s, s));
     if (it + 1 < iters)
-      SLR_LAUNCH(kKSvooUpdate, s, launch_svoo_update(q, q_perm, w.start, w.cq, n_qc, sh.BH, sh.d, sh.s, s));
+      SLR_LAUNCH(kKSvooUpdate, s, launch_svoo_update(q, q_perm, w.start, w.poff, w.part, w.cq, n_qc, sh.BH, sh.d,
+                                                     sh.s, s));
   }
   return SLR_OK;
 }
