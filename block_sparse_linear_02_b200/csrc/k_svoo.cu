@@ -64,12 +64,15 @@ __global__ void svoo_anchor_kernel(const __nv_bfloat16* __restrict__ x, const in
 // ------------------------------------------------------------------ metric
 // For own centre n (< Cs): a_m = R_m . s_n over the Cr centres of the other side,
 // u_n = sum_m a_m R_m, b_n = sum_m a_m^2, all in fp64 with a fixed summation order.
+// The Cr x d rows of R are staged in shared memory first (one coalesced pass).
 // u_n is written as bf16 hi | mid | lo rows of 3d columns; rows n >= Cs are zero.
 __global__ void __launch_bounds__(128) svoo_metric_kernel(const float* __restrict__ R, int Cr, int Cpr,
                                                           const float* __restrict__ S, int Cs, int Cps, int d,
                                                           __nv_bfloat16* __restrict__ ub, float* __restrict__ bias) {
+  extern __shared__ float4 sR4[];           // Cr x d fp32
   __shared__ double s_n[128];
   __shared__ double a[128];
+  const float* sR = reinterpret_cast<const float*>(sR4);
   const int n = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   __nv_bfloat16* row = ub + ((size_t)bh * Cps + n) * 3 * d;
   if (n >= Cs) {
@@ -77,12 +80,13 @@ __global__ void __launch_bounds__(128) svoo_metric_kernel(const float* __restric
     if (tid == 0) bias[(size_t)bh * Cps + n] = 0.f;
     return;
   }
-  const float* Rb = R + (size_t)bh * Cpr * d;
+  const float4* src = reinterpret_cast<const float4*>(R + (size_t)bh * Cpr * d);
+  for (int i = tid; i < Cr * d / 4; i += blockDim.x) sR4[i] = src[i];
   if (tid < d) s_n[tid] = (double)S[((size_t)bh * Cps + n) * d + tid];
   __syncthreads();
   for (int m = warp; m < Cr; m += 4) {
     double p = 0.0;
-    for (int c = lane; c < d; c += 32) p += (double)Rb[(size_t)m * d + c] * s_n[c];
+    for (int c = lane; c < d; c += 32) p += (double)sR[m * d + c] * s_n[c];
     #pragma unroll
     for (int off = 16; off > 0; off >>= 1) p += __shfl_xor_sync(0xFFFFFFFFu, p, off);
     if (lane == 0) a[m] = p;
@@ -90,7 +94,7 @@ __global__ void __launch_bounds__(128) svoo_metric_kernel(const float* __restric
   __syncthreads();
   if (tid < d) {
     double u = 0.0;
-    for (int m = 0; m < Cr; ++m) u += a[m] * (double)Rb[(size_t)m * d + tid];
+    for (int m = 0; m < Cr; ++m) u += a[m] * (double)sR[m * d + tid];
     const __nv_bfloat16 hi = __double2bfloat16(u);
     const double r1 = u - (double)__bfloat162float(hi);
     const __nv_bfloat16 mid = __double2bfloat16(r1);
@@ -109,18 +113,20 @@ __global__ void __launch_bounds__(128) svoo_metric_kernel(const float* __restric
 // ------------------------------------------------------------------ assignment
 // One CTA per 1024-token chunk of one head (8 tiles of 128 tokens), one CTA per SM.
 // Shared memory (offsets from a 1024-byte aligned base):
-//   X  a ring of kXStages token tiles, each D/64 chunks of 128 rows x 64 bf16 (16 KB),
+//   X  a ring of nst token tiles (4, or 3 when the metric takes 128 rows), each D/64
+//      chunks of 128 rows x 64 bf16 (16 KB),
 //      128-byte swizzled
 //   U  3D/64 chunks of Cp centre rows x 64 bf16: the hi chunks, the mid chunks, the lo
 //      chunks (loaded once: the chunk's head has one metric)
 //   then the Cp biases, the label histogram, the mbarriers, the TMEM slot, the abort flag
 // Thread 0 loads and issues the MMAs; tile i's scores go to TMEM columns (i & 1) * Cp, so
 // that the four warps' argmin of tile i - 1 overlaps the MMAs of tile i, and the load of
-// tile i + kXStages - 1 is issued as soon as the MMAs of tile i - 1 have read their stage.
+// tile i + nst - 1 is issued as soon as the MMAs of tile i - 1 have read their stage.
 constexpr int kMaxClusters = 128;
 constexpr int kHistSlots = 160;       // >= kMaxClusters + 1 buckets
 constexpr int kAsgTiles = kSortChunk / kAsgRows;
-constexpr int kXStages = 3;
+constexpr int kXStagesMax = 4;
+constexpr size_t kAsgSmemCap = 200 * 1024;   // a fourth stage only below this
 template <int D>
 struct AsgLayout {
   static constexpr int kAChunks = D / 64;
@@ -128,9 +134,12 @@ struct AsgLayout {
   static constexpr int kAChunkBytes = kAsgRows * 128;
   static constexpr int kXBytes = kAChunks * kAChunkBytes;
   __host__ __device__ static size_t b_chunk_bytes(int Cp) { return (size_t)Cp * 128; }
-  __host__ __device__ static size_t u_off() { return (size_t)kXStages * kXBytes; }
-  __host__ __device__ static size_t bias_off(int Cp) { return u_off() + kBChunks * b_chunk_bytes(Cp); }
-  __host__ __device__ static size_t bytes(int Cp) { return bias_off(Cp) + kMaxClusters * 4 + kHistSlots * 4 + 128 + 1024; }
+  __host__ __device__ static size_t u_off(int nst) { return (size_t)nst * kXBytes; }
+  __host__ __device__ static size_t bias_off(int Cp, int nst) { return u_off(nst) + kBChunks * b_chunk_bytes(Cp); }
+  __host__ __device__ static size_t bytes(int Cp, int nst) {
+    return bias_off(Cp, nst) + kMaxClusters * 4 + kHistSlots * 4 + 128 + 1024;
+  }
+  static int stages(int Cp) { return bytes(Cp, kXStagesMax) <= kAsgSmemCap ? kXStagesMax : kXStagesMax - 1; }
 };
 
 template <int D>
@@ -139,17 +148,17 @@ __global__ void __launch_bounds__(128, 1) svoo_assign_kernel(const __grid_consta
                                                              const float* __restrict__ bias, int C, int Cp,
                                                              int32_t* __restrict__ labels,
                                                              int32_t* __restrict__ counts, int n_chunks, SeqShape s,
-                                                             int* status) {
+                                                             int nst, int* status) {
   using L = AsgLayout<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t b_chunk = (uint32_t)L::b_chunk_bytes(Cp);
   uint8_t* sX = smem;
-  uint8_t* sU = smem + L::u_off();
-  float* sbias = reinterpret_cast<float*>(smem + L::bias_off(Cp));
+  uint8_t* sU = smem + L::u_off(nst);
+  float* sbias = reinterpret_cast<float*>(smem + L::bias_off(Cp, nst));
   int* hist = reinterpret_cast<int*>(sbias + kMaxClusters);
-  uint64_t* x_full = reinterpret_cast<uint64_t*>(hist + kHistSlots);   // [kXStages]
-  uint64_t* u_full = x_full + kXStages;
+  uint64_t* x_full = reinterpret_cast<uint64_t*>(hist + kHistSlots);   // [kXStagesMax]
+  uint64_t* u_full = x_full + kXStagesMax;
   uint64_t* mma_done = u_full + 1;                                     // [2]
   uint64_t* drain = mma_done + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
@@ -160,7 +169,7 @@ __global__ void __launch_bounds__(128, 1) svoo_assign_kernel(const __grid_consta
   int tiles = (s.n_pad - m_base + kAsgRows - 1) / kAsgRows;
   if (tiles > kAsgTiles) tiles = kAsgTiles;
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kXStages; ++i) mbar_init(&x_full[i], 1);
+    for (int i = 0; i < kXStagesMax; ++i) mbar_init(&x_full[i], 1);
     mbar_init(u_full, 1);
     mbar_init(&mma_done[0], 1);
     mbar_init(&mma_done[1], 1);
@@ -178,19 +187,18 @@ __global__ void __launch_bounds__(128, 1) svoo_assign_kernel(const __grid_consta
   const uint32_t id = idesc_bf16(kAsgRows, Cp, false, false);
   int issued = 0, landed = 0;              // thread 0: token tiles loaded / waited for
   auto load_x = [&](int i) {
-    uint64_t* bar = &x_full[i % kXStages];
+    uint64_t* bar = &x_full[i % nst];
     mbar_arrive_expect_tx(bar, (uint32_t)L::kXBytes);
     #pragma unroll
     for (int c = 0; c < L::kAChunks; ++c)
-      tma_load_3d(sX + (i % kXStages) * L::kXBytes + c * L::kAChunkBytes, &tmX, bar, c * 64,
-                  m_base + i * kAsgRows, bh);
+      tma_load_3d(sX + (i % nst) * L::kXBytes + c * L::kAChunkBytes, &tmX, bar, c * 64, m_base + i * kAsgRows, bh);
     ++issued;
   };
   if (threadIdx.x == 0) {
     mbar_arrive_expect_tx(u_full, (uint32_t)(L::kBChunks * b_chunk));
     #pragma unroll
     for (int c = 0; c < L::kBChunks; ++c) tma_load_3d(sU + c * b_chunk, &tmU, u_full, c * 64, 0, bh);
-    for (int i = 0; i < kXStages - 1 && i < tiles; ++i) load_x(i);
+    for (int i = 0; i < nst - 1 && i < tiles; ++i) load_x(i);
   }
 
   // labels of tile j from TMEM buffer j & 1 (all four warps, one row each)
@@ -209,18 +217,18 @@ __global__ void __launch_bounds__(128, 1) svoo_assign_kernel(const __grid_consta
       }
     }
     const int t = m_base + j * kAsgRows + warp * 32 + lane;
-    if (t < s.n_pad) {
-      const int lab = token_valid(s, t) ? best : C;
-      labels[(size_t)bh * s.n_pad + t] = lab;
-      atomicAdd(&hist[lab], 1);
-    }
+    const int lab = t < s.n_pad ? (token_valid(s, t) ? best : C) : -1;
+    if (lab >= 0) labels[(size_t)bh * s.n_pad + t] = lab;
+    // one shared-memory atomic per distinct label of the warp
+    const unsigned peers = __match_any_sync(0xFFFFFFFFu, lab);
+    if (lab >= 0 && (peers & ((1u << lane) - 1u)) == 0) atomicAdd(&hist[lab], __popc(peers));
   };
 
   for (int i = 0; i <= tiles; ++i) {
     if (*abort_flag) break;                 // uniform: read after the barrier that ends each pass
     if (i < tiles && threadIdx.x == 0) {
       bool ok = (i > 0 || mbar_wait(u_full, 0, abort_flag, status)) &&
-                mbar_wait(&x_full[i % kXStages], (uint32_t)(i / kXStages) & 1u, abort_flag, status);
+                mbar_wait(&x_full[i % nst], (uint32_t)(i / nst) & 1u, abort_flag, status);
       if (ok) {
         ++landed;
         tc_fence_after();
@@ -230,7 +238,7 @@ __global__ void __launch_bounds__(128, 1) svoo_assign_kernel(const __grid_consta
         for (int part = 0; part < 3; ++part) {
           #pragma unroll
           for (int c = 0; c < L::kAChunks; ++c) {
-            const uint32_t a = smem_u32(sX + (i % kXStages) * L::kXBytes + c * L::kAChunkBytes);
+            const uint32_t a = smem_u32(sX + (i % nst) * L::kXBytes + c * L::kAChunkBytes);
             const uint32_t b = smem_u32(sU + (part * L::kAChunks + c) * b_chunk);
             #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
@@ -240,10 +248,10 @@ __global__ void __launch_bounds__(128, 1) svoo_assign_kernel(const __grid_consta
           }
         }
         mma_commit(&mma_done[i & 1]);
-        // the stage of tile i - 1 is free once its MMAs are done: load tile i + kXStages - 1 into it
-        if (i + kXStages - 1 < tiles &&
+        // the stage of tile i - 1 is free once its MMAs are done: load tile i + nst - 1 into it
+        if (i + nst - 1 < tiles &&
             (i == 0 || mbar_wait(&mma_done[(i - 1) & 1], (uint32_t)((i - 1) >> 1) & 1u, abort_flag, status)))
-          load_x(i + kXStages - 1);
+          load_x(i + nst - 1);
       }
     }
     if (i > 0) {
@@ -262,7 +270,7 @@ __global__ void __launch_bounds__(128, 1) svoo_assign_kernel(const __grid_consta
     // so far are done before TMEM is released
     for (int i = landed; i < issued; ++i) {
       const long long t0 = clock64();
-      while (!mbar_try_wait(&x_full[i % kXStages], (uint32_t)(i / kXStages) & 1u) &&
+      while (!mbar_try_wait(&x_full[i % nst], (uint32_t)(i / nst) & 1u) &&
              clock64() - t0 < kWaitBudgetCycles) {}
     }
     mma_commit(drain);
@@ -539,12 +547,13 @@ cudaError_t launch_assign_d(const void* x, const __nv_bfloat16* ub, const float*
   const uint64_t us[2] = {(uint64_t)(3 * D) * 2, (uint64_t)(3 * D) * 2 * Cp};
   const uint32_t ubx[3] = {64, (uint32_t)Cp, 1};
   if (!make_tile_map(&mu, ub, 3, ud, us, ubx)) return cudaErrorInvalidValue;
-  const size_t smem = L::bytes(Cp);
+  const int nst = L::stages(Cp);
+  const size_t smem = L::bytes(Cp, nst);
   cudaError_t e = cudaFuncSetAttribute(svoo_assign_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid(svoo_sort_chunks(s.n_pad), BH);
   svoo_assign_kernel<D><<<grid, 128, smem, st>>>(mx, mu, bias, C, Cp, labels, counts, svoo_sort_chunks(s.n_pad), s,
-                                                 status);
+                                                 nst, status);
   return cudaGetLastError();
 }
 
@@ -552,8 +561,11 @@ cudaError_t launch_svoo_assign(const void* x, const float* other, int C_other, f
                                __nv_bfloat16* ub, float* bias, int32_t* labels, int32_t* counts, int BH, int d,
                                SeqShape s, int* status, cudaStream_t st) {
   const int Cpo = svoo_padded_clusters(C_other), Cp = svoo_padded_clusters(C_own);
-  svoo_metric_kernel<<<dim3(Cp, BH), 128, 0, st>>>(other, C_other, Cpo, own, C_own, Cp, d, ub, bias);
-  cudaError_t e = cudaGetLastError();
+  const int msmem = C_other * d * (int)sizeof(float);
+  cudaError_t e = cudaFuncSetAttribute(svoo_metric_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, msmem);
+  if (e != cudaSuccess) return e;
+  svoo_metric_kernel<<<dim3(Cp, BH), 128, msmem, st>>>(other, C_other, Cpo, own, C_own, Cp, d, ub, bias);
+  e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   return d == 128 ? launch_assign_d<128>(x, ub, bias, C_own, Cp, labels, counts, BH, s, status, st)
                   : launch_assign_d<64>(x, ub, bias, C_own, Cp, labels, counts, BH, s, status, st);
