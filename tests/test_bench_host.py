@@ -92,3 +92,27 @@ def test_lvsa_flops_counts_attended_frame_blocks():
     # every frame attends C = 21 frames of 25 blocks: 121 * 25 * 21 * 25 block pairs
     assert bench.lvsa_flops(w, sets) == 4 * 64 * 64 * 128 * 121 * 25 * 21 * 25 * 12
     assert abs(bench.lvsa_flops(w, sets) / 1e12 - 39.97) < 0.01
+
+
+def test_svoo_flops_and_config():
+    # 103 kept key blocks (ceil(0.2 * 512)) per query block, 512 query blocks, 12 heads, d = 128
+    w = workloads.SVOO
+    f = bench.svoo_flops(w, 103)
+    assert f == 4 * 64 * 64 * 128 * 512 * 103 * 12
+    assert abs(f / 1e12 - 1.327) < 1e-3
+    c = bench.config_dict(w)
+    assert c["seq_len"] == 32768 and c["heads"] == 12
+    assert "64 query + 64 key clusters" in c["workload"] and "top 20% key blocks" in c["workload"]
+    assert "co-clustering + attention" in c["workload"]
+
+
+def test_svoo_anchors_are_distinct_valid_tokens():
+    w = workloads.SVOO
+    for which, C in (("q", w.clusters[0]), ("k", w.clusters[1])):
+        a = workloads.make_anchors(w, which, heads=3)
+        assert a.shape == (1, 3, C)
+        for h in range(3):
+            row = a[0, h].tolist()
+            assert len(set(row)) == C and min(row) >= 0 and max(row) < w.seg_len
+    # the draw of a head does not depend on how many heads are drawn
+    assert (workloads.make_anchors(w, "q", heads=2)[0, 1] == workloads.make_anchors(w, "q", heads=4)[0, 1]).all()
