@@ -10,6 +10,10 @@ three source write-ups define:
                        percentile classification, sparse softmax attention on
                        critical blocks, linear attention on marginal blocks and
                        the learnable projection of the linear output.
+* ``oracle.sla_grad`` -- the SLA backward (same page, section 3, last paragraph):
+                       FlashAttention-style gradients of the sparse part and
+                       the gradients of the normalised linear part, the block
+                       mask held fixed.
 * ``oracle.lvsa``   -- LVSA (arXiv 2605.31057), as described on the rainbus
                        paper-digest page, sections "核心方法" and "方法步骤详情":
                        the global period T_per, the rotating global set G_s,
@@ -35,4 +39,4 @@ All arithmetic is fp64.  Parity status of every function is listed in each
 module's header; every function is pinned by a test in ``tests/test_oracle_*.py``
 against closed forms, special cases, library routines or hand-worked examples.
 """
-from . import sla, lvsa, tile3d, sta, svoo  # noqa: F401
+from . import sla, sla_grad, lvsa, tile3d, sta, svoo  # noqa: F401
