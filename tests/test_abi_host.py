@@ -198,3 +198,15 @@ def test_svoo_workspace_and_arguments(lib):
                              None) == slr.SLR_ERR_ARG
     assert lib.slr_svoo_attn(fake, fake, fake, ctypes.byref(segs), fake, fake, 0.5, fake, None, ws, 1 << 30,
                              None) == slr.SLR_ERR_UNSUPPORTED
+
+
+def test_svoo_binding_rejects_host_tensors_and_bad_shapes(lib):
+    import torch
+    seq = slr.make_seq(1, 1, 64, 1, 256, 256)
+    q = torch.zeros(1, 1, 256, 64, dtype=torch.bfloat16)
+    anchors = torch.zeros(1, 1, 4, dtype=torch.int32)
+    with pytest.raises(ValueError):           # host tensors never reach the library
+        slr.slr_svoo_cocluster(q, q, seq, anchors, anchors)
+    perm = torch.arange(256, dtype=torch.int32).reshape(1, 1, 256)
+    with pytest.raises(ValueError):
+        slr.slr_svoo_attn(q, q, q, seq, perm, perm, 0.5)
